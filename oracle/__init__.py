@@ -1,0 +1,204 @@
+"""CPU oracle for the MSA hot path (test infrastructure only).
+
+Only the tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  It wraps ``msa_oracle.c`` (plain C,
+double precision, OpenMP over rows) through ctypes and shares no code with
+the CUDA library.
+
+Each function cites the page passage it follows in ``msa_oracle.c``:
+  * ``index_pooled``  -- index-branch token scores + block max-pool
+    ("MSA 稀疏注意力三国杀" page, section "MSA 架构：粗筛 + 精算", steps 1-2;
+    sparse-attention survey page, MSA entry);
+  * ``topk`` / ``topk_f32`` -- 16 blocks per query and group, own block
+    forced (same section, step 3; survey MSA entry);
+  * ``attention`` -- exact softmax attention over the selected tokens (same
+    section, "第二步：精算"; softmax(QK^T/sqrt(d)) V from the chenxutan page);
+  * ``merge`` -- log-sum-exp combination of per-block softmax pieces (the
+    identity the KV-block-outer "Outer Gather Q" scheme relies on);
+  * ``block_query_lists`` -- query->block lists inverted into block->query
+    lists ("Kernel 创新：Outer Gather Q" section).
+
+Parity is pinned by ``tests/test_oracle_pins.py`` (brute force, closed forms,
+invariants and hand-derived fixtures under ``tests/golden/``).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "msa_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "libmsa_oracle.so")
+_lock = threading.Lock()
+_lib = None
+
+BLOCK = 128
+TOPK = 16
+HEAD_DIM = 128
+
+
+def build(force: bool = False) -> str:
+    """Compile ``msa_oracle.c`` into ``libmsa_oracle.so`` next to it."""
+    if (not force and os.path.exists(_LIB_PATH)
+            and os.path.getmtime(_LIB_PATH) >= os.path.getmtime(_SRC)):
+        return _LIB_PATH
+    tmp = _LIB_PATH + f".tmp{os.getpid()}"
+    subprocess.check_call(["gcc", "-std=c99", "-O2", "-fopenmp", "-fPIC", "-shared",
+                           "-o", tmp, _SRC, "-lm"])
+    os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = ctypes.CDLL(build())
+            P = ctypes.c_void_p
+            I64, I32, F64 = ctypes.c_int64, ctypes.c_int32, ctypes.c_double
+            lib.msa_oracle_index_pooled.argtypes = [I64, I32, I32, I64, I32, P, P, P, P, I64, P]
+            lib.msa_oracle_topk.argtypes = [I64, I32, P, I64, P, P]
+            lib.msa_oracle_topk_f32.argtypes = [I64, I64, P, P, P]
+            lib.msa_oracle_attention.argtypes = [I64, I32, I32, I64, P, P, P, P, P, P, F64, P, P]
+            lib.msa_oracle_merge.argtypes = [I64, I32, I32, P, P, P, P, P, P]
+            lib.msa_oracle_block_query_lists.argtypes = [I64, I32, I64, I64, P, P, P]
+            for f in (lib.msa_oracle_index_pooled, lib.msa_oracle_topk, lib.msa_oracle_topk_f32,
+                      lib.msa_oracle_attention, lib.msa_oracle_merge,
+                      lib.msa_oracle_block_query_lists):
+                f.restype = None
+            _lib = lib
+    return _lib
+
+
+def _c(a: np.ndarray, dtype) -> np.ndarray:
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+def _p(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def bf16_bits(x) -> np.ndarray:
+    """Raw uint16 bit patterns of a bf16 torch tensor (or pass uint16 through)."""
+    if isinstance(x, np.ndarray):
+        assert x.dtype == np.uint16
+        return np.ascontiguousarray(x)
+    import torch
+    return x.detach().contiguous().cpu().view(torch.int16).numpy().view(np.uint16)
+
+
+def bits_to_f64(bits: np.ndarray) -> np.ndarray:
+    """bf16 bit patterns -> float64 (exact)."""
+    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def num_blocks(n_kv: int) -> int:
+    return (n_kv + BLOCK - 1) // BLOCK
+
+
+def index_pooled(q_idx_rows, row_pos, row_batch, k_idx, out_stride=None):
+    """Pooled block scores for the given query rows.
+
+    q_idx_rows: uint16 [n_rows, G, d_idx]; row_pos/row_batch: int64 [n_rows];
+    k_idx: uint16 [B', h_kidx, n_kv, d_idx].  Returns float64
+    [n_rows, G, out_stride] with NaN at c >= own(t).
+    """
+    lib = _load()
+    q = _c(q_idx_rows, np.uint16)
+    k = _c(k_idx, np.uint16)
+    pos = _c(row_pos, np.int64)
+    bat = _c(row_batch, np.int64)
+    n_rows, G, d_idx = q.shape
+    _, h_kidx, n_kv, d2 = k.shape
+    assert d2 == d_idx and d_idx <= 256 and h_kidx in (1, G)
+    stride = out_stride or num_blocks(n_kv)
+    out = np.empty((n_rows, G, stride), np.float64)
+    lib.msa_oracle_index_pooled(n_rows, G, d_idx, n_kv, h_kidx, _p(q), _p(pos), _p(bat),
+                                _p(k), stride, _p(out))
+    return out
+
+
+def topk(pooled, row_pos):
+    """Selected blocks [n_rows, G, 16] (ascending, -1 padded) from float64 scores."""
+    lib = _load()
+    s = _c(pooled, np.float64)
+    pos = _c(row_pos, np.int64)
+    n_rows, G, stride = s.shape
+    sel = np.empty((n_rows, G, TOPK), np.int32)
+    lib.msa_oracle_topk(n_rows, G, _p(pos), stride, _p(s), _p(sel))
+    return sel
+
+
+def topk_f32(pooled_f32, own):
+    """Selection on float32 scores [n_rows, stride] with own block per row."""
+    lib = _load()
+    s = _c(pooled_f32, np.float32)
+    o = _c(own, np.int64)
+    n_rows, stride = s.shape
+    sel = np.empty((n_rows, TOPK), np.int32)
+    lib.msa_oracle_topk_f32(n_rows, stride, _p(o), _p(s), _p(sel))
+    return sel
+
+
+def attention(q_rows, row_pos, row_batch, k, v, sel, scale):
+    """Exact softmax attention of the rows over their selected tokens.
+
+    q_rows uint16 [n_rows, H, 128]; k, v uint16 [B', G, n_kv, 128];
+    sel int32 [n_rows, G, 16].  Returns (out float64 [n_rows, H, 128],
+    lse float64 [n_rows, H]).
+    """
+    lib = _load()
+    q = _c(q_rows, np.uint16)
+    kk = _c(k, np.uint16)
+    vv = _c(v, np.uint16)
+    s = _c(sel, np.int32)
+    pos = _c(row_pos, np.int64)
+    bat = _c(row_batch, np.int64)
+    n_rows, H, D = q.shape
+    _, G, n_kv, D2 = kk.shape
+    assert D == HEAD_DIM and D2 == HEAD_DIM and H % G == 0 and vv.shape == kk.shape
+    assert s.shape == (n_rows, G, TOPK)
+    out = np.empty((n_rows, H, HEAD_DIM), np.float64)
+    lse = np.empty((n_rows, H), np.float64)
+    lib.msa_oracle_attention(n_rows, H, G, n_kv, _p(q), _p(pos), _p(bat), _p(kk), _p(vv),
+                             _p(s), float(scale), _p(out), _p(lse))
+    return out, lse
+
+
+def merge(valid, m, l, acc):
+    """Log-sum-exp combination of softmax pieces: valid/m/l [n, S], acc [n, S, D]."""
+    lib = _load()
+    va = _c(valid, np.int32)
+    mm = _c(m, np.float64)
+    ll = _c(l, np.float64)
+    aa = _c(acc, np.float64)
+    n, S, D = aa.shape
+    out = np.empty((n, D), np.float64)
+    lse = np.empty((n,), np.float64)
+    lib.msa_oracle_merge(n, S, D, _p(va), _p(mm), _p(ll), _p(aa), _p(out), _p(lse))
+    return out, lse
+
+
+def block_query_lists(sel, nblk):
+    """CSR inversion of sel [B, G, n_q, 16] -> (offsets int64 [B*G*nblk+1], entries int32)."""
+    lib = _load()
+    s = _c(sel, np.int32)
+    B, G, n_q, T = s.shape
+    assert T == TOPK
+    offsets = np.empty((B * G * nblk + 1,), np.int64)
+    n_ent = int((s >= 0).sum())
+    entries = np.empty((max(n_ent, 1),), np.int32)
+    lib.msa_oracle_block_query_lists(B, G, n_q, nblk, _p(s), _p(offsets), _p(entries))
+    return offsets, entries[:n_ent]
+
+
+def forward_rows(q_rows, q_idx_rows, row_pos, row_batch, k, v, k_idx, scale):
+    """Whole path for sampled rows: pooled scores, selection, attention."""
+    pooled = index_pooled(q_idx_rows, row_pos, row_batch, k_idx)
+    sel = topk(pooled, row_pos)
+    out, lse = attention(q_rows, row_pos, row_batch, k, v, sel, scale)
+    return pooled, sel, out, lse

@@ -1,0 +1,298 @@
+/*
+ * msa_oracle.c -- plain, slow, double-precision CPU definition of the
+ * MiniMax Sparse Attention (MSA) hot path.  TEST INFRASTRUCTURE ONLY: the
+ * tests, the smoke check and the CPU baseline of the benchmark call it; the
+ * product path never does.  It shares no code, header, table or helper with
+ * the CUDA library.
+ *
+ * Sources (page title, section):
+ *  [P1] "MSA 稀疏注意力三国杀：NSA / DSA / MoBA / MSA 四方案深度对比",
+ *       section "MSA 架构：粗筛 + 精算" (index branch: 128-token blocks, one
+ *       score per token, block score = max over the block, 16 blocks with the
+ *       query's own block always taken; main branch: full attention over the
+ *       16 x 128 = 2048 selected tokens).
+ *  [P3] "sparse-attention" survey, entry "MiniMax Sparse Attention (MSA)"
+ *       (per GQA group one index query head and a shared index key head,
+ *       block max-pool, per-group top-k with the local block kept, exact
+ *       softmax attention on the selected blocks).
+ *  [P5] chenxutan.com article, section on standard self-attention, formula
+ *       softmax(Q K^T / sqrt(d_k)) V.
+ *
+ * Readings where the pages are silent (each one is listed in the design
+ * notes as well):
+ *  - index score of (query t, key j) for group g is the raw dot product
+ *    q_idx[t,g,:] . k_idx[j,:] (no scale, bias or activation);
+ *  - a block's score is taken only over keys j <= t; blocks c < own(t) are
+ *    whole, so only the own block would be cut, and it is forced anyway;
+ *  - "16 blocks" counts the forced own block: own + 15 best candidates;
+ *  - ranking is by score descending, ties to the lower block index, with
+ *    -0.0 equal to +0.0 (C comparison of doubles already does this);
+ *  - the attention scale is the caller's (1/sqrt(128) by default);
+ *  - head h belongs to group h / (H / G).
+ *
+ * Every input array is contiguous in the layout stated beside it; bf16
+ * values are passed as their raw uint16 bit patterns.  All arithmetic is
+ * double precision; a bf16 value converts to double exactly, and so does a
+ * product of two of them.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define MSA_BLOCK 128  /* B_k: tokens per KV block ([P1], [P3]) */
+#define MSA_TOPK 16    /* blocks per query and group, own block included */
+#define MSA_HEAD_DIM 128
+
+static double bf16_to_f64(uint16_t h) {
+  uint32_t u = ((uint32_t)h) << 16;
+  float f;
+  memcpy(&f, &u, sizeof f);
+  return (double)f;
+}
+
+/* ---------------------------------------------------------------------- */
+/* Step 1-2: token scores and block max-pooling ([P1] steps 1-2, [P3]).   */
+/*                                                                        */
+/* For each row r (absolute position t = row_pos[r], batch row_batch[r])  */
+/* and group g: pooled[r,g,c] = max over keys j in block c of             */
+/*   sum_k q_idx_rows[r,g,k] * k_idx[b, hk(g), j, k]                      */
+/* for every block c < own(t) = t / 128.  Entries c >= own(t) are NaN.    */
+/* hk(g) = 0 when h_kidx == 1 (shared index key head), else g.            */
+/* ---------------------------------------------------------------------- */
+void msa_oracle_index_pooled(int64_t n_rows, int32_t G, int32_t d_idx,
+                             int64_t n_kv, int32_t h_kidx,
+                             const uint16_t* q_idx_rows, /* [n_rows,G,d_idx] */
+                             const int64_t* row_pos, const int64_t* row_batch,
+                             const uint16_t* k_idx, /* [B',h_kidx,n_kv,d_idx] */
+                             int64_t out_stride,    /* >= number of blocks */
+                             double* pooled)        /* [n_rows,G,out_stride] */
+{
+#pragma omp parallel for collapse(2) schedule(dynamic, 1)
+  for (int64_t r = 0; r < n_rows; ++r) {
+    for (int32_t g = 0; g < G; ++g) {
+      const int64_t t = row_pos[r];
+      const int64_t own = t / MSA_BLOCK;
+      const int32_t hk = (h_kidx == 1) ? 0 : g;
+      const uint16_t* qv = q_idx_rows + (r * G + g) * (int64_t)d_idx;
+      const uint16_t* kb =
+          k_idx + ((row_batch[r] * h_kidx + hk) * n_kv) * (int64_t)d_idx;
+      double* out = pooled + (r * G + g) * out_stride;
+      double qd[256];
+      for (int32_t k = 0; k < d_idx; ++k) qd[k] = bf16_to_f64(qv[k]);
+      for (int64_t c = 0; c < out_stride; ++c) out[c] = NAN;
+      for (int64_t c = 0; c < own; ++c) {
+        double best = -INFINITY;
+        for (int64_t j = c * MSA_BLOCK; j < (c + 1) * MSA_BLOCK; ++j) {
+          const uint16_t* kv = kb + j * (int64_t)d_idx;
+          double s = 0.0;
+          for (int32_t k = 0; k < d_idx; ++k) s += qd[k] * bf16_to_f64(kv[k]);
+          if (s > best) best = s;
+        }
+        out[c] = best;
+      }
+    }
+  }
+}
+
+/* ---------------------------------------------------------------------- */
+/* Step 3: block selection ([P1] step 3; [P3] per-group top-k with the    */
+/* local block kept).  nsel = min(16, own+1).  The own block is always    */
+/* in; the other nsel-1 are the best candidates c < own ranked by         */
+/* (score descending, block index ascending).  Output is the selected     */
+/* block ids in ascending order, padded with -1 to 16.                    */
+/* ---------------------------------------------------------------------- */
+typedef struct {
+  double score;
+  int32_t idx;
+} cand_t;
+
+static int cand_cmp(const void* pa, const void* pb) {
+  const cand_t* a = (const cand_t*)pa;
+  const cand_t* b = (const cand_t*)pb;
+  if (a->score > b->score) return -1;
+  if (a->score < b->score) return 1;
+  return (a->idx < b->idx) ? -1 : (a->idx > b->idx);
+}
+
+static int int_cmp(const void* pa, const void* pb) {
+  int32_t a = *(const int32_t*)pa, b = *(const int32_t*)pb;
+  return (a > b) - (a < b);
+}
+
+void msa_oracle_select_row(int64_t own, const double* scores, int32_t* sel) {
+  int32_t out[MSA_TOPK];
+  int32_t n = 0;
+  if (own + 1 <= MSA_TOPK) {
+    for (int32_t c = 0; c <= own; ++c) out[n++] = c;
+  } else {
+    cand_t* cands = (cand_t*)malloc(sizeof(cand_t) * (size_t)own);
+    for (int64_t c = 0; c < own; ++c) {
+      cands[c].score = scores[c];
+      cands[c].idx = (int32_t)c;
+    }
+    qsort(cands, (size_t)own, sizeof(cand_t), cand_cmp);
+    for (int32_t i = 0; i < MSA_TOPK - 1; ++i) out[n++] = cands[i].idx;
+    out[n++] = (int32_t)own;
+    free(cands);
+    qsort(out, (size_t)n, sizeof(int32_t), int_cmp);
+  }
+  for (int32_t i = 0; i < MSA_TOPK; ++i) sel[i] = (i < n) ? out[i] : -1;
+}
+
+void msa_oracle_topk(int64_t n_rows, int32_t G, const int64_t* row_pos,
+                     int64_t stride, const double* pooled, /* [n_rows,G,stride] */
+                     int32_t* sel)                          /* [n_rows,G,16] */
+{
+#pragma omp parallel for collapse(2) schedule(static)
+  for (int64_t r = 0; r < n_rows; ++r)
+    for (int32_t g = 0; g < G; ++g)
+      msa_oracle_select_row(row_pos[r] / MSA_BLOCK,
+                            pooled + (r * G + g) * stride,
+                            sel + (r * G + g) * MSA_TOPK);
+}
+
+/* Same selection on fp32 scores (the scores a caller hands to the select
+ * step), so that a float-valued input is ranked exactly as given. */
+void msa_oracle_topk_f32(int64_t n_rows, int64_t stride, const int64_t* own,
+                         const float* pooled, int32_t* sel) {
+#pragma omp parallel for schedule(static)
+  for (int64_t r = 0; r < n_rows; ++r) {
+    double* tmp = (double*)malloc(sizeof(double) * (size_t)(own[r] + 1));
+    for (int64_t c = 0; c < own[r]; ++c) tmp[c] = (double)pooled[r * stride + c];
+    msa_oracle_select_row(own[r], tmp, sel + r * MSA_TOPK);
+    free(tmp);
+  }
+}
+
+/* ---------------------------------------------------------------------- */
+/* Step 4: exact softmax attention over the selected tokens ([P1] main     */
+/* branch, [P3] "exact softmax attention", [P5] softmax(QK^T/sqrt(d))V).   */
+/* For row r, head h (group g = h / (H/G), KV head g): the token set is    */
+/* the union of the selected blocks, restricted to j <= t.                 */
+/*   o = sum_j p_j v_j,  p_j = exp(s_j - m) / l,  s_j = scale * q.k_j,     */
+/*   m = max_j s_j, l = sum_j exp(s_j - m), lse = m + log(l).              */
+/* ---------------------------------------------------------------------- */
+void msa_oracle_attention(int64_t n_rows, int32_t H, int32_t G, int64_t n_kv,
+                          const uint16_t* q_rows,   /* [n_rows,H,128] */
+                          const int64_t* row_pos, const int64_t* row_batch,
+                          const uint16_t* k, const uint16_t* v, /* [B',G,n_kv,128] */
+                          const int32_t* sel,        /* [n_rows,G,16] */
+                          double scale,
+                          double* out,               /* [n_rows,H,128] */
+                          double* lse)               /* [n_rows,H] */
+{
+  const int32_t R = H / G;
+#pragma omp parallel for collapse(2) schedule(dynamic, 1)
+  for (int64_t r = 0; r < n_rows; ++r) {
+    for (int32_t h = 0; h < H; ++h) {
+      const int64_t t = row_pos[r];
+      const int32_t g = h / R;
+      const int32_t* srow = sel + (r * G + g) * MSA_TOPK;
+      const uint16_t* qh = q_rows + (r * H + h) * (int64_t)MSA_HEAD_DIM;
+      const int64_t kvbase = (row_batch[r] * G + g) * n_kv;
+      double qd[MSA_HEAD_DIM];
+      for (int32_t d = 0; d < MSA_HEAD_DIM; ++d) qd[d] = bf16_to_f64(qh[d]);
+
+      /* logits of every selected causal token */
+      double logit[MSA_TOPK * MSA_BLOCK];
+      int64_t tok[MSA_TOPK * MSA_BLOCK];
+      int32_t n = 0;
+      for (int32_t s = 0; s < MSA_TOPK; ++s) {
+        const int32_t c = srow[s];
+        if (c < 0) continue;
+        for (int64_t j = (int64_t)c * MSA_BLOCK; j < (int64_t)(c + 1) * MSA_BLOCK; ++j) {
+          if (j > t || j >= n_kv) break;
+          const uint16_t* kj = k + (kvbase + j) * MSA_HEAD_DIM;
+          double dot = 0.0;
+          for (int32_t d = 0; d < MSA_HEAD_DIM; ++d) dot += qd[d] * bf16_to_f64(kj[d]);
+          logit[n] = scale * dot;
+          tok[n] = j;
+          ++n;
+        }
+      }
+      double m = -INFINITY;
+      for (int32_t i = 0; i < n; ++i) if (logit[i] > m) m = logit[i];
+      double l = 0.0;
+      double o[MSA_HEAD_DIM];
+      for (int32_t d = 0; d < MSA_HEAD_DIM; ++d) o[d] = 0.0;
+      for (int32_t i = 0; i < n; ++i) {
+        const double p = exp(logit[i] - m);
+        l += p;
+        const uint16_t* vj = v + (kvbase + tok[i]) * MSA_HEAD_DIM;
+        for (int32_t d = 0; d < MSA_HEAD_DIM; ++d) o[d] += p * bf16_to_f64(vj[d]);
+      }
+      double* orow = out + (r * H + h) * (int64_t)MSA_HEAD_DIM;
+      for (int32_t d = 0; d < MSA_HEAD_DIM; ++d) orow[d] = o[d] / l;
+      lse[r * H + h] = m + log(l);
+    }
+  }
+}
+
+/* ---------------------------------------------------------------------- */
+/* Combination of per-block softmax pieces.  A piece s of one (query,      */
+/* head) carries m_s (max logit of its tokens), l_s = sum exp(s_j - m_s)   */
+/* and acc_s = sum exp(s_j - m_s) v_j.  Softmax over the union of the      */
+/* pieces' tokens is                                                       */
+/*   M = max_s m_s, L = sum_s l_s e^{m_s-M}, o = sum_s acc_s e^{m_s-M} / L, */
+/*   lse = M + log L.                                                      */
+/* Pieces with valid[s] == 0 are ignored.                                  */
+/* ---------------------------------------------------------------------- */
+void msa_oracle_merge(int64_t n, int32_t nslot, int32_t dim,
+                      const int32_t* valid, /* [n,nslot] */
+                      const double* m, const double* l, /* [n,nslot] */
+                      const double* acc,                /* [n,nslot,dim] */
+                      double* out, double* lse)         /* [n,dim], [n] */
+{
+#pragma omp parallel for schedule(static)
+  for (int64_t i = 0; i < n; ++i) {
+    double M = -INFINITY;
+    for (int32_t s = 0; s < nslot; ++s)
+      if (valid[i * nslot + s] && m[i * nslot + s] > M) M = m[i * nslot + s];
+    double L = 0.0;
+    for (int32_t d = 0; d < dim; ++d) out[i * dim + d] = 0.0;
+    for (int32_t s = 0; s < nslot; ++s) {
+      if (!valid[i * nslot + s]) continue;
+      const double w = exp(m[i * nslot + s] - M);
+      L += w * l[i * nslot + s];
+      for (int32_t d = 0; d < dim; ++d)
+        out[i * dim + d] += w * acc[(i * nslot + s) * dim + d];
+    }
+    for (int32_t d = 0; d < dim; ++d) out[i * dim + d] /= L;
+    lse[i] = M + log(L);
+  }
+}
+
+/* ---------------------------------------------------------------------- */
+/* Inversion of the query -> block lists into block -> query lists, the    */
+/* data structure a KV-block-outer kernel walks ([P1] "Outer Gather Q":    */
+/* all queries that chose a block are gathered and computed together).    */
+/* Segments are ordered by (batch, group, block); inside a segment the     */
+/* entries are (q << 4) | slot with q ascending.  offsets has              */
+/* B*G*nblk + 1 entries, offsets[seg] .. offsets[seg+1] bound segment seg. */
+/* ---------------------------------------------------------------------- */
+void msa_oracle_block_query_lists(int64_t B, int32_t G, int64_t n_q, int64_t nblk,
+                                  const int32_t* sel, /* [B,G,n_q,16] */
+                                  int64_t* offsets,   /* [B*G*nblk+1] */
+                                  int32_t* entries)
+{
+  const int64_t nseg = B * G * nblk;
+  int64_t* cursor = (int64_t*)calloc((size_t)nseg, sizeof(int64_t));
+  for (int64_t i = 0; i <= nseg; ++i) offsets[i] = 0;
+  for (int64_t bg = 0; bg < B * G; ++bg)
+    for (int64_t q = 0; q < n_q; ++q)
+      for (int32_t s = 0; s < MSA_TOPK; ++s) {
+        const int32_t c = sel[(bg * n_q + q) * MSA_TOPK + s];
+        if (c >= 0) offsets[bg * nblk + c + 1] += 1;
+      }
+  for (int64_t i = 0; i < nseg; ++i) offsets[i + 1] += offsets[i];
+  for (int64_t i = 0; i < nseg; ++i) cursor[i] = offsets[i];
+  for (int64_t bg = 0; bg < B * G; ++bg)
+    for (int64_t q = 0; q < n_q; ++q)
+      for (int32_t s = 0; s < MSA_TOPK; ++s) {
+        const int32_t c = sel[(bg * n_q + q) * MSA_TOPK + s];
+        if (c < 0) continue;
+        entries[cursor[bg * nblk + c]++] = (int32_t)((q << 4) | s);
+      }
+  free(cursor);
+}

@@ -1,0 +1,339 @@
+"""Pins for the CPU oracle: each test checks it against something other than
+itself -- brute force, closed forms, invariants and hand-derived fixtures.
+
+The statements pinned come from the MSA pages: "MSA 稀疏注意力三国杀"
+(section "MSA 架构：粗筛 + 精算": 128-token blocks, token scores max-pooled
+per block, 16 blocks with the own block always in, attention over the
+selected 2048 tokens; section "试过的强制规则都被砍掉": no forced sink or
+window; section "MSA 性能数据": 28.4x theoretical saving at 1M), the
+sparse-attention survey (MSA entry: per GQA group, shared index key head,
+exact softmax) and the chenxutan page (softmax(QK^T/sqrt(d))V).
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+BLOCK = 128
+
+
+def _bf16_round(x: np.ndarray) -> np.ndarray:
+    """float -> bf16 bits (round to nearest even)."""
+    f = np.ascontiguousarray(x, dtype=np.float32)
+    u = f.view(np.uint32).astype(np.uint64)
+    u = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
+    return u.astype(np.uint16)
+
+
+def _rand_bits(rng, shape, scale=1.0):
+    return _bf16_round(rng.standard_normal(shape) * scale)
+
+
+def _dense_scores(q_idx_rows, k_idx, b_of_row, hk_of_group):
+    """Full token-score matrix for each row and group via matrix products."""
+    qf = oracle.bits_to_f64(q_idx_rows)                      # [n, G, d]
+    kf = oracle.bits_to_f64(k_idx)                           # [B, hk, n_kv, d]
+    n, G, _ = qf.shape
+    out = np.empty((n, G, kf.shape[2]))
+    for r in range(n):
+        for g in range(G):
+            out[r, g] = kf[b_of_row[r], hk_of_group(g)] @ qf[r, g]
+    return out
+
+
+# ----------------------------------------------------------------------------
+# index branch: block max-pool of token scores
+# ----------------------------------------------------------------------------
+@pytest.mark.parametrize("h_kidx", [1, 3])
+def test_pooled_equals_block_max_of_dense_scores(h_kidx):
+    rng = np.random.default_rng(1)
+    B, G, d_idx, n_kv = 2, 3, 64, 700                        # ragged last block (700 = 5*128 + 60)
+    k_idx = _rand_bits(rng, (B, h_kidx, n_kv, d_idx))
+    rows = np.array([0, 127, 128, 300, 640, 699, 511, 256], np.int64)
+    bats = np.array([0, 1, 0, 1, 1, 0, 1, 0], np.int64)
+    q_rows = _rand_bits(rng, (len(rows), G, d_idx))
+    pooled = oracle.index_pooled(q_rows, rows, bats, k_idx)
+    dense = _dense_scores(q_rows, k_idx, bats, (lambda g: 0) if h_kidx == 1 else (lambda g: g))
+    nblk = oracle.num_blocks(n_kv)
+    for r, t in enumerate(rows):
+        own = t // BLOCK
+        for g in range(G):
+            for c in range(nblk):
+                if c < own:
+                    want = dense[r, g, c * BLOCK:(c + 1) * BLOCK].max()
+                    assert pooled[r, g, c] == pytest.approx(want, rel=1e-12, abs=1e-12)
+                else:
+                    assert math.isnan(pooled[r, g, c])
+
+
+def test_worked_case_index_and_selection():
+    fx = json.load(open(os.path.join(GOLD, "index_select_worked_case.json")))
+    n_kv, t = fx["n_kv"], fx["t"]
+    k = np.zeros((1, 1, n_kv, 2), np.float32)
+    k[..., 0] = -100.0
+    for c, (tok, val) in enumerate(zip(fx["plant_token_in_block"], fx["plant"])):
+        k[0, 0, c * BLOCK + tok, 0] = val
+    q = np.array([[[1.0, 0.0]]], np.float32)
+    pooled = oracle.index_pooled(_bf16_round(q), np.array([t]), np.array([0]), _bf16_round(k))
+    own = t // BLOCK
+    assert list(pooled[0, 0, :own]) == fx["expected_pooled"]
+    sel = oracle.topk(pooled, np.array([t]))
+    assert list(sel[0, 0]) == fx["expected_sel"]
+
+
+# ----------------------------------------------------------------------------
+# selection
+# ----------------------------------------------------------------------------
+def _golden_rows():
+    cases = []
+    for line in open(os.path.join(GOLD, "select_rows_f32.txt")):
+        if line.startswith("#") or not line.strip():
+            continue
+        a, b, c = line.split("|")
+        cases.append((int(a), [float(x) for x in b.split()], [int(x) for x in c.split()]))
+    return cases
+
+
+def test_selection_golden_rows():
+    cases = _golden_rows()
+    stride = max(max(own, 1) for own, _, _ in cases)
+    scores = np.full((len(cases), stride), np.nan, np.float32)
+    owns = np.array([own for own, _, _ in cases], np.int64)
+    for i, (own, sc, _) in enumerate(cases):
+        scores[i, :len(sc)] = sc
+    sel = oracle.topk_f32(scores, owns)
+    for i, (_, _, want) in enumerate(cases):
+        assert list(sel[i]) == want, (i, list(sel[i]), want)
+    # the float64 entry point ranks the same way
+    sel64 = oracle.topk(scores.astype(np.float64)[:, None, :], owns * BLOCK + 5)
+    assert (sel64[:, 0, :] == sel).all()
+
+
+def _check_selection_certificate(scores, own, sel_row):
+    """Invariants + optimality certificate of one selected row."""
+    nsel = min(16, own + 1)
+    chosen = [c for c in sel_row if c >= 0]
+    assert len(chosen) == nsel
+    assert chosen == sorted(chosen) and len(set(chosen)) == nsel
+    assert own in chosen and all(0 <= c <= own for c in chosen)
+    assert all(c == -1 for c in sel_row[nsel:])
+    picked = [c for c in chosen if c != own]
+    rejected = [c for c in range(own) if c not in picked]
+    # every rejected candidate ranks below every picked one under (score desc, idx asc)
+    for p in picked:
+        for r in rejected:
+            assert (scores[p] > scores[r]) or (scores[p] == scores[r] and p < r)
+
+
+def test_selection_certificate_random_rows():
+    rng = np.random.default_rng(2)
+    owns = np.array([0, 1, 14, 15, 16, 17, 40, 255, 1023, 2047, 3000], np.int64)
+    stride = int(owns.max())
+    sc = rng.standard_normal((len(owns), stride)).astype(np.float32)
+    sc[:, ::7] = np.round(sc[:, ::7])           # plenty of exact ties
+    sel = oracle.topk_f32(sc, owns)
+    for i, own in enumerate(owns):
+        _check_selection_certificate(sc[i].astype(np.float64), int(own), list(sel[i]))
+
+
+def test_no_sink_or_window_forcing():
+    """Only the own block is forced: a low first block or a low preceding block is dropped."""
+    own = 40
+    sc = np.linspace(1.0, 2.0, own).astype(np.float32)
+    sc[0] = -10.0
+    sc[own - 1] = -9.0
+    sel = oracle.topk_f32(sc[None, :], np.array([own]))[0]
+    assert 0 not in sel and (own - 1) not in sel and own in sel
+
+
+# ----------------------------------------------------------------------------
+# attention over the selected tokens
+# ----------------------------------------------------------------------------
+def _dense_masked_attention(q, k, v, mask, scale):
+    """softmax(q k^T * scale + log mask) v for one (row, head): numpy, float64."""
+    logits = (k @ q) * scale
+    logits = np.where(mask, logits, -np.inf)
+    m = logits.max()
+    p = np.exp(logits - m)
+    p /= p.sum()
+    return p @ v, m + math.log(np.exp(logits - m).sum())
+
+
+def _make_qkv(rng, B, n_q, n_kv, H, G, q_scale=1.0):
+    q = _rand_bits(rng, (B, n_q, H, 128), q_scale)
+    k = _rand_bits(rng, (B, G, n_kv, 128))
+    v = _rand_bits(rng, (B, G, n_kv, 128))
+    return q, k, v
+
+
+def test_sixteen_blocks_or_fewer_is_full_causal_attention():
+    """With at most 16 blocks of context every block is selected, so MSA equals
+    full causal attention (follows from the 16 x 128 budget and the forced own block)."""
+    rng = np.random.default_rng(3)
+    B, n, H, G = 1, 2048, 4, 2
+    q, k, v = _make_qkv(rng, B, n, n, H, G)
+    rows = np.array([0, 1, 127, 128, 1000, 2047], np.int64)
+    bats = np.zeros_like(rows)
+    q_rows = q[0, rows]
+    q_idx = _rand_bits(rng, (len(rows), G, 64))
+    k_idx = _rand_bits(rng, (B, 1, n, 64))
+    _, sel, out, lse = oracle.forward_rows(q_rows, q_idx, rows, bats, k, v, k_idx, 1 / math.sqrt(128))
+    kf, vf, qf = oracle.bits_to_f64(k), oracle.bits_to_f64(v), oracle.bits_to_f64(q_rows)
+    for r, t in enumerate(rows):
+        for h in range(H):
+            g = h // (H // G)
+            mask = np.arange(n) <= t
+            o, l = _dense_masked_attention(qf[r, h], kf[0, g], vf[0, g], mask, 1 / math.sqrt(128))
+            np.testing.assert_allclose(out[r, h], o, rtol=0, atol=1e-12)
+            assert abs(lse[r, h] - l) < 1e-12
+
+
+def test_attention_equals_dense_masked_attention():
+    """Sparse attention on a selected set == dense attention with the set's mask."""
+    rng = np.random.default_rng(4)
+    B, n_kv, H, G = 2, 40 * 128 + 17, 8, 2
+    q, k, v = _make_qkv(rng, B, 1, n_kv, H, G)
+    rows = np.array([n_kv - 1, 20 * 128 + 5, 16 * 128, 33 * 128 + 127], np.int64)
+    bats = np.array([0, 1, 1, 0], np.int64)
+    q_rows = _rand_bits(rng, (len(rows), H, 128), 2.0)
+    sel = np.full((len(rows), G, 16), -1, np.int32)
+    for r, t in enumerate(rows):
+        own = t // BLOCK
+        for g in range(G):
+            pick = rng.choice(own, size=min(15, own), replace=False)
+            sel[r, g, :len(pick) + 1] = np.sort(np.append(pick, own))
+    out, lse = oracle.attention(q_rows, rows, bats, k, v, sel, 1 / math.sqrt(128))
+    kf, vf, qf = oracle.bits_to_f64(k), oracle.bits_to_f64(v), oracle.bits_to_f64(q_rows)
+    for r, t in enumerate(rows):
+        for h in range(H):
+            g = h // (H // G)
+            blocks = np.arange(n_kv) // BLOCK
+            mask = np.isin(blocks, sel[r, g][sel[r, g] >= 0]) & (np.arange(n_kv) <= t)
+            o, l = _dense_masked_attention(qf[r, h], kf[bats[r], g], vf[bats[r], g], mask,
+                                           1 / math.sqrt(128))
+            np.testing.assert_allclose(out[r, h], o, rtol=0, atol=1e-12)
+            assert abs(lse[r, h] - l) < 1e-11
+
+
+def test_equal_keys_give_the_mean_of_values():
+    """All keys equal -> uniform softmax -> output is the mean of V over the selected causal tokens."""
+    rng = np.random.default_rng(5)
+    n_kv, H, G = 20 * 128, 2, 1
+    k = np.tile(_rand_bits(rng, (1, 1, 1, 128)), (1, G, n_kv, 1))
+    v = _rand_bits(rng, (1, G, n_kv, 128))
+    t = 19 * 128 + 40
+    q_rows = _rand_bits(rng, (1, H, 128))
+    sel = np.array([[[0, 2, 3, 5, 7, 8, 9, 10, 11, 12, 13, 14, 15, 16, 18, 19]]], np.int32)
+    out, lse = oracle.attention(q_rows, np.array([t]), np.array([0]), k, v, sel, 0.25)
+    toks = np.concatenate([np.arange(c * 128, min(c * 128 + 128, t + 1)) for c in sel[0, 0]])
+    want = oracle.bits_to_f64(v)[0, 0, toks].mean(axis=0)
+    for h in range(H):
+        np.testing.assert_allclose(out[0, h], want, rtol=0, atol=1e-12)
+        s = 0.25 * float(oracle.bits_to_f64(q_rows)[0, h] @ oracle.bits_to_f64(k)[0, 0, 0])
+        assert abs(lse[0, h] - (s + math.log(len(toks)))) < 1e-10
+
+
+def test_single_token_row_returns_its_value():
+    """Query 0 sees only key 0: o = v_0 and lse = scale * q.k_0."""
+    rng = np.random.default_rng(6)
+    q, k, v = _make_qkv(rng, 1, 1, 300, 4, 2)
+    sel = np.full((1, 2, 16), -1, np.int32)
+    sel[0, :, 0] = 0
+    out, lse = oracle.attention(q[0], np.array([0]), np.array([0]), k, v, sel, 0.1)
+    for h in range(4):
+        g = h // 2
+        np.testing.assert_array_equal(out[0, h], oracle.bits_to_f64(v)[0, g, 0])
+        want = 0.1 * float(oracle.bits_to_f64(q)[0, 0, h] @ oracle.bits_to_f64(k)[0, g, 0])
+        assert abs(lse[0, h] - want) < 1e-12
+
+
+def test_output_is_a_convex_combination():
+    rng = np.random.default_rng(7)
+    q, k, v = _make_qkv(rng, 1, 1, 64 * 128, 4, 1, q_scale=4.0)
+    t = 64 * 128 - 1
+    sel = np.array([[list(range(0, 60, 4)) + [63]]], np.int32)
+    out, _ = oracle.attention(q[0], np.array([t]), np.array([0]), k, v, sel, 1 / math.sqrt(128))
+    toks = np.concatenate([np.arange(c * 128, c * 128 + 128) for c in sel[0, 0]])
+    vf = oracle.bits_to_f64(v)[0, 0, toks]
+    assert (out[0] >= vf.min(axis=0) - 1e-12).all() and (out[0] <= vf.max(axis=0) + 1e-12).all()
+
+
+# ----------------------------------------------------------------------------
+# merge of softmax pieces
+# ----------------------------------------------------------------------------
+def test_merge_of_per_block_pieces_equals_attention_over_the_union():
+    """Pieces over disjoint block subsets, combined by log-sum-exp, equal the
+    attention over the union: the identity a KV-block-outer kernel needs."""
+    rng = np.random.default_rng(8)
+    n_kv, H, G = 30 * 128, 4, 1
+    q, k, v = _make_qkv(rng, 1, 1, n_kv, H, G, q_scale=3.0)
+    t = n_kv - 1
+    full = np.array([[[1, 3, 4, 6, 8, 9, 11, 13, 15, 17, 20, 22, 24, 26, 28, 29]]], np.int32)
+    out_full, lse_full = oracle.attention(q[0], np.array([t]), np.array([0]), k, v, full, 0.1)
+    # one piece per selected block (what the block-outer kernel produces)
+    S = 16
+    m = np.zeros((H, S)); l = np.zeros((H, S)); acc = np.zeros((H, S, 128))
+    for s in range(S):
+        one = np.full((1, 1, 16), -1, np.int32)
+        one[0, 0, 0] = full[0, 0, s]
+        o_s, lse_s = oracle.attention(q[0], np.array([t]), np.array([0]), k, v, one, 0.1)
+        # a piece (m, l, acc) is any triple with acc / l = o_s and m + log l = lse_s
+        scale_l = rng.uniform(0.5, 2.0)
+        l[:, s] = scale_l
+        m[:, s] = lse_s[0] - math.log(scale_l)
+        acc[:, s] = o_s[0] * scale_l
+    perm = rng.permutation(S)
+    out, lse = oracle.merge(np.ones((H, S), np.int32), m[:, perm], l[:, perm], acc[:, perm])
+    np.testing.assert_allclose(out, out_full[0], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, lse_full[0], rtol=0, atol=1e-11)
+    # invalid pieces are ignored
+    valid = np.ones((H, S), np.int32); valid[:, 5] = 0
+    m2 = m.copy(); m2[:, 5] = 1e6
+    out2, _ = oracle.merge(valid, m2, l, acc)
+    keep = [s for s in range(S) if s != 5]
+    out3, _ = oracle.merge(np.ones((H, S - 1), np.int32), m[:, keep], l[:, keep], acc[:, keep])
+    np.testing.assert_allclose(out2, out3, rtol=0, atol=1e-14)
+
+
+# ----------------------------------------------------------------------------
+# block -> query lists
+# ----------------------------------------------------------------------------
+def test_block_query_lists_against_a_stable_sort():
+    rng = np.random.default_rng(9)
+    B, G, n_q, nblk = 2, 3, 300, 7
+    sel = np.full((B, G, n_q, 16), -1, np.int32)
+    for b in range(B):
+        for g in range(G):
+            for q in range(n_q):
+                k = rng.integers(1, 8)
+                sel[b, g, q, :k] = np.sort(rng.choice(nblk, size=k, replace=False))
+    offsets, entries = oracle.block_query_lists(sel, nblk)
+    # independent construction: sort all (segment, q, slot) triples
+    bb, gg, qq, ss = np.nonzero(sel >= 0)
+    cc = sel[bb, gg, qq, ss]
+    seg = (bb * G + gg) * nblk + cc
+    order = np.lexsort((ss, qq, seg))
+    want = (qq[order] << 4) | ss[order]
+    np.testing.assert_array_equal(entries, want.astype(np.int32))
+    counts = np.bincount(seg, minlength=B * G * nblk)
+    np.testing.assert_array_equal(offsets, np.concatenate([[0], np.cumsum(counts)]))
+    assert len(entries) == (sel >= 0).sum()
+
+
+# ----------------------------------------------------------------------------
+# cost model
+# ----------------------------------------------------------------------------
+def test_cost_model_reproduces_the_pages_28x():
+    """Full/MSA attention FLOPs at 1M context.  The pages give 28.4x for the
+    109B experimental model; with R = 16 query heads per group and
+    d = d_idx = 128 (inferred, not printed), causal full attention costs
+    R*d*n/2*4 per group and query, MSA costs R*d*2048*4 + d_idx*n/2*2."""
+    n, R, d, d_idx = 2 ** 20, 16, 128, 128
+    full = R * d * (n / 2) * 4
+    msa = R * d * 2048 * 4 + d_idx * (n / 2) * 2
+    assert round(full / msa, 1) == 28.4
