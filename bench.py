@@ -1,0 +1,374 @@
+"""Benchmark of the MSA hot path on B200.
+
+One step = one pass of the whole path over one batch of synthetic input:
+index scores + block max-pool, top-16 selection, block->query lists,
+KV-block-outer attention and the log-sum-exp merge, for the 128K-token
+prefill workload (batch 1, 131072 tokens, 64 query heads / 8 KV heads,
+d_idx 128).  The headline metric is queries/s of that pass; the selected-token
+attention TFLOP/s and a decode pass (64 sequences x 256K cached tokens, one
+new token each) are reported alongside.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl msa|reference]
+
+With N > 1 (launched by torchrun) every rank runs its own independent
+instance of the workload (the problems share nothing: weak scaling, no
+collective on the data path); `value` = all ranks' queries / the slowest
+rank's time.  `--impl reference` times the CPU oracle on a bounded sample of
+rows of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    try:
+        with open(PEAKS_PATH) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return FALLBACK, "fallback"
+
+
+def work_counts(w):
+    """Algorithmic FLOPs / bytes of one pass (formulas stated in the design notes)."""
+    B, G, R, d_idx = w.batch, w.h_kv, w.h_q // w.h_kv, w.d_idx
+    t = w.q_pos0 + np.arange(w.n_q, dtype=np.int64)
+    own = t // 128
+    # index: every token of every candidate block c < own(t), per group: 2*d_idx FLOP
+    idx_flops = float(B * G * 2 * d_idx * 128 * own.sum())
+    # attention: 4*128 FLOP per (query, head, selected causal token)
+    nsel_full = np.minimum(16, own + 1)
+    # selected tokens: own block contributes t%128+1, the others 128 each
+    toks = (nsel_full - 1) * 128 + (t % 128) + 1
+    attn_flops = float(B * w.h_q * 4 * 128 * toks.sum())
+    n_entries = int(B * G * nsel_full.sum())
+    return idx_flops, attn_flops, n_entries
+
+
+def sample_clocks(stop_file, out_path):
+    cmd = ["nvidia-smi", "--query-gpu=index,clocks.sm,clocks.max.sm,power.draw,"
+           "clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+           "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+           "clocks_event_reasons.sw_power_cap", "--format=csv,noheader,nounits", "-lms", "200"]
+    try:
+        return subprocess.Popen(cmd, stdout=open(out_path, "w"), stderr=subprocess.DEVNULL)
+    except OSError:
+        return None
+
+
+def summarize_clocks(path, gpu_index):
+    sm, mx, reasons = [], [], set()
+    try:
+        for line in open(path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9 or f[0] != str(gpu_index):
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for name, val in zip(["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
+                                  "sw_power_cap"], f[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+    except OSError:
+        pass
+    if not sm:
+        return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+    return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons)}
+
+
+class Stages:
+    """CUDA events between the C-ABI calls of a step (same stream)."""
+
+    NAMES = ["index", "topk", "block_lists", "attn", "merge"]
+
+    def __init__(self):
+        self.ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(self.NAMES) + 1)]
+
+    def ms(self):
+        return {n: self.ev[i].elapsed_time(self.ev[i + 1]) for i, n in enumerate(self.NAMES)}
+
+
+def run_step(pipeline, capi, buf, inp, stages=None):
+    d = buf.dims
+    ev = stages.ev if stages else None
+    if ev: ev[0].record()
+    capi.msa_index_score_maxpool(d, inp["q_idx"], inp["k_idx"], buf.pooled, buf.pooled_stride,
+                                 buf.dev_err)
+    if ev: ev[1].record()
+    capi.msa_topk_blocks(d, buf.pooled, buf.pooled_stride, buf.sel, buf.dev_err)
+    if ev: ev[2].record()
+    capi.msa_build_block_query_lists(d, buf.sel, buf.blk_offsets, buf.entries, buf.ws,
+                                     buf.dev_err)
+    if ev: ev[3].record()
+    capi.msa_sparse_attn_fwd(d, inp["q"], inp["k"], inp["v"], buf.blk_offsets, buf.entries,
+                             buf.part_ml, buf.part_acc, buf.dev_err)
+    if ev: ev[4].record()
+    capi.msa_merge_partials(d, buf.sel, buf.part_ml, buf.part_acc, buf.out, buf.lse,
+                            buf.dev_err)
+    if ev: ev[5].record()
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def bench_workload(w, steps, warmup, world, rank, with_e2e=True):
+    from block_sparse_attention_32_b200 import capi, pipeline, workloads as wl
+    d = pipeline.dims_for(w)
+    buf = pipeline.Buffers.allocate(d)
+    inp = wl.make_inputs(w, "cuda")
+    torch.cuda.synchronize()
+    for _ in range(warmup):
+        run_step(pipeline, capi, buf, inp)
+    torch.cuda.synchronize()
+    if int(buf.dev_err[0]) != 0:
+        raise RuntimeError(f"device error {int(buf.dev_err[0])} during warm-up")
+
+    stages = [Stages() for _ in range(steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    start.record()
+    for s in range(steps):
+        run_step(pipeline, capi, buf, inp, stages[s])
+    end.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    total_ms = start.elapsed_time(end)
+    per_stage = {n: statistics.median(st.ms()[n] for st in stages) for n in Stages.NAMES}
+    per_stage_mean = {n: sum(st.ms()[n] for st in stages) / steps for n in Stages.NAMES}
+    if int(buf.dev_err[0]) != 0:
+        raise RuntimeError(f"device error {int(buf.dev_err[0])} during timing")
+
+    e2e = None
+    if with_e2e:
+        e2e = bench_e2e(w, buf, inp, max(2, min(steps, 3)), world)
+    del inp
+    del buf
+    torch.cuda.empty_cache()
+    return total_ms, per_stage, per_stage_mean, e2e
+
+
+def bench_e2e(w, buf, dev_inp, steps, world):
+    """Same pass through the C ABI with host buffers: pinned H2D of the inputs,
+    the five calls, D2H of the output and lse, all inside the timed region."""
+    from block_sparse_attention_32_b200 import capi, pipeline
+    host = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in dev_inp.items()}
+    for k, v in dev_inp.items():
+        host[k].copy_(v)
+    out_h = torch.empty(buf.out.shape, dtype=buf.out.dtype, pin_memory=True)
+    lse_h = torch.empty(buf.lse.shape, dtype=buf.lse.dtype, pin_memory=True)
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_h.numel() * out_h.element_size() + lse_h.numel() * lse_h.element_size()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    start.record()
+    for _ in range(steps):
+        for k in dev_inp:
+            dev_inp[k].copy_(host[k], non_blocking=True)
+        run_step(pipeline, capi, buf, dev_inp)
+        out_h.copy_(buf.out, non_blocking=True)
+        lse_h.copy_(buf.lse, non_blocking=True)
+    end.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(start.elapsed_time(end) / steps, world)
+    return {"ms_per_step": ms, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+
+class CpuOracleSample:
+    """The oracle, as it stands, on a bounded sample of the workload's query rows."""
+
+    def __init__(self, w, n_rows=16, seed=0):
+        import oracle
+        from block_sparse_attention_32_b200 import workloads as wl
+        self.oracle, self.w = oracle, w
+        inp = wl.make_inputs(w, "cpu")
+        rng = np.random.default_rng(seed)
+        self.rows = np.sort(rng.choice(w.n_q, size=min(n_rows, w.n_q), replace=False)).astype(np.int64)
+        bits = oracle.bf16_bits
+        self.k, self.v, self.ki = bits(inp["k"]), bits(inp["v"]), bits(inp["k_idx"])
+        self.q_rows = bits(inp["q"][0, self.rows])
+        self.qi_rows = bits(inp["q_idx"][0, self.rows])
+        self.pos = w.q_pos0 + self.rows
+        self.bat = np.zeros_like(self.rows)
+
+    def run(self):
+        t0 = time.perf_counter()
+        self.oracle.forward_rows(self.q_rows, self.qi_rows, self.pos, self.bat, self.k, self.v,
+                                 self.ki, self.w.scale)
+        dt = time.perf_counter() - t0
+        cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+        w = self.w
+        return {"value": len(self.rows) / dt, "unit": "queries/s", "cores": cores,
+                "kind": "oracle",
+                "sample": f"{len(self.rows)} random query rows of {w.name} (all {w.h_kv} groups, "
+                          f"{w.h_q} heads): fp64 index scores + selection + attention; "
+                          f"{dt:.1f} s"}
+
+
+def cpu_baseline(w, n_rows=16):
+    return CpuOracleSample(w, n_rows).run()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="msa", choices=["msa", "reference"])
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    args = ap.parse_args()
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    from block_sparse_attention_32_b200 import workloads as wl
+    w = wl.P128
+    idx_flops, attn_flops, n_ent = work_counts(w)
+    peaks, peak_src = load_peaks()
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        sample = CpuOracleSample(w, n_rows=4)
+        vals = []
+        for _ in range(args.warmup):
+            sample.run()
+        for _ in range(args.steps):
+            vals.append(sample.run())
+        v = statistics.median(x["value"] for x in vals)
+        line = {"impl": "reference", "metric": "prefill_128k_queries_per_s", "value": v,
+                "unit": "queries/s", "n_gpus": 0, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": 1000.0 * 4 / v, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "config": {"workload": w.name, "batch": w.batch, "seq_len": w.n_kv,
+                           "h_q": w.h_q, "h_kv": w.h_kv, "d_idx": w.d_idx, "topk_blocks": 16,
+                           "block": 128},
+                "cpu_baseline": dict(vals[-1], value=v),
+                "e2e": {"value": v, "unit": "queries/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line))
+        return
+
+    if world > 1:
+        torch.distributed.init_process_group("nccl", device_id=torch.device("cuda", local),
+                                             timeout=__import__("datetime").timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    import __graft_entry__
+    __graft_entry__.build()
+
+    clk_path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{rank}.csv")
+    os.makedirs(os.path.dirname(clk_path), exist_ok=True)
+    proc = sample_clocks(None, clk_path) if rank == 0 else None
+    total_ms, stage_med, stage_mean, e2e = bench_workload(w, args.steps, args.warmup, world, rank)
+    if proc is not None:
+        proc.terminate()
+        proc.wait()
+    clocks = summarize_clocks(clk_path, local) if rank == 0 else None
+
+    total_ms = max_over_ranks(total_ms, world)
+    ms_step = total_ms / args.steps
+    qps = world * w.n_q / (ms_step / 1000.0)
+
+    decode = None
+    if not args.no_decode:
+        dw = wl.DECODE
+        dms, dstage, _, _ = bench_workload(dw, max(3, args.steps), args.warmup, world, rank,
+                                           with_e2e=False)
+        dms = max_over_ranks(dms, world) / max(3, args.steps)
+        kidx_bytes = dw.batch * dw.n_kv * dw.d_idx * 2
+        sel_kv_bytes = dw.batch * dw.h_kv * 16 * 128 * 128 * 2 * 2
+        decode = {"workload": dw.name, "tokens_per_s": world * dw.batch / (dms / 1000.0),
+                  "ms_per_step": dms, "stages_ms": dstage,
+                  "index_scan_gbs": kidx_bytes / (dstage["index"] / 1000.0) / 1e9,
+                  "bytes_read_per_step": kidx_bytes + sel_kv_bytes}
+
+    if rank != 0:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
+
+    # dominant kernel: the longest stage
+    dom = max(stage_mean, key=stage_mean.get)
+    sustained = peaks.get("bf16_tflops_sustained", FALLBACK["bf16_tflops_sustained"])
+    if dom in ("index", "attn"):
+        flops = idx_flops if dom == "index" else attn_flops
+        ach = flops / (stage_mean[dom] / 1000.0) / 1e12
+        roof = {"kernel": dom, "bound": "tensor", "achieved": ach, "peak": sustained,
+                "unit": "TFLOP/s", "frac": ach / sustained, "traffic": None,
+                "peak_source": f"{peak_src} bf16_tflops_sustained"}
+    else:
+        part_bytes = w.batch * w.n_q * w.h_q * 16 * (128 + 2) * 4
+        byts = {"merge": part_bytes + w.batch * w.n_q * w.h_q * (256 + 4) + n_ent * 4,
+                "topk": w.batch * w.h_kv * (idx_flops / (2 * w.d_idx * 128 * w.batch * w.h_kv)) * 4,
+                "block_lists": n_ent * 4 * 4}[dom]
+        ach = byts / (stage_mean[dom] / 1000.0) / 1e9
+        roof = {"kernel": dom, "bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": ach / peaks["hbm_gbs"], "traffic": None,
+                "peak_source": f"{peak_src} hbm_gbs"}
+
+    attn_tflops = attn_flops / (stage_mean["attn"] / 1000.0) / 1e12
+    attn_merge_tflops = attn_flops / ((stage_mean["attn"] + stage_mean["merge"]) / 1000.0) / 1e12
+    line = {
+        "metric": "prefill_128k_queries_per_s", "value": qps, "unit": "queries/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.batch, "seq_len": w.n_kv, "h_q": w.h_q,
+                   "h_kv": w.h_kv, "d_idx": w.d_idx, "topk_blocks": 16, "block": 128,
+                   "parallelism": f"replicas{world}",
+                   "l2": "inputs larger than L2 (partials 69 GB per pass)"},
+        "selected_token_attn_tflops": attn_tflops,
+        "selected_token_attn_merge_tflops": attn_merge_tflops,
+        "index_tflops": idx_flops / (stage_mean["index"] / 1000.0) / 1e12,
+        "stages_ms": stage_mean,
+        "decode": decode,
+        "roofline": roof,
+        "clocks": clocks,
+        "gpu_launches": args.steps * 8,
+        "e2e": {"value": world * w.n_q / (e2e["ms_per_step"] / 1000.0), "unit": "queries/s",
+                "h2d_bytes_per_step": e2e["h2d_bytes_per_step"],
+                "d2h_bytes_per_step": e2e["d2h_bytes_per_step"]} if e2e else None,
+    }
+    if not args.no_cpu:
+        line["cpu_baseline"] = cpu_baseline(w)
+    print(json.dumps(line))
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,155 @@
+"""Thin ctypes binding of ``libmsa.so`` -- argument marshalling only.
+
+Each function has the name of the C entry point it calls (``include/msa.h``)
+and takes torch CUDA tensors; it passes raw device pointers, element strides
+and the current CUDA stream, raises ``MSAError`` on a non-OK status, and does
+no arithmetic of its own.  If the library is missing this module raises on
+first use: there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "lib", "libmsa.so")
+
+BLOCK = 128
+TOPK = 16
+HEAD_DIM = 128
+
+STATUS = {0: "MSA_OK", 1: "MSA_ERR_INVALID_ARG", 2: "MSA_ERR_UNSUPPORTED",
+          3: "MSA_ERR_ALIGNMENT", 4: "MSA_ERR_WORKSPACE_TOO_SMALL", 5: "MSA_ERR_CUDA"}
+DEVERR = {1: "MSA_DEVERR_TIMEOUT", 2: "MSA_DEVERR_BAD_BLOCK", 3: "MSA_DEVERR_BAD_ENTRY"}
+
+
+class MSAError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} returned {STATUS.get(status, status)}")
+        self.status = status
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int64), ("n_q", ctypes.c_int64), ("n_kv", ctypes.c_int64),
+                ("q_pos0", ctypes.c_int64), ("h_q", ctypes.c_int32), ("h_kv", ctypes.c_int32),
+                ("h_kidx", ctypes.c_int32), ("d_idx", ctypes.c_int32), ("scale", ctypes.c_float)]
+
+
+class Tensor(ctypes.Structure):
+    _fields_ = [("ptr", ctypes.c_void_p), ("s_batch", ctypes.c_int64), ("s_tok", ctypes.c_int64),
+                ("s_head", ctypes.c_int64)]
+
+
+_lib = None
+_lock = threading.Lock()
+_P = ctypes.c_void_p
+_PD = ctypes.POINTER(Dims)
+
+
+def lib() -> ctypes.CDLL:
+    """Load libmsa.so (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(
+                    f"{LIB_PATH} is missing: build it with "
+                    "`python -m block_sparse_attention_32_b200.build` (no CPU fallback exists)")
+            L = ctypes.CDLL(LIB_PATH)
+            L.msa_num_blocks.argtypes = [_PD]
+            L.msa_num_blocks.restype = ctypes.c_int64
+            L.msa_num_entries.argtypes = [_PD]
+            L.msa_num_entries.restype = ctypes.c_int64
+            L.msa_index_score_maxpool.argtypes = [_PD, Tensor, Tensor, _P, ctypes.c_int64, _P, _P]
+            L.msa_topk_blocks.argtypes = [_PD, _P, ctypes.c_int64, _P, _P, _P]
+            L.msa_block_query_lists_workspace.argtypes = [_PD]
+            L.msa_block_query_lists_workspace.restype = ctypes.c_size_t
+            L.msa_build_block_query_lists.argtypes = [_PD, _P, _P, _P, _P, ctypes.c_size_t, _P, _P]
+            L.msa_sparse_attn_fwd.argtypes = [_PD, Tensor, Tensor, Tensor, _P, _P, _P, _P, _P, _P]
+            L.msa_merge_partials.argtypes = [_PD, _P, _P, _P, _P, _P, _P, _P]
+            L.msa_status_string.argtypes = [ctypes.c_int]
+            L.msa_status_string.restype = ctypes.c_char_p
+            for f in (L.msa_index_score_maxpool, L.msa_topk_blocks, L.msa_build_block_query_lists,
+                      L.msa_sparse_attn_fwd, L.msa_merge_partials):
+                f.restype = ctypes.c_int
+            _lib = L
+    return _lib
+
+
+def make_dims(batch, n_q, n_kv, q_pos0, h_q, h_kv, d_idx, h_kidx=1, scale=None) -> Dims:
+    if scale is None:
+        scale = HEAD_DIM ** -0.5
+    return Dims(batch, n_q, n_kv, q_pos0, h_q, h_kv, h_kidx, d_idx, scale)
+
+
+def _ptr(t) -> int:
+    return 0 if t is None else t.data_ptr()
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def tensor_btd(t: torch.Tensor) -> Tensor:
+    """[B, T, H, D] layout (q, q_idx)."""
+    assert t.dim() == 4 and t.stride(3) == 1 and t.dtype == torch.bfloat16 and t.is_cuda
+    return Tensor(t.data_ptr(), t.stride(0), t.stride(1), t.stride(2))
+
+
+def tensor_bhtd(t: torch.Tensor) -> Tensor:
+    """[B, H, T, D] layout (k, v, k_idx)."""
+    assert t.dim() == 4 and t.stride(3) == 1 and t.dtype == torch.bfloat16 and t.is_cuda
+    return Tensor(t.data_ptr(), t.stride(0), t.stride(2), t.stride(1))
+
+
+def _check(fn, status):
+    if status != 0:
+        raise MSAError(fn, status)
+
+
+def msa_num_blocks(d: Dims) -> int:
+    return lib().msa_num_blocks(ctypes.byref(d))
+
+
+def msa_num_entries(d: Dims) -> int:
+    return lib().msa_num_entries(ctypes.byref(d))
+
+
+def msa_block_query_lists_workspace(d: Dims) -> int:
+    return lib().msa_block_query_lists_workspace(ctypes.byref(d))
+
+
+def msa_index_score_maxpool(d: Dims, q_idx, k_idx, pooled, pooled_row_stride, dev_err=None):
+    _check("msa_index_score_maxpool",
+           lib().msa_index_score_maxpool(ctypes.byref(d), tensor_btd(q_idx), tensor_bhtd(k_idx),
+                                         _ptr(pooled), pooled_row_stride, _ptr(dev_err), _stream()))
+
+
+def msa_topk_blocks(d: Dims, pooled, pooled_row_stride, sel, dev_err=None):
+    _check("msa_topk_blocks",
+           lib().msa_topk_blocks(ctypes.byref(d), _ptr(pooled), pooled_row_stride, _ptr(sel),
+                                 _ptr(dev_err), _stream()))
+
+
+def msa_build_block_query_lists(d: Dims, sel, blk_offsets, entries, ws, dev_err=None):
+    nbytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check("msa_build_block_query_lists",
+           lib().msa_build_block_query_lists(ctypes.byref(d), _ptr(sel), _ptr(blk_offsets),
+                                             _ptr(entries), _ptr(ws), nbytes, _ptr(dev_err),
+                                             _stream()))
+
+
+def msa_sparse_attn_fwd(d: Dims, q, k, v, blk_offsets, entries, part_ml, part_acc, dev_err=None):
+    _check("msa_sparse_attn_fwd",
+           lib().msa_sparse_attn_fwd(ctypes.byref(d), tensor_btd(q), tensor_bhtd(k),
+                                     tensor_bhtd(v), _ptr(blk_offsets), _ptr(entries),
+                                     _ptr(part_ml), _ptr(part_acc), _ptr(dev_err), _stream()))
+
+
+def msa_merge_partials(d: Dims, sel, part_ml, part_acc, out, lse, dev_err=None):
+    _check("msa_merge_partials",
+           lib().msa_merge_partials(ctypes.byref(d), _ptr(sel), _ptr(part_ml), _ptr(part_acc),
+                                    _ptr(out), _ptr(lse), _ptr(dev_err), _stream()))

@@ -1,0 +1,167 @@
+// Inversion of the per-query block lists into per-block query lists (CSR),
+// the index the KV-block-outer attention kernel walks.
+//
+// Source: page "MSA 稀疏注意力三国杀", section "Kernel 创新：Outer Gather Q":
+// the KV block is the outer loop and all queries that chose it are gathered
+// and computed together, so each block is read once.  The inversion itself is
+// not spelled out on the pages; this is a deterministic counting sort.
+//
+// Segments are (batch, group, block) in that order; inside a segment the
+// entries (i << 4 | slot) are ascending in the query index i.  Steps:
+//   1. count:   per 128-query tile, a shared-memory histogram over blocks;
+//   2. colscan: per block, exclusive prefix over tiles (in place) + totals;
+//   3. offsets: exclusive scan of the totals over all segments;
+//   4. scatter: per tile, queries in ascending order claim consecutive slots
+//      of each block's range, so the order never depends on timing.
+// Workspace: tile histograms [B*G, ntiles, nblk] + totals [B*G*nblk], int32.
+#include "common.cuh"
+
+namespace msa {
+
+constexpr int kCsrTile = 128;   // queries per tile
+
+__global__ void __launch_bounds__(256)
+    csr_count_kernel(const int32_t* __restrict__ sel, int64_t n_q, int64_t q_pos0,
+                     int32_t nblk, int32_t ntiles, int32_t* __restrict__ tile_counts,
+                     int32_t* err) {
+  extern __shared__ int32_t hist[];
+  const int tile = blockIdx.x;
+  const int64_t bg = blockIdx.y;
+  for (int c = threadIdx.x; c < nblk; c += blockDim.x) hist[c] = 0;
+  __syncthreads();
+  const int64_t q0 = (int64_t)tile * kCsrTile;
+  const int64_t nq = min64(kCsrTile, n_q - q0);
+  const int32_t* srow = sel + (bg * n_q + q0) * kTopK;
+  for (int idx = threadIdx.x; idx < nq * kTopK; idx += blockDim.x) {
+    const int32_t c = srow[idx];
+    if (c < 0) continue;
+    const int64_t own = (q_pos0 + q0 + idx / kTopK) / kBlock;
+    if (c > own || c >= nblk) {
+      report(err, MSA_DEVERR_BAD_BLOCK);
+      continue;
+    }
+    atomicAdd(&hist[c], 1);
+  }
+  __syncthreads();
+  int32_t* dst = tile_counts + (bg * ntiles + tile) * (int64_t)nblk;
+  for (int c = threadIdx.x; c < nblk; c += blockDim.x) dst[c] = hist[c];
+}
+
+__global__ void __launch_bounds__(256)
+    csr_colscan_kernel(int32_t* __restrict__ tile_counts, int32_t* __restrict__ totals,
+                       int32_t nblk, int32_t ntiles) {
+  const int c = blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t bg = blockIdx.y;
+  if (c >= nblk) return;
+  int32_t* col = tile_counts + bg * ntiles * (int64_t)nblk + c;
+  int32_t run = 0;
+  for (int t = 0; t < ntiles; ++t) {
+    const int32_t v = col[(int64_t)t * nblk];
+    col[(int64_t)t * nblk] = run;
+    run += v;
+  }
+  totals[bg * nblk + c] = run;
+}
+
+// single block, 1024 threads: exclusive scan of n values into out[0..n]
+__global__ void __launch_bounds__(1024)
+    csr_offsets_kernel(const int32_t* __restrict__ totals, int64_t n,
+                       int32_t* __restrict__ offsets) {
+  __shared__ int32_t warp_sums[32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t per = (n + 1023) / 1024;
+  const int64_t lo = min64(n, tid * per), hi = min64(n, lo + per);
+  int32_t s = 0;
+  for (int64_t i = lo; i < hi; ++i) s += totals[i];
+  // block exclusive scan of s
+  int32_t incl = s;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (lane == 31) warp_sums[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int32_t w = warp_sums[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int32_t v = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += v;
+    }
+    warp_sums[lane] = w;   // inclusive over warps
+  }
+  __syncthreads();
+  int32_t run = incl - s + (warp > 0 ? warp_sums[warp - 1] : 0);
+  for (int64_t i = lo; i < hi; ++i) {
+    offsets[i] = run;
+    run += totals[i];
+  }
+  if (tid == 1023) offsets[n] = warp_sums[31];
+}
+
+__global__ void __launch_bounds__(32)
+    csr_scatter_kernel(const int32_t* __restrict__ sel, int64_t n_q, int64_t q_pos0,
+                       int32_t nblk, int32_t ntiles, const int32_t* __restrict__ tile_counts,
+                       const int32_t* __restrict__ offsets, int32_t* __restrict__ entries,
+                       int64_t cap) {
+  extern __shared__ int32_t base[];
+  const int tile = blockIdx.x;
+  const int64_t bg = blockIdx.y;
+  const int lane = threadIdx.x;
+  const int32_t* tc = tile_counts + (bg * ntiles + tile) * (int64_t)nblk;
+  const int32_t* off = offsets + bg * nblk;
+  for (int c = lane; c < nblk; c += 32) base[c] = off[c] + tc[c];
+  __syncwarp();
+  const int64_t q0 = (int64_t)tile * kCsrTile;
+  const int64_t nq = min64(kCsrTile, n_q - q0);
+  for (int64_t i = 0; i < nq; ++i) {
+    const int64_t qi = q0 + i;
+    if (lane < kTopK) {
+      const int32_t c = sel[(bg * n_q + qi) * kTopK + lane];
+      const int64_t own = (q_pos0 + qi) / kBlock;
+      if (c >= 0 && c <= own && c < nblk) {
+        const int32_t p = base[c];
+        base[c] = p + 1;                // blocks within one row are distinct
+        if (p >= 0 && p < cap) entries[p] = (int32_t)((qi << 4) | lane);
+      }
+    }
+    __syncwarp();
+  }
+}
+
+size_t block_lists_workspace(int64_t bgcount, int64_t n_q, int64_t nblk) {
+  const int64_t ntiles = (n_q + kCsrTile - 1) / kCsrTile;
+  return (size_t)(bgcount * nblk * (ntiles + 1)) * sizeof(int32_t);
+}
+
+cudaError_t launch_block_lists(const int32_t* sel, int64_t bgcount, int64_t n_q,
+                               int64_t q_pos0, int64_t nblk, int32_t* offsets,
+                               int32_t* entries, int64_t cap, void* ws, int32_t* err,
+                               cudaStream_t st) {
+  const int64_t ntiles = (n_q + kCsrTile - 1) / kCsrTile;
+  int32_t* tile_counts = reinterpret_cast<int32_t*>(ws);
+  int32_t* totals = tile_counts + bgcount * ntiles * nblk;
+  const size_t hist_bytes = (size_t)nblk * sizeof(int32_t);
+  cudaError_t e;
+  if (hist_bytes > 48 * 1024) {
+    e = cudaFuncSetAttribute(csr_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)hist_bytes);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(csr_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)hist_bytes);
+    if (e != cudaSuccess) return e;
+  }
+  dim3 g1((unsigned)ntiles, (unsigned)bgcount);
+  csr_count_kernel<<<g1, 256, hist_bytes, st>>>(sel, n_q, q_pos0, (int32_t)nblk,
+                                                (int32_t)ntiles, tile_counts, err);
+  dim3 g2((unsigned)((nblk + 255) / 256), (unsigned)bgcount);
+  csr_colscan_kernel<<<g2, 256, 0, st>>>(tile_counts, totals, (int32_t)nblk, (int32_t)ntiles);
+  csr_offsets_kernel<<<1, 1024, 0, st>>>(totals, bgcount * nblk, offsets);
+  csr_scatter_kernel<<<g1, 32, hist_bytes, st>>>(sel, n_q, q_pos0, (int32_t)nblk,
+                                                 (int32_t)ntiles, tile_counts, offsets, entries,
+                                                 cap);
+  return cudaGetLastError();
+}
+
+}  // namespace msa

@@ -1,0 +1,329 @@
+// Index branch: token scores q_idx . k_idx and causal block max-pool, without
+// ever storing the score matrix.
+//
+// Source: page "MSA 稀疏注意力三国杀", section "MSA 架构：粗筛 + 精算", first
+// step items 1-2 (score every token of a 128-token block, the block's score is
+// its highest token score); sparse-attention survey page, MSA entry (one index
+// query head per GQA group, shared index key head, block max-pool).
+//
+// Two kernels:
+//  * index_score_maxpool_kernel -- prefill / chunked prefill.  A 128-query x
+//    128-key tile of scores is one tcgen05 MMA (M=128, N=128, K=d_idx) whose
+//    fp32 accumulator lives in TMEM; the block max is the row max of that
+//    tile, read back with tcgen05.ld (one thread per query row).  Warp roles:
+//    warp 0 issues TMA loads (q_idx tile once, k_idx blocks through a 4-stage
+//    ring), warp 1 issues the MMAs into 4 TMEM accumulators, warps 2-9 reduce
+//    the accumulators (two groups alternating blocks) and stage the maxima in
+//    shared memory, which is written out row-contiguously at the end.
+//  * index_score_decode_kernel -- one query per sequence (decode): a
+//    streaming scan of k_idx, HBM-bound.  Each warp reads 16-key tiles
+//    straight into mma.sync fragments (16-byte loads) and multiplies them by
+//    the G <= 8 index queries of the sequence (m16n8k16: keys x groups).
+#include "common.cuh"
+
+namespace msa {
+
+template <int D>
+struct IdxCfg {
+  static constexpr int kHalves = D / 64;            // 128-byte column panels
+  static constexpr int kTileBytes = 128 * D * 2;    // 128 rows of d_idx bf16
+  static constexpr int kStages = 4;                 // k_idx ring depth
+  static constexpr int kChunkBlocks = 64;           // key blocks per CTA
+  static constexpr int kAcc = 4;                    // TMEM accumulators (128 columns each)
+  static constexpr int kStageStride = kChunkBlocks + 1;
+  static constexpr int kThreads = 320;              // 10 warps
+  static constexpr int kSmemBytes =
+      1024 + kTileBytes * (1 + kStages) + 128 * kStageStride * 4 + 17 * 8 + 16;
+};
+
+template <int D>
+__global__ void __launch_bounds__(320, 1)
+    index_score_maxpool_kernel(const __grid_constant__ CUtensorMap tm_q,
+                               const __grid_constant__ CUtensorMap tm_k, int64_t n_q,
+                               int64_t q_pos0, int32_t G, int32_t h_kidx, int32_t n_qtiles,
+                               float* __restrict__ pooled, int64_t stride, int32_t* err) {
+  using C = IdxCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* sq = base;
+  uint8_t* sk = base + C::kTileBytes;
+  float* stage = reinterpret_cast<float*>(sk + C::kStages * C::kTileBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(stage + 128 * C::kStageStride);
+  uint64_t* full = bars;          // [4] k stage loaded
+  uint64_t* empty = bars + 4;     // [4] k stage consumed by the MMAs
+  uint64_t* qfull = bars + 8;     // q tile loaded
+  uint64_t* accfull = bars + 9;   // [4] accumulator ready
+  uint64_t* accempty = bars + 13; // [4] accumulator drained
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 17);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = blockIdx.x % G;
+  const int kc = blockIdx.x / G;
+  const int qt = n_qtiles - 1 - (int)blockIdx.y;   // longest rows first
+  const int b = blockIdx.z;
+  const int64_t q0 = (int64_t)qt * 128;
+  const int64_t q_last = min64(q0 + 127, n_q - 1);
+  const int64_t nb_tile = (q_pos0 + q_last) / kBlock;   // candidates of the tile's last row
+  const int64_t c0 = (int64_t)kc * C::kChunkBlocks;
+  if (c0 >= nb_tile) return;                            // uniform: nothing to score
+  const int nb = (int)min64(C::kChunkBlocks, nb_tile - c0);
+  const int hk = (h_kidx == 1) ? 0 : g;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(full + i, 1);
+      mbar_init(empty + i, 1);
+      mbar_init(accfull + i, 1);
+      mbar_init(accempty + i, 4);
+    }
+    mbar_init(qfull, 1);
+    *abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      prefetch_tensormap(&tm_q);
+      prefetch_tensormap(&tm_k);
+      mbar_arrive_expect_tx(qfull, C::kTileBytes);
+      for (int h = 0; h < C::kHalves; ++h)
+        tma_load_4d(sq + h * 16384, &tm_q, qfull, h * 64, g, (int32_t)q0, b);
+      for (int i = 0; i < nb; ++i) {
+        const int s = i % C::kStages;
+        if (i >= C::kStages &&
+            !mbar_wait(empty + s, ((i / C::kStages) - 1) & 1, abort_flag, err))
+          break;
+        mbar_arrive_expect_tx(full + s, C::kTileBytes);
+        for (int h = 0; h < C::kHalves; ++h)
+          tma_load_4d(sk + s * C::kTileBytes + h * 16384, &tm_k, full + s, h * 64,
+                      (int32_t)((c0 + i) * kBlock), hk, b);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(128, 128, 0);
+      const uint32_t qa = smem_u32(sq);
+      bool ok = mbar_wait(qfull, 0, abort_flag, err);
+      for (int i = 0; ok && i < nb; ++i) {
+        const int s = i % C::kStages, a = i % C::kAcc;
+        if (!mbar_wait(full + s, (i / C::kStages) & 1, abort_flag, err)) break;
+        if (i >= C::kAcc && !mbar_wait(accempty + a, ((i / C::kAcc) - 1) & 1, abort_flag, err))
+          break;
+        tc_fence_after();
+        const uint32_t ka = smem_u32(sk + s * C::kTileBytes);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          umma_bf16(tmem + a * 128, smem_desc_sw128(qa + off, 16, 1024),
+                    smem_desc_sw128(ka + off, 16, 1024), idesc, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(empty + s);
+        umma_commit(accfull + a);
+      }
+    }
+  } else {
+    const int grp = (warp - 2) >> 2;     // accumulators a with a % 2 == grp
+    const int quarter = warp & 3;        // TMEM lanes 32*quarter .. +31
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    for (int i = grp; i < nb; i += 2) {
+      const int a = i % C::kAcc;
+      if (!mbar_wait(accfull + a, (i / C::kAcc) & 1, abort_flag, err)) break;
+      tc_fence_after();
+      float m = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(tmem + lane_base + a * 128 + j * 32, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int x = 0; x < 32; ++x) m = fmaxf(m, u2f(r[x]));
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(accempty + a);
+      stage[row * C::kStageStride + i] = m;
+    }
+  }
+  __syncthreads();
+
+  // row-contiguous write-out of the staged block maxima (only blocks c < own(t))
+  float* prow = pooled + ((int64_t)b * G + g) * n_q * stride;
+  for (int idx = threadIdx.x; idx < 128 * nb; idx += C::kThreads) {
+    const int r = idx / nb, i = idx - r * nb;
+    const int64_t q = q0 + r;
+    if (q >= n_q) continue;
+    const int64_t c = c0 + i;
+    if (c < (q_pos0 + q) / kBlock) prow[q * stride + c] = stage[r * C::kStageStride + i];
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// decode: one query per sequence, d_idx = 128, shared index key head, G <= 8
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
+__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint32_t a1,
+                                               uint32_t a2, uint32_t a3, uint32_t b0,
+                                               uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+      "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t u4get(const uint4& v, int i) {
+  return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
+}
+
+// Fragment trick: the reduction over the 128 index dimensions is order-free,
+// so the k index of the m16n8k16 fragments is mapped to physical dimensions
+// such that every thread reads 64 contiguous bytes of each of its two key
+// rows: at k-step s, thread column-group cq covers logical k {2cq, 2cq+1} ->
+// dims 32cq + 4s + {0,1} and logical k {2cq+8, 2cq+9} -> dims 32cq + 4s + {2,3}.
+// A (keys) and B (index queries) use the same map.
+constexpr int kDecodeBlocksPerWarp = 4;
+
+__global__ void __launch_bounds__(128)
+    index_score_decode_kernel(const __nv_bfloat16* __restrict__ q_idx, int64_t qs_b,
+                              int64_t qs_h, const __nv_bfloat16* __restrict__ k_idx,
+                              int64_t ks_b, int64_t ks_t, int64_t q_pos0, int32_t G,
+                              float* __restrict__ pooled, int64_t stride) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int b = blockIdx.y;
+  const int64_t own = q_pos0 / kBlock;
+  const int64_t cbeg = ((int64_t)blockIdx.x * 4 + warp) * kDecodeBlocksPerWarp;
+  if (cbeg >= own) return;
+  const int64_t cend = min64(cbeg + kDecodeBlocksPerWarp, own);
+  const int gq = lane >> 2, cq = lane & 3;
+
+  uint4 qv[4];
+  if (gq < G) {
+    const __nv_bfloat16* qp = q_idx + (int64_t)b * qs_b + (int64_t)gq * qs_h + 32 * cq;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) qv[i] = *reinterpret_cast<const uint4*>(qp + 8 * i);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) qv[i] = make_uint4(0, 0, 0, 0);
+  }
+
+  for (int64_t c = cbeg; c < cend; ++c) {
+    const __nv_bfloat16* kb = k_idx + (int64_t)b * ks_b + (c * kBlock) * ks_t + 32 * cq;
+    float mx0 = -INFINITY, mx1 = -INFINITY;
+    uint4 cur[8], nxt[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      cur[i] = ld_stream_v4(kb + (int64_t)gq * ks_t + 8 * i);
+      cur[4 + i] = ld_stream_v4(kb + (int64_t)(gq + 8) * ks_t + 8 * i);
+    }
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt) {
+      if (mt < 7) {
+        const __nv_bfloat16* kn = kb + (int64_t)(16 * (mt + 1)) * ks_t;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          nxt[i] = ld_stream_v4(kn + (int64_t)gq * ks_t + 8 * i);
+          nxt[4 + i] = ld_stream_v4(kn + (int64_t)(gq + 8) * ks_t + 8 * i);
+        }
+      }
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int s = 0; s < 8; ++s) {
+        // pair p = 2s / 2s+1 of the thread's 16 bf16 pairs; uint4 index p/4, component p%4
+        const uint32_t a0 = u4get(cur[(2 * s) >> 2], (2 * s) & 3);
+        const uint32_t a2 = u4get(cur[(2 * s + 1) >> 2], (2 * s + 1) & 3);
+        const uint32_t a1 = u4get(cur[4 + ((2 * s) >> 2)], (2 * s) & 3);
+        const uint32_t a3 = u4get(cur[4 + ((2 * s + 1) >> 2)], (2 * s + 1) & 3);
+        const uint32_t b0 = u4get(qv[(2 * s) >> 2], (2 * s) & 3);
+        const uint32_t b1 = u4get(qv[(2 * s + 1) >> 2], (2 * s + 1) & 3);
+        mma_bf16_16816(acc, a0, a1, a2, a3, b0, b1);
+      }
+      mx0 = fmaxf(mx0, fmaxf(acc[0], acc[2]));
+      mx1 = fmaxf(mx1, fmaxf(acc[1], acc[3]));
+      if (mt < 7) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) cur[i] = nxt[i];
+      }
+    }
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+    }
+    if (gq == 0) {
+      const int g0 = 2 * cq, g1 = 2 * cq + 1;
+      if (g0 < G) pooled[((int64_t)b * G + g0) * stride + c] = mx0;
+      if (g1 < G) pooled[((int64_t)b * G + g1) * stride + c] = mx1;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host launchers (called from the C ABI after validation)
+// ---------------------------------------------------------------------------
+cudaError_t launch_index_score_prefill(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
+                                       int d_idx, int64_t batch, int64_t n_q, int64_t q_pos0,
+                                       int32_t G, int32_t h_kidx, float* pooled,
+                                       int64_t stride, int32_t* err, cudaStream_t st) {
+  const int64_t n_qtiles = (n_q + 127) / 128;
+  const int64_t max_nb = (q_pos0 + n_q - 1) / kBlock;
+  if (max_nb == 0) return cudaSuccess;
+  const int64_t n_chunks = (max_nb + 63) / 64;
+  dim3 grid((unsigned)(n_chunks * G), (unsigned)n_qtiles, (unsigned)batch);
+  if (d_idx == 128) {
+    auto k = index_score_maxpool_kernel<128>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         IdxCfg<128>::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    k<<<grid, IdxCfg<128>::kThreads, IdxCfg<128>::kSmemBytes, st>>>(
+        tm_q, tm_k, n_q, q_pos0, G, h_kidx, (int32_t)n_qtiles, pooled, stride, err);
+  } else {
+    auto k = index_score_maxpool_kernel<64>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         IdxCfg<64>::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    k<<<grid, IdxCfg<64>::kThreads, IdxCfg<64>::kSmemBytes, st>>>(
+        tm_q, tm_k, n_q, q_pos0, G, h_kidx, (int32_t)n_qtiles, pooled, stride, err);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_index_score_decode(const void* q_idx, int64_t qs_b, int64_t qs_h,
+                                      const void* k_idx, int64_t ks_b, int64_t ks_t,
+                                      int64_t batch, int64_t q_pos0, int32_t G, float* pooled,
+                                      int64_t stride, cudaStream_t st) {
+  const int64_t own = q_pos0 / kBlock;
+  if (own == 0) return cudaSuccess;
+  const int64_t per_cta = 4 * kDecodeBlocksPerWarp;
+  dim3 grid((unsigned)((own + per_cta - 1) / per_cta), (unsigned)batch);
+  index_score_decode_kernel<<<grid, 128, 0, st>>>(
+      reinterpret_cast<const __nv_bfloat16*>(q_idx), qs_b, qs_h,
+      reinterpret_cast<const __nv_bfloat16*>(k_idx), ks_b, ks_t, q_pos0, G, pooled, stride);
+  return cudaGetLastError();
+}
+
+}  // namespace msa

@@ -1,0 +1,82 @@
+// Log-sum-exp merge of the per-(query, head, block) softmax pieces written by
+// the KV-block-outer attention kernel, in fixed slot order (deterministic):
+//   M = max_s m_s, L = sum_s l_s e^{m_s-M}, o = sum_s acc_s e^{m_s-M} / L,
+//   lse = M + ln L.
+// Softmax over a union of disjoint token sets factors this way, which is
+// what lets the "Outer Gather Q" scheme (page "MSA 稀疏注意力三国杀", section
+// "Kernel 创新：Outer Gather Q") compute each selected block separately.
+//
+// One warp per (batch, query, head); lane l owns output dims 4l .. 4l+3.
+// HBM-bound: it reads each piece once.
+#include "common.cuh"
+
+namespace msa {
+
+__global__ void __launch_bounds__(256)
+    merge_partials_kernel(const int32_t* __restrict__ sel, const float* __restrict__ part_ml,
+                          const float* __restrict__ part_acc, __nv_bfloat16* __restrict__ out,
+                          float* __restrict__ lse, int64_t n_rows, int64_t n_q, int32_t H,
+                          int32_t G) {
+  const int lane = threadIdx.x & 31;
+  const int64_t r = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (r >= n_rows) return;
+  const int32_t R = H / G;
+  const int32_t h = (int32_t)(r % H);
+  const int64_t bq = r / H;            // b * n_q + qi
+  const int64_t b = bq / n_q, qi = bq - b * n_q;
+  const int32_t g = h / R;
+  const int32_t* srow = sel + ((b * G + g) * n_q + qi) * kTopK;
+
+  float m = -INFINITY, l = 0.f;
+  bool v = false;
+  if (lane < kTopK) {
+    v = srow[lane] >= 0;
+    if (v) {
+      const float2 ml = *reinterpret_cast<const float2*>(part_ml + (r * kTopK + lane) * 2);
+      m = ml.x;
+      l = ml.y;
+    }
+  }
+  const uint32_t vmask = __ballot_sync(0xffffffffu, v);
+  float M = m;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  const float w = v ? expf(m - M) : 0.f;
+  float L = w * l;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  const float* pa = part_acc + r * kTopK * kHeadDim + 4 * lane;
+#pragma unroll
+  for (int s = 0; s < kTopK; ++s) {
+    const float ws = __shfl_sync(0xffffffffu, w, s);
+    if ((vmask >> s) & 1u) {
+      const float4 a = *reinterpret_cast<const float4*>(pa + s * kHeadDim);
+      acc.x = fmaf(ws, a.x, acc.x);
+      acc.y = fmaf(ws, a.y, acc.y);
+      acc.z = fmaf(ws, a.z, acc.z);
+      acc.w = fmaf(ws, a.w, acc.w);
+    }
+  }
+  const float inv = 1.0f / L;
+  const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+  const __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+  uint2 packed;
+  packed.x = *reinterpret_cast<const uint32_t*>(&lo);
+  packed.y = *reinterpret_cast<const uint32_t*>(&hi);
+  *reinterpret_cast<uint2*>(out + r * kHeadDim + 4 * lane) = packed;
+  if (lane == 0) lse[r] = M + logf(L);
+}
+
+cudaError_t launch_merge(const int32_t* sel, const float* part_ml, const float* part_acc,
+                         void* out, float* lse, int64_t n_rows, int64_t n_q, int32_t H,
+                         int32_t G, cudaStream_t st) {
+  if (n_rows == 0) return cudaSuccess;
+  const int64_t threads = n_rows * 32;
+  merge_partials_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(
+      sel, part_ml, part_acc, reinterpret_cast<__nv_bfloat16*>(out), lse, n_rows, n_q, H, G);
+  return cudaGetLastError();
+}
+
+}  // namespace msa

@@ -1,0 +1,252 @@
+// C ABI of the MSA hot path: host-side argument checks, TMA tensor-map
+// encoding and kernel dispatch.  Every call validates first and enqueues on
+// the caller's stream; nothing here allocates, frees or synchronises.
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <mutex>
+
+#include "common.cuh"
+
+namespace msa {
+cudaError_t launch_index_score_prefill(const CUtensorMap&, const CUtensorMap&, int, int64_t,
+                                       int64_t, int64_t, int32_t, int32_t, float*, int64_t,
+                                       int32_t*, cudaStream_t);
+cudaError_t launch_index_score_decode(const void*, int64_t, int64_t, const void*, int64_t,
+                                      int64_t, int64_t, int64_t, int32_t, float*, int64_t,
+                                      cudaStream_t);
+cudaError_t launch_topk_blocks(const float*, int64_t, int64_t, int64_t, int64_t, int32_t*,
+                               cudaStream_t);
+size_t block_lists_workspace(int64_t, int64_t, int64_t);
+cudaError_t launch_block_lists(const int32_t*, int64_t, int64_t, int64_t, int64_t, int32_t*,
+                               int32_t*, int64_t, void*, int32_t*, cudaStream_t);
+cudaError_t launch_sparse_attn(const CUtensorMap&, const CUtensorMap&, const void*, int64_t,
+                               int64_t, int64_t, const int32_t*, const int32_t*, int64_t,
+                               int64_t, int64_t, int64_t, int32_t, int32_t, int32_t, float,
+                               float*, float*, int32_t*, cudaStream_t);
+cudaError_t launch_merge(const int32_t*, const float*, const float*, void*, float*, int64_t,
+                         int64_t, int32_t, int32_t, cudaStream_t);
+}  // namespace msa
+
+namespace {
+
+constexpr int64_t kMaxBlocks = 50000;   // shared-memory histogram bound of the inversion
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool is_pow2(int64_t x) { return x > 0 && (x & (x - 1)) == 0; }
+
+msa_status check_dims(const msa_dims* d) {
+  if (d == nullptr) return MSA_ERR_INVALID_ARG;
+  if (d->batch < 1 || d->n_q < 1 || d->n_kv < 1 || d->q_pos0 < 0) return MSA_ERR_INVALID_ARG;
+  if (d->q_pos0 + d->n_q > d->n_kv) return MSA_ERR_INVALID_ARG;
+  if (d->h_kv < 1 || d->h_q < 1 || d->h_q % d->h_kv != 0) return MSA_ERR_INVALID_ARG;
+  if (d->h_kidx != 1 && d->h_kidx != d->h_kv) return MSA_ERR_INVALID_ARG;
+  if (!(d->scale > 0.f) || !std::isfinite(d->scale)) return MSA_ERR_INVALID_ARG;
+  const int64_t R = d->h_q / d->h_kv;
+  if (!is_pow2(R) || R > 16) return MSA_ERR_UNSUPPORTED;
+  if (d->d_idx != 64 && d->d_idx != 128) return MSA_ERR_UNSUPPORTED;
+  const int64_t nblk = (d->n_kv + MSA_BLOCK_TOKENS - 1) / MSA_BLOCK_TOKENS;
+  if (nblk > kMaxBlocks) return MSA_ERR_UNSUPPORTED;
+  if (d->n_kv > (int64_t(1) << 31) - 1) return MSA_ERR_UNSUPPORTED;
+  if (d->n_q > (int64_t(1) << 26)) return MSA_ERR_UNSUPPORTED;   // entries pack i << 4
+  if (d->batch > 65535 || d->batch * d->h_kv > 65535) return MSA_ERR_UNSUPPORTED;
+  if (d->n_q / 128 + 1 > 65535) return MSA_ERR_UNSUPPORTED;
+  return MSA_OK;
+}
+
+msa_status check_tensor(const msa_tensor& t) {
+  if (t.ptr == nullptr) return MSA_ERR_INVALID_ARG;
+  if (!aligned16(t.ptr)) return MSA_ERR_ALIGNMENT;
+  if (t.s_batch < 0 || t.s_tok < 0 || t.s_head < 0) return MSA_ERR_INVALID_ARG;
+  if ((t.s_batch % 8) || (t.s_tok % 8) || (t.s_head % 8)) return MSA_ERR_ALIGNMENT;
+  return MSA_OK;
+}
+
+// total (query, selected block) pairs of one (batch, group)
+int64_t entries_per_bg(const msa_dims* d) {
+  int64_t total = 0;
+  // queries with own(t) >= 15 contribute 16; earlier ones own + 1
+  const int64_t t0 = d->q_pos0, t1 = d->q_pos0 + d->n_q;   // [t0, t1)
+  const int64_t full_from = 15 * MSA_BLOCK_TOKENS;           // first t with own >= 15
+  const int64_t a = t0, bnd = std::min(t1, std::max(t0, full_from));
+  for (int64_t t = a; t < bnd; ++t) total += t / MSA_BLOCK_TOKENS + 1;
+  if (t1 > bnd) total += (t1 - bnd) * MSA_TOPK_BLOCKS;
+  return total;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 4-D bf16 map: dims {inner, d1, d2, d3} with byte strides of d1..d3, box
+// {64, b1, b2, 1}, 128-byte swizzle, zero fill out of bounds.
+msa_status make_map(CUtensorMap* map, const void* ptr, uint64_t inner, uint64_t d1, uint64_t d2,
+                    uint64_t d3, int64_t s1, int64_t s2, int64_t s3, uint32_t b1, uint32_t b2) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return MSA_ERR_CUDA;
+  cuuint64_t dims[4] = {inner, d1, d2, d3};
+  cuuint64_t strides[3] = {(cuuint64_t)s1 * 2, (cuuint64_t)s2 * 2, (cuuint64_t)s3 * 2};
+  // a dimension of extent 1 still needs a legal stride
+  for (int i = 0; i < 3; ++i)
+    if (strides[i] == 0) strides[i] = 16;
+  cuuint32_t box[4] = {64, b1, b2, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? MSA_OK : MSA_ERR_CUDA;
+}
+
+msa_status from_cuda(cudaError_t e) { return e == cudaSuccess ? MSA_OK : MSA_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+int64_t msa_num_blocks(const msa_dims* d) {
+  if (d == nullptr || d->n_kv < 1) return 0;
+  return (d->n_kv + MSA_BLOCK_TOKENS - 1) / MSA_BLOCK_TOKENS;
+}
+
+int64_t msa_num_entries(const msa_dims* d) {
+  if (check_dims(d) != MSA_OK) return 0;
+  return d->batch * d->h_kv * entries_per_bg(d);
+}
+
+msa_status msa_index_score_maxpool(const msa_dims* d, msa_tensor q_idx, msa_tensor k_idx,
+                                   float* pooled, int64_t pooled_row_stride, int32_t* dev_err,
+                                   void* stream) {
+  msa_status s = check_dims(d);
+  if (s != MSA_OK) return s;
+  if ((s = check_tensor(q_idx)) != MSA_OK) return s;
+  if ((s = check_tensor(k_idx)) != MSA_OK) return s;
+  if (pooled == nullptr) return MSA_ERR_INVALID_ARG;
+  if (!aligned16(pooled)) return MSA_ERR_ALIGNMENT;
+  const int64_t nblk = msa_num_blocks(d);
+  if (pooled_row_stride < nblk || pooled_row_stride % 4 != 0) return MSA_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int32_t G = d->h_kv;
+  if (d->n_q == 1 && d->h_kidx == 1 && d->d_idx == 128 && G <= 8) {
+    return from_cuda(msa::launch_index_score_decode(q_idx.ptr, q_idx.s_batch, q_idx.s_head,
+                                                    k_idx.ptr, k_idx.s_batch, k_idx.s_tok,
+                                                    d->batch, d->q_pos0, G, pooled,
+                                                    pooled_row_stride, st));
+  }
+  CUtensorMap tq, tk;
+  // q_idx [B, n_q, G, d_idx]: dims {d_idx, G, n_q, B}, box {64, 1, 128, 1}
+  if ((s = make_map(&tq, q_idx.ptr, d->d_idx, G, d->n_q, d->batch, q_idx.s_head, q_idx.s_tok,
+                    q_idx.s_batch, 1, 128)) != MSA_OK)
+    return s;
+  // k_idx [B, h_kidx, n_kv, d_idx]: dims {d_idx, n_kv, h_kidx, B}, box {64, 128, 1, 1}
+  if ((s = make_map(&tk, k_idx.ptr, d->d_idx, d->n_kv, d->h_kidx, d->batch, k_idx.s_tok,
+                    k_idx.s_head, k_idx.s_batch, 128, 1)) != MSA_OK)
+    return s;
+  return from_cuda(msa::launch_index_score_prefill(tq, tk, d->d_idx, d->batch, d->n_q,
+                                                   d->q_pos0, G, d->h_kidx, pooled,
+                                                   pooled_row_stride, dev_err, st));
+}
+
+msa_status msa_topk_blocks(const msa_dims* d, const float* pooled, int64_t pooled_row_stride,
+                           int32_t* sel, int32_t* dev_err, void* stream) {
+  (void)dev_err;
+  msa_status s = check_dims(d);
+  if (s != MSA_OK) return s;
+  if (pooled == nullptr || sel == nullptr) return MSA_ERR_INVALID_ARG;
+  if (!aligned16(pooled) || !aligned16(sel)) return MSA_ERR_ALIGNMENT;
+  if (pooled_row_stride < msa_num_blocks(d) || pooled_row_stride % 4 != 0)
+    return MSA_ERR_INVALID_ARG;
+  const int64_t n_rows = d->batch * d->h_kv * d->n_q;
+  return from_cuda(msa::launch_topk_blocks(pooled, pooled_row_stride, n_rows, d->n_q, d->q_pos0,
+                                           sel, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t msa_block_query_lists_workspace(const msa_dims* d) {
+  if (check_dims(d) != MSA_OK) return 0;
+  return msa::block_lists_workspace(d->batch * d->h_kv, d->n_q, msa_num_blocks(d));
+}
+
+msa_status msa_build_block_query_lists(const msa_dims* d, const int32_t* sel,
+                                       int32_t* blk_offsets, int32_t* entries, void* ws,
+                                       size_t ws_bytes, int32_t* dev_err, void* stream) {
+  msa_status s = check_dims(d);
+  if (s != MSA_OK) return s;
+  if (sel == nullptr || blk_offsets == nullptr || entries == nullptr || ws == nullptr)
+    return MSA_ERR_INVALID_ARG;
+  if (!aligned16(sel) || !aligned16(ws)) return MSA_ERR_ALIGNMENT;
+  if (ws_bytes < msa_block_query_lists_workspace(d)) return MSA_ERR_WORKSPACE_TOO_SMALL;
+  const int64_t total = msa_num_entries(d);
+  if (total >= (int64_t(1) << 31)) return MSA_ERR_UNSUPPORTED;
+  return from_cuda(msa::launch_block_lists(sel, d->batch * d->h_kv, d->n_q, d->q_pos0,
+                                           msa_num_blocks(d), blk_offsets, entries, total, ws,
+                                           dev_err, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+msa_status msa_sparse_attn_fwd(const msa_dims* d, msa_tensor q, msa_tensor k, msa_tensor v,
+                               const int32_t* blk_offsets, const int32_t* entries,
+                               float* part_ml, float* part_acc, int32_t* dev_err,
+                               void* stream) {
+  msa_status s = check_dims(d);
+  if (s != MSA_OK) return s;
+  if ((s = check_tensor(q)) != MSA_OK) return s;
+  if ((s = check_tensor(k)) != MSA_OK) return s;
+  if ((s = check_tensor(v)) != MSA_OK) return s;
+  if (blk_offsets == nullptr || entries == nullptr || part_ml == nullptr || part_acc == nullptr)
+    return MSA_ERR_INVALID_ARG;
+  if (!aligned16(part_ml) || !aligned16(part_acc)) return MSA_ERR_ALIGNMENT;
+  const int64_t nblk = msa_num_blocks(d);
+  const int64_t n_seg = d->batch * d->h_kv * nblk;
+  const int64_t total = msa_num_entries(d);
+  if (total >= (int64_t(1) << 31)) return MSA_ERR_UNSUPPORTED;
+  CUtensorMap tk, tv;
+  // k, v [B, h_kv, n_kv, 128]: dims {128, n_kv, h_kv, B}, box {64, 128, 1, 1}
+  if ((s = make_map(&tk, k.ptr, MSA_HEAD_DIM, d->n_kv, d->h_kv, d->batch, k.s_tok, k.s_head,
+                    k.s_batch, 128, 1)) != MSA_OK)
+    return s;
+  if ((s = make_map(&tv, v.ptr, MSA_HEAD_DIM, d->n_kv, d->h_kv, d->batch, v.s_tok, v.s_head,
+                    v.s_batch, 128, 1)) != MSA_OK)
+    return s;
+  return from_cuda(msa::launch_sparse_attn(
+      tk, tv, q.ptr, q.s_batch, q.s_tok, q.s_head, blk_offsets, entries, n_seg, total, d->n_q,
+      d->q_pos0, d->h_kv, d->h_q, (int32_t)nblk, d->scale, part_ml, part_acc, dev_err,
+      reinterpret_cast<cudaStream_t>(stream)));
+}
+
+msa_status msa_merge_partials(const msa_dims* d, const int32_t* sel, const float* part_ml,
+                              const float* part_acc, void* out, float* lse, int32_t* dev_err,
+                              void* stream) {
+  (void)dev_err;
+  msa_status s = check_dims(d);
+  if (s != MSA_OK) return s;
+  if (sel == nullptr || part_ml == nullptr || part_acc == nullptr || out == nullptr ||
+      lse == nullptr)
+    return MSA_ERR_INVALID_ARG;
+  if (!aligned16(part_ml) || !aligned16(part_acc) || !aligned16(out))
+    return MSA_ERR_ALIGNMENT;
+  const int64_t n_rows = d->batch * d->n_q * d->h_q;
+  return from_cuda(msa::launch_merge(sel, part_ml, part_acc, out, lse, n_rows, d->n_q, d->h_q,
+                                     d->h_kv, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+const char* msa_status_string(msa_status s) {
+  switch (s) {
+    case MSA_OK: return "MSA_OK";
+    case MSA_ERR_INVALID_ARG: return "MSA_ERR_INVALID_ARG";
+    case MSA_ERR_UNSUPPORTED: return "MSA_ERR_UNSUPPORTED";
+    case MSA_ERR_ALIGNMENT: return "MSA_ERR_ALIGNMENT";
+    case MSA_ERR_WORKSPACE_TOO_SMALL: return "MSA_ERR_WORKSPACE_TOO_SMALL";
+    case MSA_ERR_CUDA: return "MSA_ERR_CUDA";
+  }
+  return "MSA_ERR_UNKNOWN";
+}
+
+}  // extern "C"

@@ -209,6 +209,10 @@ def random_selection(w: Workload, device="cpu", seed_offset: int = 11):
                 top = torch.topk(key, k, dim=1)
                 picked = torch.where(top.values >= 0, top.indices, torch.full_like(top.indices, -1))
                 rows = torch.cat([picked, o[:, None]], dim=1)
+                if rows.shape[1] < TOPK:
+                    pad = torch.full((rows.shape[0], TOPK - rows.shape[1]), -1,
+                                     dtype=rows.dtype, device=device)
+                    rows = torch.cat([rows, pad], dim=1)
                 big = torch.full_like(rows, 1 << 30)
                 rows = torch.where(rows >= 0, rows, big).sort(dim=1).values
                 rows = torch.where(rows == (1 << 30), torch.full_like(rows, -1), rows)

@@ -1,0 +1,181 @@
+/*
+ * msa.h -- C ABI of the MiniMax Sparse Attention (MSA) hot path on B200
+ * (sm_100a).
+ *
+ * The method (page "MSA 稀疏注意力三国杀：NSA / DSA / MoBA / MSA 四方案深度对比",
+ * section "MSA 架构：粗筛 + 精算"; sparse-attention survey page, entry
+ * "MiniMax Sparse Attention (MSA)"):
+ *   1. an index branch scores every causal (query, key token) pair with one
+ *      index query head per GQA group and a shared index key head;
+ *   2. token scores are max-pooled over 128-token KV blocks and each query
+ *      keeps 16 blocks per group, its own block always among them;
+ *   3. the main branch runs exact softmax attention over the 16 x 128 = 2048
+ *      selected tokens.
+ * Step 3 runs KV-block-outer ("Kernel 创新：Outer Gather Q" section of the
+ * first page): each selected KV block is read once and every query row that
+ * chose it is gathered into one tensor-core tile; the per-(query, block)
+ * softmax pieces are then merged by log-sum-exp.
+ *
+ * Conventions for every entry point:
+ *   - All pointers are DEVICE pointers unless stated; the caller owns every
+ *     buffer.  The library never allocates, frees or synchronises; each call
+ *     validates its arguments on the host, then enqueues its kernels on
+ *     `stream` (a cudaStream_t; NULL = legacy default stream) and returns.
+ *   - A non-OK status is returned before anything is enqueued, except
+ *     MSA_ERR_CUDA, which reports a launch error.
+ *   - `dev_err` (may be NULL) is a device int32 the caller zeroes; a kernel
+ *     that detects a problem at run time (an out-of-range block id, a wait
+ *     that ran past its time limit) stores an MSA_DEVERR_* code there and
+ *     returns early.  Nothing traps.
+ *   - Results are deterministic: bit-identical from run to run.
+ *   - Fixed sizes: block B_k = 128 tokens, top-k = 16 blocks (own included),
+ *     head_dim = 128, d_idx in {64, 128}.
+ *   - Layouts are given as [outer, ..., inner]; the innermost dimension is
+ *     contiguous, the other strides are element strides in msa_tensor.
+ */
+#ifndef MSA_H_
+#define MSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define MSA_API __attribute__((visibility("default")))
+#else
+#define MSA_API
+#endif
+
+#define MSA_BLOCK_TOKENS 128
+#define MSA_TOPK_BLOCKS 16
+#define MSA_HEAD_DIM 128
+
+typedef enum {
+  MSA_OK = 0,
+  MSA_ERR_INVALID_ARG = 1,        /* null pointer, bad size, inconsistent dims */
+  MSA_ERR_UNSUPPORTED = 2,        /* valid but not implemented (e.g. d_idx 96) */
+  MSA_ERR_ALIGNMENT = 3,          /* pointer or stride not 16-byte aligned */
+  MSA_ERR_WORKSPACE_TOO_SMALL = 4,
+  MSA_ERR_CUDA = 5                /* a CUDA runtime/driver call failed */
+} msa_status;
+
+/* device-side error codes written to *dev_err */
+#define MSA_DEVERR_TIMEOUT 1      /* a bounded wait on a barrier ran out */
+#define MSA_DEVERR_BAD_BLOCK 2    /* a selected block id outside [0, own] */
+#define MSA_DEVERR_BAD_ENTRY 3    /* a block->query entry out of range */
+
+/* Problem sizes.  Query i of batch b sits at absolute position
+ * t = q_pos0 + i and may attend keys j <= t; keys are 0 .. n_kv-1 and
+ * q_pos0 + n_q <= n_kv.  Prefill: q_pos0 = 0, n_q = n_kv.  Decode: n_q = 1,
+ * q_pos0 = n_kv - 1.  Chunked prefill: q_pos0 = length of the cached prefix.
+ * G = h_kv GQA groups; h_q / h_kv query heads per group (a power of two
+ * <= 128); head h belongs to group h / (h_q / h_kv).  h_kidx is 1 (one index
+ * key head shared by all groups) or h_kv (one per group).  scale multiplies
+ * q.k in the main branch (1/sqrt(128) for the textbook softmax). */
+typedef struct {
+  int64_t batch, n_q, n_kv, q_pos0;
+  int32_t h_q, h_kv, h_kidx, d_idx;
+  float scale;
+} msa_dims;
+
+/* A strided bf16 tensor: element strides of the batch, token and head
+ * dimensions; the innermost (feature) dimension is contiguous.  ptr and
+ * every stride * 2 bytes must be multiples of 16 bytes. */
+typedef struct {
+  const void* ptr;
+  int64_t s_batch, s_tok, s_head;
+} msa_tensor;
+
+/* Number of KV blocks, ceil(n_kv / 128). */
+MSA_API int64_t msa_num_blocks(const msa_dims* dims);
+
+/* Number of (query, selected block) pairs over the whole problem:
+ * batch * h_kv * sum_i min(16, own(q_pos0 + i) + 1), own(t) = t / 128.
+ * It sizes the `entries` array of msa_build_block_query_lists. */
+MSA_API int64_t msa_num_entries(const msa_dims* dims);
+
+/* Step 1+2a: index scores and causal block max-pool
+ * (first page, "第一步：粗筛" items 1-2: score each token, a block's score is
+ * its highest token score; survey page MSA entry: one index query head per
+ * GQA group, shared index key head, block max-pool).
+ *   q_idx  [B, n_q, G, d_idx]            bf16
+ *   k_idx  [B, h_kidx, n_kv, d_idx]      bf16 (s_head = stride between index key heads)
+ *   pooled [B, G, n_q, pooled_row_stride] fp32, written for every block
+ *          c < own(t): pooled = max_{j in block c} sum_k q_idx[t,g,k] k_idx[j,k],
+ *          accumulated in fp32 from the exact bf16 products.  Entries
+ *          c >= own(t) are left untouched.  The n_q x n_kv score matrix is
+ *          never stored.
+ * pooled_row_stride >= msa_num_blocks(dims) and a multiple of 4. */
+MSA_API msa_status msa_index_score_maxpool(const msa_dims* dims, msa_tensor q_idx, msa_tensor k_idx,
+                                   float* pooled, int64_t pooled_row_stride,
+                                   int32_t* dev_err, void* stream);
+
+/* Step 2b: block selection (first page, "第一步：粗筛" item 3: 16 blocks, the
+ * current position's block always taken, the rest by score; survey page:
+ * top-k per GQA group with the local block kept).
+ *   pooled [B, G, n_q, pooled_row_stride] fp32 as written above
+ *   sel    [B, G, n_q, 16] int32: own(t) plus the min(15, own(t)) best blocks
+ *          c < own(t) ranked by (score descending, block index ascending;
+ *          -0.0 equals +0.0), in ascending block order, padded with -1 to 16.
+ * No other block (first block, sink, window) is forced. */
+MSA_API msa_status msa_topk_blocks(const msa_dims* dims, const float* pooled, int64_t pooled_row_stride,
+                           int32_t* sel, int32_t* dev_err, void* stream);
+
+/* Bytes of device workspace msa_build_block_query_lists needs. */
+MSA_API size_t msa_block_query_lists_workspace(const msa_dims* dims);
+
+/* Step 3a: inversion of the query->block lists into block->query lists, the
+ * index a KV-block-outer kernel walks (first page, "Kernel 创新：Outer Gather
+ * Q": the queries that chose a block are gathered and computed together).
+ *   sel         [B, G, n_q, 16] int32 (as written by msa_topk_blocks; any
+ *               valid selection works)
+ *   blk_offsets [B * G * nblk + 1] int32: segment s = (b * G + g) * nblk + c
+ *               holds entries[blk_offsets[s] .. blk_offsets[s+1])
+ *   entries     [msa_num_entries(dims)] int32: (i << 4) | slot for each query
+ *               index i (within its batch) and the slot of c in sel[b,g,i,:],
+ *               ascending in i inside a segment (deterministic counting sort)
+ *   ws          device workspace of at least msa_block_query_lists_workspace()
+ *               bytes, 16-byte aligned; contents on entry do not matter. */
+MSA_API msa_status msa_build_block_query_lists(const msa_dims* dims, const int32_t* sel,
+                                       int32_t* blk_offsets, int32_t* entries,
+                                       void* ws, size_t ws_bytes,
+                                       int32_t* dev_err, void* stream);
+
+/* Step 3b: KV-block-outer sparse attention (first page "第二步：精算": full
+ * attention over the selected blocks only; survey page: exact softmax
+ * attention; softmax(Q K^T * scale) V from the chenxutan page).  For every
+ * segment (b, g, c) each K/V block is brought into shared memory once and the
+ * R = h_q / h_kv head rows of every listed query are gathered into 128-row
+ * tensor-core tiles.  For each (query i, head h in g, slot) it writes the
+ * piece over the tokens j of block c with j <= t:
+ *   part_ml [B, n_q, h_q, 16, 2] fp32: m = max_j scale * q.k_j,
+ *                                      l = sum_j e^{scale q.k_j - m}
+ *   part_acc[B, n_q, h_q, 16, 128] fp32: sum_j e^{scale q.k_j - m} v_j
+ * (the weights e^{...} are rounded to bf16 before they multiply V and before
+ * they are summed into l, so acc / l is an exact convex combination).
+ *   q [B, n_q, h_q, 128] bf16; k, v [B, h_kv, n_kv, 128] bf16
+ *   (msa_tensor strides; for k/v s_head is the stride between KV heads). */
+MSA_API msa_status msa_sparse_attn_fwd(const msa_dims* dims, msa_tensor q, msa_tensor k, msa_tensor v,
+                               const int32_t* blk_offsets, const int32_t* entries,
+                               float* part_ml, float* part_acc,
+                               int32_t* dev_err, void* stream);
+
+/* Step 3c: log-sum-exp merge of the pieces, in slot order:
+ *   M = max_s m_s, L = sum_s l_s e^{m_s - M}, o = sum_s acc_s e^{m_s - M} / L,
+ *   lse = M + ln L, over the slots s with sel[b, g, i, s] >= 0.
+ *   out [B, n_q, h_q, 128] bf16 contiguous; lse [B, n_q, h_q] fp32. */
+MSA_API msa_status msa_merge_partials(const msa_dims* dims, const int32_t* sel,
+                              const float* part_ml, const float* part_acc,
+                              void* out, float* lse, int32_t* dev_err, void* stream);
+
+/* Human-readable name of a status code (static storage). */
+MSA_API const char* msa_status_string(msa_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MSA_H_ */

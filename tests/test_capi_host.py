@@ -1,0 +1,113 @@
+"""Host-only checks of the C ABI (no GPU needed): the library loads, exports
+every entry point include/msa.h declares, sizes work out, and argument
+validation rejects bad input before anything reaches the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from block_sparse_attention_32_b200 import build as msa_build
+from block_sparse_attention_32_b200 import capi
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    msa_build.build()
+    return capi.lib()
+
+
+def _declared():
+    names = []
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            txt = open(os.path.join(ROOT, "include", fn)).read()
+            names += re.findall(r"MSA_API\s+[\w\s\*]+?\b(msa_\w+)\s*\(", txt)
+    return names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared()
+    assert len(names) >= 9
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_block_and_entry_counts(lib):
+    d = capi.make_dims(1, 4096, 4096, 0, 4, 1, 64)
+    assert capi.msa_num_blocks(d) == 32
+    # queries t < 1920 keep own+1 blocks, later ones 16
+    want = sum(min(16, t // 128 + 1) for t in range(4096))
+    assert capi.msa_num_entries(d) == want
+    d = capi.make_dims(64, 1, 262144, 262143, 64, 8, 128)
+    assert capi.msa_num_blocks(d) == 2048
+    assert capi.msa_num_entries(d) == 64 * 8 * 16
+    d = capi.make_dims(1, 8192, 1056768, 1048576, 64, 8, 128)
+    assert capi.msa_num_blocks(d) == 8256
+    assert capi.msa_num_entries(d) == 8 * 8192 * 16
+    d = capi.make_dims(1, 1000, 2600, 1000, 4, 2, 64)   # unaligned chunk start
+    want = sum(min(16, t // 128 + 1) for t in range(1000, 2000)) * 2
+    assert capi.msa_num_entries(d) == want
+
+
+def test_workspace_size(lib):
+    d = capi.make_dims(2, 300, 1000, 700, 8, 2, 64)
+    nblk, ntiles = 8, 3
+    assert capi.msa_block_query_lists_workspace(d) == 4 * 2 * 2 * nblk * (ntiles + 1)
+
+
+BAD_DIMS = [
+    dict(batch=0), dict(n_q=0), dict(n_kv=0), dict(q_pos0=-1), dict(q_pos0=5000),
+    dict(h_q=6), dict(h_kv=3), dict(h_kidx=3), dict(scale=0.0), dict(scale=float("nan")),
+]
+
+
+@pytest.mark.parametrize("bad", BAD_DIMS, ids=lambda b: ",".join(f"{k}={v}" for k, v in b.items()))
+def test_invalid_dims_are_rejected(lib, bad):
+    args = dict(batch=1, n_q=1000, n_kv=4096, q_pos0=0, h_q=8, h_kv=2, d_idx=128, h_kidx=1,
+                scale=0.088)
+    args.update(bad)
+    d = capi.Dims(args["batch"], args["n_q"], args["n_kv"], args["q_pos0"], args["h_q"],
+                  args["h_kv"], args["h_kidx"], args["d_idx"], args["scale"])
+    t = capi.Tensor(0x100000, 0, 256, 128)
+    st = lib.msa_index_score_maxpool(ctypes.byref(d), t, t, ctypes.c_void_p(0x200000), 32, None,
+                                     None)
+    assert st in (1, 2)          # INVALID_ARG or UNSUPPORTED, nothing enqueued
+
+
+def test_unsupported_sizes(lib):
+    for d in (capi.make_dims(1, 100, 100, 0, 8, 2, 96),          # d_idx 96
+              capi.make_dims(1, 100, 100, 0, 12, 4, 64),         # R = 3
+              capi.make_dims(1, 100, 100, 0, 64, 2, 64)):        # R = 32
+        t = capi.Tensor(0x100000, 0, 256, 128)
+        assert lib.msa_index_score_maxpool(ctypes.byref(d), t, t, ctypes.c_void_p(0x200000),
+                                           4, None, None) == 2
+
+
+def test_pointer_and_stride_checks(lib):
+    d = capi.make_dims(1, 1000, 4096, 0, 8, 2, 128)
+    good = capi.Tensor(0x100000, 0, 256, 128)
+    null = capi.Tensor(0, 0, 256, 128)
+    mis = capi.Tensor(0x100008, 0, 256, 128)
+    odd = capi.Tensor(0x100000, 0, 260, 128)
+    P = ctypes.c_void_p
+    f = lib.msa_index_score_maxpool
+    assert f(ctypes.byref(d), null, good, P(0x200000), 32, None, None) == 1
+    assert f(ctypes.byref(d), mis, good, P(0x200000), 32, None, None) == 3
+    assert f(ctypes.byref(d), good, odd, P(0x200000), 32, None, None) == 3
+    assert f(ctypes.byref(d), good, good, P(0x200004), 32, None, None) == 3
+    assert f(ctypes.byref(d), good, good, P(0x200000), 30, None, None) == 1   # stride < nblk
+    assert f(ctypes.byref(d), good, good, P(0x200000), 33, None, None) == 1   # not a multiple of 4
+    assert f(None, good, good, P(0x200000), 32, None, None) == 1
+    ws = capi.msa_block_query_lists_workspace(d)
+    g = lib.msa_build_block_query_lists
+    assert g(ctypes.byref(d), P(0x1000), P(0x2000), P(0x3000), P(0x4000), ws - 4, None, None) == 4
+    assert g(ctypes.byref(d), P(0x1000), None, P(0x3000), P(0x4000), ws, None, None) == 1
+    h = lib.msa_sparse_attn_fwd
+    assert h(ctypes.byref(d), good, good, mis, P(0x1000), P(0x2000), P(0x3000), P(0x4000),
+             None, None) == 3
+    m = lib.msa_merge_partials
+    assert m(ctypes.byref(d), P(0x1000), P(0x2000), P(0x3000), None, P(0x5000), None, None) == 1
+    assert lib.msa_status_string(4) == b"MSA_ERR_WORKSPACE_TOO_SMALL"

@@ -1,0 +1,81 @@
+"""GPU parity at the full workload sizes, in the launch configuration the
+benchmark times (the five C-ABI calls of pipeline.forward on one stream).
+
+The whole path runs on the GPU for every query; the oracle recomputes a
+stratified sample of query rows (first rows, the 16-block boundary, planted
+targets, random rows) from the same inputs: pooled scores, the selected set
+(bit-exact apart from counted near-ties) and the attention output.
+Selection invariants are checked on every row of the GPU result.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from block_sparse_attention_32_b200 import pipeline, workloads as wl
+
+from _helpers import (OUT_MAX_ABS, OUT_MEAN_ABS, bits, compare_out, compare_pooled,
+                      compare_sets, pooled_tolerance, sample_rows)
+
+pytestmark = pytest.mark.gpu
+
+
+def _invariants_all_rows(sel: torch.Tensor, w):
+    """own(t) in the set, count = min(16, own+1), ascending, distinct, all <= own."""
+    pos = w.q_pos0 + torch.arange(w.n_q, device=sel.device)
+    own = (pos // 128).view(1, 1, -1)
+    nsel = torch.clamp(own + 1, max=16)
+    valid = sel >= 0
+    assert torch.equal(valid.sum(-1), nsel.expand_as(valid.sum(-1)))
+    big = torch.where(valid, sel, torch.full_like(sel, 1 << 30))
+    assert bool((big[..., 1:] > big[..., :-1]).all())           # strictly ascending
+    assert bool(((sel <= own[..., None]) | ~valid).all())
+    last = torch.gather(sel, -1, (nsel - 1).expand(sel.shape[:-1]).unsqueeze(-1).long())
+    assert torch.equal(last.squeeze(-1), own.expand(sel.shape[:-1]).to(sel.dtype))
+
+
+@pytest.mark.parametrize("name,n_rows,batches", [
+    ("prefill_32k", 40, None),
+    ("prefill_128k", 28, None),
+    ("chunked_prefill_1m", 12, None),
+    ("decode_64x256k", 1, [0, 37]),
+])
+def test_full_size_sampled_parity(name, n_rows, batches):
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    w = wl.CONFIGS[name]
+    torch.cuda.empty_cache()
+    inp = wl.make_inputs(w, "cuda")
+    buf = pipeline.Buffers.allocate(pipeline.dims_for(w))
+    out, lse = pipeline.forward(buf, inp["q"], inp["k"], inp["v"], inp["q_idx"], inp["k_idx"])
+    torch.cuda.synchronize()
+    assert int(buf.dev_err[0]) == 0
+    _invariants_all_rows(buf.sel, w)
+
+    bsel = batches or [0]
+    rows = sample_rows(w.n_q, w.q_pos0, n_rows, seed=1)
+    pos = np.concatenate([w.q_pos0 + rows for _ in bsel])
+    bat = np.concatenate([np.full(len(rows), i, np.int64) for i in range(len(bsel))])
+    qi = np.concatenate([rows for _ in bsel])
+    bt = torch.tensor(bsel)
+    rt = torch.tensor(rows)
+    q_rows = bits(inp["q"][bt][:, rt].reshape(-1, w.h_q, 128))
+    qidx_rows = bits(inp["q_idx"][bt][:, rt].reshape(-1, w.h_kv, w.d_idx))
+    k_b, v_b, ki_b = (bits(inp[n][bt]) for n in ("k", "v", "k_idx"))
+    pooled_o, sel_o, out_o, _ = oracle.forward_rows(q_rows, qidx_rows, pos, bat, k_b, v_b, ki_b,
+                                                    w.scale)
+    gp = buf.pooled[bt][:, :, rt].permute(0, 2, 1, 3).reshape(len(pos), w.h_kv, -1).cpu().numpy()
+    tol = pooled_tolerance(qidx_rows, ki_b, pos, bat, w.h_kidx)
+    worst = compare_pooled(gp, pooled_o, tol, pos)
+    gs = buf.sel[bt][:, :, rt].permute(0, 2, 1, 3).reshape(len(pos), w.h_kv, 16).cpu().numpy()
+    bad, ties, bad_cert, ok = compare_sets(gs, sel_o, pooled_o, pos)
+    go = out[bt][:, rt].float().reshape(len(pos), w.h_q, 128).cpu().numpy()
+    mx, mean = compare_out(go[ok], out_o[ok])
+    print(f"{name}: rows={len(pos)} pooled_err/tol={worst:.3f} near_ties={ties} "
+          f"set_mismatch={bad} out_max={mx:.3g} out_mean={mean:.3g}")
+    del inp, buf
+    torch.cuda.empty_cache()
+    assert worst <= 1.0
+    assert bad == 0 and bad_cert == 0
+    assert ok.sum() >= len(pos) - ties
+    assert mx <= OUT_MAX_ABS and mean <= OUT_MEAN_ABS

@@ -1,0 +1,238 @@
+"""GPU parity: every C-ABI step against the CPU oracle on seeded inputs.
+
+Small workloads span several tiles, ragged tails (n_kv and n_q not multiples
+of 128), a chunk start inside a block, every group size R in {1,2,4,8,16},
+d_idx in {64,128}, shared and per-group index key heads, batch > 1 and the
+one-query decode path.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from block_sparse_attention_32_b200 import capi, pipeline, workloads as wl
+
+from _helpers import (LSE_MAX_ABS, OUT_MAX_ABS, OUT_MEAN_ABS, bits, compare_out,
+                      compare_pooled, compare_sets, pooled_tolerance)
+
+pytestmark = pytest.mark.gpu
+
+CASES = [
+    wl.TINY,
+    wl.small("ragged_r4", 1, 2500, 2500, 0, 8, 2, 128, seed=11),
+    wl.small("chunk_unaligned_r2_hk2", 1, 1600, 2600, 1000, 4, 2, 64, seed=12, h_kidx=2),
+    wl.small("batch2_r8", 2, 640, 3000, 2360, 16, 2, 128, seed=13),
+    wl.small("r16_peaked", 1, 2100, 2100, 0, 16, 1, 64, seed=14, q_scale=4.0),
+    wl.small("r1", 1, 2300, 2300, 0, 2, 2, 128, seed=15),
+    wl.small("decode_b3", 3, 1, 5000, 4999, 32, 8, 128, seed=16),
+    wl.small("decode_d64", 2, 1, 3000, 2999, 8, 2, 64, seed=17),
+    wl.small("one_block", 1, 100, 100, 0, 4, 1, 64, seed=18),
+    wl.small("sixteen_blocks", 1, 2048, 2048, 0, 8, 2, 128, seed=19),
+]
+
+
+def _need_gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+
+
+def _all_rows(w):
+    rows = np.arange(w.n_q, dtype=np.int64)
+    pos = np.tile(w.q_pos0 + rows, w.batch)
+    bat = np.repeat(np.arange(w.batch, dtype=np.int64), w.n_q)
+    idx = np.tile(rows, w.batch)
+    return idx, pos, bat
+
+
+def _run_select(w, inp):
+    d = pipeline.dims_for(w)
+    buf = pipeline.Buffers.allocate(d)
+    buf.pooled.fill_(float("nan"))
+    pipeline.select(buf, inp["q_idx"], inp["k_idx"])
+    torch.cuda.synchronize()
+    assert int(buf.dev_err[0]) == 0
+    return buf
+
+
+@pytest.mark.parametrize("w", CASES, ids=lambda w: w.name)
+def test_index_pooled_and_selection(w):
+    _need_gpu()
+    inp = wl.make_inputs(w, "cuda")
+    buf = _run_select(w, inp)
+    idx, pos, bat = _all_rows(w)
+    qib = bits(inp["q_idx"])                               # [B, n_q, G, d]
+    q_rows = qib.reshape(-1, w.h_kv, w.d_idx)
+    kib = bits(inp["k_idx"])
+    ora_pooled = oracle.index_pooled(q_rows, pos, bat, kib)
+    gpu_pooled = buf.pooled.permute(0, 2, 1, 3).reshape(-1, w.h_kv, buf.pooled_stride).cpu().numpy()
+    tol = pooled_tolerance(q_rows, kib, pos, bat, w.h_kidx)
+    worst = compare_pooled(gpu_pooled, ora_pooled, tol, pos)
+    assert worst <= 1.0, f"pooled error {worst:.3f} x tolerance"
+    ora_sel = oracle.topk(ora_pooled, pos)
+    gpu_sel = buf.sel.permute(0, 2, 1, 3).reshape(-1, w.h_kv, 16).cpu().numpy()
+    bad, ties, bad_cert, _ = compare_sets(gpu_sel, ora_sel, ora_pooled, pos)
+    assert bad == 0 and bad_cert == 0, (bad, ties, bad_cert)
+
+
+def test_selection_golden_rows_on_gpu():
+    """The hand-derived selection rows, fed to the select kernel as pooled scores."""
+    _need_gpu()
+    from test_oracle_pins import _golden_rows
+    for own, sc, want in _golden_rows():
+        n_kv = (own + 1) * 128
+        d = capi.make_dims(1, 1, n_kv, own * 128 + 3, 8, 1, 128)
+        stride = (own + 4) // 4 * 4
+        pooled = torch.full((1, 1, 1, stride), float("nan"), device="cuda")
+        if sc:
+            pooled[0, 0, 0, :len(sc)] = torch.tensor(sc, dtype=torch.float32)
+        sel = torch.empty((1, 1, 1, 16), dtype=torch.int32, device="cuda")
+        capi.msa_topk_blocks(d, pooled, stride, sel)
+        assert sel[0, 0, 0].tolist() == want
+
+
+@pytest.mark.parametrize("n_q,n_kv,q_pos0,G", [(3000, 3000, 0, 3), (700, 9000, 8300, 2),
+                                                (1, 300000, 299999, 8), (5, 1056768, 1056763, 1)])
+def test_selection_random_scores_bit_exact(n_q, n_kv, q_pos0, G):
+    """fp32 scores with many exact ties and signed zeros: the select kernel and
+    the oracle take the same decision on the same float32 values."""
+    _need_gpu()
+    d = capi.make_dims(1, n_q, n_kv, q_pos0, G, G, 128)
+    nblk = capi.msa_num_blocks(d)
+    stride = (nblk + 3) // 4 * 4
+    g = torch.Generator(device="cpu").manual_seed(n_q + n_kv)
+    sc = torch.randn((G, n_q, stride), generator=g)
+    sc = torch.where(torch.rand(sc.shape, generator=g) < 0.3, torch.round(sc * 2) / 2, sc)
+    sc = torch.where(sc == 0, torch.where(torch.rand(sc.shape, generator=g) < 0.5,
+                                          torch.tensor(-0.0), torch.tensor(0.0)), sc)
+    pooled = sc[None].contiguous().cuda()
+    sel = torch.empty((1, G, n_q, 16), dtype=torch.int32, device="cuda")
+    capi.msa_topk_blocks(d, pooled, stride, sel)
+    own = (q_pos0 + np.arange(n_q)) // 128
+    want = oracle.topk_f32(sc.reshape(G * n_q, stride).numpy(), np.tile(own, G))
+    np.testing.assert_array_equal(sel.cpu().numpy().reshape(G * n_q, 16), want)
+
+
+@pytest.mark.parametrize("w", CASES, ids=lambda w: w.name)
+def test_block_query_lists_bit_exact(w):
+    _need_gpu()
+    d = pipeline.dims_for(w)
+    buf = pipeline.Buffers.allocate(d)
+    sel = wl.random_selection(w, "cpu")
+    buf.sel.copy_(sel)
+    buf.blk_offsets.fill_(-7)
+    buf.entries.fill_(-7)
+    buf.ws.fill_(12345)                      # stale workspace must not matter
+    capi.msa_build_block_query_lists(d, buf.sel, buf.blk_offsets, buf.entries, buf.ws, buf.dev_err)
+    torch.cuda.synchronize()
+    assert int(buf.dev_err[0]) == 0
+    off, ent = oracle.block_query_lists(sel.numpy(), capi.msa_num_blocks(d))
+    np.testing.assert_array_equal(buf.blk_offsets.cpu().numpy(), off.astype(np.int32))
+    np.testing.assert_array_equal(buf.entries.cpu().numpy()[:len(ent)], ent)
+    assert len(ent) == capi.msa_num_entries(d)
+
+
+@pytest.mark.parametrize("w", CASES, ids=lambda w: w.name)
+def test_attention_on_given_selection(w):
+    """Block lists + KV-block-outer attention + merge on a random valid selection."""
+    _need_gpu()
+    d = pipeline.dims_for(w)
+    buf = pipeline.Buffers.allocate(d)
+    inp = wl.make_inputs(w, "cuda")
+    sel = wl.random_selection(w, "cpu")
+    buf.sel.copy_(sel)
+    buf.part_ml.fill_(float("nan"))
+    buf.part_acc.fill_(float("nan"))
+    buf.out.fill_(float("nan"))
+    pipeline.attend(buf, inp["q"], inp["k"], inp["v"])
+    torch.cuda.synchronize()
+    assert int(buf.dev_err[0]) == 0
+    idx, pos, bat = _all_rows(w)
+    q_rows = bits(inp["q"]).reshape(-1, w.h_q, 128)
+    sel_rows = sel.permute(0, 2, 1, 3).reshape(-1, w.h_kv, 16).numpy()
+    out, lse = oracle.attention(q_rows, pos, bat, bits(inp["k"]), bits(inp["v"]), sel_rows, w.scale)
+    gpu_out = buf.out.float().reshape(-1, w.h_q, 128).cpu().numpy()
+    mx, mean = compare_out(gpu_out, out)
+    assert mx <= OUT_MAX_ABS and mean <= OUT_MEAN_ABS, (mx, mean)
+    gpu_lse = buf.lse.reshape(-1, w.h_q).cpu().numpy()
+    assert np.abs(gpu_lse - lse).max() <= LSE_MAX_ABS
+
+
+def test_merge_kernel_against_oracle_merge():
+    """Random pieces (some slots unused) merged by the kernel and by the oracle."""
+    _need_gpu()
+    w = wl.small("merge", 2, 300, 3000, 2700, 8, 2, 64, seed=21)
+    d = pipeline.dims_for(w)
+    sel = wl.random_selection(w, "cpu")
+    g = torch.Generator().manual_seed(5)
+    B, n_q, H = w.batch, w.n_q, w.h_q
+    m = torch.randn((B, n_q, H, 16), generator=g) * 3
+    l = torch.rand((B, n_q, H, 16), generator=g) * 5 + 0.5
+    acc = torch.randn((B, n_q, H, 16, 128), generator=g) * l[..., None]
+    ml = torch.stack([m, l], dim=-1).contiguous()
+    out = torch.empty((B, n_q, H, 128), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((B, n_q, H), device="cuda")
+    capi.msa_merge_partials(d, sel.cuda(), ml.cuda(), acc.contiguous().cuda(), out, lse)
+    R = H // w.h_kv
+    valid = (sel.permute(0, 2, 1, 3)[:, :, torch.arange(H) // R] >= 0).reshape(-1, 16).numpy()
+    o_ref, lse_ref = oracle.merge(valid.astype(np.int32), m.reshape(-1, 16).double().numpy(),
+                                  l.reshape(-1, 16).double().numpy(),
+                                  acc.reshape(-1, 16, 128).double().numpy())
+    o = out.float().reshape(-1, 128).cpu().numpy()
+    assert np.abs(o - o_ref).max() <= 1e-2 * max(1.0, np.abs(o_ref).max())
+    assert np.abs(lse.reshape(-1).cpu().numpy() - lse_ref).max() <= 1e-4
+
+
+@pytest.mark.parametrize("w", [CASES[0], CASES[3], CASES[6]], ids=lambda w: w.name)
+def test_end_to_end_against_oracle(w):
+    """The five calls in sequence vs the oracle's selection and attention."""
+    _need_gpu()
+    d = pipeline.dims_for(w)
+    buf = pipeline.Buffers.allocate(d)
+    inp = wl.make_inputs(w, "cuda")
+    out, lse = pipeline.forward(buf, inp["q"], inp["k"], inp["v"], inp["q_idx"], inp["k_idx"])
+    torch.cuda.synchronize()
+    assert int(buf.dev_err[0]) == 0
+    idx, pos, bat = _all_rows(w)
+    q_idx_rows = bits(inp["q_idx"]).reshape(-1, w.h_kv, w.d_idx)
+    q_rows = bits(inp["q"]).reshape(-1, w.h_q, 128)
+    pooled, sel, o_ref, lse_ref = oracle.forward_rows(q_rows, q_idx_rows, pos, bat, bits(inp["k"]),
+                                                      bits(inp["v"]), bits(inp["k_idx"]), w.scale)
+    gpu_sel = buf.sel.permute(0, 2, 1, 3).reshape(-1, w.h_kv, 16).cpu().numpy()
+    bad, ties, bad_cert, ok = compare_sets(gpu_sel, sel, pooled, pos)
+    assert bad == 0 and bad_cert == 0, (bad, ties, bad_cert)
+    gpu_out = out.float().reshape(-1, w.h_q, 128).cpu().numpy()
+    mx, mean = compare_out(gpu_out[ok], o_ref[ok])
+    assert mx <= OUT_MAX_ABS and mean <= OUT_MEAN_ABS, (mx, mean)
+
+
+def test_repeat_runs_bit_identical():
+    _need_gpu()
+    w = CASES[1]
+    d = pipeline.dims_for(w)
+    inp = wl.make_inputs(w, "cuda")
+    res = []
+    for _ in range(2):
+        buf = pipeline.Buffers.allocate(d)
+        buf.pooled.zero_()
+        o, l = pipeline.forward(buf, inp["q"], inp["k"], inp["v"], inp["q_idx"], inp["k_idx"])
+        res.append((o.view(torch.int16).clone(), l.clone(), buf.sel.clone(), buf.pooled.clone(),
+                    buf.entries.clone()))
+    torch.cuda.synchronize()
+    for a, b in zip(res[0], res[1]):
+        assert torch.equal(a, b)
+
+
+def test_device_error_on_bad_selection():
+    """A selection naming a block after the query's own is reported, not trapped."""
+    _need_gpu()
+    w = wl.small("bad", 1, 300, 300, 0, 4, 1, 64, seed=22)
+    d = pipeline.dims_for(w)
+    buf = pipeline.Buffers.allocate(d)
+    sel = wl.random_selection(w, "cpu")
+    sel[0, 0, 5, 1] = 2          # query 5 lives in block 0
+    buf.sel.copy_(sel)
+    capi.msa_build_block_query_lists(d, buf.sel, buf.blk_offsets, buf.entries, buf.ws, buf.dev_err)
+    torch.cuda.synchronize()
+    assert int(buf.dev_err[0]) == capi.__dict__.get("MSA_DEVERR_BAD_BLOCK", 2)
