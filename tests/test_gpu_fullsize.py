@@ -28,7 +28,7 @@ def _invariants_all_rows(sel: torch.Tensor, w):
     valid = sel >= 0
     assert torch.equal(valid.sum(-1), nsel.expand_as(valid.sum(-1)))
     big = torch.where(valid, sel, torch.full_like(sel, 1 << 30))
-    assert bool((big[..., 1:] > big[..., :-1]).all())           # strictly ascending
+    assert bool(((big[..., 1:] > big[..., :-1]) | ~valid[..., 1:]).all())   # ascending
     assert bool(((sel <= own[..., None]) | ~valid).all())
     last = torch.gather(sel, -1, (nsel - 1).expand(sel.shape[:-1]).unsqueeze(-1).long())
     assert torch.equal(last.squeeze(-1), own.expand(sel.shape[:-1]).to(sel.dtype))
