@@ -128,6 +128,11 @@ def run_step(pipeline, capi, buf, inp, stages=None):
     if ev: ev[5].record()
 
 
+def pipeline_launches():
+    from block_sparse_attention_32_b200 import pipeline
+    return pipeline.LAUNCHES_PER_STEP
+
+
 def barrier(world):
     if world > 1:
         torch.distributed.barrier()
@@ -358,7 +363,7 @@ def main():
         "decode": decode,
         "roofline": roof,
         "clocks": clocks,
-        "gpu_launches": args.steps * 8,
+        "gpu_launches": args.steps * sum(pipeline_launches().values()),
         "e2e": {"value": world * w.n_q / (e2e["ms_per_step"] / 1000.0), "unit": "queries/s",
                 "h2d_bytes_per_step": e2e["h2d_bytes_per_step"],
                 "d2h_bytes_per_step": e2e["d2h_bytes_per_step"]} if e2e else None,

@@ -49,33 +49,38 @@ _P = ctypes.c_void_p
 _PD = ctypes.POINTER(Dims)
 
 
+def load_library(path: str) -> ctypes.CDLL:
+    """Load a build of the library from `path` with every signature declared."""
+    if not os.path.exists(path):
+        raise RuntimeError(
+            f"{path} is missing: build it with "
+            "`python -m block_sparse_attention_32_b200.build` (no CPU fallback exists)")
+    L = ctypes.CDLL(path)
+    L.msa_num_blocks.argtypes = [_PD]
+    L.msa_num_blocks.restype = ctypes.c_int64
+    L.msa_num_entries.argtypes = [_PD]
+    L.msa_num_entries.restype = ctypes.c_int64
+    L.msa_index_score_maxpool.argtypes = [_PD, Tensor, Tensor, _P, ctypes.c_int64, _P, _P]
+    L.msa_topk_blocks.argtypes = [_PD, _P, ctypes.c_int64, _P, _P, _P]
+    L.msa_block_query_lists_workspace.argtypes = [_PD]
+    L.msa_block_query_lists_workspace.restype = ctypes.c_size_t
+    L.msa_build_block_query_lists.argtypes = [_PD, _P, _P, _P, _P, ctypes.c_size_t, _P, _P]
+    L.msa_sparse_attn_fwd.argtypes = [_PD, Tensor, Tensor, Tensor, _P, _P, _P, _P, _P, _P]
+    L.msa_merge_partials.argtypes = [_PD, _P, _P, _P, _P, _P, _P, _P]
+    L.msa_status_string.argtypes = [ctypes.c_int]
+    L.msa_status_string.restype = ctypes.c_char_p
+    for f in (L.msa_index_score_maxpool, L.msa_topk_blocks, L.msa_build_block_query_lists,
+              L.msa_sparse_attn_fwd, L.msa_merge_partials):
+        f.restype = ctypes.c_int
+    return L
+
+
 def lib() -> ctypes.CDLL:
     """Load libmsa.so (raises if it has not been built)."""
     global _lib
     with _lock:
         if _lib is None:
-            if not os.path.exists(LIB_PATH):
-                raise RuntimeError(
-                    f"{LIB_PATH} is missing: build it with "
-                    "`python -m block_sparse_attention_32_b200.build` (no CPU fallback exists)")
-            L = ctypes.CDLL(LIB_PATH)
-            L.msa_num_blocks.argtypes = [_PD]
-            L.msa_num_blocks.restype = ctypes.c_int64
-            L.msa_num_entries.argtypes = [_PD]
-            L.msa_num_entries.restype = ctypes.c_int64
-            L.msa_index_score_maxpool.argtypes = [_PD, Tensor, Tensor, _P, ctypes.c_int64, _P, _P]
-            L.msa_topk_blocks.argtypes = [_PD, _P, ctypes.c_int64, _P, _P, _P]
-            L.msa_block_query_lists_workspace.argtypes = [_PD]
-            L.msa_block_query_lists_workspace.restype = ctypes.c_size_t
-            L.msa_build_block_query_lists.argtypes = [_PD, _P, _P, _P, _P, ctypes.c_size_t, _P, _P]
-            L.msa_sparse_attn_fwd.argtypes = [_PD, Tensor, Tensor, Tensor, _P, _P, _P, _P, _P, _P]
-            L.msa_merge_partials.argtypes = [_PD, _P, _P, _P, _P, _P, _P, _P]
-            L.msa_status_string.argtypes = [ctypes.c_int]
-            L.msa_status_string.restype = ctypes.c_char_p
-            for f in (L.msa_index_score_maxpool, L.msa_topk_blocks, L.msa_build_block_query_lists,
-                      L.msa_sparse_attn_fwd, L.msa_merge_partials):
-                f.restype = ctypes.c_int
-            _lib = L
+            _lib = load_library(LIB_PATH)
     return _lib
 
 

@@ -10,10 +10,12 @@
 // entries (i << 4 | slot) are ascending in the query index i.  Steps:
 //   1. count:   per 128-query tile, a shared-memory histogram over blocks;
 //   2. colscan: per block, exclusive prefix over tiles (in place) + totals;
-//   3. offsets: exclusive scan of the totals over all segments;
+//   3. offsets: exclusive scan of the totals over all segments (chunk sums,
+//      scan of the chunk sums, chunk-local scans);
 //   4. scatter: per tile, queries in ascending order claim consecutive slots
 //      of each block's range, so the order never depends on timing.
-// Workspace: tile histograms [B*G, ntiles, nblk] + totals [B*G*nblk], int32.
+// Workspace: tile histograms [B*G, ntiles, nblk] + totals [B*G*nblk] + chunk
+// sums [ceil(B*G*nblk / 4096)], int32.
 #include "common.cuh"
 
 namespace msa {
@@ -63,22 +65,23 @@ __global__ void __launch_bounds__(256)
   totals[bg * nblk + c] = run;
 }
 
-// single block, 1024 threads: exclusive scan of n values into out[0..n]
-__global__ void __launch_bounds__(1024)
-    csr_offsets_kernel(const int32_t* __restrict__ totals, int64_t n,
-                       int32_t* __restrict__ offsets) {
-  __shared__ int32_t warp_sums[32];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int64_t per = (n + 1023) / 1024;
-  const int64_t lo = min64(n, tid * per), hi = min64(n, lo + per);
-  int32_t s = 0;
-  for (int64_t i = lo; i < hi; ++i) s += totals[i];
-  // block exclusive scan of s
-  int32_t incl = s;
+// Exclusive scan of the per-segment totals into offsets[0..n], in three
+// steps over chunks of kScanChunk values: chunk sums, a scan of the chunk
+// sums, then a block-local scan of each chunk plus its chunk prefix.
+constexpr int kScanThreads = 1024;
+constexpr int kScanPerThread = 4;
+constexpr int kScanChunk = kScanThreads * kScanPerThread;
+
+// inclusive block scan of one value per thread (1024 threads); returns the
+// inclusive prefix, *block_total receives the sum
+__device__ __forceinline__ int32_t block_scan_incl(int32_t v, int32_t* warp_sums,
+                                                   int32_t* block_total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int32_t incl = v;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    const int32_t v = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += v;
+    const int32_t u = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += u;
   }
   if (lane == 31) warp_sums[warp] = incl;
   __syncthreads();
@@ -86,18 +89,69 @@ __global__ void __launch_bounds__(1024)
     int32_t w = warp_sums[lane];
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      const int32_t v = __shfl_up_sync(0xffffffffu, w, o);
-      if (lane >= o) w += v;
+      const int32_t u = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += u;
     }
-    warp_sums[lane] = w;   // inclusive over warps
+    warp_sums[lane] = w;
   }
   __syncthreads();
-  int32_t run = incl - s + (warp > 0 ? warp_sums[warp - 1] : 0);
-  for (int64_t i = lo; i < hi; ++i) {
-    offsets[i] = run;
-    run += totals[i];
+  const int32_t r = incl + (warp > 0 ? warp_sums[warp - 1] : 0);
+  *block_total = warp_sums[31];
+  __syncthreads();
+  return r;
+}
+
+__global__ void __launch_bounds__(kScanThreads)
+    csr_chunk_sums_kernel(const int32_t* __restrict__ totals, int64_t n,
+                          int32_t* __restrict__ chunk_sums) {
+  __shared__ int32_t ws[32];
+  const int64_t base = (int64_t)blockIdx.x * kScanChunk + threadIdx.x * kScanPerThread;
+  int32_t s = 0;
+#pragma unroll
+  for (int k = 0; k < kScanPerThread; ++k)
+    if (base + k < n) s += totals[base + k];
+  int32_t tot;
+  block_scan_incl(s, ws, &tot);
+  if (threadIdx.x == 0) chunk_sums[blockIdx.x] = tot;
+}
+
+// single block: exclusive scan of the chunk sums in place; total to offsets[n]
+__global__ void __launch_bounds__(kScanThreads)
+    csr_chunk_scan_kernel(int32_t* __restrict__ chunk_sums, int64_t nchunks, int64_t n,
+                          int32_t* __restrict__ offsets) {
+  __shared__ int32_t ws[32];
+  int32_t carry = 0;
+  for (int64_t base = 0; base < nchunks; base += kScanThreads) {
+    const int64_t i = base + threadIdx.x;
+    const int32_t v = (i < nchunks) ? chunk_sums[i] : 0;
+    int32_t tot;
+    const int32_t incl = block_scan_incl(v, ws, &tot);
+    if (i < nchunks) chunk_sums[i] = carry + incl - v;
+    carry += tot;
   }
-  if (tid == 1023) offsets[n] = warp_sums[31];
+  if (threadIdx.x == 0) offsets[n] = carry;
+}
+
+__global__ void __launch_bounds__(kScanThreads)
+    csr_chunk_apply_kernel(const int32_t* __restrict__ totals, int64_t n,
+                           const int32_t* __restrict__ chunk_prefix,
+                           int32_t* __restrict__ offsets) {
+  __shared__ int32_t ws[32];
+  const int64_t base = (int64_t)blockIdx.x * kScanChunk + threadIdx.x * kScanPerThread;
+  int32_t v[kScanPerThread];
+  int32_t s = 0;
+#pragma unroll
+  for (int k = 0; k < kScanPerThread; ++k) {
+    v[k] = (base + k < n) ? totals[base + k] : 0;
+    s += v[k];
+  }
+  int32_t tot;
+  int32_t run = block_scan_incl(s, ws, &tot) - s + chunk_prefix[blockIdx.x];
+#pragma unroll
+  for (int k = 0; k < kScanPerThread; ++k) {
+    if (base + k < n) offsets[base + k] = run;
+    run += v[k];
+  }
 }
 
 __global__ void __launch_bounds__(32)
@@ -132,7 +186,9 @@ __global__ void __launch_bounds__(32)
 
 size_t block_lists_workspace(int64_t bgcount, int64_t n_q, int64_t nblk) {
   const int64_t ntiles = (n_q + kCsrTile - 1) / kCsrTile;
-  return (size_t)(bgcount * nblk * (ntiles + 1)) * sizeof(int32_t);
+  const int64_t nseg = bgcount * nblk;
+  const int64_t nchunks = (nseg + kScanChunk - 1) / kScanChunk;
+  return (size_t)(nseg * (ntiles + 1) + nchunks) * sizeof(int32_t);
 }
 
 cudaError_t launch_block_lists(const int32_t* sel, int64_t bgcount, int64_t n_q,
@@ -157,7 +213,13 @@ cudaError_t launch_block_lists(const int32_t* sel, int64_t bgcount, int64_t n_q,
                                                 (int32_t)ntiles, tile_counts, err);
   dim3 g2((unsigned)((nblk + 255) / 256), (unsigned)bgcount);
   csr_colscan_kernel<<<g2, 256, 0, st>>>(tile_counts, totals, (int32_t)nblk, (int32_t)ntiles);
-  csr_offsets_kernel<<<1, 1024, 0, st>>>(totals, bgcount * nblk, offsets);
+  const int64_t nseg = bgcount * nblk;
+  const int64_t nchunks = (nseg + kScanChunk - 1) / kScanChunk;
+  int32_t* chunk_sums = totals + nseg;
+  csr_chunk_sums_kernel<<<(unsigned)nchunks, kScanThreads, 0, st>>>(totals, nseg, chunk_sums);
+  csr_chunk_scan_kernel<<<1, kScanThreads, 0, st>>>(chunk_sums, nchunks, nseg, offsets);
+  csr_chunk_apply_kernel<<<(unsigned)nchunks, kScanThreads, 0, st>>>(totals, nseg, chunk_sums,
+                                                                     offsets);
   csr_scatter_kernel<<<g1, 32, hist_bytes, st>>>(sel, n_q, q_pos0, (int32_t)nblk,
                                                  (int32_t)ntiles, tile_counts, offsets, entries,
                                                  cap);

@@ -74,26 +74,47 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// As above, but the thread may sleep (up to `hint_ns`) until the phase
+// completes, so that waiting warps leave the issue slots to working ones.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity,
+                                                    uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Time limit of every barrier wait.  A wait that runs out sets *abort (a
 // shared flag every role polls), reports MSA_DEVERR_TIMEOUT and returns
 // false, so the block winds down instead of hanging.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
+constexpr uint32_t kWaitSleepNs = 1000000u;       // longest single sleep: 1 ms
 
+static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                           int32_t* err) {
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t it = 0;; ++it) {
+    if (mbar_try_wait_sleep(bar, parity, kWaitSleepNs)) return true;
+    if (*abort) return false;
+    if (global_timer_ns() - t0 > kWaitLimitNs || it > (1u << 30)) {
+      *abort = 1;
+      report(err, MSA_DEVERR_TIMEOUT);
+      return false;
+    }
+  }
+}
+
+// Fast path inline, the bounded sleeping loop out of line (keeps the
+// instruction footprint of the many wait sites small).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           int32_t* err) {
   if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = global_timer_ns();
-  for (uint32_t it = 0;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 63u) {
-      if (*abort) return false;
-      if (global_timer_ns() - t0 > kWaitLimitNs || it > (1u << 30)) {
-        *abort = 1;
-        report(err, MSA_DEVERR_TIMEOUT);
-        return false;
-      }
-    }
-  }
+  return mbar_wait_slow(bar, parity, abort, err);
 }
 
 // ---------------------------------------------------------------------------
@@ -218,6 +239,13 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int b_mn_maj
 // small numeric helpers
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ float u2f(uint32_t u) { return __uint_as_float(u); }
+
+// 2^x with the hardware approximation (MUFU); inputs <= 0 here, results in [0, 1]
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 
 __host__ __device__ __forceinline__ int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
 __host__ __device__ __forceinline__ int64_t max64(int64_t a, int64_t b) { return a > b ? a : b; }

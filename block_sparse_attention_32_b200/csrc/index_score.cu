@@ -8,13 +8,14 @@
 //
 // Two kernels:
 //  * index_score_maxpool_kernel -- prefill / chunked prefill.  A 128-query x
-//    128-key tile of scores is one tcgen05 MMA (M=128, N=128, K=d_idx) whose
+//    256-key tile of scores is one tcgen05 MMA (M=128, N=256, K=d_idx) whose
 //    fp32 accumulator lives in TMEM; the block max is the row max of that
-//    tile, read back with tcgen05.ld (one thread per query row).  Warp roles:
-//    warp 0 issues TMA loads (q_idx tile once, k_idx blocks through a 4-stage
-//    ring), warp 1 issues the MMAs into 4 TMEM accumulators, warps 2-9 reduce
-//    the accumulators (two groups alternating blocks) and stage the maxima in
-//    shared memory, which is written out row-contiguously at the end.
+//    tile, read back with tcgen05.ld (one thread per query row).  Each MMA
+//    step covers two key blocks (N = 256, halving shared-memory operand
+//    traffic per FLOP).  Warp roles: warp 0 issues TMA loads (the q_idx tile
+//    once, pairs of k_idx blocks through a 3-5 stage ring), warp 1 issues the
+//    MMAs into two 256-column TMEM accumulators, warps 2-5 take the two row
+//    maxima of each accumulator and store them.
 //  * index_score_decode_kernel -- one query per sequence (decode): a
 //    streaming scan of k_idx, HBM-bound.  Each warp reads 16-key tiles
 //    straight into mma.sync fragments (16-byte loads) and multiplies them by
@@ -25,19 +26,18 @@ namespace msa {
 
 template <int D>
 struct IdxCfg {
-  static constexpr int kHalves = D / 64;            // 128-byte column panels
-  static constexpr int kTileBytes = 128 * D * 2;    // 128 rows of d_idx bf16
-  static constexpr int kStages = 4;                 // k_idx ring depth
-  static constexpr int kChunkBlocks = 64;           // key blocks per CTA
-  static constexpr int kAcc = 4;                    // TMEM accumulators (128 columns each)
-  static constexpr int kStageStride = kChunkBlocks + 1;
-  static constexpr int kThreads = 320;              // 10 warps
-  static constexpr int kSmemBytes =
-      1024 + kTileBytes * (1 + kStages) + 128 * kStageStride * 4 + 17 * 8 + 16;
+  static constexpr int kHalves = D / 64;             // 128-byte column panels
+  static constexpr int kQBytes = 128 * D * 2;        // 128 query rows
+  static constexpr int kPairBytes = 256 * D * 2;     // two key blocks (256 key rows)
+  static constexpr int kStages = (D == 128) ? 3 : 5; // k_idx ring depth (pairs)
+  static constexpr int kChunkPairs = 64;             // key-block pairs per CTA
+  static constexpr int kThreads = 192;               // TMA, MMA, 4 epilogue warps
+  static constexpr int kBars = 2 * kStages + 1 + 4;
+  static constexpr int kSmemBytes = 1024 + kQBytes + kStages * kPairBytes + kBars * 8 + 16;
 };
 
 template <int D>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(192, 1)
     index_score_maxpool_kernel(const __grid_constant__ CUtensorMap tm_q,
                                const __grid_constant__ CUtensorMap tm_k, int64_t n_q,
                                int64_t q_pos0, int32_t G, int32_t h_kidx, int32_t n_qtiles,
@@ -47,15 +47,14 @@ __global__ void __launch_bounds__(320, 1)
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   uint8_t* sq = base;
-  uint8_t* sk = base + C::kTileBytes;
-  float* stage = reinterpret_cast<float*>(sk + C::kStages * C::kTileBytes);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(stage + 128 * C::kStageStride);
-  uint64_t* full = bars;          // [4] k stage loaded
-  uint64_t* empty = bars + 4;     // [4] k stage consumed by the MMAs
-  uint64_t* qfull = bars + 8;     // q tile loaded
-  uint64_t* accfull = bars + 9;   // [4] accumulator ready
-  uint64_t* accempty = bars + 13; // [4] accumulator drained
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 17);
+  uint8_t* sk = base + C::kQBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sk + C::kStages * C::kPairBytes);
+  uint64_t* full = bars;                        // [kStages] key pair loaded
+  uint64_t* empty = bars + C::kStages;          // [kStages] key pair consumed by the MMAs
+  uint64_t* qfull = bars + 2 * C::kStages;      // q tile loaded
+  uint64_t* accfull = qfull + 1;                // [2] accumulator ready
+  uint64_t* accempty = qfull + 3;               // [2] accumulator drained
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -66,19 +65,22 @@ __global__ void __launch_bounds__(320, 1)
   const int64_t q0 = (int64_t)qt * 128;
   const int64_t q_last = min64(q0 + 127, n_q - 1);
   const int64_t nb_tile = (q_pos0 + q_last) / kBlock;   // candidates of the tile's last row
-  const int64_t c0 = (int64_t)kc * C::kChunkBlocks;
+  const int64_t c0 = (int64_t)kc * 2 * C::kChunkPairs;
   if (c0 >= nb_tile) return;                            // uniform: nothing to score
-  const int nb = (int)min64(C::kChunkBlocks, nb_tile - c0);
+  const int nb = (int)min64(2 * C::kChunkPairs, nb_tile - c0);
+  const int np = (nb + 1) >> 1;                         // MMA steps of 256 keys
   const int hk = (h_kidx == 1) ? 0 : g;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < C::kStages; ++i) {
       mbar_init(full + i, 1);
       mbar_init(empty + i, 1);
+    }
+    mbar_init(qfull, 1);
+    for (int i = 0; i < 2; ++i) {
       mbar_init(accfull + i, 1);
       mbar_init(accempty + i, 4);
     }
-    mbar_init(qfull, 1);
     *abort_flag = 0;
     fence_mbarrier_init();
   }
@@ -95,76 +97,82 @@ __global__ void __launch_bounds__(320, 1)
     if (lane == 0) {
       prefetch_tensormap(&tm_q);
       prefetch_tensormap(&tm_k);
-      mbar_arrive_expect_tx(qfull, C::kTileBytes);
+      mbar_arrive_expect_tx(qfull, C::kQBytes);
       for (int h = 0; h < C::kHalves; ++h)
         tma_load_4d(sq + h * 16384, &tm_q, qfull, h * 64, g, (int32_t)q0, b);
-      for (int i = 0; i < nb; ++i) {
+      for (int i = 0; i < np; ++i) {
         const int s = i % C::kStages;
         if (i >= C::kStages &&
             !mbar_wait(empty + s, ((i / C::kStages) - 1) & 1, abort_flag, err))
           break;
-        mbar_arrive_expect_tx(full + s, C::kTileBytes);
+        mbar_arrive_expect_tx(full + s, C::kPairBytes);
+        // one box of 256 key rows per 64-column panel (rows past n_kv read as 0)
         for (int h = 0; h < C::kHalves; ++h)
-          tma_load_4d(sk + s * C::kTileBytes + h * 16384, &tm_k, full + s, h * 64,
-                      (int32_t)((c0 + i) * kBlock), hk, b);
+          tma_load_4d(sk + s * C::kPairBytes + h * 32768, &tm_k, full + s, h * 64,
+                      (int32_t)((c0 + 2 * i) * kBlock), hk, b);
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(128, 128, 0);
+      constexpr uint32_t idesc = idesc_bf16_f32(128, 256, 0);
       const uint32_t qa = smem_u32(sq);
       bool ok = mbar_wait(qfull, 0, abort_flag, err);
-      for (int i = 0; ok && i < nb; ++i) {
-        const int s = i % C::kStages, a = i % C::kAcc;
+      for (int i = 0; ok && i < np; ++i) {
+        const int s = i % C::kStages, a = i & 1;
         if (!mbar_wait(full + s, (i / C::kStages) & 1, abort_flag, err)) break;
-        if (i >= C::kAcc && !mbar_wait(accempty + a, ((i / C::kAcc) - 1) & 1, abort_flag, err))
-          break;
+        if (i >= 2 && !mbar_wait(accempty + a, ((i >> 1) - 1) & 1, abort_flag, err)) break;
         tc_fence_after();
-        const uint32_t ka = smem_u32(sk + s * C::kTileBytes);
+        const uint32_t ka = smem_u32(sk + s * C::kPairBytes);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          umma_bf16(tmem + a * 128, smem_desc_sw128(qa + off, 16, 1024),
-                    smem_desc_sw128(ka + off, 16, 1024), idesc, kk > 0 ? 1u : 0u);
+          umma_bf16(tmem + a * 256,
+                    smem_desc_sw128(qa + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                    smem_desc_sw128(ka + (kk >> 2) * 32768 + (kk & 3) * 32, 16, 1024), idesc,
+                    kk > 0 ? 1u : 0u);
         }
         umma_commit(empty + s);
         umma_commit(accfull + a);
       }
     }
   } else {
-    const int grp = (warp - 2) >> 2;     // accumulators a with a % 2 == grp
-    const int quarter = warp & 3;        // TMEM lanes 32*quarter .. +31
+    // epilogue: thread = query row; columns [0,128) = block c, [128,256) = block c+1
+    const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
-    for (int i = grp; i < nb; i += 2) {
-      const int a = i % C::kAcc;
-      if (!mbar_wait(accfull + a, (i / C::kAcc) & 1, abort_flag, err)) break;
+    const int64_t q = q0 + row;
+    const int64_t own = (q_pos0 + q) / kBlock;
+    float* prow = pooled + (((int64_t)b * G + g) * n_q + q) * stride;
+    for (int i = 0; i < np; ++i) {
+      const int a = i & 1;
+      if (!mbar_wait(accfull + a, (i >> 1) & 1, abort_flag, err)) break;
       tc_fence_after();
-      float m = -INFINITY;
+      float m[2];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(tmem + lane_base + a * 128 + j * 32, r);
-        tmem_ld_wait();
+      for (int hb = 0; hb < 2; ++hb) {
+        float mx = -INFINITY;
 #pragma unroll
-        for (int x = 0; x < 32; ++x) m = fmaxf(m, u2f(r[x]));
+        for (int j = 0; j < 4; j += 2) {
+          uint32_t r0[32], r1[32];
+          tmem_ld_32x32b_x32(tmem + lane_base + a * 256 + hb * 128 + j * 32, r0);
+          tmem_ld_32x32b_x32(tmem + lane_base + a * 256 + hb * 128 + (j + 1) * 32, r1);
+          tmem_ld_wait();
+#pragma unroll
+          for (int x = 0; x < 32; ++x) mx = fmaxf(mx, fmaxf(u2f(r0[x]), u2f(r1[x])));
+        }
+        m[hb] = mx;
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(accempty + a);
-      stage[row * C::kStageStride + i] = m;
+      const int64_t c = c0 + 2 * i;
+      if (q < n_q) {
+        if (c + 1 < own && 2 * i + 1 < nb) {
+          *reinterpret_cast<float2*>(prow + c) = make_float2(m[0], m[1]);
+        } else if (c < own) {
+          prow[c] = m[0];
+        }
+      }
     }
-  }
-  __syncthreads();
-
-  // row-contiguous write-out of the staged block maxima (only blocks c < own(t))
-  float* prow = pooled + ((int64_t)b * G + g) * n_q * stride;
-  for (int idx = threadIdx.x; idx < 128 * nb; idx += C::kThreads) {
-    const int r = idx / nb, i = idx - r * nb;
-    const int64_t q = q0 + r;
-    if (q >= n_q) continue;
-    const int64_t c = c0 + i;
-    if (c < (q_pos0 + q) / kBlock) prow[q * stride + c] = stage[r * C::kStageStride + i];
   }
 
   tc_fence_before();
@@ -292,7 +300,8 @@ cudaError_t launch_index_score_prefill(const CUtensorMap& tm_q, const CUtensorMa
   const int64_t n_qtiles = (n_q + 127) / 128;
   const int64_t max_nb = (q_pos0 + n_q - 1) / kBlock;
   if (max_nb == 0) return cudaSuccess;
-  const int64_t n_chunks = (max_nb + 63) / 64;
+  const int64_t per_cta = 2 * IdxCfg<128>::kChunkPairs;
+  const int64_t n_chunks = (max_nb + per_cta - 1) / per_cta;
   dim3 grid((unsigned)(n_chunks * G), (unsigned)n_qtiles, (unsigned)batch);
   if (d_idx == 128) {
     auto k = index_score_maxpool_kernel<128>;

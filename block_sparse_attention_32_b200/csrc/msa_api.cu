@@ -147,9 +147,10 @@ msa_status msa_index_score_maxpool(const msa_dims* d, msa_tensor q_idx, msa_tens
   if ((s = make_map(&tq, q_idx.ptr, d->d_idx, G, d->n_q, d->batch, q_idx.s_head, q_idx.s_tok,
                     q_idx.s_batch, 1, 128)) != MSA_OK)
     return s;
-  // k_idx [B, h_kidx, n_kv, d_idx]: dims {d_idx, n_kv, h_kidx, B}, box {64, 128, 1, 1}
+  // k_idx [B, h_kidx, n_kv, d_idx]: dims {d_idx, n_kv, h_kidx, B}, box {64, 256, 1, 1}
+  // (two key blocks per load)
   if ((s = make_map(&tk, k_idx.ptr, d->d_idx, d->n_kv, d->h_kidx, d->batch, k_idx.s_tok,
-                    k_idx.s_head, k_idx.s_batch, 128, 1)) != MSA_OK)
+                    k_idx.s_head, k_idx.s_batch, 256, 1)) != MSA_OK)
     return s;
   return from_cuda(msa::launch_index_score_prefill(tq, tk, d->d_idx, d->batch, d->n_q,
                                                    d->q_pos0, G, d->h_kidx, pooled,

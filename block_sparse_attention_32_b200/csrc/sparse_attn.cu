@@ -1,9 +1,9 @@
 // KV-block-outer sparse attention: for every (batch, group, KV block) segment
 // of the block->query lists, the block's K and V tiles are loaded into shared
-// memory by TMA once, the query rows that chose it are gathered into 128-row
-// tiles, and S = Q K^T, the softmax piece and O = P V run on the tcgen05 tensor
-// cores with fp32 accumulators in TMEM.  Each (query, head, slot) gets a
-// piece (m, l, acc) that the merge kernel combines.
+// memory by TMA once per work item, the query rows that chose the block are
+// gathered into 128-row tiles, and S = Q K^T, the softmax piece and O = P V
+// run on the tcgen05 tensor cores with fp32 accumulators in TMEM.  Each
+// (query, head, slot) gets a piece (m, l, acc) that the merge kernel combines.
 //
 // Source: page "MSA 稀疏注意力三国杀", section "MSA 架构：粗筛 + 精算" (main
 // branch: full attention over the selected blocks only) and section "Kernel
@@ -12,151 +12,350 @@
 // survey page, MSA entry (exact softmax attention); chenxutan page, standard
 // attention softmax(Q K^T / sqrt(d_k)) V.
 //
-// Tile shapes: a 128-row tile holds 128 / R query entries x R heads of the
-// group (R = h_q / h_kv).  Shared memory (per CTA, 96 KB, two CTAs per SM):
-//   sq: Q tile, later overwritten by P (bf16, 128 x 128, K-major, 128B swizzle)
-//   sk: K block (keys x dims, K-major for S = Q K^T)
-//   sv: V block (keys x dims, N(dims)-major for O = P V)
-// TMEM: columns [0,128) hold S, [128,256) hold O.
+// A 128-row tile ("chunk") holds 128 / R query entries x R heads of one group
+// (R = h_q / h_kv).  Work items are runs of W consecutive entries; an item
+// splits into pieces (one per segment = one K/V block) and pieces into
+// chunks.  The kernel is persistent (one CTA per SM) and warp-specialised so
+// that consecutive chunks overlap:
+//   warp 0      scheduler:    walks the CTA's items (32-ary search of the
+//                             segment offsets) and publishes one descriptor
+//                             per chunk -- (b, g, block, count, piece, flags)
+//                             and its entries -- in an 8-deep shared ring
+//   warp 1      MMA issuer:   S(n) = Q K^T, then O(n-1) = P V  (TMEM owner)
+//   warp 2      TMA producer: K and V of each piece; K of the next piece is
+//                             loaded as soon as the last S MMA of the current
+//                             one is done, V as soon as its last P V is done
+//   warps 3-6   gather:       cp.async of the chunk's Q rows into a 4-deep ring
+//   warps 7-10  softmax:      S -> (m, l), P = bf16(e^{s-m}) into the Q buffer
+//   warps 11-14 epilogue:     O -> the (m, l, acc) pieces in global memory
+// Shared memory: K 32 KB, V 32 KB, 4 x 32 KB Q/P (128B-swizzled K-major
+// tiles; V is read N-major for P V).  TMEM: S in columns [0,256), O in
+// [256,512), two buffers of 128 columns each.
 #include "common.cuh"
 
 namespace msa {
 
-constexpr int kAttnThreads = 128;
-constexpr int kAttnChunksPerItem = 8;
-constexpr int kAttnSmemBytes = 1024 + 3 * 32768 + 256 + 128 * 4;
+constexpr int kAttnThreads = 480;
+constexpr int kAttnMaxChunksPerItem = 8;
+constexpr int kQRing = 4;              // Q/P tiles in flight
+constexpr int kDescRing = 8;           // chunk descriptors in flight
+
+struct alignas(16) ChunkDesc {
+  int32_t b, g, c, cnt;                // cnt < 0: no more work
+  int32_t piece, first, last, pad;
+  int32_t ent[128];
+};
+
+constexpr int kOffK = 0;               // 32768: [K lo | K hi]
+constexpr int kOffV = 32768;           // 32768: [V lo | V hi]
+constexpr int kOffQP = 65536;          // kQRing x 32768: Q tile, then P
+constexpr int kOffML = kOffQP + kQRing * 32768;          // 2 x 128 float2: (m, l) per row
+constexpr int kOffDesc = kOffML + 2048;                  // kDescRing descriptors
+constexpr int kOffBar = kOffDesc + kDescRing * (int)sizeof(ChunkDesc);
+constexpr int kNumBars = 4 + 3 * kQRing + 6 + 2 * kDescRing;
+constexpr int kOffMisc = kOffBar + kNumBars * 8;         // TMEM base, abort flag
+constexpr int kAttnSmemBytes = 1024 + kOffMisc + 64;
+
+enum {
+  BAR_K_FULL = 0, BAR_K_EMPTY = 1, BAR_V_FULL = 2, BAR_V_EMPTY = 3,
+  BAR_Q_FULL = 4, BAR_QP_EMPTY = 4 + kQRing, BAR_P_FULL = 4 + 2 * kQRing,
+  BAR_S_FULL = 4 + 3 * kQRing, BAR_O_FULL = BAR_S_FULL + 2, BAR_O_EMPTY = BAR_S_FULL + 4,
+  BAR_D_FULL = BAR_S_FULL + 6, BAR_D_EMPTY = BAR_D_FULL + kDescRing
+};
+
+__device__ __forceinline__ void st_global_v8(float* p, const uint32_t* r) {
+  asm volatile("st.global.v8.f32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p),
+               "f"(u2f(r[0])), "f"(u2f(r[1])), "f"(u2f(r[2])), "f"(u2f(r[3])), "f"(u2f(r[4])),
+               "f"(u2f(r[5])), "f"(u2f(r[6])), "f"(u2f(r[7]))
+               : "memory");
+}
+
+struct AttnArgs {
+  const __nv_bfloat16* q;
+  int64_t qs_b, qs_t, qs_h;
+  const int32_t* blk_offsets;
+  const int32_t* entries;
+  int64_t n_seg, n_entries, n_items, W;
+  int64_t n_q, q_pos0;
+  int32_t G, H, nblk;
+  float scale;
+  float* part_ml;
+  float* part_acc;
+  int32_t* err;
+};
+
+// Largest s in [lo, n_seg) with off[s] <= pos, by a 32-ary search: each round
+// the 31 probes of the warp split the range.  Called by a full warp.
+__device__ __forceinline__ int64_t warp_find_segment(const int32_t* off, int64_t lo,
+                                                     int64_t hi, int64_t pos, int lane) {
+  while (hi - lo > 1) {
+    const int64_t step = (hi - lo + 31) >> 5;
+    const int64_t idx = lo + (int64_t)lane * step;
+    const bool le = lane >= 1 && idx < hi && off[idx] <= pos;
+    const int k = __popc(__ballot_sync(0xffffffffu, le));
+    lo = lo + (int64_t)k * step;
+    hi = min64(hi, lo + step);
+  }
+  return lo;
+}
 
 template <int R>
-__global__ void __launch_bounds__(kAttnThreads, 2)
+__global__ void __launch_bounds__(kAttnThreads, 1)
     sparse_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k,
                            const __grid_constant__ CUtensorMap tm_v,
-                           const __nv_bfloat16* __restrict__ q, int64_t qs_b, int64_t qs_t,
-                           int64_t qs_h, const int32_t* __restrict__ blk_offsets,
-                           const int32_t* __restrict__ entries, int64_t n_seg,
-                           int64_t n_entries, int64_t n_q, int64_t q_pos0, int32_t G,
-                           int32_t H, int32_t nblk, float scale, float* __restrict__ part_ml,
-                           float* __restrict__ part_acc, int32_t* err) {
-  constexpr int CH = 128 / R;                       // query entries per 128-row tile
-  constexpr int W = CH * kAttnChunksPerItem;        // entries per CTA
+                           const __grid_constant__ AttnArgs a) {
+  constexpr int CH = 128 / R;
   constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128, 0);
   constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 128, 1);
-  const float scale_log2 = scale * 1.4426950408889634f;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint8_t* sq = base;
-  uint8_t* sk = base + 32768;
-  uint8_t* sv = base + 65536;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(base + 98304);
-  uint64_t* kv_full = bars;
-  uint64_t* mma_done = bars + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  int32_t* ent_s = reinterpret_cast<int32_t*>(base + 98304 + 256);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(base + kOffBar);
+  float2* ml_s = reinterpret_cast<float2*>(base + kOffML);
+  ChunkDesc* desc = reinterpret_cast<ChunkDesc*>(base + kOffDesc);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(base + kOffMisc + 4);
 
-  const int tid = threadIdx.x, warp = tid >> 5;
-  const int64_t e0 = (int64_t)blockIdx.x * W;
-  const int64_t e1 = min64(e0 + W, n_entries);
-
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) {
-    mbar_init(kv_full, 1);
-    mbar_init(mma_done, 1);
+    mbar_init(bar + BAR_K_FULL, 1);
+    mbar_init(bar + BAR_K_EMPTY, 1);
+    mbar_init(bar + BAR_V_FULL, 1);
+    mbar_init(bar + BAR_V_EMPTY, 1);
+    for (int i = 0; i < kQRing; ++i) {
+      mbar_init(bar + BAR_Q_FULL + i, 128);
+      mbar_init(bar + BAR_QP_EMPTY + i, 1);
+      mbar_init(bar + BAR_P_FULL + i, 128);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar + BAR_S_FULL + i, 1);
+      mbar_init(bar + BAR_O_FULL + i, 1);
+      mbar_init(bar + BAR_O_EMPTY + i, 128);
+    }
+    for (int i = 0; i < kDescRing; ++i) {
+      mbar_init(bar + BAR_D_FULL + i, 1);
+      mbar_init(bar + BAR_D_EMPTY + i, 128 + 1);   // epilogue threads + TMA producer
+    }
     *abort_flag = 0;
     fence_mbarrier_init();
   }
-  if (warp == 0) {
-    tmem_alloc(tmem_slot, 256);
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-  const uint32_t sq_a = smem_u32(sq), sk_a = smem_u32(sk), sv_a = smem_u32(sv);
+  int32_t* err = a.err;
+  // ring of depth D: the n-th use is ready / the (n-D)-th use has been released
+  auto Wuse = [&](int id, int depth, int64_t n) {
+    return mbar_wait(bar + id + (int)(n % depth), (uint32_t)((n / depth) & 1), abort_flag, err);
+  };
+  auto Wfree = [&](int id, int depth, int64_t n) {
+    return n < depth || mbar_wait(bar + id + (int)(n % depth),
+                                  (uint32_t)(((n / depth) + 1) & 1), abort_flag, err);
+  };
 
-  uint32_t kv_phase = 0, mma_phase = 0;
-  int64_t pos = e0;
-  while (pos < e1) {
-    if (__syncthreads_or(*abort_flag != 0)) break;
-    // segment holding entry `pos`: the last s with blk_offsets[s] <= pos
-    int64_t lo = 0, hi = n_seg;   // invariant: offsets[lo] <= pos < offsets[hi]
-    while (hi - lo > 1) {
-      const int64_t mid = (lo + hi) >> 1;
-      if (blk_offsets[mid] <= pos) lo = mid; else hi = mid;
+  if (warp == 0) {
+    // ---------------- scheduler ----------------
+    int64_t chunk = 0, piece = 0;
+    bool ok = true;
+    auto claim = [&](int64_t n) {      // lane 0 waits, the warp follows
+      bool r = true;
+      if (lane == 0) r = Wfree(BAR_D_EMPTY, kDescRing, n);
+      return __shfl_sync(0xffffffffu, r ? 1 : 0, 0) != 0;
+    };
+    for (int64_t item = blockIdx.x; ok && item < a.n_items; item += gridDim.x) {
+      const int64_t e0 = item * a.W;
+      const int64_t e1 = min64(e0 + a.W, a.n_entries);
+      int64_t pos = e0;
+      int64_t seg = warp_find_segment(a.blk_offsets, 0, a.n_seg, pos, lane);
+      while (pos < e1) {
+        const int64_t pend = min64(e1, (int64_t)a.blk_offsets[seg + 1]);
+        if (pend <= pos) {             // fewer entries listed than the sizes imply
+          if (lane == 0) {
+            report(err, MSA_DEVERR_BAD_ENTRY);
+            *abort_flag = 1;
+          }
+          ok = false;
+          break;
+        }
+        const int64_t bg = seg / a.nblk;
+        const int32_t c = (int32_t)(seg - bg * a.nblk);
+        const int32_t b = (int32_t)(bg / a.G), g = (int32_t)(bg - (int64_t)b * a.G);
+        for (int64_t cpos = pos; cpos < pend; cpos += CH) {
+          if (!claim(chunk)) {
+            ok = false;
+            break;
+          }
+          ChunkDesc& d = desc[chunk % kDescRing];
+          const int cnt = (int)min64(CH, pend - cpos);
+          for (int i = lane; i < CH; i += 32) d.ent[i] = (i < cnt) ? a.entries[cpos + i] : -1;
+          if (lane == 0) {
+            d.b = b;
+            d.g = g;
+            d.c = c;
+            d.cnt = cnt;
+            d.piece = (int32_t)piece;
+            d.first = cpos == pos;
+            d.last = cpos + CH >= pend;
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar + BAR_D_FULL + (int)(chunk % kDescRing));
+          ++chunk;
+        }
+        if (!ok) break;
+        ++piece;
+        pos = pend;
+        if (pos < e1) seg = warp_find_segment(a.blk_offsets, seg + 1, a.n_seg, pos, lane);
+      }
     }
-    const int64_t seg = lo;
-    const int64_t pend = min64(e1, blk_offsets[seg + 1]);
-    if (pend <= pos) {               // fewer entries listed than expected
-      if (tid == 0) report(err, MSA_DEVERR_BAD_ENTRY);
-      break;
+    if (ok && claim(chunk)) {          // end marker
+      if (lane == 0) {
+        desc[chunk % kDescRing].cnt = -1;
+        mbar_arrive(bar + BAR_D_FULL + (int)(chunk % kDescRing));
+      }
     }
-    const int64_t bg = seg / nblk;
-    const int32_t c = (int32_t)(seg - bg * nblk);
-    const int32_t b = (int32_t)(bg / G), g = (int32_t)(bg - (int64_t)b * G);
-
-    if (tid == 0) {
-      mbar_arrive_expect_tx(kv_full, 65536);
-      tma_load_4d(sk, &tm_k, kv_full, 0, c * kBlock, g, b);
-      tma_load_4d(sk + 16384, &tm_k, kv_full, 64, c * kBlock, g, b);
-      tma_load_4d(sv, &tm_v, kv_full, 0, c * kBlock, g, b);
-      tma_load_4d(sv + 16384, &tm_v, kv_full, 64, c * kBlock, g, b);
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      int64_t pn = -1, pp = 0, v_ready = -1, last_s_piece = -1;
+      bool plast = false, ok = true;
+      auto issue_pv = [&](int64_t n, int64_t p, bool last) {
+        const int qb = (int)(n % kQRing), ob = (int)(n & 1);
+        if (p != v_ready) {
+          if (!Wuse(BAR_V_FULL, 1, p)) return false;
+          v_ready = p;
+        }
+        if (!Wuse(BAR_P_FULL, kQRing, n)) return false;
+        tc_fence_after();
+        const uint32_t pa = smem_u32(base + kOffQP + qb * 32768);
+        const uint32_t va = smem_u32(base + kOffV);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t aoff = (kk >> 2) * 16384 + (kk & 3) * 32;
+          umma_bf16(tmem + 256 + ob * 128, smem_desc_sw128(pa + aoff, 16, 1024),
+                    smem_desc_sw128(va + kk * 2048, 16384, 1024), kIdescPV, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(bar + BAR_O_FULL + ob);
+        umma_commit(bar + BAR_QP_EMPTY + qb);
+        if (last) umma_commit(bar + BAR_V_EMPTY);
+        return true;
+      };
+      for (int64_t n = 0;; ++n) {
+        if (!Wuse(BAR_D_FULL, kDescRing, n)) { ok = false; break; }
+        const ChunkDesc& d = desc[n % kDescRing];
+        if (d.cnt < 0) break;
+        const int64_t p = d.piece;
+        const bool first = d.first != 0, last = d.last != 0;
+        const int qb = (int)(n % kQRing), sb = (int)(n & 1);
+        if (first) {
+          // drain the pending P V before waiting for the next block's K
+          if (pn >= 0 && !issue_pv(pn, pp, plast)) { ok = false; break; }
+          pn = -1;
+          if (!Wuse(BAR_K_FULL, 1, p)) { ok = false; break; }
+        }
+        if (!Wuse(BAR_Q_FULL, kQRing, n)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t qa = smem_u32(base + kOffQP + qb * 32768);
+        const uint32_t ka = smem_u32(base + kOffK);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          umma_bf16(tmem + sb * 128, smem_desc_sw128(qa + off, 16, 1024),
+                    smem_desc_sw128(ka + off, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(bar + BAR_S_FULL + sb);
+        if (last) {
+          umma_commit(bar + BAR_K_EMPTY);
+          last_s_piece = p;
+        }
+        if (pn >= 0 && !issue_pv(pn, pp, plast)) { ok = false; break; }
+        pn = n;
+        pp = p;
+        plast = last;
+      }
+      if (ok && pn >= 0 && issue_pv(pn, pp, plast)) {
+        // let the last completions land before the block can exit
+        Wuse(BAR_QP_EMPTY, kQRing, pn);
+        if (plast) Wuse(BAR_V_EMPTY, 1, pp);
+        if (last_s_piece >= 0) Wuse(BAR_K_EMPTY, 1, last_s_piece);
+      }
     }
-
-    for (int64_t cpos = pos; cpos < pend; cpos += CH) {
-      const int cnt = (int)min64(CH, pend - cpos);
-      if (tid < CH) ent_s[tid] = (tid < cnt) ? entries[cpos + tid] : -1;
-      if (__syncthreads_or(*abort_flag != 0)) break;
-
-      // gather the Q rows of this tile (zero rows past the entry count)
+  } else if (warp == 2) {
+    // ---------------- TMA producer: K/V of every piece ----------------
+    if (lane == 0) {
+      prefetch_tensormap(&tm_k);
+      prefetch_tensormap(&tm_v);
+      for (int64_t n = 0;; ++n) {
+        if (!Wuse(BAR_D_FULL, kDescRing, n)) break;
+        const ChunkDesc& d = desc[n % kDescRing];
+        if (d.cnt < 0) break;
+        if (d.first) {
+          const int64_t p = d.piece;
+          const int32_t b = d.b, g = d.g, c = d.c;
+          if (!Wfree(BAR_K_EMPTY, 1, p)) break;
+          mbar_arrive_expect_tx(bar + BAR_K_FULL, 32768);
+          tma_load_4d(base + kOffK, &tm_k, bar + BAR_K_FULL, 0, c * kBlock, g, b);
+          tma_load_4d(base + kOffK + 16384, &tm_k, bar + BAR_K_FULL, 64, c * kBlock, g, b);
+          if (!Wfree(BAR_V_EMPTY, 1, p)) break;
+          mbar_arrive_expect_tx(bar + BAR_V_FULL, 32768);
+          tma_load_4d(base + kOffV, &tm_v, bar + BAR_V_FULL, 0, c * kBlock, g, b);
+          tma_load_4d(base + kOffV + 16384, &tm_v, bar + BAR_V_FULL, 64, c * kBlock, g, b);
+        }
+        mbar_arrive(bar + BAR_D_EMPTY + (int)(n % kDescRing));
+      }
+    }
+  } else if (warp < 7) {
+    // ---------------- gather: Q rows of each chunk ----------------
+    const int gt = tid - 96;   // 0..127
+    const int ch = gt & 15;
+    for (int64_t n = 0;; ++n) {
+      if (!Wuse(BAR_D_FULL, kDescRing, n)) break;
+      const ChunkDesc& d = desc[n % kDescRing];
+      if (d.cnt < 0) break;
+      const int qb = (int)(n % kQRing);
+      const int32_t b = d.b, g = d.g;
+      if (!Wfree(BAR_QP_EMPTY, kQRing, n)) break;
+      uint8_t* sq = base + kOffQP + qb * 32768;
+      const __nv_bfloat16* qbase = a.q + (int64_t)b * a.qs_b + (int64_t)(g * R) * a.qs_h + ch * 8;
 #pragma unroll 4
       for (int it = 0; it < 16; ++it) {
-        const int idx = it * kAttnThreads + tid;
-        const int row = idx >> 4, ch = idx & 15;
-        const int e = ent_s[row / R];
-        const int hr = row % R;
+        const int row = it * 8 + (gt >> 4);
+        const int e = d.ent[row / R];
         const int64_t qi = (int64_t)(e >> 4);
-        const bool ok = (e >= 0) && (qi < n_q);
-        const __nv_bfloat16* src =
-            ok ? q + (int64_t)b * qs_b + qi * qs_t + (int64_t)(g * R + hr) * qs_h + ch * 8 : q;
-        uint8_t* dst = sq + (ch >> 3) * 16384 + row * 128 + ((((ch & 7) ^ (row & 7))) << 4);
+        const bool ok = (e >= 0) && (qi < a.n_q);
+        const __nv_bfloat16* src = ok ? qbase + qi * a.qs_t + (int64_t)(row % R) * a.qs_h : a.q;
+        uint8_t* dst = sq + (ch >> 3) * 16384 + row * 128 + (((ch & 7) ^ (row & 7)) << 4);
         cp_async_16(dst, src, ok ? 16u : 0u);
       }
       cp_async_wait_all();
       fence_proxy_async_smem();
-      __syncthreads();
-
-      // S = Q K^T
-      if (tid == 0) {
-        bool ok = true;
-        if (cpos == pos) ok = mbar_wait(kv_full, kv_phase, abort_flag, err);
-        if (ok) {
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-            umma_bf16(tmem, smem_desc_sw128(sq_a + off, 16, 1024),
-                      smem_desc_sw128(sk_a + off, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
-          }
-          umma_commit(mma_done);
-        }
-      }
-      mbar_wait(mma_done, mma_phase, abort_flag, err);
-      mma_phase ^= 1;
+      mbar_arrive(bar + BAR_Q_FULL + qb);
+    }
+  } else if (warp < 11) {
+    // ---------------- softmax: S -> P, (m, l) ----------------
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    const float scale_log2 = a.scale * 1.4426950408889634f;
+    for (int64_t n = 0;; ++n) {
+      if (!Wuse(BAR_D_FULL, kDescRing, n)) break;
+      const ChunkDesc& d = desc[n % kDescRing];
+      if (d.cnt < 0) break;
+      const int qb = (int)(n % kQRing), sb = (int)(n & 1);
+      const int e = d.ent[row / R];
+      const int32_t c = d.c;
+      if (!Wuse(BAR_S_FULL, 2, n)) break;
+      if (!Wfree(BAR_O_EMPTY, 2, n)) break;
       tc_fence_after();
-
-      // softmax piece of row `tid`
-      const int row = tid;
-      const int e = ent_s[row / R];
-      const int hr = row % R;
       const int64_t qi = (int64_t)(e >> 4);
-      const int slot = e & 15;
-      bool valid = (e >= 0) && (qi < n_q);
-      int lim = 127;   // last key offset inside the block visible to the row
+      bool valid = (e >= 0) && (qi < a.n_q);
+      int lim = 127;
       if (valid) {
-        const int64_t t = q_pos0 + qi;
-        const int64_t rel = t - (int64_t)c * kBlock;
+        const int64_t rel = a.q_pos0 + qi - (int64_t)c * kBlock;
         if (rel < 0) {
           valid = false;
           report(err, MSA_DEVERR_BAD_ENTRY);
@@ -164,106 +363,123 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
           lim = (int)rel;
         }
       }
-      float sv_[128];
-#pragma unroll
+      const uint32_t s_addr = tmem + lane_base + sb * 128;
+      float mx = -INFINITY;
+#pragma unroll 1
       for (int j = 0; j < 4; ++j) {
         uint32_t r[32];
-        tmem_ld_32x32b_x32(tmem + lane_base + j * 32, r);
+        tmem_ld_32x32b_x32(s_addr + j * 32, r);
         tmem_ld_wait();
 #pragma unroll
-        for (int x = 0; x < 32; ++x) sv_[j * 32 + x] = u2f(r[x]);
+        for (int x = 0; x < 32; ++x)
+          if (j * 32 + x <= lim) mx = fmaxf(mx, u2f(r[x]));
       }
-      float mx = -INFINITY;
-#pragma unroll
-      for (int x = 0; x < 128; ++x)
-        if (x <= lim) mx = fmaxf(mx, sv_[x]);
-      if (!valid) mx = 0.f;
+      if (!valid) {
+        mx = 0.f;
+        lim = -1;                             // every weight of the row is zero
+      }
       const float mneg = -mx * scale_log2;
-      float l = 0.f;
+      float lsum[4] = {0.f, 0.f, 0.f, 0.f};
+      uint8_t* sp = base + kOffQP + qb * 32768;
+#pragma unroll 1
+      for (int j = 0; j < 4; ++j) {
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(s_addr + j * 32, r);
+        tmem_ld_wait();
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        uint32_t w[4];
+        for (int cc = 0; cc < 4; ++cc) {      // 8 keys per 16-byte chunk
+          uint32_t w[4];
 #pragma unroll
-        for (int x = 0; x < 4; ++x) {
-          const int k0 = j * 8 + 2 * x;
-          float p0 = (valid && k0 <= lim) ? exp2f(fmaf(sv_[k0], scale_log2, mneg)) : 0.f;
-          float p1 = (valid && k0 + 1 <= lim) ? exp2f(fmaf(sv_[k0 + 1], scale_log2, mneg)) : 0.f;
-          const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
-          l += __low2float(h2) + __high2float(h2);
-          w[x] = *reinterpret_cast<const uint32_t*>(&h2);
+          for (int x = 0; x < 4; ++x) {
+            const int k0 = j * 32 + cc * 8 + 2 * x;
+            // branch-free: exponentiate every key, then zero the ones past lim
+            float p0 = ex2_approx(fmaf(u2f(r[cc * 8 + 2 * x]), scale_log2, mneg));
+            float p1 = ex2_approx(fmaf(u2f(r[cc * 8 + 2 * x + 1]), scale_log2, mneg));
+            p0 = (k0 <= lim) ? p0 : 0.f;
+            p1 = (k0 + 1 <= lim) ? p1 : 0.f;
+            const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+            lsum[x] += __low2float(h2) + __high2float(h2);
+            w[x] = *reinterpret_cast<const uint32_t*>(&h2);
+          }
+          const int chunk16 = j * 4 + cc;     // 0..15
+          uint8_t* dst = sp + (chunk16 >> 3) * 16384 + row * 128 +
+                         ((((chunk16 & 7) ^ (row & 7))) << 4);
+          *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
         }
-        uint8_t* dst = sq + (j >> 3) * 16384 + row * 128 + ((((j & 7) ^ (row & 7))) << 4);
-        *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
       }
+      const float l = (lsum[0] + lsum[1]) + (lsum[2] + lsum[3]);
+      ml_s[sb * 128 + row] = make_float2(mx * a.scale, l);
       fence_proxy_async_smem();
       tc_fence_before();
-      __syncthreads();
-
-      // O = P V
-      if (tid == 0) {
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t aoff = (kk >> 2) * 16384 + (kk & 3) * 32;
-          umma_bf16(tmem + 128, smem_desc_sw128(sq_a + aoff, 16, 1024),
-                    smem_desc_sw128(sv_a + kk * 2048, 16384, 1024), kIdescPV, kk > 0 ? 1u : 0u);
-        }
-        umma_commit(mma_done);
-      }
-      mbar_wait(mma_done, mma_phase, abort_flag, err);
-      mma_phase ^= 1;
+      mbar_arrive(bar + BAR_P_FULL + qb);
+    }
+  } else {
+    // ---------------- epilogue: O -> pieces ----------------
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    for (int64_t n = 0;; ++n) {
+      if (!Wuse(BAR_D_FULL, kDescRing, n)) break;
+      const ChunkDesc& d = desc[n % kDescRing];
+      if (d.cnt < 0) break;
+      const int ob = (int)(n & 1);
+      const int e = d.ent[row / R];
+      const int32_t b = d.b, g = d.g, c = d.c;
+      if (!Wuse(BAR_O_FULL, 2, n)) break;
+      if (!Wuse(BAR_P_FULL, kQRing, n)) break;   // acquire the softmax's (m, l)
       tc_fence_after();
-
-      // write the piece
+      const int hr = row % R;
+      const int64_t qi = (int64_t)(e >> 4);
+      const bool valid = (e >= 0) && (qi < a.n_q) && (a.q_pos0 + qi >= (int64_t)c * kBlock);
       const int64_t pidx =
-          valid ? ((((int64_t)b * n_q + qi) * H + (g * R + hr)) * kTopK + slot) : 0;
-      if (valid) {
-        *reinterpret_cast<float2*>(part_ml + pidx * 2) = make_float2(mx * scale, l);
-      }
-#pragma unroll
+          valid ? (((int64_t)b * a.n_q + qi) * a.H + (g * R + hr)) * kTopK + (e & 15) : 0;
+      if (valid) *reinterpret_cast<float2*>(a.part_ml + pidx * 2) = ml_s[ob * 128 + row];
+      float* dst = a.part_acc + pidx * kHeadDim;
+#pragma unroll 1
       for (int j = 0; j < 4; ++j) {
         uint32_t r[32];
-        tmem_ld_32x32b_x32(tmem + lane_base + 128 + j * 32, r);
+        tmem_ld_32x32b_x32(tmem + lane_base + 256 + ob * 128 + j * 32, r);
         tmem_ld_wait();
         if (valid) {
-          float4* dst = reinterpret_cast<float4*>(part_acc + pidx * kHeadDim + j * 32);
 #pragma unroll
-          for (int x = 0; x < 8; ++x)
-            dst[x] = make_float4(u2f(r[4 * x]), u2f(r[4 * x + 1]), u2f(r[4 * x + 2]),
-                                 u2f(r[4 * x + 3]));
+          for (int x = 0; x < 4; ++x) st_global_v8(dst + j * 32 + x * 8, r + x * 8);
         }
       }
       tc_fence_before();
+      mbar_arrive(bar + BAR_O_EMPTY + ob);
+      mbar_arrive(bar + BAR_D_EMPTY + (int)(n % kDescRing));
     }
-    kv_phase ^= 1;
-    pos = pend;
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) {
+  if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(tmem, 512);
   }
 }
 
 template <int R>
-static cudaError_t launch_attn_r(const CUtensorMap& tm_k, const CUtensorMap& tm_v, const void* q,
-                                 int64_t qs_b, int64_t qs_t, int64_t qs_h,
-                                 const int32_t* blk_offsets, const int32_t* entries,
-                                 int64_t n_seg, int64_t n_entries, int64_t n_q, int64_t q_pos0,
-                                 int32_t G, int32_t H, int32_t nblk, float scale, float* part_ml,
-                                 float* part_acc, int32_t* err, cudaStream_t st) {
-  constexpr int W = (128 / R) * kAttnChunksPerItem;
+static cudaError_t launch_attn_r(const CUtensorMap& tm_k, const CUtensorMap& tm_v, AttnArgs a,
+                                 cudaStream_t st) {
+  constexpr int CH = 128 / R;
   auto k = sparse_attn_fwd_kernel<R>;
   cudaError_t e =
       cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kAttnSmemBytes);
   if (e != cudaSuccess) return e;
-  const int64_t items = (n_entries + W - 1) / W;
-  if (items == 0) return cudaSuccess;
-  k<<<(unsigned)items, kAttnThreads, kAttnSmemBytes, st>>>(
-      tm_k, tm_v, reinterpret_cast<const __nv_bfloat16*>(q), qs_b, qs_t, qs_h, blk_offsets,
-      entries, n_seg, n_entries, n_q, q_pos0, G, H, nblk, scale, part_ml, part_acc, err);
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  // items of W consecutive entries: at most 8 tiles each, and enough items
+  // (about 8 per SM) to keep every SM busy on small problems
+  const int64_t target_items = (int64_t)sms * 8;
+  int64_t W = (a.n_entries + target_items - 1) / target_items;
+  W = max64(1, min64(W, (int64_t)CH * kAttnMaxChunksPerItem));
+  a.W = W;
+  a.n_items = (a.n_entries + W - 1) / W;
+  if (a.n_items == 0) return cudaSuccess;
+  const int64_t grid = min64(a.n_items, sms);
+  k<<<(unsigned)grid, kAttnThreads, kAttnSmemBytes, st>>>(tm_k, tm_v, a);
   return cudaGetLastError();
 }
 
@@ -273,22 +489,34 @@ cudaError_t launch_sparse_attn(const CUtensorMap& tm_k, const CUtensorMap& tm_v,
                                int64_t n_seg, int64_t n_entries, int64_t n_q, int64_t q_pos0,
                                int32_t G, int32_t H, int32_t nblk, float scale, float* part_ml,
                                float* part_acc, int32_t* err, cudaStream_t st) {
-  const int R = H / G;
-#define MSA_ATTN_CASE(RR)                                                                     \
-  case RR:                                                                                    \
-    return launch_attn_r<RR>(tm_k, tm_v, q, qs_b, qs_t, qs_h, blk_offsets, entries, n_seg,    \
-                             n_entries, n_q, q_pos0, G, H, nblk, scale, part_ml, part_acc, err, \
-                             st);
-  switch (R) {
-    MSA_ATTN_CASE(1)
-    MSA_ATTN_CASE(2)
-    MSA_ATTN_CASE(4)
-    MSA_ATTN_CASE(8)
-    MSA_ATTN_CASE(16)
-    default:
-      return cudaErrorInvalidValue;
+  AttnArgs a;
+  a.q = reinterpret_cast<const __nv_bfloat16*>(q);
+  a.qs_b = qs_b;
+  a.qs_t = qs_t;
+  a.qs_h = qs_h;
+  a.blk_offsets = blk_offsets;
+  a.entries = entries;
+  a.n_seg = n_seg;
+  a.n_entries = n_entries;
+  a.n_items = 0;
+  a.W = 1;
+  a.n_q = n_q;
+  a.q_pos0 = q_pos0;
+  a.G = G;
+  a.H = H;
+  a.nblk = nblk;
+  a.scale = scale;
+  a.part_ml = part_ml;
+  a.part_acc = part_acc;
+  a.err = err;
+  switch (H / G) {
+    case 1: return launch_attn_r<1>(tm_k, tm_v, a, st);
+    case 2: return launch_attn_r<2>(tm_k, tm_v, a, st);
+    case 4: return launch_attn_r<4>(tm_k, tm_v, a, st);
+    case 8: return launch_attn_r<8>(tm_k, tm_v, a, st);
+    case 16: return launch_attn_r<16>(tm_k, tm_v, a, st);
+    default: return cudaErrorInvalidValue;
   }
-#undef MSA_ATTN_CASE
 }
 
 }  // namespace msa

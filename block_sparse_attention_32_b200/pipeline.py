@@ -18,7 +18,7 @@ import torch
 from . import capi
 
 # kernels each step launches (for launch accounting)
-LAUNCHES_PER_STEP = {"index": 1, "topk": 1, "block_lists": 4, "attn": 1, "merge": 1}
+LAUNCHES_PER_STEP = {"index": 1, "topk": 1, "block_lists": 6, "attn": 1, "merge": 1}
 
 
 @dataclasses.dataclass

@@ -55,7 +55,9 @@ def test_block_and_entry_counts(lib):
 def test_workspace_size(lib):
     d = capi.make_dims(2, 300, 1000, 700, 8, 2, 64)
     nblk, ntiles = 8, 3
-    assert capi.msa_block_query_lists_workspace(d) == 4 * 2 * 2 * nblk * (ntiles + 1)
+    nseg = 2 * 2 * nblk
+    nchunks = (nseg + 4095) // 4096
+    assert capi.msa_block_query_lists_workspace(d) == 4 * (nseg * (ntiles + 1) + nchunks)
 
 
 BAD_DIMS = [
