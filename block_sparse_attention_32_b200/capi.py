@@ -22,7 +22,8 @@ TOPK = 16
 HEAD_DIM = 128
 
 STATUS = {0: "MSA_OK", 1: "MSA_ERR_INVALID_ARG", 2: "MSA_ERR_UNSUPPORTED",
-          3: "MSA_ERR_ALIGNMENT", 4: "MSA_ERR_WORKSPACE_TOO_SMALL", 5: "MSA_ERR_CUDA"}
+          3: "MSA_ERR_ALIGNMENT", 4: "MSA_ERR_WORKSPACE_TOO_SMALL", 5: "MSA_ERR_CUDA",
+          6: "MSA_ERR_SCRATCH_LIMIT"}
 DEVERR = {1: "MSA_DEVERR_TIMEOUT", 2: "MSA_DEVERR_BAD_BLOCK", 3: "MSA_DEVERR_BAD_ENTRY"}
 
 
@@ -65,12 +66,13 @@ def load_library(path: str) -> ctypes.CDLL:
     L.msa_block_query_lists_workspace.argtypes = [_PD]
     L.msa_block_query_lists_workspace.restype = ctypes.c_size_t
     L.msa_build_block_query_lists.argtypes = [_PD, _P, _P, _P, _P, ctypes.c_size_t, _P, _P]
+    L.msa_build_block_query_lists_noalloc.argtypes = [_PD, _P, _P, _P, _P, _P]
     L.msa_sparse_attn_fwd.argtypes = [_PD, Tensor, Tensor, Tensor, _P, _P, _P, _P, _P, _P]
     L.msa_merge_partials.argtypes = [_PD, _P, _P, _P, _P, _P, _P, _P]
     L.msa_status_string.argtypes = [ctypes.c_int]
     L.msa_status_string.restype = ctypes.c_char_p
     for f in (L.msa_index_score_maxpool, L.msa_topk_blocks, L.msa_build_block_query_lists,
-              L.msa_sparse_attn_fwd, L.msa_merge_partials):
+              L.msa_build_block_query_lists_noalloc, L.msa_sparse_attn_fwd, L.msa_merge_partials):
         f.restype = ctypes.c_int
     return L
 
@@ -145,6 +147,14 @@ def msa_build_block_query_lists(d: Dims, sel, blk_offsets, entries, ws, dev_err=
            lib().msa_build_block_query_lists(ctypes.byref(d), _ptr(sel), _ptr(blk_offsets),
                                              _ptr(entries), _ptr(ws), nbytes, _ptr(dev_err),
                                              _stream()))
+
+
+def msa_build_block_query_lists_noalloc(d: Dims, sel, blk_offsets, entries, dev_err=None):
+    """Same lists as msa_build_block_query_lists, with the library's built-in
+    device scratch instead of a caller workspace (nothing is allocated)."""
+    _check("msa_build_block_query_lists_noalloc",
+           lib().msa_build_block_query_lists_noalloc(ctypes.byref(d), _ptr(sel), _ptr(blk_offsets),
+                                                     _ptr(entries), _ptr(dev_err), _stream()))
 
 
 def msa_sparse_attn_fwd(d: Dims, q, k, v, blk_offsets, entries, part_ml, part_acc, dev_err=None):

@@ -1,0 +1,71 @@
+// Allocation-free variant of msa_build_block_query_lists.
+//
+// Some callers cannot call cudaMalloc (or any allocating routine) at the point
+// where they build the block->query lists: a plugin running inside a serving
+// process whose host owns all device memory through its own pool, or a
+// latency-critical loop that must not allocate.  For them this entry point
+// takes no workspace: the inversion's scratch lives in a file-scope device
+// array of fixed size that every GPU loading the library keeps until the
+// process exits.  The arithmetic is exactly that of the workspace version (the
+// same kernels are launched, only the scratch pointer differs).
+#include <mutex>
+
+#include "common.cuh"
+
+namespace msa {
+size_t block_lists_workspace(int64_t bgcount, int64_t n_q, int64_t nblk);
+cudaError_t launch_block_lists(const int32_t* sel, int64_t bgcount, int64_t n_q, int64_t q_pos0,
+                               int64_t nblk, int32_t* offsets, int32_t* entries, int64_t cap,
+                               void* ws, int32_t* err, cudaStream_t st);
+}  // namespace msa
+
+// The scratch.  In host code this name is only a host-side stand-in for the
+// device symbol: its device address must be obtained with
+// cudaGetSymbolAddress on each device before it is handed to a kernel.
+static __device__ __align__(256) unsigned char g_block_lists_scratch[MSA_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mutex;
+void* g_scratch_ptr[kMaxDevices] = {};
+
+// Device address of the scratch on the current device (looked up once per
+// device, with that device current).
+cudaError_t scratch_address(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (g_scratch_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_block_lists_scratch);
+    if (e != cudaSuccess) return e;
+    if (p == nullptr) return cudaErrorInvalidSymbol;
+    g_scratch_ptr[dev] = p;
+  }
+  *out = g_scratch_ptr[dev];
+  return cudaSuccess;
+}
+
+}  // namespace
+
+extern "C" msa_status msa_build_block_query_lists_noalloc(const msa_dims* d, const int32_t* sel,
+                                                          int32_t* blk_offsets, int32_t* entries,
+                                                          int32_t* dev_err, void* stream) {
+  // same argument checks as the workspace version
+  const size_t need = msa_block_query_lists_workspace(d);
+  if (need == 0) return MSA_ERR_INVALID_ARG;            // dims rejected
+  if (sel == nullptr || blk_offsets == nullptr || entries == nullptr) return MSA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(sel) & 15u) != 0) return MSA_ERR_ALIGNMENT;
+  if (need > (size_t)MSA_NOALLOC_SCRATCH_BYTES) return MSA_ERR_SCRATCH_LIMIT;
+  const int64_t total = msa_num_entries(d);
+  if (total >= (int64_t(1) << 31)) return MSA_ERR_UNSUPPORTED;
+  void* ws = nullptr;
+  if (scratch_address(&ws) != cudaSuccess) return MSA_ERR_CUDA;
+  const cudaError_t e = msa::launch_block_lists(
+      sel, d->batch * d->h_kv, d->n_q, d->q_pos0, msa_num_blocks(d), blk_offsets, entries, total,
+      ws, dev_err, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MSA_OK : MSA_ERR_CUDA;
+}

@@ -246,6 +246,7 @@ const char* msa_status_string(msa_status s) {
     case MSA_ERR_ALIGNMENT: return "MSA_ERR_ALIGNMENT";
     case MSA_ERR_WORKSPACE_TOO_SMALL: return "MSA_ERR_WORKSPACE_TOO_SMALL";
     case MSA_ERR_CUDA: return "MSA_ERR_CUDA";
+    case MSA_ERR_SCRATCH_LIMIT: return "MSA_ERR_SCRATCH_LIMIT";
   }
   return "MSA_ERR_UNKNOWN";
 }

@@ -59,7 +59,9 @@ typedef enum {
   MSA_ERR_UNSUPPORTED = 2,        /* valid but not implemented (e.g. d_idx 96) */
   MSA_ERR_ALIGNMENT = 3,          /* pointer or stride not 16-byte aligned */
   MSA_ERR_WORKSPACE_TOO_SMALL = 4,
-  MSA_ERR_CUDA = 5                /* a CUDA runtime/driver call failed */
+  MSA_ERR_CUDA = 5,               /* a CUDA runtime/driver call failed */
+  MSA_ERR_SCRATCH_LIMIT = 6       /* needs more than the built-in scratch of the
+                                     allocation-free entry point */
 } msa_status;
 
 /* device-side error codes written to *dev_err */
@@ -143,6 +145,33 @@ MSA_API msa_status msa_build_block_query_lists(const msa_dims* dims, const int32
                                        int32_t* blk_offsets, int32_t* entries,
                                        void* ws, size_t ws_bytes,
                                        int32_t* dev_err, void* stream);
+
+/* Size of the device scratch array behind msa_build_block_query_lists_noalloc
+ * (32 MiB, held on every GPU that loads the library until the process exits). */
+#define MSA_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+/* Allocation-free variant of msa_build_block_query_lists (the paper has no
+ * counterpart: it is a convenience of this library).  It is meant for callers
+ * that cannot call cudaMalloc or any allocating routine where they build the
+ * lists -- e.g. a plugin inside a serving process whose host owns all device
+ * memory through its own pool, or a latency-critical loop that must not
+ * allocate.  Same arguments and results as msa_build_block_query_lists, minus
+ * the workspace: the scratch is a file-scope device array of
+ * MSA_NOALLOC_SCRATCH_BYTES, and problems needing more
+ * (msa_block_query_lists_workspace(dims) > MSA_NOALLOC_SCRATCH_BYTES) are
+ * rejected with MSA_ERR_SCRATCH_LIMIT before anything is enqueued.  For
+ * example the 32K prefill (8 groups), the 64 x 256K decode and an 8192-query
+ * chunk after a 1M-token cache fit; a 128K-token prefill with 8 groups does not.
+ *   - The first call on a device looks up the array's device address with
+ *     cudaGetSymbolAddress (with that device current); make that first call
+ *     before any stream capture.
+ *   - Nothing is allocated or freed.  Every call shares the one array, which
+ *     keeps the previous call's contents; its contents on entry do not matter
+ *     (every word is written before it is read).  Calls that overlap on the
+ *     GPU (on different streams without ordering) race on the array. */
+MSA_API msa_status msa_build_block_query_lists_noalloc(const msa_dims* dims, const int32_t* sel,
+                                                       int32_t* blk_offsets, int32_t* entries,
+                                                       int32_t* dev_err, void* stream);
 
 /* Step 3b: KV-block-outer sparse attention (first page "第二步：精算": full
  * attention over the selected blocks only; survey page: exact softmax
