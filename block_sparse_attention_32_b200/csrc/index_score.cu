@@ -3,7 +3,7 @@
 //
 // Source: page "MSA 稀疏注意力三国杀", section "MSA 架构：粗筛 + 精算", first
 // step items 1-2 (score every token of a 128-token block, the block's score is
-// its highest token score); sparse-attention survey page, MSA entry (one index
+// its highest token score); page "稀疏注意力速览", section 4, MSA entry (one index
 // query head per GQA group, shared index key head, block max-pool).
 //
 // Two kernels:

@@ -26,13 +26,15 @@ __global__ void __launch_bounds__(256)
   const int64_t b = bq / n_q, qi = bq - b * n_q;
   const int32_t g = h / R;
   const int32_t* srow = sel + ((b * G + g) * n_q + qi) * kTopK;
+  // pieces are [B, n_q, G, 16 slots, R, ...]: slot s of this head is row prow0 + s * R
+  const int64_t prow0 = ((b * n_q + qi) * G + g) * kTopK * R + (h - g * R);
 
   float m = -INFINITY, l = 0.f;
   bool v = false;
   if (lane < kTopK) {
     v = srow[lane] >= 0;
     if (v) {
-      const float2 ml = *reinterpret_cast<const float2*>(part_ml + (r * kTopK + lane) * 2);
+      const float2 ml = *reinterpret_cast<const float2*>(part_ml + (prow0 + lane * R) * 2);
       m = ml.x;
       l = ml.y;
     }
@@ -47,12 +49,12 @@ __global__ void __launch_bounds__(256)
   for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
 
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  const float* pa = part_acc + r * kTopK * kHeadDim + 4 * lane;
+  const float* pa = part_acc + prow0 * kHeadDim + 4 * lane;
 #pragma unroll
   for (int s = 0; s < kTopK; ++s) {
     const float ws = __shfl_sync(0xffffffffu, w, s);
     if ((vmask >> s) & 1u) {
-      const float4 a = *reinterpret_cast<const float4*>(pa + s * kHeadDim);
+      const float4 a = *reinterpret_cast<const float4*>(pa + (int64_t)s * R * kHeadDim);
       acc.x = fmaf(ws, a.x, acc.x);
       acc.y = fmaf(ws, a.y, acc.y);
       acc.z = fmaf(ws, a.z, acc.z);

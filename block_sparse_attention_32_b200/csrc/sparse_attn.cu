@@ -9,8 +9,8 @@
 // branch: full attention over the selected blocks only) and section "Kernel
 // 创新：Outer Gather Q" (the KV block is the outer loop, all queries that chose
 // it are computed together so the block is read once); sparse-attention
-// survey page, MSA entry (exact softmax attention); chenxutan page, standard
-// attention softmax(Q K^T / sqrt(d_k)) V.
+// "稀疏注意力速览" page, section 4, MSA entry (exact softmax attention); page
+// "稀疏注意力架构革命", section 1.1 (standard attention softmax(Q K^T / sqrt(d_k)) V).
 //
 // A 128-row tile ("chunk") holds 128 / R query entries x R heads of one group
 // (R = h_q / h_kv).  Work items are runs of W consecutive entries; an item
@@ -25,19 +25,22 @@
 //   warp 2      TMA producer: K and V of each piece; K of the next piece is
 //                             loaded as soon as the last S MMA of the current
 //                             one is done, V as soon as its last P V is done
-//   warps 3-6   gather:       cp.async of the chunk's Q rows into a 4-deep ring
+//   warps 3-6   gather:       cp.async of the chunk's Q rows into a 2-deep ring
 //   warps 7-10  softmax:      S -> (m, l), P = bf16(e^{s-m}) into the Q buffer
-//   warps 11-14 epilogue:     O -> the (m, l, acc) pieces in global memory
-// Shared memory: K 32 KB, V 32 KB, 4 x 32 KB Q/P (128B-swizzled K-major
-// tiles; V is read N-major for P V).  TMEM: S in columns [0,256), O in
-// [256,512), two buffers of 128 columns each.
+//   warps 11-14 epilogue:     O -> shared staging (one 512-byte row per
+//                             thread) -> one bulk async copy per row into the
+//                             (m, l, acc) pieces in global memory
+// Shared memory: K 32 KB, V 32 KB, 2 x 32 KB Q/P (128B-swizzled K-major
+// tiles; V is read N-major for P V), 66 KB output staging (rows padded to
+// 528 bytes so a warp's row-per-thread writes spread over all banks).  TMEM:
+// S in columns [0,256), O in [256,512), two buffers of 128 columns each.
 #include "common.cuh"
 
 namespace msa {
 
 constexpr int kAttnThreads = 480;
 constexpr int kAttnMaxChunksPerItem = 8;
-constexpr int kQRing = 4;              // Q/P tiles in flight
+constexpr int kQRing = 2;              // Q/P tiles in flight
 constexpr int kDescRing = 8;           // chunk descriptors in flight
 
 struct alignas(16) ChunkDesc {
@@ -49,7 +52,9 @@ struct alignas(16) ChunkDesc {
 constexpr int kOffK = 0;               // 32768: [K lo | K hi]
 constexpr int kOffV = 32768;           // 32768: [V lo | V hi]
 constexpr int kOffQP = 65536;          // kQRing x 32768: Q tile, then P
-constexpr int kOffML = kOffQP + kQRing * 32768;          // 2 x 128 float2: (m, l) per row
+constexpr int kStageRow = 528;                           // staged output row (512 B + pad)
+constexpr int kOffStage = kOffQP + kQRing * 32768;       // 128 staged rows
+constexpr int kOffML = kOffStage + 128 * kStageRow;      // 2 x 128 float2: (m, l) per row
 constexpr int kOffDesc = kOffML + 2048;                  // kDescRing descriptors
 constexpr int kOffBar = kOffDesc + kDescRing * (int)sizeof(ChunkDesc);
 constexpr int kNumBars = 4 + 3 * kQRing + 6 + 2 * kDescRing;
@@ -62,13 +67,6 @@ enum {
   BAR_S_FULL = 4 + 3 * kQRing, BAR_O_FULL = BAR_S_FULL + 2, BAR_O_EMPTY = BAR_S_FULL + 4,
   BAR_D_FULL = BAR_S_FULL + 6, BAR_D_EMPTY = BAR_D_FULL + kDescRing
 };
-
-__device__ __forceinline__ void st_global_v8(float* p, const uint32_t* r) {
-  asm volatile("st.global.v8.f32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p),
-               "f"(u2f(r[0])), "f"(u2f(r[1])), "f"(u2f(r[2])), "f"(u2f(r[3])), "f"(u2f(r[4])),
-               "f"(u2f(r[5])), "f"(u2f(r[6])), "f"(u2f(r[7]))
-               : "memory");
-}
 
 struct AttnArgs {
   const __nv_bfloat16* q;
@@ -320,7 +318,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const int32_t b = d.b, g = d.g;
       if (!Wfree(BAR_QP_EMPTY, kQRing, n)) break;
       uint8_t* sq = base + kOffQP + qb * 32768;
-      const __nv_bfloat16* qbase = a.q + (int64_t)b * a.qs_b + (int64_t)(g * R) * a.qs_h + ch * 8;
+      const __nv_bfloat16* qbase =
+          a.q + (int64_t)b * a.qs_b + (int64_t)(g * R) * a.qs_h + ch * 8;
 #pragma unroll 4
       for (int it = 0; it < 16; ++it) {
         const int row = it * 8 + (gt >> 4);
@@ -431,24 +430,32 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const int hr = row % R;
       const int64_t qi = (int64_t)(e >> 4);
       const bool valid = (e >= 0) && (qi < a.n_q) && (a.q_pos0 + qi >= (int64_t)c * kBlock);
+      // piece row of (b, qi, g, slot, hr): the R head rows of one entry are adjacent
       const int64_t pidx =
-          valid ? (((int64_t)b * a.n_q + qi) * a.H + (g * R + hr)) * kTopK + (e & 15) : 0;
+          valid ? ((((int64_t)b * a.n_q + qi) * a.G + g) * kTopK + (e & 15)) * R + hr : 0;
       if (valid) *reinterpret_cast<float2*>(a.part_ml + pidx * 2) = ml_s[ob * 128 + row];
-      float* dst = a.part_acc + pidx * kHeadDim;
+      uint8_t* srow = base + kOffStage + row * kStageRow;
+      bulk_wait_read();                         // the previous row copy has left the staging
 #pragma unroll 1
       for (int j = 0; j < 4; ++j) {
         uint32_t r[32];
         tmem_ld_32x32b_x32(tmem + lane_base + 256 + ob * 128 + j * 32, r);
         tmem_ld_wait();
-        if (valid) {
 #pragma unroll
-          for (int x = 0; x < 4; ++x) st_global_v8(dst + j * 32 + x * 8, r + x * 8);
-        }
+        for (int x = 0; x < 8; ++x)
+          *reinterpret_cast<uint4*>(srow + j * 128 + x * 16) =
+              make_uint4(r[4 * x], r[4 * x + 1], r[4 * x + 2], r[4 * x + 3]);
       }
       tc_fence_before();
       mbar_arrive(bar + BAR_O_EMPTY + ob);
+      if (valid) {
+        fence_proxy_async_smem();
+        bulk_store_s2g(a.part_acc + pidx * kHeadDim, srow, kHeadDim * 4);
+        bulk_commit();
+      }
       mbar_arrive(bar + BAR_D_EMPTY + (int)(n % kDescRing));
     }
+    bulk_wait_all();
   }
 
   tc_fence_before();

@@ -4,15 +4,22 @@
 //
 // Source: page "MSA 稀疏注意力三国杀", section "MSA 架构：粗筛 + 精算", first
 // step item 3 (16 blocks, the current position's block always taken, the rest
-// by score); sparse-attention survey page, MSA entry (per-group top-k with the
+// by score); page "稀疏注意力速览", section 4, MSA entry (per-group top-k with the
 // local block kept).  The tie rule is the stated reading where the pages are
 // silent.
 //
-// One warp per row.  The 15th-best score is found by an exact radix select on
-// order-preserving 32-bit keys (4 passes of 8 bits, warp-aggregated shared
-// histograms); candidates strictly above it are taken, and among those equal
-// to it the lowest block indices fill the remaining places.  The row is read
-// from global memory once per pass (L1-resident after the first).
+// One warp per row; keys are (score, block) pairs ordered by score, then lower
+// block first (a 64-bit key: order-preserving score bits over the complemented
+// block index).  The row is scanned in chunks of 32 x 32 candidates:
+//   1. every lane takes the maximum of its 32 scores; the 15th largest lane
+//      maximum is a lower bound for the 15th-best score (15 distinct
+//      candidates reach it), and so is the current 15th-best of the row;
+//   2. the candidates at or above the larger of the two bounds (usually a few
+//      dozen) join the current best 15 in a 64-slot shared buffer, which a
+//      warp bitonic network sorts; its first 15 entries are the new best 15.
+// If more than 64 keys pass the bound (many equal scores), the row falls back
+// to an exact radix select over the whole row (4 passes of 8 bits with
+// warp-aggregated shared histograms).  Both give the same set.
 #include "common.cuh"
 
 namespace msa {
@@ -26,12 +33,130 @@ __device__ __forceinline__ uint32_t order_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// exact radix select over a row of n candidates: the 15 best in ascending
+// block order into out[0..14]
+__device__ __noinline__ void select_row_radix(const float* __restrict__ row, int n, int32_t* out,
+                                              uint32_t* hist, int lane) {
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  uint32_t prefix = 0, mask = 0;
+  int k = kTopK - 1;
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int i = lane; i < 256; i += 32) hist[i] = 0;
+    __syncwarp();
+    for (int i0 = 0; i0 < n; i0 += 32) {
+      const int i = i0 + lane;
+      bool act = false;
+      uint32_t bin = 0;
+      if (i < n) {
+        const uint32_t u = order_key(row[i]);
+        act = (u & mask) == prefix;
+        bin = (u >> shift) & 255u;
+      }
+      const uint32_t am = __ballot_sync(0xffffffffu, act);
+      if (act) {
+        const uint32_t peers = __match_any_sync(am, bin);
+        if ((peers & lt_mask) == 0) atomicAdd(&hist[bin], __popc(peers));
+      }
+    }
+    __syncwarp();
+    uint32_t mine = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) mine += hist[8 * lane + j];
+    uint32_t incl = mine;   // inclusive suffix sum over lanes
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t v = __shfl_down_sync(0xffffffffu, incl, o);
+      if (lane + o < 32) incl += v;
+    }
+    int digit = -1;
+    uint32_t cum_at = 0, cum = incl - mine;
+#pragma unroll
+    for (int j = 7; j >= 0; --j) {
+      const uint32_t h = hist[8 * lane + j];
+      if (digit < 0 && cum < (uint32_t)k && cum + h >= (uint32_t)k) {
+        digit = 8 * lane + j;
+        cum_at = cum;
+      }
+      cum += h;
+    }
+    const int src = __ffs(__ballot_sync(0xffffffffu, digit >= 0)) - 1;
+    digit = __shfl_sync(0xffffffffu, digit, src);
+    cum_at = __shfl_sync(0xffffffffu, cum_at, src);
+    prefix |= (uint32_t)digit << shift;
+    mask |= 255u << shift;
+    k -= (int)cum_at;
+    __syncwarp();
+  }
+  const uint32_t T = prefix;   // the 15th-best score key; k keys equal to T are taken
+  int written = 0, ties = 0;
+  for (int i0 = 0; i0 < n; i0 += 32) {
+    const int i = i0 + lane;
+    const uint32_t u = (i < n) ? order_key(row[i]) : 0u;
+    const bool eq = (i < n) && (u == T);
+    const uint32_t eqm = __ballot_sync(0xffffffffu, eq);
+    const int tie_rank = ties + __popc(eqm & lt_mask);
+    ties += __popc(eqm);
+    const bool take = (i < n) && (u > T || (eq && tie_rank < k));
+    const uint32_t tm = __ballot_sync(0xffffffffu, take);
+    if (take) out[written + __popc(tm & lt_mask)] = i;
+    written += __popc(tm);
+  }
+}
+
+__device__ __forceinline__ uint64_t shfl_xor_u64(uint64_t v, int m) {
+  const uint32_t lo = __shfl_xor_sync(0xffffffffu, (uint32_t)v, m);
+  const uint32_t hi = __shfl_xor_sync(0xffffffffu, (uint32_t)(v >> 32), m);
+  return ((uint64_t)hi << 32) | lo;
+}
+
+// Sorts the 64 keys held as (a: position lane, b: position lane + 32)
+// descending with a bitonic network.
+__device__ __forceinline__ void bitonic64_desc(uint64_t& a, uint64_t& b, int lane) {
+#pragma unroll
+  for (int k = 2; k <= 64; k <<= 1) {
+#pragma unroll
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      if (j == 32) {                        // partners within the lane
+        const bool desc = true;             // only in the last stage (k = 64)
+        const uint64_t hi = a > b ? a : b, lo = a > b ? b : a;
+        a = desc ? hi : lo;
+        b = desc ? lo : hi;
+      } else {
+        const uint64_t oa = shfl_xor_u64(a, j), ob = shfl_xor_u64(b, j);
+        const bool lower = (lane & j) == 0;
+        const bool desc_a = (lane & k) == 0;          // position lane
+        const bool desc_b = ((lane + 32) & k) == 0;   // position lane + 32
+        a = (lower == desc_a) ? (a > oa ? a : oa) : (a < oa ? a : oa);
+        b = (lower == desc_b) ? (b > ob ? b : ob) : (b < ob ? b : ob);
+      }
+    }
+  }
+}
+
+// Sorts one 32-bit value per lane ascending over lanes 0..15 (lanes 16..31
+// take part with values that sort after).
+__device__ __forceinline__ int32_t bitonic16_asc(int32_t v, int lane) {
+#pragma unroll
+  for (int k = 2; k <= 16; k <<= 1) {
+#pragma unroll
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      const int32_t o = __shfl_xor_sync(0xffffffffu, v, j);
+      const bool lower = (lane & j) == 0;
+      const bool asc = (lane & k) == 0;
+      v = (lower == asc) ? min(v, o) : max(v, o);
+    }
+  }
+  return v;
+}
+
 __global__ void __launch_bounds__(kTopkWarps * 32)
     topk_blocks_kernel(const float* __restrict__ pooled, int64_t stride, int64_t n_rows,
                        int64_t n_q, int64_t q_pos0, int32_t* __restrict__ sel) {
   __shared__ uint32_t hist_all[kTopkWarps][256];
+  __shared__ uint64_t cand_all[kTopkWarps][64];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   uint32_t* hist = hist_all[warp];
+  uint64_t* cand = cand_all[warp];
   const uint32_t lt_mask = (1u << lane) - 1u;
 
   for (int64_t r = (int64_t)blockIdx.x * kTopkWarps + warp; r < n_rows;
@@ -46,79 +171,65 @@ __global__ void __launch_bounds__(kTopkWarps * 32)
     const float* row = pooled + r * stride;
     const int n = (int)own;
 
-    // radix select: threshold key T and how many keys equal to T to take
-    uint32_t prefix = 0, mask = 0;
-    int k = kTopK - 1;
-    for (int shift = 24; shift >= 0; shift -= 8) {
-      for (int i = lane; i < 256; i += 32) hist[i] = 0;
-      __syncwarp();
-      for (int i0 = 0; i0 < n; i0 += 32) {
-        const int i = i0 + lane;
-        bool act = false;
-        uint32_t bin = 0;
-        if (i < n) {
-          const uint32_t u = order_key(row[i]);
-          act = (u & mask) == prefix;
-          bin = (u >> shift) & 255u;
+    // best 15 so far, descending, in lanes 0..14 (0 = empty)
+    uint64_t best = 0;
+    bool overflow = false;
+    for (int c0 = 0; c0 < n; c0 += 1024) {
+      uint32_t u[32];
+      uint32_t lmax = 0;
+#pragma unroll
+      for (int s = 0; s < 32; ++s) {
+        const int i = c0 + s * 32 + lane;
+        u[s] = (i < n) ? order_key(__ldg(row + i)) : 0u;
+        lmax = max(lmax, u[s]);
+      }
+      // 15th largest lane maximum: sort the 32 maxima descending (score bits)
+      int32_t sm = (int32_t)(lmax ^ 0x80000000u);   // signed order = unsigned order
+#pragma unroll
+      for (int k = 2; k <= 32; k <<= 1) {
+#pragma unroll
+        for (int j = k >> 1; j > 0; j >>= 1) {
+          const int32_t o = __shfl_xor_sync(0xffffffffu, sm, j);
+          const bool lower = (lane & j) == 0;
+          const bool desc = (lane & k) == 0;
+          sm = (lower == desc) ? max(sm, o) : min(sm, o);
         }
-        const uint32_t am = __ballot_sync(0xffffffffu, act);
-        if (act) {
-          const uint32_t peers = __match_any_sync(am, bin);
-          if ((peers & lt_mask) == 0) atomicAdd(&hist[bin], __popc(peers));
-        }
+      }
+      const uint32_t t_chunk = (uint32_t)__shfl_sync(0xffffffffu, sm, 14) ^ 0x80000000u;
+      const uint32_t t_best = (uint32_t)(__shfl_sync(0xffffffffu, best, 14) >> 32);
+      const uint32_t T = max(t_chunk, t_best);
+      // candidates: score key >= T (ties at T included), plus the current best 15
+      int cnt = 0;
+#pragma unroll
+      for (int s = 0; s < 32; ++s) {
+        const int i = c0 + s * 32 + lane;
+        const bool take = (i < n) && (u[s] >= T);
+        const uint32_t m = __ballot_sync(0xffffffffu, take);
+        if (take && cnt + __popc(m & lt_mask) < 64 - (kTopK - 1))
+          cand[cnt + __popc(m & lt_mask)] =
+              ((uint64_t)u[s] << 32) | (uint32_t)(0xFFFFFFFFu - (uint32_t)i);
+        cnt += __popc(m);
+      }
+      if (cnt > 64 - (kTopK - 1)) {
+        overflow = true;
+        break;
       }
       __syncwarp();
-      // lane l owns bins 8l .. 8l+7; count of keys in higher lanes' bins
-      uint32_t mine = 0;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) mine += hist[8 * lane + j];
-      uint32_t above = 0;   // sum over lanes > lane
-      {
-        uint32_t incl = mine;   // inclusive suffix sum
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const uint32_t v = __shfl_down_sync(0xffffffffu, incl, o);
-          if (lane + o < 32) incl += v;
-        }
-        above = incl - mine;
-      }
-      int digit = -1;
-      uint32_t cum_at = 0;
-      uint32_t cum = above;
-#pragma unroll
-      for (int j = 7; j >= 0; --j) {
-        const uint32_t h = hist[8 * lane + j];
-        if (digit < 0 && cum < (uint32_t)k && cum + h >= (uint32_t)k) {
-          digit = 8 * lane + j;
-          cum_at = cum;
-        }
-        cum += h;
-      }
-      const uint32_t found = __ballot_sync(0xffffffffu, digit >= 0);
-      const int src = __ffs(found) - 1;
-      digit = __shfl_sync(0xffffffffu, digit, src);
-      cum_at = __shfl_sync(0xffffffffu, cum_at, src);
-      prefix |= (uint32_t)digit << shift;
-      mask |= 255u << shift;
-      k -= (int)cum_at;
+      if (lane < kTopK - 1) cand[cnt + lane] = best;
+      __syncwarp();
+      const int tot = cnt + kTopK - 1;
+      uint64_t a = (lane < tot) ? cand[lane] : 0, b = (lane + 32 < tot) ? cand[lane + 32] : 0;
+      bitonic64_desc(a, b, lane);
+      best = (lane < kTopK - 1) ? a : 0;
       __syncwarp();
     }
-    const uint32_t T = prefix;   // the 15th-best key; k keys equal to T are taken
-
-    // emit selected candidates in ascending index order, then the own block
-    int written = 0, ties = 0;
-    for (int i0 = 0; i0 < n; i0 += 32) {
-      const int i = i0 + lane;
-      uint32_t u = 0;
-      if (i < n) u = order_key(row[i]);
-      const bool eq = (i < n) && (u == T);
-      const uint32_t eqm = __ballot_sync(0xffffffffu, eq);
-      const int tie_rank = ties + __popc(eqm & lt_mask);
-      ties += __popc(eqm);
-      const bool take = (i < n) && (u > T || (eq && tie_rank < k));
-      const uint32_t tm = __ballot_sync(0xffffffffu, take);
-      if (take) out[written + __popc(tm & lt_mask)] = i;
-      written += __popc(tm);
+    if (overflow) {
+      select_row_radix(row, n, out, hist, lane);
+    } else {
+      // the 15 block ids ascending, then the own block
+      int32_t id = (lane < kTopK - 1) ? (int32_t)(0xFFFFFFFFu - (uint32_t)best) : 0x7FFFFFFF;
+      id = bitonic16_asc(id, lane);
+      if (lane < kTopK - 1) out[lane] = id;
     }
     if (lane == 0) out[kTopK - 1] = n;
     __syncwarp();

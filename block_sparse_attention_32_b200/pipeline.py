@@ -52,9 +52,10 @@ class Buffers:
             blk_offsets=torch.empty((B * G * nblk + 1,), dtype=torch.int32, device=dev),
             entries=torch.empty((max(n_ent, 1),), dtype=torch.int32, device=dev),
             ws=torch.empty(((ws_bytes + 15) // 16 * 4,), dtype=torch.int32, device=dev),
-            part_ml=torch.empty((B, n_q, H, capi.TOPK, 2), dtype=torch.float32, device=dev),
-            part_acc=torch.empty((B, n_q, H, capi.TOPK, capi.HEAD_DIM), dtype=torch.float32,
-                                 device=dev),
+            part_ml=torch.empty((B, n_q, G, capi.TOPK, H // G, 2), dtype=torch.float32,
+                                device=dev),
+            part_acc=torch.empty((B, n_q, G, capi.TOPK, H // G, capi.HEAD_DIM),
+                                 dtype=torch.float32, device=dev),
             out=torch.empty((B, n_q, H, capi.HEAD_DIM), dtype=torch.bfloat16, device=dev),
             lse=torch.empty((B, n_q, H), dtype=torch.float32, device=dev),
             dev_err=torch.zeros((4,), dtype=torch.int32, device=dev),

@@ -3,7 +3,8 @@
  * (sm_100a).
  *
  * The method (page "MSA 稀疏注意力三国杀：NSA / DSA / MoBA / MSA 四方案深度对比",
- * section "MSA 架构：粗筛 + 精算"; sparse-attention survey page, entry
+ * section "MSA 架构：粗筛 + 精算"; page "稀疏注意力速览（Sparse Attention，
+ * 2019 ~ 2026）", section 4, entry
  * "MiniMax Sparse Attention (MSA)"):
  *   1. an index branch scores every causal (query, key token) pair with one
  *      index query head per GQA group and a shared index key head;
@@ -101,7 +102,7 @@ MSA_API int64_t msa_num_entries(const msa_dims* dims);
 
 /* Step 1+2a: index scores and causal block max-pool
  * (first page, "第一步：粗筛" items 1-2: score each token, a block's score is
- * its highest token score; survey page MSA entry: one index query head per
+ * its highest token score; "稀疏注意力速览" page, MSA entry: one index query head per
  * GQA group, shared index key head, block max-pool).
  *   q_idx  [B, n_q, G, d_idx]            bf16
  *   k_idx  [B, h_kidx, n_kv, d_idx]      bf16 (s_head = stride between index key heads)
@@ -116,7 +117,7 @@ MSA_API msa_status msa_index_score_maxpool(const msa_dims* dims, msa_tensor q_id
                                    int32_t* dev_err, void* stream);
 
 /* Step 2b: block selection (first page, "第一步：粗筛" item 3: 16 blocks, the
- * current position's block always taken, the rest by score; survey page:
+ * current position's block always taken, the rest by score; "稀疏注意力速览" page:
  * top-k per GQA group with the local block kept).
  *   pooled [B, G, n_q, pooled_row_stride] fp32 as written above
  *   sel    [B, G, n_q, 16] int32: own(t) plus the min(15, own(t)) best blocks
@@ -174,15 +175,17 @@ MSA_API msa_status msa_build_block_query_lists_noalloc(const msa_dims* dims, con
                                                        int32_t* dev_err, void* stream);
 
 /* Step 3b: KV-block-outer sparse attention (first page "第二步：精算": full
- * attention over the selected blocks only; survey page: exact softmax
- * attention; softmax(Q K^T * scale) V from the chenxutan page).  For every
+ * attention over the selected blocks only; "稀疏注意力速览" page: exact softmax
+ * attention; softmax(Q K^T * scale) V from the "稀疏注意力架构革命" page, section 1.1).  For every
  * segment (b, g, c) each K/V block is brought into shared memory once and the
  * R = h_q / h_kv head rows of every listed query are gathered into 128-row
- * tensor-core tiles.  For each (query i, head h in g, slot) it writes the
- * piece over the tokens j of block c with j <= t:
- *   part_ml [B, n_q, h_q, 16, 2] fp32: m = max_j scale * q.k_j,
- *                                      l = sum_j e^{scale q.k_j - m}
- *   part_acc[B, n_q, h_q, 16, 128] fp32: sum_j e^{scale q.k_j - m} v_j
+ * tensor-core tiles.  For each (query i, group g, slot, head r of the group,
+ * i.e. head h = g * R + r) it writes the piece over the tokens j of block c
+ * with j <= t:
+ *   part_ml [B, n_q, G, 16, R, 2] fp32: m = max_j scale * q.k_j,
+ *                                       l = sum_j e^{scale q.k_j - m}
+ *   part_acc[B, n_q, G, 16, R, 128] fp32: sum_j e^{scale q.k_j - m} v_j
+ * (the R head rows of one (query, block) are adjacent, R = h_q / h_kv)
  * (the weights e^{...} are rounded to bf16 before they multiply V and before
  * they are summed into l, so acc / l is an exact convex combination).
  *   q [B, n_q, h_q, 128] bf16; k, v [B, h_kv, n_kv, 128] bf16

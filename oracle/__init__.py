@@ -8,11 +8,12 @@ the CUDA library.
 Each function cites the page passage it follows in ``msa_oracle.c``:
   * ``index_pooled``  -- index-branch token scores + block max-pool
     ("MSA 稀疏注意力三国杀" page, section "MSA 架构：粗筛 + 精算", steps 1-2;
-    sparse-attention survey page, MSA entry);
+    "稀疏注意力速览" page, section 4, MSA entry);
   * ``topk`` / ``topk_f32`` -- 16 blocks per query and group, own block
     forced (same section, step 3; survey MSA entry);
   * ``attention`` -- exact softmax attention over the selected tokens (same
-    section, "第二步：精算"; softmax(QK^T/sqrt(d)) V from the chenxutan page);
+    section, "第二步：精算"; softmax(QK^T/sqrt(d)) V from the "稀疏注意力架构革命"
+    page, section 1.1);
   * ``merge`` -- log-sum-exp combination of per-block softmax pieces (the
     identity the KV-block-outer "Outer Gather Q" scheme relies on);
   * ``block_query_lists`` -- query->block lists inverted into block->query

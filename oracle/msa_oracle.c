@@ -11,11 +11,13 @@
  *       score per token, block score = max over the block, 16 blocks with the
  *       query's own block always taken; main branch: full attention over the
  *       16 x 128 = 2048 selected tokens).
- *  [P3] "sparse-attention" survey, entry "MiniMax Sparse Attention (MSA)"
+ *  [P3] "稀疏注意力速览（Sparse Attention，2019 ~ 2026）", section 4 (block
+ *       级选择派), entry "MiniMax Sparse Attention（MSA）"
  *       (per GQA group one index query head and a shared index key head,
  *       block max-pool, per-group top-k with the local block kept, exact
  *       softmax attention on the selected blocks).
- *  [P5] chenxutan.com article, section on standard self-attention, formula
+ *  [P5] "稀疏注意力架构革命：2026年长上下文大模型核心技术解析", section 1.1
+ *       (标准Transformer Attention的O(n²)困境), formula
  *       softmax(Q K^T / sqrt(d_k)) V.
  *
  * Readings where the pages are silent (each one is listed in the design

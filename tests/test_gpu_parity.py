@@ -166,19 +166,21 @@ def test_merge_kernel_against_oracle_merge():
     d = pipeline.dims_for(w)
     sel = wl.random_selection(w, "cpu")
     g = torch.Generator().manual_seed(5)
-    B, n_q, H = w.batch, w.n_q, w.h_q
-    m = torch.randn((B, n_q, H, 16), generator=g) * 3
-    l = torch.rand((B, n_q, H, 16), generator=g) * 5 + 0.5
-    acc = torch.randn((B, n_q, H, 16, 128), generator=g) * l[..., None]
+    B, n_q, H, G = w.batch, w.n_q, w.h_q, w.h_kv
+    R = H // G
+    # pieces in the ABI layout [B, n_q, G, 16, R, ...]
+    m = torch.randn((B, n_q, G, 16, R), generator=g) * 3
+    l = torch.rand((B, n_q, G, 16, R), generator=g) * 5 + 0.5
+    acc = torch.randn((B, n_q, G, 16, R, 128), generator=g) * l[..., None]
     ml = torch.stack([m, l], dim=-1).contiguous()
     out = torch.empty((B, n_q, H, 128), dtype=torch.bfloat16, device="cuda")
     lse = torch.empty((B, n_q, H), device="cuda")
     capi.msa_merge_partials(d, sel.cuda(), ml.cuda(), acc.contiguous().cuda(), out, lse)
-    R = H // w.h_kv
+    # oracle view: one row per (b, q, head), 16 slots each
+    to_rows = lambda t: t.movedim(4, 3).reshape(B * n_q * H, 16, *t.shape[5:])
     valid = (sel.permute(0, 2, 1, 3)[:, :, torch.arange(H) // R] >= 0).reshape(-1, 16).numpy()
-    o_ref, lse_ref = oracle.merge(valid.astype(np.int32), m.reshape(-1, 16).double().numpy(),
-                                  l.reshape(-1, 16).double().numpy(),
-                                  acc.reshape(-1, 16, 128).double().numpy())
+    o_ref, lse_ref = oracle.merge(valid.astype(np.int32), to_rows(m).double().numpy(),
+                                  to_rows(l).double().numpy(), to_rows(acc).double().numpy())
     o = out.float().reshape(-1, 128).cpu().numpy()
     assert np.abs(o - o_ref).max() <= 1e-2 * max(1.0, np.abs(o_ref).max())
     assert np.abs(lse.reshape(-1).cpu().numpy() - lse_ref).max() <= 1e-4

@@ -4,10 +4,11 @@ itself -- brute force, closed forms, invariants and hand-derived fixtures.
 The statements pinned come from the MSA pages: "MSA 稀疏注意力三国杀"
 (section "MSA 架构：粗筛 + 精算": 128-token blocks, token scores max-pooled
 per block, 16 blocks with the own block always in, attention over the
-selected 2048 tokens; section "试过的强制规则都被砍掉": no forced sink or
-window; section "MSA 性能数据": 28.4x theoretical saving at 1M), the
-sparse-attention survey (MSA entry: per GQA group, shared index key head,
-exact softmax) and the chenxutan page (softmax(QK^T/sqrt(d))V).
+selected 2048 tokens; the appendix section on emergent head patterns: the
+forced sink and window rules were dropped; section "MSA 性能数据": 28.4x
+theoretical saving at 1M), the "稀疏注意力速览" page (section 4, MSA entry:
+per GQA group, shared index key head, exact softmax) and the "稀疏注意力架构革命"
+page (section 1.1: softmax(QK^T/sqrt(d))V).
 """
 import json
 import math
