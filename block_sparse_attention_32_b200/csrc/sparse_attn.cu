@@ -25,22 +25,28 @@
 //   warp 2      TMA producer: K and V of each piece; K of the next piece is
 //                             loaded as soon as the last S MMA of the current
 //                             one is done, V as soon as its last P V is done
-//   warps 3-6   gather:       cp.async of the chunk's Q rows into a 2-deep ring
-//   warps 7-10  softmax:      S -> (m, l), P = bf16(e^{s-m}) into the Q buffer
-//   warps 11-14 epilogue:     O -> shared staging (one 512-byte row per
-//                             thread) -> one bulk async copy per row into the
-//                             (m, l, acc) pieces in global memory
-// Shared memory: K 32 KB, V 32 KB, 2 x 32 KB Q/P (128B-swizzled K-major
-// tiles; V is read N-major for P V), 66 KB output staging (rows padded to
-// 528 bytes so a warp's row-per-thread writes spread over all banks).  TMEM:
-// S in columns [0,256), O in [256,512), two buffers of 128 columns each.
+//   warps 3-6   gather:       cp.async of the chunk's Q rows into a 3-deep ring
+//   warps 7-10  softmax:      S -> (m, l), P = bf16(e^{s-m}) written back into
+//                             the first 64 columns of its S buffer in TMEM
+//                             (the A operand of O = P V)
+//   warps 11-14 epilogue:     O -> the (m, l, acc) pieces in global memory:
+//                             each warp stages its 32 rows half a row (256 B)
+//                             at a time in shared memory and reads them back
+//                             transposed, so that one store instruction
+//                             writes two whole half rows (coalesced)
+// Shared memory: K 32 KB, V 32 KB, 3 x 32 KB Q tiles (128B-swizzled K-major;
+// V is read N-major for P V), 34 KB output staging (half rows padded to 272
+// bytes so a warp's row-per-thread writes spread over all banks).  TMEM: S/P
+// in columns [0,256), O in [256,512), two buffers of 128 columns each; a Q
+// tile is released as soon as its S MMA is done, and S(n+2) waits for
+// O(n) = P(n) V, which reads P(n) from the same columns.
 #include "common.cuh"
 
 namespace msa {
 
 constexpr int kAttnThreads = 480;
 constexpr int kAttnMaxChunksPerItem = 8;
-constexpr int kQRing = 2;              // Q/P tiles in flight
+constexpr int kQRing = 3;              // Q/P tiles in flight
 constexpr int kDescRing = 8;           // chunk descriptors in flight
 
 struct alignas(16) ChunkDesc {
@@ -52,7 +58,7 @@ struct alignas(16) ChunkDesc {
 constexpr int kOffK = 0;               // 32768: [K lo | K hi]
 constexpr int kOffV = 32768;           // 32768: [V lo | V hi]
 constexpr int kOffQP = 65536;          // kQRing x 32768: Q tile, then P
-constexpr int kStageRow = 528;                           // staged output row (512 B + pad)
+constexpr int kStageRow = 272;                           // staged half row (256 B + pad)
 constexpr int kOffStage = kOffQP + kQRing * 32768;       // 128 staged rows
 constexpr int kOffML = kOffStage + 128 * kStageRow;      // 2 x 128 float2: (m, l) per row
 constexpr int kOffDesc = kOffML + 2048;                  // kDescRing descriptors
@@ -218,29 +224,30 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
+    // S(n) and the pending P V(n-1) are issued in whichever order their
+    // inputs become ready (S(n) needs the gathered Q tile, P V(n-1) the
+    // softmax of n-1); S(n+1) always waits for P V(n-1), which frees S buffer.
     if (lane == 0) {
       int64_t pn = -1, pp = 0, v_ready = -1, last_s_piece = -1;
       bool plast = false, ok = true;
-      auto issue_pv = [&](int64_t n, int64_t p, bool last) {
-        const int qb = (int)(n % kQRing), ob = (int)(n & 1);
+      auto pv_ready = [&](int64_t n, int64_t p) {
         if (p != v_ready) {
-          if (!Wuse(BAR_V_FULL, 1, p)) return false;
+          if (!mbar_try_wait(bar + BAR_V_FULL, (uint32_t)(p & 1))) return false;
           v_ready = p;
         }
-        if (!Wuse(BAR_P_FULL, kQRing, n)) return false;
+        return mbar_try_wait(bar + BAR_P_FULL + (int)(n % kQRing),
+                             (uint32_t)((n / kQRing) & 1));
+      };
+      auto issue_pv = [&](int64_t n, bool last) {
+        const int ob = (int)(n & 1);
         tc_fence_after();
-        const uint32_t pa = smem_u32(base + kOffQP + qb * 32768);
         const uint32_t va = smem_u32(base + kOffV);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t aoff = (kk >> 2) * 16384 + (kk & 3) * 32;
-          umma_bf16(tmem + 256 + ob * 128, smem_desc_sw128(pa + aoff, 16, 1024),
-                    smem_desc_sw128(va + kk * 2048, 16384, 1024), kIdescPV, kk > 0 ? 1u : 0u);
-        }
+        for (int kk = 0; kk < 8; ++kk)
+          umma_bf16_ts(tmem + 256 + ob * 128, tmem + ob * 128 + kk * 8,
+                       smem_desc_sw128(va + kk * 2048, 16384, 1024), kIdescPV, kk > 0 ? 1u : 0u);
         umma_commit(bar + BAR_O_FULL + ob);
-        umma_commit(bar + BAR_QP_EMPTY + qb);
         if (last) umma_commit(bar + BAR_V_EMPTY);
-        return true;
       };
       for (int64_t n = 0;; ++n) {
         if (!Wuse(BAR_D_FULL, kDescRing, n)) { ok = false; break; }
@@ -249,37 +256,66 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const int64_t p = d.piece;
         const bool first = d.first != 0, last = d.last != 0;
         const int qb = (int)(n % kQRing), sb = (int)(n & 1);
-        if (first) {
-          // drain the pending P V before waiting for the next block's K
-          if (pn >= 0 && !issue_pv(pn, pp, plast)) { ok = false; break; }
-          pn = -1;
-          if (!Wuse(BAR_K_FULL, 1, p)) { ok = false; break; }
-        }
-        if (!Wuse(BAR_Q_FULL, kQRing, n)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t qa = smem_u32(base + kOffQP + qb * 32768);
-        const uint32_t ka = smem_u32(base + kOffK);
+        bool s_done = false, k_ok = !first, pv_done = pn < 0, o_ok = n < 2;
+        const uint64_t t0 = global_timer_ns();
+        while (!(s_done && pv_done)) {
+          bool progress = false;
+          if (!pv_done && pv_ready(pn, pp)) {
+            issue_pv(pn, plast);
+            pv_done = progress = true;
+          }
+          if (!s_done) {
+            if (!k_ok) k_ok = mbar_try_wait(bar + BAR_K_FULL, (uint32_t)(p & 1));
+            // S buffer sb holds P(n-2) until O(n-2) = P(n-2) V is complete
+            if (!o_ok) o_ok = mbar_try_wait(bar + BAR_O_FULL + sb, (uint32_t)(((n - 2) >> 1) & 1));
+            if (k_ok && o_ok &&
+                mbar_try_wait(bar + BAR_Q_FULL + qb, (uint32_t)((n / kQRing) & 1))) {
+              tc_fence_after();
+              const uint32_t qa = smem_u32(base + kOffQP + qb * 32768);
+              const uint32_t ka = smem_u32(base + kOffK);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          umma_bf16(tmem + sb * 128, smem_desc_sw128(qa + off, 16, 1024),
-                    smem_desc_sw128(ka + off, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
+              for (int kk = 0; kk < 8; ++kk) {
+                const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+                umma_bf16(tmem + sb * 128, smem_desc_sw128(qa + off, 16, 1024),
+                          smem_desc_sw128(ka + off, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
+              }
+              umma_commit(bar + BAR_S_FULL + sb);
+              umma_commit(bar + BAR_QP_EMPTY + qb);
+              if (last) {
+                umma_commit(bar + BAR_K_EMPTY);
+                last_s_piece = p;
+              }
+              s_done = progress = true;
+            }
+          }
+          if (!progress) {
+            if (*abort_flag) { ok = false; break; }
+            if (global_timer_ns() - t0 > kWaitLimitNs) {
+              *abort_flag = 1;
+              report(err, MSA_DEVERR_TIMEOUT);
+              ok = false;
+              break;
+            }
+            __nanosleep(32);
+          }
         }
-        umma_commit(bar + BAR_S_FULL + sb);
-        if (last) {
-          umma_commit(bar + BAR_K_EMPTY);
-          last_s_piece = p;
-        }
-        if (pn >= 0 && !issue_pv(pn, pp, plast)) { ok = false; break; }
+        if (!ok) break;
         pn = n;
         pp = p;
         plast = last;
       }
-      if (ok && pn >= 0 && issue_pv(pn, pp, plast)) {
-        // let the last completions land before the block can exit
-        Wuse(BAR_QP_EMPTY, kQRing, pn);
-        if (plast) Wuse(BAR_V_EMPTY, 1, pp);
-        if (last_s_piece >= 0) Wuse(BAR_K_EMPTY, 1, last_s_piece);
+      if (ok && pn >= 0) {
+        bool ready = false;
+        if (pp != v_ready) ready = Wuse(BAR_V_FULL, 1, pp);
+        else ready = true;
+        if (ready && Wuse(BAR_P_FULL, kQRing, pn)) {
+          issue_pv(pn, plast);
+          // let the last completions land before the block can exit
+          Wuse(BAR_QP_EMPTY, kQRing, pn);
+          Wuse(BAR_O_FULL, 2, pn);
+          if (plast) Wuse(BAR_V_EMPTY, 1, pp);
+          if (last_s_piece >= 0) Wuse(BAR_K_EMPTY, 1, last_s_piece);
+        }
       }
     }
   } else if (warp == 2) {
@@ -348,7 +384,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const int e = d.ent[row / R];
       const int32_t c = d.c;
       if (!Wuse(BAR_S_FULL, 2, n)) break;
-      if (!Wfree(BAR_O_EMPTY, 2, n)) break;
       tc_fence_after();
       const int64_t qi = (int64_t)(e >> 4);
       bool valid = (e >= 0) && (qi < a.n_q);
@@ -379,36 +414,33 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       }
       const float mneg = -mx * scale_log2;
       float lsum[4] = {0.f, 0.f, 0.f, 0.f};
-      uint8_t* sp = base + kOffQP + qb * 32768;
 #pragma unroll 1
       for (int j = 0; j < 4; ++j) {
         uint32_t r[32];
         tmem_ld_32x32b_x32(s_addr + j * 32, r);
         tmem_ld_wait();
+        uint32_t w[16];
 #pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {      // 8 keys per 16-byte chunk
-          uint32_t w[4];
-#pragma unroll
-          for (int x = 0; x < 4; ++x) {
-            const int k0 = j * 32 + cc * 8 + 2 * x;
-            // branch-free: exponentiate every key, then zero the ones past lim
-            float p0 = ex2_approx(fmaf(u2f(r[cc * 8 + 2 * x]), scale_log2, mneg));
-            float p1 = ex2_approx(fmaf(u2f(r[cc * 8 + 2 * x + 1]), scale_log2, mneg));
-            p0 = (k0 <= lim) ? p0 : 0.f;
-            p1 = (k0 + 1 <= lim) ? p1 : 0.f;
-            const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
-            lsum[x] += __low2float(h2) + __high2float(h2);
-            w[x] = *reinterpret_cast<const uint32_t*>(&h2);
-          }
-          const int chunk16 = j * 4 + cc;     // 0..15
-          uint8_t* dst = sp + (chunk16 >> 3) * 16384 + row * 128 +
-                         ((((chunk16 & 7) ^ (row & 7))) << 4);
-          *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+        for (int x = 0; x < 16; ++x) {
+          const int k0 = j * 32 + 2 * x;
+          // branch-free: exponentiate every key, then zero the ones past lim
+          float p0 = ex2_approx(fmaf(u2f(r[2 * x]), scale_log2, mneg));
+          float p1 = ex2_approx(fmaf(u2f(r[2 * x + 1]), scale_log2, mneg));
+          p0 = (k0 <= lim) ? p0 : 0.f;
+          p1 = (k0 + 1 <= lim) ? p1 : 0.f;
+          const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+          lsum[x & 3] += __low2float(h2) + __high2float(h2);
+          w[x] = *reinterpret_cast<const uint32_t*>(&h2);
         }
+        // keys 32j..32j+31 -> columns 16j..16j+15 of this S buffer (already read)
+        tmem_st_32x32b_x16(s_addr + j * 16, w);
       }
+      tmem_st_wait();
       const float l = (lsum[0] + lsum[1]) + (lsum[2] + lsum[3]);
+      // (m, l) slot sb and O buffer sb are free once the epilogue of n-2 is done;
+      // P V(n) is issued only after this arrival
+      if (!Wfree(BAR_O_EMPTY, 2, n)) break;
       ml_s[sb * 128 + row] = make_float2(mx * a.scale, l);
-      fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(bar + BAR_P_FULL + qb);
     }
@@ -435,27 +467,41 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           valid ? ((((int64_t)b * a.n_q + qi) * a.G + g) * kTopK + (e & 15)) * R + hr : 0;
       if (valid) *reinterpret_cast<float2*>(a.part_ml + pidx * 2) = ml_s[ob * 128 + row];
       uint8_t* srow = base + kOffStage + row * kStageRow;
-      bulk_wait_read();                         // the previous row copy has left the staging
+      uint8_t* swarp = base + kOffStage + (quarter * 32) * kStageRow;
+      const uint32_t o_addr = tmem + lane_base + 256 + ob * 128;
+      float* acc = a.part_acc + pidx * kHeadDim;
 #pragma unroll 1
-      for (int j = 0; j < 4; ++j) {
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(tmem + lane_base + 256 + ob * 128 + j * 32, r);
+      for (int half = 0; half < 2; ++half) {
+        uint32_t r0[32], r1[32];
+        tmem_ld_32x32b_x32(o_addr + half * 64, r0);
+        tmem_ld_32x32b_x32(o_addr + half * 64 + 32, r1);
         tmem_ld_wait();
+        if (half == 1) {
+          tc_fence_before();
+          mbar_arrive(bar + BAR_O_EMPTY + ob);
+        }
 #pragma unroll
-        for (int x = 0; x < 8; ++x)
-          *reinterpret_cast<uint4*>(srow + j * 128 + x * 16) =
-              make_uint4(r[4 * x], r[4 * x + 1], r[4 * x + 2], r[4 * x + 3]);
-      }
-      tc_fence_before();
-      mbar_arrive(bar + BAR_O_EMPTY + ob);
-      if (valid) {
-        fence_proxy_async_smem();
-        bulk_store_s2g(a.part_acc + pidx * kHeadDim, srow, kHeadDim * 4);
-        bulk_commit();
+        for (int x = 0; x < 8; ++x) {
+          *reinterpret_cast<uint4*>(srow + x * 16) =
+              make_uint4(r0[4 * x], r0[4 * x + 1], r0[4 * x + 2], r0[4 * x + 3]);
+          *reinterpret_cast<uint4*>(srow + 128 + x * 16) =
+              make_uint4(r1[4 * x], r1[4 * x + 1], r1[4 * x + 2], r1[4 * x + 3]);
+        }
+        __syncwarp();
+        // two half rows per instruction: lanes 0-15 row 2i, lanes 16-31 row 2i+1
+#pragma unroll 4
+        for (int i = 0; i < 16; ++i) {
+          const int rr = 2 * i + (lane >> 4);
+          const float* dst_row = (const float*)__shfl_sync(0xffffffffu, (unsigned long long)acc, rr);
+          const bool rv = __shfl_sync(0xffffffffu, valid ? 1 : 0, rr) != 0;
+          const uint4 v = *reinterpret_cast<const uint4*>(swarp + rr * kStageRow + (lane & 15) * 16);
+          if (rv)
+            *reinterpret_cast<uint4*>(const_cast<float*>(dst_row) + half * 64 + (lane & 15) * 4) = v;
+        }
+        __syncwarp();
       }
       mbar_arrive(bar + BAR_D_EMPTY + (int)(n % kDescRing));
     }
-    bulk_wait_all();
   }
 
   tc_fence_before();
