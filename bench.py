@@ -47,7 +47,7 @@ def load_peaks():
 
 
 def work_counts(w):
-    """Algorithmic FLOPs / bytes of one pass (formulas stated in the design notes)."""
+    """Algorithmic FLOPs and entry count of one pass (formulas stated in the design notes)."""
     B, G, R, d_idx = w.batch, w.h_kv, w.h_q // w.h_kv, w.d_idx
     t = w.q_pos0 + np.arange(w.n_q, dtype=np.int64)
     own = t // 128
@@ -60,6 +60,54 @@ def work_counts(w):
     attn_flops = float(B * w.h_q * 4 * 128 * toks.sum())
     n_entries = int(B * G * nsel_full.sum())
     return idx_flops, attn_flops, n_entries
+
+
+def bytes_model(w, n_entries, n_pieces_nonempty):
+    """Algorithmic DRAM bytes per launch of each kernel (design notes, section 7).
+
+    attention: per (query, block) entry the R gathered Q rows (256 B each) and
+    the R fp32 pieces written (512 B acc + 8 B (m, l)); per selected (batch,
+    group, block) the 64 KB K/V tile once; the entry list.  merge: the pieces
+    read once, sel, and the bf16 output + lse written."""
+    B, G, R = w.batch, w.h_kv, w.h_q // w.h_kv
+    t = w.q_pos0 + np.arange(w.n_q, dtype=np.int64)
+    own = t // 128
+    rows = B * G * w.n_q
+    return {
+        "index": float(B * w.n_q * G * w.d_idx * 2 + B * w.h_kidx * w.n_kv * w.d_idx * 2
+                       + 4 * B * G * own.sum()),
+        "topk": float(4 * B * G * own[own >= 16].sum() + 64 * rows),
+        "block_lists": float(64 * rows * 2 + 4 * n_entries * 2),
+        "attn": float(n_entries * R * (256 + 520) + n_pieces_nonempty * 65536 + 4 * n_entries),
+        "merge": float(n_entries * R * 520 + 64 * rows + B * w.n_q * w.h_q * (256 + 4)),
+    }
+
+
+def source_digest(paths):
+    import hashlib
+    h = hashlib.sha256()
+    for pth in paths:
+        with open(pth, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def measured_traffic(kernel_files, record):
+    """DRAM bytes per launch from a committed ncu summary, or None when the
+    kernel sources changed since the counters were taken."""
+    path = os.path.join(ROOT, "profiles", record)
+    try:
+        kv = dict(line.split(":", 1) for line in open(path) if ":" in line)
+    except OSError:
+        return None
+    digest = source_digest([os.path.join(ROOT, "block_sparse_attention_32_b200", "csrc", f)
+                            for f in kernel_files])
+    if kv.get("source_sha256", "").strip() != digest:
+        return None
+    try:
+        return float(kv["dram_bytes_per_launch"].strip())
+    except (KeyError, ValueError):
+        return None
 
 
 def sample_clocks(stop_file, out_path):
@@ -174,13 +222,15 @@ def bench_workload(w, steps, warmup, world, rank, with_e2e=True):
     if int(buf.dev_err[0]) != 0:
         raise RuntimeError(f"device error {int(buf.dev_err[0])} during timing")
 
+    # (batch, group, block) segments that some query selected: K/V tiles read
+    n_pieces = int((buf.blk_offsets[1:] > buf.blk_offsets[:-1]).sum().item())
     e2e = None
     if with_e2e:
         e2e = bench_e2e(w, buf, inp, max(2, min(steps, 3)), world)
     del inp
     del buf
     torch.cuda.empty_cache()
-    return total_ms, per_stage, per_stage_mean, e2e
+    return total_ms, per_stage, per_stage_mean, e2e, n_pieces
 
 
 def bench_e2e(w, buf, dev_inp, steps, world):
@@ -298,7 +348,8 @@ def main():
     clk_path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{rank}.csv")
     os.makedirs(os.path.dirname(clk_path), exist_ok=True)
     proc = sample_clocks(None, clk_path) if rank == 0 else None
-    total_ms, stage_med, stage_mean, e2e = bench_workload(w, args.steps, args.warmup, world, rank)
+    total_ms, stage_med, stage_mean, e2e, n_pieces = bench_workload(w, args.steps, args.warmup,
+                                                                    world, rank)
     if proc is not None:
         proc.terminate()
         proc.wait()
@@ -311,39 +362,49 @@ def main():
     decode = None
     if not args.no_decode:
         dw = wl.DECODE
-        dms, dstage, _, _ = bench_workload(dw, max(3, args.steps), args.warmup, world, rank,
-                                           with_e2e=False)
+        dms, dstage, _, _, dpieces = bench_workload(dw, max(3, args.steps), args.warmup, world,
+                                                    rank, with_e2e=False)
         dms = max_over_ranks(dms, world) / max(3, args.steps)
         kidx_bytes = dw.batch * dw.n_kv * dw.d_idx * 2
-        sel_kv_bytes = dw.batch * dw.h_kv * 16 * 128 * 128 * 2 * 2
+        sel_kv_bytes = dpieces * 65536
+        read_bytes = kidx_bytes + sel_kv_bytes
         decode = {"workload": dw.name, "tokens_per_s": world * dw.batch / (dms / 1000.0),
                   "ms_per_step": dms, "stages_ms": dstage,
                   "index_scan_gbs": kidx_bytes / (dstage["index"] / 1000.0) / 1e9,
-                  "bytes_read_per_step": kidx_bytes + sel_kv_bytes}
+                  "bytes_read_per_step": read_bytes,
+                  "hbm_frac_on_bytes_read": read_bytes / (dms / 1000.0) / 1e9
+                  / peaks.get("hbm_gbs", FALLBACK["hbm_gbs"])}
 
     if rank != 0:
         if world > 1:
             torch.distributed.destroy_process_group()
         return
 
-    # dominant kernel: the longest stage
+    # dominant kernel: the longest stage; its bound is the larger of its
+    # algorithmic time at the tensor peak and at the HBM peak
     dom = max(stage_mean, key=stage_mean.get)
     sustained = peaks.get("bf16_tflops_sustained", FALLBACK["bf16_tflops_sustained"])
-    if dom in ("index", "attn"):
-        flops = idx_flops if dom == "index" else attn_flops
-        ach = flops / (stage_mean[dom] / 1000.0) / 1e12
+    hbm = peaks.get("hbm_gbs", FALLBACK["hbm_gbs"])
+    nbytes = bytes_model(w, n_ent, n_pieces)
+    flops = {"index": idx_flops, "attn": attn_flops}.get(dom, 0.0)
+    secs = stage_mean[dom] / 1000.0
+    t_tensor = flops / (sustained * 1e12)
+    t_hbm = nbytes[dom] / (hbm * 1e9)
+    if t_tensor >= t_hbm:
+        ach = flops / secs / 1e12
         roof = {"kernel": dom, "bound": "tensor", "achieved": ach, "peak": sustained,
-                "unit": "TFLOP/s", "frac": ach / sustained, "traffic": None,
+                "unit": "TFLOP/s", "frac": ach / sustained,
                 "peak_source": f"{peak_src} bf16_tflops_sustained"}
     else:
-        part_bytes = w.batch * w.n_q * w.h_q * 16 * (128 + 2) * 4
-        byts = {"merge": part_bytes + w.batch * w.n_q * w.h_q * (256 + 4) + n_ent * 4,
-                "topk": w.batch * w.h_kv * (idx_flops / (2 * w.d_idx * 128 * w.batch * w.h_kv)) * 4,
-                "block_lists": n_ent * 4 * 4}[dom]
-        ach = byts / (stage_mean[dom] / 1000.0) / 1e9
-        roof = {"kernel": dom, "bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"],
-                "unit": "GB/s", "frac": ach / peaks["hbm_gbs"], "traffic": None,
-                "peak_source": f"{peak_src} hbm_gbs"}
+        ach = nbytes[dom] / secs / 1e9
+        roof = {"kernel": dom, "bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s",
+                "frac": ach / hbm, "peak_source": f"{peak_src} hbm_gbs",
+                "algorithmic_bytes": nbytes[dom]}
+        if flops:
+            roof["tensor_frac"] = flops / secs / 1e12 / sustained
+    roof["traffic"] = (measured_traffic(["sparse_attn.cu", "common.cuh"],
+                                        "sparse_attn_dram_traffic_prefill_128k.txt")
+                       if dom == "attn" else None)
 
     attn_tflops = attn_flops / (stage_mean["attn"] / 1000.0) / 1e12
     attn_merge_tflops = attn_flops / ((stage_mean["attn"] + stage_mean["merge"]) / 1000.0) / 1e12

@@ -79,6 +79,13 @@ M1 = Workload("chunked_prefill_1m", 1, 8192, 1056768, 1048576, 64, 8, 128, seed=
 
 CONFIGS = {w.name: w for w in (TINY, P32, P128, DECODE, M1)}
 
+# Profiling-sized prefill with the 128K workload's structure (R = 8, sink and
+# recency): ~2.2 GB of pieces, larger than L2, small enough for hardware
+# counter capture.
+PROFILE_8K = Workload("profile_8k_r8", 1, 8192, 8192, 0, 32, 4, 128, seed=3, sink=True,
+                      recency=True)
+ALL = dict(CONFIGS, **{PROFILE_8K.name: PROFILE_8K})
+
 
 def small(name, batch, n_q, n_kv, q_pos0, h_q, h_kv, d_idx, seed, **kw) -> Workload:
     """A parity-sized workload (ragged tails, several tiles)."""
