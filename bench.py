@@ -262,38 +262,57 @@ def bench_e2e(w, buf, dev_inp, steps, world):
 
 
 class CpuOracleSample:
-    """The oracle, as it stands, on a bounded sample of the workload's query rows."""
+    """The oracle, as it stands, on a bounded sample of the workload's query rows.
 
-    def __init__(self, w, n_rows=16, seed=0):
+    The sample size is calibrated so that one run() takes about `target_s`
+    seconds on this host: a first pass over one row per core measures the
+    per-row cost, then the row count is fixed for every later run().
+    """
+
+    def __init__(self, w, target_s=15.0, seed=0):
         import oracle
         from block_sparse_attention_32_b200 import workloads as wl
         self.oracle, self.w = oracle, w
         inp = wl.make_inputs(w, "cpu")
-        rng = np.random.default_rng(seed)
-        self.rows = np.sort(rng.choice(w.n_q, size=min(n_rows, w.n_q), replace=False)).astype(np.int64)
         bits = oracle.bf16_bits
         self.k, self.v, self.ki = bits(inp["k"]), bits(inp["v"]), bits(inp["k_idx"])
-        self.q_rows = bits(inp["q"][0, self.rows])
-        self.qi_rows = bits(inp["q_idx"][0, self.rows])
+        self.q_all, self.qi_all = inp["q"][0], inp["q_idx"][0]
+        self.cores = int(os.environ.get("OMP_NUM_THREADS", len(os.sched_getaffinity(0))))
+        self.rng = np.random.default_rng(seed)
+        self._pick(min(self.cores, w.n_q))
+        t0 = time.perf_counter()
+        self._forward()
+        per_row = (time.perf_counter() - t0) / len(self.rows)
+        n = int(max(self.cores, min(w.n_q, target_s / max(per_row, 1e-9))))
+        self._pick(n)
+
+    def _pick(self, n):
+        w = self.w
+        self.rows = np.sort(self.rng.choice(w.n_q, size=n, replace=False)).astype(np.int64)
+        bits = self.oracle.bf16_bits
+        self.q_rows = bits(self.q_all[self.rows])
+        self.qi_rows = bits(self.qi_all[self.rows])
         self.pos = w.q_pos0 + self.rows
         self.bat = np.zeros_like(self.rows)
 
-    def run(self):
-        t0 = time.perf_counter()
+    def _forward(self):
         self.oracle.forward_rows(self.q_rows, self.qi_rows, self.pos, self.bat, self.k, self.v,
                                  self.ki, self.w.scale)
+
+    def run(self):
+        t0 = time.perf_counter()
+        self._forward()
         dt = time.perf_counter() - t0
-        cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
         w = self.w
-        return {"value": len(self.rows) / dt, "unit": "queries/s", "cores": cores,
+        return {"value": len(self.rows) / dt, "unit": "queries/s", "cores": self.cores,
                 "kind": "oracle",
                 "sample": f"{len(self.rows)} random query rows of {w.name} (all {w.h_kv} groups, "
                           f"{w.h_q} heads): fp64 index scores + selection + attention; "
                           f"{dt:.1f} s"}
 
 
-def cpu_baseline(w, n_rows=16):
-    return CpuOracleSample(w, n_rows).run()
+def cpu_baseline(w, target_s=15.0):
+    return CpuOracleSample(w, target_s).run()
 
 
 def main():
@@ -318,7 +337,7 @@ def main():
     if args.impl == "reference":
         if rank != 0:
             return
-        sample = CpuOracleSample(w, n_rows=4)
+        sample = CpuOracleSample(w, target_s=6.0)
         vals = []
         for _ in range(args.warmup):
             sample.run()
@@ -327,7 +346,7 @@ def main():
         v = statistics.median(x["value"] for x in vals)
         line = {"impl": "reference", "metric": "prefill_128k_queries_per_s", "value": v,
                 "unit": "queries/s", "n_gpus": 0, "steps": args.steps, "warmup": args.warmup,
-                "ms_per_step": 1000.0 * 4 / v, "higher_is_better": True, "scaling": "weak",
+                "ms_per_step": 1000.0 * len(sample.rows) / v, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "f64", "data": "synthetic",
                 "config": {"workload": w.name, "batch": w.batch, "seq_len": w.n_kv,
                            "h_q": w.h_q, "h_kv": w.h_kv, "d_idx": w.d_idx, "topk_blocks": 16,
