@@ -25,6 +25,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 import numpy as np
@@ -47,7 +48,7 @@ def load_peaks():
 
 
 def work_counts(w):
-    """Algorithmic FLOPs and entry count of one pass (formulas stated in the design notes)."""
+    """Algorithmic FLOPs and (query, group, block) entry count of one pass."""
     B, G, R, d_idx = w.batch, w.h_kv, w.h_q // w.h_kv, w.d_idx
     t = w.q_pos0 + np.arange(w.n_q, dtype=np.int64)
     own = t // 128
@@ -63,7 +64,7 @@ def work_counts(w):
 
 
 def bytes_model(w, n_entries, n_pieces_nonempty):
-    """Algorithmic DRAM bytes per launch of each kernel (design notes, section 7).
+    """Algorithmic DRAM bytes per launch of each kernel.
 
     attention: per (query, block) entry the R gathered Q rows (256 B each) and
     the R fp32 pieces written (512 B acc + 8 B (m, l)); per selected (batch,
@@ -187,11 +188,19 @@ def barrier(world):
 
 
 def max_over_ranks(x, world):
+    """The maximum of a per-rank float over all ranks (the job's time)."""
     if world == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(units_per_rank, ms_local, world):
+    """Whole-job throughput: units of all ranks / the slowest rank's time."""
+    ms = max_over_ranks(ms_local, world)
+    return world * units_per_rank / (ms / 1000.0), ms
 
 
 def bench_workload(w, steps, warmup, world, rank, with_e2e=True):
@@ -364,8 +373,7 @@ def main():
     import __graft_entry__
     __graft_entry__.build()
 
-    clk_path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{rank}.csv")
-    os.makedirs(os.path.dirname(clk_path), exist_ok=True)
+    clk_path = os.path.join(tempfile.gettempdir(), f"msa_bench_clocks_{os.getpid()}.csv")
     proc = sample_clocks(None, clk_path) if rank == 0 else None
     total_ms, stage_med, stage_mean, e2e, n_pieces = bench_workload(w, args.steps, args.warmup,
                                                                     world, rank)
@@ -374,20 +382,18 @@ def main():
         proc.wait()
     clocks = summarize_clocks(clk_path, local) if rank == 0 else None
 
-    total_ms = max_over_ranks(total_ms, world)
-    ms_step = total_ms / args.steps
-    qps = world * w.n_q / (ms_step / 1000.0)
+    qps, ms_step = job_throughput(w.n_q, total_ms / args.steps, world)
 
     decode = None
     if not args.no_decode:
         dw = wl.DECODE
         dms, dstage, _, _, dpieces = bench_workload(dw, max(3, args.steps), args.warmup, world,
                                                     rank, with_e2e=False)
-        dms = max_over_ranks(dms, world) / max(3, args.steps)
+        dtps, dms = job_throughput(dw.batch, dms / max(3, args.steps), world)
         kidx_bytes = dw.batch * dw.n_kv * dw.d_idx * 2
         sel_kv_bytes = dpieces * 65536
         read_bytes = kidx_bytes + sel_kv_bytes
-        decode = {"workload": dw.name, "tokens_per_s": world * dw.batch / (dms / 1000.0),
+        decode = {"workload": dw.name, "tokens_per_s": dtps,
                   "ms_per_step": dms, "stages_ms": dstage,
                   "index_scan_gbs": kidx_bytes / (dstage["index"] / 1000.0) / 1e9,
                   "bytes_read_per_step": read_bytes,
