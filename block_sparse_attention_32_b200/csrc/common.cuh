@@ -117,6 +117,19 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   return mbar_wait_slow(bar, parity, abort, err);
 }
 
+// Waits, bounded but regardless of the abort flag, for a phase that an issued
+// copy completes: a block drains its copies in flight before it exits, also
+// after an abort.
+static __device__ __noinline__ void mbar_drain(uint64_t* bar, uint32_t parity, int32_t* err) {
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t it = 0; !mbar_try_wait_sleep(bar, parity, kWaitSleepNs); ++it) {
+    if (global_timer_ns() - t0 > kWaitLimitNs || it > (1u << 30)) {
+      report(err, MSA_DEVERR_TIMEOUT);
+      return;
+    }
+  }
+}
+
 // ---------------------------------------------------------------------------
 // TMA tile loads (no multicast)
 // ---------------------------------------------------------------------------

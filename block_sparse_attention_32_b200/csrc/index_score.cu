@@ -17,9 +17,10 @@
 //    MMAs into two 256-column TMEM accumulators, warps 2-5 take the two row
 //    maxima of each accumulator and store them.
 //  * index_score_decode_kernel -- one query per sequence (decode): a
-//    streaming scan of k_idx, HBM-bound.  Each warp reads 16-key tiles
-//    straight into mma.sync fragments (16-byte loads) and multiplies them by
-//    the G <= 8 index queries of the sequence (m16n8k16: keys x groups).
+//    streaming scan of k_idx, HBM-bound.  TMA streams 32 KB key blocks
+//    through a shared-memory ring; consumer warps multiply them by the
+//    G <= 8 index queries of the sequence with mma.sync (m16n8k16: keys x
+//    groups) and keep each group's block maximum.
 #include "common.cuh"
 
 namespace msa {
@@ -186,12 +187,29 @@ __global__ void __launch_bounds__(192, 1)
 // ---------------------------------------------------------------------------
 // decode: one query per sequence, d_idx = 128, shared index key head, G <= 8
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
-  uint4 r;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-               : "l"(p));
-  return r;
+// A streaming scan of k_idx.  The units are the (sequence, candidate block)
+// pairs, split into one contiguous range per CTA (persistent grid, one CTA
+// per SM).  Warp 0 streams each unit's 32 KB key block into a ring of
+// shared-memory stages with TMA (two 64-column boxes, 128-byte swizzle), so
+// that up to kDecStages x 32 KB per SM are in flight.  Each consumer warp
+// owns the stages s with s % kDecConsumers == its index (one consumer per
+// stage keeps the barrier phases unambiguous) and multiplies the block by the
+// sequence's G <= 8 index queries with mma.sync m16n8k16: A = 16 keys x 16
+// dims through ldmatrix, B = the queries held in registers; the block score
+// of group g is the maximum of column g over the 128 keys.
+constexpr int kDecStages = 6;
+constexpr int kDecConsumers = 3;
+static_assert(kDecStages % kDecConsumers == 0, "a stage must always have the same consumer");
+constexpr int kDecThreads = 32 * (1 + kDecConsumers);
+constexpr int kDecStageBytes = kBlock * 128 * 2;    // 128 keys x 128 dims bf16
+constexpr int kDecSmemBytes = 1024 + kDecStages * kDecStageBytes + 2 * kDecStages * 8 + 16;
+
+__device__ __forceinline__ void ldmatrix_x4(uint32_t addr, uint32_t& r0, uint32_t& r1,
+                                            uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr)
+               : "memory");
 }
 
 __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint32_t a1,
@@ -204,90 +222,117 @@ __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint3
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-__device__ __forceinline__ uint32_t u4get(const uint4& v, int i) {
-  return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
-}
+__global__ void __launch_bounds__(kDecThreads, 1)
+    index_score_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
+                              const __nv_bfloat16* __restrict__ q_idx, int64_t qs_b,
+                              int64_t qs_h, int64_t batch, int64_t q_pos0, int32_t G,
+                              float* __restrict__ pooled, int64_t stride, int32_t* err) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(base + kDecStages * kDecStageBytes);
+  uint64_t* empty = full + kDecStages;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + kDecStages);
 
-// Fragment trick: the reduction over the 128 index dimensions is order-free,
-// so the k index of the m16n8k16 fragments is mapped to physical dimensions
-// such that every thread reads 64 contiguous bytes of each of its two key
-// rows: at k-step s, thread column-group cq covers logical k {2cq, 2cq+1} ->
-// dims 32cq + 4s + {0,1} and logical k {2cq+8, 2cq+9} -> dims 32cq + 4s + {2,3}.
-// A (keys) and B (index queries) use the same map.
-constexpr int kDecodeBlocksPerWarp = 4;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t own = q_pos0 / kBlock;                  // candidates per sequence
+  const int64_t total = batch * own;
+  const int64_t u0 = total * blockIdx.x / gridDim.x;
+  const int n = (int)(total * (blockIdx.x + 1) / gridDim.x - u0);
 
-__global__ void __launch_bounds__(128)
-    index_score_decode_kernel(const __nv_bfloat16* __restrict__ q_idx, int64_t qs_b,
-                              int64_t qs_h, const __nv_bfloat16* __restrict__ k_idx,
-                              int64_t ks_b, int64_t ks_t, int64_t q_pos0, int32_t G,
-                              float* __restrict__ pooled, int64_t stride) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int b = blockIdx.y;
-  const int64_t own = q_pos0 / kBlock;
-  const int64_t cbeg = ((int64_t)blockIdx.x * 4 + warp) * kDecodeBlocksPerWarp;
-  if (cbeg >= own) return;
-  const int64_t cend = min64(cbeg + kDecodeBlocksPerWarp, own);
-  const int gq = lane >> 2, cq = lane & 3;
-
-  uint4 qv[4];
-  if (gq < G) {
-    const __nv_bfloat16* qp = q_idx + (int64_t)b * qs_b + (int64_t)gq * qs_h + 32 * cq;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) qv[i] = *reinterpret_cast<const uint4*>(qp + 8 * i);
-  } else {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) qv[i] = make_uint4(0, 0, 0, 0);
-  }
-
-  for (int64_t c = cbeg; c < cend; ++c) {
-    const __nv_bfloat16* kb = k_idx + (int64_t)b * ks_b + (c * kBlock) * ks_t + 32 * cq;
-    float mx0 = -INFINITY, mx1 = -INFINITY;
-    uint4 cur[8], nxt[8];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      cur[i] = ld_stream_v4(kb + (int64_t)gq * ks_t + 8 * i);
-      cur[4 + i] = ld_stream_v4(kb + (int64_t)(gq + 8) * ks_t + 8 * i);
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kDecStages; ++i) {
+      mbar_init(full + i, 1);
+      mbar_init(empty + i, 1);
     }
+    *abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  __syncthreads();
+
+  if (warp == 0) {
+    if (lane == 0) {
+      prefetch_tensormap(&tm_k);
+      int i = 0;
+      for (; i < n; ++i) {
+        const int s = i % kDecStages;
+        if (i >= kDecStages &&
+            !mbar_wait(empty + s, ((i / kDecStages) - 1) & 1, abort_flag, err))
+          break;
+        const int64_t u = u0 + i;
+        const int64_t b = u / own, c = u - b * own;
+        uint8_t* dst = base + s * kDecStageBytes;
+        mbar_arrive_expect_tx(full + s, kDecStageBytes);
+        tma_load_4d(dst, &tm_k, full + s, 0, (int32_t)(c * kBlock), 0, (int32_t)b);
+        tma_load_4d(dst + kDecStageBytes / 2, &tm_k, full + s, 64, (int32_t)(c * kBlock), 0,
+                    (int32_t)b);
+      }
+      // no copy may still be writing this block's shared memory when it exits
+      for (int j = (i > kDecStages ? i - kDecStages : 0); j < i; ++j)
+        mbar_drain(full + j % kDecStages, (j / kDecStages) & 1, err);
+    }
+  } else {
+    const int cw = warp - 1;
+    const int gq = lane >> 2, tq = lane & 3;
+    // ldmatrix row of this lane inside a 16-key tile, and its 128-byte swizzle phase
+    const int lrow = (lane & 7) + ((lane >> 3) & 1) * 8;
+    const int hi = lane >> 4;                          // second 8 dims of a k-step
+    uint32_t bq[16];
+    int64_t qb = -1;
+    for (int i = cw; i < n; i += kDecConsumers) {
+      const int s = i % kDecStages;
+      const int64_t u = u0 + i;
+      const int64_t b = u / own, c = u - b * own;
+      if (b != qb) {
+        // B fragments: k pairs (16 ks + 2 tq, +1) and (16 ks + 8 + 2 tq, +1) of group gq
+        const __nv_bfloat16* qp = q_idx + b * qs_b + (int64_t)gq * qs_h + 2 * tq;
 #pragma unroll
-    for (int mt = 0; mt < 8; ++mt) {
-      if (mt < 7) {
-        const __nv_bfloat16* kn = kb + (int64_t)(16 * (mt + 1)) * ks_t;
+        for (int ks = 0; ks < 8; ++ks) {
+          bq[2 * ks] = gq < G ? *reinterpret_cast<const uint32_t*>(qp + 16 * ks) : 0u;
+          bq[2 * ks + 1] = gq < G ? *reinterpret_cast<const uint32_t*>(qp + 16 * ks + 8) : 0u;
+        }
+        qb = b;
+      }
+      if (!mbar_wait(full + s, (i / kDecStages) & 1, abort_flag, err)) break;
+      const uint32_t sbase = smem_u32(base + s * kDecStageBytes);
+      float acc[8][4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          nxt[i] = ld_stream_v4(kn + (int64_t)gq * ks_t + 8 * i);
-          nxt[4 + i] = ld_stream_v4(kn + (int64_t)(gq + 8) * ks_t + 8 * i);
+      for (int mt = 0; mt < 8; ++mt) {
+        acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
+      }
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        // 16-byte chunk of this lane's row, swizzled by the row (row & 7 == lane & 7)
+        const uint32_t chunk = (uint32_t)((2 * (ks & 3) + hi) ^ (lane & 7));
+        const uint32_t kaddr = sbase + (ks >> 2) * (kDecStageBytes / 2) + lrow * 128 + chunk * 16;
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt) {
+          uint32_t a0, a1, a2, a3;
+          ldmatrix_x4(kaddr + mt * 16 * 128, a0, a1, a2, a3);
+          mma_bf16_16816(acc[mt], a0, a1, a2, a3, bq[2 * ks], bq[2 * ks + 1]);
         }
       }
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+      float mx0 = -INFINITY, mx1 = -INFINITY;   // groups 2 tq and 2 tq + 1
 #pragma unroll
-      for (int s = 0; s < 8; ++s) {
-        // pair p = 2s / 2s+1 of the thread's 16 bf16 pairs; uint4 index p/4, component p%4
-        const uint32_t a0 = u4get(cur[(2 * s) >> 2], (2 * s) & 3);
-        const uint32_t a2 = u4get(cur[(2 * s + 1) >> 2], (2 * s + 1) & 3);
-        const uint32_t a1 = u4get(cur[4 + ((2 * s) >> 2)], (2 * s) & 3);
-        const uint32_t a3 = u4get(cur[4 + ((2 * s + 1) >> 2)], (2 * s + 1) & 3);
-        const uint32_t b0 = u4get(qv[(2 * s) >> 2], (2 * s) & 3);
-        const uint32_t b1 = u4get(qv[(2 * s + 1) >> 2], (2 * s + 1) & 3);
-        mma_bf16_16816(acc, a0, a1, a2, a3, b0, b1);
+      for (int mt = 0; mt < 8; ++mt) {
+        mx0 = fmaxf(mx0, fmaxf(acc[mt][0], acc[mt][2]));
+        mx1 = fmaxf(mx1, fmaxf(acc[mt][1], acc[mt][3]));
       }
-      mx0 = fmaxf(mx0, fmaxf(acc[0], acc[2]));
-      mx1 = fmaxf(mx1, fmaxf(acc[1], acc[3]));
-      if (mt < 7) {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(empty + s);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) cur[i] = nxt[i];
+      for (int o = 4; o < 32; o <<= 1) {
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
       }
-    }
-#pragma unroll
-    for (int o = 4; o < 32; o <<= 1) {
-      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
-      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
-    }
-    if (gq == 0) {
-      const int g0 = 2 * cq, g1 = 2 * cq + 1;
-      if (g0 < G) pooled[((int64_t)b * G + g0) * stride + c] = mx0;
-      if (g1 < G) pooled[((int64_t)b * G + g1) * stride + c] = mx1;
+      if (gq == 0) {
+        const int g0 = 2 * tq, g1 = 2 * tq + 1;
+        if (g0 < G) pooled[(b * G + g0) * stride + c] = mx0;
+        if (g1 < G) pooled[(b * G + g1) * stride + c] = mx1;
+      }
     }
   }
+  __syncthreads();
 }
 
 // ---------------------------------------------------------------------------
@@ -321,17 +366,23 @@ cudaError_t launch_index_score_prefill(const CUtensorMap& tm_q, const CUtensorMa
   return cudaGetLastError();
 }
 
-cudaError_t launch_index_score_decode(const void* q_idx, int64_t qs_b, int64_t qs_h,
-                                      const void* k_idx, int64_t ks_b, int64_t ks_t,
-                                      int64_t batch, int64_t q_pos0, int32_t G, float* pooled,
-                                      int64_t stride, cudaStream_t st) {
-  const int64_t own = q_pos0 / kBlock;
-  if (own == 0) return cudaSuccess;
-  const int64_t per_cta = 4 * kDecodeBlocksPerWarp;
-  dim3 grid((unsigned)((own + per_cta - 1) / per_cta), (unsigned)batch);
-  index_score_decode_kernel<<<grid, 128, 0, st>>>(
-      reinterpret_cast<const __nv_bfloat16*>(q_idx), qs_b, qs_h,
-      reinterpret_cast<const __nv_bfloat16*>(k_idx), ks_b, ks_t, q_pos0, G, pooled, stride);
+cudaError_t launch_index_score_decode(const CUtensorMap& tm_k, const void* q_idx, int64_t qs_b,
+                                      int64_t qs_h, int64_t batch, int64_t q_pos0, int32_t G,
+                                      float* pooled, int64_t stride, int32_t* err,
+                                      cudaStream_t st) {
+  const int64_t total = batch * (q_pos0 / kBlock);
+  if (total == 0) return cudaSuccess;
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  auto k = index_score_decode_kernel;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       kDecSmemBytes);
+  if (e != cudaSuccess) return e;
+  const int64_t grid = min64(total, sms);
+  k<<<(unsigned)grid, kDecThreads, kDecSmemBytes, st>>>(
+      tm_k, reinterpret_cast<const __nv_bfloat16*>(q_idx), qs_b, qs_h, batch, q_pos0, G, pooled,
+      stride, err);
   return cudaGetLastError();
 }
 

@@ -12,8 +12,8 @@ namespace msa {
 cudaError_t launch_index_score_prefill(const CUtensorMap&, const CUtensorMap&, int, int64_t,
                                        int64_t, int64_t, int32_t, int32_t, float*, int64_t,
                                        int32_t*, cudaStream_t);
-cudaError_t launch_index_score_decode(const void*, int64_t, int64_t, const void*, int64_t,
-                                      int64_t, int64_t, int64_t, int32_t, float*, int64_t,
+cudaError_t launch_index_score_decode(const CUtensorMap&, const void*, int64_t, int64_t,
+                                      int64_t, int64_t, int32_t, float*, int64_t, int32_t*,
                                       cudaStream_t);
 cudaError_t launch_topk_blocks(const float*, int64_t, int64_t, int64_t, int64_t, int32_t*,
                                cudaStream_t);
@@ -137,10 +137,15 @@ msa_status msa_index_score_maxpool(const msa_dims* d, msa_tensor q_idx, msa_tens
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const int32_t G = d->h_kv;
   if (d->n_q == 1 && d->h_kidx == 1 && d->d_idx == 128 && G <= 8) {
-    return from_cuda(msa::launch_index_score_decode(q_idx.ptr, q_idx.s_batch, q_idx.s_head,
-                                                    k_idx.ptr, k_idx.s_batch, k_idx.s_tok,
+    // k_idx [B, 1, n_kv, 128]: dims {128, n_kv, 1, B}, box {64, 128, 1, 1} (one key block
+    // per pair of loads)
+    CUtensorMap tk;
+    if ((s = make_map(&tk, k_idx.ptr, d->d_idx, d->n_kv, d->h_kidx, d->batch, k_idx.s_tok,
+                      k_idx.s_head, k_idx.s_batch, 128, 1)) != MSA_OK)
+      return s;
+    return from_cuda(msa::launch_index_score_decode(tk, q_idx.ptr, q_idx.s_batch, q_idx.s_head,
                                                     d->batch, d->q_pos0, G, pooled,
-                                                    pooled_row_stride, st));
+                                                    pooled_row_stride, dev_err, st));
   }
   CUtensorMap tq, tk;
   // q_idx [B, n_q, G, d_idx]: dims {d_idx, G, n_q, B}, box {64, 1, 128, 1}
