@@ -95,8 +95,8 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 constexpr uint32_t kWaitSleepNs = 1000000u;       // longest single sleep: 1 ms
 
-static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                           int32_t* err) {
+__device__ __forceinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                               int32_t* err) {
   const uint64_t t0 = global_timer_ns();
   for (uint32_t it = 0;; ++it) {
     if (mbar_try_wait_sleep(bar, parity, kWaitSleepNs)) return true;
@@ -109,8 +109,9 @@ static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parit
   }
 }
 
-// Fast path inline, the bounded sleeping loop out of line (keeps the
-// instruction footprint of the many wait sites small).
+// Fast path first, then the bounded sleeping loop.  Both are inlined: a call
+// would pin the callee to one register budget, which kernels that resize
+// their warpgroups' registers (setmaxnreg) cannot share.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           int32_t* err) {
   if (mbar_try_wait(bar, parity)) return true;
@@ -120,7 +121,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
 // Waits, bounded but regardless of the abort flag, for a phase that an issued
 // copy completes: a block drains its copies in flight before it exits, also
 // after an abort.
-static __device__ __noinline__ void mbar_drain(uint64_t* bar, uint32_t parity, int32_t* err) {
+__device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity, int32_t* err) {
   const uint64_t t0 = global_timer_ns();
   for (uint32_t it = 0; !mbar_try_wait_sleep(bar, parity, kWaitSleepNs); ++it) {
     if (global_timer_ns() - t0 > kWaitLimitNs || it > (1u << 30)) {
@@ -142,8 +143,35 @@ __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, u
       : "memory");
 }
 
+// TMA tile store shared -> global (no multicast), tracked per thread by bulk groups
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src, int32_t x,
+                                             int32_t y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(smem_u32(src)), "r"(x), "r"(y)
+      : "memory");
+}
+
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// named barrier `id` (1..15) over `nthreads` threads (a multiple of 32)
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// per-warpgroup register reallocation (every thread of the warpgroup executes it)
+// ---------------------------------------------------------------------------
+template <int N>
+__device__ __forceinline__ void setmaxnreg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void setmaxnreg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 // ---------------------------------------------------------------------------
@@ -154,6 +182,16 @@ __device__ __forceinline__ void cp_async_16(void* dst, const void* src, uint32_t
                "r"(src_bytes)
                : "memory");
 }
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+// waits until at most N of this thread's committed cp.async groups are pending
+template <int N>
+__device__ __forceinline__ void cp_async_wait_group() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 __device__ __forceinline__ void cp_async_wait_all() {
   asm volatile("cp.async.wait_all;" ::: "memory");
 }

@@ -4,6 +4,7 @@
 #include <cudaTypedefs.h>
 
 #include <cmath>
+#include <cstring>
 #include <mutex>
 
 #include "common.cuh"
@@ -20,7 +21,8 @@ cudaError_t launch_topk_blocks(const float*, int64_t, int64_t, int64_t, int64_t,
 size_t block_lists_workspace(int64_t, int64_t, int64_t);
 cudaError_t launch_block_lists(const int32_t*, int64_t, int64_t, int64_t, int64_t, int32_t*,
                                int32_t*, int64_t, void*, int32_t*, cudaStream_t);
-cudaError_t launch_sparse_attn(const CUtensorMap&, const CUtensorMap&, const void*, int64_t,
+cudaError_t launch_sparse_attn(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
+                               const void*, int64_t,
                                int64_t, int64_t, const int32_t*, const int32_t*, int64_t,
                                int64_t, int64_t, int64_t, int32_t, int32_t, int32_t, float,
                                float*, float*, int32_t*, cudaStream_t);
@@ -104,6 +106,21 @@ msa_status make_map(CUtensorMap* map, const void* ptr, uint64_t inner, uint64_t 
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides,
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? MSA_OK : MSA_ERR_CUDA;
+}
+
+// 2-D fp32 map over rows of 128 floats (512-byte rows): dims {128, rows}, box
+// {32, box_rows}, 128-byte swizzle (the layout the writer stages in shared memory)
+msa_status make_map_rows_f32(CUtensorMap* map, void* ptr, uint64_t rows, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return MSA_ERR_CUDA;
+  cuuint64_t dims[2] = {128, rows};
+  cuuint64_t strides[1] = {128 * sizeof(float)};
+  cuuint32_t box[2] = {32, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, ptr, dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? MSA_OK : MSA_ERR_CUDA;
 }
 
@@ -221,8 +238,18 @@ msa_status msa_sparse_attn_fwd(const msa_dims* d, msa_tensor q, msa_tensor k, ms
   if ((s = make_map(&tv, v.ptr, MSA_HEAD_DIM, d->n_kv, d->h_kv, d->batch, v.s_tok, v.s_head,
                     v.s_batch, 128, 1)) != MSA_OK)
     return s;
+  // part_acc [B, n_q, G, 16, R, 128] fp32 as rows of 128 floats; for R >= 8 one
+  // entry's R rows are written by TMA stores of R x 32 floats
+  CUtensorMap to;
+  std::memset(&to, 0, sizeof(to));
+  const int64_t R = d->h_q / d->h_kv;
+  if (R >= 8) {
+    const int64_t rows = d->batch * d->n_q * d->h_kv * MSA_TOPK_BLOCKS * R;
+    if (rows >= (int64_t(1) << 31)) return MSA_ERR_UNSUPPORTED;
+    if ((s = make_map_rows_f32(&to, part_acc, (uint64_t)rows, (uint32_t)R)) != MSA_OK) return s;
+  }
   return from_cuda(msa::launch_sparse_attn(
-      tk, tv, q.ptr, q.s_batch, q.s_tok, q.s_head, blk_offsets, entries, n_seg, total, d->n_q,
+      tk, tv, to, q.ptr, q.s_batch, q.s_tok, q.s_head, blk_offsets, entries, n_seg, total, d->n_q,
       d->q_pos0, d->h_kv, d->h_q, (int32_t)nblk, d->scale, part_ml, part_acc, dev_err,
       reinterpret_cast<cudaStream_t>(stream)));
 }

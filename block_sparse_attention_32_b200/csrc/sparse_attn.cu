@@ -21,31 +21,49 @@
 //                             segment offsets) and publishes one descriptor
 //                             per chunk -- (b, g, block, count, piece, flags)
 //                             and its entries -- in an 8-deep shared ring
-//   warp 1      MMA issuer:   S(n) = Q K^T, then O(n-1) = P V  (TMEM owner)
+//   warp 1      MMA issuer:   S(n) = Q K^T, then O(n-1) = P V, in that fixed order
 //   warp 2      TMA producer: K and V of each piece; K of the next piece is
 //                             loaded as soon as the last S MMA of the current
 //                             one is done, V as soon as its last P V is done
-//   warps 3-6   gather:       cp.async of the chunk's Q rows into a 3-deep ring
-//   warps 7-10  softmax:      S -> (m, l), P = bf16(e^{s-m}) written back into
-//                             the first 64 columns of its S buffer in TMEM
+//   warp 3      idle (fills the control warpgroup)
+//   warps 4-7   gather:       cp.async of the chunk's Q rows into a 3-deep ring
+//   warps 8-15  softmax:      two warpgroups, one per half of the keys; each
+//                             holds its 64 S values of a row in registers,
+//                             the halves exchange row maxima through shared
+//                             memory, and P = bf16(e^{s-m}) goes back into
+//                             the first 64 columns of the S buffer in TMEM
 //                             (the A operand of O = P V)
-//   warps 11-14 epilogue:     O -> the (m, l, acc) pieces in global memory:
-//                             each warp stages its 32 rows half a row (256 B)
-//                             at a time in shared memory and reads them back
-//                             transposed, so that one store instruction
+//   warps 16-19 epilogue:     O from TMEM half a row at a time, then the
+//                             (m, l, acc) pieces to global memory.  R >= 8:
+//                             the half rows are staged in 128B-swizzled
+//                             panels and each entry's R rows leave by TMA
+//                             tensor stores; R < 8: staged rows are read
+//                             back transposed so that one store instruction
 //                             writes two whole half rows (coalesced)
+// The five warpgroups split the register file unevenly (setmaxnreg).
 // Shared memory: K 32 KB, V 32 KB, 3 x 32 KB Q tiles (128B-swizzled K-major;
-// V is read N-major for P V), 34 KB output staging (half rows padded to 272
-// bytes so a warp's row-per-thread writes spread over all banks).  TMEM: S/P
-// in columns [0,256), O in [256,512), two buffers of 128 columns each; a Q
-// tile is released as soon as its S MMA is done, and S(n+2) waits for
-// O(n) = P(n) V, which reads P(n) from the same columns.
+// V is read N-major for P V), 34 KB output staging, (m, l) slots and the row
+// maxima the two softmax halves exchange.  TMEM: S/P in columns [0,256), O in
+// [256,512), two buffers of 128 columns each; a Q tile is released as soon as
+// its S MMA is done, S(n+2) waits for O(n) = P(n) V, which reads P(n) from
+// the same columns, and P V(n+2) waits until the epilogue has read O(n).
 #include "common.cuh"
 
 namespace msa {
 
-constexpr int kAttnThreads = 480;
-constexpr int kAttnMaxChunksPerItem = 8;
+constexpr int kAttnThreads = 640;
+// Registers per thread: 96 at launch (65536 / 640, rounded down to the
+// allocation unit); the control and gather warpgroups give registers back,
+// the two softmax warpgroups and the epilogue take them, and the five shares
+// add up to exactly the launch allocation.  The launcher checks the compiled
+// count before the first launch.
+constexpr int kAttnRegsAtLaunch = 96;
+constexpr int kRegsControl = 88, kRegsGather = 48, kRegsSoftmax = 120, kRegsEpilogue = 104;
+static_assert(kRegsControl + kRegsGather + 2 * kRegsSoftmax + kRegsEpilogue ==
+                  5 * kAttnRegsAtLaunch,
+              "warpgroup register shares must add up to the launch allocation");
+static_assert(kAttnThreads * kAttnRegsAtLaunch <= 65536, "register file");
+constexpr int kAttnMaxChunksPerItem = 32;
 constexpr int kQRing = 3;              // Q/P tiles in flight
 constexpr int kDescRing = 8;           // chunk descriptors in flight
 
@@ -60,10 +78,11 @@ constexpr int kOffV = 32768;           // 32768: [V lo | V hi]
 constexpr int kOffQP = 65536;          // kQRing x 32768: Q tile, then P
 constexpr int kStageRow = 272;                           // staged half row (256 B + pad)
 constexpr int kOffStage = kOffQP + kQRing * 32768;       // 128 staged rows
-constexpr int kOffML = kOffStage + 128 * kStageRow;      // 2 x 128 float2: (m, l) per row
-constexpr int kOffDesc = kOffML + 2048;                  // kDescRing descriptors
+constexpr int kOffML = kOffStage + 128 * kStageRow;      // [2 slots][2 halves][128] float2 (m, l)
+constexpr int kOffMX = kOffML + 4096;                    // [2][2 halves][128] float row maxima
+constexpr int kOffDesc = kOffMX + 2048;                  // kDescRing descriptors
 constexpr int kOffBar = kOffDesc + kDescRing * (int)sizeof(ChunkDesc);
-constexpr int kNumBars = 4 + 3 * kQRing + 6 + 2 * kDescRing;
+constexpr int kNumBars = 4 + 3 * kQRing + 6 + 2 * kDescRing + 2;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;         // TMEM base, abort flag
 constexpr int kAttnSmemBytes = 1024 + kOffMisc + 64;
 
@@ -71,7 +90,8 @@ enum {
   BAR_K_FULL = 0, BAR_K_EMPTY = 1, BAR_V_FULL = 2, BAR_V_EMPTY = 3,
   BAR_Q_FULL = 4, BAR_QP_EMPTY = 4 + kQRing, BAR_P_FULL = 4 + 2 * kQRing,
   BAR_S_FULL = 4 + 3 * kQRing, BAR_O_FULL = BAR_S_FULL + 2, BAR_O_EMPTY = BAR_S_FULL + 4,
-  BAR_D_FULL = BAR_S_FULL + 6, BAR_D_EMPTY = BAR_D_FULL + kDescRing
+  BAR_D_FULL = BAR_S_FULL + 6, BAR_D_EMPTY = BAR_D_FULL + kDescRing,
+  BAR_ML_EMPTY = BAR_D_EMPTY + kDescRing
 };
 
 struct AttnArgs {
@@ -107,6 +127,7 @@ template <int R>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     sparse_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k,
                            const __grid_constant__ CUtensorMap tm_v,
+                           const __grid_constant__ CUtensorMap tm_o,
                            const __grid_constant__ AttnArgs a) {
   constexpr int CH = 128 / R;
   constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128, 0);
@@ -117,6 +138,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                                              ~uintptr_t(1023));
   uint64_t* bar = reinterpret_cast<uint64_t*>(base + kOffBar);
   float2* ml_s = reinterpret_cast<float2*>(base + kOffML);
+  float* mx_x = reinterpret_cast<float*>(base + kOffMX);
   ChunkDesc* desc = reinterpret_cast<ChunkDesc*>(base + kOffDesc);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(base + kOffMisc + 4);
@@ -130,12 +152,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     for (int i = 0; i < kQRing; ++i) {
       mbar_init(bar + BAR_Q_FULL + i, 128);
       mbar_init(bar + BAR_QP_EMPTY + i, 1);
-      mbar_init(bar + BAR_P_FULL + i, 128);
+      mbar_init(bar + BAR_P_FULL + i, 256);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar + BAR_S_FULL + i, 1);
       mbar_init(bar + BAR_O_FULL + i, 1);
       mbar_init(bar + BAR_O_EMPTY + i, 128);
+      mbar_init(bar + BAR_ML_EMPTY + i, 128);
     }
     for (int i = 0; i < kDescRing; ++i) {
       mbar_init(bar + BAR_D_FULL + i, 1);
@@ -162,154 +185,135 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                                   (uint32_t)(((n / depth) + 1) & 1), abort_flag, err);
   };
 
-  if (warp == 0) {
-    // ---------------- scheduler ----------------
-    int64_t chunk = 0, piece = 0;
-    bool ok = true;
-    auto claim = [&](int64_t n) {      // lane 0 waits, the warp follows
-      bool r = true;
-      if (lane == 0) r = Wfree(BAR_D_EMPTY, kDescRing, n);
-      return __shfl_sync(0xffffffffu, r ? 1 : 0, 0) != 0;
-    };
-    for (int64_t item = blockIdx.x; ok && item < a.n_items; item += gridDim.x) {
-      const int64_t e0 = item * a.W;
-      const int64_t e1 = min64(e0 + a.W, a.n_entries);
-      int64_t pos = e0;
-      int64_t seg = warp_find_segment(a.blk_offsets, 0, a.n_seg, pos, lane);
-      while (pos < e1) {
-        const int64_t pend = min64(e1, (int64_t)a.blk_offsets[seg + 1]);
-        if (pend <= pos) {             // fewer entries listed than the sizes imply
-          if (lane == 0) {
-            report(err, MSA_DEVERR_BAD_ENTRY);
-            *abort_flag = 1;
-          }
-          ok = false;
-          break;
-        }
-        const int64_t bg = seg / a.nblk;
-        const int32_t c = (int32_t)(seg - bg * a.nblk);
-        const int32_t b = (int32_t)(bg / a.G), g = (int32_t)(bg - (int64_t)b * a.G);
-        for (int64_t cpos = pos; cpos < pend; cpos += CH) {
-          if (!claim(chunk)) {
+  // Roles by warpgroup; each warpgroup first resizes its registers (all four
+  // of its warps execute the same setmaxnreg).
+  if (warp < 4) {
+    setmaxnreg_dec<kRegsControl>();
+    if (warp == 0) {
+      // ---------------- scheduler ----------------
+      int64_t chunk = 0, piece = 0;
+      bool ok = true;
+      auto claim = [&](int64_t n) {      // lane 0 waits, the warp follows
+        bool r = true;
+        if (lane == 0) r = Wfree(BAR_D_EMPTY, kDescRing, n);
+        return __shfl_sync(0xffffffffu, r ? 1 : 0, 0) != 0;
+      };
+      for (int64_t item = blockIdx.x; ok && item < a.n_items; item += gridDim.x) {
+        const int64_t e0 = item * a.W;
+        const int64_t e1 = min64(e0 + a.W, a.n_entries);
+        int64_t pos = e0;
+        int64_t seg = warp_find_segment(a.blk_offsets, 0, a.n_seg, pos, lane);
+        while (pos < e1) {
+          const int64_t pend = min64(e1, (int64_t)a.blk_offsets[seg + 1]);
+          if (pend <= pos) {             // fewer entries listed than the sizes imply
+            if (lane == 0) {
+              report(err, MSA_DEVERR_BAD_ENTRY);
+              *abort_flag = 1;
+            }
             ok = false;
             break;
           }
-          ChunkDesc& d = desc[chunk % kDescRing];
-          const int cnt = (int)min64(CH, pend - cpos);
-          for (int i = lane; i < CH; i += 32) d.ent[i] = (i < cnt) ? a.entries[cpos + i] : -1;
-          if (lane == 0) {
-            d.b = b;
-            d.g = g;
-            d.c = c;
-            d.cnt = cnt;
-            d.piece = (int32_t)piece;
-            d.first = cpos == pos;
-            d.last = cpos + CH >= pend;
-          }
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bar + BAR_D_FULL + (int)(chunk % kDescRing));
-          ++chunk;
-        }
-        if (!ok) break;
-        ++piece;
-        pos = pend;
-        if (pos < e1) seg = warp_find_segment(a.blk_offsets, seg + 1, a.n_seg, pos, lane);
-      }
-    }
-    if (ok && claim(chunk)) {          // end marker
-      if (lane == 0) {
-        desc[chunk % kDescRing].cnt = -1;
-        mbar_arrive(bar + BAR_D_FULL + (int)(chunk % kDescRing));
-      }
-    }
-  } else if (warp == 1) {
-    // ---------------- MMA issuer ----------------
-    // S(n) and the pending P V(n-1) are issued in whichever order their
-    // inputs become ready (S(n) needs the gathered Q tile, P V(n-1) the
-    // softmax of n-1); S(n+1) always waits for P V(n-1), which frees S buffer.
-    if (lane == 0) {
-      int64_t pn = -1, pp = 0, v_ready = -1, last_s_piece = -1;
-      bool plast = false, ok = true;
-      auto pv_ready = [&](int64_t n, int64_t p) {
-        if (p != v_ready) {
-          if (!mbar_try_wait(bar + BAR_V_FULL, (uint32_t)(p & 1))) return false;
-          v_ready = p;
-        }
-        return mbar_try_wait(bar + BAR_P_FULL + (int)(n % kQRing),
-                             (uint32_t)((n / kQRing) & 1));
-      };
-      auto issue_pv = [&](int64_t n, bool last) {
-        const int ob = (int)(n & 1);
-        tc_fence_after();
-        const uint32_t va = smem_u32(base + kOffV);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          umma_bf16_ts(tmem + 256 + ob * 128, tmem + ob * 128 + kk * 8,
-                       smem_desc_sw128(va + kk * 2048, 16384, 1024), kIdescPV, kk > 0 ? 1u : 0u);
-        umma_commit(bar + BAR_O_FULL + ob);
-        if (last) umma_commit(bar + BAR_V_EMPTY);
-      };
-      for (int64_t n = 0;; ++n) {
-        if (!Wuse(BAR_D_FULL, kDescRing, n)) { ok = false; break; }
-        const ChunkDesc& d = desc[n % kDescRing];
-        if (d.cnt < 0) break;
-        const int64_t p = d.piece;
-        const bool first = d.first != 0, last = d.last != 0;
-        const int qb = (int)(n % kQRing), sb = (int)(n & 1);
-        bool s_done = false, k_ok = !first, pv_done = pn < 0, o_ok = n < 2;
-        const uint64_t t0 = global_timer_ns();
-        while (!(s_done && pv_done)) {
-          bool progress = false;
-          if (!pv_done && pv_ready(pn, pp)) {
-            issue_pv(pn, plast);
-            pv_done = progress = true;
-          }
-          if (!s_done) {
-            if (!k_ok) k_ok = mbar_try_wait(bar + BAR_K_FULL, (uint32_t)(p & 1));
-            // S buffer sb holds P(n-2) until O(n-2) = P(n-2) V is complete
-            if (!o_ok) o_ok = mbar_try_wait(bar + BAR_O_FULL + sb, (uint32_t)(((n - 2) >> 1) & 1));
-            if (k_ok && o_ok &&
-                mbar_try_wait(bar + BAR_Q_FULL + qb, (uint32_t)((n / kQRing) & 1))) {
-              tc_fence_after();
-              const uint32_t qa = smem_u32(base + kOffQP + qb * 32768);
-              const uint32_t ka = smem_u32(base + kOffK);
-#pragma unroll
-              for (int kk = 0; kk < 8; ++kk) {
-                const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-                umma_bf16(tmem + sb * 128, smem_desc_sw128(qa + off, 16, 1024),
-                          smem_desc_sw128(ka + off, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
-              }
-              umma_commit(bar + BAR_S_FULL + sb);
-              umma_commit(bar + BAR_QP_EMPTY + qb);
-              if (last) {
-                umma_commit(bar + BAR_K_EMPTY);
-                last_s_piece = p;
-              }
-              s_done = progress = true;
-            }
-          }
-          if (!progress) {
-            if (*abort_flag) { ok = false; break; }
-            if (global_timer_ns() - t0 > kWaitLimitNs) {
-              *abort_flag = 1;
-              report(err, MSA_DEVERR_TIMEOUT);
+          const int64_t bg = seg / a.nblk;
+          const int32_t c = (int32_t)(seg - bg * a.nblk);
+          const int32_t b = (int32_t)(bg / a.G), g = (int32_t)(bg - (int64_t)b * a.G);
+          for (int64_t cpos = pos; cpos < pend; cpos += CH) {
+            if (!claim(chunk)) {
               ok = false;
               break;
             }
-            __nanosleep(32);
+            ChunkDesc& d = desc[chunk % kDescRing];
+            const int cnt = (int)min64(CH, pend - cpos);
+            for (int i = lane; i < CH; i += 32) d.ent[i] = (i < cnt) ? a.entries[cpos + i] : -1;
+            if (lane == 0) {
+              d.b = b;
+              d.g = g;
+              d.c = c;
+              d.cnt = cnt;
+              d.piece = (int32_t)piece;
+              d.first = cpos == pos;
+              d.last = cpos + CH >= pend;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar + BAR_D_FULL + (int)(chunk % kDescRing));
+            ++chunk;
           }
+          if (!ok) break;
+          ++piece;
+          pos = pend;
+          if (pos < e1) seg = warp_find_segment(a.blk_offsets, seg + 1, a.n_seg, pos, lane);
         }
-        if (!ok) break;
-        pn = n;
-        pp = p;
-        plast = last;
       }
-      if (ok && pn >= 0) {
-        bool ready = false;
-        if (pp != v_ready) ready = Wuse(BAR_V_FULL, 1, pp);
-        else ready = true;
-        if (ready && Wuse(BAR_P_FULL, kQRing, pn)) {
-          issue_pv(pn, plast);
+      if (ok && claim(chunk)) {          // end marker
+        if (lane == 0) {
+          desc[chunk % kDescRing].cnt = -1;
+          mbar_arrive(bar + BAR_D_FULL + (int)(chunk % kDescRing));
+        }
+      }
+    } else if (warp == 1) {
+      // ---------------- MMA issuer ----------------
+      // Fixed order S(0), S(1), P V(0), S(2), P V(1), ...: S(n) needs the
+      // gathered Q tile, the piece's K and its S buffer back from P V(n-2);
+      // P V(n-1) needs the softmax of n-1 and the piece's V.  Every wait
+      // suspends in hardware (no polling).
+      if (lane == 0) {
+        int64_t pn = -1, pp = -1, v_ready = -1, last_s_piece = -1;
+        bool plast = false, ok = true;
+        auto issue_pv = [&](int64_t n, int64_t p, bool last) {
+          if (p != v_ready) {
+            if (!Wuse(BAR_V_FULL, 1, p)) return false;
+            v_ready = p;
+          }
+          if (!Wuse(BAR_P_FULL, kQRing, n)) return false;
+          // O buffer n & 1 is free once the epilogue of n-2 has read it
+          if (!Wfree(BAR_O_EMPTY, 2, n)) return false;
+          const int ob = (int)(n & 1);
+          tc_fence_after();
+          const uint32_t va = smem_u32(base + kOffV);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            umma_bf16_ts(tmem + 256 + ob * 128, tmem + ob * 128 + kk * 8,
+                         smem_desc_sw128(va + kk * 2048, 16384, 1024), kIdescPV,
+                         kk > 0 ? 1u : 0u);
+          umma_commit(bar + BAR_O_FULL + ob);
+          if (last) umma_commit(bar + BAR_V_EMPTY);
+          return true;
+        };
+        int64_t k_ready = -1;
+        for (int64_t n = 0;; ++n) {
+          if (!Wuse(BAR_D_FULL, kDescRing, n)) { ok = false; break; }
+          const ChunkDesc& d = desc[n % kDescRing];
+          if (d.cnt < 0) break;
+          const int64_t p = d.piece;
+          const bool last = d.last != 0;
+          const int qb = (int)(n % kQRing), sb = (int)(n & 1);
+          if (p != k_ready) {
+            if (!Wuse(BAR_K_FULL, 1, p)) { ok = false; break; }
+            k_ready = p;
+          }
+          // S buffer sb holds P(n-2) until O(n-2) = P(n-2) V is complete
+          if (n >= 2 && !Wuse(BAR_O_FULL, 2, n - 2)) { ok = false; break; }
+          if (!Wuse(BAR_Q_FULL, kQRing, n)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t qa = smem_u32(base + kOffQP + qb * 32768);
+          const uint32_t ka = smem_u32(base + kOffK);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+            umma_bf16(tmem + sb * 128, smem_desc_sw128(qa + off, 16, 1024),
+                      smem_desc_sw128(ka + off, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(bar + BAR_S_FULL + sb);
+          umma_commit(bar + BAR_QP_EMPTY + qb);
+          if (last) {
+            umma_commit(bar + BAR_K_EMPTY);
+            last_s_piece = p;
+          }
+          if (pn >= 0 && !issue_pv(pn, pp, plast)) { ok = false; break; }
+          pn = n;
+          pp = p;
+          plast = last;
+        }
+        if (ok && pn >= 0 && issue_pv(pn, pp, plast)) {
           // let the last completions land before the block can exit
           Wuse(BAR_QP_EMPTY, kQRing, pn);
           Wuse(BAR_O_FULL, 2, pn);
@@ -317,34 +321,38 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           if (last_s_piece >= 0) Wuse(BAR_K_EMPTY, 1, last_s_piece);
         }
       }
-    }
-  } else if (warp == 2) {
-    // ---------------- TMA producer: K/V of every piece ----------------
-    if (lane == 0) {
-      prefetch_tensormap(&tm_k);
-      prefetch_tensormap(&tm_v);
-      for (int64_t n = 0;; ++n) {
-        if (!Wuse(BAR_D_FULL, kDescRing, n)) break;
-        const ChunkDesc& d = desc[n % kDescRing];
-        if (d.cnt < 0) break;
-        if (d.first) {
-          const int64_t p = d.piece;
-          const int32_t b = d.b, g = d.g, c = d.c;
-          if (!Wfree(BAR_K_EMPTY, 1, p)) break;
-          mbar_arrive_expect_tx(bar + BAR_K_FULL, 32768);
-          tma_load_4d(base + kOffK, &tm_k, bar + BAR_K_FULL, 0, c * kBlock, g, b);
-          tma_load_4d(base + kOffK + 16384, &tm_k, bar + BAR_K_FULL, 64, c * kBlock, g, b);
-          if (!Wfree(BAR_V_EMPTY, 1, p)) break;
-          mbar_arrive_expect_tx(bar + BAR_V_FULL, 32768);
-          tma_load_4d(base + kOffV, &tm_v, bar + BAR_V_FULL, 0, c * kBlock, g, b);
-          tma_load_4d(base + kOffV + 16384, &tm_v, bar + BAR_V_FULL, 64, c * kBlock, g, b);
+    } else if (warp == 2) {
+      // ---------------- TMA producer: K/V of every piece ----------------
+      if (lane == 0) {
+        prefetch_tensormap(&tm_k);
+        prefetch_tensormap(&tm_v);
+        for (int64_t n = 0;; ++n) {
+          if (!Wuse(BAR_D_FULL, kDescRing, n)) break;
+          const ChunkDesc& d = desc[n % kDescRing];
+          if (d.cnt < 0) break;
+          if (d.first) {
+            const int64_t p = d.piece;
+            const int32_t b = d.b, g = d.g, c = d.c;
+            if (!Wfree(BAR_K_EMPTY, 1, p)) break;
+            mbar_arrive_expect_tx(bar + BAR_K_FULL, 32768);
+            tma_load_4d(base + kOffK, &tm_k, bar + BAR_K_FULL, 0, c * kBlock, g, b);
+            tma_load_4d(base + kOffK + 16384, &tm_k, bar + BAR_K_FULL, 64, c * kBlock, g, b);
+            if (!Wfree(BAR_V_EMPTY, 1, p)) break;
+            mbar_arrive_expect_tx(bar + BAR_V_FULL, 32768);
+            tma_load_4d(base + kOffV, &tm_v, bar + BAR_V_FULL, 0, c * kBlock, g, b);
+            tma_load_4d(base + kOffV + 16384, &tm_v, bar + BAR_V_FULL, 64, c * kBlock, g, b);
+          }
+          mbar_arrive(bar + BAR_D_EMPTY + (int)(n % kDescRing));
         }
-        mbar_arrive(bar + BAR_D_EMPTY + (int)(n % kDescRing));
       }
     }
-  } else if (warp < 7) {
+    // warp 3: idle
+  } else if (warp < 8) {
     // ---------------- gather: Q rows of each chunk ----------------
-    const int gt = tid - 96;   // 0..127
+    setmaxnreg_dec<kRegsGather>();
+    // thread = (row within an 8-row group, 16-byte column chunk); a warp
+    // instruction copies two whole 256-byte rows
+    const int gt = tid - 128;   // 0..127
     const int ch = gt & 15;
     for (int64_t n = 0;; ++n) {
       if (!Wuse(BAR_D_FULL, kDescRing, n)) break;
@@ -370,8 +378,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       fence_proxy_async_smem();
       mbar_arrive(bar + BAR_Q_FULL + qb);
     }
-  } else if (warp < 11) {
+  } else if (warp < 16) {
     // ---------------- softmax: S -> P, (m, l) ----------------
+    // warpgroup h (0, 1) takes keys 64h .. 64h+63 of every row; the two
+    // halves of a row exchange their maxima through shared memory (named
+    // barrier 1 + quarter, 64 threads) and each writes its own sum.
+    setmaxnreg_inc<kRegsSoftmax>();
+    const int h = (warp >> 2) - 2;
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
@@ -385,6 +398,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const int32_t c = d.c;
       if (!Wuse(BAR_S_FULL, 2, n)) break;
       tc_fence_after();
+      const uint32_t s_addr = tmem + lane_base + sb * 128;
+      uint32_t r0[32], r1[32];
+      tmem_ld_32x32b_x32(s_addr + 64 * h, r0);
+      tmem_ld_32x32b_x32(s_addr + 64 * h + 32, r1);
       const int64_t qi = (int64_t)(e >> 4);
       bool valid = (e >= 0) && (qi < a.n_q);
       int lim = 127;
@@ -392,63 +409,95 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const int64_t rel = a.q_pos0 + qi - (int64_t)c * kBlock;
         if (rel < 0) {
           valid = false;
-          report(err, MSA_DEVERR_BAD_ENTRY);
+          if (h == 0) report(err, MSA_DEVERR_BAD_ENTRY);
         } else if (rel < 127) {
           lim = (int)rel;
         }
       }
-      const uint32_t s_addr = tmem + lane_base + sb * 128;
-      float mx = -INFINITY;
-#pragma unroll 1
-      for (int j = 0; j < 4; ++j) {
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(s_addr + j * 32, r);
-        tmem_ld_wait();
+      if (!valid) lim = -1;                   // every weight of the row is zero
+      const int k0 = 64 * h;
+      // only rows of the query's own block mask keys (past the query); a warp
+      // with no such row skips every per-key compare
+      const bool masked = __any_sync(0xffffffffu, lim >= 0 && lim < 127);
+      tmem_ld_wait();
+      float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      if (!masked) {
 #pragma unroll
-        for (int x = 0; x < 32; ++x)
-          if (j * 32 + x <= lim) mx = fmaxf(mx, u2f(r[x]));
+        for (int x = 0; x < 32; x += 2) {
+          m4[0] = fmaxf(m4[0], u2f(r0[x]));
+          m4[1] = fmaxf(m4[1], u2f(r0[x + 1]));
+          m4[2] = fmaxf(m4[2], u2f(r1[x]));
+          m4[3] = fmaxf(m4[3], u2f(r1[x + 1]));
+        }
+      } else {
+#pragma unroll
+        for (int x = 0; x < 32; x += 2) {
+          m4[0] = fmaxf(m4[0], k0 + x <= lim ? u2f(r0[x]) : -INFINITY);
+          m4[1] = fmaxf(m4[1], k0 + x + 1 <= lim ? u2f(r0[x + 1]) : -INFINITY);
+          m4[2] = fmaxf(m4[2], k0 + 32 + x <= lim ? u2f(r1[x]) : -INFINITY);
+          m4[3] = fmaxf(m4[3], k0 + 33 + x <= lim ? u2f(r1[x + 1]) : -INFINITY);
+        }
       }
-      if (!valid) {
-        mx = 0.f;
-        lim = -1;                             // every weight of the row is zero
-      }
-      const float mneg = -mx * scale_log2;
+      const float mloc = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+      float* mxn = mx_x + (int)(n & 1) * 256;   // by parity: the partner reads it before n+2
+      mxn[h * 128 + row] = mloc;
+      tc_fence_before();                       // this half's S reads precede the other's P writes
+      named_bar_sync(1 + quarter, 64);
+      tc_fence_after();
+      float mx = fmaxf(mloc, mxn[(1 - h) * 128 + row]);
+      if (!valid) mx = 0.f;
+      // e^{s-m} = 2^{s log2(e) scale - m log2(e) scale}; a row with no valid
+      // key gets weight 2^-inf = 0 everywhere
+      const float mneg = valid ? -mx * scale_log2 : -INFINITY;
       float lsum[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 1
-      for (int j = 0; j < 4; ++j) {
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(s_addr + j * 32, r);
-        tmem_ld_wait();
+      // keys 32j..32j+31 -> columns 16j..16j+15 of this S buffer (already read).
+      // P is rounded to bf16 for the P V product; l sums the fp32 weights.
+      auto exp_pack_store = [&](const uint32_t (&r)[32], int j, bool mask) {
         uint32_t w[16];
 #pragma unroll
         for (int x = 0; x < 16; ++x) {
-          const int k0 = j * 32 + 2 * x;
-          // branch-free: exponentiate every key, then zero the ones past lim
           float p0 = ex2_approx(fmaf(u2f(r[2 * x]), scale_log2, mneg));
           float p1 = ex2_approx(fmaf(u2f(r[2 * x + 1]), scale_log2, mneg));
-          p0 = (k0 <= lim) ? p0 : 0.f;
-          p1 = (k0 + 1 <= lim) ? p1 : 0.f;
-          const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
-          lsum[x & 3] += __low2float(h2) + __high2float(h2);
-          w[x] = *reinterpret_cast<const uint32_t*>(&h2);
+          if (mask) {
+            const int kk = j * 32 + 2 * x;
+            p0 = (kk <= lim) ? p0 : 0.f;
+            p1 = (kk + 1 <= lim) ? p1 : 0.f;
+          }
+          lsum[x & 3] += p0 + p1;
+          w[x] = pack_bf16x2(p0, p1);
         }
-        // keys 32j..32j+31 -> columns 16j..16j+15 of this S buffer (already read)
         tmem_st_32x32b_x16(s_addr + j * 16, w);
+      };
+      if (!masked) {
+        exp_pack_store(r0, 2 * h, false);
+        exp_pack_store(r1, 2 * h + 1, false);
+      } else {
+        exp_pack_store(r0, 2 * h, true);
+        exp_pack_store(r1, 2 * h + 1, true);
       }
       tmem_st_wait();
       const float l = (lsum[0] + lsum[1]) + (lsum[2] + lsum[3]);
-      // (m, l) slot sb and O buffer sb are free once the epilogue of n-2 is done;
-      // P V(n) is issued only after this arrival
-      if (!Wfree(BAR_O_EMPTY, 2, n)) break;
-      ml_s[sb * 128 + row] = make_float2(mx * a.scale, l);
+      // (m, l) slot sb is free once the epilogue of n-2 has read it; P V(n)
+      // is issued only after both halves arrive
+      if (!Wfree(BAR_ML_EMPTY, 2, n)) break;
+      ml_s[(sb * 2 + h) * 128 + row] = make_float2(mx * a.scale, l);
       tc_fence_before();
       mbar_arrive(bar + BAR_P_FULL + qb);
     }
   } else {
     // ---------------- epilogue: O -> pieces ----------------
+    setmaxnreg_inc<kRegsEpilogue>();
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    // R >= 8: each warp stages half rows in two 32-column panels (32 rows x
+    // 128 B, 128-byte swizzle) and the first lane of each entry writes the
+    // entry's R rows with one TMA store per panel.  R < 8: half rows padded
+    // to 272 B, read back transposed, two half rows per store instruction.
+    constexpr bool kTmaStore = R >= 8;
+    uint8_t* stage = base + kOffStage + quarter * 8192;
+    uint8_t* srow = base + kOffStage + row * kStageRow;
+    uint8_t* swarp = base + kOffStage + (quarter * 32) * kStageRow;
     for (int64_t n = 0;; ++n) {
       if (!Wuse(BAR_D_FULL, kDescRing, n)) break;
       const ChunkDesc& d = desc[n % kDescRing];
@@ -459,15 +508,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (!Wuse(BAR_O_FULL, 2, n)) break;
       if (!Wuse(BAR_P_FULL, kQRing, n)) break;   // acquire the softmax's (m, l)
       tc_fence_after();
+      const float2 ml0 = ml_s[(ob * 2) * 128 + row];
+      const float2 ml1 = ml_s[(ob * 2 + 1) * 128 + row];
+      mbar_arrive(bar + BAR_ML_EMPTY + ob);      // (m, l) slot ob is free
       const int hr = row % R;
       const int64_t qi = (int64_t)(e >> 4);
       const bool valid = (e >= 0) && (qi < a.n_q) && (a.q_pos0 + qi >= (int64_t)c * kBlock);
       // piece row of (b, qi, g, slot, hr): the R head rows of one entry are adjacent
       const int64_t pidx =
           valid ? ((((int64_t)b * a.n_q + qi) * a.G + g) * kTopK + (e & 15)) * R + hr : 0;
-      if (valid) *reinterpret_cast<float2*>(a.part_ml + pidx * 2) = ml_s[ob * 128 + row];
-      uint8_t* srow = base + kOffStage + row * kStageRow;
-      uint8_t* swarp = base + kOffStage + (quarter * 32) * kStageRow;
+      if (valid)
+        *reinterpret_cast<float2*>(a.part_ml + pidx * 2) = make_float2(ml0.x, ml0.y + ml1.y);
       const uint32_t o_addr = tmem + lane_base + 256 + ob * 128;
       float* acc = a.part_acc + pidx * kHeadDim;
 #pragma unroll 1
@@ -478,30 +529,54 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         tmem_ld_wait();
         if (half == 1) {
           tc_fence_before();
-          mbar_arrive(bar + BAR_O_EMPTY + ob);
+          mbar_arrive(bar + BAR_O_EMPTY + ob);   // O buffer ob is free
         }
+        if constexpr (kTmaStore) {
+          bulk_wait_read();                      // the previous stores have read the panels
+          __syncwarp();
+          const int sw = lane & 7;
 #pragma unroll
-        for (int x = 0; x < 8; ++x) {
-          *reinterpret_cast<uint4*>(srow + x * 16) =
-              make_uint4(r0[4 * x], r0[4 * x + 1], r0[4 * x + 2], r0[4 * x + 3]);
-          *reinterpret_cast<uint4*>(srow + 128 + x * 16) =
-              make_uint4(r1[4 * x], r1[4 * x + 1], r1[4 * x + 2], r1[4 * x + 3]);
-        }
-        __syncwarp();
-        // two half rows per instruction: lanes 0-15 row 2i, lanes 16-31 row 2i+1
+          for (int j = 0; j < 8; ++j) {
+            *reinterpret_cast<uint4*>(stage + lane * 128 + ((j ^ sw) << 4)) =
+                make_uint4(r0[4 * j], r0[4 * j + 1], r0[4 * j + 2], r0[4 * j + 3]);
+            *reinterpret_cast<uint4*>(stage + 4096 + lane * 128 + ((j ^ sw) << 4)) =
+                make_uint4(r1[4 * j], r1[4 * j + 1], r1[4 * j + 2], r1[4 * j + 3]);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (valid && hr == 0) {                // first row of an entry: R rows per store
+            tma_store_2d(&tm_o, stage + lane * 128, half * 64, (int32_t)pidx);
+            tma_store_2d(&tm_o, stage + 4096 + lane * 128, half * 64 + 32, (int32_t)pidx);
+          }
+          bulk_commit();
+        } else {
+#pragma unroll
+          for (int x = 0; x < 8; ++x) {
+            *reinterpret_cast<uint4*>(srow + x * 16) =
+                make_uint4(r0[4 * x], r0[4 * x + 1], r0[4 * x + 2], r0[4 * x + 3]);
+            *reinterpret_cast<uint4*>(srow + 128 + x * 16) =
+                make_uint4(r1[4 * x], r1[4 * x + 1], r1[4 * x + 2], r1[4 * x + 3]);
+          }
+          __syncwarp();
+          // two half rows per instruction: lanes 0-15 row 2i, lanes 16-31 row 2i+1
 #pragma unroll 4
-        for (int i = 0; i < 16; ++i) {
-          const int rr = 2 * i + (lane >> 4);
-          const float* dst_row = (const float*)__shfl_sync(0xffffffffu, (unsigned long long)acc, rr);
-          const bool rv = __shfl_sync(0xffffffffu, valid ? 1 : 0, rr) != 0;
-          const uint4 v = *reinterpret_cast<const uint4*>(swarp + rr * kStageRow + (lane & 15) * 16);
-          if (rv)
-            *reinterpret_cast<uint4*>(const_cast<float*>(dst_row) + half * 64 + (lane & 15) * 4) = v;
+          for (int i = 0; i < 16; ++i) {
+            const int rr = 2 * i + (lane >> 4);
+            const float* dst_row =
+                (const float*)__shfl_sync(0xffffffffu, (unsigned long long)acc, rr);
+            const bool rv = __shfl_sync(0xffffffffu, valid ? 1 : 0, rr) != 0;
+            const uint4 v =
+                *reinterpret_cast<const uint4*>(swarp + rr * kStageRow + (lane & 15) * 16);
+            if (rv)
+              *reinterpret_cast<uint4*>(const_cast<float*>(dst_row) + half * 64 +
+                                        (lane & 15) * 4) = v;
+          }
+          __syncwarp();
         }
-        __syncwarp();
       }
       mbar_arrive(bar + BAR_D_EMPTY + (int)(n % kDescRing));
     }
+    if constexpr (kTmaStore) bulk_wait_all();    // every store has landed
   }
 
   tc_fence_before();
@@ -513,12 +588,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 }
 
 template <int R>
-static cudaError_t launch_attn_r(const CUtensorMap& tm_k, const CUtensorMap& tm_v, AttnArgs a,
-                                 cudaStream_t st) {
+static cudaError_t launch_attn_r(const CUtensorMap& tm_k, const CUtensorMap& tm_v,
+                                 const CUtensorMap& tm_o, AttnArgs a, cudaStream_t st) {
   constexpr int CH = 128 / R;
   auto k = sparse_attn_fwd_kernel<R>;
-  cudaError_t e =
-      cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kAttnSmemBytes);
+  // the register split above is only safe with exactly this many registers
+  // per thread at launch
+  cudaFuncAttributes fa;
+  cudaError_t e = cudaFuncGetAttributes(&fa, k);
+  if (e != cudaSuccess) return e;
+  if (fa.numRegs != kAttnRegsAtLaunch) return cudaErrorInvalidConfiguration;
+  e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kAttnSmemBytes);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess)
@@ -532,11 +612,12 @@ static cudaError_t launch_attn_r(const CUtensorMap& tm_k, const CUtensorMap& tm_
   a.n_items = (a.n_entries + W - 1) / W;
   if (a.n_items == 0) return cudaSuccess;
   const int64_t grid = min64(a.n_items, sms);
-  k<<<(unsigned)grid, kAttnThreads, kAttnSmemBytes, st>>>(tm_k, tm_v, a);
+  k<<<(unsigned)grid, kAttnThreads, kAttnSmemBytes, st>>>(tm_k, tm_v, tm_o, a);
   return cudaGetLastError();
 }
 
-cudaError_t launch_sparse_attn(const CUtensorMap& tm_k, const CUtensorMap& tm_v, const void* q,
+cudaError_t launch_sparse_attn(const CUtensorMap& tm_k, const CUtensorMap& tm_v,
+                               const CUtensorMap& tm_o, const void* q,
                                int64_t qs_b, int64_t qs_t, int64_t qs_h,
                                const int32_t* blk_offsets, const int32_t* entries,
                                int64_t n_seg, int64_t n_entries, int64_t n_q, int64_t q_pos0,
@@ -563,11 +644,11 @@ cudaError_t launch_sparse_attn(const CUtensorMap& tm_k, const CUtensorMap& tm_v,
   a.part_acc = part_acc;
   a.err = err;
   switch (H / G) {
-    case 1: return launch_attn_r<1>(tm_k, tm_v, a, st);
-    case 2: return launch_attn_r<2>(tm_k, tm_v, a, st);
-    case 4: return launch_attn_r<4>(tm_k, tm_v, a, st);
-    case 8: return launch_attn_r<8>(tm_k, tm_v, a, st);
-    case 16: return launch_attn_r<16>(tm_k, tm_v, a, st);
+    case 1: return launch_attn_r<1>(tm_k, tm_v, tm_o, a, st);
+    case 2: return launch_attn_r<2>(tm_k, tm_v, tm_o, a, st);
+    case 4: return launch_attn_r<4>(tm_k, tm_v, tm_o, a, st);
+    case 8: return launch_attn_r<8>(tm_k, tm_v, tm_o, a, st);
+    case 16: return launch_attn_r<16>(tm_k, tm_v, tm_o, a, st);
     default: return cudaErrorInvalidValue;
   }
 }
