@@ -22,7 +22,7 @@ size_t block_lists_workspace(int64_t, int64_t, int64_t);
 cudaError_t launch_block_lists(const int32_t*, int64_t, int64_t, int64_t, int64_t, int32_t*,
                                int32_t*, int64_t, void*, int32_t*, cudaStream_t);
 cudaError_t launch_sparse_attn(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
-                               const void*, int64_t,
+                               const CUtensorMap&, const void*, int64_t,
                                int64_t, int64_t, const int32_t*, const int32_t*, int64_t,
                                int64_t, int64_t, int64_t, int32_t, int32_t, int32_t, float,
                                float*, float*, int32_t*, cudaStream_t);
@@ -240,16 +240,21 @@ msa_status msa_sparse_attn_fwd(const msa_dims* d, msa_tensor q, msa_tensor k, ms
     return s;
   // part_acc [B, n_q, G, 16, R, 128] fp32 as rows of 128 floats; for R >= 8 one
   // entry's R rows are written by TMA stores of R x 32 floats
-  CUtensorMap to;
+  CUtensorMap to, tq;
   std::memset(&to, 0, sizeof(to));
+  std::memset(&tq, 0, sizeof(tq));
   const int64_t R = d->h_q / d->h_kv;
   if (R >= 8) {
+    // q [B, n_q, H, 128]: dims {128, H, n_q, B}, box {64, R, 1, 1} (one entry's heads)
+    if ((s = make_map(&tq, q.ptr, MSA_HEAD_DIM, d->h_q, d->n_q, d->batch, q.s_head, q.s_tok,
+                      q.s_batch, (uint32_t)R, 1)) != MSA_OK)
+      return s;
     const int64_t rows = d->batch * d->n_q * d->h_kv * MSA_TOPK_BLOCKS * R;
     if (rows >= (int64_t(1) << 31)) return MSA_ERR_UNSUPPORTED;
     if ((s = make_map_rows_f32(&to, part_acc, (uint64_t)rows, (uint32_t)R)) != MSA_OK) return s;
   }
   return from_cuda(msa::launch_sparse_attn(
-      tk, tv, to, q.ptr, q.s_batch, q.s_tok, q.s_head, blk_offsets, entries, n_seg, total, d->n_q,
+      tq, tk, tv, to, q.ptr, q.s_batch, q.s_tok, q.s_head, blk_offsets, entries, n_seg, total, d->n_q,
       d->q_pos0, d->h_kv, d->h_q, (int32_t)nblk, d->scale, part_ml, part_acc, dev_err,
       reinterpret_cast<cudaStream_t>(stream)));
 }

@@ -26,7 +26,10 @@
 //                             loaded as soon as the last S MMA of the current
 //                             one is done, V as soon as its last P V is done
 //   warp 3      idle (fills the control warpgroup)
-//   warps 4-7   gather:       cp.async of the chunk's Q rows into a 3-deep ring
+//   warps 4-7   gather:       the chunk's Q rows into a 3-deep ring: for R >= 8
+//                             one TMA box per entry and 64-column panel
+//                             (an entry's R head rows are contiguous),
+//                             otherwise 16-byte cp.async
 //   warps 8-15  softmax:      two warpgroups, one per half of the keys; each
 //                             holds its 64 S values of a row in registers,
 //                             the halves exchange row maxima through shared
@@ -125,11 +128,14 @@ __device__ __forceinline__ int64_t warp_find_segment(const int32_t* off, int64_t
 
 template <int R>
 __global__ void __launch_bounds__(kAttnThreads, 1)
-    sparse_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_k,
+    sparse_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
+                           const __grid_constant__ CUtensorMap tm_k,
                            const __grid_constant__ CUtensorMap tm_v,
                            const __grid_constant__ CUtensorMap tm_o,
                            const __grid_constant__ AttnArgs a) {
   constexpr int CH = 128 / R;
+  // R >= 8: an entry's R head rows (R x 256 contiguous bytes) arrive by TMA
+  constexpr bool kTmaGather = R >= 8;
   constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128, 0);
   constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 128, 1);
 
@@ -150,7 +156,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     mbar_init(bar + BAR_V_FULL, 1);
     mbar_init(bar + BAR_V_EMPTY, 1);
     for (int i = 0; i < kQRing; ++i) {
-      mbar_init(bar + BAR_Q_FULL + i, 128);
+      mbar_init(bar + BAR_Q_FULL + i, kTmaGather ? 4 : 128);
       mbar_init(bar + BAR_QP_EMPTY + i, 1);
       mbar_init(bar + BAR_P_FULL + i, 256);
     }
@@ -167,6 +173,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     *abort_flag = 0;
     fence_mbarrier_init();
   }
+  // Q tiles start zeroed: rows that no entry fills keep finite old data
+  for (int i = tid; i < kQRing * 32768 / 16; i += kAttnThreads)
+    reinterpret_cast<uint4*>(base + kOffQP)[i] = make_uint4(0, 0, 0, 0);
+  fence_proxy_async_smem();
   if (warp == 1) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
@@ -350,33 +360,68 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   } else if (warp < 8) {
     // ---------------- gather: Q rows of each chunk ----------------
     setmaxnreg_dec<kRegsGather>();
-    // thread = (row within an 8-row group, 16-byte column chunk); a warp
-    // instruction copies two whole 256-byte rows
-    const int gt = tid - 128;   // 0..127
-    const int ch = gt & 15;
-    for (int64_t n = 0;; ++n) {
-      if (!Wuse(BAR_D_FULL, kDescRing, n)) break;
-      const ChunkDesc& d = desc[n % kDescRing];
-      if (d.cnt < 0) break;
-      const int qb = (int)(n % kQRing);
-      const int32_t b = d.b, g = d.g;
-      if (!Wfree(BAR_QP_EMPTY, kQRing, n)) break;
-      uint8_t* sq = base + kOffQP + qb * 32768;
-      const __nv_bfloat16* qbase =
-          a.q + (int64_t)b * a.qs_b + (int64_t)(g * R) * a.qs_h + ch * 8;
-#pragma unroll 4
-      for (int it = 0; it < 16; ++it) {
-        const int row = it * 8 + (gt >> 4);
-        const int e = d.ent[row / R];
-        const int64_t qi = (int64_t)(e >> 4);
-        const bool ok = (e >= 0) && (qi < a.n_q);
-        const __nv_bfloat16* src = ok ? qbase + qi * a.qs_t + (int64_t)(row % R) * a.qs_h : a.q;
-        uint8_t* dst = sq + (ch >> 3) * 16384 + row * 128 + (((ch & 7) ^ (row & 7)) << 4);
-        cp_async_16(dst, src, ok ? 16u : 0u);
+    if constexpr (kTmaGather) {
+      // lane 0 of gather warp w loads entries w, w+4, ...: one TMA box of R
+      // rows x 64 columns per 128-byte panel, completing on Q_FULL
+      const int wq = warp - 4;
+      for (int64_t n = 0;; ++n) {
+        if (!Wuse(BAR_D_FULL, kDescRing, n)) break;
+        const ChunkDesc& d = desc[n % kDescRing];
+        if (d.cnt < 0) break;
+        const int qb = (int)(n % kQRing);
+        int ok = 1;
+        if (lane == 0) {
+          if (!Wfree(BAR_QP_EMPTY, kQRing, n)) {
+            ok = 0;
+          } else {
+            uint8_t* sq = base + kOffQP + qb * 32768;
+            uint32_t bytes = 0;
+            for (int k = wq; k < CH; k += 4) {
+              const int e = d.ent[k];
+              if (e >= 0 && (int64_t)(e >> 4) < a.n_q) bytes += R * 256;
+            }
+            mbar_arrive_expect_tx(bar + BAR_Q_FULL + qb, bytes);
+            for (int k = wq; k < CH; k += 4) {
+              const int e = d.ent[k];
+              if (e < 0 || (int64_t)(e >> 4) >= a.n_q) continue;
+              for (int p = 0; p < 2; ++p)
+                tma_load_4d(sq + p * 16384 + k * R * 128, &tm_q, bar + BAR_Q_FULL + qb, p * 64,
+                            d.g * R, e >> 4, d.b);
+            }
+          }
+        }
+        if (!__shfl_sync(0xffffffffu, ok, 0)) break;
       }
-      cp_async_wait_all();
-      fence_proxy_async_smem();
-      mbar_arrive(bar + BAR_Q_FULL + qb);
+    } else {
+      // thread = (row within an 8-row group, 16-byte column chunk); a warp
+      // instruction copies two whole 256-byte rows
+      const int gt = tid - 128;   // 0..127
+      const int ch = gt & 15;
+      for (int64_t n = 0;; ++n) {
+        if (!Wuse(BAR_D_FULL, kDescRing, n)) break;
+        const ChunkDesc& d = desc[n % kDescRing];
+        if (d.cnt < 0) break;
+        const int qb = (int)(n % kQRing);
+        const int32_t b = d.b, g = d.g;
+        if (!Wfree(BAR_QP_EMPTY, kQRing, n)) break;
+        uint8_t* sq = base + kOffQP + qb * 32768;
+        const __nv_bfloat16* qbase =
+            a.q + (int64_t)b * a.qs_b + (int64_t)(g * R) * a.qs_h + ch * 8;
+#pragma unroll 4
+        for (int it = 0; it < 16; ++it) {
+          const int row = it * 8 + (gt >> 4);
+          const int e = d.ent[row / R];
+          const int64_t qi = (int64_t)(e >> 4);
+          const bool ok = (e >= 0) && (qi < a.n_q);
+          const __nv_bfloat16* src =
+              ok ? qbase + qi * a.qs_t + (int64_t)(row % R) * a.qs_h : a.q;
+          uint8_t* dst = sq + (ch >> 3) * 16384 + row * 128 + (((ch & 7) ^ (row & 7)) << 4);
+          cp_async_16(dst, src, ok ? 16u : 0u);
+        }
+        cp_async_wait_all();
+        fence_proxy_async_smem();
+        mbar_arrive(bar + BAR_Q_FULL + qb);
+      }
     }
   } else if (warp < 16) {
     // ---------------- softmax: S -> P, (m, l) ----------------
@@ -588,8 +633,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 }
 
 template <int R>
-static cudaError_t launch_attn_r(const CUtensorMap& tm_k, const CUtensorMap& tm_v,
-                                 const CUtensorMap& tm_o, AttnArgs a, cudaStream_t st) {
+static cudaError_t launch_attn_r(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
+                                 const CUtensorMap& tm_v, const CUtensorMap& tm_o, AttnArgs a,
+                                 cudaStream_t st) {
   constexpr int CH = 128 / R;
   auto k = sparse_attn_fwd_kernel<R>;
   // the register split above is only safe with exactly this many registers
@@ -612,12 +658,12 @@ static cudaError_t launch_attn_r(const CUtensorMap& tm_k, const CUtensorMap& tm_
   a.n_items = (a.n_entries + W - 1) / W;
   if (a.n_items == 0) return cudaSuccess;
   const int64_t grid = min64(a.n_items, sms);
-  k<<<(unsigned)grid, kAttnThreads, kAttnSmemBytes, st>>>(tm_k, tm_v, tm_o, a);
+  k<<<(unsigned)grid, kAttnThreads, kAttnSmemBytes, st>>>(tm_q, tm_k, tm_v, tm_o, a);
   return cudaGetLastError();
 }
 
-cudaError_t launch_sparse_attn(const CUtensorMap& tm_k, const CUtensorMap& tm_v,
-                               const CUtensorMap& tm_o, const void* q,
+cudaError_t launch_sparse_attn(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
+                               const CUtensorMap& tm_v, const CUtensorMap& tm_o, const void* q,
                                int64_t qs_b, int64_t qs_t, int64_t qs_h,
                                const int32_t* blk_offsets, const int32_t* entries,
                                int64_t n_seg, int64_t n_entries, int64_t n_q, int64_t q_pos0,
@@ -644,11 +690,11 @@ cudaError_t launch_sparse_attn(const CUtensorMap& tm_k, const CUtensorMap& tm_v,
   a.part_acc = part_acc;
   a.err = err;
   switch (H / G) {
-    case 1: return launch_attn_r<1>(tm_k, tm_v, tm_o, a, st);
-    case 2: return launch_attn_r<2>(tm_k, tm_v, tm_o, a, st);
-    case 4: return launch_attn_r<4>(tm_k, tm_v, tm_o, a, st);
-    case 8: return launch_attn_r<8>(tm_k, tm_v, tm_o, a, st);
-    case 16: return launch_attn_r<16>(tm_k, tm_v, tm_o, a, st);
+    case 1: return launch_attn_r<1>(tm_q, tm_k, tm_v, tm_o, a, st);
+    case 2: return launch_attn_r<2>(tm_q, tm_k, tm_v, tm_o, a, st);
+    case 4: return launch_attn_r<4>(tm_q, tm_k, tm_v, tm_o, a, st);
+    case 8: return launch_attn_r<8>(tm_q, tm_k, tm_v, tm_o, a, st);
+    case 16: return launch_attn_r<16>(tm_q, tm_k, tm_v, tm_o, a, st);
     default: return cudaErrorInvalidValue;
   }
 }
