@@ -15,8 +15,9 @@
 //      maximum is a lower bound for the 15th-best score (15 distinct
 //      candidates reach it), and so is the current 15th-best of the row;
 //   2. the candidates at or above the larger of the two bounds (usually a few
-//      dozen) join the current best 15 in a 64-slot shared buffer, which a
-//      warp bitonic network sorts; its first 15 entries are the new best 15.
+//      dozen) are compacted by a warp prefix sum into a shared buffer next to
+//      the current best 15 and sorted by a warp bitonic network (one key per
+//      lane when they fit in 32, else two); the first 15 are the new best.
 // If more than 64 keys pass the bound (many equal scores), the row falls back
 // to an exact radix select over the whole row (4 passes of 8 bits with
 // warp-aggregated shared histograms).  Both give the same set.
@@ -116,11 +117,10 @@ __device__ __forceinline__ void bitonic64_desc(uint64_t& a, uint64_t& b, int lan
   for (int k = 2; k <= 64; k <<= 1) {
 #pragma unroll
     for (int j = k >> 1; j > 0; j >>= 1) {
-      if (j == 32) {                        // partners within the lane
-        const bool desc = true;             // only in the last stage (k = 64)
+      if (j == 32) {                        // partners within the lane (last stage only)
         const uint64_t hi = a > b ? a : b, lo = a > b ? b : a;
-        a = desc ? hi : lo;
-        b = desc ? lo : hi;
+        a = hi;
+        b = lo;
       } else {
         const uint64_t oa = shfl_xor_u64(a, j), ob = shfl_xor_u64(b, j);
         const bool lower = (lane & j) == 0;
@@ -131,6 +131,20 @@ __device__ __forceinline__ void bitonic64_desc(uint64_t& a, uint64_t& b, int lan
       }
     }
   }
+}
+
+// Sorts one 64-bit key per lane descending over the warp.
+__device__ __forceinline__ uint64_t bitonic32_desc(uint64_t a, int lane) {
+#pragma unroll
+  for (int k = 2; k <= 32; k <<= 1) {
+#pragma unroll
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      const uint64_t o = shfl_xor_u64(a, j);
+      const bool keep_max = ((lane & j) == 0) == ((lane & k) == 0);
+      a = keep_max ? (a > o ? a : o) : (a < o ? a : o);
+    }
+  }
+  return a;
 }
 
 // Sorts one 32-bit value per lane ascending over lanes 0..15 (lanes 16..31
@@ -149,7 +163,7 @@ __device__ __forceinline__ int32_t bitonic16_asc(int32_t v, int lane) {
   return v;
 }
 
-__global__ void __launch_bounds__(kTopkWarps * 32)
+__global__ void __launch_bounds__(kTopkWarps * 32, 3)
     topk_blocks_kernel(const float* __restrict__ pooled, int64_t stride, int64_t n_rows,
                        int64_t n_q, int64_t q_pos0, int32_t* __restrict__ sel) {
   __shared__ uint32_t hist_all[kTopkWarps][256];
@@ -157,7 +171,6 @@ __global__ void __launch_bounds__(kTopkWarps * 32)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   uint32_t* hist = hist_all[warp];
   uint64_t* cand = cand_all[warp];
-  const uint32_t lt_mask = (1u << lane) - 1u;
 
   for (int64_t r = (int64_t)blockIdx.x * kTopkWarps + warp; r < n_rows;
        r += (int64_t)gridDim.x * kTopkWarps) {
@@ -170,57 +183,80 @@ __global__ void __launch_bounds__(kTopkWarps * 32)
     }
     const float* row = pooled + r * stride;
     const int n = (int)own;
+    {
+      // pull the warp's next row toward L2 while this one is processed (one
+      // 128-byte line per lane covers rows of up to 1024 candidates)
+      const int64_t rn = r + (int64_t)gridDim.x * kTopkWarps;
+      if (rn < n_rows && lane * 32 < n)
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(pooled + rn * stride + lane * 32));
+    }
 
-    // best 15 so far, descending, in lanes 0..14 (0 = empty)
+    // best 15 so far, descending, in lanes 0..14 (0 = empty, below every key)
     uint64_t best = 0;
     bool overflow = false;
     for (int c0 = 0; c0 < n; c0 += 1024) {
-      uint32_t u[32];
-      uint32_t lmax = 0;
+      float v[32];
+      float lmax = -INFINITY;
 #pragma unroll
       for (int s = 0; s < 32; ++s) {
         const int i = c0 + s * 32 + lane;
-        u[s] = (i < n) ? order_key(__ldg(row + i)) : 0u;
-        lmax = max(lmax, u[s]);
+        v[s] = (i < n) ? __ldg(row + i) : -INFINITY;
+        lmax = fmaxf(lmax, v[s]);
       }
-      // 15th largest lane maximum: sort the 32 maxima descending (score bits)
-      int32_t sm = (int32_t)(lmax ^ 0x80000000u);   // signed order = unsigned order
+      // 15th largest lane maximum: bitonic sort of the 32 maxima, descending
+      float sm = lmax;
 #pragma unroll
       for (int k = 2; k <= 32; k <<= 1) {
 #pragma unroll
         for (int j = k >> 1; j > 0; j >>= 1) {
-          const int32_t o = __shfl_xor_sync(0xffffffffu, sm, j);
-          const bool lower = (lane & j) == 0;
-          const bool desc = (lane & k) == 0;
-          sm = (lower == desc) ? max(sm, o) : min(sm, o);
+          const float o = __shfl_xor_sync(0xffffffffu, sm, j);
+          const bool keep_max = ((lane & j) == 0) == ((lane & k) == 0);
+          sm = keep_max ? fmaxf(sm, o) : fminf(sm, o);
         }
       }
-      const uint32_t t_chunk = (uint32_t)__shfl_sync(0xffffffffu, sm, 14) ^ 0x80000000u;
-      const uint32_t t_best = (uint32_t)(__shfl_sync(0xffffffffu, best, 14) >> 32);
-      const uint32_t T = max(t_chunk, t_best);
-      // candidates: score key >= T (ties at T included), plus the current best 15
+      float T = __shfl_sync(0xffffffffu, sm, 14);
+      if (c0 > 0) {
+        // the 15th best so far, back from its order-preserving key
+        const uint32_t kb = (uint32_t)(__shfl_sync(0xffffffffu, best, 14) >> 32);
+        const float tb = __uint_as_float((kb & 0x80000000u) ? (kb & 0x7FFFFFFFu) : ~kb);
+        T = fmaxf(T, tb);
+      }
+      // candidates: score >= T (ties at T included), compacted by a prefix sum
       int cnt = 0;
 #pragma unroll
-      for (int s = 0; s < 32; ++s) {
-        const int i = c0 + s * 32 + lane;
-        const bool take = (i < n) && (u[s] >= T);
-        const uint32_t m = __ballot_sync(0xffffffffu, take);
-        if (take && cnt + __popc(m & lt_mask) < 64 - (kTopK - 1))
-          cand[cnt + __popc(m & lt_mask)] =
-              ((uint64_t)u[s] << 32) | (uint32_t)(0xFFFFFFFFu - (uint32_t)i);
-        cnt += __popc(m);
+      for (int s = 0; s < 32; ++s) cnt += (c0 + s * 32 + lane < n && v[s] >= T) ? 1 : 0;
+      int incl = cnt;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
       }
-      if (cnt > 64 - (kTopK - 1)) {
+      const int total = __shfl_sync(0xffffffffu, incl, 31);
+      const int nbest = (c0 > 0) ? kTopK - 1 : 0;
+      if (total + nbest > 64) {
         overflow = true;
         break;
       }
+      int pos = incl - cnt;
+#pragma unroll
+      for (int s = 0; s < 32; ++s) {
+        const int i = c0 + s * 32 + lane;
+        if (i < n && v[s] >= T) {
+          cand[pos++] = ((uint64_t)order_key(v[s]) << 32) | (uint32_t)(0xFFFFFFFFu - (uint32_t)i);
+        }
+      }
+      if (lane < nbest) cand[total + lane] = best;
       __syncwarp();
-      if (lane < kTopK - 1) cand[cnt + lane] = best;
-      __syncwarp();
-      const int tot = cnt + kTopK - 1;
-      uint64_t a = (lane < tot) ? cand[lane] : 0, b = (lane + 32 < tot) ? cand[lane + 32] : 0;
-      bitonic64_desc(a, b, lane);
-      best = (lane < kTopK - 1) ? a : 0;
+      const int m = total + nbest;
+      if (m <= 32) {
+        uint64_t k1 = (lane < m) ? cand[lane] : 0;
+        k1 = bitonic32_desc(k1, lane);
+        best = (lane < kTopK - 1) ? k1 : 0;
+      } else {
+        uint64_t a = (lane < m) ? cand[lane] : 0, b = (lane + 32 < m) ? cand[lane + 32] : 0;
+        bitonic64_desc(a, b, lane);
+        best = (lane < kTopK - 1) ? a : 0;
+      }
       __syncwarp();
     }
     if (overflow) {

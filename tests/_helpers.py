@@ -21,9 +21,11 @@ POOLED_REL = 1e-5
 NEAR_TIE_REL = 1e-5
 OUT_MAX_ABS = 2e-2
 OUT_MEAN_ABS = 2e-3
-# The kernel rounds each softmax weight to bf16 before it enters both P.V and the
-# normaliser l, so l may differ from the exact sum by the bf16 unit roundoff 2^-8
-# in relative terms: |lse_gpu - lse| <= log(1 + 2^-8) < 4e-3 (plus fp32 rounding).
+# The kernel sums the fp32 softmax weights into l and rounds them to bf16 only for
+# the P.V product; l may still differ from the exact sum by the rounding of the
+# bf16 logits' fp32 accumulation and of ex2.approx, far below the bf16 unit
+# roundoff 2^-8 of a weight.  The bound log(1 + 2^-8) < 4e-3 covers even a
+# normaliser built from bf16-rounded weights.
 LSE_MAX_ABS = 4e-3
 BLOCK = 128
 
