@@ -9,7 +9,8 @@
 // Segments are (batch, group, block) in that order; inside a segment the
 // entries (i << 4 | slot) are ascending in the query index i.  Steps:
 //   1. count:   per 128-query tile, a shared-memory histogram over blocks;
-//   2. colscan: per block, exclusive prefix over tiles (in place) + totals;
+//   2. colscan: per block, exclusive prefix over tiles (in place) + totals
+//      (coalesced two-pass form for many tiles, one thread per column else);
 //   3. offsets: exclusive scan of the totals over all segments (chunk sums,
 //      scan of the chunk sums, chunk-local scans);
 //   4. scatter: per tile, queries in ascending order claim consecutive slots
@@ -49,9 +50,10 @@ __global__ void __launch_bounds__(256)
   for (int c = threadIdx.x; c < nblk; c += blockDim.x) dst[c] = hist[c];
 }
 
+// Column scan for few tiles (decode): one thread per (segment), walking its tiles.
 __global__ void __launch_bounds__(256)
-    csr_colscan_kernel(int32_t* __restrict__ tile_counts, int32_t* __restrict__ totals,
-                       int32_t nblk, int32_t ntiles) {
+    csr_colscan_small_kernel(int32_t* __restrict__ tile_counts, int32_t* __restrict__ totals,
+                             int32_t nblk, int32_t ntiles) {
   const int c = blockIdx.x * blockDim.x + threadIdx.x;
   const int64_t bg = blockIdx.y;
   if (c >= nblk) return;
@@ -63,6 +65,46 @@ __global__ void __launch_bounds__(256)
     run += v;
   }
   totals[bg * nblk + c] = run;
+}
+
+// Column scan, coalesced: a block takes 32 adjacent blocks (one per lane) of
+// one (batch, group) and its 8 warps split the query tiles; each warp sums its
+// tiles, the warps' partial sums give each warp its starting prefix, and a
+// second pass writes the exclusive prefixes in place.
+constexpr int kColWarps = 8;
+
+__global__ void __launch_bounds__(kColWarps * 32)
+    csr_colscan_kernel(int32_t* __restrict__ tile_counts, int32_t* __restrict__ totals,
+                       int32_t nblk, int32_t ntiles) {
+  __shared__ int32_t part[kColWarps][32];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int c = blockIdx.x * 32 + lane;
+  const int64_t bg = blockIdx.y;
+  int32_t* col = tile_counts + bg * ntiles * (int64_t)nblk + c;
+  const int per = (ntiles + kColWarps - 1) / kColWarps;
+  const int t0 = min(ntiles, w * per), t1 = min(ntiles, t0 + per);
+  int32_t s = 0;
+  if (c < nblk) {
+#pragma unroll 8
+    for (int t = t0; t < t1; ++t) s += col[(int64_t)t * nblk];
+  }
+  part[w][lane] = s;
+  __syncthreads();
+  int32_t run = 0, total = 0;
+#pragma unroll
+  for (int k = 0; k < kColWarps; ++k) {
+    run += (k < w) ? part[k][lane] : 0;
+    total += part[k][lane];
+  }
+  if (c < nblk) {
+#pragma unroll 8
+    for (int t = t0; t < t1; ++t) {
+      const int32_t v = col[(int64_t)t * nblk];
+      col[(int64_t)t * nblk] = run;
+      run += v;
+    }
+    if (w == 0) totals[bg * nblk + c] = total;
+  }
 }
 
 // Exclusive scan of the per-segment totals into offsets[0..n], in three
@@ -211,8 +253,15 @@ cudaError_t launch_block_lists(const int32_t* sel, int64_t bgcount, int64_t n_q,
   dim3 g1((unsigned)ntiles, (unsigned)bgcount);
   csr_count_kernel<<<g1, 256, hist_bytes, st>>>(sel, n_q, q_pos0, (int32_t)nblk,
                                                 (int32_t)ntiles, tile_counts, err);
-  dim3 g2((unsigned)((nblk + 255) / 256), (unsigned)bgcount);
-  csr_colscan_kernel<<<g2, 256, 0, st>>>(tile_counts, totals, (int32_t)nblk, (int32_t)ntiles);
+  if (ntiles < 4 * kColWarps) {
+    dim3 g2((unsigned)((nblk + 255) / 256), (unsigned)bgcount);
+    csr_colscan_small_kernel<<<g2, 256, 0, st>>>(tile_counts, totals, (int32_t)nblk,
+                                                 (int32_t)ntiles);
+  } else {
+    dim3 g2((unsigned)((nblk + 31) / 32), (unsigned)bgcount);
+    csr_colscan_kernel<<<g2, kColWarps * 32, 0, st>>>(tile_counts, totals, (int32_t)nblk,
+                                                      (int32_t)ntiles);
+  }
   const int64_t nseg = bgcount * nblk;
   const int64_t nchunks = (nseg + kScanChunk - 1) / kScanChunk;
   int32_t* chunk_sums = totals + nseg;

@@ -204,24 +204,6 @@ constexpr int kDecThreads = 32 * (1 + kDecConsumers);
 constexpr int kDecStageBytes = kBlock * 128 * 2;    // 128 keys x 128 dims bf16
 constexpr int kDecSmemBytes = 1024 + kDecStages * kDecStageBytes + 2 * kDecStages * 8 + 16;
 
-__device__ __forceinline__ void ldmatrix_x4(uint32_t addr, uint32_t& r0, uint32_t& r1,
-                                            uint32_t& r2, uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-               : "r"(addr)
-               : "memory");
-}
-
-__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint32_t a1,
-                                               uint32_t a2, uint32_t a3, uint32_t b0,
-                                               uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
-      "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
 __global__ void __launch_bounds__(kDecThreads, 1)
     index_score_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
                               const __nv_bfloat16* __restrict__ q_idx, int64_t qs_b,

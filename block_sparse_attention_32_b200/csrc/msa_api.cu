@@ -26,6 +26,10 @@ cudaError_t launch_sparse_attn(const CUtensorMap&, const CUtensorMap&, const CUt
                                int64_t, int64_t, const int32_t*, const int32_t*, int64_t,
                                int64_t, int64_t, int64_t, int32_t, int32_t, int32_t, float,
                                float*, float*, int32_t*, cudaStream_t);
+cudaError_t launch_sparse_attn_decode(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
+                                      const int32_t*, const int32_t*, int64_t, int64_t, int64_t,
+                                      int32_t, int32_t, int32_t, float, float*, float*, int32_t*,
+                                      cudaStream_t);
 cudaError_t launch_merge(const int32_t*, const float*, const float*, void*, float*, int64_t,
                          int64_t, int32_t, int32_t, cudaStream_t);
 }  // namespace msa
@@ -244,6 +248,17 @@ msa_status msa_sparse_attn_fwd(const msa_dims* d, msa_tensor q, msa_tensor k, ms
   std::memset(&to, 0, sizeof(to));
   std::memset(&tq, 0, sizeof(tq));
   const int64_t R = d->h_q / d->h_kv;
+  if (d->n_q == 1 && R <= 8) {
+    // one query per sequence: warp-level tiles, heads as the 8-wide side.
+    // q [B, 1, H, 128]: dims {128, H, 1, B}, box {64, R, 1, 1} (the query's heads of a group)
+    if ((s = make_map(&tq, q.ptr, MSA_HEAD_DIM, d->h_q, d->n_q, d->batch, q.s_head, q.s_tok,
+                      q.s_batch, (uint32_t)R, 1)) != MSA_OK)
+      return s;
+    return from_cuda(msa::launch_sparse_attn_decode(
+        tq, tk, tv, blk_offsets, entries, d->batch * d->h_kv, d->n_q, d->q_pos0, d->h_kv,
+        d->h_q, (int32_t)nblk, d->scale, part_ml, part_acc, dev_err,
+        reinterpret_cast<cudaStream_t>(stream)));
+  }
   if (R >= 8) {
     // q [B, n_q, H, 128]: dims {128, H, n_q, B}, box {64, R, 1, 1} (one entry's heads)
     if ((s = make_map(&tq, q.ptr, MSA_HEAD_DIM, d->h_q, d->n_q, d->batch, q.s_head, q.s_tok,

@@ -30,6 +30,10 @@ CASES = [
     wl.small("decode_d64", 2, 1, 3000, 2999, 8, 2, 64, seed=17),
     wl.small("one_block", 1, 100, 100, 0, 4, 1, 64, seed=18),
     wl.small("sixteen_blocks", 1, 2048, 2048, 0, 8, 2, 128, seed=19),
+    # one query per sequence with R = 1, 16 (general kernel) and a context of 8 blocks
+    wl.small("decode_r1", 2, 1, 2200, 2199, 4, 4, 128, seed=20),
+    wl.small("decode_r16", 2, 1, 2500, 2499, 32, 2, 128, seed=21),
+    wl.small("decode_r8_short", 4, 1, 1000, 999, 16, 2, 128, seed=22),
 ]
 
 
