@@ -143,13 +143,21 @@ __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, u
       : "memory");
 }
 
-// TMA tile store shared -> global (no multicast), tracked per thread by bulk groups
-__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src, int32_t x,
-                                             int32_t y) {
+// L2 cache policy for bulk copies: lines a copy writes are evicted first
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+// TMA tile store shared -> global with an L2 cache policy (no multicast), tracked
+// per thread by bulk groups
+__device__ __forceinline__ void tma_store_2d_hint(const CUtensorMap* map, const void* src,
+                                                  int32_t x, int32_t y, uint64_t policy) {
   asm volatile(
-      "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
-          reinterpret_cast<uint64_t>(map)),
-      "r"(smem_u32(src)), "r"(x), "r"(y)
+      "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group.L2::cache_hint [%0, {%2, %3}], [%1], "
+      "%4;" ::"l"(reinterpret_cast<uint64_t>(map)),
+      "r"(smem_u32(src)), "r"(x), "r"(y), "l"(policy)
       : "memory");
 }
 

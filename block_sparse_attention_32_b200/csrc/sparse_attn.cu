@@ -540,6 +540,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     // entry's R rows with one TMA store per panel.  R < 8: half rows padded
     // to 272 B, read back transposed, two half rows per store instruction.
     constexpr bool kTmaStore = R >= 8;
+    // pieces are read back only by the merge kernel: keep them from displacing Q rows in L2
+    const uint64_t pol_st = l2_policy_evict_first();
     uint8_t* stage = base + kOffStage + quarter * 8192;
     uint8_t* srow = base + kOffStage + row * kStageRow;
     uint8_t* swarp = base + kOffStage + (quarter * 32) * kStageRow;
@@ -590,8 +592,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           fence_proxy_async_smem();
           __syncwarp();
           if (valid && hr == 0) {                // first row of an entry: R rows per store
-            tma_store_2d(&tm_o, stage + lane * 128, half * 64, (int32_t)pidx);
-            tma_store_2d(&tm_o, stage + 4096 + lane * 128, half * 64 + 32, (int32_t)pidx);
+            tma_store_2d_hint(&tm_o, stage + lane * 128, half * 64, (int32_t)pidx, pol_st);
+            tma_store_2d_hint(&tm_o, stage + 4096 + lane * 128, half * 64 + 32,
+                              (int32_t)pidx, pol_st);
           }
           bulk_commit();
         } else {

@@ -84,7 +84,11 @@ CONFIGS = {w.name: w for w in (TINY, P32, P128, DECODE, M1)}
 # counter capture.
 PROFILE_8K = Workload("profile_8k_r8", 1, 8192, 8192, 0, 32, 4, 128, seed=3, sink=True,
                       recency=True)
-ALL = dict(CONFIGS, **{PROFILE_8K.name: PROFILE_8K})
+# Profiling-sized decode: 4 sequences of the decode workload's shape (k_idx 268 MB,
+# K/V 4.3 GB), larger than L2.
+PROFILE_DECODE = Workload("profile_decode_b4", 4, 1, 262144, 262143, 64, 8, 128, seed=5,
+                          plants_per_group=2, plant_targets=1)
+ALL = dict(CONFIGS, **{PROFILE_8K.name: PROFILE_8K, PROFILE_DECODE.name: PROFILE_DECODE})
 
 
 def small(name, batch, n_q, n_kv, q_pos0, h_q, h_kv, d_idx, seed, **kw) -> Workload:
