@@ -16,7 +16,8 @@
 //   4. scatter: per tile, queries in ascending order claim consecutive slots
 //      of each block's range, so the order never depends on timing.
 // Workspace: tile histograms [B*G, ntiles, nblk] + totals [B*G*nblk] + chunk
-// sums [ceil(B*G*nblk / 4096)], int32.
+// sums [ceil(B*G*nblk / 4096)], int32.  One query per row (decode) takes a
+// two-launch path that needs only the per-row counts.
 #include "common.cuh"
 
 namespace msa {
@@ -226,6 +227,76 @@ __global__ void __launch_bounds__(32)
   }
 }
 
+// One query per (batch, group) row (decode).  Each segment then holds at most
+// one entry, and the lists follow from the rows directly: the offset of block
+// c in row r is (entries of the rows before r) + (selected blocks of r below
+// c), and each selected block gets its entry at that offset.  Two launches:
+// per-row counts, then one warp per row writes its offsets and entries.
+constexpr int kRowWarps = 8;
+
+__global__ void __launch_bounds__(kRowWarps * 32)
+    csr_rows_count_kernel(const int32_t* __restrict__ sel, int64_t n_rows, int64_t q_pos0,
+                          int32_t nblk, int32_t* __restrict__ counts, int32_t* err) {
+  const int lane = threadIdx.x & 31;
+  const int64_t r = (int64_t)blockIdx.x * kRowWarps + (threadIdx.x >> 5);
+  if (r >= n_rows) return;
+  const int64_t own = q_pos0 / kBlock;
+  const int32_t c = (lane < kTopK) ? sel[r * kTopK + lane] : -1;
+  const bool v = c >= 0 && c <= own && c < nblk;
+  if (c >= 0 && !v) report(err, MSA_DEVERR_BAD_BLOCK);
+  const int32_t cnt = __popc(__ballot_sync(0xffffffffu, v));
+  if (lane == 0) counts[r] = cnt;
+}
+
+__global__ void __launch_bounds__(kRowWarps * 32)
+    csr_rows_fill_kernel(const int32_t* __restrict__ sel, int64_t n_rows, int64_t q_pos0,
+                         int32_t nblk, const int32_t* __restrict__ counts,
+                         int32_t* __restrict__ offsets, int32_t* __restrict__ entries,
+                         int64_t cap) {
+  __shared__ int32_t part[kRowWarps * 32];
+  __shared__ int32_t row_base[kRowWarps + 1];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int64_t r0 = (int64_t)blockIdx.x * kRowWarps;
+  // entries of all rows before this block's first row
+  int32_t s = 0;
+  for (int64_t i = threadIdx.x; i < r0; i += blockDim.x) s += counts[i];
+  part[threadIdx.x] = s;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int32_t b = 0;
+    for (int i = 0; i < kRowWarps * 32; ++i) b += part[i];
+    for (int k = 0; k <= kRowWarps; ++k) {
+      row_base[k] = b;
+      if (r0 + k < n_rows) b += counts[r0 + k];
+    }
+  }
+  __syncthreads();
+  const int64_t r = r0 + w;
+  if (r >= n_rows) return;
+  const int64_t own = q_pos0 / kBlock;
+  const int32_t base = row_base[w];
+  const int32_t raw = (lane < kTopK) ? sel[r * kTopK + lane] : -1;
+  const int32_t mine = (raw >= 0 && raw <= own && raw < nblk) ? raw : 0x7FFFFFFF;
+  int32_t ck[kTopK];
+#pragma unroll
+  for (int k = 0; k < kTopK; ++k) ck[k] = __shfl_sync(0xffffffffu, mine, k);
+  int32_t* off = offsets + r * nblk;
+  for (int c = lane; c < nblk; c += 32) {
+    int32_t below = 0;
+#pragma unroll
+    for (int k = 0; k < kTopK; ++k) below += (ck[k] < c) ? 1 : 0;
+    off[c] = base + below;
+  }
+  if (lane < kTopK && mine != 0x7FFFFFFF) {
+    int32_t below = 0;
+#pragma unroll
+    for (int k = 0; k < kTopK; ++k) below += (ck[k] < mine) ? 1 : 0;
+    const int64_t p = (int64_t)base + below;
+    if (p < cap) entries[p] = lane;          // query 0 of the row, slot `lane`
+  }
+  if (r == n_rows - 1 && lane == 0) offsets[n_rows * nblk] = row_base[w + 1];
+}
+
 size_t block_lists_workspace(int64_t bgcount, int64_t n_q, int64_t nblk) {
   const int64_t ntiles = (n_q + kCsrTile - 1) / kCsrTile;
   const int64_t nseg = bgcount * nblk;
@@ -237,6 +308,15 @@ cudaError_t launch_block_lists(const int32_t* sel, int64_t bgcount, int64_t n_q,
                                int64_t q_pos0, int64_t nblk, int32_t* offsets,
                                int32_t* entries, int64_t cap, void* ws, int32_t* err,
                                cudaStream_t st) {
+  if (n_q == 1) {
+    int32_t* counts = reinterpret_cast<int32_t*>(ws);
+    const unsigned grid = (unsigned)((bgcount + kRowWarps - 1) / kRowWarps);
+    csr_rows_count_kernel<<<grid, kRowWarps * 32, 0, st>>>(sel, bgcount, q_pos0, (int32_t)nblk,
+                                                           counts, err);
+    csr_rows_fill_kernel<<<grid, kRowWarps * 32, 0, st>>>(sel, bgcount, q_pos0, (int32_t)nblk,
+                                                          counts, offsets, entries, cap);
+    return cudaGetLastError();
+  }
   const int64_t ntiles = (n_q + kCsrTile - 1) / kCsrTile;
   int32_t* tile_counts = reinterpret_cast<int32_t*>(ws);
   int32_t* totals = tile_counts + bgcount * ntiles * nblk;

@@ -17,7 +17,8 @@ import torch
 
 from . import capi
 
-# kernels each step launches (for launch accounting)
+# kernels each step launches (for launch accounting; with one query per row the
+# block lists take 2 launches instead of 6)
 LAUNCHES_PER_STEP = {"index": 1, "topk": 1, "block_lists": 6, "attn": 1, "merge": 1}
 
 
