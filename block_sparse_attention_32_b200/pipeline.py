@@ -93,6 +93,65 @@ def forward(buf: Buffers, q, k, v, q_idx, k_idx):
     return buf.out, buf.lse
 
 
+INPUT_NAMES = ("q", "k", "v", "q_idx", "k_idx")
+
+
+class HostPipeline:
+    """The hot path on batches held in pinned host memory, copies overlapped.
+
+    ``run(host_in, host_out)`` takes a list of host input dicts (pinned q, k,
+    v, q_idx, k_idx of the problem ``buf`` was allocated for) and a matching
+    list of pinned host (out, lse) pairs.  For every batch it enqueues the
+    host-to-device copy of the inputs (upload stream), the five library calls
+    (the caller's current stream) and the device-to-host copy of out and lse
+    (download stream).  Two device sets of inputs and outputs alternate, so
+    batch i+1's upload and batch i-1's download run while batch i's kernels
+    do; events order the three streams.  On return the caller's stream has
+    waited for every download.
+    """
+
+    def __init__(self, buf: Buffers, like: dict):
+        self.buf = buf
+        self.dev_in = [{k: torch.empty_like(like[k]) for k in INPUT_NAMES} for _ in range(2)]
+        self.dev_out = [(buf.out, buf.lse), (torch.empty_like(buf.out), torch.empty_like(buf.lse))]
+        self.s_up = torch.cuda.Stream()
+        self.s_down = torch.cuda.Stream()
+
+    def run(self, host_in, host_out):
+        comp = torch.cuda.current_stream()
+        n = len(host_in)
+        comp_done, down_done = [None] * n, [None] * n
+        try:
+            for i in range(n):
+                slot = i % 2
+                dev = self.dev_in[slot]
+                out, lse = self.dev_out[slot]
+                up = torch.cuda.Event()
+                with torch.cuda.stream(self.s_up):
+                    if i >= 2:                      # the kernels of batch i-2 read this set
+                        self.s_up.wait_event(comp_done[i - 2])
+                    for k in INPUT_NAMES:
+                        dev[k].copy_(host_in[i][k], non_blocking=True)
+                    up.record(self.s_up)
+                comp.wait_event(up)
+                if i >= 2:                          # batch i-2's output has left this set
+                    comp.wait_event(down_done[i - 2])
+                self.buf.out, self.buf.lse = out, lse
+                forward(self.buf, dev["q"], dev["k"], dev["v"], dev["q_idx"], dev["k_idx"])
+                comp_done[i] = torch.cuda.Event()
+                comp_done[i].record(comp)
+                down_done[i] = torch.cuda.Event()
+                with torch.cuda.stream(self.s_down):
+                    self.s_down.wait_event(comp_done[i])
+                    host_out[i][0].copy_(out, non_blocking=True)
+                    host_out[i][1].copy_(lse, non_blocking=True)
+                    down_done[i].record(self.s_down)
+            if n:
+                comp.wait_event(down_done[n - 1])
+        finally:
+            self.buf.out, self.buf.lse = self.dev_out[0]
+
+
 def check_device_errors(buf: Buffers):
     """Raise if any kernel reported a device-side error (synchronises)."""
     code = int(buf.dev_err[0].item())

@@ -242,3 +242,32 @@ def test_device_error_on_bad_selection():
     capi.msa_build_block_query_lists(d, buf.sel, buf.blk_offsets, buf.entries, buf.ws, buf.dev_err)
     torch.cuda.synchronize()
     assert int(buf.dev_err[0]) == capi.__dict__.get("MSA_DEVERR_BAD_BLOCK", 2)
+
+
+def test_host_pipeline_matches_device_runs():
+    """Overlapped upload / kernels / download over several host batches gives the
+    same bytes as running each batch on the device directly."""
+    _need_gpu()
+    import dataclasses
+    base = wl.small("host_batches", 1, 1500, 1500, 0, 16, 2, 128, seed=30)
+    ws = [dataclasses.replace(base, seed=30 + i) for i in range(3)]
+    d = pipeline.dims_for(base)
+    buf = pipeline.Buffers.allocate(d)
+    expect = []
+    dev_inputs = []
+    for w in ws:
+        inp = wl.make_inputs(w, "cuda")
+        dev_inputs.append(inp)
+        out, lse = pipeline.forward(buf, inp["q"], inp["k"], inp["v"], inp["q_idx"], inp["k_idx"])
+        expect.append((out.clone(), lse.clone()))
+    torch.cuda.synchronize()
+    host_in = [{k: v.cpu().pin_memory() for k, v in inp.items()} for inp in dev_inputs]
+    host_out = [(torch.empty(buf.out.shape, dtype=buf.out.dtype, pin_memory=True),
+                 torch.empty(buf.lse.shape, dtype=buf.lse.dtype, pin_memory=True)) for _ in ws]
+    runner = pipeline.HostPipeline(buf, dev_inputs[0])
+    runner.run(host_in, host_out)
+    torch.cuda.synchronize()
+    assert int(buf.dev_err[0]) == 0
+    for (o, l), (eo, el) in zip(host_out, expect):
+        assert torch.equal(o, eo.cpu())
+        assert torch.equal(l, el.cpu())
