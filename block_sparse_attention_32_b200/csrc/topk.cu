@@ -104,6 +104,12 @@ __device__ __noinline__ void select_row_radix(const float* __restrict__ row, int
   }
 }
 
+__device__ __forceinline__ uint64_t shfl_u64(uint64_t v, int src) {
+  const uint32_t lo = __shfl_sync(0xffffffffu, (uint32_t)v, src);
+  const uint32_t hi = __shfl_sync(0xffffffffu, (uint32_t)(v >> 32), src);
+  return ((uint64_t)hi << 32) | lo;
+}
+
 __device__ __forceinline__ uint64_t shfl_xor_u64(uint64_t v, int m) {
   const uint32_t lo = __shfl_xor_sync(0xffffffffu, (uint32_t)v, m);
   const uint32_t hi = __shfl_xor_sync(0xffffffffu, (uint32_t)(v >> 32), m);
@@ -237,23 +243,33 @@ __global__ void __launch_bounds__(kTopkWarps * 32, 3)
         overflow = true;
         break;
       }
+      // raw (score bits, block) pairs; the sort keys are formed after the compaction
+      uint2* raw = reinterpret_cast<uint2*>(cand);
       int pos = incl - cnt;
 #pragma unroll
       for (int s = 0; s < 32; ++s) {
         const int i = c0 + s * 32 + lane;
-        if (i < n && v[s] >= T) {
-          cand[pos++] = ((uint64_t)order_key(v[s]) << 32) | (uint32_t)(0xFFFFFFFFu - (uint32_t)i);
-        }
+        if (i < n && v[s] >= T) raw[pos++] = make_uint2(__float_as_uint(v[s]), (uint32_t)i);
       }
-      if (lane < nbest) cand[total + lane] = best;
       __syncwarp();
       const int m = total + nbest;
+      // key j of the merged list: compacted candidates first, then the best so far
+      // (the shuffle runs on every lane, whichever side its j falls on)
+      auto key_at = [&](int j) -> uint64_t {
+        const uint64_t bk = shfl_u64(best, (j - total) & 31);
+        if (j < total) {
+          const uint2 c = raw[j];
+          return ((uint64_t)order_key(__uint_as_float(c.x)) << 32) |
+                 (uint32_t)(0xFFFFFFFFu - c.y);
+        }
+        return (j < m) ? bk : 0;
+      };
       if (m <= 32) {
-        uint64_t k1 = (lane < m) ? cand[lane] : 0;
+        uint64_t k1 = key_at(lane);
         k1 = bitonic32_desc(k1, lane);
         best = (lane < kTopK - 1) ? k1 : 0;
       } else {
-        uint64_t a = (lane < m) ? cand[lane] : 0, b = (lane + 32 < m) ? cand[lane + 32] : 0;
+        uint64_t a = key_at(lane), b = key_at(lane + 32);
         bitonic64_desc(a, b, lane);
         best = (lane < kTopK - 1) ? a : 0;
       }

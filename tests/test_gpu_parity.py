@@ -34,6 +34,10 @@ CASES = [
     wl.small("decode_r1", 2, 1, 2200, 2199, 4, 4, 128, seed=20),
     wl.small("decode_r16", 2, 1, 2500, 2499, 32, 2, 128, seed=21),
     wl.small("decode_r8_short", 4, 1, 1000, 999, 16, 2, 128, seed=22),
+    # one query per sequence with a key head per group, and with 16 groups: the
+    # index branch falls back from the streaming scan to the tiled kernel
+    wl.small("decode_hk_per_group", 2, 1, 1900, 1899, 16, 4, 128, seed=23, h_kidx=4),
+    wl.small("decode_g16", 2, 1, 1700, 1699, 32, 16, 64, seed=24),
 ]
 
 
