@@ -17,7 +17,10 @@ Each function cites the page passage it follows in ``msa_oracle.c``:
   * ``merge`` -- log-sum-exp combination of per-block softmax pieces (the
     identity the KV-block-outer "Outer Gather Q" scheme relies on);
   * ``block_query_lists`` -- query->block lists inverted into block->query
-    lists ("Kernel 创新：Outer Gather Q" section).
+    lists ("Kernel 创新：Outer Gather Q" section);
+  * ``selection_recall`` -- the main branch's attention mass per block (the
+    teacher), the recall of the chosen blocks and the KL divergences to the
+    index branch's block softmax (section "索引分支训练：KL 对齐").
 
 Parity is pinned by ``tests/test_oracle_pins.py`` (brute force, closed forms,
 invariants and hand-derived fixtures under ``tests/golden/``).
@@ -67,9 +70,11 @@ def _load():
             lib.msa_oracle_attention.argtypes = [I64, I32, I32, I64, P, P, P, P, P, P, F64, P, P]
             lib.msa_oracle_merge.argtypes = [I64, I32, I32, P, P, P, P, P, P]
             lib.msa_oracle_block_query_lists.argtypes = [I64, I32, I64, I64, P, P, P]
+            lib.msa_oracle_selection_recall.argtypes = [I64, I32, I32, I32, I64, I32, P, P, P, P,
+                                                         P, P, P, F64, I64, P, P, P, P]
             for f in (lib.msa_oracle_index_pooled, lib.msa_oracle_topk, lib.msa_oracle_topk_f32,
                       lib.msa_oracle_attention, lib.msa_oracle_merge,
-                      lib.msa_oracle_block_query_lists):
+                      lib.msa_oracle_block_query_lists, lib.msa_oracle_selection_recall):
                 f.restype = None
             _lib = lib
     return _lib
@@ -203,3 +208,35 @@ def forward_rows(q_rows, q_idx_rows, row_pos, row_batch, k, v, k_idx, scale):
     sel = topk(pooled, row_pos)
     out, lse = attention(q_rows, row_pos, row_batch, k, v, sel, scale)
     return pooled, sel, out, lse
+
+
+def selection_recall(q_rows, q_idx_rows, row_pos, row_batch, k, k_idx, sel, scale, stride=None):
+    """Teacher block mass, recall and KL divergences for the given rows.
+
+    q_rows uint16 [n, H, 128]; q_idx_rows uint16 [n, G, d_idx]; k uint16
+    [B', G, n_kv, 128]; k_idx uint16 [B', h_kidx, n_kv, d_idx]; sel int32
+    [n, G, 16].  Returns (block_mass [n, G, stride], recall [n, G],
+    kl_pq [n, G], kl_qp [n, G]) in float64.
+    """
+    lib = _load()
+    q = _c(q_rows, np.uint16)
+    qi = _c(q_idx_rows, np.uint16)
+    kk = _c(k, np.uint16)
+    ki = _c(k_idx, np.uint16)
+    s = _c(sel, np.int32)
+    pos = _c(row_pos, np.int64)
+    bat = _c(row_batch, np.int64)
+    n, H, D = q.shape
+    _, G, d_idx = qi.shape
+    _, G2, n_kv, _ = kk.shape
+    h_kidx = ki.shape[1]
+    assert D == HEAD_DIM and G2 == G and s.shape == (n, G, TOPK)
+    stride = stride or num_blocks(n_kv)
+    mass = np.empty((n, G, stride), np.float64)
+    rec = np.empty((n, G), np.float64)
+    kpq = np.empty((n, G), np.float64)
+    kqp = np.empty((n, G), np.float64)
+    lib.msa_oracle_selection_recall(n, H, G, d_idx, n_kv, h_kidx, _p(q), _p(qi), _p(pos), _p(bat),
+                                    _p(kk), _p(ki), _p(s), float(scale), stride, _p(mass), _p(rec),
+                                    _p(kpq), _p(kqp))
+    return mass, rec, kpq, kqp

@@ -298,3 +298,100 @@ void msa_oracle_block_query_lists(int64_t B, int32_t G, int64_t n_q, int64_t nbl
       }
   free(cursor);
 }
+
+/* ---------------------------------------------------------------------- */
+/* Selection recall and the index branch's alignment target ([P1] section */
+/* "索引分支训练：KL 对齐": the index branch learns from the main branch's   */
+/* attention distribution through a KL divergence with the teacher's      */
+/* gradient stopped, and its chosen blocks are reported to hold over 90 % */
+/* of the main branch's attention weight; [P3] MSA entry: a KL loss       */
+/* aligns the index distribution to the main branch's probabilities).     */
+/* For row r (position t, own = t / 128) and group g, over blocks         */
+/* c = 0 .. own and keys j <= t:                                          */
+/*   teacher P(c) = (1/R) sum_{h in g} sum_{j in c} softmax_h(j), with    */
+/*                  softmax_h over all keys j <= t of scale * q_h . k_j   */
+/*   student Q(c) = softmax over c of z(c), z(c) = max_{j in c} of the    */
+/*                  index score q_idx[g] . k_idx[j] (own block: j <= t)   */
+/*   recall = sum of P(c) over the selected blocks                        */
+/*   kl_pq = sum_c P(c) log(P(c) / Q(c)), kl_qp = sum_c Q(c) log(Q(c)/P(c)) */
+/* block_mass[r,g,c] = P(c) for c <= own and 0 for own < c < stride.      */
+/* The teacher of a group is the mean over its R heads (the group shares  */
+/* one selection); the index logits are unscaled, as in step 1.           */
+/* ---------------------------------------------------------------------- */
+void msa_oracle_selection_recall(int64_t n_rows, int32_t H, int32_t G, int32_t d_idx,
+                                 int64_t n_kv, int32_t h_kidx,
+                                 const uint16_t* q_rows,     /* [n_rows,H,128] */
+                                 const uint16_t* q_idx_rows, /* [n_rows,G,d_idx] */
+                                 const int64_t* row_pos, const int64_t* row_batch,
+                                 const uint16_t* k,          /* [B',G,n_kv,128] */
+                                 const uint16_t* k_idx,      /* [B',h_kidx,n_kv,d_idx] */
+                                 const int32_t* sel,         /* [n_rows,G,16] */
+                                 double scale, int64_t stride,
+                                 double* block_mass,         /* [n_rows,G,stride] */
+                                 double* recall, double* kl_pq, double* kl_qp) /* [n_rows,G] */
+{
+  const int32_t R = H / G;
+#pragma omp parallel for collapse(2) schedule(dynamic, 1)
+  for (int64_t r = 0; r < n_rows; ++r) {
+    for (int32_t g = 0; g < G; ++g) {
+      const int64_t t = row_pos[r];
+      const int64_t own = t / MSA_BLOCK;
+      const int64_t nb = own + 1;
+      const int64_t kvbase = (row_batch[r] * G + g) * n_kv;
+      const int64_t kibase = (row_batch[r] * h_kidx + (h_kidx == 1 ? 0 : g)) * n_kv;
+      double* P = block_mass + (r * G + g) * stride;
+      double* z = (double*)malloc((size_t)nb * sizeof(double));
+      double* logit = (double*)malloc((size_t)(t + 1) * sizeof(double));
+      for (int64_t c = 0; c < stride; ++c) P[c] = 0.0;
+      /* teacher: each head's softmax over every key j <= t, summed per block */
+      for (int32_t hr = 0; hr < R; ++hr) {
+        const uint16_t* qh = q_rows + (r * H + g * R + hr) * (int64_t)MSA_HEAD_DIM;
+        double qd[MSA_HEAD_DIM];
+        for (int32_t d = 0; d < MSA_HEAD_DIM; ++d) qd[d] = bf16_to_f64(qh[d]);
+        double m = -INFINITY;
+        for (int64_t j = 0; j <= t; ++j) {
+          const uint16_t* kj = k + (kvbase + j) * MSA_HEAD_DIM;
+          double dot = 0.0;
+          for (int32_t d = 0; d < MSA_HEAD_DIM; ++d) dot += qd[d] * bf16_to_f64(kj[d]);
+          logit[j] = scale * dot;
+          if (logit[j] > m) m = logit[j];
+        }
+        double l = 0.0;
+        for (int64_t j = 0; j <= t; ++j) l += exp(logit[j] - m);
+        for (int64_t j = 0; j <= t; ++j) P[j / MSA_BLOCK] += exp(logit[j] - m) / l / R;
+      }
+      /* student: softmax of the block-max index scores */
+      const uint16_t* qi = q_idx_rows + (r * G + g) * (int64_t)d_idx;
+      double zmax = -INFINITY;
+      for (int64_t c = 0; c < nb; ++c) {
+        double best = -INFINITY;
+        for (int64_t j = c * MSA_BLOCK; j < (c + 1) * MSA_BLOCK && j <= t; ++j) {
+          const uint16_t* kj = k_idx + (kibase + j) * d_idx;
+          double dot = 0.0;
+          for (int32_t d = 0; d < d_idx; ++d) dot += bf16_to_f64(qi[d]) * bf16_to_f64(kj[d]);
+          if (dot > best) best = dot;
+        }
+        z[c] = best;
+        if (best > zmax) zmax = best;
+      }
+      double zs = 0.0;
+      for (int64_t c = 0; c < nb; ++c) zs += exp(z[c] - zmax);
+      double kpq = 0.0, kqp = 0.0;
+      for (int64_t c = 0; c < nb; ++c) {
+        const double logq = z[c] - zmax - log(zs);
+        const double q = exp(logq);
+        if (P[c] > 0.0) kpq += P[c] * (log(P[c]) - logq);
+        if (q > 0.0) kqp += q * (logq - log(P[c]));
+      }
+      double rc = 0.0;
+      const int32_t* srow = sel + (r * G + g) * MSA_TOPK;
+      for (int32_t s = 0; s < MSA_TOPK; ++s)
+        if (srow[s] >= 0 && srow[s] <= own) rc += P[srow[s]];
+      recall[r * G + g] = rc;
+      kl_pq[r * G + g] = kpq;
+      kl_qp[r * G + g] = kqp;
+      free(z);
+      free(logit);
+    }
+  }
+}

@@ -338,3 +338,112 @@ def test_cost_model_reproduces_the_pages_28x():
     full = R * d * (n / 2) * 4
     msa = R * d * 2048 * 4 + d_idx * (n / 2) * 2
     assert round(full / msa, 1) == 28.4
+
+
+# ----------------------------------------------------------------------------
+# selection recall and the KL alignment target ("MSA 稀疏注意力三国杀", section
+# "索引分支训练：KL 对齐": the main branch's attention distribution is the index
+# branch's teacher; the chosen blocks hold most of its weight)
+# ----------------------------------------------------------------------------
+def _recall_case(rng, n, rows, H=4, G=2, d_idx=64, k=None, k_idx=None):
+    q = _rand_bits(rng, (1, n, H, 128))
+    k = _rand_bits(rng, (1, G, n, 128)) if k is None else k
+    q_idx = _rand_bits(rng, (len(rows), G, d_idx))
+    k_idx = _rand_bits(rng, (1, 1, n, d_idx)) if k_idx is None else k_idx
+    return q[0, rows], q_idx, k, k_idx
+
+
+def test_recall_is_one_when_every_causal_block_is_selected():
+    """Within 16 blocks of context every causal block is selected: recall 1, and the
+    teacher's block masses sum to 1 for every group."""
+    rng = np.random.default_rng(40)
+    n = 1700
+    rows = np.array([0, 5, 127, 128, 900, 1699], np.int64)
+    q_rows, q_idx, k, k_idx = _recall_case(rng, n, rows)
+    pooled = oracle.index_pooled(q_idx, rows, np.zeros_like(rows), k_idx)
+    sel = oracle.topk(pooled, rows)
+    mass, rec, kpq, kqp = oracle.selection_recall(q_rows, q_idx, rows, np.zeros_like(rows), k, k_idx,
+                                                  sel, 1 / math.sqrt(128))
+    np.testing.assert_allclose(rec, 1.0, atol=1e-12)
+    np.testing.assert_allclose(mass.sum(axis=2), 1.0, atol=1e-12)
+    assert (kpq >= -1e-12).all() and (kqp >= -1e-12).all()
+
+
+def test_recall_equals_ratio_of_attention_normalisers():
+    """The mass of a block subset is exp(lse over the subset - lse over all causal
+    blocks), averaged over the group's heads -- two separate oracle routines agree."""
+    rng = np.random.default_rng(41)
+    n, H, G = 1900, 4, 2
+    rows = np.array([1500, 1899], np.int64)
+    q_rows, q_idx, k, k_idx = _recall_case(rng, n, rows, H=H, G=G)
+    v = _rand_bits(rng, (1, G, n, 128))
+    bats = np.zeros_like(rows)
+    own = rows // BLOCK
+    sel_all = np.full((len(rows), G, 16), -1, np.int32)
+    sel_sub = np.full((len(rows), G, 16), -1, np.int32)
+    for r in range(len(rows)):
+        for g in range(G):
+            sel_all[r, g, :own[r] + 1] = np.arange(own[r] + 1)
+            sub = sorted({0, 3, int(own[r]) - 2 - g, int(own[r])})
+            sel_sub[r, g, :len(sub)] = sub
+    _, lse_all = oracle.attention(q_rows, rows, bats, k, v, sel_all, 1 / math.sqrt(128))
+    _, lse_sub = oracle.attention(q_rows, rows, bats, k, v, sel_sub, 1 / math.sqrt(128))
+    _, rec, _, _ = oracle.selection_recall(q_rows, q_idx, rows, bats, k, k_idx, sel_sub,
+                                           1 / math.sqrt(128))
+    R = H // G
+    for r in range(len(rows)):
+        for g in range(G):
+            expect = np.mean(np.exp(lse_sub[r, g * R:(g + 1) * R] - lse_all[r, g * R:(g + 1) * R]))
+            assert abs(rec[r, g] - expect) < 1e-12
+
+
+def test_teacher_is_uniform_over_tokens_for_equal_keys():
+    """Equal keys give every causal token the same weight: block mass = tokens / (t+1)."""
+    rng = np.random.default_rng(42)
+    n = 1000
+    rows = np.array([700, 999], np.int64)
+    kvec = _rand_bits(rng, (128,))
+    k = np.broadcast_to(kvec, (1, 2, n, 128)).copy()
+    q_rows, q_idx, k, k_idx = _recall_case(rng, n, rows, k=k)
+    sel = np.full((len(rows), 2, 16), -1, np.int32)
+    sel[:, :, 0] = rows[:, None] // BLOCK
+    mass, rec, _, _ = oracle.selection_recall(q_rows, q_idx, rows, np.zeros_like(rows), k, k_idx,
+                                              sel, 1 / math.sqrt(128))
+    for r, t in enumerate(rows):
+        counts = np.bincount(np.arange(t + 1) // BLOCK, minlength=mass.shape[2]).astype(float)
+        np.testing.assert_allclose(mass[r], np.broadcast_to(counts / (t + 1), mass[r].shape),
+                                   atol=1e-12)
+        np.testing.assert_allclose(rec[r], (t % BLOCK + 1) / (t + 1), atol=1e-12)
+
+
+def test_kl_closed_forms():
+    """Full blocks, equal keys (teacher uniform over blocks): equal index keys give a
+    uniform student and zero divergence; two index-key values give the textbook KL
+    of (1/2, 1/2) against softmax(z0, z1)."""
+    rng = np.random.default_rng(43)
+    n = 256
+    rows = np.array([255], np.int64)                  # two full blocks
+    kvec = _rand_bits(rng, (128,))
+    k = np.broadcast_to(kvec, (1, 2, n, 128)).copy()
+    u = _rand_bits(rng, (64,))
+    w = _rand_bits(rng, (64,))
+    sel = np.full((1, 2, 16), -1, np.int32)
+    sel[0, :, :2] = [0, 1]
+    # equal index keys
+    k_idx = np.broadcast_to(u, (1, 1, n, 64)).copy()
+    q_rows, q_idx, k, k_idx = _recall_case(rng, n, rows, k=k, k_idx=k_idx)
+    _, _, kpq, kqp = oracle.selection_recall(q_rows, q_idx, rows, np.zeros_like(rows), k, k_idx,
+                                             sel, 1 / math.sqrt(128))
+    np.testing.assert_allclose(kpq, 0.0, atol=1e-12)
+    np.testing.assert_allclose(kqp, 0.0, atol=1e-12)
+    # block 0 keys u, block 1 keys w
+    k_idx2 = np.concatenate([np.broadcast_to(u, (128, 64)), np.broadcast_to(w, (128, 64))])[None, None]
+    _, _, kpq, kqp = oracle.selection_recall(q_rows, q_idx, rows, np.zeros_like(rows), k,
+                                             np.ascontiguousarray(k_idx2), sel, 1 / math.sqrt(128))
+    qf = oracle.bits_to_f64(q_idx)[0]                     # [G, 64]
+    uf, wf = oracle.bits_to_f64(u), oracle.bits_to_f64(w)
+    for g in range(2):
+        z = np.array([qf[g] @ uf, qf[g] @ wf])
+        qd = np.exp(z - z.max()) / np.exp(z - z.max()).sum()
+        assert abs(kpq[0, g] - np.sum(0.5 * np.log(0.5 / qd))) < 1e-12
+        assert abs(kqp[0, g] - np.sum(qd * np.log(qd / 0.5))) < 1e-12
