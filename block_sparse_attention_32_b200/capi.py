@@ -69,10 +69,15 @@ def load_library(path: str) -> ctypes.CDLL:
     L.msa_build_block_query_lists_noalloc.argtypes = [_PD, _P, _P, _P, _P, _P]
     L.msa_sparse_attn_fwd.argtypes = [_PD, Tensor, Tensor, Tensor, _P, _P, _P, _P, _P, _P]
     L.msa_merge_partials.argtypes = [_PD, _P, _P, _P, _P, _P, _P, _P]
+    L.msa_selection_recall_workspace.argtypes = [_PD, ctypes.c_int64]
+    L.msa_selection_recall_workspace.restype = ctypes.c_size_t
+    L.msa_selection_recall.argtypes = [_PD, Tensor, Tensor, Tensor, Tensor, _P, _P, ctypes.c_int64,
+                                       _P, ctypes.c_int64, _P, _P, _P, _P, ctypes.c_size_t, _P, _P]
     L.msa_status_string.argtypes = [ctypes.c_int]
     L.msa_status_string.restype = ctypes.c_char_p
     for f in (L.msa_index_score_maxpool, L.msa_topk_blocks, L.msa_build_block_query_lists,
-              L.msa_build_block_query_lists_noalloc, L.msa_sparse_attn_fwd, L.msa_merge_partials):
+              L.msa_build_block_query_lists_noalloc, L.msa_sparse_attn_fwd, L.msa_merge_partials,
+              L.msa_selection_recall):
         f.restype = ctypes.c_int
     return L
 
@@ -168,3 +173,20 @@ def msa_merge_partials(d: Dims, sel, part_ml, part_acc, out, lse, dev_err=None):
     _check("msa_merge_partials",
            lib().msa_merge_partials(ctypes.byref(d), _ptr(sel), _ptr(part_ml), _ptr(part_acc),
                                     _ptr(out), _ptr(lse), _ptr(dev_err), _stream()))
+
+
+def msa_selection_recall_workspace(d: Dims, n_rows: int) -> int:
+    return int(lib().msa_selection_recall_workspace(ctypes.byref(d), n_rows))
+
+
+def msa_selection_recall(d: Dims, q, k, q_idx, k_idx, sel, rows, block_mass, recall, kl_pq, kl_qp,
+                         ws, dev_err=None):
+    """Teacher block mass, recall and KL divergences for the sampled rows
+    (rows: int64 device tensor of b * n_q + qi; block_mass [n * G, >= nblk])."""
+    nbytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check("msa_selection_recall",
+           lib().msa_selection_recall(ctypes.byref(d), tensor_btd(q), tensor_bhtd(k),
+                                      tensor_btd(q_idx), tensor_bhtd(k_idx), _ptr(sel), _ptr(rows),
+                                      rows.numel(), _ptr(block_mass), block_mass.stride(0),
+                                      _ptr(recall), _ptr(kl_pq), _ptr(kl_qp), _ptr(ws), nbytes,
+                                      _ptr(dev_err), _stream()))

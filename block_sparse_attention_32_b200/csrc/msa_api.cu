@@ -30,6 +30,13 @@ cudaError_t launch_sparse_attn_decode(const CUtensorMap&, const CUtensorMap&, co
                                       const int32_t*, const int32_t*, int64_t, int64_t, int64_t,
                                       int32_t, int32_t, int32_t, float, float*, float*, int32_t*,
                                       cudaStream_t);
+size_t recall_workspace(int64_t, int32_t, int32_t, int32_t);
+cudaError_t launch_selection_recall(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
+                                    const int64_t*, int64_t, const void*, int64_t, int64_t,
+                                    int64_t, int64_t, int64_t, int64_t, int32_t, int32_t,
+                                    int32_t, int32_t, int32_t, float, const int32_t*, float*,
+                                    int64_t, float*, float*, float*, void*, int32_t*,
+                                    cudaStream_t);
 cudaError_t launch_merge(const int32_t*, const float*, const float*, void*, float*, int64_t,
                          int64_t, int32_t, int32_t, cudaStream_t);
 }  // namespace msa
@@ -288,6 +295,53 @@ msa_status msa_merge_partials(const msa_dims* d, const int32_t* sel, const float
   const int64_t n_rows = d->batch * d->n_q * d->h_q;
   return from_cuda(msa::launch_merge(sel, part_ml, part_acc, out, lse, n_rows, d->n_q, d->h_q,
                                      d->h_kv, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t msa_selection_recall_workspace(const msa_dims* d, int64_t n_rows) {
+  if (check_dims(d) != MSA_OK || n_rows < 0) return 0;
+  return msa::recall_workspace(n_rows, d->h_kv, d->h_q / d->h_kv, (int32_t)msa_num_blocks(d));
+}
+
+msa_status msa_selection_recall(const msa_dims* d, msa_tensor q, msa_tensor k, msa_tensor q_idx,
+                                msa_tensor k_idx, const int32_t* sel, const int64_t* rows,
+                                int64_t n_rows, float* block_mass, int64_t mass_stride,
+                                float* recall, float* kl_pq, float* kl_qp, void* ws,
+                                size_t ws_bytes, int32_t* dev_err, void* stream) {
+  msa_status s = check_dims(d);
+  if (s != MSA_OK) return s;
+  if ((s = check_tensor(q)) != MSA_OK) return s;
+  if ((s = check_tensor(k)) != MSA_OK) return s;
+  if ((s = check_tensor(q_idx)) != MSA_OK) return s;
+  if ((s = check_tensor(k_idx)) != MSA_OK) return s;
+  if (n_rows < 0) return MSA_ERR_INVALID_ARG;
+  if (n_rows == 0) return MSA_OK;
+  if (sel == nullptr || rows == nullptr || block_mass == nullptr || recall == nullptr ||
+      kl_pq == nullptr || kl_qp == nullptr || ws == nullptr)
+    return MSA_ERR_INVALID_ARG;
+  if (!aligned16(ws)) return MSA_ERR_ALIGNMENT;
+  const int64_t nblk = msa_num_blocks(d);
+  const int64_t R = d->h_q / d->h_kv;
+  if (R > 8) return MSA_ERR_UNSUPPORTED;            // heads are the 8-wide side of the tiles
+  if (mass_stride < nblk) return MSA_ERR_INVALID_ARG;
+  if (n_rows * d->h_kv > 0x7FFFFFFF) return MSA_ERR_UNSUPPORTED;
+  if (ws_bytes < msa_selection_recall_workspace(d, n_rows)) return MSA_ERR_WORKSPACE_TOO_SMALL;
+  CUtensorMap tq, tk, tki;
+  // q [B, n_q, H, 128]: box {64, R, 1, 1} (one query's heads of a group)
+  if ((s = make_map(&tq, q.ptr, MSA_HEAD_DIM, d->h_q, d->n_q, d->batch, q.s_head, q.s_tok,
+                    q.s_batch, (uint32_t)R, 1)) != MSA_OK)
+    return s;
+  // k [B, h_kv, n_kv, 128] and k_idx [B, h_kidx, n_kv, d_idx]: one 128-token block per box
+  if ((s = make_map(&tk, k.ptr, MSA_HEAD_DIM, d->n_kv, d->h_kv, d->batch, k.s_tok, k.s_head,
+                    k.s_batch, 128, 1)) != MSA_OK)
+    return s;
+  if ((s = make_map(&tki, k_idx.ptr, d->d_idx, d->n_kv, d->h_kidx, d->batch, k_idx.s_tok,
+                    k_idx.s_head, k_idx.s_batch, 128, 1)) != MSA_OK)
+    return s;
+  return from_cuda(msa::launch_selection_recall(
+      tq, tk, tki, rows, n_rows, q_idx.ptr, q_idx.s_batch, q_idx.s_tok, q_idx.s_head, d->batch,
+      d->n_q, d->q_pos0, d->h_kv, d->h_q, d->d_idx, d->h_kidx, (int32_t)nblk, d->scale, sel,
+      block_mass, mass_stride, recall, kl_pq, kl_qp, ws, dev_err,
+      reinterpret_cast<cudaStream_t>(stream)));
 }
 
 const char* msa_status_string(msa_status s) {

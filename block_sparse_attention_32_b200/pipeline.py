@@ -93,6 +93,24 @@ def forward(buf: Buffers, q, k, v, q_idx, k_idx):
     return buf.out, buf.lse
 
 
+def selection_recall(buf: Buffers, q, k, q_idx, k_idx, rows):
+    """For sampled rows (int64 device tensor of b * n_q + qi): the main branch's
+    block mass [n, G, nblk], the recall of buf.sel and KL(P||Q), KL(Q||P) [n, G]."""
+    d = buf.dims
+    n, G = rows.numel(), d.h_kv
+    nblk = capi.msa_num_blocks(d)
+    dev = rows.device
+    mass = torch.empty((n, G, nblk), dtype=torch.float32, device=dev)
+    rec = torch.empty((n, G), dtype=torch.float32, device=dev)
+    kpq = torch.empty((n, G), dtype=torch.float32, device=dev)
+    kqp = torch.empty((n, G), dtype=torch.float32, device=dev)
+    ws_bytes = capi.msa_selection_recall_workspace(d, n)
+    ws = torch.empty(((ws_bytes + 15) // 16 * 4,), dtype=torch.int32, device=dev)
+    capi.msa_selection_recall(d, q, k, q_idx, k_idx, buf.sel, rows, mass.view(n * G, nblk), rec,
+                              kpq, kqp, ws, buf.dev_err)
+    return mass, rec, kpq, kqp
+
+
 INPUT_NAMES = ("q", "k", "v", "q_idx", "k_idx")
 
 

@@ -186,8 +186,9 @@ MSA_API msa_status msa_build_block_query_lists_noalloc(const msa_dims* dims, con
  *                                       l = sum_j e^{scale q.k_j - m}
  *   part_acc[B, n_q, G, 16, R, 128] fp32: sum_j e^{scale q.k_j - m} v_j
  * (the R head rows of one (query, block) are adjacent, R = h_q / h_kv)
- * (the weights e^{...} are rounded to bf16 before they multiply V and before
- * they are summed into l, so acc / l is an exact convex combination).
+ * (l sums the fp32 weights e^{...}; they are rounded to bf16 only where they
+ * multiply V, as in standard flash attention).  With one query per sequence
+ * (n_q = 1) and R <= 8 the work runs on warp-level tiles instead; same output.
  *   q [B, n_q, h_q, 128] bf16; k, v [B, h_kv, n_kv, 128] bf16
  *   (msa_tensor strides; for k/v s_head is the stride between KV heads). */
 MSA_API msa_status msa_sparse_attn_fwd(const msa_dims* dims, msa_tensor q, msa_tensor k, msa_tensor v,
@@ -202,6 +203,32 @@ MSA_API msa_status msa_sparse_attn_fwd(const msa_dims* dims, msa_tensor q, msa_t
 MSA_API msa_status msa_merge_partials(const msa_dims* dims, const int32_t* sel,
                               const float* part_ml, const float* part_acc,
                               void* out, float* lse, int32_t* dev_err, void* stream);
+
+/* Selection recall and the index branch's alignment target, for sampled query
+ * rows ("MSA 稀疏注意力三国杀" page, section "索引分支训练：KL 对齐": the index
+ * branch learns the main branch's attention distribution through a KL
+ * divergence with the teacher's gradient stopped, and its chosen blocks hold
+ * most of the main branch's weight; "稀疏注意力速览" page, section 4, MSA entry).
+ * For sampled row rows[i] = b * n_q + qi (position t = q_pos0 + qi) and group
+ * g, over blocks c = 0 .. t / 128 and keys j <= t:
+ *   teacher P(c) = mean over the group's R heads of the full causal softmax
+ *                  mass of block c, softmax over all j <= t of scale * q.k_j
+ *   student Q(c) = softmax over c of z(c) = max_{j in c} q_idx[g] . k_idx[j]
+ *   recall = sum of P over the blocks sel[b, g, qi, :] selects
+ *   kl_pq = sum_c P log(P / Q), kl_qp = sum_c Q log(Q / P)
+ * Outputs (device, fp32): block_mass [n_rows, G, mass_stride] (P, 0 beyond the
+ * causal blocks), recall, kl_pq, kl_qp [n_rows, G].  rows: device int64
+ * [n_rows]; sel: [B, G, n_q, 16] as from msa_topk_blocks.  Needs R = h_q/h_kv
+ * <= 8 (else MSA_ERR_UNSUPPORTED), mass_stride >= the block count, and a
+ * device workspace of msa_selection_recall_workspace(dims, n_rows) bytes
+ * (16-byte aligned).  A row outside [0, B * n_q) sets MSA_DEVERR_BAD_ENTRY. */
+MSA_API size_t msa_selection_recall_workspace(const msa_dims* dims, int64_t n_rows);
+MSA_API msa_status msa_selection_recall(const msa_dims* dims, msa_tensor q, msa_tensor k,
+                                        msa_tensor q_idx, msa_tensor k_idx,
+                                        const int32_t* sel, const int64_t* rows, int64_t n_rows,
+                                        float* block_mass, int64_t mass_stride, float* recall,
+                                        float* kl_pq, float* kl_qp, void* ws, size_t ws_bytes,
+                                        int32_t* dev_err, void* stream);
 
 /* Human-readable name of a status code (static storage). */
 MSA_API const char* msa_status_string(msa_status status);
