@@ -242,6 +242,47 @@ def bench_workload(w, steps, warmup, world, rank, with_e2e=True):
     return total_ms, per_stage, per_stage_mean, e2e, n_pieces
 
 
+def bench_recall(w, n_rows=64, reps=3):
+    """Selection recall and KL alignment target on n_rows sampled rows of the
+    workload (the next scoped measurement): mean recall / KL and the kernel time,
+    and the bytes it streams into shared memory (every causal K and k_idx block of
+    each (row, group), mostly L2 hits since rows share blocks)."""
+    from block_sparse_attention_32_b200 import pipeline, workloads as wl
+    d = pipeline.dims_for(w)
+    buf = pipeline.Buffers.allocate(d)
+    inp = wl.make_inputs(w, "cuda")
+    pipeline.select(buf, inp["q_idx"], inp["k_idx"])
+    rng = np.random.default_rng(7)
+    rows = np.sort(rng.choice(w.batch * w.n_q, size=n_rows, replace=False)).astype(np.int64)
+    rows_d = torch.from_numpy(rows).cuda()
+    args = (buf, inp["q"], inp["k"], inp["q_idx"], inp["k_idx"], rows_d)
+    pipeline.selection_recall(*args)
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    ev[0].record()
+    for _ in range(reps):
+        mass, rec, kpq, kqp = pipeline.selection_recall(*args)
+    ev[1].record()
+    torch.cuda.synchronize()
+    if int(buf.dev_err[0]) != 0:
+        raise RuntimeError(f"device error {int(buf.dev_err[0])} in the recall measurement")
+    ms = ev[0].elapsed_time(ev[1]) / reps
+    # every (row, group) streams its causal K and k_idx blocks into shared memory;
+    # rows of one batch share those blocks, so DRAM sees each at most once
+    nb = (w.q_pos0 + rows % w.n_q) // 128 + 1
+    streamed = float(nb.sum()) * w.h_kv * (128 * 128 * 2 + 128 * w.d_idx * 2)
+    blocks = int(nb.max())
+    unique = float(w.batch * blocks * 128 * (w.h_kv * 128 * 2 + w.h_kidx * w.d_idx * 2))
+    out = {"rows": n_rows, "mean_recall": float(rec.mean()),
+           "mean_kl_teacher_student": float(kpq.mean()),
+           "mean_kl_student_teacher": float(kqp.mean()), "ms": ms,
+           "streamed_bytes": streamed, "streamed_gbs": streamed / (ms / 1000.0) / 1e9,
+           "dram_bytes_at_most": unique}
+    del buf, inp
+    torch.cuda.empty_cache()
+    return out
+
+
 def bench_e2e(w, buf, dev_inp, steps, world):
     """The pass through the public API with host buffers: every step uploads its
     inputs from pinned host memory, runs the five calls and downloads the output
@@ -333,6 +374,7 @@ def main():
     ap.add_argument("--impl", default="msa", choices=["msa", "reference"])
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-recall", action="store_true")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -406,6 +448,10 @@ def main():
             torch.distributed.destroy_process_group()
         return
 
+    recall = None
+    if not args.no_recall:
+        recall = bench_recall(w)
+
     # dominant kernel: the longest stage; its bound is the larger of its
     # algorithmic time at the tensor peak and at the HBM peak
     dom = max(stage_mean, key=stage_mean.get)
@@ -448,6 +494,7 @@ def main():
         "index_tflops": idx_flops / (stage_mean["index"] / 1000.0) / 1e12,
         "stages_ms": stage_mean,
         "decode": decode,
+        "selection_recall": recall,
         "roofline": roof,
         "clocks": clocks,
         "gpu_launches": args.steps * sum(pipeline_launches().values()),
