@@ -18,6 +18,9 @@ Each function cites the page passage it follows in ``msa_oracle.c``:
     identity the KV-block-outer "Outer Gather Q" scheme relies on);
   * ``block_query_lists`` -- query->block lists inverted into block->query
     lists ("Kernel 创新：Outer Gather Q" section);
+  * ``e4m3_value``, ``quantize_e4m3``, ``index_pooled_e4m3`` -- the 8-bit
+    (e4m3) variant of steps 1-2: per-tensor scale amax / 448, nearest code
+    with ties to even, pooled scores from the codes;
   * ``selection_recall`` -- the main branch's attention mass per block (the
     teacher), the recall of the chosen blocks and the KL divergences to the
     index branch's block softmax (section "索引分支训练：KL 对齐").
@@ -70,11 +73,17 @@ def _load():
             lib.msa_oracle_attention.argtypes = [I64, I32, I32, I64, P, P, P, P, P, P, F64, P, P]
             lib.msa_oracle_merge.argtypes = [I64, I32, I32, P, P, P, P, P, P]
             lib.msa_oracle_block_query_lists.argtypes = [I64, I32, I64, I64, P, P, P]
+            lib.msa_oracle_e4m3_value.argtypes = [ctypes.c_uint8]
+            lib.msa_oracle_e4m3_value.restype = F64
+            lib.msa_oracle_quantize_e4m3.argtypes = [I64, P, P, P]
+            lib.msa_oracle_index_pooled_e4m3.argtypes = [I64, I32, I32, I64, I32, P, P, P, P, F64,
+                                                         F64, I64, P]
             lib.msa_oracle_selection_recall.argtypes = [I64, I32, I32, I32, I64, I32, P, P, P, P,
                                                          P, P, P, F64, I64, P, P, P, P]
             for f in (lib.msa_oracle_index_pooled, lib.msa_oracle_topk, lib.msa_oracle_topk_f32,
                       lib.msa_oracle_attention, lib.msa_oracle_merge,
-                      lib.msa_oracle_block_query_lists, lib.msa_oracle_selection_recall):
+                      lib.msa_oracle_block_query_lists, lib.msa_oracle_selection_recall,
+                      lib.msa_oracle_quantize_e4m3, lib.msa_oracle_index_pooled_e4m3):
                 f.restype = None
             _lib = lib
     return _lib
@@ -240,3 +249,35 @@ def selection_recall(q_rows, q_idx_rows, row_pos, row_batch, k, k_idx, sel, scal
                                     _p(kk), _p(ki), _p(s), float(scale), stride, _p(mass), _p(rec),
                                     _p(kpq), _p(kqp))
     return mass, rec, kpq, kqp
+
+
+def e4m3_value(code: int) -> float:
+    """Value of one e4m3 code."""
+    return float(_load().msa_oracle_e4m3_value(int(code) & 0xFF))
+
+
+def quantize_e4m3(x_bits):
+    """bf16 bits (any shape) -> (codes uint8 same shape, scale float)."""
+    lib = _load()
+    x = _c(x_bits, np.uint16)
+    codes = np.empty(x.shape, np.uint8)
+    scale = np.zeros((1,), np.float32)
+    lib.msa_oracle_quantize_e4m3(x.size, _p(x), _p(scale), _p(codes))
+    return codes, float(scale[0])
+
+
+def index_pooled_e4m3(q_codes_rows, row_pos, row_batch, k_codes, s_q, s_k, out_stride=None):
+    """Pooled block scores from e4m3 codes (see index_pooled): float64
+    [n_rows, G, out_stride], NaN at c >= own(t)."""
+    lib = _load()
+    q = _c(q_codes_rows, np.uint8)
+    k = _c(k_codes, np.uint8)
+    pos = _c(row_pos, np.int64)
+    bat = _c(row_batch, np.int64)
+    n_rows, G, d_idx = q.shape
+    _, h_kidx, n_kv, _ = k.shape
+    stride = out_stride or num_blocks(n_kv)
+    out = np.empty((n_rows, G, stride), np.float64)
+    lib.msa_oracle_index_pooled_e4m3(n_rows, G, d_idx, n_kv, h_kidx, _p(q), _p(pos), _p(bat), _p(k),
+                                     float(s_q), float(s_k), stride, _p(out))
+    return out

@@ -395,3 +395,82 @@ void msa_oracle_selection_recall(int64_t n_rows, int32_t H, int32_t G, int32_t d
     }
   }
 }
+
+/* ---------------------------------------------------------------------- */
+/* FP8 (e4m3) index branch: the next scoped variant of steps 1-2, the     */
+/* index scores computed from 8-bit copies of q_idx and k_idx.            */
+/* e4m3: sign, 4 exponent bits (bias 7), 3 mantissa bits; exponent 0 is   */
+/* subnormal (2^-6 * m / 8); exponent 15 with mantissa 7 is NaN; there is */
+/* no infinity, the largest finite magnitude is 448.                      */
+/* Quantisation of a tensor x: amax = max |x|, scale = amax / 448 (fp32,  */
+/* 1 when amax is 0), code(x) = e4m3 nearest to x / scale (fp32 division),*/
+/* ties to the even code, magnitudes past 448 saturate to 448.            */
+/* ---------------------------------------------------------------------- */
+double msa_oracle_e4m3_value(uint8_t code) {
+  const int s = code >> 7, e = (code >> 3) & 15, m = code & 7;
+  if (e == 15 && m == 7) return NAN;
+  const double mag = (e == 0) ? ldexp((double)m / 8.0, -6) : ldexp(1.0 + (double)m / 8.0, e - 7);
+  return s ? -mag : mag;
+}
+
+static uint8_t e4m3_nearest(float y) {
+  /* brute force over the 127 finite non-negative codes 0x00 .. 0x7E */
+  const double a = fabs((double)y);
+  uint8_t best = 0;
+  double bd = INFINITY;
+  for (int c = 0; c <= 0x7E; ++c) {
+    const double d = fabs(msa_oracle_e4m3_value((uint8_t)c) - a);
+    if (d < bd || (d == bd && (c & 1) == 0 && (best & 1) == 1)) {
+      bd = d;
+      best = (uint8_t)c;
+    }
+  }
+  if (a >= 448.0) best = 0x7E;
+  return (uint8_t)(best | (signbit(y) ? 0x80 : 0));   /* the sign survives rounding to zero */
+}
+
+void msa_oracle_quantize_e4m3(int64_t n, const uint16_t* x_bf16, float* scale_out,
+                              uint8_t* codes) {
+  float amax = 0.0f;
+  for (int64_t i = 0; i < n; ++i) {
+    const float v = fabsf((float)bf16_to_f64(x_bf16[i]));
+    if (v > amax) amax = v;
+  }
+  const float scale = (amax > 0.0f) ? amax / 448.0f : 1.0f;
+  *scale_out = scale;
+#pragma omp parallel for schedule(static)
+  for (int64_t i = 0; i < n; ++i) codes[i] = e4m3_nearest((float)bf16_to_f64(x_bf16[i]) / scale);
+}
+
+/* Steps 1-2 on the codes: pooled[r,g,c] = s_q s_k max over keys j of block c */
+/* of sum_k value(q_codes[r,g,k]) value(k_codes[b,hk(g),j,k]), c < own(t).   */
+void msa_oracle_index_pooled_e4m3(int64_t n_rows, int32_t G, int32_t d_idx, int64_t n_kv,
+                                  int32_t h_kidx,
+                                  const uint8_t* q_codes,   /* [n_rows,G,d_idx] */
+                                  const int64_t* row_pos, const int64_t* row_batch,
+                                  const uint8_t* k_codes,   /* [B',h_kidx,n_kv,d_idx] */
+                                  double s_q, double s_k, int64_t stride,
+                                  double* out)              /* [n_rows,G,stride] */
+{
+#pragma omp parallel for collapse(2) schedule(dynamic, 1)
+  for (int64_t r = 0; r < n_rows; ++r) {
+    for (int32_t g = 0; g < G; ++g) {
+      const int64_t own = row_pos[r] / MSA_BLOCK;
+      const uint8_t* qr = q_codes + (r * G + g) * (int64_t)d_idx;
+      const int64_t kb = (row_batch[r] * h_kidx + (h_kidx == 1 ? 0 : g)) * n_kv;
+      double* o = out + (r * G + g) * stride;
+      for (int64_t c = 0; c < stride; ++c) o[c] = NAN;
+      for (int64_t c = 0; c < own; ++c) {
+        double best = -INFINITY;
+        for (int64_t j = c * MSA_BLOCK; j < (c + 1) * MSA_BLOCK && j < n_kv; ++j) {
+          const uint8_t* kr = k_codes + (kb + j) * d_idx;
+          double dot = 0.0;
+          for (int32_t d = 0; d < d_idx; ++d)
+            dot += msa_oracle_e4m3_value(qr[d]) * msa_oracle_e4m3_value(kr[d]);
+          if (dot > best) best = dot;
+        }
+        o[c] = s_q * s_k * best;
+      }
+    }
+  }
+}

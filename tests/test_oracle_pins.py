@@ -447,3 +447,51 @@ def test_kl_closed_forms():
         qd = np.exp(z - z.max()) / np.exp(z - z.max()).sum()
         assert abs(kpq[0, g] - np.sum(0.5 * np.log(0.5 / qd))) < 1e-12
         assert abs(kqp[0, g] - np.sum(qd * np.log(qd / 0.5))) < 1e-12
+
+
+# ----------------------------------------------------------------------------
+# 8-bit (e4m3) index branch: format and quantisation from the e4m3 definition
+# ----------------------------------------------------------------------------
+def test_e4m3_values_from_the_format_definition():
+    """sign | 4 exponent bits (bias 7) | 3 mantissa bits; exponent 0 subnormal."""
+    cases = {0x00: 0.0, 0x38: 1.0, 0x39: 1.125, 0x3F: 1.875, 0x40: 2.0, 0xC0: -2.0,
+             0x08: 2.0 ** -6, 0x01: 2.0 ** -9, 0x07: 7 * 2.0 ** -9, 0x7E: 448.0, 0x79: 288.0,
+             0x30: 0.5, 0xB8: -1.0}
+    for code, val in cases.items():
+        assert oracle.e4m3_value(code) == val, hex(code)
+    assert math.isnan(oracle.e4m3_value(0x7F)) and math.isnan(oracle.e4m3_value(0xFF))
+
+
+def test_e4m3_quantisation_rounds_to_nearest_even_and_saturates():
+    """With amax = 448 the scale is 1: each value goes to its nearest code, ties to
+    the even code, and the sign of a value that rounds to zero is kept."""
+    vals = np.array([448.0, 1.0, 1.0625, 1.1875, -2.0, 300.0, 2.0 ** -10, -(2.0 ** -10),
+                     3 * 2.0 ** -10, 0.0, -0.0, 5.0, 240.0], np.float32)
+    expect = [0x7E, 0x38, 0x38, 0x3A, 0xC0, 0x79, 0x00, 0x80, 0x02, 0x00, 0x80, 0x4A, 0x77]
+    codes, scale = oracle.quantize_e4m3(_bf16_round(vals))
+    assert scale == 1.0
+    assert [int(c) for c in codes] == expect
+    # a tensor whose amax is 896 has scale 2: every value halves before rounding
+    codes2, scale2 = oracle.quantize_e4m3(_bf16_round(np.array([896.0, 2.0, -1.0], np.float32)))
+    assert scale2 == 2.0 and [int(c) for c in codes2] == [0x7E, 0x38, 0xB0]
+
+
+def test_e4m3_pooled_equals_bf16_pooled_on_exact_values():
+    """Inputs the 8-bit format holds exactly (scale 1) give the bf16 pooled scores."""
+    rng = np.random.default_rng(44)
+    n_kv, G, d = 700, 2, 128
+    pick = np.array([-2.0, -1.0, -0.5, 0.5, 1.0, 2.0], np.float32)
+    qv = rng.choice(pick, size=(5, G, d)).astype(np.float32)
+    kv = rng.choice(pick, size=(1, 1, n_kv, d)).astype(np.float32)
+    qv[0, 0, 0] = 448.0
+    kv[0, 0, 0, 0] = 448.0
+    rows = np.array([130, 256, 400, 511, 699], np.int64)
+    bats = np.zeros_like(rows)
+    qb, kb = _bf16_round(qv), _bf16_round(kv)
+    qc, sq = oracle.quantize_e4m3(qb)
+    kc, sk = oracle.quantize_e4m3(kb)
+    assert sq == 1.0 and sk == 1.0
+    p8 = oracle.index_pooled_e4m3(qc, rows, bats, kc, sq, sk)
+    p16 = oracle.index_pooled(qb, rows, bats, kb)
+    np.testing.assert_array_equal(np.isnan(p8), np.isnan(p16))
+    np.testing.assert_allclose(p8[~np.isnan(p8)], p16[~np.isnan(p16)], rtol=0, atol=0)
