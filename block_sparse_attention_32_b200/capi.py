@@ -69,6 +69,9 @@ def load_library(path: str) -> ctypes.CDLL:
     L.msa_build_block_query_lists_noalloc.argtypes = [_PD, _P, _P, _P, _P, _P]
     L.msa_sparse_attn_fwd.argtypes = [_PD, Tensor, Tensor, Tensor, _P, _P, _P, _P, _P, _P]
     L.msa_merge_partials.argtypes = [_PD, _P, _P, _P, _P, _P, _P, _P]
+    L.msa_quantize_e4m3.argtypes = [_P, ctypes.c_int64, _P, _P, _P]
+    L.msa_index_score_maxpool_e4m3.argtypes = [_PD, Tensor, Tensor, _P, _P, _P, ctypes.c_int64,
+                                               _P, _P]
     L.msa_selection_recall_workspace.argtypes = [_PD, ctypes.c_int64]
     L.msa_selection_recall_workspace.restype = ctypes.c_size_t
     L.msa_selection_recall.argtypes = [_PD, Tensor, Tensor, Tensor, Tensor, _P, _P, ctypes.c_int64,
@@ -77,7 +80,7 @@ def load_library(path: str) -> ctypes.CDLL:
     L.msa_status_string.restype = ctypes.c_char_p
     for f in (L.msa_index_score_maxpool, L.msa_topk_blocks, L.msa_build_block_query_lists,
               L.msa_build_block_query_lists_noalloc, L.msa_sparse_attn_fwd, L.msa_merge_partials,
-              L.msa_selection_recall):
+              L.msa_selection_recall, L.msa_quantize_e4m3, L.msa_index_score_maxpool_e4m3):
         f.restype = ctypes.c_int
     return L
 
@@ -190,3 +193,28 @@ def msa_selection_recall(d: Dims, q, k, q_idx, k_idx, sel, rows, block_mass, rec
                                       rows.numel(), _ptr(block_mass), block_mass.stride(0),
                                       _ptr(recall), _ptr(kl_pq), _ptr(kl_qp), _ptr(ws), nbytes,
                                       _ptr(dev_err), _stream()))
+
+
+def tensor_u8(t: torch.Tensor, bhtd: bool) -> Tensor:
+    """uint8 [B, T, H, D] (q_idx codes) or [B, H, T, D] (k_idx codes), strides in bytes."""
+    assert t.dim() == 4 and t.stride(3) == 1 and t.dtype == torch.uint8 and t.is_cuda
+    if bhtd:
+        return Tensor(t.data_ptr(), t.stride(0), t.stride(2), t.stride(1))
+    return Tensor(t.data_ptr(), t.stride(0), t.stride(1), t.stride(2))
+
+
+def msa_quantize_e4m3(x, codes, scale):
+    """x bf16 contiguous -> codes uint8 (same numel); scale: 2 device floats."""
+    assert x.is_contiguous() and codes.is_contiguous() and codes.numel() == x.numel()
+    assert scale.dtype == torch.float32 and scale.numel() >= 2
+    _check("msa_quantize_e4m3",
+           lib().msa_quantize_e4m3(_ptr(x), x.numel(), _ptr(codes), _ptr(scale), _stream()))
+
+
+def msa_index_score_maxpool_e4m3(d: Dims, q_idx8, k_idx8, scale_q, scale_k, pooled, stride,
+                                 dev_err=None):
+    _check("msa_index_score_maxpool_e4m3",
+           lib().msa_index_score_maxpool_e4m3(ctypes.byref(d), tensor_u8(q_idx8, False),
+                                              tensor_u8(k_idx8, True), _ptr(scale_q),
+                                              _ptr(scale_k), _ptr(pooled), stride,
+                                              _ptr(dev_err), _stream()))

@@ -25,25 +25,30 @@
 
 namespace msa {
 
-template <int D>
+template <int D, bool F8 = false>
 struct IdxCfg {
-  static constexpr int kHalves = D / 64;             // 128-byte column panels
-  static constexpr int kQBytes = 128 * D * 2;        // 128 query rows
-  static constexpr int kPairBytes = 256 * D * 2;     // two key blocks (256 key rows)
-  static constexpr int kStages = (D == 128) ? 3 : 5; // k_idx ring depth (pairs)
+  static constexpr int kEsz = F8 ? 1 : 2;            // bytes per element
+  static constexpr int kHalves = D * kEsz / 128;     // 128-byte column panels
+  static constexpr int kPanelElems = 128 / kEsz;     // elements per panel row
+  static constexpr int kQBytes = 128 * D * kEsz;     // 128 query rows
+  static constexpr int kPairBytes = 256 * D * kEsz;  // two key blocks (256 key rows)
+  static constexpr int kKSteps = D * kEsz / 32;      // MMA steps of 32 bytes along K
+  static constexpr int kStages = (kPairBytes == 65536) ? 3 : 5;   // k_idx ring depth (pairs)
   static constexpr int kChunkPairs = 64;             // key-block pairs per CTA
   static constexpr int kThreads = 192;               // TMA, MMA, 4 epilogue warps
   static constexpr int kBars = 2 * kStages + 1 + 4;
   static constexpr int kSmemBytes = 1024 + kQBytes + kStages * kPairBytes + kBars * 8 + 16;
 };
 
-template <int D>
+template <int D, bool F8 = false>
 __global__ void __launch_bounds__(192, 1)
     index_score_maxpool_kernel(const __grid_constant__ CUtensorMap tm_q,
                                const __grid_constant__ CUtensorMap tm_k, int64_t n_q,
                                int64_t q_pos0, int32_t G, int32_t h_kidx, int32_t n_qtiles,
-                               float* __restrict__ pooled, int64_t stride, int32_t* err) {
-  using C = IdxCfg<D>;
+                               float* __restrict__ pooled, int64_t stride, int32_t* err,
+                               const float* __restrict__ scale_q,
+                               const float* __restrict__ scale_k) {
+  using C = IdxCfg<D, F8>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -100,7 +105,7 @@ __global__ void __launch_bounds__(192, 1)
       prefetch_tensormap(&tm_k);
       mbar_arrive_expect_tx(qfull, C::kQBytes);
       for (int h = 0; h < C::kHalves; ++h)
-        tma_load_4d(sq + h * 16384, &tm_q, qfull, h * 64, g, (int32_t)q0, b);
+        tma_load_4d(sq + h * 16384, &tm_q, qfull, h * C::kPanelElems, g, (int32_t)q0, b);
       for (int i = 0; i < np; ++i) {
         const int s = i % C::kStages;
         if (i >= C::kStages &&
@@ -109,13 +114,13 @@ __global__ void __launch_bounds__(192, 1)
         mbar_arrive_expect_tx(full + s, C::kPairBytes);
         // one box of 256 key rows per 64-column panel (rows past n_kv read as 0)
         for (int h = 0; h < C::kHalves; ++h)
-          tma_load_4d(sk + s * C::kPairBytes + h * 32768, &tm_k, full + s, h * 64,
+          tma_load_4d(sk + s * C::kPairBytes + h * 32768, &tm_k, full + s, h * C::kPanelElems,
                       (int32_t)((c0 + 2 * i) * kBlock), hk, b);
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(128, 256, 0);
+      constexpr uint32_t idesc = F8 ? idesc_e4m3_f32(128, 256) : idesc_bf16_f32(128, 256, 0);
       const uint32_t qa = smem_u32(sq);
       bool ok = mbar_wait(qfull, 0, abort_flag, err);
       for (int i = 0; ok && i < np; ++i) {
@@ -125,11 +130,13 @@ __global__ void __launch_bounds__(192, 1)
         tc_fence_after();
         const uint32_t ka = smem_u32(sk + s * C::kPairBytes);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          umma_bf16(tmem + a * 256,
-                    smem_desc_sw128(qa + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                    smem_desc_sw128(ka + (kk >> 2) * 32768 + (kk & 3) * 32, 16, 1024), idesc,
-                    kk > 0 ? 1u : 0u);
+        for (int kk = 0; kk < C::kKSteps; ++kk) {
+          const uint64_t ad = smem_desc_sw128(qa + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+          const uint64_t bd = smem_desc_sw128(ka + (kk >> 2) * 32768 + (kk & 3) * 32, 16, 1024);
+          if constexpr (F8)
+            umma_e4m3(tmem + a * 256, ad, bd, idesc, kk > 0 ? 1u : 0u);
+          else
+            umma_bf16(tmem + a * 256, ad, bd, idesc, kk > 0 ? 1u : 0u);
         }
         umma_commit(empty + s);
         umma_commit(accfull + a);
@@ -143,6 +150,8 @@ __global__ void __launch_bounds__(192, 1)
     const int64_t q = q0 + row;
     const int64_t own = (q_pos0 + q) / kBlock;
     float* prow = pooled + (((int64_t)b * G + g) * n_q + q) * stride;
+    // 8-bit inputs: the codes' product times both tensors' scales
+    const float sc = F8 ? scale_q[0] * scale_k[0] : 1.0f;
     for (int i = 0; i < np; ++i) {
       const int a = i & 1;
       if (!mbar_wait(accfull + a, (i >> 1) & 1, abort_flag, err)) break;
@@ -160,7 +169,7 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
           for (int x = 0; x < 32; ++x) mx = fmaxf(mx, fmaxf(u2f(r0[x]), u2f(r1[x])));
         }
-        m[hb] = mx;
+        m[hb] = F8 ? mx * sc : mx;
       }
       tc_fence_before();
       __syncwarp();
@@ -331,20 +340,99 @@ cudaError_t launch_index_score_prefill(const CUtensorMap& tm_q, const CUtensorMa
   const int64_t n_chunks = (max_nb + per_cta - 1) / per_cta;
   dim3 grid((unsigned)(n_chunks * G), (unsigned)n_qtiles, (unsigned)batch);
   if (d_idx == 128) {
-    auto k = index_score_maxpool_kernel<128>;
+    auto k = index_score_maxpool_kernel<128, false>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          IdxCfg<128>::kSmemBytes);
     if (e != cudaSuccess) return e;
     k<<<grid, IdxCfg<128>::kThreads, IdxCfg<128>::kSmemBytes, st>>>(
-        tm_q, tm_k, n_q, q_pos0, G, h_kidx, (int32_t)n_qtiles, pooled, stride, err);
+        tm_q, tm_k, n_q, q_pos0, G, h_kidx, (int32_t)n_qtiles, pooled, stride, err, nullptr,
+        nullptr);
   } else {
-    auto k = index_score_maxpool_kernel<64>;
+    auto k = index_score_maxpool_kernel<64, false>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          IdxCfg<64>::kSmemBytes);
     if (e != cudaSuccess) return e;
     k<<<grid, IdxCfg<64>::kThreads, IdxCfg<64>::kSmemBytes, st>>>(
-        tm_q, tm_k, n_q, q_pos0, G, h_kidx, (int32_t)n_qtiles, pooled, stride, err);
+        tm_q, tm_k, n_q, q_pos0, G, h_kidx, (int32_t)n_qtiles, pooled, stride, err, nullptr,
+        nullptr);
   }
+  return cudaGetLastError();
+}
+
+// 8-bit (e4m3) index scores: d_idx = 128, maps over uint8 codes, box {128, ...}.
+cudaError_t launch_index_score_e4m3(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
+                                   int64_t batch, int64_t n_q, int64_t q_pos0, int32_t G,
+                                   int32_t h_kidx, float* pooled, int64_t stride,
+                                   const float* scale_q, const float* scale_k, int32_t* err,
+                                   cudaStream_t st) {
+  using C = IdxCfg<128, true>;
+  const int64_t n_qtiles = (n_q + 127) / 128;
+  const int64_t max_nb = (q_pos0 + n_q - 1) / kBlock;
+  if (max_nb == 0) return cudaSuccess;
+  const int64_t per_cta = 2 * C::kChunkPairs;
+  const int64_t n_chunks = (max_nb + per_cta - 1) / per_cta;
+  dim3 grid((unsigned)(n_chunks * G), (unsigned)n_qtiles, (unsigned)batch);
+  auto k = index_score_maxpool_kernel<128, true>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       C::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  k<<<grid, C::kThreads, C::kSmemBytes, st>>>(tm_q, tm_k, n_q, q_pos0, G, h_kidx,
+                                               (int32_t)n_qtiles, pooled, stride, err, scale_q,
+                                               scale_k);
+  return cudaGetLastError();
+}
+
+// Per-tensor e4m3 quantisation: amax of |x| (atomic max on the float bits of
+// non-negative values), scale = amax / 448 (1 when amax is 0), codes = x /
+// scale rounded to the nearest e4m3 value (ties to even, saturating at 448).
+__global__ void __launch_bounds__(256)
+    amax_bf16_kernel(const __nv_bfloat16* __restrict__ x, int64_t n, uint32_t* amax_bits) {
+  float m = 0.f;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x)
+    m = fmaxf(m, fabsf(__bfloat162float(x[i])));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 31) == 0) atomicMax(amax_bits, __float_as_uint(m));
+}
+
+__global__ void __launch_bounds__(256)
+    quantize_e4m3_kernel(const __nv_bfloat16* __restrict__ x, int64_t n,
+                         const uint32_t* __restrict__ amax_bits, uint8_t* __restrict__ codes,
+                         float* __restrict__ scale_out) {
+  const float amax = __uint_as_float(*amax_bits);
+  const float scale = amax > 0.f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+  if (blockIdx.x == 0 && threadIdx.x == 0) *scale_out = scale;
+  for (int64_t i = 2 * ((int64_t)blockIdx.x * blockDim.x + threadIdx.x); i < n;
+       i += 2 * (int64_t)gridDim.x * blockDim.x) {
+    const float y0 = __fdiv_rn(__bfloat162float(x[i]), scale);
+    const float y1 = (i + 1 < n) ? __fdiv_rn(__bfloat162float(x[i + 1]), scale) : 0.f;
+    uint16_t pair;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(pair) : "f"(y1), "f"(y0));
+    codes[i] = (uint8_t)(pair & 0xFF);
+    if (i + 1 < n) codes[i + 1] = (uint8_t)(pair >> 8);
+  }
+}
+
+cudaError_t launch_quantize_e4m3(const void* x, int64_t n, void* codes, float* scale,
+                                 cudaStream_t st) {
+  uint32_t* amax_bits = reinterpret_cast<uint32_t*>(scale + 1);
+  cudaError_t e = cudaMemsetAsync(amax_bits, 0, sizeof(uint32_t), st);
+  if (e != cudaSuccess) return e;
+  if (n == 0) {
+    quantize_e4m3_kernel<<<1, 32, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(x), 0,
+                                           amax_bits, reinterpret_cast<uint8_t*>(codes), scale);
+    return cudaGetLastError();
+  }
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t blocks = min64((n + 511) / 512, (int64_t)sms * 8);
+  amax_bf16_kernel<<<(unsigned)blocks, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(x),
+                                                     n, amax_bits);
+  quantize_e4m3_kernel<<<(unsigned)blocks, 256, 0, st>>>(
+      reinterpret_cast<const __nv_bfloat16*>(x), n, amax_bits, reinterpret_cast<uint8_t*>(codes),
+      scale);
   return cudaGetLastError();
 }
 

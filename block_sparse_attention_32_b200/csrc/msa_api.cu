@@ -37,6 +37,10 @@ cudaError_t launch_selection_recall(const CUtensorMap&, const CUtensorMap&, cons
                                     int32_t, int32_t, int32_t, float, const int32_t*, float*,
                                     int64_t, float*, float*, float*, void*, int32_t*,
                                     cudaStream_t);
+cudaError_t launch_index_score_e4m3(const CUtensorMap&, const CUtensorMap&, int64_t, int64_t,
+                                   int64_t, int32_t, int32_t, float*, int64_t, const float*,
+                                   const float*, int32_t*, cudaStream_t);
+cudaError_t launch_quantize_e4m3(const void*, int64_t, void*, float*, cudaStream_t);
 cudaError_t launch_merge(const int32_t*, const float*, const float*, void*, float*, int64_t,
                          int64_t, int32_t, int32_t, cudaStream_t);
 }  // namespace msa
@@ -136,6 +140,35 @@ msa_status make_map_rows_f32(CUtensorMap* map, void* ptr, uint64_t rows, uint32_
 }
 
 msa_status from_cuda(cudaError_t e) { return e == cudaSuccess ? MSA_OK : MSA_ERR_CUDA; }
+
+// 4-D uint8 map (e4m3 codes): dims {inner, d1, d2, d3}, byte strides, box
+// {128, b1, b2, 1}, 128-byte swizzle, zero fill out of bounds.
+msa_status make_map_u8(CUtensorMap* map, const void* ptr, uint64_t inner, uint64_t d1,
+                       uint64_t d2, uint64_t d3, int64_t s1, int64_t s2, int64_t s3, uint32_t b1,
+                       uint32_t b2) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return MSA_ERR_CUDA;
+  cuuint64_t dims[4] = {inner, d1, d2, d3};
+  cuuint64_t strides[3] = {(cuuint64_t)s1, (cuuint64_t)s2, (cuuint64_t)s3};
+  for (int i = 0; i < 3; ++i)
+    if (strides[i] == 0) strides[i] = 16;
+  cuuint32_t box[4] = {128, b1, b2, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(ptr), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? MSA_OK : MSA_ERR_CUDA;
+}
+
+msa_status check_tensor_u8(const msa_tensor& t) {
+  if (t.ptr == nullptr) return MSA_ERR_INVALID_ARG;
+  if (!aligned16(t.ptr)) return MSA_ERR_ALIGNMENT;
+  if (t.s_batch < 0 || t.s_tok < 0 || t.s_head < 0) return MSA_ERR_INVALID_ARG;
+  if ((t.s_batch % 16) || (t.s_tok % 16) || (t.s_head % 16)) return MSA_ERR_ALIGNMENT;
+  return MSA_OK;
+}
+
+
 
 }  // namespace
 
@@ -295,6 +328,42 @@ msa_status msa_merge_partials(const msa_dims* d, const int32_t* sel, const float
   const int64_t n_rows = d->batch * d->n_q * d->h_q;
   return from_cuda(msa::launch_merge(sel, part_ml, part_acc, out, lse, n_rows, d->n_q, d->h_q,
                                      d->h_kv, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+msa_status msa_quantize_e4m3(const void* x, int64_t n, void* codes, float* scale,
+                             void* stream) {
+  if (n < 0) return MSA_ERR_INVALID_ARG;
+  if (scale == nullptr || (n > 0 && (x == nullptr || codes == nullptr))) return MSA_ERR_INVALID_ARG;
+  return from_cuda(msa::launch_quantize_e4m3(x, n, codes, scale,
+                                             reinterpret_cast<cudaStream_t>(stream)));
+}
+
+msa_status msa_index_score_maxpool_e4m3(const msa_dims* d, msa_tensor q_idx8, msa_tensor k_idx8,
+                                        const float* scale_q, const float* scale_k,
+                                        float* pooled, int64_t pooled_row_stride,
+                                        int32_t* dev_err, void* stream) {
+  msa_status s = check_dims(d);
+  if (s != MSA_OK) return s;
+  if (d->d_idx != 128) return MSA_ERR_UNSUPPORTED;   // one 128-byte row per index vector
+  if ((s = check_tensor_u8(q_idx8)) != MSA_OK) return s;
+  if ((s = check_tensor_u8(k_idx8)) != MSA_OK) return s;
+  if (pooled == nullptr || scale_q == nullptr || scale_k == nullptr) return MSA_ERR_INVALID_ARG;
+  if (!aligned16(pooled)) return MSA_ERR_ALIGNMENT;
+  if (pooled_row_stride < msa_num_blocks(d) || pooled_row_stride % 4 != 0)
+    return MSA_ERR_INVALID_ARG;
+  CUtensorMap tq, tk;
+  // q_idx codes [B, n_q, G, 128]: dims {128, G, n_q, B}, box {128, 1, 128, 1}
+  if ((s = make_map_u8(&tq, q_idx8.ptr, 128, d->h_kv, d->n_q, d->batch, q_idx8.s_head,
+                       q_idx8.s_tok, q_idx8.s_batch, 1, 128)) != MSA_OK)
+    return s;
+  // k_idx codes [B, h_kidx, n_kv, 128]: dims {128, n_kv, h_kidx, B}, box {128, 256, 1, 1}
+  if ((s = make_map_u8(&tk, k_idx8.ptr, 128, d->n_kv, d->h_kidx, d->batch, k_idx8.s_tok,
+                       k_idx8.s_head, k_idx8.s_batch, 256, 1)) != MSA_OK)
+    return s;
+  return from_cuda(msa::launch_index_score_e4m3(tq, tk, d->batch, d->n_q, d->q_pos0, d->h_kv,
+                                                d->h_kidx, pooled, pooled_row_stride, scale_q,
+                                                scale_k, dev_err,
+                                                reinterpret_cast<cudaStream_t>(stream)));
 }
 
 size_t msa_selection_recall_workspace(const msa_dims* d, int64_t n_rows) {

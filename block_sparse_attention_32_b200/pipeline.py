@@ -76,6 +76,23 @@ def select(buf: Buffers, q_idx, k_idx):
     capi.msa_topk_blocks(d, buf.pooled, buf.pooled_stride, buf.sel, buf.dev_err)
 
 
+def select_e4m3(buf: Buffers, q_idx, k_idx):
+    """Selection from 8-bit index scores: per-tensor e4m3 copies of q_idx and
+    k_idx, the tcgen05 kind::f8f6f4 score + max-pool kernel, then top-16 ->
+    buf.sel.  Returns the codes and the two scales (device)."""
+    d = buf.dims
+    q8 = torch.empty(q_idx.shape, dtype=torch.uint8, device=q_idx.device)
+    k8 = torch.empty(k_idx.shape, dtype=torch.uint8, device=k_idx.device)
+    sq = torch.empty((2,), dtype=torch.float32, device=q_idx.device)
+    sk = torch.empty((2,), dtype=torch.float32, device=q_idx.device)
+    capi.msa_quantize_e4m3(q_idx, q8, sq)
+    capi.msa_quantize_e4m3(k_idx, k8, sk)
+    capi.msa_index_score_maxpool_e4m3(d, q8, k8, sq, sk, buf.pooled, buf.pooled_stride,
+                                      buf.dev_err)
+    capi.msa_topk_blocks(d, buf.pooled, buf.pooled_stride, buf.sel, buf.dev_err)
+    return q8, k8, sq, sk
+
+
 def attend(buf: Buffers, q, k, v, sel=None):
     """Block lists + KV-block-outer attention + merge over `sel` (default buf.sel)."""
     d = buf.dims

@@ -204,6 +204,30 @@ MSA_API msa_status msa_merge_partials(const msa_dims* dims, const int32_t* sel,
                               const float* part_ml, const float* part_acc,
                               void* out, float* lse, int32_t* dev_err, void* stream);
 
+/* 8-bit (e4m3) index branch, an opt-in variant of step 1 that the MSA pages do
+ * not describe: the "推理系统基础设施手记（三）" page (sections "4. CSA：先压缩，
+ * 再稀疏选择" and "8. 常见坑") reports a low-precision indexer that makes selection
+ * cheap and warns that its inputs must be clamped to the format's range.
+ * msa_quantize_e4m3: n bf16 values x (device, contiguous) -> n e4m3 codes
+ * (device, contiguous bytes) with one per-tensor scale: amax = max |x|,
+ * scale = amax / 448 (1 when amax is 0), code = e4m3 nearest to x / scale
+ * (ties to even; magnitudes past 448 saturate).  scale points to 2 device
+ * floats: scale[0] receives the scale, scale[1] is scratch for amax. */
+MSA_API msa_status msa_quantize_e4m3(const void* x_bf16, int64_t n, void* codes, float* scale,
+                                     void* stream);
+
+/* Step 1 on e4m3 codes (d_idx = 128 only): pooled[b, g, i, c] =
+ * scale_q[0] * scale_k[0] * max over keys j of block c of sum_k code_q . code_k,
+ * for c < own(t), tcgen05 kind::f8f6f4 tiles.  q_idx8 [B, n_q, G, 128] and
+ * k_idx8 [B, h_kidx, n_kv, 128] are uint8 codes (msa_tensor strides in bytes,
+ * multiples of 16); the scales are device floats from msa_quantize_e4m3.
+ * Feed `pooled` to msa_topk_blocks as usual. */
+MSA_API msa_status msa_index_score_maxpool_e4m3(const msa_dims* dims, msa_tensor q_idx8,
+                                                msa_tensor k_idx8, const float* scale_q,
+                                                const float* scale_k, float* pooled,
+                                                int64_t pooled_row_stride, int32_t* dev_err,
+                                                void* stream);
+
 /* Selection recall and the index branch's alignment target, for sampled query
  * rows ("MSA 稀疏注意力三国杀" page, section "索引分支训练：KL 对齐": the index
  * branch learns the main branch's attention distribution through a KL
