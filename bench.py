@@ -242,6 +242,46 @@ def bench_workload(w, steps, warmup, world, rank, with_e2e=True):
     return total_ms, per_stage, per_stage_mean, e2e, n_pieces
 
 
+def bench_e4m3(w, reps=3):
+    """The 8-bit index branch on the workload: time of quantisation + scores +
+    top-k against the bf16 selection step, and how many (query, group) sets
+    and selected blocks the two selections share."""
+    from block_sparse_attention_32_b200 import pipeline, workloads as wl
+    d = pipeline.dims_for(w)
+    buf = pipeline.Buffers.allocate(d)
+    inp = wl.make_inputs(w, "cuda", with_qkv=False)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    pipeline.select(buf, inp["q_idx"], inp["k_idx"])
+    pipeline.select_e4m3(buf, inp["q_idx"], inp["k_idx"])
+    torch.cuda.synchronize()
+    ev[0].record()
+    for _ in range(reps):
+        pipeline.select(buf, inp["q_idx"], inp["k_idx"])
+    ev[1].record()
+    sel16 = buf.sel.clone()
+    ev[2].record()
+    for _ in range(reps):
+        pipeline.select_e4m3(buf, inp["q_idx"], inp["k_idx"])
+    ev[3].record()
+    torch.cuda.synchronize()
+    if int(buf.dev_err[0]) != 0:
+        raise RuntimeError(f"device error {int(buf.dev_err[0])} in the e4m3 measurement")
+    sel8 = buf.sel
+    same_sets = float((sel8 == sel16).all(dim=-1).float().mean())
+    # blocks of the 8-bit set that the bf16 set also holds (both ascending, -1 padded)
+    valid = sel16 >= 0
+    hits = (sel8.unsqueeze(-1) == sel16.unsqueeze(-2)).any(dim=-1) & (sel8 >= 0)
+    shared = float(hits.sum()) / float(valid.sum())
+    ms16 = ev[0].elapsed_time(ev[1]) / reps
+    ms8 = ev[2].elapsed_time(ev[3]) / reps
+    idx_flops, _, _ = work_counts(w)
+    del buf, inp
+    torch.cuda.empty_cache()
+    return {"select_ms_bf16": ms16, "select_ms_e4m3": ms8, "speedup": ms16 / ms8,
+            "identical_sets": same_sets, "shared_blocks": shared,
+            "index_tflops_e4m3_incl_quant_and_topk": idx_flops / (ms8 / 1000.0) / 1e12}
+
+
 def bench_recall(w, n_rows=64, reps=3):
     """Selection recall and KL alignment target on n_rows sampled rows of the
     workload (the next scoped measurement): mean recall / KL and the kernel time,
@@ -375,6 +415,7 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-recall", action="store_true")
+    ap.add_argument("--no-e4m3", action="store_true")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -451,6 +492,7 @@ def main():
     recall = None
     if not args.no_recall:
         recall = bench_recall(w)
+    e4m3 = None if args.no_e4m3 else bench_e4m3(w)
 
     # dominant kernel: the longest stage; its bound is the larger of its
     # algorithmic time at the tensor peak and at the HBM peak
@@ -495,6 +537,7 @@ def main():
         "stages_ms": stage_mean,
         "decode": decode,
         "selection_recall": recall,
+        "index_e4m3": e4m3,
         "roofline": roof,
         "clocks": clocks,
         "gpu_launches": args.steps * sum(pipeline_launches().values()),

@@ -14,8 +14,9 @@
 //    step covers two key blocks (N = 256, halving shared-memory operand
 //    traffic per FLOP).  Warp roles: warp 0 issues TMA loads (the q_idx tile
 //    once, pairs of k_idx blocks through a 3-5 stage ring), warp 1 issues the
-//    MMAs into two 256-column TMEM accumulators, warps 2-5 take the two row
-//    maxima of each accumulator and store them.
+//    MMAs into two 256-column TMEM accumulators, warps 2-9 take the row maxima
+//    (one warp per TMEM lane quarter and block of the pair, all 128 columns in
+//    one round of loads) and store them.
 //  * index_score_decode_kernel -- one query per sequence (decode): a
 //    streaming scan of k_idx, HBM-bound.  TMA streams 32 KB key blocks
 //    through a shared-memory ring; consumer warps multiply them by the
@@ -35,13 +36,13 @@ struct IdxCfg {
   static constexpr int kKSteps = D * kEsz / 32;      // MMA steps of 32 bytes along K
   static constexpr int kStages = (kPairBytes == 65536) ? 3 : 5;   // k_idx ring depth (pairs)
   static constexpr int kChunkPairs = 64;             // key-block pairs per CTA
-  static constexpr int kThreads = 192;               // TMA, MMA, 4 epilogue warps
+  static constexpr int kThreads = 320;               // TMA, MMA, 8 epilogue warps
   static constexpr int kBars = 2 * kStages + 1 + 4;
   static constexpr int kSmemBytes = 1024 + kQBytes + kStages * kPairBytes + kBars * 8 + 16;
 };
 
 template <int D, bool F8 = false>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     index_score_maxpool_kernel(const __grid_constant__ CUtensorMap tm_q,
                                const __grid_constant__ CUtensorMap tm_k, int64_t n_q,
                                int64_t q_pos0, int32_t G, int32_t h_kidx, int32_t n_qtiles,
@@ -85,7 +86,7 @@ __global__ void __launch_bounds__(192, 1)
     mbar_init(qfull, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(accfull + i, 1);
-      mbar_init(accempty + i, 4);
+      mbar_init(accempty + i, 8);
     }
     *abort_flag = 0;
     fence_mbarrier_init();
@@ -143,8 +144,10 @@ __global__ void __launch_bounds__(192, 1)
       }
     }
   } else {
-    // epilogue: thread = query row; columns [0,128) = block c, [128,256) = block c+1
+    // epilogue: thread = query row; warps 2-5 take columns [0,128) of each
+    // accumulator (block c), warps 6-9 columns [128,256) (block c+1)
     const int quarter = warp & 3;
+    const int hb = (warp - 2) >> 2;
     const int row = quarter * 32 + lane;
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     const int64_t q = q0 + row;
@@ -156,32 +159,28 @@ __global__ void __launch_bounds__(192, 1)
       const int a = i & 1;
       if (!mbar_wait(accfull + a, (i >> 1) & 1, abort_flag, err)) break;
       tc_fence_after();
-      float m[2];
-#pragma unroll
-      for (int hb = 0; hb < 2; ++hb) {
-        float mx = -INFINITY;
-#pragma unroll
-        for (int j = 0; j < 4; j += 2) {
-          uint32_t r0[32], r1[32];
-          tmem_ld_32x32b_x32(tmem + lane_base + a * 256 + hb * 128 + j * 32, r0);
-          tmem_ld_32x32b_x32(tmem + lane_base + a * 256 + hb * 128 + (j + 1) * 32, r1);
-          tmem_ld_wait();
-#pragma unroll
-          for (int x = 0; x < 32; ++x) mx = fmaxf(mx, fmaxf(u2f(r0[x]), u2f(r1[x])));
-        }
-        m[hb] = F8 ? mx * sc : mx;
-      }
+      uint32_t r0[32], r1[32], r2[32], r3[32];
+      const uint32_t col = tmem + lane_base + a * 256 + hb * 128;
+      tmem_ld_32x32b_x32(col, r0);
+      tmem_ld_32x32b_x32(col + 32, r1);
+      tmem_ld_32x32b_x32(col + 64, r2);
+      tmem_ld_32x32b_x32(col + 96, r3);
+      tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(accempty + a);
-      const int64_t c = c0 + 2 * i;
-      if (q < n_q) {
-        if (c + 1 < own && 2 * i + 1 < nb) {
-          *reinterpret_cast<float2*>(prow + c) = make_float2(m[0], m[1]);
-        } else if (c < own) {
-          prow[c] = m[0];
-        }
+      float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+      for (int x = 0; x < 32; ++x) {
+        m4[0] = fmaxf(m4[0], u2f(r0[x]));
+        m4[1] = fmaxf(m4[1], u2f(r1[x]));
+        m4[2] = fmaxf(m4[2], u2f(r2[x]));
+        m4[3] = fmaxf(m4[3], u2f(r3[x]));
       }
+      float m = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+      if (F8) m *= sc;
+      const int64_t c = c0 + 2 * i + hb;
+      if (q < n_q && c < own && 2 * i + hb < nb) prow[c] = m;
     }
   }
 
