@@ -21,6 +21,9 @@ Each function cites the page passage it follows in ``msa_oracle.c``:
   * ``e4m3_value``, ``quantize_e4m3``, ``index_pooled_e4m3`` -- the 8-bit
     (e4m3) variant of steps 1-2: per-tensor scale amax / 448, nearest code
     with ties to even, pooled scores from the codes;
+  * ``token_select_attention`` -- the token-level variant at the same
+    budget: top-2048 tokens by index score, attention over them, and the full
+    causal attention's lse;
   * ``selection_recall`` -- the main branch's attention mass per block (the
     teacher), the recall of the chosen blocks and the KL divergences to the
     index branch's block softmax (section "索引分支训练：KL 对齐").
@@ -78,12 +81,16 @@ def _load():
             lib.msa_oracle_quantize_e4m3.argtypes = [I64, P, P, P]
             lib.msa_oracle_index_pooled_e4m3.argtypes = [I64, I32, I32, I64, I32, P, P, P, P, F64,
                                                          F64, I64, P]
+            lib.msa_oracle_token_select_attention.argtypes = [I64, I32, I32, I32, I64, I32, I64,
+                                                              P, P, P, P, P, P, P, F64, P, P,
+                                                              P, P]
             lib.msa_oracle_selection_recall.argtypes = [I64, I32, I32, I32, I64, I32, P, P, P, P,
                                                          P, P, P, F64, I64, P, P, P, P]
             for f in (lib.msa_oracle_index_pooled, lib.msa_oracle_topk, lib.msa_oracle_topk_f32,
                       lib.msa_oracle_attention, lib.msa_oracle_merge,
                       lib.msa_oracle_block_query_lists, lib.msa_oracle_selection_recall,
-                      lib.msa_oracle_quantize_e4m3, lib.msa_oracle_index_pooled_e4m3):
+                      lib.msa_oracle_quantize_e4m3, lib.msa_oracle_index_pooled_e4m3,
+                      lib.msa_oracle_token_select_attention):
                 f.restype = None
             _lib = lib
     return _lib
@@ -281,3 +288,28 @@ def index_pooled_e4m3(q_codes_rows, row_pos, row_batch, k_codes, s_q, s_k, out_s
     lib.msa_oracle_index_pooled_e4m3(n_rows, G, d_idx, n_kv, h_kidx, _p(q), _p(pos), _p(bat), _p(k),
                                      float(s_q), float(s_k), stride, _p(out))
     return out
+
+
+def token_select_attention(q_rows, q_idx_rows, row_pos, row_batch, k, v, k_idx, scale, budget=2048):
+    """Top-`budget` tokens by index score per (row, group) (ascending, -1 padded,
+    int64 [n, G, budget]), attention over them (out [n, H, 128], lse [n, H]) and
+    the full causal lse [n, H], all float64."""
+    lib = _load()
+    q = _c(q_rows, np.uint16)
+    qi = _c(q_idx_rows, np.uint16)
+    kk = _c(k, np.uint16)
+    vv = _c(v, np.uint16)
+    ki = _c(k_idx, np.uint16)
+    pos = _c(row_pos, np.int64)
+    bat = _c(row_batch, np.int64)
+    n, H, _ = q.shape
+    _, G, d_idx = qi.shape
+    n_kv = kk.shape[2]
+    tokens = np.empty((n, G, budget), np.int64)
+    out = np.empty((n, H, HEAD_DIM), np.float64)
+    lse = np.empty((n, H), np.float64)
+    lse_full = np.empty((n, H), np.float64)
+    lib.msa_oracle_token_select_attention(n, H, G, d_idx, n_kv, ki.shape[1], budget, _p(q), _p(qi),
+                                          _p(pos), _p(bat), _p(kk), _p(vv), _p(ki), float(scale),
+                                          _p(tokens), _p(out), _p(lse), _p(lse_full))
+    return tokens, out, lse, lse_full

@@ -474,3 +474,99 @@ void msa_oracle_index_pooled_e4m3(int64_t n_rows, int32_t G, int32_t d_idx, int6
     }
   }
 }
+
+/* ---------------------------------------------------------------------- */
+/* Token-level selection at the same budget: the top min(2048, t+1) keys  */
+/* j <= t by index score q_idx[g] . k_idx[j] (score descending, lower      */
+/* index first), the granularity the other selection-based method of the  */
+/* pages (DSA) uses ([P1] section "分歧一：颗粒度——token 级还是块级？";   */
+/* [P3] section 4; [P4] "Sparse attention · DSA và MSA chọn vị trí").      */
+/* Exact softmax attention                                                */
+/* over the chosen tokens, per head of the group, with its lse; and the   */
+/* full causal attention's lse for the same heads.                        */
+/* ---------------------------------------------------------------------- */
+typedef struct { double s; int64_t j; } tok_t;
+
+static int tok_cmp(const void* pa, const void* pb) {
+  const tok_t* a = (const tok_t*)pa;
+  const tok_t* b = (const tok_t*)pb;
+  if (a->s > b->s) return -1;
+  if (a->s < b->s) return 1;
+  return (a->j < b->j) ? -1 : (a->j > b->j);
+}
+
+static int i64_cmp(const void* pa, const void* pb) {
+  const int64_t a = *(const int64_t*)pa, b = *(const int64_t*)pb;
+  return (a > b) - (a < b);
+}
+
+void msa_oracle_token_select_attention(int64_t n_rows, int32_t H, int32_t G, int32_t d_idx,
+                                       int64_t n_kv, int32_t h_kidx, int64_t budget,
+                                       const uint16_t* q_rows,     /* [n_rows,H,128] */
+                                       const uint16_t* q_idx_rows, /* [n_rows,G,d_idx] */
+                                       const int64_t* row_pos, const int64_t* row_batch,
+                                       const uint16_t* k, const uint16_t* v, /* [B',G,n_kv,128] */
+                                       const uint16_t* k_idx,      /* [B',h_kidx,n_kv,d_idx] */
+                                       double scale,
+                                       int64_t* tokens,            /* [n_rows,G,budget], -1 pad */
+                                       double* out,                /* [n_rows,H,128] */
+                                       double* lse,                /* [n_rows,H] */
+                                       double* lse_full)           /* [n_rows,H] */
+{
+  const int32_t R = H / G;
+#pragma omp parallel for collapse(2) schedule(dynamic, 1)
+  for (int64_t r = 0; r < n_rows; ++r) {
+    for (int32_t g = 0; g < G; ++g) {
+      const int64_t t = row_pos[r];
+      const int64_t kvbase = (row_batch[r] * G + g) * n_kv;
+      const int64_t kibase = (row_batch[r] * h_kidx + (h_kidx == 1 ? 0 : g)) * n_kv;
+      const uint16_t* qi = q_idx_rows + (r * G + g) * (int64_t)d_idx;
+      tok_t* sc = (tok_t*)malloc((size_t)(t + 1) * sizeof(tok_t));
+      for (int64_t j = 0; j <= t; ++j) {
+        const uint16_t* kj = k_idx + (kibase + j) * d_idx;
+        double dot = 0.0;
+        for (int32_t d = 0; d < d_idx; ++d) dot += bf16_to_f64(qi[d]) * bf16_to_f64(kj[d]);
+        sc[j].s = dot;
+        sc[j].j = j;
+      }
+      qsort(sc, (size_t)(t + 1), sizeof(tok_t), tok_cmp);
+      const int64_t m = (t + 1 < budget) ? t + 1 : budget;
+      int64_t* tk = tokens + (r * G + g) * budget;
+      for (int64_t i = 0; i < m; ++i) tk[i] = sc[i].j;
+      qsort(tk, (size_t)m, sizeof(int64_t), i64_cmp);
+      for (int64_t i = m; i < budget; ++i) tk[i] = -1;
+      free(sc);
+      for (int32_t hr = 0; hr < R; ++hr) {
+        const int32_t h = g * R + hr;
+        const uint16_t* qh = q_rows + (r * H + h) * (int64_t)MSA_HEAD_DIM;
+        double qd[MSA_HEAD_DIM];
+        for (int32_t d = 0; d < MSA_HEAD_DIM; ++d) qd[d] = bf16_to_f64(qh[d]);
+        double* logit = (double*)malloc((size_t)(t + 1) * sizeof(double));
+        double mf = -INFINITY;
+        for (int64_t j = 0; j <= t; ++j) {
+          const uint16_t* kj = k + (kvbase + j) * MSA_HEAD_DIM;
+          double dot = 0.0;
+          for (int32_t d = 0; d < MSA_HEAD_DIM; ++d) dot += qd[d] * bf16_to_f64(kj[d]);
+          logit[j] = scale * dot;
+          if (logit[j] > mf) mf = logit[j];
+        }
+        double lf = 0.0;
+        for (int64_t j = 0; j <= t; ++j) lf += exp(logit[j] - mf);
+        lse_full[r * H + h] = mf + log(lf);
+        double ms = -INFINITY;
+        for (int64_t i = 0; i < m; ++i) if (logit[tk[i]] > ms) ms = logit[tk[i]];
+        double ls = 0.0, o[MSA_HEAD_DIM];
+        for (int32_t d = 0; d < MSA_HEAD_DIM; ++d) o[d] = 0.0;
+        for (int64_t i = 0; i < m; ++i) {
+          const double p = exp(logit[tk[i]] - ms);
+          ls += p;
+          const uint16_t* vj = v + (kvbase + tk[i]) * MSA_HEAD_DIM;
+          for (int32_t d = 0; d < MSA_HEAD_DIM; ++d) o[d] += p * bf16_to_f64(vj[d]);
+        }
+        for (int32_t d = 0; d < MSA_HEAD_DIM; ++d) out[(r * H + h) * (int64_t)MSA_HEAD_DIM + d] = o[d] / ls;
+        lse[r * H + h] = ms + log(ls);
+        free(logit);
+      }
+    }
+  }
+}

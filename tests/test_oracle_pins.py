@@ -495,3 +495,79 @@ def test_e4m3_pooled_equals_bf16_pooled_on_exact_values():
     p16 = oracle.index_pooled(qb, rows, bats, kb)
     np.testing.assert_array_equal(np.isnan(p8), np.isnan(p16))
     np.testing.assert_allclose(p8[~np.isnan(p8)], p16[~np.isnan(p16)], rtol=0, atol=0)
+
+
+# ----------------------------------------------------------------------------
+# token-level selection at the same budget ("MSA 稀疏注意力三国杀", section
+# "分歧一：颗粒度——token 级还是块级？"): top-2048 tokens by index score
+# ----------------------------------------------------------------------------
+def test_token_selection_within_budget_is_full_attention():
+    """With t + 1 <= 2048 every causal token is chosen: the lse equals the full
+    causal lse, and the output equals the all-blocks output of the block routine."""
+    rng = np.random.default_rng(45)
+    n, H, G = 1500, 4, 2
+    rows = np.array([0, 300, 1499], np.int64)
+    bats = np.zeros_like(rows)
+    q, k, v = _make_qkv(rng, 1, n, n, H, G)
+    q_idx = _rand_bits(rng, (len(rows), G, 64))
+    k_idx = _rand_bits(rng, (1, 1, n, 64))
+    toks, out, lse, lse_full = oracle.token_select_attention(q[0, rows], q_idx, rows, bats, k, v,
+                                                             k_idx, 1 / math.sqrt(128))
+    np.testing.assert_allclose(lse, lse_full, atol=1e-12)
+    sel = np.full((len(rows), G, 16), -1, np.int32)
+    for r, t in enumerate(rows):
+        sel[r, :, :t // BLOCK + 1] = np.arange(t // BLOCK + 1)
+        for g in range(G):
+            assert list(toks[r, g, :t + 1]) == list(range(t + 1)) and (toks[r, g, t + 1:] == -1).all()
+    o_blk, l_blk = oracle.attention(q[0, rows], rows, bats, k, v, sel, 1 / math.sqrt(128))
+    np.testing.assert_allclose(out, o_blk, atol=1e-12)
+    np.testing.assert_allclose(lse, l_blk, atol=1e-12)
+
+
+def test_token_selection_order_and_ties():
+    """Keys that are multiples of one vector rank by the multiple; equal scores go
+    to the lower token index (hand-derived sets for a budget of 5)."""
+    rng = np.random.default_rng(46)
+    n = 40
+    u = _rand_bits(rng, (64,))
+    qv = oracle.bits_to_f64(u)
+    mult = np.array([(j * 7) % 5 for j in range(n)], np.float32)   # 0..4, many ties
+    kf = (mult[:, None] * qv[None, :]).astype(np.float32)           # score = mult * |u|^2
+    k_idx = _bf16_round(kf)[None, None]
+    q_idx = np.broadcast_to(u, (1, 1, 64)).copy()
+    q, k, v = _make_qkv(rng, 1, n, n, 1, 1)
+    rows = np.array([39], np.int64)
+    toks, _, _, _ = oracle.token_select_attention(q[0, rows], q_idx, rows, np.zeros_like(rows), k, v,
+                                                  k_idx, 1 / math.sqrt(128), budget=5)
+    # mult 4 at j = 2, 7, 12, ...: the five lowest such indices
+    assert list(toks[0, 0]) == [2, 7, 12, 17, 22]
+    toks, _, _, _ = oracle.token_select_attention(q[0, [10]], q_idx, np.array([10]), np.array([0]), k,
+                                                  v, k_idx, 1 / math.sqrt(128), budget=5)
+    # keys 0..10: mult 4 at 2, 7; mult 3 at 4, 9; mult 2 at 1, 6: ties to the lower index
+    assert list(toks[0, 0]) == [1, 2, 4, 7, 9]
+
+
+def test_token_selection_of_whole_blocks_matches_block_attention():
+    """When the 2048 highest-scoring tokens are exactly 16 whole blocks, token-level
+    and block-level attention over them agree (two separate oracle routines)."""
+    rng = np.random.default_rng(47)
+    n, H, G = 3072, 2, 1
+    rows = np.array([3071], np.int64)                                 # own block 23 is full
+    bats = np.zeros_like(rows)
+    q, k, v = _make_qkv(rng, 1, n, n, H, G)
+    u = _rand_bits(rng, (64,))
+    blocks = [0, 2, 3, 5, 6, 7, 9, 10, 11, 12, 13, 15, 17, 18, 19, 23]
+    kf = rng.standard_normal((n, 64)).astype(np.float32) * 0.01
+    uf = oracle.bits_to_f64(u).astype(np.float32)
+    for c in blocks:
+        kf[c * 128:(c + 1) * 128] += 50.0 * uf
+    k_idx = _bf16_round(kf)[None, None]
+    q_idx = np.broadcast_to(u, (1, 1, 64)).copy()
+    toks, out, lse, _ = oracle.token_select_attention(q[0, rows], q_idx, rows, bats, k, v, k_idx,
+                                                      1 / math.sqrt(128))
+    expect = np.concatenate([np.arange(c * 128, (c + 1) * 128) for c in blocks])
+    np.testing.assert_array_equal(toks[0, 0], expect)
+    sel = np.array(blocks, np.int32)[None, None]
+    o_blk, l_blk = oracle.attention(q[0, rows], rows, bats, k, v, sel, 1 / math.sqrt(128))
+    np.testing.assert_allclose(out, o_blk, atol=1e-12)
+    np.testing.assert_allclose(lse, l_blk, atol=1e-12)
