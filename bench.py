@@ -307,6 +307,30 @@ def bench_recall(w, n_rows=64, reps=3):
     if int(buf.dev_err[0]) != 0:
         raise RuntimeError(f"device error {int(buf.dev_err[0])} in the recall measurement")
     ms = ev[0].elapsed_time(ev[1]) / reps
+    # token-level selection at the same key budget (2048 = 16 x 128) on the same
+    # rows: its captured share of each head's full attention mass,
+    # exp(lse_tokens - lse_full), against the block selection's recall
+    lse_full = torch.empty((n_rows, w.h_q), dtype=torch.float32, device="cuda")
+    pipeline.selection_recall(*args, lse_full=lse_full)
+    targs = (d, inp["q"], inp["k"], inp["v"], inp["q_idx"], inp["k_idx"], rows_d, 2048,
+             buf.dev_err)
+    pipeline.token_select_attention(*targs)
+    torch.cuda.synchronize()
+    ev[0].record()
+    for _ in range(reps):
+        _, _, lse_tok = pipeline.token_select_attention(*targs)
+    ev[1].record()
+    torch.cuda.synchronize()
+    if int(buf.dev_err[0]) != 0:
+        raise RuntimeError(f"device error {int(buf.dev_err[0])} in the token-level measurement")
+    ms_tok = ev[0].elapsed_time(ev[1]) / reps
+    tok_share = torch.exp(lse_tok.double() - lse_full.double())          # [n, H]
+    tok_rec = tok_share.view(n_rows, w.h_kv, -1).mean(dim=2)             # [n, G]
+    token_level = {"budget_tokens": 2048, "mean_recall": float(tok_rec.mean()),
+                   "min_recall": float(tok_rec.min()),
+                   "block_min_recall": float(rec.min()),
+                   "units_token_above_block": float((tok_rec > rec.double()).float().mean()),
+                   "ms": ms_tok}
     # every (row, group) streams its causal K and k_idx blocks into shared memory;
     # rows of one batch share those blocks, so DRAM sees each at most once
     nb = (w.q_pos0 + rows % w.n_q) // 128 + 1
@@ -317,7 +341,7 @@ def bench_recall(w, n_rows=64, reps=3):
            "mean_kl_teacher_student": float(kpq.mean()),
            "mean_kl_student_teacher": float(kqp.mean()), "ms": ms,
            "streamed_bytes": streamed, "streamed_gbs": streamed / (ms / 1000.0) / 1e9,
-           "dram_bytes_at_most": unique}
+           "dram_bytes_at_most": unique, "token_level": token_level}
     del buf, inp
     torch.cuda.empty_cache()
     return out

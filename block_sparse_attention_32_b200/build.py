@@ -21,7 +21,8 @@ LIB = os.path.join(OUT_DIR, "libmsa.so")
 OBJ_DIR = os.path.join(ROOT, "_build", "msa")
 
 SOURCES = ["msa_api.cu", "index_score.cu", "topk.cu", "block_lists.cu", "block_lists_noalloc.cu",
-           "sparse_attn.cu", "sparse_attn_decode.cu", "merge.cu", "recall.cu"]
+           "sparse_attn.cu", "sparse_attn_decode.cu", "merge.cu", "recall.cu",
+           "token_select.cu"]
 HEADERS = ["common.cuh"]
 
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",

@@ -75,12 +75,19 @@ def load_library(path: str) -> ctypes.CDLL:
     L.msa_selection_recall_workspace.argtypes = [_PD, ctypes.c_int64]
     L.msa_selection_recall_workspace.restype = ctypes.c_size_t
     L.msa_selection_recall.argtypes = [_PD, Tensor, Tensor, Tensor, Tensor, _P, _P, ctypes.c_int64,
-                                       _P, ctypes.c_int64, _P, _P, _P, _P, ctypes.c_size_t, _P, _P]
+                                       _P, ctypes.c_int64, _P, _P, _P, _P, _P, ctypes.c_size_t,
+                                       _P, _P]
+    L.msa_token_select_workspace.argtypes = [_PD, ctypes.c_int64]
+    L.msa_token_select_workspace.restype = ctypes.c_size_t
+    L.msa_token_select_attention.argtypes = [_PD, Tensor, Tensor, Tensor, Tensor, Tensor, _P,
+                                             ctypes.c_int64, ctypes.c_int64, _P, _P, _P, _P,
+                                             ctypes.c_size_t, _P, _P]
     L.msa_status_string.argtypes = [ctypes.c_int]
     L.msa_status_string.restype = ctypes.c_char_p
     for f in (L.msa_index_score_maxpool, L.msa_topk_blocks, L.msa_build_block_query_lists,
               L.msa_build_block_query_lists_noalloc, L.msa_sparse_attn_fwd, L.msa_merge_partials,
-              L.msa_selection_recall, L.msa_quantize_e4m3, L.msa_index_score_maxpool_e4m3):
+              L.msa_selection_recall, L.msa_quantize_e4m3, L.msa_index_score_maxpool_e4m3,
+              L.msa_token_select_attention):
         f.restype = ctypes.c_int
     return L
 
@@ -183,16 +190,35 @@ def msa_selection_recall_workspace(d: Dims, n_rows: int) -> int:
 
 
 def msa_selection_recall(d: Dims, q, k, q_idx, k_idx, sel, rows, block_mass, recall, kl_pq, kl_qp,
-                         ws, dev_err=None):
+                         ws, dev_err=None, lse_full=None):
     """Teacher block mass, recall and KL divergences for the sampled rows
-    (rows: int64 device tensor of b * n_q + qi; block_mass [n * G, >= nblk])."""
+    (rows: int64 device tensor of b * n_q + qi; block_mass [n * G, >= nblk]);
+    lse_full [n, H] (optional) receives each head's full causal log-normaliser."""
     nbytes = 0 if ws is None else ws.numel() * ws.element_size()
     _check("msa_selection_recall",
            lib().msa_selection_recall(ctypes.byref(d), tensor_btd(q), tensor_bhtd(k),
                                       tensor_btd(q_idx), tensor_bhtd(k_idx), _ptr(sel), _ptr(rows),
                                       rows.numel(), _ptr(block_mass), block_mass.stride(0),
-                                      _ptr(recall), _ptr(kl_pq), _ptr(kl_qp), _ptr(ws), nbytes,
-                                      _ptr(dev_err), _stream()))
+                                      _ptr(recall), _ptr(kl_pq), _ptr(kl_qp), _ptr(lse_full),
+                                      _ptr(ws), nbytes, _ptr(dev_err), _stream()))
+
+
+def msa_token_select_workspace(d: Dims, n_rows: int) -> int:
+    return int(lib().msa_token_select_workspace(ctypes.byref(d), n_rows))
+
+
+def msa_token_select_attention(d: Dims, q, k, v, q_idx, k_idx, rows, budget, tokens, out, lse, ws,
+                               dev_err=None):
+    """Top-budget tokens by index score per (sampled row, group) and attention
+    over them: tokens int32 [n, G, budget], out fp32 [n, H, 128], lse fp32 [n, H]."""
+    nbytes = 0 if ws is None else ws.numel() * ws.element_size()
+    assert tokens.dtype == torch.int32 and out.dtype == torch.float32 and lse.dtype == torch.float32
+    _check("msa_token_select_attention",
+           lib().msa_token_select_attention(ctypes.byref(d), tensor_btd(q), tensor_bhtd(k),
+                                            tensor_bhtd(v), tensor_btd(q_idx), tensor_bhtd(k_idx),
+                                            _ptr(rows), rows.numel(), budget, _ptr(tokens),
+                                            _ptr(out), _ptr(lse), _ptr(ws), nbytes,
+                                            _ptr(dev_err), _stream()))
 
 
 def tensor_u8(t: torch.Tensor, bhtd: bool) -> Tensor:

@@ -35,8 +35,16 @@ cudaError_t launch_selection_recall(const CUtensorMap&, const CUtensorMap&, cons
                                     const int64_t*, int64_t, const void*, int64_t, int64_t,
                                     int64_t, int64_t, int64_t, int64_t, int32_t, int32_t,
                                     int32_t, int32_t, int32_t, float, const int32_t*, float*,
-                                    int64_t, float*, float*, float*, void*, int32_t*,
+                                    int64_t, float*, float*, float*, float*, void*, int32_t*,
                                     cudaStream_t);
+size_t token_select_workspace(int64_t, int32_t, int64_t);
+cudaError_t launch_token_select_attention(const CUtensorMap&, const int64_t*, int64_t,
+                                          const void*, int64_t, int64_t, int64_t, const void*,
+                                          int64_t, int64_t, int64_t, const void*, int64_t,
+                                          int64_t, int64_t, const void*, int64_t, int64_t,
+                                          int64_t, int64_t, int64_t, int64_t, int64_t, int32_t,
+                                          int32_t, int32_t, int32_t, float, int64_t, int32_t*,
+                                          float*, float*, void*, int32_t*, cudaStream_t);
 cudaError_t launch_index_score_e4m3(const CUtensorMap&, const CUtensorMap&, int64_t, int64_t,
                                    int64_t, int32_t, int32_t, float*, int64_t, const float*,
                                    const float*, int32_t*, cudaStream_t);
@@ -374,7 +382,8 @@ size_t msa_selection_recall_workspace(const msa_dims* d, int64_t n_rows) {
 msa_status msa_selection_recall(const msa_dims* d, msa_tensor q, msa_tensor k, msa_tensor q_idx,
                                 msa_tensor k_idx, const int32_t* sel, const int64_t* rows,
                                 int64_t n_rows, float* block_mass, int64_t mass_stride,
-                                float* recall, float* kl_pq, float* kl_qp, void* ws,
+                                float* recall, float* kl_pq, float* kl_qp, float* lse_full,
+                                void* ws,
                                 size_t ws_bytes, int32_t* dev_err, void* stream) {
   msa_status s = check_dims(d);
   if (s != MSA_OK) return s;
@@ -409,8 +418,46 @@ msa_status msa_selection_recall(const msa_dims* d, msa_tensor q, msa_tensor k, m
   return from_cuda(msa::launch_selection_recall(
       tq, tk, tki, rows, n_rows, q_idx.ptr, q_idx.s_batch, q_idx.s_tok, q_idx.s_head, d->batch,
       d->n_q, d->q_pos0, d->h_kv, d->h_q, d->d_idx, d->h_kidx, (int32_t)nblk, d->scale, sel,
-      block_mass, mass_stride, recall, kl_pq, kl_qp, ws, dev_err,
+      block_mass, mass_stride, recall, kl_pq, kl_qp, lse_full, ws, dev_err,
       reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t msa_token_select_workspace(const msa_dims* d, int64_t n_rows) {
+  if (check_dims(d) != MSA_OK || n_rows < 0) return 0;
+  return msa::token_select_workspace(n_rows, d->h_kv, d->n_kv);
+}
+
+msa_status msa_token_select_attention(const msa_dims* d, msa_tensor q, msa_tensor k,
+                                      msa_tensor v, msa_tensor q_idx, msa_tensor k_idx,
+                                      const int64_t* rows, int64_t n_rows, int64_t budget,
+                                      int32_t* tokens, float* out, float* lse, void* ws,
+                                      size_t ws_bytes, int32_t* dev_err, void* stream) {
+  msa_status s = check_dims(d);
+  if (s != MSA_OK) return s;
+  if ((s = check_tensor(q)) != MSA_OK) return s;
+  if ((s = check_tensor(k)) != MSA_OK) return s;
+  if ((s = check_tensor(v)) != MSA_OK) return s;
+  if ((s = check_tensor(q_idx)) != MSA_OK) return s;
+  if ((s = check_tensor(k_idx)) != MSA_OK) return s;
+  if (n_rows < 0 || budget < 1 || budget > 0x7FFFFFFF) return MSA_ERR_INVALID_ARG;
+  if (n_rows == 0) return MSA_OK;
+  if (rows == nullptr || tokens == nullptr || out == nullptr || lse == nullptr || ws == nullptr)
+    return MSA_ERR_INVALID_ARG;
+  if (!aligned16(ws) || !aligned16(out)) return MSA_ERR_ALIGNMENT;
+  const int64_t R = d->h_q / d->h_kv;
+  if (R > 8) return MSA_ERR_UNSUPPORTED;            // heads are the 8-wide side of the tiles
+  if (n_rows * d->h_kv > 0x7FFFFFFF) return MSA_ERR_UNSUPPORTED;
+  if (ws_bytes < msa_token_select_workspace(d, n_rows)) return MSA_ERR_WORKSPACE_TOO_SMALL;
+  CUtensorMap tki;
+  // k_idx [B, h_kidx, n_kv, d_idx]: one 128-token block of 64 dims per box
+  if ((s = make_map(&tki, k_idx.ptr, d->d_idx, d->n_kv, d->h_kidx, d->batch, k_idx.s_tok,
+                    k_idx.s_head, k_idx.s_batch, 128, 1)) != MSA_OK)
+    return s;
+  return from_cuda(msa::launch_token_select_attention(
+      tki, rows, n_rows, q.ptr, q.s_batch, q.s_tok, q.s_head, q_idx.ptr, q_idx.s_batch,
+      q_idx.s_tok, q_idx.s_head, k.ptr, k.s_batch, k.s_tok, k.s_head, v.ptr, v.s_batch, v.s_tok,
+      v.s_head, d->batch, d->n_q, d->n_kv, d->q_pos0, d->h_kv, d->h_q, d->d_idx, d->h_kidx,
+      d->scale, budget, tokens, out, lse, ws, dev_err, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 const char* msa_status_string(msa_status s) {

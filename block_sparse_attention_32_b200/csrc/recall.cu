@@ -22,7 +22,8 @@
 //    mma.sync, heads as the 8-wide side) and the block's index score z(c)
 //    (k_idx times the index query, mma.sync with one live column);
 //  * recall_reduce_kernel -- one warp per (row, group): lse_h = log sum_c
-//    exp(a_h(c)), P(c) = mean_h exp(a_h(c) - lse_h), Q from z, recall, KL.
+//    exp(a_h(c)), P(c) = mean_h exp(a_h(c) - lse_h), Q from z, recall, KL,
+//    and (optionally) lse_h itself, the full causal attention's log-normaliser.
 #include "common.cuh"
 
 namespace msa {
@@ -231,7 +232,7 @@ __global__ void __launch_bounds__(256)
     recall_reduce_kernel(const RecallArgs a, int32_t R, const int32_t* __restrict__ sel,
                          float* __restrict__ block_mass, int64_t mass_stride,
                          float* __restrict__ recall, float* __restrict__ kl_pq,
-                         float* __restrict__ kl_qp) {
+                         float* __restrict__ kl_qp, float* __restrict__ lse_full) {
   const int lane = threadIdx.x & 31;
   const int64_t unit = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   if (unit >= a.n_rows * a.G) return;
@@ -296,6 +297,8 @@ __global__ void __launch_bounds__(256)
     recall[unit] = rc;
     kl_pq[unit] = kpq;
     kl_qp[unit] = kqp;
+    if (lse_full != nullptr)                       // [n_rows, H], head g R + h
+      for (int h = 0; h < R; ++h) lse_full[unit * R + h] = lse[h];
   }
 }
 
@@ -323,8 +326,8 @@ cudaError_t launch_selection_recall(const CUtensorMap& tm_q, const CUtensorMap& 
                                     int32_t h_kidx,
                                     int32_t nblk, float scale, const int32_t* sel,
                                     float* block_mass, int64_t mass_stride, float* recall,
-                                    float* kl_pq, float* kl_qp, void* ws, int32_t* err,
-                                    cudaStream_t st) {
+                                    float* kl_pq, float* kl_qp, float* lse_full, void* ws,
+                                    int32_t* err, cudaStream_t st) {
   if (n_rows == 0) return cudaSuccess;
   const int32_t R = H / G;
   RecallArgs a;
@@ -356,7 +359,7 @@ cudaError_t launch_selection_recall(const CUtensorMap& tm_q, const CUtensorMap& 
   if (e != cudaSuccess) return e;
   const int64_t threads = n_rows * G * 32;
   recall_reduce_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(
-      a, R, sel, block_mass, mass_stride, recall, kl_pq, kl_qp);
+      a, R, sel, block_mass, mass_stride, recall, kl_pq, kl_qp, lse_full);
   return cudaGetLastError();
 }
 

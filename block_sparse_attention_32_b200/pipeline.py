@@ -110,9 +110,10 @@ def forward(buf: Buffers, q, k, v, q_idx, k_idx):
     return buf.out, buf.lse
 
 
-def selection_recall(buf: Buffers, q, k, q_idx, k_idx, rows):
+def selection_recall(buf: Buffers, q, k, q_idx, k_idx, rows, lse_full=None):
     """For sampled rows (int64 device tensor of b * n_q + qi): the main branch's
-    block mass [n, G, nblk], the recall of buf.sel and KL(P||Q), KL(Q||P) [n, G]."""
+    block mass [n, G, nblk], the recall of buf.sel and KL(P||Q), KL(Q||P) [n, G].
+    A given lse_full [n, H] fp32 receives each head's full causal log-normaliser."""
     d = buf.dims
     n, G = rows.numel(), d.h_kv
     nblk = capi.msa_num_blocks(d)
@@ -124,8 +125,24 @@ def selection_recall(buf: Buffers, q, k, q_idx, k_idx, rows):
     ws_bytes = capi.msa_selection_recall_workspace(d, n)
     ws = torch.empty(((ws_bytes + 15) // 16 * 4,), dtype=torch.int32, device=dev)
     capi.msa_selection_recall(d, q, k, q_idx, k_idx, buf.sel, rows, mass.view(n * G, nblk), rec,
-                              kpq, kqp, ws, buf.dev_err)
+                              kpq, kqp, ws, buf.dev_err, lse_full=lse_full)
     return mass, rec, kpq, kqp
+
+
+def token_select_attention(d, q, k, v, q_idx, k_idx, rows, budget=2048, dev_err=None):
+    """Token-level selection at the same key budget for sampled rows: tokens
+    int32 [n, G, budget] (ascending, -1 padded), out fp32 [n, H, 128] and lse
+    fp32 [n, H] of the attention over them."""
+    n, G, H = rows.numel(), d.h_kv, d.h_q
+    dev = rows.device
+    tokens = torch.empty((n, G, budget), dtype=torch.int32, device=dev)
+    out = torch.empty((n, H, 128), dtype=torch.float32, device=dev)
+    lse = torch.empty((n, H), dtype=torch.float32, device=dev)
+    ws_bytes = capi.msa_token_select_workspace(d, n)
+    ws = torch.empty(((ws_bytes + 15) // 16 * 4,), dtype=torch.int32, device=dev)
+    capi.msa_token_select_attention(d, q, k, v, q_idx, k_idx, rows, budget, tokens, out, lse, ws,
+                                    dev_err)
+    return tokens, out, lse
 
 
 INPUT_NAMES = ("q", "k", "v", "q_idx", "k_idx")

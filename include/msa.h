@@ -241,7 +241,9 @@ MSA_API msa_status msa_index_score_maxpool_e4m3(const msa_dims* dims, msa_tensor
  *   recall = sum of P over the blocks sel[b, g, qi, :] selects
  *   kl_pq = sum_c P log(P / Q), kl_qp = sum_c Q log(Q / P)
  * Outputs (device, fp32): block_mass [n_rows, G, mass_stride] (P, 0 beyond the
- * causal blocks), recall, kl_pq, kl_qp [n_rows, G].  rows: device int64
+ * causal blocks), recall, kl_pq, kl_qp [n_rows, G], and, when lse_full is not
+ * NULL, lse_full [n_rows, H]: each head's log sum_{j <= t} exp(scale * q.k_j),
+ * the full causal attention's log-normaliser.  rows: device int64
  * [n_rows]; sel: [B, G, n_q, 16] as from msa_topk_blocks.  Needs R = h_q/h_kv
  * <= 8 (else MSA_ERR_UNSUPPORTED), mass_stride >= the block count, and a
  * device workspace of msa_selection_recall_workspace(dims, n_rows) bytes
@@ -251,8 +253,35 @@ MSA_API msa_status msa_selection_recall(const msa_dims* dims, msa_tensor q, msa_
                                         msa_tensor q_idx, msa_tensor k_idx,
                                         const int32_t* sel, const int64_t* rows, int64_t n_rows,
                                         float* block_mass, int64_t mass_stride, float* recall,
-                                        float* kl_pq, float* kl_qp, void* ws, size_t ws_bytes,
-                                        int32_t* dev_err, void* stream);
+                                        float* kl_pq, float* kl_qp, float* lse_full, void* ws,
+                                        size_t ws_bytes, int32_t* dev_err, void* stream);
+
+/* Token-level selection at the same key budget, for sampled query rows: the
+ * selection granularity the pages set against MSA's 128-token blocks ("MSA 稀疏
+ * 注意力三国杀" page, section "分歧一：颗粒度——token 级还是块级？"; "稀疏注意力速览"
+ * page, section 4; "Sparse attention · DSA và MSA chọn vị trí" page), here with
+ * MSA's own index branch as the scorer.  For sampled row rows[i] = b * n_q + qi
+ * (position t = q_pos0 + qi) and group g:
+ *   score(j) = q_idx[b, qi, g] . k_idx[b, g or 0, j] for every key j <= t (fp32),
+ *   T = the min(budget, t + 1) keys of highest score, the lower index first
+ *       among equal scores, written ascending to tokens[i, g, :] (int32,
+ *       [n_rows, G, budget], -1 after the last),
+ *   out[i, h] = sum_{j in T} softmax_{j in T}(scale * q_h.k_j) v_j and
+ *   lse[i, h] = log sum_{j in T} exp(scale * q_h.k_j) for the group's heads h
+ *   (device fp32, [n_rows, H, 128] and [n_rows, H]).
+ * exp(lse - lse_full) (lse_full from msa_selection_recall) is the share of the
+ * full attention mass the tokens hold, the token-level counterpart of recall.
+ * budget >= 1 (2048 spends the 16 x 128 keys of the block selection); R =
+ * h_q/h_kv <= 8 (else MSA_ERR_UNSUPPORTED); a device workspace of
+ * msa_token_select_workspace(dims, n_rows) bytes (16-byte aligned; it holds
+ * the score rows).  A row outside [0, B * n_q) sets MSA_DEVERR_BAD_ENTRY. */
+MSA_API size_t msa_token_select_workspace(const msa_dims* dims, int64_t n_rows);
+MSA_API msa_status msa_token_select_attention(const msa_dims* dims, msa_tensor q, msa_tensor k,
+                                              msa_tensor v, msa_tensor q_idx, msa_tensor k_idx,
+                                              const int64_t* rows, int64_t n_rows,
+                                              int64_t budget, int32_t* tokens, float* out,
+                                              float* lse, void* ws, size_t ws_bytes,
+                                              int32_t* dev_err, void* stream);
 
 /* Human-readable name of a status code (static storage). */
 MSA_API const char* msa_status_string(msa_status status);
