@@ -24,6 +24,9 @@ Each function cites the page passage it follows in ``msa_oracle.c``:
   * ``token_select_attention`` -- the token-level variant at the same
     budget: top-2048 tokens by index score, attention over them, and the full
     causal attention's lse;
+  * ``attention_bwd`` -- gradients dQ, dK, dV of the main branch's attention
+    over a fixed selection, for sparse training (section "MSA 能力不掉：3T token
+    对照实验": MSA-PT and MSA-CPT train through the sparse attention);
   * ``selection_recall`` -- the main branch's attention mass per block (the
     teacher), the recall of the chosen blocks and the KL divergences to the
     index branch's block softmax (section "索引分支训练：KL 对齐").
@@ -84,13 +87,15 @@ def _load():
             lib.msa_oracle_token_select_attention.argtypes = [I64, I32, I32, I32, I64, I32, I64,
                                                               P, P, P, P, P, P, P, F64, P, P,
                                                               P, P]
+            lib.msa_oracle_attention_bwd.argtypes = [I64, I64, I64, I64, I32, I32, P, P, P, P, P,
+                                                     F64, P, P, P, P, P]
             lib.msa_oracle_selection_recall.argtypes = [I64, I32, I32, I32, I64, I32, P, P, P, P,
                                                          P, P, P, F64, I64, P, P, P, P]
             for f in (lib.msa_oracle_index_pooled, lib.msa_oracle_topk, lib.msa_oracle_topk_f32,
                       lib.msa_oracle_attention, lib.msa_oracle_merge,
                       lib.msa_oracle_block_query_lists, lib.msa_oracle_selection_recall,
                       lib.msa_oracle_quantize_e4m3, lib.msa_oracle_index_pooled_e4m3,
-                      lib.msa_oracle_token_select_attention):
+                      lib.msa_oracle_token_select_attention, lib.msa_oracle_attention_bwd):
                 f.restype = None
             _lib = lib
     return _lib
@@ -313,3 +318,29 @@ def token_select_attention(q_rows, q_idx_rows, row_pos, row_batch, k, v, k_idx, 
                                           _p(pos), _p(bat), _p(kk), _p(vv), _p(ki), float(scale),
                                           _p(tokens), _p(out), _p(lse), _p(lse_full))
     return tokens, out, lse, lse_full
+
+
+def attention_bwd(q, k, v, dout, sel, scale, q_pos0=0):
+    """Gradients of the sparse attention for an upstream dout, the selection
+    fixed.  q, dout [B, n_q, H, 128]; k, v [B, G, n_kv, 128] (float64 arrays,
+    or bf16 bit patterns as uint16, converted exactly); sel [B, G, n_q, 16]
+    int32.  Returns dq [B, n_q, H, 128], dk, dv [B, G, n_kv, 128], lse and
+    delta = dO.o [B, n_q, H], all float64."""
+    lib = _load()
+
+    def f64(a):
+        return _c(bits_to_f64(a) if a.dtype == np.uint16 else a, np.float64)
+
+    qq, kk, vv, do = f64(q), f64(k), f64(v), f64(dout)
+    ss = _c(sel, np.int32)
+    B, n_q, H, _ = qq.shape
+    G, n_kv = kk.shape[1], kk.shape[2]
+    assert ss.shape == (B, G, n_q, TOPK) and do.shape == qq.shape and vv.shape == kk.shape
+    dq = np.empty_like(qq)
+    dk = np.empty_like(kk)
+    dv = np.empty_like(vv)
+    lse = np.empty((B, n_q, H), np.float64)
+    delta = np.empty((B, n_q, H), np.float64)
+    lib.msa_oracle_attention_bwd(B, n_q, n_kv, int(q_pos0), H, G, _p(qq), _p(kk), _p(vv), _p(do),
+                                 _p(ss), float(scale), _p(dq), _p(dk), _p(dv), _p(lse), _p(delta))
+    return dq, dk, dv, lse, delta

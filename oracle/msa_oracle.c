@@ -570,3 +570,131 @@ void msa_oracle_token_select_attention(int64_t n_rows, int32_t H, int32_t G, int
     }
   }
 }
+
+/* ---------------------------------------------------------------------- */
+/* Backward of step 4 for sparse training ([P1] section "MSA 能力不掉：3T    */
+/* token 对照实验": a model trained with MSA from the start (MSA-PT) and a   */
+/* dense model converted by continued training (MSA-CPT), both of which    */
+/* back-propagate through the main branch; [P1] section "索引分支训练：KL    */
+/* 对齐": the index branch learns only through its own KL term, so the top-k */
+/* selection is a fixed input here and carries no gradient).               */
+/*                                                                        */
+/* The gradients of o = sum_j p_j v_j, p = softmax_j(scale q.k_j) over the  */
+/* selected causal tokens J(t, g) of the forward, for an upstream dO:      */
+/*   dP_j = dO.v_j,  D = sum_j p_j dP_j (= dO.o),  dS_j = p_j (dP_j - D),   */
+/*   dQ = scale sum_j dS_j k_j,  dK_j += scale dS_j q,  dV_j += p_j dO,     */
+/* summed over every (query, head) whose token set holds j.                */
+/* Inputs are doubles so that the finite-difference pins can perturb them; */
+/* bf16 callers convert exactly.  All arrays contiguous:                   */
+/*   q, dout, dq [B, n_q, H, 128];  k, v, dk, dv [B, G, n_kv, 128];         */
+/*   sel [B, G, n_q, 16] (-1 = unused slot); query i sits at t = q_pos0+i. */
+/* Two passes, each over independent units: (1) per (batch, query, head):  */
+/* lse, D and dQ; (2) per (batch, group, KV block c): dK and dV of c's     */
+/* tokens, summed over the queries that selected c in ascending order and  */
+/* over the group's heads.                                                 */
+/* ---------------------------------------------------------------------- */
+static int32_t bwd_tokens(const int32_t* srow, int64_t t, int64_t n_kv, int64_t* tok) {
+  int32_t n = 0;
+  for (int32_t s = 0; s < MSA_TOPK; ++s) {
+    const int32_t c = srow[s];
+    if (c < 0) continue;
+    for (int64_t j = (int64_t)c * MSA_BLOCK; j < (int64_t)(c + 1) * MSA_BLOCK; ++j) {
+      if (j > t || j >= n_kv) break;
+      tok[n++] = j;
+    }
+  }
+  return n;
+}
+
+static double dot128(const double* a, const double* b) {
+  double s = 0.0;
+  for (int32_t d = 0; d < MSA_HEAD_DIM; ++d) s += a[d] * b[d];
+  return s;
+}
+
+void msa_oracle_attention_bwd(int64_t B, int64_t n_q, int64_t n_kv, int64_t q_pos0, int32_t H,
+                              int32_t G, const double* q, const double* k, const double* v,
+                              const double* dout, const int32_t* sel, double scale,
+                              double* dq, double* dk, double* dv,
+                              double* lse_out, double* delta_out) /* [B, n_q, H] each */
+{
+  const int32_t R = H / G;
+  const int64_t nblk = (n_kv + MSA_BLOCK - 1) / MSA_BLOCK;
+  /* pass 1: per (b, i, h) */
+#pragma omp parallel for collapse(3) schedule(dynamic, 16)
+  for (int64_t b = 0; b < B; ++b) {
+    for (int64_t i = 0; i < n_q; ++i) {
+      for (int32_t h = 0; h < H; ++h) {
+        const int64_t t = q_pos0 + i;
+        const int32_t g = h / R;
+        const int64_t row = (b * n_q + i) * H + h;
+        const double* qh = q + row * MSA_HEAD_DIM;
+        const double* doh = dout + row * MSA_HEAD_DIM;
+        const double* kb = k + (b * G + g) * n_kv * MSA_HEAD_DIM;
+        const double* vb = v + (b * G + g) * n_kv * MSA_HEAD_DIM;
+        int64_t tok[MSA_TOPK * MSA_BLOCK];
+        double s[MSA_TOPK * MSA_BLOCK], p[MSA_TOPK * MSA_BLOCK], dp[MSA_TOPK * MSA_BLOCK];
+        const int32_t n = bwd_tokens(sel + ((b * G + g) * n_q + i) * MSA_TOPK, t, n_kv, tok);
+        double m = -INFINITY;
+        for (int32_t a = 0; a < n; ++a) {
+          s[a] = scale * dot128(qh, kb + tok[a] * MSA_HEAD_DIM);
+          if (s[a] > m) m = s[a];
+        }
+        double l = 0.0;
+        for (int32_t a = 0; a < n; ++a) l += exp(s[a] - m);
+        const double lse = m + log(l);
+        double D = 0.0;
+        for (int32_t a = 0; a < n; ++a) {
+          p[a] = exp(s[a] - lse);
+          dp[a] = dot128(doh, vb + tok[a] * MSA_HEAD_DIM);
+          D += p[a] * dp[a];
+        }
+        double* dqh = dq + row * MSA_HEAD_DIM;
+        for (int32_t d = 0; d < MSA_HEAD_DIM; ++d) dqh[d] = 0.0;
+        for (int32_t a = 0; a < n; ++a) {
+          const double ds = p[a] * (dp[a] - D);
+          const double* kj = kb + tok[a] * MSA_HEAD_DIM;
+          for (int32_t d = 0; d < MSA_HEAD_DIM; ++d) dqh[d] += scale * ds * kj[d];
+        }
+        lse_out[row] = lse;
+        delta_out[row] = D;
+      }
+    }
+  }
+  /* pass 2: per (b, g, c) */
+#pragma omp parallel for collapse(3) schedule(dynamic, 1)
+  for (int64_t b = 0; b < B; ++b) {
+    for (int32_t g = 0; g < G; ++g) {
+      for (int64_t c = 0; c < nblk; ++c) {
+        const int64_t j0 = c * MSA_BLOCK;
+        const int64_t j1 = (j0 + MSA_BLOCK < n_kv) ? j0 + MSA_BLOCK : n_kv;
+        const double* kb = k + (b * G + g) * n_kv * MSA_HEAD_DIM;
+        const double* vb = v + (b * G + g) * n_kv * MSA_HEAD_DIM;
+        double* dkb = dk + (b * G + g) * n_kv * MSA_HEAD_DIM;
+        double* dvb = dv + (b * G + g) * n_kv * MSA_HEAD_DIM;
+        for (int64_t j = j0; j < j1; ++j)
+          for (int32_t d = 0; d < MSA_HEAD_DIM; ++d) dkb[j * MSA_HEAD_DIM + d] = dvb[j * MSA_HEAD_DIM + d] = 0.0;
+        for (int64_t i = 0; i < n_q; ++i) {
+          const int64_t t = q_pos0 + i;
+          const int32_t* srow = sel + ((b * G + g) * n_q + i) * MSA_TOPK;
+          int chosen = 0;
+          for (int32_t s2 = 0; s2 < MSA_TOPK; ++s2) chosen |= (srow[s2] == (int32_t)c);
+          if (!chosen || j0 > t) continue;
+          for (int32_t r = 0; r < R; ++r) {
+            const int64_t row = (b * n_q + i) * H + g * R + r;
+            const double* qh = q + row * MSA_HEAD_DIM;
+            const double* doh = dout + row * MSA_HEAD_DIM;
+            for (int64_t j = j0; j < j1 && j <= t; ++j) {
+              const double pj = exp(scale * dot128(qh, kb + j * MSA_HEAD_DIM) - lse_out[row]);
+              const double ds = pj * (dot128(doh, vb + j * MSA_HEAD_DIM) - delta_out[row]);
+              for (int32_t d = 0; d < MSA_HEAD_DIM; ++d) {
+                dkb[j * MSA_HEAD_DIM + d] += scale * ds * qh[d];
+                dvb[j * MSA_HEAD_DIM + d] += pj * doh[d];
+              }
+            }
+          }
+        }
+      }
+    }
+  }
+}

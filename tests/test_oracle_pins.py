@@ -571,3 +571,142 @@ def test_token_selection_of_whole_blocks_matches_block_attention():
     o_blk, l_blk = oracle.attention(q[0, rows], rows, bats, k, v, sel, 1 / math.sqrt(128))
     np.testing.assert_allclose(out, o_blk, atol=1e-12)
     np.testing.assert_allclose(lse, l_blk, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# backward of the main branch (sparse training: "MSA 稀疏注意力三国杀", section
+# "MSA 能力不掉：3T token 对照实验"; the selection is a fixed input)
+# ---------------------------------------------------------------------------
+def _bwd_problem(seed, B, n_q, n_kv, q_pos0, H, G, sparse):
+    """Random fp64 inputs and a selection: every causal block when not sparse,
+    otherwise the own block plus up to 15 random earlier ones."""
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((B, n_q, H, 128))
+    k = rng.standard_normal((B, G, n_kv, 128))
+    v = rng.standard_normal((B, G, n_kv, 128))
+    do = rng.standard_normal((B, n_q, H, 128))
+    sel = np.full((B, G, n_q, 16), -1, np.int32)
+    for b in range(B):
+        for g in range(G):
+            for i in range(n_q):
+                own = (q_pos0 + i) // BLOCK
+                cands = np.arange(own)
+                if sparse and own > 15:
+                    cands = np.sort(rng.choice(own, size=15, replace=False))
+                blocks = np.concatenate([cands, [own]]).astype(np.int32)
+                sel[b, g, i, :len(blocks)] = np.sort(blocks)
+    return q, k, v, do, sel
+
+
+def _torch_masked_grads(q, k, v, do, sel, scale, q_pos0):
+    """Gradients by autograd of dense attention in float64 with the mask that
+    admits exactly the selected causal tokens (GQA: head h reads KV head h // R)."""
+    import torch
+    B, n_q, H, _ = q.shape
+    G, n_kv = k.shape[1], k.shape[2]
+    R = H // G
+    tq = torch.tensor(q, requires_grad=True)
+    tk = torch.tensor(k, requires_grad=True)
+    tv = torch.tensor(v, requires_grad=True)
+    allowed = np.zeros((B, G, n_q, n_kv), bool)
+    j = np.arange(n_kv)
+    for b in range(B):
+        for g in range(G):
+            for i in range(n_q):
+                blk = sel[b, g, i][sel[b, g, i] >= 0]
+                allowed[b, g, i] = np.isin(j // BLOCK, blk) & (j <= q_pos0 + i)
+    kk = tk.repeat_interleave(R, dim=1)                       # [B, H, n_kv, 128]
+    vv = tv.repeat_interleave(R, dim=1)
+    s = torch.einsum("bihd,bhjd->bhij", tq, kk) * scale
+    mask = torch.tensor(np.repeat(allowed, R, axis=1))
+    s = s.masked_fill(~mask, float("-inf"))
+    o = torch.einsum("bhij,bhjd->bihd", torch.softmax(s, dim=-1), vv)
+    (o * torch.tensor(do)).sum().backward()
+    return tq.grad.numpy(), tk.grad.numpy(), tv.grad.numpy(), o.detach().numpy()
+
+
+@pytest.mark.parametrize("sparse,q_pos0,n_q,n_kv", [(False, 0, 600, 600), (False, 300, 300, 600),
+                                                    (True, 0, 2300, 2300)],
+                         ids=["dense", "chunk_after_cache", "sparse_selection"])
+def test_attention_bwd_matches_autograd(sparse, q_pos0, n_q, n_kv):
+    """dQ, dK, dV equal autograd's gradients of dense fp64 attention masked to
+    the selected causal tokens (with a full selection: plain causal attention)."""
+    scale = 1.0 / math.sqrt(128)
+    q, k, v, do, sel = _bwd_problem(41, 1, n_q, n_kv, q_pos0, 4, 2, sparse)
+    dq, dk, dv, lse, delta = oracle.attention_bwd(q, k, v, do, sel, scale, q_pos0)
+    gq, gk, gv, o = _torch_masked_grads(q, k, v, do, sel, scale, q_pos0)
+    for mine, ref in ((dq, gq), (dk, gk), (dv, gv)):
+        assert np.abs(mine - ref).max() <= 1e-10 * max(1.0, np.abs(ref).max())
+    np.testing.assert_allclose(delta, np.einsum("bihd,bihd->bih", do, o), atol=1e-10)
+
+
+def test_attention_bwd_finite_differences():
+    """Central differences of L = sum(dO * o) along random directions of q, k
+    and v agree with <grad, direction> (sparse selection, two batches)."""
+    import torch
+    scale = 0.1
+    q, k, v, do, sel = _bwd_problem(43, 2, 2200, 2200, 0, 2, 1, True)
+    dq, dk, dv, _, _ = oracle.attention_bwd(q, k, v, do, sel, scale)
+    rng = np.random.default_rng(44)
+
+    def loss(qq, kk, vv):
+        # the forward through the same masked formulation, no autograd
+        with torch.no_grad():
+            _, _, _, o = _torch_masked_grads_fwd(qq, kk, vv, sel, scale)
+        return float((o * do).sum())
+
+    for which, grad in ((0, dq), (1, dk), (2, dv)):
+        direc = rng.standard_normal(grad.shape)
+        eps = 1e-5
+        args_p = [q, k, v]
+        args_m = [q, k, v]
+        args_p[which] = args_p[which] + eps * direc
+        args_m[which] = args_m[which] - eps * direc
+        fd = (loss(*args_p) - loss(*args_m)) / (2 * eps)
+        an = float((grad * direc).sum())
+        assert abs(fd - an) <= 1e-6 * max(1.0, abs(an)), (which, fd, an)
+
+
+def _torch_masked_grads_fwd(q, k, v, sel, scale):
+    import torch
+    B, n_q, H, _ = q.shape
+    G, n_kv = k.shape[1], k.shape[2]
+    R = H // G
+    j = np.arange(n_kv)
+    allowed = np.zeros((B, G, n_q, n_kv), bool)
+    for b in range(B):
+        for g in range(G):
+            for i in range(n_q):
+                blk = sel[b, g, i][sel[b, g, i] >= 0]
+                allowed[b, g, i] = np.isin(j // BLOCK, blk) & (j <= i)
+    kk = torch.tensor(k).repeat_interleave(R, dim=1)
+    vv = torch.tensor(v).repeat_interleave(R, dim=1)
+    s = torch.einsum("bihd,bhjd->bhij", torch.tensor(q), kk) * scale
+    s = s.masked_fill(~torch.tensor(np.repeat(allowed, R, axis=1)), float("-inf"))
+    o = torch.einsum("bhij,bhjd->bihd", torch.softmax(s, dim=-1), vv)
+    return None, None, None, o.numpy()
+
+
+def test_attention_bwd_invariants_and_first_query():
+    """Per (batch, group): sum_j dK_j = 0 (each row's dS sums to zero) and
+    sum_j dV_j = sum of dO over the group's heads and queries (each row's
+    weights sum to one); the first query sees one token, so its dQ is zero."""
+    scale = 1.0 / math.sqrt(128)
+    q, k, v, do, sel = _bwd_problem(45, 2, 2100, 2100, 0, 8, 2, True)
+    dq, dk, dv, _, _ = oracle.attention_bwd(q, k, v, do, sel, scale)
+    R = 4
+    for b in range(2):
+        for g in range(2):
+            assert np.abs(dk[b, g].sum(axis=0)).max() <= 1e-9 * np.abs(dk[b, g]).sum(axis=0).max()
+            want = do[b, :, g * R:(g + 1) * R].sum(axis=(0, 1))
+            np.testing.assert_allclose(dv[b, g].sum(axis=0), want, rtol=1e-10, atol=1e-9)
+    assert np.abs(dq[:, 0]).max() == 0.0
+    # keys no query selected get no gradient
+    picked = np.zeros((2, 2, 2100 // BLOCK + 1), bool)
+    for b in range(2):
+        for g in range(2):
+            picked[b, g, np.unique(sel[b, g][sel[b, g] >= 0])] = True
+    for b in range(2):
+        for g in range(2):
+            for c in np.nonzero(~picked[b, g])[0]:
+                assert not dk[b, g, c * BLOCK:(c + 1) * BLOCK].any()
