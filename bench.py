@@ -347,6 +347,38 @@ def bench_recall(w, n_rows=64, reps=3):
     return out
 
 
+def bench_backward(w, attn_flops, reps=3):
+    """The attention's backward (dq, dk, dv for a seeded upstream gradient,
+    selection fixed by the forward) on the workload: its time, and TFLOP/s
+    over the five products per (row, head, selected causal token) -- S, dP,
+    dV, dK and dQ, 2.5x the forward's two."""
+    from block_sparse_attention_32_b200 import pipeline, workloads as wl
+    d = pipeline.dims_for(w)
+    buf = pipeline.Buffers.allocate(d)
+    grads = pipeline.Grads.allocate(d)
+    inp = wl.make_inputs(w, "cuda")
+    d_out = wl.upstream_grad(w, "cuda")
+    pipeline.forward(buf, inp["q"], inp["k"], inp["v"], inp["q_idx"], inp["k_idx"])
+    args = (buf, grads, inp["q"], inp["k"], inp["v"], d_out)
+    pipeline.backward(*args)
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    ev[0].record()
+    for _ in range(reps):
+        pipeline.backward(*args)
+    ev[1].record()
+    torch.cuda.synchronize()
+    if int(buf.dev_err[0]) != 0:
+        raise RuntimeError(f"device error {int(buf.dev_err[0])} in the backward measurement")
+    ms = ev[0].elapsed_time(ev[1]) / reps
+    flops = 2.5 * attn_flops
+    out = {"workload": w.name, "ms": ms, "tflops": flops / (ms / 1000.0) / 1e12,
+           "algorithmic_flops": flops, "kernels": "mma.sync m16n8k16 (bf16, fp32 accumulate)"}
+    del buf, grads, inp, d_out
+    torch.cuda.empty_cache()
+    return out
+
+
 def bench_e2e(w, buf, dev_inp, steps, world):
     """The pass through the public API with host buffers: every step uploads its
     inputs from pinned host memory, runs the five calls and downloads the output
@@ -440,6 +472,7 @@ def main():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-recall", action="store_true")
     ap.add_argument("--no-e4m3", action="store_true")
+    ap.add_argument("--no-bwd", action="store_true")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -517,6 +550,7 @@ def main():
     if not args.no_recall:
         recall = bench_recall(w)
     e4m3 = None if args.no_e4m3 else bench_e4m3(w)
+    backward = None if args.no_bwd else bench_backward(w, attn_flops)
 
     # dominant kernel: the longest stage; its bound is the larger of its
     # algorithmic time at the tensor peak and at the HBM peak
@@ -562,6 +596,7 @@ def main():
         "decode": decode,
         "selection_recall": recall,
         "index_e4m3": e4m3,
+        "backward": backward,
         "roofline": roof,
         "clocks": clocks,
         "gpu_launches": args.steps * sum(pipeline_launches().values()),

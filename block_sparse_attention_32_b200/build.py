@@ -22,7 +22,7 @@ OBJ_DIR = os.path.join(ROOT, "_build", "msa")
 
 SOURCES = ["msa_api.cu", "index_score.cu", "topk.cu", "block_lists.cu", "block_lists_noalloc.cu",
            "sparse_attn.cu", "sparse_attn_decode.cu", "merge.cu", "recall.cu",
-           "token_select.cu"]
+           "token_select.cu", "sparse_attn_bwd.cu"]
 HEADERS = ["common.cuh"]
 
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",

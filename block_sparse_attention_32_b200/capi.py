@@ -77,6 +77,8 @@ def load_library(path: str) -> ctypes.CDLL:
     L.msa_selection_recall.argtypes = [_PD, Tensor, Tensor, Tensor, Tensor, _P, _P, ctypes.c_int64,
                                        _P, ctypes.c_int64, _P, _P, _P, _P, _P, ctypes.c_size_t,
                                        _P, _P]
+    L.msa_sparse_attn_bwd.argtypes = [_PD, Tensor, Tensor, Tensor, Tensor, Tensor, _P, _P, _P,
+                                      _P, _P, _P, _P, _P, _P, _P]
     L.msa_token_select_workspace.argtypes = [_PD, ctypes.c_int64]
     L.msa_token_select_workspace.restype = ctypes.c_size_t
     L.msa_token_select_attention.argtypes = [_PD, Tensor, Tensor, Tensor, Tensor, Tensor, _P,
@@ -87,7 +89,7 @@ def load_library(path: str) -> ctypes.CDLL:
     for f in (L.msa_index_score_maxpool, L.msa_topk_blocks, L.msa_build_block_query_lists,
               L.msa_build_block_query_lists_noalloc, L.msa_sparse_attn_fwd, L.msa_merge_partials,
               L.msa_selection_recall, L.msa_quantize_e4m3, L.msa_index_score_maxpool_e4m3,
-              L.msa_token_select_attention):
+              L.msa_token_select_attention, L.msa_sparse_attn_bwd):
         f.restype = ctypes.c_int
     return L
 
@@ -177,6 +179,19 @@ def msa_sparse_attn_fwd(d: Dims, q, k, v, blk_offsets, entries, part_ml, part_ac
            lib().msa_sparse_attn_fwd(ctypes.byref(d), tensor_btd(q), tensor_bhtd(k),
                                      tensor_bhtd(v), _ptr(blk_offsets), _ptr(entries),
                                      _ptr(part_ml), _ptr(part_acc), _ptr(dev_err), _stream()))
+
+
+def msa_sparse_attn_bwd(d: Dims, q, k, v, o, d_o, lse, blk_offsets, entries, delta, part_dq, dq,
+                        dk, dv, dev_err=None):
+    """dq [B,n_q,H,128], dk/dv [B,G,n_kv,128] (fp32) for upstream d_o (bf16)."""
+    for t in (delta, part_dq, dq, dk, dv):
+        assert t.dtype == torch.float32 and t.is_contiguous()
+    _check("msa_sparse_attn_bwd",
+           lib().msa_sparse_attn_bwd(ctypes.byref(d), tensor_btd(q), tensor_bhtd(k),
+                                     tensor_bhtd(v), tensor_btd(o), tensor_btd(d_o), _ptr(lse),
+                                     _ptr(blk_offsets), _ptr(entries), _ptr(delta),
+                                     _ptr(part_dq), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dev_err),
+                                     _stream()))
 
 
 def msa_merge_partials(d: Dims, sel, part_ml, part_acc, out, lse, dev_err=None):

@@ -37,6 +37,12 @@ cudaError_t launch_selection_recall(const CUtensorMap&, const CUtensorMap&, cons
                                     int32_t, int32_t, int32_t, float, const int32_t*, float*,
                                     int64_t, float*, float*, float*, float*, void*, int32_t*,
                                     cudaStream_t);
+cudaError_t launch_sparse_attn_bwd(const CUtensorMap&, const CUtensorMap&, const void*, int64_t,
+                                   int64_t, int64_t, const void*, int64_t, int64_t, int64_t,
+                                   const void*, int64_t, int64_t, int64_t, const float*,
+                                   const int32_t*, const int32_t*, int64_t, int64_t, int64_t,
+                                   int64_t, int64_t, int32_t, int32_t, int32_t, float, float*,
+                                   float*, float*, float*, float*, int32_t*, cudaStream_t);
 size_t token_select_workspace(int64_t, int32_t, int64_t);
 cudaError_t launch_token_select_attention(const CUtensorMap&, const int64_t*, int64_t,
                                           const void*, int64_t, int64_t, int64_t, const void*,
@@ -420,6 +426,41 @@ msa_status msa_selection_recall(const msa_dims* d, msa_tensor q, msa_tensor k, m
       d->n_q, d->q_pos0, d->h_kv, d->h_q, d->d_idx, d->h_kidx, (int32_t)nblk, d->scale, sel,
       block_mass, mass_stride, recall, kl_pq, kl_qp, lse_full, ws, dev_err,
       reinterpret_cast<cudaStream_t>(stream)));
+}
+
+msa_status msa_sparse_attn_bwd(const msa_dims* d, msa_tensor q, msa_tensor k, msa_tensor v,
+                               msa_tensor o, msa_tensor d_o, const float* lse,
+                               const int32_t* blk_offsets, const int32_t* entries, float* delta,
+                               float* part_dq, float* dq, float* dk, float* dv, int32_t* dev_err,
+                               void* stream) {
+  msa_status s = check_dims(d);
+  if (s != MSA_OK) return s;
+  if ((s = check_tensor(q)) != MSA_OK) return s;
+  if ((s = check_tensor(k)) != MSA_OK) return s;
+  if ((s = check_tensor(v)) != MSA_OK) return s;
+  if ((s = check_tensor(o)) != MSA_OK) return s;
+  if ((s = check_tensor(d_o)) != MSA_OK) return s;
+  if (lse == nullptr || blk_offsets == nullptr || entries == nullptr || delta == nullptr ||
+      part_dq == nullptr || dq == nullptr || dk == nullptr || dv == nullptr)
+    return MSA_ERR_INVALID_ARG;
+  if (!aligned16(part_dq) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return MSA_ERR_ALIGNMENT;
+  const int64_t nblk = msa_num_blocks(d);
+  const int64_t total = msa_num_entries(d);
+  if (total >= (int64_t(1) << 31)) return MSA_ERR_UNSUPPORTED;
+  CUtensorMap tk, tv;
+  // k, v [B, h_kv, n_kv, 128]: dims {128, n_kv, h_kv, B}, box {64, 128, 1, 1}
+  if ((s = make_map(&tk, k.ptr, MSA_HEAD_DIM, d->n_kv, d->h_kv, d->batch, k.s_tok, k.s_head,
+                    k.s_batch, 128, 1)) != MSA_OK)
+    return s;
+  if ((s = make_map(&tv, v.ptr, MSA_HEAD_DIM, d->n_kv, d->h_kv, d->batch, v.s_tok, v.s_head,
+                    v.s_batch, 128, 1)) != MSA_OK)
+    return s;
+  return from_cuda(msa::launch_sparse_attn_bwd(
+      tk, tv, q.ptr, q.s_batch, q.s_tok, q.s_head, o.ptr, o.s_batch, o.s_tok, o.s_head, d_o.ptr,
+      d_o.s_batch, d_o.s_tok, d_o.s_head, lse, blk_offsets, entries, total, d->batch, d->n_q,
+      d->n_kv, d->q_pos0, d->h_kv, d->h_q, (int32_t)nblk, d->scale, delta, part_dq, dq, dk, dv,
+      dev_err, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 size_t msa_token_select_workspace(const msa_dims* d, int64_t n_rows) {

@@ -110,6 +110,35 @@ def forward(buf: Buffers, q, k, v, q_idx, k_idx):
     return buf.out, buf.lse
 
 
+@dataclasses.dataclass
+class Grads:
+    delta: torch.Tensor
+    dq: torch.Tensor
+    dk: torch.Tensor
+    dv: torch.Tensor
+
+    @staticmethod
+    def allocate(d: capi.Dims, device="cuda") -> "Grads":
+        B, n_q, n_kv, G, H = d.batch, d.n_q, d.n_kv, d.h_kv, d.h_q
+        dev = torch.device(device)
+        return Grads(
+            delta=torch.empty((B, n_q, H), dtype=torch.float32, device=dev),
+            dq=torch.empty((B, n_q, H, capi.HEAD_DIM), dtype=torch.float32, device=dev),
+            dk=torch.empty((B, G, n_kv, capi.HEAD_DIM), dtype=torch.float32, device=dev),
+            dv=torch.empty((B, G, n_kv, capi.HEAD_DIM), dtype=torch.float32, device=dev),
+        )
+
+
+def backward(buf: Buffers, grads: Grads, q, k, v, d_out):
+    """Gradients of the attention for upstream d_out (bf16 [B,n_q,H,128]) after a
+    forward on the same buffers (its out, lse and block lists; the selection is
+    fixed).  The forward's piece buffer holds the dQ pieces.  Returns (dq, dk, dv)."""
+    capi.msa_sparse_attn_bwd(buf.dims, q, k, v, buf.out, d_out, buf.lse, buf.blk_offsets,
+                             buf.entries, grads.delta, buf.part_acc, grads.dq, grads.dk,
+                             grads.dv, buf.dev_err)
+    return grads.dq, grads.dk, grads.dv
+
+
 def selection_recall(buf: Buffers, q, k, q_idx, k_idx, rows, lse_full=None):
     """For sampled rows (int64 device tensor of b * n_q + qi): the main branch's
     block mass [n, G, nblk], the recall of buf.sel and KL(P||Q), KL(Q||P) [n, G].

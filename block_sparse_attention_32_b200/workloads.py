@@ -229,3 +229,36 @@ def random_selection(w: Workload, device="cpu", seed_offset: int = 11):
                 rows = torch.where(rows == (1 << 30), torch.full_like(rows, -1), rows)
                 out[b, g, r0:r1] = rows.to(torch.int32)
     return out
+
+
+def upstream_grad(w: Workload, device="cpu", seed_offset: int = 101):
+    """A seeded upstream gradient dO [B, n_q, H, 128] (bf16, N(0,1)) for the
+    attention's backward."""
+    device = torch.device(device)
+    return _randn((w.batch, w.n_q, w.h_q, HEAD_DIM), _gen(device, w.seed + seed_offset), device,
+                  torch.bfloat16)
+
+
+def random_selection(w: Workload, device="cpu", seed_offset: int = 202):
+    """A seeded valid block selection [B, G, n_q, 16] int32: each query's own
+    block and up to 15 distinct earlier blocks drawn uniformly, ascending,
+    -1 after the last.  It stands in for the index branch's choice where a
+    step takes the selection as an input (the attention and its backward)."""
+    device = torch.device(device)
+    gen = _gen(device, w.seed + seed_offset)
+    B, G, n_q, nblk = w.batch, w.h_kv, w.n_q, w.nblk
+    own = (w.q_pos0 + torch.arange(n_q, device=device)) // BLOCK          # [n_q]
+    r = torch.rand((B, G, n_q, nblk), generator=gen, device=device)
+    blk = torch.arange(nblk, device=device)
+    r = torch.where(blk[None, None, None, :] < own[None, None, :, None], r, torch.full_like(r, -1.0))
+    k = min(TOPK - 1, nblk)
+    vals, idx = r.topk(k, dim=-1) if k > 0 else (r[..., :0], r[..., :0].long())
+    big = torch.iinfo(torch.int32).max
+    idx = torch.where(vals >= 0, idx, torch.full_like(idx, big))
+    sel = torch.cat([idx, own[None, None, :, None].expand(B, G, n_q, 1)], dim=-1)
+    if sel.shape[-1] < TOPK:
+        pad = torch.full((B, G, n_q, TOPK - sel.shape[-1]), big, device=device, dtype=sel.dtype)
+        sel = torch.cat([sel, pad], dim=-1)
+    sel = sel.sort(dim=-1).values
+    sel = torch.where(sel == big, torch.full_like(sel, -1), sel)
+    return sel.to(torch.int32).contiguous()

@@ -204,6 +204,35 @@ MSA_API msa_status msa_merge_partials(const msa_dims* dims, const int32_t* sel,
                               const float* part_ml, const float* part_acc,
                               void* out, float* lse, int32_t* dev_err, void* stream);
 
+/* Backward of step 3b/3c for training through the sparse attention ("MSA 稀疏
+ * 注意力三国杀" page, section "MSA 能力不掉：3T token 对照实验": a model trained
+ * with MSA from the start, MSA-PT, and a dense one converted by continued
+ * training, MSA-CPT; section "索引分支训练：KL 对齐": the index branch learns
+ * only through its KL term, so the selection is fixed here).  For every
+ * (query t, head h) of group g and its selected causal tokens J (the same
+ * block->query lists as the forward):
+ *   p_j = exp(scale q.k_j - lse),  D = dO.o,  dS_j = p_j (dO.v_j - D),
+ *   dq = scale sum_j dS_j k_j,  dk_j = scale sum dS_j q,  dv_j = sum p_j dO,
+ * the last two summed over every (query, head) whose set holds j.
+ *   q, o, d_o   [B, n_q, h_q, 128] bf16 (msa_tensor strides); o and lse are
+ *               the forward's results (msa_merge_partials)
+ *   k, v        [B, h_kv, n_kv, 128] bf16
+ *   lse         [B, n_q, h_q] fp32
+ *   delta       [B, n_q, h_q] fp32 device scratch (receives D)
+ *   part_dq     [B, n_q, h_kv, 16, R, 128] fp32 device scratch, the size and
+ *               layout of part_acc (the forward's buffer may be reused)
+ *   dq          [B, n_q, h_q, 128] fp32, contiguous
+ *   dk, dv      [B, h_kv, n_kv, 128] fp32, contiguous; zeroed by the call
+ * Blocks and keys that no query selected get zero gradients.  dq is summed in
+ * slot order (deterministic); a KV block whose queries span several work
+ * chunks sums their parts of dk, dv by atomic adds (order not fixed). */
+MSA_API msa_status msa_sparse_attn_bwd(const msa_dims* dims, msa_tensor q, msa_tensor k,
+                                       msa_tensor v, msa_tensor o, msa_tensor d_o,
+                                       const float* lse, const int32_t* blk_offsets,
+                                       const int32_t* entries, float* delta, float* part_dq,
+                                       float* dq, float* dk, float* dv, int32_t* dev_err,
+                                       void* stream);
+
 /* 8-bit (e4m3) index branch, an opt-in variant of step 1 that the MSA pages do
  * not describe: the "推理系统基础设施手记（三）" page (sections "4. CSA：先压缩，
  * 再稀疏选择" and "8. 常见坑") reports a low-precision indexer that makes selection
