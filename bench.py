@@ -347,11 +347,26 @@ def bench_recall(w, n_rows=64, reps=3):
     return out
 
 
-def bench_backward(w, attn_flops, reps=3):
+def bwd_bytes_model(w, n_entries, n_pieces):
+    """Algorithmic DRAM bytes of one backward call: per gathered row (entry x
+    head) the Q and dO rows (512 B), its lse and D (8 B), its fp32 dq piece
+    written and read back by the slot reduction (2 x 512 B); per (query, head)
+    o and dO for D (512 B), D (4 B) and dq (512 B); per selected (batch, group,
+    block) segment the 64 KB K/V tile; dk and dv written once (fp32); the
+    entry list."""
+    R = w.h_q // w.h_kv
+    rows = n_entries * R
+    qh = w.batch * w.n_q * w.h_q
+    return float(rows * (512 + 8 + 1024) + qh * (512 + 4 + 512) + n_pieces * 65536
+                 + 2 * w.batch * w.h_kv * w.n_kv * 512 + 4 * n_entries)
+
+
+def bench_backward(w, attn_flops, n_entries, peaks, reps=3):
     """The attention's backward (dq, dk, dv for a seeded upstream gradient,
-    selection fixed by the forward) on the workload: its time, and TFLOP/s
-    over the five products per (row, head, selected causal token) -- S, dP,
-    dV, dK and dQ, 2.5x the forward's two."""
+    selection fixed by the forward) on the workload: its time, TFLOP/s over
+    the five products per (row, head, selected causal token) -- S, dP, dV, dK
+    and dQ, 2.5x the forward's two -- and its algorithmic bytes against the
+    measured HBM bandwidth (the bound at these sizes)."""
     from block_sparse_attention_32_b200 import pipeline, workloads as wl
     d = pipeline.dims_for(w)
     buf = pipeline.Buffers.allocate(d)
@@ -372,8 +387,17 @@ def bench_backward(w, attn_flops, reps=3):
         raise RuntimeError(f"device error {int(buf.dev_err[0])} in the backward measurement")
     ms = ev[0].elapsed_time(ev[1]) / reps
     flops = 2.5 * attn_flops
-    out = {"workload": w.name, "ms": ms, "tflops": flops / (ms / 1000.0) / 1e12,
-           "algorithmic_flops": flops, "kernels": "mma.sync m16n8k16 (bf16, fp32 accumulate)"}
+    n_pieces = int((buf.blk_offsets[1:] > buf.blk_offsets[:-1]).sum().item())
+    nbytes = bwd_bytes_model(w, n_entries, n_pieces)
+    hbm = peaks.get("hbm_gbs", FALLBACK["hbm_gbs"])
+    sustained = peaks.get("bf16_tflops_sustained", FALLBACK["bf16_tflops_sustained"])
+    tflops = flops / (ms / 1000.0) / 1e12
+    gbs = nbytes / (ms / 1000.0) / 1e9
+    out = {"workload": w.name, "ms": ms, "tflops": tflops, "algorithmic_flops": flops,
+           "bound": "hbm" if nbytes / hbm / 1e9 > flops / sustained / 1e12 else "tensor",
+           "algorithmic_bytes": nbytes, "achieved_gbs": gbs, "hbm_frac": gbs / hbm,
+           "tensor_frac": tflops / sustained,
+           "kernels": "mma.sync m16n8k16 (bf16, fp32 accumulate)"}
     del buf, grads, inp, d_out
     torch.cuda.empty_cache()
     return out
@@ -550,7 +574,7 @@ def main():
     if not args.no_recall:
         recall = bench_recall(w)
     e4m3 = None if args.no_e4m3 else bench_e4m3(w)
-    backward = None if args.no_bwd else bench_backward(w, attn_flops)
+    backward = None if args.no_bwd else bench_backward(w, attn_flops, n_ent, peaks)
 
     # dominant kernel: the longest stage; its bound is the larger of its
     # algorithmic time at the tensor peak and at the HBM peak
