@@ -335,6 +335,12 @@ def bench_recall(w, n_rows=64, reps=3):
     # rows of one batch share those blocks, so DRAM sees each at most once
     nb = (w.q_pos0 + rows % w.n_q) // 128 + 1
     streamed = float(nb.sum()) * w.h_kv * (128 * 128 * 2 + 128 * w.d_idx * 2)
+    # token level: each (row, group) streams its causal k_idx blocks for the scores
+    # and gathers the K and V rows of its min(2048, t + 1) tokens
+    ntok = np.minimum(2048, w.q_pos0 + rows % w.n_q + 1)
+    tok_streamed = float(w.h_kv * (nb.sum() * 128 * w.d_idx * 2 + ntok.sum() * 512))
+    token_level["streamed_bytes"] = tok_streamed
+    token_level["streamed_gbs"] = tok_streamed / (ms_tok / 1000.0) / 1e9
     blocks = int(nb.max())
     unique = float(w.batch * blocks * 128 * (w.h_kv * 128 * 2 + w.h_kidx * w.d_idx * 2))
     out = {"rows": n_rows, "mean_recall": float(rec.mean()),
@@ -467,8 +473,25 @@ class CpuOracleSample:
         self.bat = np.zeros_like(self.rows)
 
     def _forward(self):
-        self.oracle.forward_rows(self.q_rows, self.qi_rows, self.pos, self.bat, self.k, self.v,
-                                 self.ki, self.w.scale)
+        _, self.sel, _, _ = self.oracle.forward_rows(self.q_rows, self.qi_rows, self.pos, self.bat,
+                                                     self.k, self.v, self.ki, self.w.scale)
+
+    def run_next_rows(self, n=None):
+        """The oracle on the first n sampled rows for the selection-recall
+        measurement and the token-level variant (rows/s, beside the GPU's)."""
+        n = min(len(self.rows), n or 2 * self.cores)
+        sl = slice(0, n)
+        args = (self.q_rows[sl], self.qi_rows[sl], self.pos[sl], self.bat[sl])
+        t0 = time.perf_counter()
+        self.oracle.selection_recall(*args, self.k, self.ki, self.sel[sl], self.w.scale)
+        t1 = time.perf_counter()
+        self.oracle.token_select_attention(*args, self.k, self.v, self.ki, self.w.scale, budget=2048)
+        t2 = time.perf_counter()
+        desc = f"{n} of the sampled rows of {self.w.name}, all groups, fp64, {self.cores} threads"
+        return ({"value": n / (t1 - t0), "unit": "rows/s", "cores": self.cores, "kind": "oracle",
+                 "sample": desc},
+                {"value": n / (t2 - t1), "unit": "rows/s", "cores": self.cores, "kind": "oracle",
+                 "sample": desc})
 
     def run(self):
         t0 = time.perf_counter()
@@ -483,7 +506,8 @@ class CpuOracleSample:
 
 
 def cpu_baseline(w, target_s=15.0):
-    return CpuOracleSample(w, target_s).run()
+    sample = CpuOracleSample(w, target_s)
+    return sample.run(), sample
 
 
 def main():
@@ -629,7 +653,14 @@ def main():
                 "d2h_bytes_per_step": e2e["d2h_bytes_per_step"]} if e2e else None,
     }
     if not args.no_cpu:
-        line["cpu_baseline"] = cpu_baseline(w)
+        line["cpu_baseline"], sample = cpu_baseline(w)
+        if recall is not None:
+            rec_cpu, tok_cpu = sample.run_next_rows()
+            recall["cpu_oracle"] = rec_cpu
+            recall["token_level"]["cpu_oracle"] = tok_cpu
+            recall["rows_per_s"] = recall["rows"] / (recall["ms"] / 1000.0)
+            recall["token_level"]["rows_per_s"] = recall["rows"] / (recall["token_level"]["ms"]
+                                                                   / 1000.0)
     print(json.dumps(line))
     if world > 1:
         torch.distributed.destroy_process_group()
