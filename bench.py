@@ -403,7 +403,7 @@ def bench_backward(w, attn_flops, n_entries, peaks, reps=3):
            "bound": "hbm" if nbytes / hbm / 1e9 > flops / sustained / 1e12 else "tensor",
            "algorithmic_bytes": nbytes, "achieved_gbs": gbs, "hbm_frac": gbs / hbm,
            "tensor_frac": tflops / sustained,
-           "kernels": "mma.sync m16n8k16 (bf16, fp32 accumulate)"}
+           "kernels": "tcgen05 kind::f16 (bf16, fp32 accumulate in TMEM)"}
     del buf, grads, inp, d_out
     torch.cuda.empty_cache()
     return out

@@ -11,25 +11,26 @@
 // Same KV-block-outer order as the forward ("Kernel 创新：Outer Gather Q"): a
 // KV block's K and V are loaded once per piece and every query row that chose
 // the block is gathered against it, so dK and dV of the block accumulate in
-// registers; dQ leaves as one fp32 piece per (query, head, slot), summed in
-// slot order by a second kernel (deterministic), exactly like the forward's
+// TMEM; dQ leaves as one fp32 piece per (query, head, slot), summed in slot
+// order by a second kernel (deterministic), exactly like the forward's
 // (m, l, acc) pieces and merge.
 //
 // Three kernels:
 //  * bwd_delta_kernel      -- D = dO.o per (query, head), one warp each;
-//  * sparse_attn_bwd_kernel<R> -- 8 warps; the entries of the block->query
-//    lists are cut into equal runs ("chunks", one CTA each, strided over a
-//    grid of at most one CTA per SM), a chunk into pieces (one per segment =
-//    KV block) and a piece into 32-row tiles (32 / R entries x R heads).
-//    Per piece: K, V by TMA (128B swizzle).  Per tile: Q and dO rows and the
-//    rows' lse and D by cp.async (double-buffered, the entries one tile
-//    further ahead in registers); warp w owns keys 16w .. 16w+15 and forms
-//    S^T = K Q^T and dP^T = V dO^T (mma.sync m16n8k16), P^T and dS^T in
-//    registers, then dV += P^T dO and dK += dS^T Q from those registers;
-//    dS^T goes to shared memory for dQ = dS K (warp w: 16 rows x 32 dims).
-//    At the end of a piece dK and dV are added to fp32 accumulators in
-//    global memory (one vector atomic per element pair: a block split over
-//    several chunks sums its parts there);
+//  * sparse_attn_bwd_tc_kernel<R> -- the entries of the block->query lists
+//    are cut into equal runs ("chunks", strided over a grid of at most one
+//    CTA per SM), a chunk into pieces (one per segment = KV block) and a
+//    piece into 128-row tiles (128 / R entries x R heads).  Warp roles
+//    (512 threads): a TMA warp loads each piece's K and V; four gather warps
+//    bring each tile's Q and dO rows by cp.async into two buffers; an MMA
+//    warp issues, per tile, S^T = K Q^T and dP^T = V dO^T (tcgen05, M = 128
+//    keys, N = 128 rows), then -- once four softmax warps (thread = key) have
+//    turned them into P^T and dS^T (bf16, back into TMEM, and dS^T also into
+//    shared memory) -- dV += P^T dO and dK += dS^T Q with A read from TMEM,
+//    and dQ = dS K with A read from shared memory; four epilogue warps store
+//    the dQ pieces and, at the end of a piece, add dK and dV into the fp32
+//    outputs (vector atomics: a block split over several chunks sums its
+//    parts there);
 //  * bwd_dq_reduce_kernel  -- dQ = sum over the slots of the pieces, one warp
 //    per (query, head).
 #include "common.cuh"
@@ -37,24 +38,6 @@
 namespace msa {
 
 namespace {
-
-constexpr int kBwThreads = 256;
-constexpr int kBwRows = 32;                      // gathered rows per tile
-constexpr int kBwOffK = 0, kBwOffV = 32768;
-constexpr int kBwOffQ = 65536;                   // 2 buffers x 8 KB (2 panels x 32 rows x 128 B)
-constexpr int kBwOffDO = kBwOffQ + 2 * 8192;
-constexpr int kBwOffDS = kBwOffDO + 2 * 8192;    // dS^T [128 keys][32 rows] bf16, 64 B per key
-constexpr int kBwOffMeta = kBwOffDS + 8192;
-// meta per buffer: lse[32], D[32] (fp32), ent[32] (int32)
-constexpr int kBwMetaBytes = 3 * kBwRows * 4;
-constexpr int kBwOffBar = kBwOffMeta + 2 * kBwMetaBytes;
-constexpr int kBwSmemBytes = 1024 + kBwOffBar + 16;
-
-__device__ __forceinline__ void cp_async_4(void* dst, const void* src, uint32_t src_bytes) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(dst)), "l"(src),
-               "r"(src_bytes)
-               : "memory");
-}
 
 struct BwdArgs {
   const __nv_bfloat16* q;     // [B, n_q, H, 128] (strided)
@@ -108,312 +91,402 @@ __global__ void __launch_bounds__(256)
   if (lane == 0) delta[r] = s;
 }
 
+// ---------------------------------------------------------------------------
+// main kernel: 128-row tiles on tcgen05, accumulators in TMEM
+// ---------------------------------------------------------------------------
+// TMEM columns (lanes = keys unless noted): [0,128) S^T, then P^T as bf16 in
+// [0,64), then dQ (lanes = rows); [128,256) dP^T, then dS^T as bf16 in
+// [128,192); [256,384) dV; [384,512) dK.  Shared memory: K, V (32 KB each,
+// TMA, 128B swizzle, two 64-column panels), two Q and two dO tiles (128
+// gathered rows each, same layout, cp.async), dS^T [128 keys][128 rows] (the
+// A operand of dQ = dS K, stored rows-contiguous: an MN-major operand), the
+// tile's row data (t, lse, D), barriers.
+namespace {
+constexpr int kTcThreads = 512;
+constexpr int kTcOffK = 0, kTcOffV = 32768;
+constexpr int kTcOffQ = 65536;                   // 2 x 32 KB
+constexpr int kTcOffDO = kTcOffQ + 2 * 32768;    // 2 x 32 KB
+constexpr int kTcOffDS = kTcOffDO + 2 * 32768;   // 32 KB
+constexpr int kTcOffMeta = kTcOffDS + 32768;     // t[128] (int32), lse[128], D[128]
+constexpr int kTcOffBar = kTcOffMeta + 3 * 128 * 4;
+enum {
+  TB_KV_FULL = 0, TB_KV_EMPTY, TB_QDO_FULL0, TB_QDO_FULL1, TB_QDO_EMPTY0, TB_QDO_EMPTY1,
+  TB_S_FULL, TB_P_FULL, TB_DVK_DONE, TB_DQ_FULL, TB_DQ_EMPTY, TB_DKV_FULL, TB_DKV_EMPTY,
+  TB_COUNT
+};
+constexpr int kTcOffMisc = kTcOffBar + TB_COUNT * 8;
+constexpr int kTcSmemBytes = 1024 + kTcOffMisc + 16;
+static_assert(kTcSmemBytes <= 232448, "shared memory per block");
+// kind::f16, bf16 A and B, fp32 D, M = N = 128; a_mn / b_mn: operand stored
+// M- / N-contiguous
+constexpr uint32_t idesc_tc(int a_mn, int b_mn) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) |
+         ((uint32_t)(128 >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+}
+
+// The CTA's sequence of pieces: runs of chunk_entries entries (chunks
+// blockIdx.x, + gridDim.x, ...), each cut at segment boundaries.  Every role
+// walks the same sequence.
+struct PieceWalk {
+  int64_t chunk, c_end, e, seg;
+};
+struct Piece {
+  int64_t b, e0, e1;
+  int32_t g, c;
+};
+__device__ __forceinline__ void walk_start(PieceWalk& w, const BwdArgs& a) {
+  w.chunk = blockIdx.x;
+  w.e = w.chunk * a.chunk_entries;
+  w.c_end = min64(w.e + a.chunk_entries, a.total);
+  w.seg = -1;
+}
+// false at the end of the CTA's work, or (with *bad set) when the lists hold
+// fewer entries than the sizes imply
+__device__ __forceinline__ bool walk_next(PieceWalk& w, const BwdArgs& a, Piece& pc, bool* bad) {
+  *bad = false;
+  while (w.e >= w.c_end) {
+    w.chunk += gridDim.x;
+    if (w.chunk * a.chunk_entries >= a.total) return false;
+    w.e = w.chunk * a.chunk_entries;
+    w.c_end = min64(w.e + a.chunk_entries, a.total);
+    w.seg = -1;
+  }
+  int64_t s2 = w.seg + 1;
+  const int64_t lim = w.seg < 0 ? 0 : min64(w.seg + 5, a.nseg);
+  while (s2 < lim && a.offsets[s2 + 1] <= w.e) ++s2;
+  w.seg = (s2 < lim) ? s2 : segment_of(a.offsets, a.nseg, w.e);
+  const int64_t p_end = min64((int64_t)a.offsets[w.seg + 1], w.c_end);
+  if (p_end <= w.e) {
+    *bad = true;
+    return false;
+  }
+  pc.e0 = w.e;
+  pc.e1 = p_end;
+  w.e = p_end;
+  pc.c = (int32_t)(w.seg % a.nblk);
+  const int64_t bg = w.seg / a.nblk;
+  pc.g = (int32_t)(bg % a.G);
+  pc.b = bg / a.G;
+  return true;
+}
+}  // namespace
+
 template <int R>
-__global__ void __launch_bounds__(kBwThreads, 1)
-    sparse_attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_k,
-                           const __grid_constant__ CUtensorMap tm_v,
-                           const __grid_constant__ BwdArgs a) {
-  static_assert(R >= 1 && R <= 16 && (kBwRows % R) == 0, "32 rows hold whole entries");
-  constexpr int kEnt = kBwRows / R;              // entries per tile
+__global__ void __launch_bounds__(kTcThreads, 1)
+    sparse_attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k,
+                              const __grid_constant__ CUtensorMap tm_v,
+                              const __grid_constant__ BwdArgs a) {
+  static_assert(R >= 1 && R <= 16 && (128 % R) == 0, "128 rows hold whole entries");
+  constexpr int kEnt = 128 / R;                  // entries per tile
+  constexpr uint32_t kIdKK = idesc_tc(0, 0);     // S^T = K Q^T, dP^T = V dO^T
+  constexpr uint32_t kIdKN = idesc_tc(0, 1);     // dV += P^T dO, dK += dS^T Q (A in TMEM)
+  constexpr uint32_t kIdNN = idesc_tc(1, 1);     // dQ = dS K
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint64_t* kv_bar = reinterpret_cast<uint64_t*>(base + kBwOffBar);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(base + kBwOffBar + 8);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(base + kTcOffBar);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + kTcOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(base + kTcOffMisc + 4);
+  int32_t* m_t = reinterpret_cast<int32_t*>(base + kTcOffMeta);
+  float* m_lse = reinterpret_cast<float*>(base + kTcOffMeta + 512);
+  float* m_d = reinterpret_cast<float*>(base + kTcOffMeta + 1024);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int gq = lane >> 2, tq = lane & 3;
-  const float scale_log2 = a.scale * 1.4426950408889634f;
-  const float log2e = 1.4426950408889634f;
+  int32_t* err = a.err;
 
   if (tid == 0) {
-    mbar_init(kv_bar, 1);
+    mbar_init(bar + TB_KV_FULL, 1);
+    mbar_init(bar + TB_KV_EMPTY, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar + TB_QDO_FULL0 + i, 128);
+      mbar_init(bar + TB_QDO_EMPTY0 + i, 1);
+    }
+    mbar_init(bar + TB_S_FULL, 1);
+    mbar_init(bar + TB_P_FULL, 128);
+    mbar_init(bar + TB_DVK_DONE, 1);
+    mbar_init(bar + TB_DQ_FULL, 1);
+    mbar_init(bar + TB_DQ_EMPTY, 128);
+    mbar_init(bar + TB_DKV_FULL, 1);
+    mbar_init(bar + TB_DKV_EMPTY, 128);
     *abort_flag = 0;
     fence_mbarrier_init();
-    prefetch_tensormap(&tm_k);
-    prefetch_tensormap(&tm_v);
   }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
   __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  // k-th completion of a barrier has parity k & 1
+  auto W = [&](int id, int64_t k) {
+    return mbar_wait(bar + id, (uint32_t)(k & 1), abort_flag, err);
+  };
+  auto ntiles_of = [](const Piece& pc) { return (pc.e1 - pc.e0 + kEnt - 1) / kEnt; };
 
-  const uint32_t k_s = smem_u32(base + kBwOffK), v_s = smem_u32(base + kBwOffV);
-  const uint32_t ds_s = smem_u32(base + kBwOffDS);
-  // prefetch role: row pr = tid / 8 of the tile, 16-byte chunks 2 (tid % 8) and + 1
-  const int pr = tid >> 3, pc = (tid & 7) * 2;
-  uint32_t kv_phase = 0;
-  bool stop = false, kv_phase_used = false;
+  PieceWalk wk;
+  walk_start(wk, a);
+  Piece pc;
+  bool bad = false;
 
-  const int64_t nchunks = (a.total + a.chunk_entries - 1) / a.chunk_entries;
-  for (int64_t chunk = blockIdx.x; chunk < nchunks; chunk += gridDim.x) {
-    const int64_t c_begin = chunk * a.chunk_entries;
-    const int64_t c_end = min64(c_begin + a.chunk_entries, a.total);
-    int64_t e = c_begin;
-    int64_t seg = -1;
-    while (e < c_end) {
-      // the segment holding entry e: a few steps past the previous one, else a search
-      {
-        int64_t s2 = seg + 1;
-        const int64_t lim = seg < 0 ? 0 : min64(seg + 5, a.nseg);
-        while (s2 < lim && a.offsets[s2 + 1] <= e) ++s2;
-        seg = (s2 < lim) ? s2 : segment_of(a.offsets, a.nseg, e);
-      }
-      const int64_t p_end = min64((int64_t)a.offsets[seg + 1], c_end);
-      const int64_t p_begin = e;
-      if (p_end <= p_begin) {                    // fewer entries listed than the sizes imply
-        if (tid == 0) report(a.err, MSA_DEVERR_BAD_ENTRY);
-        stop = true;                             // uniform: every thread read the same offsets
-        break;
-      }
-      e = p_end;
-      const int32_t c = (int32_t)(seg % a.nblk);
-      const int64_t bg = seg / a.nblk;
-      const int32_t g = (int32_t)(bg % a.G);
-      const int64_t b = bg / a.G;
-      const int64_t ntiles = (p_end - p_begin + kEnt - 1) / kEnt;
-
-      __syncthreads();                           // K, V, the buffers and dS^T are free
-      if (tid == 0) {
-        mbar_arrive_expect_tx(kv_bar, 65536u);
-        for (int p = 0; p < 2; ++p) {
-          tma_load_4d(base + kBwOffK + p * 16384, &tm_k, kv_bar, p * 64, c * kBlock, g, (int32_t)b);
-          tma_load_4d(base + kBwOffV + p * 16384, &tm_v, kv_bar, p * 64, c * kBlock, g, (int32_t)b);
+  if (warp == 0) {
+    // ---------------- K, V of every piece by TMA ----------------
+    if (lane == 0) {
+      prefetch_tensormap(&tm_k);
+      prefetch_tensormap(&tm_v);
+      for (int64_t p = 0; walk_next(wk, a, pc, &bad); ++p) {
+        if (p > 0 && !W(TB_KV_EMPTY, p - 1)) break;
+        mbar_arrive_expect_tx(bar + TB_KV_FULL, 65536u);
+        for (int h = 0; h < 2; ++h) {
+          tma_load_4d(base + kTcOffK + h * 16384, &tm_k, bar + TB_KV_FULL, h * 64, pc.c * kBlock,
+                      pc.g, (int32_t)pc.b);
+          tma_load_4d(base + kTcOffV + h * 16384, &tm_v, bar + TB_KV_FULL, h * 64, pc.c * kBlock,
+                      pc.g, (int32_t)pc.b);
         }
       }
-
-      // the prefetch of tile n into buffer n & 1: this thread's row's entry
-      // value for tile n is `ent_cur`; rows past the piece load zeros
-      auto prefetch = [&](int64_t n, int32_t ent) {
-        const int buf = (int)(n & 1);
-        uint8_t* qd = base + kBwOffQ + buf * 8192;
-        uint8_t* dd = base + kBwOffDO + buf * 8192;
-        uint8_t* meta = base + kBwOffMeta + buf * kBwMetaBytes;
-        const bool ok = ent >= 0;
-        const int64_t qi = ok ? (ent >> 4) : 0;
-        const int64_t h = (int64_t)g * R + (pr % R);
-        const __nv_bfloat16* qrow = a.q + b * a.qs_b + qi * a.qs_t + h * a.qs_h;
-        const __nv_bfloat16* drow = a.dout + b * a.ds_b + qi * a.ds_t + h * a.ds_h;
-#pragma unroll
-        for (int x = 0; x < 2; ++x) {
-          const int ch = pc + x;
-          const uint32_t off = (uint32_t)((ch >> 3) * 4096 + pr * 128 + (((ch & 7) ^ (pr & 7)) << 4));
-          cp_async_16(qd + off, ok ? (const void*)(qrow + ch * 8) : (const void*)a.q, ok ? 16u : 0u);
-          cp_async_16(dd + off, ok ? (const void*)(drow + ch * 8) : (const void*)a.dout, ok ? 16u : 0u);
-        }
-        if ((tid & 7) == 0) {
-          const int64_t mrow = (b * a.n_q + qi) * a.H + h;
-          cp_async_4(meta + pr * 4, ok ? (const void*)(a.lse + mrow) : (const void*)a.lse, ok ? 4u : 0u);
-          cp_async_4(meta + 128 + pr * 4, ok ? (const void*)(a.delta + mrow) : (const void*)a.delta,
-                     ok ? 4u : 0u);
-          reinterpret_cast<int32_t*>(meta + 256)[pr] = ent;
-        }
-        cp_async_commit();
-      };
-      auto load_ent = [&](int64_t n) -> int32_t {
-        const int64_t ei = p_begin + n * kEnt + pr / R;
-        return (n < ntiles && ei < p_end) ? __ldg(a.entries + ei) : -1;
-      };
-
-      float dv_acc[16][4], dk_acc[16][4];
-#pragma unroll
-      for (int i = 0; i < 16; ++i)
-#pragma unroll
-        for (int x = 0; x < 4; ++x) dv_acc[i][x] = dk_acc[i][x] = 0.f;
-
-      int32_t ent_next = load_ent(0);
-      prefetch(0, ent_next);
-      ent_next = load_ent(1);
-      bool kv_ok = true;
-      for (int64_t n = 0; n < ntiles; ++n) {
-        const int buf = (int)(n & 1);
-        if (n + 1 < ntiles) {
-          prefetch(n + 1, ent_next);
-          ent_next = load_ent(n + 2);
-          cp_async_wait_group<1>();
-        } else {
-          cp_async_wait_group<0>();
-        }
-        __syncthreads();                         // tile n in shared memory
-        if (n == 0) {
-          kv_ok = mbar_wait(kv_bar, kv_phase, abort_flag, a.err);
-          kv_phase ^= 1u;
-          kv_phase_used = true;
-        }
-        const uint32_t q_s = smem_u32(base + kBwOffQ + buf * 8192);
-        const uint32_t do_s = smem_u32(base + kBwOffDO + buf * 8192);
-        const float* m_lse = reinterpret_cast<const float*>(base + kBwOffMeta + buf * kBwMetaBytes);
-        const float* m_d = m_lse + kBwRows;
-        const int32_t* m_ent = reinterpret_cast<const int32_t*>(m_d + kBwRows);
-
-        // S^T and dP^T: keys 16 warp + gq (+8) x rows 8 j + 2 tq (+1)
-        float st[4][4], dpt[4][4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-#pragma unroll
-          for (int x = 0; x < 4; ++x) st[j][x] = dpt[j][x] = 0.f;
-        {
-          const int krow = 16 * warp + (lane & 7) + ((lane >> 3) & 1) * 8;
-          const int qrow_l = (lane & 7) + 8 * (lane >> 4);
-#pragma unroll
-          for (int ks = 0; ks < 8; ++ks) {
-            const int ach = 2 * ks + (lane >> 4);              // A: K / V rows
-            const uint32_t aoff = (uint32_t)((ach >> 3) * 16384 + krow * 128 +
-                                             (((ach & 7) ^ (krow & 7)) << 4));
-            uint32_t ka0, ka1, ka2, ka3, va0, va1, va2, va3;
-            ldmatrix_x4(k_s + aoff, ka0, ka1, ka2, ka3);
-            ldmatrix_x4(v_s + aoff, va0, va1, va2, va3);
-            const int bch = 2 * ks + ((lane >> 3) & 1);        // B: Q / dO rows
-#pragma unroll
-            for (int jp = 0; jp < 2; ++jp) {
-              const int rr = 16 * jp + qrow_l;
-              const uint32_t boff = (uint32_t)((bch >> 3) * 4096 + rr * 128 +
-                                               (((bch & 7) ^ (rr & 7)) << 4));
-              uint32_t b0, b1, b2, b3;
-              ldmatrix_x4(q_s + boff, b0, b1, b2, b3);
-              mma_bf16_16816(st[2 * jp], ka0, ka1, ka2, ka3, b0, b1);
-              mma_bf16_16816(st[2 * jp + 1], ka0, ka1, ka2, ka3, b2, b3);
-              ldmatrix_x4(do_s + boff, b0, b1, b2, b3);
-              mma_bf16_16816(dpt[2 * jp], va0, va1, va2, va3, b0, b1);
-              mma_bf16_16816(dpt[2 * jp + 1], va0, va1, va2, va3, b2, b3);
-            }
-          }
-        }
-        // P^T and dS^T; rows with no entry carry t = -1, so every key masks them
-        uint32_t pa[4][2], sa[4][2];             // bf16 pairs: [n-tile][key half]
-        {
-          const int64_t key0 = (int64_t)c * kBlock + 16 * warp + gq;
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int row = 8 * j + 2 * tq;
-            const float2 lse2 = *reinterpret_cast<const float2*>(m_lse + row);
-            const float2 d2 = *reinterpret_cast<const float2*>(m_d + row);
-            const int32_t e0 = m_ent[row], e1 = m_ent[row + 1];
-            const int64_t t0 = e0 >= 0 ? a.q_pos0 + (e0 >> 4) : -1;
-            const int64_t t1 = e1 >= 0 ? a.q_pos0 + (e1 >> 4) : -1;
-            float p[4], s[4];
-#pragma unroll
-            for (int x = 0; x < 4; ++x) {
-              const int64_t key = key0 + ((x >> 1) ? 8 : 0);
-              const bool col1 = x & 1;
-              const int64_t tt = col1 ? t1 : t0;
-              const float lv = col1 ? lse2.y : lse2.x;
-              const float dd = col1 ? d2.y : d2.x;
-              p[x] = key <= tt ? ex2_approx(st[j][x] * scale_log2 - lv * log2e) : 0.f;
-              s[x] = p[x] * (dpt[j][x] - dd);
-            }
-            pa[j][0] = pack_bf16x2(p[0], p[1]);
-            pa[j][1] = pack_bf16x2(p[2], p[3]);
-            sa[j][0] = pack_bf16x2(s[0], s[1]);
-            sa[j][1] = pack_bf16x2(s[2], s[3]);
-          }
-        }
-        // dS^T to shared memory: key row 64 B, 16-byte chunk j holds rows 8j .. 8j+7,
-        // stored at chunk j ^ ((key >> 1) & 3)
-        {
-          const int k0 = 16 * warp + gq, k1 = k0 + 8;
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const uint32_t o0 = (uint32_t)(k0 * 64 + ((j ^ ((k0 >> 1) & 3)) << 4) + tq * 4);
-            const uint32_t o1 = (uint32_t)(k1 * 64 + ((j ^ ((k1 >> 1) & 3)) << 4) + tq * 4);
-            asm volatile("st.shared.b32 [%0], %1;" ::"r"(ds_s + o0), "r"(sa[j][0]) : "memory");
-            asm volatile("st.shared.b32 [%0], %1;" ::"r"(ds_s + o1), "r"(sa[j][1]) : "memory");
-          }
-        }
-        // dV += P^T dO and dK += dS^T Q: k-steps over the 32 rows, B by transposing loads
-        {
-          const int rrow = (lane & 7) + ((lane >> 3) & 1) * 8;
-#pragma unroll
-          for (int kk = 0; kk < 2; ++kk) {
-            const uint32_t pa0 = pa[2 * kk][0], pa1 = pa[2 * kk][1];
-            const uint32_t pa2 = pa[2 * kk + 1][0], pa3 = pa[2 * kk + 1][1];
-            const uint32_t sa0 = sa[2 * kk][0], sa1 = sa[2 * kk][1];
-            const uint32_t sa2 = sa[2 * kk + 1][0], sa3 = sa[2 * kk + 1][1];
-            const int rr = 16 * kk + rrow;
-#pragma unroll
-            for (int np = 0; np < 8; ++np) {               // dim tiles 2 np, 2 np + 1
-              const int ch = 2 * np + (lane >> 4);
-              const uint32_t off = (uint32_t)((ch >> 3) * 4096 + rr * 128 +
-                                              (((ch & 7) ^ (rr & 7)) << 4));
-              uint32_t b0, b1, b2, b3;
-              ldmatrix_x4_trans(do_s + off, b0, b1, b2, b3);
-              mma_bf16_16816(dv_acc[2 * np], pa0, pa1, pa2, pa3, b0, b1);
-              mma_bf16_16816(dv_acc[2 * np + 1], pa0, pa1, pa2, pa3, b2, b3);
-              ldmatrix_x4_trans(q_s + off, b0, b1, b2, b3);
-              mma_bf16_16816(dk_acc[2 * np], sa0, sa1, sa2, sa3, b0, b1);
-              mma_bf16_16816(dk_acc[2 * np + 1], sa0, sa1, sa2, sa3, b2, b3);
-            }
-          }
-        }
-        const int32_t dq_ent0 = m_ent[16 * (warp & 1) + gq];
-        const int32_t dq_ent1 = m_ent[16 * (warp & 1) + gq + 8];
-        __syncthreads();                         // dS^T complete; buffer n & 1 read
-        // dQ = scale dS K: warp -> rows 16 (warp & 1) + .., dims 32 (warp >> 1) + ..
-        {
-          float dq[4][4];
-#pragma unroll
-          for (int j = 0; j < 4; ++j) dq[j][0] = dq[j][1] = dq[j][2] = dq[j][3] = 0.f;
-          const int mrow = warp & 1, dcol = warp >> 1;
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const int key = 16 * kk + (lane & 7) + 8 * (lane >> 4);
-            const int rch = 2 * mrow + ((lane >> 3) & 1);
-            uint32_t a0, a1, a2, a3;
-            ldmatrix_x4_trans(ds_s + (uint32_t)(key * 64 + ((rch ^ ((key >> 1) & 3)) << 4)),
-                              a0, a1, a2, a3);
-            const int kkey = 16 * kk + (lane & 7) + ((lane >> 3) & 1) * 8;
-#pragma unroll
-            for (int np = 0; np < 2; ++np) {
-              const int ch = 4 * dcol + 2 * np + (lane >> 4);
-              const uint32_t off = (uint32_t)((ch >> 3) * 16384 + kkey * 128 +
-                                              (((ch & 7) ^ (kkey & 7)) << 4));
-              uint32_t b0, b1, b2, b3;
-              ldmatrix_x4_trans(k_s + off, b0, b1, b2, b3);
-              mma_bf16_16816(dq[2 * np], a0, a1, a2, a3, b0, b1);
-              mma_bf16_16816(dq[2 * np + 1], a0, a1, a2, a3, b2, b3);
-            }
-          }
-          // rows 16 mrow + gq and + 8: piece row (b, i, g, slot, r) of [B, n_q, G, 16, R]
-#pragma unroll
-          for (int hf = 0; hf < 2; ++hf) {
-            const int row = 16 * mrow + gq + 8 * hf;
-            const int32_t ent = hf ? dq_ent1 : dq_ent0;
-            if (ent >= 0 && kv_ok) {
-              const int64_t prow = ((b * a.n_q + (ent >> 4)) * a.G + g) * (int64_t)kTopK * R +
-                                   (int64_t)(ent & 15) * R + (row % R);
-              float* dst = a.part_dq + prow * kHeadDim + 32 * dcol + 2 * tq;
-#pragma unroll
-              for (int j = 0; j < 4; ++j)
-                *reinterpret_cast<float2*>(dst + 8 * j) =
-                    make_float2(a.scale * dq[j][2 * hf], a.scale * dq[j][2 * hf + 1]);
-            }
-          }
-        }
-      }
-      // the piece's dK, dV rows: keys 16 warp + gq (+8), dims 8 n + 2 tq (+1)
-      if (kv_ok) {
-        const int64_t kbase = ((b * a.G + g) * a.n_kv) * kHeadDim;
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          const int64_t key = (int64_t)c * kBlock + 16 * warp + gq + 8 * hf;
-          if (key < a.n_kv) {
-            float* dkr = a.dk + kbase + key * kHeadDim + 2 * tq;
-            float* dvr = a.dv + kbase + key * kHeadDim + 2 * tq;
-#pragma unroll
-            for (int nt = 0; nt < 16; ++nt) {
-              atomicAdd(reinterpret_cast<float2*>(dkr + 8 * nt),
-                        make_float2(a.scale * dk_acc[nt][2 * hf], a.scale * dk_acc[nt][2 * hf + 1]));
-              atomicAdd(reinterpret_cast<float2*>(dvr + 8 * nt),
-                        make_float2(dv_acc[nt][2 * hf], dv_acc[nt][2 * hf + 1]));
-            }
-          }
-        }
-      }
-      if (__syncthreads_or(*abort_flag != 0)) {
-        stop = true;
-        break;
+      if (bad) {
+        report(err, MSA_DEVERR_BAD_ENTRY);
+        *abort_flag = 1;
       }
     }
-    if (stop) break;
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      int64_t n = 0, p = 0;
+      bool ok = true;
+      const uint32_t ka = smem_u32(base + kTcOffK), va = smem_u32(base + kTcOffV);
+      const uint32_t dsa = smem_u32(base + kTcOffDS);
+      for (; ok && walk_next(wk, a, pc, &bad); ++p) {
+        if (!W(TB_KV_FULL, p)) { ok = false; break; }
+        const int64_t nt = ntiles_of(pc);
+        for (int64_t t = 0; t < nt; ++t, ++n) {
+          const int buf = (int)(n & 1);
+          if (!W(TB_QDO_FULL0 + buf, n >> 1)) { ok = false; break; }
+          if (n > 0 && !W(TB_DQ_EMPTY, n - 1)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t qa = smem_u32(base + kTcOffQ + buf * 32768);
+          const uint32_t da = smem_u32(base + kTcOffDO + buf * 32768);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+            umma_bf16(tmem, smem_desc_sw128(ka + off, 16, 1024), smem_desc_sw128(qa + off, 16, 1024),
+                      kIdKK, kk > 0 ? 1u : 0u);
+          }
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+            umma_bf16(tmem + 128, smem_desc_sw128(va + off, 16, 1024),
+                      smem_desc_sw128(da + off, 16, 1024), kIdKK, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(bar + TB_S_FULL);
+          if (!W(TB_P_FULL, n)) { ok = false; break; }
+          if (t == 0 && p > 0 && !W(TB_DKV_EMPTY, p - 1)) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t acc = (t > 0 || kk > 0) ? 1u : 0u;
+            umma_bf16_ts(tmem + 256, tmem + kk * 8, smem_desc_sw128(da + kk * 2048, 16384, 1024),
+                         kIdKN, acc);
+            umma_bf16_ts(tmem + 384, tmem + 128 + kk * 8,
+                         smem_desc_sw128(qa + kk * 2048, 16384, 1024), kIdKN, acc);
+          }
+          umma_commit(bar + TB_QDO_EMPTY0 + buf);
+          umma_commit(bar + TB_DVK_DONE);
+          // dQ overwrites the columns P^T was read from: wait for dV, dK first
+          if (!W(TB_DVK_DONE, n)) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            umma_bf16(tmem, smem_desc_sw128(dsa + kk * 2048, 16384, 1024),
+                      smem_desc_sw128(ka + kk * 2048, 16384, 1024), kIdNN, kk > 0 ? 1u : 0u);
+          umma_commit(bar + TB_DQ_FULL);
+          if (t + 1 == nt) {
+            umma_commit(bar + TB_KV_EMPTY);
+            umma_commit(bar + TB_DKV_FULL);
+          }
+        }
+      }
+      if (ok && n > 0) {                         // let the last completions land
+        W(TB_DQ_FULL, n - 1);
+        W(TB_DKV_FULL, p - 1);
+      }
+    }
+  } else if (warp >= 4 && warp < 8) {
+    // ---------------- gather: Q and dO rows of each tile ----------------
+    const int gt = tid - 128;                    // 0..127
+    const int ch = gt & 15;
+    int64_t n = 0;
+    bool ok = true;
+    for (int64_t p = 0; ok && walk_next(wk, a, pc, &bad); ++p) {
+      const int64_t nt = ntiles_of(pc);
+      const __nv_bfloat16* qb = a.q + pc.b * a.qs_b + (int64_t)(pc.g * R) * a.qs_h + ch * 8;
+      const __nv_bfloat16* db = a.dout + pc.b * a.ds_b + (int64_t)(pc.g * R) * a.ds_h + ch * 8;
+      for (int64_t t = 0; t < nt; ++t, ++n) {
+        const int buf = (int)(n & 1);
+        if (n >= 2 && !W(TB_QDO_EMPTY0 + buf, (n >> 1) - 1)) { ok = false; break; }
+        uint8_t* sq = base + kTcOffQ + buf * 32768;
+        uint8_t* sd = base + kTcOffDO + buf * 32768;
+        const int64_t et = pc.e0 + t * kEnt;
+#pragma unroll 4
+        for (int it = 0; it < 16; ++it) {
+          const int row = it * 8 + (gt >> 4);
+          const int64_t ei = et + row / R;
+          const int32_t ent = ei < pc.e1 ? __ldg(a.entries + ei) : -1;
+          const bool v = ent >= 0;
+          const int64_t qi = v ? (int64_t)(ent >> 4) : 0;
+          const int64_t hoff = (int64_t)(row % R);
+          const uint32_t off = (uint32_t)((ch >> 3) * 16384 + row * 128 + (((ch & 7) ^ (row & 7)) << 4));
+          cp_async_16(sq + off, v ? (const void*)(qb + qi * a.qs_t + hoff * a.qs_h) : (const void*)a.q,
+                      v ? 16u : 0u);
+          cp_async_16(sd + off, v ? (const void*)(db + qi * a.ds_t + hoff * a.ds_h) : (const void*)a.dout,
+                      v ? 16u : 0u);
+        }
+        cp_async_wait_all();
+        fence_proxy_async_smem();
+        mbar_arrive(bar + TB_QDO_FULL0 + buf);
+      }
+    }
+  } else if (warp >= 8 && warp < 12) {
+    // ---------------- P^T and dS^T (thread = key) ----------------
+    const int quarter = warp & 3;
+    const int key = quarter * 32 + lane;
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    const float scale_log2 = a.scale * 1.4426950408889634f;
+    const float log2e = 1.4426950408889634f;
+    uint8_t* ds = base + kTcOffDS;
+    int64_t n = 0;
+    bool ok = true;
+    for (int64_t p = 0; ok && walk_next(wk, a, pc, &bad); ++p) {
+      const int64_t nt = ntiles_of(pc);
+      const int64_t key_abs = (int64_t)pc.c * kBlock + key;
+      for (int64_t t = 0; t < nt; ++t, ++n) {
+        // this thread's row (row = key index) data for the tile
+        const int64_t ei = pc.e0 + t * kEnt + key / R;
+        const int32_t ent = ei < pc.e1 ? __ldg(a.entries + ei) : -1;
+        int32_t trow = -1;
+        float lse_r = 0.f, d_r = 0.f;
+        if (ent >= 0) {
+          const int64_t qi = (int64_t)(ent >> 4);
+          const int64_t mrow = (pc.b * a.n_q + qi) * a.H + pc.g * R + (key % R);
+          trow = (int32_t)(a.q_pos0 + qi);
+          lse_r = __ldg(a.lse + mrow);
+          d_r = __ldg(a.delta + mrow);
+        }
+        if (!W(TB_S_FULL, n)) { ok = false; break; }
+        m_t[key] = trow;
+        m_lse[key] = lse_r * log2e;
+        m_d[key] = d_r;
+        named_bar_sync(1, 128);
+        tc_fence_after();
+        const uint32_t taddr = tmem + lane_base;
+#pragma unroll 1
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t sr[32], dr[32];
+          tmem_ld_32x32b_x32(taddr + 32 * cc, sr);
+          tmem_ld_32x32b_x32(taddr + 128 + 32 * cc, dr);
+          tmem_ld_wait();
+          uint32_t pp[16], sp[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            float pv[2], sv[2];
+#pragma unroll
+            for (int x = 0; x < 2; ++x) {
+              const int row = 32 * cc + 2 * j + x;
+              const bool live = key_abs <= (int64_t)m_t[row];
+              const float pr = live ? ex2_approx(u2f(sr[2 * j + x]) * scale_log2 - m_lse[row]) : 0.f;
+              pv[x] = pr;
+              sv[x] = live ? pr * (u2f(dr[2 * j + x]) - m_d[row]) : 0.f;
+            }
+            pp[j] = pack_bf16x2(pv[0], pv[1]);
+            sp[j] = pack_bf16x2(sv[0], sv[1]);
+          }
+          tmem_st_32x32b_x16(taddr + 16 * cc, pp);
+          tmem_st_32x32b_x16(taddr + 128 + 16 * cc, sp);
+          // dS^T row `key`, rows 32 cc .. 32 cc + 31: panel cc / 2, 16-byte chunks
+          // 4 (cc % 2) .. + 3, at chunk ^ (key % 8)
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            const int chk = 4 * (cc & 1) + q4;
+            uint4 v4 = make_uint4(sp[4 * q4], sp[4 * q4 + 1], sp[4 * q4 + 2], sp[4 * q4 + 3]);
+            *reinterpret_cast<uint4*>(ds + (cc >> 1) * 16384 + key * 128 + ((chk ^ (key & 7)) << 4)) = v4;
+          }
+        }
+        tmem_st_wait();
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(bar + TB_P_FULL);
+      }
+    }
+  } else if (warp >= 12) {
+    // ---------------- epilogue: dQ pieces, then dK, dV of each piece ----------------
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;         // dQ: lane = row; dK, dV: lane = key
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    int64_t n = 0;
+    bool ok = true;
+    for (int64_t p = 0; ok && walk_next(wk, a, pc, &bad); ++p) {
+      const int64_t nt = ntiles_of(pc);
+      for (int64_t t = 0; t < nt; ++t, ++n) {
+        const int64_t ei = pc.e0 + t * kEnt + row / R;
+        const int32_t ent = ei < pc.e1 ? __ldg(a.entries + ei) : -1;
+        float* dst = nullptr;
+        if (ent >= 0) {
+          const int64_t prow = ((pc.b * a.n_q + (ent >> 4)) * a.G + pc.g) * (int64_t)kTopK * R +
+                               (int64_t)(ent & 15) * R + (row % R);
+          dst = a.part_dq + prow * kHeadDim;
+        }
+        if (!W(TB_DQ_FULL, n)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll 1
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(tmem + lane_base + 32 * cc, r);
+          tmem_ld_wait();
+          if (dst != nullptr) {
+#pragma unroll
+            for (int x = 0; x < 8; ++x)
+              *reinterpret_cast<float4*>(dst + 32 * cc + 4 * x) =
+                  make_float4(a.scale * u2f(r[4 * x]), a.scale * u2f(r[4 * x + 1]),
+                              a.scale * u2f(r[4 * x + 2]), a.scale * u2f(r[4 * x + 3]));
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(bar + TB_DQ_EMPTY);
+        if (t + 1 == nt) {
+          if (!W(TB_DKV_FULL, p)) { ok = false; break; }
+          tc_fence_after();
+          const int64_t key_abs = (int64_t)pc.c * kBlock + row;
+          const bool live = key_abs < a.n_kv;
+          const int64_t kb = ((pc.b * a.G + pc.g) * a.n_kv + key_abs) * kHeadDim;
+#pragma unroll 1
+          for (int which = 0; which < 2; ++which) {      // 0: dV, 1: dK (scaled)
+            float* outp = which ? a.dk : a.dv;
+            const float f = which ? a.scale : 1.f;
+#pragma unroll 1
+            for (int cc = 0; cc < 4; ++cc) {
+              uint32_t r[32];
+              tmem_ld_32x32b_x32(tmem + lane_base + 256 + 128 * which + 32 * cc, r);
+              tmem_ld_wait();
+              if (live) {
+#pragma unroll
+                for (int x = 0; x < 8; ++x)
+                  atomicAdd(reinterpret_cast<float4*>(outp + kb + 32 * cc + 4 * x),
+                            make_float4(f * u2f(r[4 * x]), f * u2f(r[4 * x + 1]),
+                                        f * u2f(r[4 * x + 2]), f * u2f(r[4 * x + 3])));
+              }
+            }
+          }
+          tc_fence_before();
+          mbar_arrive(bar + TB_DKV_EMPTY);
+        }
+      }
+    }
   }
-  // after an abort, the last K/V load may still be in flight
-  if (stop && kv_phase_used && tid == 0) mbar_drain(kv_bar, kv_phase ^ 1u, a.err);
+  // warps 2, 3: idle
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, 512);
 }
 
 __global__ void __launch_bounds__(256)
@@ -440,13 +513,13 @@ __global__ void __launch_bounds__(256)
 }
 
 template <int R>
-static cudaError_t launch_bwd_r(const CUtensorMap& tm_k, const CUtensorMap& tm_v,
-                                const BwdArgs& a, int grid, cudaStream_t st) {
-  auto k = sparse_attn_bwd_kernel<R>;
+static cudaError_t launch_bwd_tc_r(const CUtensorMap& tm_k, const CUtensorMap& tm_v,
+                                   const BwdArgs& a, int grid, cudaStream_t st) {
+  auto k = sparse_attn_bwd_tc_kernel<R>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       kBwSmemBytes);
+                                       kTcSmemBytes);
   if (e != cudaSuccess) return e;
-  k<<<grid, kBwThreads, kBwSmemBytes, st>>>(tm_k, tm_v, a);
+  k<<<grid, kTcThreads, kTcSmemBytes, st>>>(tm_k, tm_v, a);
   return cudaGetLastError();
 }
 
@@ -501,20 +574,20 @@ cudaError_t launch_sparse_attn_bwd(const CUtensorMap& tm_k, const CUtensorMap& t
   a.nblk = nblk;
   a.scale = scale;
   a.err = err;
-  // equal runs of entries, whole tiles each, about 8 per SM
-  const int64_t ent_per_tile = kBwRows / R;
+  // equal runs of entries, whole 128-row tiles each, about 8 per SM
+  const int64_t ent_per_tile = 128 / R;
   const int64_t tiles = (total_entries + ent_per_tile - 1) / ent_per_tile;
-  const int64_t tiles_per_chunk = max64(16, (tiles + 8LL * sms - 1) / (8LL * sms));
+  const int64_t tiles_per_chunk = max64(4, (tiles + 8LL * sms - 1) / (8LL * sms));
   a.chunk_entries = tiles_per_chunk * ent_per_tile;
   const int64_t nchunks = (total_entries + a.chunk_entries - 1) / a.chunk_entries;
   const int grid = (int)min64(nchunks, sms);
   if (grid > 0) {
     switch (R) {
-      case 1: e = launch_bwd_r<1>(tm_k, tm_v, a, grid, st); break;
-      case 2: e = launch_bwd_r<2>(tm_k, tm_v, a, grid, st); break;
-      case 4: e = launch_bwd_r<4>(tm_k, tm_v, a, grid, st); break;
-      case 8: e = launch_bwd_r<8>(tm_k, tm_v, a, grid, st); break;
-      case 16: e = launch_bwd_r<16>(tm_k, tm_v, a, grid, st); break;
+      case 1: e = launch_bwd_tc_r<1>(tm_k, tm_v, a, grid, st); break;
+      case 2: e = launch_bwd_tc_r<2>(tm_k, tm_v, a, grid, st); break;
+      case 4: e = launch_bwd_tc_r<4>(tm_k, tm_v, a, grid, st); break;
+      case 8: e = launch_bwd_tc_r<8>(tm_k, tm_v, a, grid, st); break;
+      case 16: e = launch_bwd_tc_r<16>(tm_k, tm_v, a, grid, st); break;
       default: return cudaErrorInvalidValue;
     }
     if (e != cudaSuccess) return e;
