@@ -95,8 +95,9 @@ __global__ void __launch_bounds__(256)
 // main kernel: 128-row tiles on tcgen05, accumulators in TMEM
 // ---------------------------------------------------------------------------
 // TMEM columns (lanes = keys unless noted): [0,128) S^T, then P^T as bf16 in
-// [0,64), then dQ (lanes = rows); [128,256) dP^T, then dS^T as bf16 in
-// [128,192); [256,384) dV; [384,512) dK.  Shared memory: K, V (32 KB each,
+// [0,64); [128,256) dP^T, then dS^T as bf16 in [128,192), then dQ (lanes =
+// rows); [256,384) dV; [384,512) dK.  S^T of the next tile of a piece goes in
+// as soon as dV and dK have read P^T, while the epilogue still reads dQ.  Shared memory: K, V (32 KB each,
 // TMA, 128B swizzle, two 64-column panels), two Q and two dO tiles (128
 // gathered rows each, same layout, cp.async), dS^T [128 keys][128 rows] (the
 // A operand of dQ = dS K, stored rows-contiguous: an MN-major operand), the
@@ -259,19 +260,28 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       for (; ok && walk_next(wk, a, pc, &bad); ++p) {
         if (!W(TB_KV_FULL, p)) { ok = false; break; }
         const int64_t nt = ntiles_of(pc);
-        for (int64_t t = 0; t < nt; ++t, ++n) {
-          const int buf = (int)(n & 1);
-          if (!W(TB_QDO_FULL0 + buf, n >> 1)) { ok = false; break; }
-          if (n > 0 && !W(TB_DQ_EMPTY, n - 1)) { ok = false; break; }
+        // S^T(n) = K Q(n)^T into [0,128): for the first tile of a piece here, for
+        // the others right after dQ(n-1) (it only needs P^T(n-1) consumed)
+        auto issue_s = [&](int64_t nn) {
+          if (!W(TB_QDO_FULL0 + (int)(nn & 1), nn >> 1)) return false;
           tc_fence_after();
-          const uint32_t qa = smem_u32(base + kTcOffQ + buf * 32768);
-          const uint32_t da = smem_u32(base + kTcOffDO + buf * 32768);
+          const uint32_t qa = smem_u32(base + kTcOffQ + (int)(nn & 1) * 32768);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
             const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
             umma_bf16(tmem, smem_desc_sw128(ka + off, 16, 1024), smem_desc_sw128(qa + off, 16, 1024),
                       kIdKK, kk > 0 ? 1u : 0u);
           }
+          return true;
+        };
+        if (nt > 0 && !issue_s(n)) { ok = false; break; }
+        for (int64_t t = 0; t < nt; ++t, ++n) {
+          const int buf = (int)(n & 1);
+          // dP^T(n) into [128,256), once the epilogue has read dQ(n-1) there
+          if (n > 0 && !W(TB_DQ_EMPTY, n - 1)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t qa = smem_u32(base + kTcOffQ + buf * 32768);
+          const uint32_t da = smem_u32(base + kTcOffDO + buf * 32768);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
             const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
@@ -292,17 +302,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           }
           umma_commit(bar + TB_QDO_EMPTY0 + buf);
           umma_commit(bar + TB_DVK_DONE);
-          // dQ overwrites the columns P^T was read from: wait for dV, dK first
+          // dQ overwrites the columns dS^T was read from, and S^T(n+1) those of
+          // P^T: wait for dV, dK first
           if (!W(TB_DVK_DONE, n)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            umma_bf16(tmem, smem_desc_sw128(dsa + kk * 2048, 16384, 1024),
+            umma_bf16(tmem + 128, smem_desc_sw128(dsa + kk * 2048, 16384, 1024),
                       smem_desc_sw128(ka + kk * 2048, 16384, 1024), kIdNN, kk > 0 ? 1u : 0u);
           umma_commit(bar + TB_DQ_FULL);
           if (t + 1 == nt) {
             umma_commit(bar + TB_KV_EMPTY);
             umma_commit(bar + TB_DKV_FULL);
+          } else if (!issue_s(n + 1)) {
+            ok = false;
+            break;
           }
         }
       }
@@ -387,18 +401,24 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           tmem_ld_wait();
           uint32_t pp[16], sp[16];
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            float pv[2], sv[2];
+          for (int q = 0; q < 8; ++q) {            // rows 32 cc + 4 q .. + 3
+            const int4 t4 = reinterpret_cast<const int4*>(m_t)[8 * cc + q];
+            const float4 l4 = reinterpret_cast<const float4*>(m_lse)[8 * cc + q];
+            const float4 d4 = reinterpret_cast<const float4*>(m_d)[8 * cc + q];
+            const int32_t tv[4] = {t4.x, t4.y, t4.z, t4.w};
+            const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dv4[4] = {d4.x, d4.y, d4.z, d4.w};
+            float pv[4], sv[4];
 #pragma unroll
-            for (int x = 0; x < 2; ++x) {
-              const int row = 32 * cc + 2 * j + x;
-              const bool live = key_abs <= (int64_t)m_t[row];
-              const float pr = live ? ex2_approx(u2f(sr[2 * j + x]) * scale_log2 - m_lse[row]) : 0.f;
+            for (int x = 0; x < 4; ++x) {
+              const bool live = key_abs <= (int64_t)tv[x];
+              const float pr = live ? ex2_approx(u2f(sr[4 * q + x]) * scale_log2 - lv[x]) : 0.f;
               pv[x] = pr;
-              sv[x] = live ? pr * (u2f(dr[2 * j + x]) - m_d[row]) : 0.f;
+              sv[x] = live ? pr * (u2f(dr[4 * q + x]) - dv4[x]) : 0.f;
             }
-            pp[j] = pack_bf16x2(pv[0], pv[1]);
-            sp[j] = pack_bf16x2(sv[0], sv[1]);
+            pp[2 * q] = pack_bf16x2(pv[0], pv[1]);
+            pp[2 * q + 1] = pack_bf16x2(pv[2], pv[3]);
+            sp[2 * q] = pack_bf16x2(sv[0], sv[1]);
+            sp[2 * q + 1] = pack_bf16x2(sv[2], sv[3]);
           }
           tmem_st_32x32b_x16(taddr + 16 * cc, pp);
           tmem_st_32x32b_x16(taddr + 128 + 16 * cc, sp);
@@ -440,7 +460,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll 1
         for (int cc = 0; cc < 4; ++cc) {
           uint32_t r[32];
-          tmem_ld_32x32b_x32(tmem + lane_base + 32 * cc, r);
+          tmem_ld_32x32b_x32(tmem + lane_base + 128 + 32 * cc, r);
           tmem_ld_wait();
           if (dst != nullptr) {
 #pragma unroll
