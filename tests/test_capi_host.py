@@ -113,3 +113,37 @@ def test_pointer_and_stride_checks(lib):
     m = lib.msa_merge_partials
     assert m(ctypes.byref(d), P(0x1000), P(0x2000), P(0x3000), None, P(0x5000), None, None) == 1
     assert lib.msa_status_string(4) == b"MSA_ERR_WORKSPACE_TOO_SMALL"
+
+
+def test_token_select_and_backward_validation(lib):
+    """The token-level and backward entry points reject bad arguments on the
+    host, before anything is enqueued."""
+    P = ctypes.c_void_p
+    d = capi.make_dims(1, 1000, 4096, 0, 8, 2, 128)
+    good = capi.Tensor(0x100000, 0, 256, 128)
+    mis = capi.Tensor(0x100008, 0, 256, 128)
+    # workspace: one fp32 score row per (sampled row, group)
+    assert capi.msa_token_select_workspace(d, 3) == 3 * 2 * 4096 * 4
+    ws = capi.msa_token_select_workspace(d, 3)
+    t = lib.msa_token_select_attention
+    args = lambda budget, out, wsb, rows=P(0x1000): (ctypes.byref(d), good, good, good, good, good,
+                                                     rows, 3, budget, P(0x2000), out, P(0x4000),
+                                                     P(0x5000), wsb, None, None)
+    assert t(*args(0, P(0x3000), ws)) == 1                 # budget < 1
+    assert t(*args(2048, P(0x3000), ws - 4)) == 4          # workspace too small
+    assert t(*args(2048, P(0x3004), ws)) == 3              # misaligned out
+    assert t(*args(2048, P(0x3000), ws, rows=None)) == 1   # no rows
+    d16 = capi.make_dims(1, 1000, 4096, 0, 32, 2, 128)    # R = 16: heads exceed the 8-wide tiles
+    assert t(ctypes.byref(d16), good, good, good, good, good, P(0x1000), 3, 2048, P(0x2000),
+             P(0x3000), P(0x4000), P(0x5000), capi.msa_token_select_workspace(d16, 3), None,
+             None) == 2
+    b = lib.msa_sparse_attn_bwd
+    ptrs = [P(0x1000 * (i + 1)) for i in range(8)]      # lse, offsets, entries, delta, part, dq, dk, dv
+    bad = list(ptrs)
+    bad[5] = None
+    assert b(ctypes.byref(d), good, good, good, good, good, *bad, None, None) == 1
+    bad = list(ptrs)
+    bad[6] = P(0x7008)
+    assert b(ctypes.byref(d), good, good, good, good, good, *bad, None, None) == 3
+    assert b(ctypes.byref(d), good, good, good, mis, good, *ptrs, None, None) == 3
+    assert b(None, good, good, good, good, good, *ptrs, None, None) == 1
