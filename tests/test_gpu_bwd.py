@@ -175,3 +175,26 @@ def test_backward_full_size_rows_and_identities():
             q_rows[r][None, None], kf, vf, do_rows[r][None, None],
             sel[r][None, :, None, :].astype(np.int32), w.scale, int(pos[r]))
         _check(f"dq row {rows[r]}", g_dq[r], e_dq[0, 0])
+
+
+def test_backward_reports_short_selection():
+    """A selection with fewer entries than the sizes imply (a query keeping 15
+    of its 16 blocks) is reported by the backward on the device flag
+    (MSA_DEVERR_BAD_ENTRY), after which the call returns."""
+    _need_gpu()
+    w = CASES[5]                                  # 333 queries after 1889 cached tokens
+    d = pipeline.dims_for(w)
+    buf = pipeline.Buffers.allocate(d)
+    grads = pipeline.Grads.allocate(d)
+    inp = wl.make_inputs(w, "cuda")
+    s_np = wl.random_selection(w, "cpu").numpy()
+    keep = s_np[0, 0, 300][s_np[0, 0, 300] >= 0][1:]      # query 300 of group 0 drops one block
+    s_np[0, 0, 300] = np.concatenate([keep, np.full(16 - len(keep), -1)])
+    sel = torch.from_numpy(s_np).cuda()
+    d_out = wl.upstream_grad(w, "cuda")
+    pipeline.attend(buf, inp["q"], inp["k"], inp["v"], sel=sel)
+    torch.cuda.synchronize()
+    buf.dev_err.zero_()
+    pipeline.backward(buf, grads, inp["q"], inp["k"], inp["v"], d_out)
+    torch.cuda.synchronize()
+    assert int(buf.dev_err[0]) == 3                          # MSA_DEVERR_BAD_ENTRY
