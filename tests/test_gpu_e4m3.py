@@ -76,3 +76,39 @@ def test_e4m3_codes_pooled_and_selection(w):
     gpu_sel = buf.sel.permute(0, 2, 1, 3).reshape(-1, w.h_kv, 16).cpu().numpy()
     bad, ties, bad_cert, _ = compare_sets(gpu_sel, ora_sel, ora, pos)
     assert bad == 0 and bad_cert == 0, (bad, ties, bad_cert)
+
+
+def test_e4m3_full_size_rows():
+    """The 128K prefill's index branch (8 groups, d_idx 128): every code and both
+    scales bit for bit, pooled scores and selections of sampled rows against the
+    oracle."""
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    w = wl.P128
+    d = pipeline.dims_for(w)
+    buf = pipeline.Buffers.allocate(d)
+    inp = wl.make_inputs(w, "cuda", with_qkv=False)
+    q8, k8, sq, sk = pipeline.select_e4m3(buf, inp["q_idx"], inp["k_idx"])
+    torch.cuda.synchronize()
+    assert int(buf.dev_err[0]) == 0
+    qb, kb = oracle.bf16_bits(inp["q_idx"]), oracle.bf16_bits(inp["k_idx"])
+    oq, osq = oracle.quantize_e4m3(qb)
+    ok, osk = oracle.quantize_e4m3(kb)
+    assert float(sq[0]) == osq and float(sk[0]) == osk
+    np.testing.assert_array_equal(q8.cpu().numpy(), oq)
+    np.testing.assert_array_equal(k8.cpu().numpy(), ok)
+    rows = np.array([1000, 70000, w.n_q - 1], np.int64)
+    pos = w.q_pos0 + rows
+    bat = np.zeros_like(rows)
+    q_rows = oq[0, rows]
+    ora = oracle.index_pooled_e4m3(q_rows, pos, bat, ok, osq, osk, out_stride=buf.pooled_stride)
+    gpu = buf.pooled[0, :, torch.from_numpy(rows).cuda()].permute(1, 0, 2).cpu().numpy()
+    dec = np.vectorize(oracle.e4m3_value)
+    lut = dec(np.arange(256)).astype(np.float64)
+    lut[np.isnan(lut)] = 0.0
+    tol = _tolerance(lut[q_rows], lut[ok], pos, bat, w.h_kidx, osq * osk)
+    assert compare_pooled(gpu, ora[:, :, :tol.shape[2]], tol, pos) <= 1.0
+    ora_sel = oracle.topk(ora, pos)
+    gpu_sel = buf.sel[0, :, torch.from_numpy(rows).cuda()].permute(1, 0, 2).cpu().numpy()
+    bad, ties, bad_cert, _ = compare_sets(gpu_sel, ora_sel, ora, pos)
+    assert bad == 0 and bad_cert == 0, (bad, ties, bad_cert)
