@@ -6,8 +6,13 @@ library itself never allocates); ``forward`` enqueues
   msa_index_score_maxpool -> msa_topk_blocks -> msa_build_block_query_lists
   -> msa_sparse_attn_fwd -> msa_merge_partials
 
-and returns the bf16 output and the fp32 log-sum-exp.  Every step runs in the
-library's kernels; this module only marshals arguments.
+and returns the bf16 output and the fp32 log-sum-exp.  Beside it:
+``select_e4m3`` (8-bit index branch), ``selection_recall`` (recall / KL
+alignment target, optionally the full causal lse), ``token_select_attention``
+(token-level selection at the same key budget), ``backward`` with ``Grads``
+(dq, dk, dv for an upstream gradient) and ``HostPipeline`` (host buffers,
+copies overlapped).  Every step runs in the library's kernels; this module
+only marshals arguments.
 """
 from __future__ import annotations
 

@@ -17,6 +17,11 @@
  * chose it is gathered into one tensor-core tile; the per-(query, block)
  * softmax pieces are then merged by log-sum-exp.
  *
+ * Beside the path: an 8-bit (e4m3) index branch, the selection recall / KL
+ * alignment target of the index branch, token-level selection at the same
+ * key budget, and the backward of the attention (dq, dk, dv) for training
+ * through the sparse attention.
+ *
  * Conventions for every entry point:
  *   - All pointers are DEVICE pointers unless stated; the caller owns every
  *     buffer.  The library never allocates, frees or synchronises; each call
@@ -28,7 +33,8 @@
  *     that detects a problem at run time (an out-of-range block id, a wait
  *     that ran past its time limit) stores an MSA_DEVERR_* code there and
  *     returns early.  Nothing traps.
- *   - Results are deterministic: bit-identical from run to run.
+ *   - Results are deterministic: bit-identical from run to run (except dk
+ *     and dv of msa_sparse_attn_bwd, summed with atomic adds).
  *   - Fixed sizes: block B_k = 128 tokens, top-k = 16 blocks (own included),
  *     head_dim = 128, d_idx in {64, 128}.
  *   - Layouts are given as [outer, ..., inner]; the innermost dimension is
