@@ -10,7 +10,7 @@ Each function cites the page passage it follows in ``msa_oracle.c``:
     ("MSA 稀疏注意力三国杀" page, section "MSA 架构：粗筛 + 精算", steps 1-2;
     "稀疏注意力速览" page, section 4, MSA entry);
   * ``topk`` / ``topk_f32`` -- 16 blocks per query and group, own block
-    forced (same section, step 3; survey MSA entry);
+    forced (same section, step 3; "稀疏注意力速览" page, MSA entry);
   * ``attention`` -- exact softmax attention over the selected tokens (same
     section, "第二步：精算"; softmax(QK^T/sqrt(d)) V from the "稀疏注意力架构革命"
     page, section 1.1);
