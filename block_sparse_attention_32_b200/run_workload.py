@@ -2,10 +2,12 @@
 
     python -m block_sparse_attention_32_b200.run_workload --workload profile_8k_r8 --passes 2
     python -m block_sparse_attention_32_b200.run_workload --workload prefill_32k --select-only
+    python -m block_sparse_attention_32_b200.run_workload --workload profile_bwd_4k_r8 --backward
 
 Each pass enqueues the five C-ABI calls (or only index scoring + selection
-with --select-only) on the current stream; the process exits non-zero if a
-kernel reports a device-side error.
+with --select-only; or, after one forward, the attention's backward for a
+seeded upstream gradient with --backward) on the current stream; the process
+exits non-zero if a kernel reports a device-side error.
 """
 from __future__ import annotations
 
@@ -23,6 +25,7 @@ def main(argv=None) -> int:
                     choices=sorted(workloads.ALL))
     ap.add_argument("--passes", type=int, default=2)
     ap.add_argument("--select-only", action="store_true")
+    ap.add_argument("--backward", action="store_true")
     args = ap.parse_args(argv)
     w = workloads.ALL[args.workload]
     d = pipeline.dims_for(w)
@@ -36,6 +39,14 @@ def main(argv=None) -> int:
         for _ in range(args.passes):
             capi.msa_index_score_maxpool(d, inp["q_idx"], inp["k_idx"], pooled, stride, err)
             capi.msa_topk_blocks(d, pooled, stride, sel, err)
+    elif args.backward:
+        buf = pipeline.Buffers.allocate(d)
+        grads = pipeline.Grads.allocate(d)
+        err = buf.dev_err
+        d_out = workloads.upstream_grad(w, "cuda")
+        pipeline.forward(buf, inp["q"], inp["k"], inp["v"], inp["q_idx"], inp["k_idx"])
+        for _ in range(args.passes):
+            pipeline.backward(buf, grads, inp["q"], inp["k"], inp["v"], d_out)
     else:
         buf = pipeline.Buffers.allocate(d)
         err = buf.dev_err

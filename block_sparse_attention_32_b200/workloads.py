@@ -88,7 +88,10 @@ PROFILE_8K = Workload("profile_8k_r8", 1, 8192, 8192, 0, 32, 4, 128, seed=3, sin
 # K/V 4.3 GB), larger than L2.
 PROFILE_DECODE = Workload("profile_decode_b4", 4, 1, 262144, 262143, 64, 8, 128, seed=5,
                           plants_per_group=2, plant_targets=1)
-ALL = dict(CONFIGS, **{PROFILE_8K.name: PROFILE_8K, PROFILE_DECODE.name: PROFILE_DECODE})
+# Profiling-sized backward: 4096 queries with the 128K workload's heads (dq pieces 2.1 GB).
+PROFILE_BWD = Workload("profile_bwd_4k_r8", 1, 4096, 4096, 0, 64, 8, 128, seed=9)
+ALL = dict(CONFIGS, **{PROFILE_8K.name: PROFILE_8K, PROFILE_DECODE.name: PROFILE_DECODE,
+                       PROFILE_BWD.name: PROFILE_BWD})
 
 
 def small(name, batch, n_q, n_kv, q_pos0, h_q, h_kv, d_idx, seed, **kw) -> Workload:
