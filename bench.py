@@ -594,11 +594,13 @@ def main():
             torch.distributed.destroy_process_group()
         return
 
-    recall = None
-    if not args.no_recall:
-        recall = bench_recall(w)
-    e4m3 = None if args.no_e4m3 else bench_e4m3(w)
-    backward = None if args.no_bwd else bench_backward(w, attn_flops, n_ent, peaks)
+    # the side measurements and the CPU baseline run on a single-GPU run only: with
+    # N > 1 every GPU of the job would stay held while rank 0 alone works
+    single = world == 1
+    recall = bench_recall(w) if single and not args.no_recall else None
+    e4m3 = bench_e4m3(w) if single and not args.no_e4m3 else None
+    backward = (bench_backward(w, attn_flops, n_ent, peaks) if single and not args.no_bwd
+                else None)
 
     # dominant kernel: the longest stage; its bound is the larger of its
     # algorithmic time at the tensor peak and at the HBM peak
@@ -652,7 +654,7 @@ def main():
                 "h2d_bytes_per_step": e2e["h2d_bytes_per_step"],
                 "d2h_bytes_per_step": e2e["d2h_bytes_per_step"]} if e2e else None,
     }
-    if not args.no_cpu:
+    if single and not args.no_cpu:
         line["cpu_baseline"], sample = cpu_baseline(w)
         if recall is not None:
             rec_cpu, tok_cpu = sample.run_next_rows()
