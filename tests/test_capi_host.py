@@ -147,3 +147,17 @@ def test_token_select_and_backward_validation(lib):
     assert b(ctypes.byref(d), good, good, good, good, good, *bad, None, None) == 3
     assert b(ctypes.byref(d), good, good, good, mis, good, *ptrs, None, None) == 3
     assert b(None, good, good, good, good, good, *ptrs, None, None) == 1
+
+
+def test_header_is_plain_c(tmp_path):
+    """include/msa.h compiles as C99 on its own (no C++ or CUDA types in the ABI)."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc") or shutil.which("cc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "use_msa.c"
+    src.write_text('#include "msa.h"\nint main(void) { msa_dims d; (void)d; '
+                   'return (int)msa_num_blocks((const msa_dims*)0) * 0; }\n')
+    subprocess.check_call([gcc, "-std=c99", "-Wall", "-Werror", "-pedantic", "-fsyntax-only",
+                           "-I", os.path.join(ROOT, "include"), str(src)])
