@@ -186,6 +186,12 @@ msa_status check_tensor_u8(const msa_tensor& t) {
 
 }  // namespace
 
+namespace msa {
+// the dims check of every entry point, for the allocation-free list builder
+// (library-internal: hidden like everything but the C ABI)
+msa_status validate_dims(const msa_dims* d) { return check_dims(d); }
+}  // namespace msa
+
 extern "C" {
 
 int64_t msa_num_blocks(const msa_dims* d) {

@@ -200,40 +200,6 @@ def _add_recency(w: Workload, q_idx_b: torch.Tensor, k_idx_b: torch.Tensor):
                 kb.float() + qs[lo:]).to(torch.bfloat16).view(-1, w.d_idx)
 
 
-def random_selection(w: Workload, device="cpu", seed_offset: int = 11):
-    """A valid selection [B, G, n_q, 16] drawn at random (own block + distinct
-    earlier blocks, ascending, -1 padded) -- an input for testing the
-    inversion and attention steps on their own."""
-    device = torch.device(device)
-    gen = _gen(device, w.seed + seed_offset)
-    B, G, n_q = w.batch, w.h_kv, w.n_q
-    pos = w.q_pos0 + torch.arange(n_q, device=device)
-    own = pos // BLOCK
-    out = torch.empty((B, G, n_q, TOPK), dtype=torch.int32, device=device)
-    chunk = max(1, (1 << 26) // max(w.nblk, 1))
-    cidx = torch.arange(w.nblk, device=device)
-    for b in range(B):
-        for g in range(G):
-            for r0 in range(0, n_q, chunk):
-                r1 = min(n_q, r0 + chunk)
-                o = own[r0:r1]
-                key = torch.rand((r1 - r0, w.nblk), generator=gen, device=device)
-                key = torch.where(cidx[None, :] < o[:, None], key, torch.full_like(key, -1.0))
-                k = min(TOPK - 1, w.nblk)
-                top = torch.topk(key, k, dim=1)
-                picked = torch.where(top.values >= 0, top.indices, torch.full_like(top.indices, -1))
-                rows = torch.cat([picked, o[:, None]], dim=1)
-                if rows.shape[1] < TOPK:
-                    pad = torch.full((rows.shape[0], TOPK - rows.shape[1]), -1,
-                                     dtype=rows.dtype, device=device)
-                    rows = torch.cat([rows, pad], dim=1)
-                big = torch.full_like(rows, 1 << 30)
-                rows = torch.where(rows >= 0, rows, big).sort(dim=1).values
-                rows = torch.where(rows == (1 << 30), torch.full_like(rows, -1), rows)
-                out[b, g, r0:r1] = rows.to(torch.int32)
-    return out
-
-
 def upstream_grad(w: Workload, device="cpu", seed_offset: int = 101):
     """A seeded upstream gradient dO [B, n_q, H, 128] (bf16, N(0,1)) for the
     attention's backward."""

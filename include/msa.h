@@ -154,7 +154,8 @@ MSA_API msa_status msa_build_block_query_lists(const msa_dims* dims, const int32
                                        int32_t* dev_err, void* stream);
 
 /* Size of the device scratch array behind msa_build_block_query_lists_noalloc
- * (32 MiB, held on every GPU that loads the library until the process exits). */
+ * (32 MiB per device on which that entry point has run, kept until the
+ * process exits). */
 #define MSA_NOALLOC_SCRATCH_BYTES (32u << 20)
 
 /* Allocation-free variant of msa_build_block_query_lists (the paper has no
@@ -162,16 +163,23 @@ MSA_API msa_status msa_build_block_query_lists(const msa_dims* dims, const int32
  * that cannot call cudaMalloc or any allocating routine where they build the
  * lists -- e.g. a plugin inside a serving process whose host owns all device
  * memory through its own pool, or a latency-critical loop that must not
- * allocate.  Same arguments and results as msa_build_block_query_lists, minus
- * the workspace: the scratch is a file-scope device array of
- * MSA_NOALLOC_SCRATCH_BYTES, and problems needing more
- * (msa_block_query_lists_workspace(dims) > MSA_NOALLOC_SCRATCH_BYTES) are
+ * allocate.  Same arguments, results and status codes as
+ * msa_build_block_query_lists, minus the workspace: the scratch is a
+ * file-scope device array of MSA_NOALLOC_SCRATCH_BYTES, and problems needing
+ * more (msa_block_query_lists_workspace(dims) > MSA_NOALLOC_SCRATCH_BYTES) are
  * rejected with MSA_ERR_SCRATCH_LIMIT before anything is enqueued.  For
  * example the 32K prefill (8 groups), the 64 x 256K decode and an 8192-query
  * chunk after a 1M-token cache fit; a 128K-token prefill with 8 groups does not.
- *   - The first call on a device looks up the array's device address with
- *     cudaGetSymbolAddress (with that device current); make that first call
- *     before any stream capture.
+ *   - The array is committed on a device when the library's module that holds
+ *     it is loaded there.  Under CUDA's default lazy module loading that is the
+ *     first call of this entry point on the device (under
+ *     CUDA_MODULE_LOADING=EAGER, the creation of the context).  A host that
+ *     reserves device memory for its own pool should make that first call
+ *     before the reservation; otherwise the call can fail with MSA_ERR_CUDA.
+ *   - The first call in a context looks up the array's device address with
+ *     cudaGetSymbolAddress (with that device current); so does the first call
+ *     after the device's context changed (e.g. after cudaDeviceReset).  Make
+ *     that first call before any stream capture.
  *   - Nothing is allocated or freed.  Every call shares the one array, which
  *     keeps the previous call's contents; its contents on entry do not matter
  *     (every word is written before it is read).  Calls that overlap on the

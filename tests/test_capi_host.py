@@ -115,6 +115,27 @@ def test_pointer_and_stride_checks(lib):
     assert lib.msa_status_string(4) == b"MSA_ERR_WORKSPACE_TOO_SMALL"
 
 
+def test_noalloc_builder_returns_the_workspace_builders_statuses(lib):
+    """On rejected arguments the allocation-free list builder returns the same
+    status as the workspace one (both stop before any CUDA call)."""
+    P = ctypes.c_void_p
+    ws_fn, na_fn = lib.msa_build_block_query_lists, lib.msa_build_block_query_lists_noalloc
+    cases = [capi.make_dims(1, 100, 100, 0, 64, 2, 64),       # R = 32: unsupported
+             capi.make_dims(1, 100, 100, 0, 8, 2, 96),        # d_idx 96: unsupported
+             capi.make_dims(1, 100, 100, 0, 12, 4, 64),       # R = 3: unsupported
+             capi.make_dims(0, 100, 100, 0, 8, 2, 64),        # batch 0: invalid
+             capi.make_dims(1, 100, 100, 50, 8, 2, 64)]       # q_pos0 + n_q > n_kv: invalid
+    for d in cases:
+        want = ws_fn(ctypes.byref(d), P(0x1000), P(0x2000), P(0x3000), P(0x4000), 1 << 30,
+                     None, None)
+        got = na_fn(ctypes.byref(d), P(0x1000), P(0x2000), P(0x3000), None, None)
+        assert want in (1, 2) and got == want, (want, got)
+    assert na_fn(None, P(0x1000), P(0x2000), P(0x3000), None, None) == 1
+    d = capi.make_dims(1, 1000, 4096, 0, 8, 2, 128)
+    assert na_fn(ctypes.byref(d), P(0x1000), None, P(0x3000), None, None) == 1
+    assert na_fn(ctypes.byref(d), P(0x1004), P(0x2000), P(0x3000), None, None) == 3
+
+
 def test_token_select_and_backward_validation(lib):
     """The token-level and backward entry points reject bad arguments on the
     host, before anything is enqueued."""
