@@ -63,11 +63,11 @@ def work_counts(w):
     return idx_flops, attn_flops, n_entries
 
 
-def bytes_model(w, n_entries, n_pieces_nonempty):
+def bytes_model(w, n_entries, n_pieces_nonempty, piece_bytes=520):
     """Algorithmic DRAM bytes per launch of each kernel.
 
     attention: per (query, block) entry the R gathered Q rows (256 B each) and
-    the R fp32 pieces written (512 B acc + 8 B (m, l)); per selected (batch,
+    the R pieces written (fp32: 512 B acc + 8 B (m, l); compact: 256 + 8); per selected (batch,
     group, block) the 64 KB K/V tile once; the entry list.  merge: the pieces
     read once, sel, and the bf16 output + lse written."""
     B, G, R = w.batch, w.h_kv, w.h_q // w.h_kv
@@ -79,8 +79,9 @@ def bytes_model(w, n_entries, n_pieces_nonempty):
                        + 4 * B * G * own.sum()),
         "topk": float(4 * B * G * own[own >= 16].sum() + 64 * rows),
         "block_lists": float(64 * rows * 2 + 4 * n_entries * 2),
-        "attn": float(n_entries * R * (256 + 520) + n_pieces_nonempty * 65536 + 4 * n_entries),
-        "merge": float(n_entries * R * 520 + 64 * rows + B * w.n_q * w.h_q * (256 + 4)),
+        "attn": float(n_entries * R * (256 + piece_bytes) + n_pieces_nonempty * 65536
+                      + 4 * n_entries),
+        "merge": float(n_entries * R * piece_bytes + 64 * rows + B * w.n_q * w.h_q * (256 + 4)),
     }
 
 
@@ -157,6 +158,26 @@ class Stages:
         return {n: self.ev[i].elapsed_time(self.ev[i + 1]) for i, n in enumerate(self.NAMES)}
 
 
+def percentile(xs, q):
+    """q-th percentile (0..100) of xs by linear interpolation between order statistics."""
+    v = sorted(xs)
+    if len(v) == 1:
+        return v[0]
+    pos = (len(v) - 1) * q / 100.0
+    lo = int(math.floor(pos))
+    hi = min(lo + 1, len(v) - 1)
+    return v[lo] + (v[hi] - v[lo]) * (pos - lo)
+
+
+def stage_percentiles(per_step):
+    """{stage: {p50, p95, p99, min, max}} over the timed steps' event times (ms)."""
+    return {n: {"p50": percentile([x[n] for x in per_step], 50),
+                "p95": percentile([x[n] for x in per_step], 95),
+                "p99": percentile([x[n] for x in per_step], 99),
+                "min": min(x[n] for x in per_step), "max": max(x[n] for x in per_step)}
+            for n in Stages.NAMES}
+
+
 def run_step(pipeline, capi, buf, inp, stages=None):
     d = buf.dims
     ev = stages.ev if stages else None
@@ -169,11 +190,12 @@ def run_step(pipeline, capi, buf, inp, stages=None):
     capi.msa_build_block_query_lists(d, buf.sel, buf.blk_offsets, buf.entries, buf.ws,
                                      buf.dev_err)
     if ev: ev[3].record()
-    capi.msa_sparse_attn_fwd(d, inp["q"], inp["k"], inp["v"], buf.blk_offsets, buf.entries,
-                             buf.part_ml, buf.part_acc, buf.dev_err)
+    fwd = capi.msa_sparse_attn_fwd_compact if buf.compact else capi.msa_sparse_attn_fwd
+    merge = capi.msa_merge_partials_compact if buf.compact else capi.msa_merge_partials
+    fwd(d, inp["q"], inp["k"], inp["v"], buf.blk_offsets, buf.entries, buf.part_ml, buf.part_acc,
+        buf.dev_err)
     if ev: ev[4].record()
-    capi.msa_merge_partials(d, buf.sel, buf.part_ml, buf.part_acc, buf.out, buf.lse,
-                            buf.dev_err)
+    merge(d, buf.sel, buf.part_ml, buf.part_acc, buf.out, buf.lse, buf.dev_err)
     if ev: ev[5].record()
 
 
@@ -203,10 +225,10 @@ def job_throughput(units_per_rank, ms_local, world):
     return world * units_per_rank / (ms / 1000.0), ms
 
 
-def bench_workload(w, steps, warmup, world, rank, with_e2e=True):
+def bench_workload(w, steps, warmup, world, rank, with_e2e=True, compact=False):
     from block_sparse_attention_32_b200 import capi, pipeline, workloads as wl
     d = pipeline.dims_for(w)
-    buf = pipeline.Buffers.allocate(d)
+    buf = pipeline.Buffers.allocate(d, compact=compact)
     inp = wl.make_inputs(w, "cuda")
     torch.cuda.synchronize()
     for _ in range(warmup):
@@ -226,8 +248,9 @@ def bench_workload(w, steps, warmup, world, rank, with_e2e=True):
     torch.cuda.synchronize()
     barrier(world)
     total_ms = start.elapsed_time(end)
-    per_stage = {n: statistics.median(st.ms()[n] for st in stages) for n in Stages.NAMES}
-    per_stage_mean = {n: sum(st.ms()[n] for st in stages) / steps for n in Stages.NAMES}
+    per_step = [st.ms() for st in stages]
+    per_stage = stage_percentiles(per_step)
+    per_stage_mean = {n: sum(x[n] for x in per_step) / steps for n in Stages.NAMES}
     if int(buf.dev_err[0]) != 0:
         raise RuntimeError(f"device error {int(buf.dev_err[0])} during timing")
 
@@ -349,6 +372,85 @@ def bench_recall(w, n_rows=64, reps=3):
            "streamed_bytes": streamed, "streamed_gbs": streamed / (ms / 1000.0) / 1e9,
            "dram_bytes_at_most": unique, "token_level": token_level}
     del buf, inp
+    torch.cuda.empty_cache()
+    return out
+
+
+def attention_roofline(w, stage_mean, attn_flops, n_pieces, nbytes, peaks, peak_src):
+    """Roofline of the KV-block-outer attention (A4) on the basis the scope
+    table fixes: a dense bf16 contraction, so tensor-bound, achieved =
+    selected-token FLOPs / its mean event time against the sustained bf16 peak
+    (it runs inside a long step).  Beside it: the same over attention + merge,
+    the algorithmic bytes (Q read once, the selected K/V blocks once, O written
+    once), the measured DRAM traffic per launch when the committed ncu record
+    matches the current sources, and the design's own byte model (gathered Q
+    rows, fp32 pieces, K/V per segment) as an HBM fraction."""
+    sustained = peaks.get("bf16_tflops_sustained", FALLBACK["bf16_tflops_sustained"])
+    burst = peaks.get("bf16_tflops", FALLBACK["bf16_tflops"])
+    hbm = peaks.get("hbm_gbs", FALLBACK["hbm_gbs"])
+    secs = stage_mean["attn"] / 1000.0
+    secs_m = (stage_mean["attn"] + stage_mean["merge"]) / 1000.0
+    ach = attn_flops / secs / 1e12
+    ach_m = attn_flops / secs_m / 1e12
+    qo = float(w.batch * w.n_q * w.h_q * 128 * 2)
+    algo = 2 * qo + float(n_pieces) * 65536
+    traffic = measured_traffic(["sparse_attn.cu", "common.cuh"],
+                               "sparse_attn_dram_traffic_prefill_128k.txt")
+    return {"bound": "tensor", "achieved": ach, "peak": sustained, "unit": "TFLOP/s",
+            "frac": ach / sustained, "frac_of_burst": ach / burst,
+            "peak_source": f"{peak_src} bf16_tflops_sustained",
+            "with_merge": {"achieved": ach_m, "frac": ach_m / sustained},
+            "algorithmic_flops": attn_flops,
+            "algorithmic_bytes": algo,
+            "traffic": traffic,
+            "traffic_over_algorithmic": (traffic / algo) if traffic else None,
+            "design_bytes": nbytes["attn"],
+            "design_bytes_hbm_frac": nbytes["attn"] / secs / 1e9 / hbm,
+            "merge_bytes": nbytes["merge"],
+            "merge_hbm_frac": nbytes["merge"] / (stage_mean["merge"] / 1000.0) / 1e9 / hbm}
+
+
+def bench_compact(w, steps, warmup, peaks, peak_src):
+    """The same pass with compact pieces (acc / l in bf16, fp32 m and l; an
+    opt-in of the library): queries/s, stage times and the attention's
+    roofline, with the piece bytes of this format in the design byte model."""
+    total_ms, pct, mean, _, n_pieces = bench_workload(w, steps, warmup, 1, 0, with_e2e=False,
+                                                      compact=True)
+    idx_flops, attn_flops, n_ent = work_counts(w)
+    nbytes = bytes_model(w, n_ent, n_pieces, piece_bytes=264)
+    roof = attention_roofline(w, mean, attn_flops, n_pieces, nbytes, peaks, peak_src)
+    roof["traffic"] = None
+    roof["traffic_over_algorithmic"] = None
+    ms = total_ms / steps
+    return {"workload": w.name, "pieces": "bf16 acc / l + fp32 (m, l): 264 B per (query, head, block)",
+            "queries_per_s": w.batch * w.n_q / (ms / 1000.0), "ms_per_step": ms, "steps": steps,
+            "stages_ms": mean, "stages_ms_pct": pct, "attention_roofline": roof,
+            "selected_token_attn_tflops": attn_flops / (mean["attn"] / 1000.0) / 1e12,
+            "selected_token_attn_merge_tflops":
+                attn_flops / ((mean["attn"] + mean["merge"]) / 1000.0) / 1e12}
+
+
+def bench_config(w, steps, warmup, peaks, with_cpu=True):
+    """One more configuration of the pages' long-context workloads timed the
+    same way as the headline pass (device-resident inputs, events between the
+    five calls): queries/s, per-stage times with percentiles, the index and
+    attention contractions against the bf16 peaks, and the CPU oracle's
+    queries/s on a bounded sample of the same rows (about 4 s)."""
+    total_ms, pct, mean, _, n_pieces = bench_workload(w, steps, warmup, 1, 0, with_e2e=False)
+    idx_flops, attn_flops, n_ent = work_counts(w)
+    sustained = peaks.get("bf16_tflops_sustained", FALLBACK["bf16_tflops_sustained"])
+    burst = peaks.get("bf16_tflops", FALLBACK["bf16_tflops"])
+    ms = total_ms / steps
+    idx_t = idx_flops / (mean["index"] / 1000.0) / 1e12
+    attn_t = attn_flops / (mean["attn"] / 1000.0) / 1e12
+    out = {"workload": w.name, "queries_per_s": w.batch * w.n_q / (ms / 1000.0),
+           "ms_per_step": ms, "steps": steps, "stages_ms": mean, "stages_ms_pct": pct,
+           "index": {"tflops": idx_t, "frac_sustained": idx_t / sustained,
+                     "frac_burst": idx_t / burst, "algorithmic_flops": idx_flops},
+           "attn": {"tflops": attn_t, "frac_sustained": attn_t / sustained,
+                    "algorithmic_flops": attn_flops, "entries": n_ent}}
+    if with_cpu:
+        out["cpu_baseline"] = CpuOracleSample(w, target_s=4.0).run()
     torch.cuda.empty_cache()
     return out
 
@@ -521,6 +623,8 @@ def main():
     ap.add_argument("--no-recall", action="store_true")
     ap.add_argument("--no-e4m3", action="store_true")
     ap.add_argument("--no-bwd", action="store_true")
+    ap.add_argument("--no-configs", action="store_true")
+    ap.add_argument("--no-compact", action="store_true")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -564,7 +668,7 @@ def main():
 
     clk_path = os.path.join(tempfile.gettempdir(), f"msa_bench_clocks_{os.getpid()}.csv")
     proc = sample_clocks(None, clk_path) if rank == 0 else None
-    total_ms, stage_med, stage_mean, e2e, n_pieces = bench_workload(w, args.steps, args.warmup,
+    total_ms, stage_pct, stage_mean, e2e, n_pieces = bench_workload(w, args.steps, args.warmup,
                                                                     world, rank)
     if proc is not None:
         proc.terminate()
@@ -576,15 +680,16 @@ def main():
     decode = None
     if not args.no_decode:
         dw = wl.DECODE
-        dms, dstage, _, _, dpieces = bench_workload(dw, max(3, args.steps), args.warmup, world,
-                                                    rank, with_e2e=False)
-        dtps, dms = job_throughput(dw.batch, dms / max(3, args.steps), world)
+        dsteps = max(3, args.steps)
+        dms, dpct, dmean, _, dpieces = bench_workload(dw, dsteps, args.warmup, world, rank,
+                                                      with_e2e=False)
+        dtps, dms = job_throughput(dw.batch, dms / dsteps, world)
         kidx_bytes = dw.batch * dw.n_kv * dw.d_idx * 2
         sel_kv_bytes = dpieces * 65536
         read_bytes = kidx_bytes + sel_kv_bytes
         decode = {"workload": dw.name, "tokens_per_s": dtps,
-                  "ms_per_step": dms, "stages_ms": dstage,
-                  "index_scan_gbs": kidx_bytes / (dstage["index"] / 1000.0) / 1e9,
+                  "ms_per_step": dms, "stages_ms": dmean, "stages_ms_pct": dpct,
+                  "index_scan_gbs": kidx_bytes / (dmean["index"] / 1000.0) / 1e9,
                   "bytes_read_per_step": read_bytes,
                   "hbm_frac_on_bytes_read": read_bytes / (dms / 1000.0) / 1e9
                   / peaks.get("hbm_gbs", FALLBACK["hbm_gbs"])}
@@ -601,32 +706,37 @@ def main():
     e4m3 = bench_e4m3(w) if single and not args.no_e4m3 else None
     backward = (bench_backward(w, attn_flops, n_ent, peaks) if single and not args.no_bwd
                 else None)
+    compact = (bench_compact(w, max(3, args.steps // 2), args.warmup, peaks, peak_src)
+               if single and not args.no_compact else None)
+    configs = ({c.name: bench_config(c, max(3, args.steps // 2), args.warmup, peaks,
+                                     with_cpu=not args.no_cpu)
+                for c in (wl.P32, wl.M1)} if single and not args.no_configs else None)
 
-    # dominant kernel: the longest stage; its bound is the larger of its
-    # algorithmic time at the tensor peak and at the HBM peak
-    dom = max(stage_mean, key=stage_mean.get)
     sustained = peaks.get("bf16_tflops_sustained", FALLBACK["bf16_tflops_sustained"])
+    burst = peaks.get("bf16_tflops", FALLBACK["bf16_tflops"])
     hbm = peaks.get("hbm_gbs", FALLBACK["hbm_gbs"])
     nbytes = bytes_model(w, n_ent, n_pieces)
-    flops = {"index": idx_flops, "attn": attn_flops}.get(dom, 0.0)
-    secs = stage_mean[dom] / 1000.0
-    t_tensor = flops / (sustained * 1e12)
-    t_hbm = nbytes[dom] / (hbm * 1e9)
-    if t_tensor >= t_hbm:
-        ach = flops / secs / 1e12
-        roof = {"kernel": dom, "bound": "tensor", "achieved": ach, "peak": sustained,
+    attn_roof = attention_roofline(w, stage_mean, attn_flops, n_pieces, nbytes, peaks, peak_src)
+    # dominant kernel: the longest stage.  Index scoring and the attention are
+    # dense bf16 contractions (tensor-bound by the algorithmic work, SURVEY-style
+    # FLOP counts); the other stages are HBM-bound on the bytes they must move.
+    dom = max(stage_mean, key=stage_mean.get)
+    if dom == "attn":
+        roof = dict(attn_roof)
+        roof["kernel"] = "attn"
+    elif dom == "index":
+        secs = stage_mean["index"] / 1000.0
+        ach = idx_flops / secs / 1e12
+        roof = {"kernel": "index", "bound": "tensor", "achieved": ach, "peak": sustained,
                 "unit": "TFLOP/s", "frac": ach / sustained,
-                "peak_source": f"{peak_src} bf16_tflops_sustained"}
+                "peak_source": f"{peak_src} bf16_tflops_sustained",
+                "frac_of_burst": ach / burst, "traffic": None}
     else:
+        secs = stage_mean[dom] / 1000.0
         ach = nbytes[dom] / secs / 1e9
         roof = {"kernel": dom, "bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s",
                 "frac": ach / hbm, "peak_source": f"{peak_src} hbm_gbs",
-                "algorithmic_bytes": nbytes[dom]}
-        if flops:
-            roof["tensor_frac"] = flops / secs / 1e12 / sustained
-    roof["traffic"] = (measured_traffic(["sparse_attn.cu", "common.cuh"],
-                                        "sparse_attn_dram_traffic_prefill_128k.txt")
-                       if dom == "attn" else None)
+                "algorithmic_bytes": nbytes[dom], "traffic": None}
 
     attn_tflops = attn_flops / (stage_mean["attn"] / 1000.0) / 1e12
     attn_merge_tflops = attn_flops / ((stage_mean["attn"] + stage_mean["merge"]) / 1000.0) / 1e12
@@ -643,7 +753,14 @@ def main():
         "selected_token_attn_merge_tflops": attn_merge_tflops,
         "index_tflops": idx_flops / (stage_mean["index"] / 1000.0) / 1e12,
         "stages_ms": stage_mean,
+        "stages_ms_pct": stage_pct,
+        "stage_conditions": {"steps": args.steps, "stream": "one stream, events between calls",
+                             "sm_mhz_median": clocks["sm_mhz"] if clocks else None,
+                             "reasons": clocks["reasons"] if clocks else None},
+        "attention_roofline": attn_roof,
+        "compact_pieces": compact,
         "decode": decode,
+        "configs": configs,
         "selection_recall": recall,
         "index_e4m3": e4m3,
         "backward": backward,

@@ -36,7 +36,8 @@ class MSAError(RuntimeError):
 class Dims(ctypes.Structure):
     _fields_ = [("batch", ctypes.c_int64), ("n_q", ctypes.c_int64), ("n_kv", ctypes.c_int64),
                 ("q_pos0", ctypes.c_int64), ("h_q", ctypes.c_int32), ("h_kv", ctypes.c_int32),
-                ("h_kidx", ctypes.c_int32), ("d_idx", ctypes.c_int32), ("scale", ctypes.c_float)]
+                ("h_kidx", ctypes.c_int32), ("d_idx", ctypes.c_int32), ("scale", ctypes.c_float),
+                ("q_window", ctypes.c_int32)]
 
 
 class Tensor(ctypes.Structure):
@@ -61,6 +62,10 @@ def load_library(path: str) -> ctypes.CDLL:
     L.msa_num_blocks.restype = ctypes.c_int64
     L.msa_num_entries.argtypes = [_PD]
     L.msa_num_entries.restype = ctypes.c_int64
+    L.msa_query_window.argtypes = [_PD]
+    L.msa_query_window.restype = ctypes.c_int64
+    L.msa_num_segments.argtypes = [_PD]
+    L.msa_num_segments.restype = ctypes.c_int64
     L.msa_index_score_maxpool.argtypes = [_PD, Tensor, Tensor, _P, ctypes.c_int64, _P, _P]
     L.msa_topk_blocks.argtypes = [_PD, _P, ctypes.c_int64, _P, _P, _P]
     L.msa_block_query_lists_workspace.argtypes = [_PD]
@@ -69,6 +74,9 @@ def load_library(path: str) -> ctypes.CDLL:
     L.msa_build_block_query_lists_noalloc.argtypes = [_PD, _P, _P, _P, _P, _P]
     L.msa_sparse_attn_fwd.argtypes = [_PD, Tensor, Tensor, Tensor, _P, _P, _P, _P, _P, _P]
     L.msa_merge_partials.argtypes = [_PD, _P, _P, _P, _P, _P, _P, _P]
+    L.msa_sparse_attn_fwd_compact.argtypes = [_PD, Tensor, Tensor, Tensor, _P, _P, _P, _P, _P,
+                                              _P]
+    L.msa_merge_partials_compact.argtypes = [_PD, _P, _P, _P, _P, _P, _P, _P]
     L.msa_quantize_e4m3.argtypes = [_P, ctypes.c_int64, _P, _P, _P]
     L.msa_index_score_maxpool_e4m3.argtypes = [_PD, Tensor, Tensor, _P, _P, _P, ctypes.c_int64,
                                                _P, _P]
@@ -84,10 +92,13 @@ def load_library(path: str) -> ctypes.CDLL:
     L.msa_token_select_attention.argtypes = [_PD, Tensor, Tensor, Tensor, Tensor, Tensor, _P,
                                              ctypes.c_int64, ctypes.c_int64, _P, _P, _P, _P,
                                              ctypes.c_size_t, _P, _P]
+    L.msa_debug_set_attn_wait_limit_ns.argtypes = [ctypes.c_uint64]
+    L.msa_debug_set_attn_wait_limit_ns.restype = ctypes.c_uint64
     L.msa_status_string.argtypes = [ctypes.c_int]
     L.msa_status_string.restype = ctypes.c_char_p
     for f in (L.msa_index_score_maxpool, L.msa_topk_blocks, L.msa_build_block_query_lists,
               L.msa_build_block_query_lists_noalloc, L.msa_sparse_attn_fwd, L.msa_merge_partials,
+              L.msa_sparse_attn_fwd_compact, L.msa_merge_partials_compact,
               L.msa_selection_recall, L.msa_quantize_e4m3, L.msa_index_score_maxpool_e4m3,
               L.msa_token_select_attention, L.msa_sparse_attn_bwd):
         f.restype = ctypes.c_int
@@ -103,10 +114,11 @@ def lib() -> ctypes.CDLL:
     return _lib
 
 
-def make_dims(batch, n_q, n_kv, q_pos0, h_q, h_kv, d_idx, h_kidx=1, scale=None) -> Dims:
+def make_dims(batch, n_q, n_kv, q_pos0, h_q, h_kv, d_idx, h_kidx=1, scale=None,
+              q_window=0) -> Dims:
     if scale is None:
         scale = HEAD_DIM ** -0.5
-    return Dims(batch, n_q, n_kv, q_pos0, h_q, h_kv, h_kidx, d_idx, scale)
+    return Dims(batch, n_q, n_kv, q_pos0, h_q, h_kv, h_kidx, d_idx, scale, q_window)
 
 
 def _ptr(t) -> int:
@@ -140,6 +152,20 @@ def msa_num_blocks(d: Dims) -> int:
 
 def msa_num_entries(d: Dims) -> int:
     return lib().msa_num_entries(ctypes.byref(d))
+
+
+def msa_query_window(d: Dims) -> int:
+    return lib().msa_query_window(ctypes.byref(d))
+
+
+def msa_num_segments(d: Dims) -> int:
+    return lib().msa_num_segments(ctypes.byref(d))
+
+
+def msa_debug_set_attn_wait_limit_ns(ns: int) -> int:
+    """Time limit (ns) of the attention kernel's barrier waits for later calls;
+    returns the previous one (0 restores the default 2 s)."""
+    return int(lib().msa_debug_set_attn_wait_limit_ns(ns))
 
 
 def msa_block_query_lists_workspace(d: Dims) -> int:
@@ -179,6 +205,26 @@ def msa_sparse_attn_fwd(d: Dims, q, k, v, blk_offsets, entries, part_ml, part_ac
            lib().msa_sparse_attn_fwd(ctypes.byref(d), tensor_btd(q), tensor_bhtd(k),
                                      tensor_bhtd(v), _ptr(blk_offsets), _ptr(entries),
                                      _ptr(part_ml), _ptr(part_acc), _ptr(dev_err), _stream()))
+
+
+def msa_sparse_attn_fwd_compact(d: Dims, q, k, v, blk_offsets, entries, part_ml, part_acc16,
+                                dev_err=None):
+    """As msa_sparse_attn_fwd with compact pieces: part_acc16 bf16 [B,n_q,G,16,R,128]
+    holds acc / l."""
+    assert part_acc16.dtype == torch.bfloat16
+    _check("msa_sparse_attn_fwd_compact",
+           lib().msa_sparse_attn_fwd_compact(ctypes.byref(d), tensor_btd(q), tensor_bhtd(k),
+                                             tensor_bhtd(v), _ptr(blk_offsets), _ptr(entries),
+                                             _ptr(part_ml), _ptr(part_acc16), _ptr(dev_err),
+                                             _stream()))
+
+
+def msa_merge_partials_compact(d: Dims, sel, part_ml, part_acc16, out, lse, dev_err=None):
+    assert part_acc16.dtype == torch.bfloat16
+    _check("msa_merge_partials_compact",
+           lib().msa_merge_partials_compact(ctypes.byref(d), _ptr(sel), _ptr(part_ml),
+                                            _ptr(part_acc16), _ptr(out), _ptr(lse),
+                                            _ptr(dev_err), _stream()))
 
 
 def msa_sparse_attn_bwd(d: Dims, q, k, v, o, d_o, lse, blk_offsets, entries, delta, part_dq, dq,

@@ -6,18 +6,25 @@
 // and computed together, so each block is read once.  The inversion itself is
 // not spelled out on the pages; this is a deterministic counting sort.
 //
-// Segments are (batch, group, block) in that order; inside a segment the
-// entries (i << 4 | slot) are ascending in the query index i.  Steps:
+// The query indices are cut into windows of W consecutive queries (W a
+// multiple of the 128-query tile); segments are (batch, group, window, block)
+// in that order, and inside a segment the entries (i << 4 | slot) are
+// ascending in the query index i.  A KV-block-outer kernel that walks the
+// segments in order then gathers, at any time, the query rows of one window
+// only, which stay in L2.  Steps:
 //   1. count:   per 128-query tile, a shared-memory histogram over blocks;
-//   2. colscan: per block, exclusive prefix over tiles (in place) + totals
-//      (coalesced two-pass form for many tiles, one thread per column else);
+//   2. colscan: per (window, block), exclusive prefix over the window's tiles
+//      (in place) + totals (coalesced two-pass form for many tiles, one
+//      thread per column else);
 //   3. offsets: exclusive scan of the totals over all segments (chunk sums,
 //      scan of the chunk sums, chunk-local scans);
 //   4. scatter: per tile, queries in ascending order claim consecutive slots
 //      of each block's range, so the order never depends on timing.
-// Workspace: tile histograms [B*G, ntiles, nblk] + totals [B*G*nblk] + chunk
-// sums [ceil(B*G*nblk / 4096)], int32.  One query per row (decode) takes a
+// Workspace: tile histograms [B*G, ntiles, nblk] + totals [B*G*nwin*nblk] +
+// chunk sums [ceil(B*G*nwin*nblk / 4096)], int32.  One query per row (decode) takes a
 // two-launch path that needs only the per-row counts.
+#include <algorithm>
+
 #include "common.cuh"
 
 namespace msa {
@@ -51,39 +58,49 @@ __global__ void __launch_bounds__(256)
   for (int c = threadIdx.x; c < nblk; c += blockDim.x) dst[c] = hist[c];
 }
 
-// Column scan for few tiles (decode): one thread per (segment), walking its tiles.
+// Column scan for few tiles per window: one thread per (batch-group, block),
+// walking all tiles; the prefix restarts at every window boundary (tw tiles).
 __global__ void __launch_bounds__(256)
     csr_colscan_small_kernel(int32_t* __restrict__ tile_counts, int32_t* __restrict__ totals,
-                             int32_t nblk, int32_t ntiles) {
+                             int32_t nblk, int32_t ntiles, int32_t tw, int32_t nwin) {
   const int c = blockIdx.x * blockDim.x + threadIdx.x;
   const int64_t bg = blockIdx.y;
   if (c >= nblk) return;
   int32_t* col = tile_counts + bg * ntiles * (int64_t)nblk + c;
   int32_t run = 0;
+  int w = 0;
   for (int t = 0; t < ntiles; ++t) {
+    if (t == (w + 1) * tw) {
+      totals[(bg * nwin + w) * nblk + c] = run;
+      run = 0;
+      ++w;
+    }
     const int32_t v = col[(int64_t)t * nblk];
     col[(int64_t)t * nblk] = run;
     run += v;
   }
-  totals[bg * nblk + c] = run;
+  totals[(bg * nwin + w) * nblk + c] = run;
 }
 
 // Column scan, coalesced: a block takes 32 adjacent blocks (one per lane) of
-// one (batch, group) and its 8 warps split the query tiles; each warp sums its
-// tiles, the warps' partial sums give each warp its starting prefix, and a
-// second pass writes the exclusive prefixes in place.
+// one (batch, group, window) and its 8 warps split the window's query tiles;
+// each warp sums its tiles, the warps' partial sums give each warp its
+// starting prefix, and a second pass writes the exclusive prefixes in place.
 constexpr int kColWarps = 8;
 
 __global__ void __launch_bounds__(kColWarps * 32)
     csr_colscan_kernel(int32_t* __restrict__ tile_counts, int32_t* __restrict__ totals,
-                       int32_t nblk, int32_t ntiles) {
+                       int32_t nblk, int32_t ntiles, int32_t tw, int32_t nwin) {
   __shared__ int32_t part[kColWarps][32];
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   const int c = blockIdx.x * 32 + lane;
-  const int64_t bg = blockIdx.y;
+  const int64_t bgw = blockIdx.y;                 // (batch-group) * nwin + window
+  const int64_t bg = bgw / nwin;
+  const int win = (int)(bgw - bg * nwin);
   int32_t* col = tile_counts + bg * ntiles * (int64_t)nblk + c;
-  const int per = (ntiles + kColWarps - 1) / kColWarps;
-  const int t0 = min(ntiles, w * per), t1 = min(ntiles, t0 + per);
+  const int wt0 = win * tw, wt1 = min(ntiles, wt0 + tw);
+  const int per = (wt1 - wt0 + kColWarps - 1) / kColWarps;
+  const int t0 = min(wt1, wt0 + w * per), t1 = min(wt1, t0 + per);
   int32_t s = 0;
   if (c < nblk) {
 #pragma unroll 8
@@ -104,7 +121,7 @@ __global__ void __launch_bounds__(kColWarps * 32)
       col[(int64_t)t * nblk] = run;
       run += v;
     }
-    if (w == 0) totals[bg * nblk + c] = total;
+    if (w == 0) totals[bgw * nblk + c] = total;
   }
 }
 
@@ -199,7 +216,8 @@ __global__ void __launch_bounds__(kScanThreads)
 
 __global__ void __launch_bounds__(32)
     csr_scatter_kernel(const int32_t* __restrict__ sel, int64_t n_q, int64_t q_pos0,
-                       int32_t nblk, int32_t ntiles, const int32_t* __restrict__ tile_counts,
+                       int32_t nblk, int32_t ntiles, int32_t tw, int32_t nwin,
+                       const int32_t* __restrict__ tile_counts,
                        const int32_t* __restrict__ offsets, int32_t* __restrict__ entries,
                        int64_t cap) {
   extern __shared__ int32_t base[];
@@ -207,7 +225,7 @@ __global__ void __launch_bounds__(32)
   const int64_t bg = blockIdx.y;
   const int lane = threadIdx.x;
   const int32_t* tc = tile_counts + (bg * ntiles + tile) * (int64_t)nblk;
-  const int32_t* off = offsets + bg * nblk;
+  const int32_t* off = offsets + (bg * nwin + tile / tw) * nblk;
   for (int c = lane; c < nblk; c += 32) base[c] = off[c] + tc[c];
   __syncwarp();
   const int64_t q0 = (int64_t)tile * kCsrTile;
@@ -297,18 +315,20 @@ __global__ void __launch_bounds__(kRowWarps * 32)
   if (r == n_rows - 1 && lane == 0) offsets[n_rows * nblk] = row_base[w + 1];
 }
 
-size_t block_lists_workspace(int64_t bgcount, int64_t n_q, int64_t nblk) {
+size_t block_lists_workspace(int64_t bgcount, int64_t n_q, int64_t nblk, int64_t window) {
   const int64_t ntiles = (n_q + kCsrTile - 1) / kCsrTile;
-  const int64_t nseg = bgcount * nblk;
+  const int64_t nwin = (n_q + window - 1) / window;
+  const int64_t nseg = bgcount * nwin * nblk;
   const int64_t nchunks = (nseg + kScanChunk - 1) / kScanChunk;
-  return (size_t)(nseg * (ntiles + 1) + nchunks) * sizeof(int32_t);
+  return (size_t)(bgcount * ntiles * nblk + nseg + nchunks) * sizeof(int32_t);
 }
 
 cudaError_t launch_block_lists(const int32_t* sel, int64_t bgcount, int64_t n_q,
-                               int64_t q_pos0, int64_t nblk, int32_t* offsets,
+                               int64_t q_pos0, int64_t nblk, int64_t window, int32_t* offsets,
                                int32_t* entries, int64_t cap, void* ws, int32_t* err,
                                cudaStream_t st) {
   if (n_q == 1) {
+    // one window: segment (bg, c) = bg * nblk + c
     int32_t* counts = reinterpret_cast<int32_t*>(ws);
     const unsigned grid = (unsigned)((bgcount + kRowWarps - 1) / kRowWarps);
     csr_rows_count_kernel<<<grid, kRowWarps * 32, 0, st>>>(sel, bgcount, q_pos0, (int32_t)nblk,
@@ -318,6 +338,8 @@ cudaError_t launch_block_lists(const int32_t* sel, int64_t bgcount, int64_t n_q,
     return cudaGetLastError();
   }
   const int64_t ntiles = (n_q + kCsrTile - 1) / kCsrTile;
+  const int64_t nwin = (n_q + window - 1) / window;
+  const int32_t tw = (int32_t)(window / kCsrTile);        // tiles per window
   int32_t* tile_counts = reinterpret_cast<int32_t*>(ws);
   int32_t* totals = tile_counts + bgcount * ntiles * nblk;
   const size_t hist_bytes = (size_t)nblk * sizeof(int32_t);
@@ -333,16 +355,16 @@ cudaError_t launch_block_lists(const int32_t* sel, int64_t bgcount, int64_t n_q,
   dim3 g1((unsigned)ntiles, (unsigned)bgcount);
   csr_count_kernel<<<g1, 256, hist_bytes, st>>>(sel, n_q, q_pos0, (int32_t)nblk,
                                                 (int32_t)ntiles, tile_counts, err);
-  if (ntiles < 4 * kColWarps) {
+  if (std::min<int64_t>(tw, ntiles) < 4 * kColWarps) {
     dim3 g2((unsigned)((nblk + 255) / 256), (unsigned)bgcount);
     csr_colscan_small_kernel<<<g2, 256, 0, st>>>(tile_counts, totals, (int32_t)nblk,
-                                                 (int32_t)ntiles);
+                                                 (int32_t)ntiles, tw, (int32_t)nwin);
   } else {
-    dim3 g2((unsigned)((nblk + 31) / 32), (unsigned)bgcount);
+    dim3 g2((unsigned)((nblk + 31) / 32), (unsigned)(bgcount * nwin));
     csr_colscan_kernel<<<g2, kColWarps * 32, 0, st>>>(tile_counts, totals, (int32_t)nblk,
-                                                      (int32_t)ntiles);
+                                                      (int32_t)ntiles, tw, (int32_t)nwin);
   }
-  const int64_t nseg = bgcount * nblk;
+  const int64_t nseg = bgcount * nwin * nblk;
   const int64_t nchunks = (nseg + kScanChunk - 1) / kScanChunk;
   int32_t* chunk_sums = totals + nseg;
   csr_chunk_sums_kernel<<<(unsigned)nchunks, kScanThreads, 0, st>>>(totals, nseg, chunk_sums);
@@ -350,8 +372,8 @@ cudaError_t launch_block_lists(const int32_t* sel, int64_t bgcount, int64_t n_q,
   csr_chunk_apply_kernel<<<(unsigned)nchunks, kScanThreads, 0, st>>>(totals, nseg, chunk_sums,
                                                                      offsets);
   csr_scatter_kernel<<<g1, 32, hist_bytes, st>>>(sel, n_q, q_pos0, (int32_t)nblk,
-                                                 (int32_t)ntiles, tile_counts, offsets, entries,
-                                                 cap);
+                                                 (int32_t)ntiles, tw, (int32_t)nwin,
+                                                 tile_counts, offsets, entries, cap);
   return cudaGetLastError();
 }
 

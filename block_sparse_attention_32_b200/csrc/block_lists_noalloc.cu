@@ -15,10 +15,9 @@
 #include "common.cuh"
 
 namespace msa {
-size_t block_lists_workspace(int64_t bgcount, int64_t n_q, int64_t nblk);
 cudaError_t launch_block_lists(const int32_t* sel, int64_t bgcount, int64_t n_q, int64_t q_pos0,
-                               int64_t nblk, int32_t* offsets, int32_t* entries, int64_t cap,
-                               void* ws, int32_t* err, cudaStream_t st);
+                               int64_t nblk, int64_t window, int32_t* offsets, int32_t* entries,
+                               int64_t cap, void* ws, int32_t* err, cudaStream_t st);
 msa_status validate_dims(const msa_dims* d);
 }  // namespace msa
 
@@ -106,7 +105,7 @@ extern "C" msa_status msa_build_block_query_lists_noalloc(const msa_dims* d, con
     return MSA_ERR_CUDA;
   }
   const cudaError_t e = msa::launch_block_lists(
-      sel, d->batch * d->h_kv, d->n_q, d->q_pos0, msa_num_blocks(d), blk_offsets, entries, total,
-      ws, dev_err, reinterpret_cast<cudaStream_t>(stream));
+      sel, d->batch * d->h_kv, d->n_q, d->q_pos0, msa_num_blocks(d), msa_query_window(d),
+      blk_offsets, entries, total, ws, dev_err, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? MSA_OK : MSA_ERR_CUDA;
 }

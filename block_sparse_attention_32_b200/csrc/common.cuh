@@ -91,17 +91,21 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
 
 // Time limit of every barrier wait.  A wait that runs out sets *abort (a
 // shared flag every role polls), reports MSA_DEVERR_TIMEOUT and returns
-// false, so the block winds down instead of hanging.
+// false, so the block winds down instead of hanging.  Kernels may pass a
+// shorter limit (the attention kernel takes one from its launcher); the
+// drains below always use the full limit, since they wait for hardware that
+// is still working.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 constexpr uint32_t kWaitSleepNs = 1000000u;       // longest single sleep: 1 ms
 
 __device__ __forceinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                               int32_t* err) {
+                                               int32_t* err, uint64_t limit_ns = kWaitLimitNs) {
   const uint64_t t0 = global_timer_ns();
+  const uint32_t hint = limit_ns < kWaitSleepNs ? (uint32_t)limit_ns : kWaitSleepNs;
   for (uint32_t it = 0;; ++it) {
-    if (mbar_try_wait_sleep(bar, parity, kWaitSleepNs)) return true;
+    if (mbar_try_wait_sleep(bar, parity, hint)) return true;
     if (*abort) return false;
-    if (global_timer_ns() - t0 > kWaitLimitNs || it > (1u << 30)) {
+    if (global_timer_ns() - t0 > limit_ns || it > (1u << 30)) {
       *abort = 1;
       report(err, MSA_DEVERR_TIMEOUT);
       return false;
@@ -113,9 +117,9 @@ __device__ __forceinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, v
 // would pin the callee to one register budget, which kernels that resize
 // their warpgroups' registers (setmaxnreg) cannot share.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                          int32_t* err) {
+                                          int32_t* err, uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
-  return mbar_wait_slow(bar, parity, abort, err);
+  return mbar_wait_slow(bar, parity, abort, err, limit_ns);
 }
 
 // Waits, bounded but regardless of the abort flag, for a phase that an issued

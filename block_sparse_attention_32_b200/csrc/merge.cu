@@ -7,14 +7,16 @@
 // "Kernel 创新：Outer Gather Q") compute each selected block separately.
 //
 // One warp per (batch, query, head); lane l owns output dims 4l .. 4l+3.
-// HBM-bound: it reads each piece once.
+// HBM-bound: it reads each piece once.  Compact pieces hold accn_s = acc_s /
+// l_s in bf16; then o = sum_s (l_s e^{m_s-M}) accn_s / L.
 #include "common.cuh"
 
 namespace msa {
 
+template <bool kCompact>
 __global__ void __launch_bounds__(256)
     merge_partials_kernel(const int32_t* __restrict__ sel, const float* __restrict__ part_ml,
-                          const float* __restrict__ part_acc, __nv_bfloat16* __restrict__ out,
+                          const void* __restrict__ part_acc, __nv_bfloat16* __restrict__ out,
                           float* __restrict__ lse, int64_t n_rows, int64_t n_q, int32_t H,
                           int32_t G) {
   const int lane = threadIdx.x & 31;
@@ -49,16 +51,36 @@ __global__ void __launch_bounds__(256)
   for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
 
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  const float* pa = part_acc + prow0 * kHeadDim + 4 * lane;
+  if constexpr (kCompact) {
+    // weight of piece s: l_s e^{m_s - M}
+    const float wl = w * l;
+    const __nv_bfloat16* pa =
+        reinterpret_cast<const __nv_bfloat16*>(part_acc) + prow0 * kHeadDim + 4 * lane;
 #pragma unroll
-  for (int s = 0; s < kTopK; ++s) {
-    const float ws = __shfl_sync(0xffffffffu, w, s);
-    if ((vmask >> s) & 1u) {
-      const float4 a = *reinterpret_cast<const float4*>(pa + (int64_t)s * R * kHeadDim);
-      acc.x = fmaf(ws, a.x, acc.x);
-      acc.y = fmaf(ws, a.y, acc.y);
-      acc.z = fmaf(ws, a.z, acc.z);
-      acc.w = fmaf(ws, a.w, acc.w);
+    for (int s = 0; s < kTopK; ++s) {
+      const float ws = __shfl_sync(0xffffffffu, wl, s);
+      if ((vmask >> s) & 1u) {
+        const uint2 u = *reinterpret_cast<const uint2*>(pa + (int64_t)s * R * kHeadDim);
+        const float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+        const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+        acc.x = fmaf(ws, lo.x, acc.x);
+        acc.y = fmaf(ws, lo.y, acc.y);
+        acc.z = fmaf(ws, hi.x, acc.z);
+        acc.w = fmaf(ws, hi.y, acc.w);
+      }
+    }
+  } else {
+    const float* pa = reinterpret_cast<const float*>(part_acc) + prow0 * kHeadDim + 4 * lane;
+#pragma unroll
+    for (int s = 0; s < kTopK; ++s) {
+      const float ws = __shfl_sync(0xffffffffu, w, s);
+      if ((vmask >> s) & 1u) {
+        const float4 a = *reinterpret_cast<const float4*>(pa + (int64_t)s * R * kHeadDim);
+        acc.x = fmaf(ws, a.x, acc.x);
+        acc.y = fmaf(ws, a.y, acc.y);
+        acc.z = fmaf(ws, a.z, acc.z);
+        acc.w = fmaf(ws, a.w, acc.w);
+      }
     }
   }
   const float inv = 1.0f / L;
@@ -71,13 +93,19 @@ __global__ void __launch_bounds__(256)
   if (lane == 0) lse[r] = M + logf(L);
 }
 
-cudaError_t launch_merge(const int32_t* sel, const float* part_ml, const float* part_acc,
-                         void* out, float* lse, int64_t n_rows, int64_t n_q, int32_t H,
-                         int32_t G, cudaStream_t st) {
+cudaError_t launch_merge(const int32_t* sel, const float* part_ml, const void* part_acc,
+                         bool compact, void* out, float* lse, int64_t n_rows, int64_t n_q,
+                         int32_t H, int32_t G, cudaStream_t st) {
   if (n_rows == 0) return cudaSuccess;
   const int64_t threads = n_rows * 32;
-  merge_partials_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(
-      sel, part_ml, part_acc, reinterpret_cast<__nv_bfloat16*>(out), lse, n_rows, n_q, H, G);
+  const unsigned grid = (unsigned)((threads + 255) / 256);
+  __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(out);
+  if (compact)
+    merge_partials_kernel<true><<<grid, 256, 0, st>>>(sel, part_ml, part_acc, o, lse, n_rows,
+                                                      n_q, H, G);
+  else
+    merge_partials_kernel<false><<<grid, 256, 0, st>>>(sel, part_ml, part_acc, o, lse, n_rows,
+                                                       n_q, H, G);
   return cudaGetLastError();
 }
 

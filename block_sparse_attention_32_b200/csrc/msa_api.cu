@@ -18,14 +18,14 @@ cudaError_t launch_index_score_decode(const CUtensorMap&, const void*, int64_t, 
                                       cudaStream_t);
 cudaError_t launch_topk_blocks(const float*, int64_t, int64_t, int64_t, int64_t, int32_t*,
                                cudaStream_t);
-size_t block_lists_workspace(int64_t, int64_t, int64_t);
-cudaError_t launch_block_lists(const int32_t*, int64_t, int64_t, int64_t, int64_t, int32_t*,
-                               int32_t*, int64_t, void*, int32_t*, cudaStream_t);
+size_t block_lists_workspace(int64_t, int64_t, int64_t, int64_t);
+cudaError_t launch_block_lists(const int32_t*, int64_t, int64_t, int64_t, int64_t, int64_t,
+                               int32_t*, int32_t*, int64_t, void*, int32_t*, cudaStream_t);
 cudaError_t launch_sparse_attn(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
                                const CUtensorMap&, const void*, int64_t,
                                int64_t, int64_t, const int32_t*, const int32_t*, int64_t,
-                               int64_t, int64_t, int64_t, int32_t, int32_t, int32_t, float,
-                               float*, float*, int32_t*, cudaStream_t);
+                               int64_t, int64_t, int64_t, int32_t, int32_t, int32_t, int32_t,
+                               float, float*, void*, bool, int32_t*, cudaStream_t);
 cudaError_t launch_sparse_attn_decode(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
                                       const int32_t*, const int32_t*, int64_t, int64_t, int64_t,
                                       int32_t, int32_t, int32_t, float, float*, float*, int32_t*,
@@ -41,8 +41,9 @@ cudaError_t launch_sparse_attn_bwd(const CUtensorMap&, const CUtensorMap&, const
                                    int64_t, int64_t, const void*, int64_t, int64_t, int64_t,
                                    const void*, int64_t, int64_t, int64_t, const float*,
                                    const int32_t*, const int32_t*, int64_t, int64_t, int64_t,
-                                   int64_t, int64_t, int32_t, int32_t, int32_t, float, float*,
-                                   float*, float*, float*, float*, int32_t*, cudaStream_t);
+                                   int64_t, int64_t, int32_t, int32_t, int32_t, int32_t, float,
+                                   float*, float*, float*, float*, float*, int32_t*,
+                                   cudaStream_t);
 size_t token_select_workspace(int64_t, int32_t, int64_t);
 cudaError_t launch_token_select_attention(const CUtensorMap&, const int64_t*, int64_t,
                                           const void*, int64_t, int64_t, int64_t, const void*,
@@ -55,8 +56,9 @@ cudaError_t launch_index_score_e4m3(const CUtensorMap&, const CUtensorMap&, int6
                                    int64_t, int32_t, int32_t, float*, int64_t, const float*,
                                    const float*, int32_t*, cudaStream_t);
 cudaError_t launch_quantize_e4m3(const void*, int64_t, void*, float*, cudaStream_t);
-cudaError_t launch_merge(const int32_t*, const float*, const float*, void*, float*, int64_t,
-                         int64_t, int32_t, int32_t, cudaStream_t);
+uint64_t set_attn_wait_limit(uint64_t);
+cudaError_t launch_merge(const int32_t*, const float*, const void*, bool, void*, float*,
+                         int64_t, int64_t, int32_t, int32_t, cudaStream_t);
 }  // namespace msa
 
 namespace {
@@ -65,6 +67,22 @@ constexpr int64_t kMaxBlocks = 50000;   // shared-memory histogram bound of the 
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool is_pow2(int64_t x) { return x > 0 && (x & (x - 1)) == 0; }
+
+// Query window of the block->query lists: dims->q_window when positive, else
+// the largest power of two W >= 128 whose gathered query rows of one group,
+// W * (h_q / h_kv) * 256 bytes, fit in 32 MiB (about a quarter of L2).
+int64_t query_window(const msa_dims* d) {
+  if (d->q_window > 0) return d->q_window;
+  const int64_t R = d->h_q / d->h_kv;
+  int64_t w = MSA_BLOCK_TOKENS;
+  while (2 * w * R * 256 <= (int64_t(32) << 20)) w *= 2;
+  return w;
+}
+
+int64_t num_windows(const msa_dims* d) {
+  const int64_t w = query_window(d);
+  return (d->n_q + w - 1) / w;
+}
 
 msa_status check_dims(const msa_dims* d) {
   if (d == nullptr) return MSA_ERR_INVALID_ARG;
@@ -82,6 +100,8 @@ msa_status check_dims(const msa_dims* d) {
   if (d->n_q > (int64_t(1) << 26)) return MSA_ERR_UNSUPPORTED;   // entries pack i << 4
   if (d->batch > 65535 || d->batch * d->h_kv > 65535) return MSA_ERR_UNSUPPORTED;
   if (d->n_q / 128 + 1 > 65535) return MSA_ERR_UNSUPPORTED;
+  if (d->q_window < 0 || d->q_window % MSA_BLOCK_TOKENS != 0) return MSA_ERR_INVALID_ARG;
+  if (d->batch * d->h_kv * num_windows(d) > 65535) return MSA_ERR_UNSUPPORTED;
   return MSA_OK;
 }
 
@@ -153,6 +173,22 @@ msa_status make_map_rows_f32(CUtensorMap* map, void* ptr, uint64_t rows, uint32_
   return r == CUDA_SUCCESS ? MSA_OK : MSA_ERR_CUDA;
 }
 
+// 2-D bf16 map over rows of 128 values (256-byte rows): dims {128, rows}, box
+// {64, box_rows}, 128-byte swizzle (compact pieces, staged by the writer in
+// that layout)
+msa_status make_map_rows_bf16(CUtensorMap* map, void* ptr, uint64_t rows, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return MSA_ERR_CUDA;
+  cuuint64_t dims[2] = {128, rows};
+  cuuint64_t strides[1] = {128 * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ptr, dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? MSA_OK : MSA_ERR_CUDA;
+}
+
 msa_status from_cuda(cudaError_t e) { return e == cudaSuccess ? MSA_OK : MSA_ERR_CUDA; }
 
 // 4-D uint8 map (e4m3 codes): dims {inner, d1, d2, d3}, byte strides, box
@@ -202,6 +238,16 @@ int64_t msa_num_blocks(const msa_dims* d) {
 int64_t msa_num_entries(const msa_dims* d) {
   if (check_dims(d) != MSA_OK) return 0;
   return d->batch * d->h_kv * entries_per_bg(d);
+}
+
+int64_t msa_query_window(const msa_dims* d) {
+  if (check_dims(d) != MSA_OK) return 0;
+  return query_window(d);
+}
+
+int64_t msa_num_segments(const msa_dims* d) {
+  if (check_dims(d) != MSA_OK) return 0;
+  return d->batch * d->h_kv * num_windows(d) * msa_num_blocks(d);
 }
 
 msa_status msa_index_score_maxpool(const msa_dims* d, msa_tensor q_idx, msa_tensor k_idx,
@@ -259,7 +305,8 @@ msa_status msa_topk_blocks(const msa_dims* d, const float* pooled, int64_t poole
 
 size_t msa_block_query_lists_workspace(const msa_dims* d) {
   if (check_dims(d) != MSA_OK) return 0;
-  return msa::block_lists_workspace(d->batch * d->h_kv, d->n_q, msa_num_blocks(d));
+  return msa::block_lists_workspace(d->batch * d->h_kv, d->n_q, msa_num_blocks(d),
+                                   query_window(d));
 }
 
 msa_status msa_build_block_query_lists(const msa_dims* d, const int32_t* sel,
@@ -274,14 +321,18 @@ msa_status msa_build_block_query_lists(const msa_dims* d, const int32_t* sel,
   const int64_t total = msa_num_entries(d);
   if (total >= (int64_t(1) << 31)) return MSA_ERR_UNSUPPORTED;
   return from_cuda(msa::launch_block_lists(sel, d->batch * d->h_kv, d->n_q, d->q_pos0,
-                                           msa_num_blocks(d), blk_offsets, entries, total, ws,
-                                           dev_err, reinterpret_cast<cudaStream_t>(stream)));
+                                           msa_num_blocks(d), query_window(d), blk_offsets,
+                                           entries, total, ws, dev_err,
+                                           reinterpret_cast<cudaStream_t>(stream)));
 }
 
-msa_status msa_sparse_attn_fwd(const msa_dims* d, msa_tensor q, msa_tensor k, msa_tensor v,
-                               const int32_t* blk_offsets, const int32_t* entries,
-                               float* part_ml, float* part_acc, int32_t* dev_err,
-                               void* stream) {
+}  // extern "C"
+
+namespace {
+
+msa_status sparse_attn_fwd(const msa_dims* d, msa_tensor q, msa_tensor k, msa_tensor v,
+                           const int32_t* blk_offsets, const int32_t* entries, float* part_ml,
+                           void* part_acc, bool compact, int32_t* dev_err, void* stream) {
   msa_status s = check_dims(d);
   if (s != MSA_OK) return s;
   if ((s = check_tensor(q)) != MSA_OK) return s;
@@ -291,9 +342,15 @@ msa_status msa_sparse_attn_fwd(const msa_dims* d, msa_tensor q, msa_tensor k, ms
     return MSA_ERR_INVALID_ARG;
   if (!aligned16(part_ml) || !aligned16(part_acc)) return MSA_ERR_ALIGNMENT;
   const int64_t nblk = msa_num_blocks(d);
-  const int64_t n_seg = d->batch * d->h_kv * nblk;
+  const int64_t nwin = num_windows(d);
+  const int64_t n_seg = d->batch * d->h_kv * nwin * nblk;
   const int64_t total = msa_num_entries(d);
   if (total >= (int64_t(1) << 31)) return MSA_ERR_UNSUPPORTED;
+  const int64_t R = d->h_q / d->h_kv;
+  // one query per sequence with R <= 8 runs on the warp-level decode kernel,
+  // which writes fp32 pieces only
+  const bool decode = d->n_q == 1 && R <= 8;
+  if (compact && decode) return MSA_ERR_UNSUPPORTED;
   CUtensorMap tk, tv;
   // k, v [B, h_kv, n_kv, 128]: dims {128, n_kv, h_kv, B}, box {64, 128, 1, 1}
   if ((s = make_map(&tk, k.ptr, MSA_HEAD_DIM, d->n_kv, d->h_kv, d->batch, k.s_tok, k.s_head,
@@ -302,13 +359,12 @@ msa_status msa_sparse_attn_fwd(const msa_dims* d, msa_tensor q, msa_tensor k, ms
   if ((s = make_map(&tv, v.ptr, MSA_HEAD_DIM, d->n_kv, d->h_kv, d->batch, v.s_tok, v.s_head,
                     v.s_batch, 128, 1)) != MSA_OK)
     return s;
-  // part_acc [B, n_q, G, 16, R, 128] fp32 as rows of 128 floats; for R >= 8 one
-  // entry's R rows are written by TMA stores of R x 32 floats
+  // part_acc [B, n_q, G, 16, R, 128] as rows of 128 values; for R >= 8 one
+  // entry's R rows are written by TMA stores of R x 32 floats (or R x 64 bf16)
   CUtensorMap to, tq;
   std::memset(&to, 0, sizeof(to));
   std::memset(&tq, 0, sizeof(tq));
-  const int64_t R = d->h_q / d->h_kv;
-  if (d->n_q == 1 && R <= 8) {
+  if (decode) {
     // one query per sequence: warp-level tiles, heads as the 8-wide side.
     // q [B, 1, H, 128]: dims {128, H, 1, B}, box {64, R, 1, 1} (the query's heads of a group)
     if ((s = make_map(&tq, q.ptr, MSA_HEAD_DIM, d->h_q, d->n_q, d->batch, q.s_head, q.s_tok,
@@ -316,7 +372,7 @@ msa_status msa_sparse_attn_fwd(const msa_dims* d, msa_tensor q, msa_tensor k, ms
       return s;
     return from_cuda(msa::launch_sparse_attn_decode(
         tq, tk, tv, blk_offsets, entries, d->batch * d->h_kv, d->n_q, d->q_pos0, d->h_kv,
-        d->h_q, (int32_t)nblk, d->scale, part_ml, part_acc, dev_err,
+        d->h_q, (int32_t)nblk, d->scale, part_ml, reinterpret_cast<float*>(part_acc), dev_err,
         reinterpret_cast<cudaStream_t>(stream)));
   }
   if (R >= 8) {
@@ -326,18 +382,19 @@ msa_status msa_sparse_attn_fwd(const msa_dims* d, msa_tensor q, msa_tensor k, ms
       return s;
     const int64_t rows = d->batch * d->n_q * d->h_kv * MSA_TOPK_BLOCKS * R;
     if (rows >= (int64_t(1) << 31)) return MSA_ERR_UNSUPPORTED;
-    if ((s = make_map_rows_f32(&to, part_acc, (uint64_t)rows, (uint32_t)R)) != MSA_OK) return s;
+    s = compact ? make_map_rows_bf16(&to, part_acc, (uint64_t)rows, (uint32_t)R)
+                : make_map_rows_f32(&to, part_acc, (uint64_t)rows, (uint32_t)R);
+    if (s != MSA_OK) return s;
   }
   return from_cuda(msa::launch_sparse_attn(
-      tq, tk, tv, to, q.ptr, q.s_batch, q.s_tok, q.s_head, blk_offsets, entries, n_seg, total, d->n_q,
-      d->q_pos0, d->h_kv, d->h_q, (int32_t)nblk, d->scale, part_ml, part_acc, dev_err,
-      reinterpret_cast<cudaStream_t>(stream)));
+      tq, tk, tv, to, q.ptr, q.s_batch, q.s_tok, q.s_head, blk_offsets, entries, n_seg, total,
+      d->n_q, d->q_pos0, d->h_kv, d->h_q, (int32_t)nblk, (int32_t)nwin, d->scale, part_ml,
+      part_acc, compact, dev_err, reinterpret_cast<cudaStream_t>(stream)));
 }
 
-msa_status msa_merge_partials(const msa_dims* d, const int32_t* sel, const float* part_ml,
-                              const float* part_acc, void* out, float* lse, int32_t* dev_err,
-                              void* stream) {
-  (void)dev_err;
+msa_status merge_partials(const msa_dims* d, const int32_t* sel, const float* part_ml,
+                          const void* part_acc, bool compact, void* out, float* lse,
+                          void* stream) {
   msa_status s = check_dims(d);
   if (s != MSA_OK) return s;
   if (sel == nullptr || part_ml == nullptr || part_acc == nullptr || out == nullptr ||
@@ -346,8 +403,42 @@ msa_status msa_merge_partials(const msa_dims* d, const int32_t* sel, const float
   if (!aligned16(part_ml) || !aligned16(part_acc) || !aligned16(out))
     return MSA_ERR_ALIGNMENT;
   const int64_t n_rows = d->batch * d->n_q * d->h_q;
-  return from_cuda(msa::launch_merge(sel, part_ml, part_acc, out, lse, n_rows, d->n_q, d->h_q,
-                                     d->h_kv, reinterpret_cast<cudaStream_t>(stream)));
+  return from_cuda(msa::launch_merge(sel, part_ml, part_acc, compact, out, lse, n_rows, d->n_q,
+                                     d->h_q, d->h_kv, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+}  // namespace
+
+extern "C" {
+
+msa_status msa_sparse_attn_fwd(const msa_dims* d, msa_tensor q, msa_tensor k, msa_tensor v,
+                               const int32_t* blk_offsets, const int32_t* entries,
+                               float* part_ml, float* part_acc, int32_t* dev_err,
+                               void* stream) {
+  return sparse_attn_fwd(d, q, k, v, blk_offsets, entries, part_ml, part_acc, false, dev_err,
+                         stream);
+}
+
+msa_status msa_sparse_attn_fwd_compact(const msa_dims* d, msa_tensor q, msa_tensor k,
+                                       msa_tensor v, const int32_t* blk_offsets,
+                                       const int32_t* entries, float* part_ml,
+                                       void* part_acc_bf16, int32_t* dev_err, void* stream) {
+  return sparse_attn_fwd(d, q, k, v, blk_offsets, entries, part_ml, part_acc_bf16, true,
+                         dev_err, stream);
+}
+
+msa_status msa_merge_partials(const msa_dims* d, const int32_t* sel, const float* part_ml,
+                              const float* part_acc, void* out, float* lse, int32_t* dev_err,
+                              void* stream) {
+  (void)dev_err;
+  return merge_partials(d, sel, part_ml, part_acc, false, out, lse, stream);
+}
+
+msa_status msa_merge_partials_compact(const msa_dims* d, const int32_t* sel,
+                                      const float* part_ml, const void* part_acc_bf16,
+                                      void* out, float* lse, int32_t* dev_err, void* stream) {
+  (void)dev_err;
+  return merge_partials(d, sel, part_ml, part_acc_bf16, true, out, lse, stream);
 }
 
 msa_status msa_quantize_e4m3(const void* x, int64_t n, void* codes, float* scale,
@@ -465,8 +556,8 @@ msa_status msa_sparse_attn_bwd(const msa_dims* d, msa_tensor q, msa_tensor k, ms
   return from_cuda(msa::launch_sparse_attn_bwd(
       tk, tv, q.ptr, q.s_batch, q.s_tok, q.s_head, o.ptr, o.s_batch, o.s_tok, o.s_head, d_o.ptr,
       d_o.s_batch, d_o.s_tok, d_o.s_head, lse, blk_offsets, entries, total, d->batch, d->n_q,
-      d->n_kv, d->q_pos0, d->h_kv, d->h_q, (int32_t)nblk, d->scale, delta, part_dq, dq, dk, dv,
-      dev_err, reinterpret_cast<cudaStream_t>(stream)));
+      d->n_kv, d->q_pos0, d->h_kv, d->h_q, (int32_t)nblk, (int32_t)num_windows(d), d->scale,
+      delta, part_dq, dq, dk, dv, dev_err, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 size_t msa_token_select_workspace(const msa_dims* d, int64_t n_rows) {
@@ -505,6 +596,12 @@ msa_status msa_token_select_attention(const msa_dims* d, msa_tensor q, msa_tenso
       q_idx.s_tok, q_idx.s_head, k.ptr, k.s_batch, k.s_tok, k.s_head, v.ptr, v.s_batch, v.s_tok,
       v.s_head, d->batch, d->n_q, d->n_kv, d->q_pos0, d->h_kv, d->h_q, d->d_idx, d->h_kidx,
       d->scale, budget, tokens, out, lse, ws, dev_err, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+uint64_t msa_debug_set_attn_wait_limit_ns(uint64_t ns) {
+  if (ns == 0) ns = msa::kWaitLimitNs;
+  if (ns > msa::kWaitLimitNs) ns = msa::kWaitLimitNs;
+  return msa::set_attn_wait_limit(ns);
 }
 
 const char* msa_status_string(msa_status s) {

@@ -4,6 +4,9 @@
 // gathered into 128-row tiles, and S = Q K^T, the softmax piece and O = P V
 // run on the tcgen05 tensor cores with fp32 accumulators in TMEM.  Each
 // (query, head, slot) gets a piece (m, l, acc) that the merge kernel combines.
+// Pieces are fp32 by default; the compact form (an opt-in of the C ABI) keeps
+// (m, l) in fp32 and stores acc / l rounded to bf16 (a convex combination of
+// V rows, so it cannot overflow), which halves the piece traffic.
 //
 // Source: page "MSA 稀疏注意力三国杀", section "MSA 架构：粗筛 + 精算" (main
 // branch: full attention over the selected blocks only) and section "Kernel
@@ -27,13 +30,15 @@
 //                             one is done, V as soon as its last P V is done
 //   warp 3      idle (fills the control warpgroup)
 //   warps 4-7   gather:       the chunk's Q rows into a 3-deep ring: for R >= 8
-//                             one TMA box per entry and 64-column panel
-//                             (an entry's R head rows are contiguous),
-//                             otherwise 16-byte cp.async
+//                             warp 4 alone, one TMA box per entry and
+//                             64-column panel (an entry's R head rows are
+//                             contiguous), otherwise 16-byte cp.async by all
+//                             four warps
 //   warps 8-15  softmax:      two warpgroups, one per half of the keys; each
 //                             holds its 64 S values of a row in registers,
 //                             the halves exchange row maxima through shared
-//                             memory, and P = bf16(e^{s-m}) goes back into
+//                             memory (an mbarrier per quarter and chunk
+//                             parity), and P = bf16(e^{s-m}) goes back into
 //                             the first 64 columns of the S buffer in TMEM
 //                             (the A operand of O = P V)
 //   warps 16-19 epilogue:     O from TMEM half a row at a time, then the
@@ -50,6 +55,11 @@
 // [256,512), two buffers of 128 columns each; a Q tile is released as soon as
 // its S MMA is done, S(n+2) waits for O(n) = P(n) V, which reads P(n) from
 // the same columns, and P V(n+2) waits until the epilogue has read O(n).
+// Every wait is bounded (a time limit, then the block winds down and reports
+// MSA_DEVERR_TIMEOUT); whatever path a role leaves by, the loads it issued
+// and the MMAs in flight are drained before TMEM is freed and the block exits.
+#include <atomic>
+
 #include "common.cuh"
 
 namespace msa {
@@ -85,7 +95,7 @@ constexpr int kOffML = kOffStage + 128 * kStageRow;      // [2 slots][2 halves][
 constexpr int kOffMX = kOffML + 4096;                    // [2][2 halves][128] float row maxima
 constexpr int kOffDesc = kOffMX + 2048;                  // kDescRing descriptors
 constexpr int kOffBar = kOffDesc + kDescRing * (int)sizeof(ChunkDesc);
-constexpr int kNumBars = 4 + 3 * kQRing + 6 + 2 * kDescRing + 2;
+constexpr int kNumBars = 4 + 3 * kQRing + 6 + 2 * kDescRing + 2 + 1 + 8;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;         // TMEM base, abort flag
 constexpr int kAttnSmemBytes = 1024 + kOffMisc + 64;
 
@@ -94,7 +104,10 @@ enum {
   BAR_Q_FULL = 4, BAR_QP_EMPTY = 4 + kQRing, BAR_P_FULL = 4 + 2 * kQRing,
   BAR_S_FULL = 4 + 3 * kQRing, BAR_O_FULL = BAR_S_FULL + 2, BAR_O_EMPTY = BAR_S_FULL + 4,
   BAR_D_FULL = BAR_S_FULL + 6, BAR_D_EMPTY = BAR_D_FULL + kDescRing,
-  BAR_ML_EMPTY = BAR_D_EMPTY + kDescRing
+  BAR_ML_EMPTY = BAR_D_EMPTY + kDescRing,
+  BAR_DRAIN = BAR_ML_EMPTY + 2,     // the MMA issuer's last commit (all its MMAs done)
+  BAR_MX = BAR_DRAIN + 1            // [quarter][chunk parity]: the two softmax halves'
+                                    // row maxima of a chunk are written
 };
 
 struct AttnArgs {
@@ -104,11 +117,12 @@ struct AttnArgs {
   const int32_t* entries;
   int64_t n_seg, n_entries, n_items, W;
   int64_t n_q, q_pos0;
-  int32_t G, H, nblk;
+  int32_t G, H, nblk, nwin;   // segments are (batch, group, query window, block)
   float scale;
   float* part_ml;
-  float* part_acc;
+  void* part_acc;             // fp32 rows, or bf16 rows of acc / l (compact pieces)
   int32_t* err;
+  uint64_t wait_limit_ns;     // time limit of every barrier wait (drains excepted)
 };
 
 // Largest s in [lo, n_seg) with off[s] <= pos, by a 32-ary search: each round
@@ -126,7 +140,7 @@ __device__ __forceinline__ int64_t warp_find_segment(const int32_t* off, int64_t
   return lo;
 }
 
-template <int R>
+template <int R, bool kCompact>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     sparse_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                            const __grid_constant__ CUtensorMap tm_k,
@@ -156,7 +170,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     mbar_init(bar + BAR_V_FULL, 1);
     mbar_init(bar + BAR_V_EMPTY, 1);
     for (int i = 0; i < kQRing; ++i) {
-      mbar_init(bar + BAR_Q_FULL + i, kTmaGather ? 4 : 128);
+      mbar_init(bar + BAR_Q_FULL + i, kTmaGather ? 1 : 128);
       mbar_init(bar + BAR_QP_EMPTY + i, 1);
       mbar_init(bar + BAR_P_FULL + i, 256);
     }
@@ -170,6 +184,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_init(bar + BAR_D_FULL + i, 1);
       mbar_init(bar + BAR_D_EMPTY + i, 128 + 1);   // epilogue threads + TMA producer
     }
+    mbar_init(bar + BAR_DRAIN, 1);
+    for (int i = 0; i < 8; ++i) mbar_init(bar + BAR_MX + i, 2);   // one warp of each half
     *abort_flag = 0;
     fence_mbarrier_init();
   }
@@ -187,12 +203,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const uint32_t tmem = *tmem_slot;
   int32_t* err = a.err;
   // ring of depth D: the n-th use is ready / the (n-D)-th use has been released
+  const uint64_t wait_lim = a.wait_limit_ns;
   auto Wuse = [&](int id, int depth, int64_t n) {
-    return mbar_wait(bar + id + (int)(n % depth), (uint32_t)((n / depth) & 1), abort_flag, err);
+    return mbar_wait(bar + id + (int)(n % depth), (uint32_t)((n / depth) & 1), abort_flag, err,
+                     wait_lim);
   };
   auto Wfree = [&](int id, int depth, int64_t n) {
     return n < depth || mbar_wait(bar + id + (int)(n % depth),
-                                  (uint32_t)(((n / depth) + 1) & 1), abort_flag, err);
+                                  (uint32_t)(((n / depth) + 1) & 1), abort_flag, err, wait_lim);
   };
 
   // Roles by warpgroup; each warpgroup first resizes its registers (all four
@@ -223,8 +241,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             ok = false;
             break;
           }
-          const int64_t bg = seg / a.nblk;
-          const int32_t c = (int32_t)(seg - bg * a.nblk);
+          const int64_t bgw = seg / a.nblk;
+          const int32_t c = (int32_t)(seg - bgw * a.nblk);
+          const int64_t bg = bgw / a.nwin;
           const int32_t b = (int32_t)(bg / a.G), g = (int32_t)(bg - (int64_t)b * a.G);
           for (int64_t cpos = pos; cpos < pend; cpos += CH) {
             if (!claim(chunk)) {
@@ -330,12 +349,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           if (plast) Wuse(BAR_V_EMPTY, 1, pp);
           if (last_s_piece >= 0) Wuse(BAR_K_EMPTY, 1, last_s_piece);
         }
+        // On every exit path, also after an abort: one more commit arrives once
+        // every MMA this thread issued has completed (commits complete in issue
+        // order), so no MMA still reads shared memory or writes TMEM when the
+        // block deallocates TMEM and exits.
+        umma_commit(bar + BAR_DRAIN);
+        mbar_drain(bar + BAR_DRAIN, 0, err);
       }
     } else if (warp == 2) {
       // ---------------- TMA producer: K/V of every piece ----------------
       if (lane == 0) {
         prefetch_tensormap(&tm_k);
         prefetch_tensormap(&tm_v);
+        int64_t k_issued = -1, v_issued = -1;    // last piece whose K / V load was issued
         for (int64_t n = 0;; ++n) {
           if (!Wuse(BAR_D_FULL, kDescRing, n)) break;
           const ChunkDesc& d = desc[n % kDescRing];
@@ -347,13 +373,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             mbar_arrive_expect_tx(bar + BAR_K_FULL, 32768);
             tma_load_4d(base + kOffK, &tm_k, bar + BAR_K_FULL, 0, c * kBlock, g, b);
             tma_load_4d(base + kOffK + 16384, &tm_k, bar + BAR_K_FULL, 64, c * kBlock, g, b);
+            k_issued = p;
             if (!Wfree(BAR_V_EMPTY, 1, p)) break;
             mbar_arrive_expect_tx(bar + BAR_V_FULL, 32768);
             tma_load_4d(base + kOffV, &tm_v, bar + BAR_V_FULL, 0, c * kBlock, g, b);
             tma_load_4d(base + kOffV + 16384, &tm_v, bar + BAR_V_FULL, 64, c * kBlock, g, b);
+            v_issued = p;
           }
           mbar_arrive(bar + BAR_D_EMPTY + (int)(n % kDescRing));
         }
+        // the loads in flight land before the block exits (piece p is the p-th
+        // phase of each full barrier)
+        if (k_issued >= 0) mbar_drain(bar + BAR_K_FULL, (uint32_t)(k_issued & 1), err);
+        if (v_issued >= 0) mbar_drain(bar + BAR_V_FULL, (uint32_t)(v_issued & 1), err);
       }
     }
     // warp 3: idle
@@ -361,36 +393,44 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     // ---------------- gather: Q rows of each chunk ----------------
     setmaxnreg_dec<kRegsGather>();
     if constexpr (kTmaGather) {
-      // lane 0 of gather warp w loads entries w, w+4, ...: one TMA box of R
-      // rows x 64 columns per 128-byte panel, completing on Q_FULL
-      const int wq = warp - 4;
-      for (int64_t n = 0;; ++n) {
-        if (!Wuse(BAR_D_FULL, kDescRing, n)) break;
-        const ChunkDesc& d = desc[n % kDescRing];
-        if (d.cnt < 0) break;
-        const int qb = (int)(n % kQRing);
-        int ok = 1;
-        if (lane == 0) {
-          if (!Wfree(BAR_QP_EMPTY, kQRing, n)) {
-            ok = 0;
-          } else {
-            uint8_t* sq = base + kOffQP + qb * 32768;
-            uint32_t bytes = 0;
-            for (int k = wq; k < CH; k += 4) {
-              const int e = d.ent[k];
-              if (e >= 0 && (int64_t)(e >> 4) < a.n_q) bytes += R * 256;
-            }
-            mbar_arrive_expect_tx(bar + BAR_Q_FULL + qb, bytes);
-            for (int k = wq; k < CH; k += 4) {
-              const int e = d.ent[k];
-              if (e < 0 || (int64_t)(e >> 4) >= a.n_q) continue;
-              for (int p = 0; p < 2; ++p)
-                tma_load_4d(sq + p * 16384 + k * R * 128, &tm_q, bar + BAR_Q_FULL + qb, p * 64,
-                            d.g * R, e >> 4, d.b);
+      // warp 4 alone: lane 0 arms Q_FULL with the chunk's bytes, then lane l
+      // issues the TMA boxes (R rows x 64 columns) of entries l, l+32, ... for
+      // both 128-byte panels.  One thread arms each phase, so on an abort it
+      // knows which loads are in flight and drains exactly those.
+      if (warp == 4) {
+        int64_t armed = -1;                      // last chunk whose loads were issued
+        for (int64_t n = 0;; ++n) {
+          if (!Wuse(BAR_D_FULL, kDescRing, n)) break;
+          const ChunkDesc& d = desc[n % kDescRing];
+          if (d.cnt < 0) break;
+          const int qb = (int)(n % kQRing);
+          int ok = 1;
+          if (lane == 0) {
+            if (!Wfree(BAR_QP_EMPTY, kQRing, n)) {
+              ok = 0;
+            } else {
+              uint32_t bytes = 0;
+              for (int k = 0; k < CH; ++k) {
+                const int e = d.ent[k];
+                if (e >= 0 && (int64_t)(e >> 4) < a.n_q) bytes += R * 256;
+              }
+              mbar_arrive_expect_tx(bar + BAR_Q_FULL + qb, bytes);
             }
           }
+          if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+          armed = n;
+          uint8_t* sq = base + kOffQP + qb * 32768;
+          for (int t = lane; t < 2 * CH; t += 32) {
+            const int k = t >> 1, p = t & 1;
+            const int e = d.ent[k];
+            if (e < 0 || (int64_t)(e >> 4) >= a.n_q) continue;
+            tma_load_4d(sq + p * 16384 + k * R * 128, &tm_q, bar + BAR_Q_FULL + qb, p * 64,
+                        d.g * R, e >> 4, d.b);
+          }
         }
-        if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+        if (lane == 0 && armed >= 0)
+          mbar_drain(bar + BAR_Q_FULL + (int)(armed % kQRing),
+                     (uint32_t)((armed / kQRing) & 1), err);
       }
     } else {
       // thread = (row within an 8-row group, 16-byte column chunk); a warp
@@ -426,8 +466,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   } else if (warp < 16) {
     // ---------------- softmax: S -> P, (m, l) ----------------
     // warpgroup h (0, 1) takes keys 64h .. 64h+63 of every row; the two
-    // halves of a row exchange their maxima through shared memory (named
-    // barrier 1 + quarter, 64 threads) and each writes its own sum.
+    // halves of a row exchange their maxima through shared memory (an
+    // mbarrier per quarter and chunk parity, one arrival per warp) and each
+    // writes its own sum.
     setmaxnreg_inc<kRegsSoftmax>();
     const int h = (warp >> 2) - 2;
     const int quarter = warp & 3;
@@ -487,7 +528,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       float* mxn = mx_x + (int)(n & 1) * 256;   // by parity: the partner reads it before n+2
       mxn[h * 128 + row] = mloc;
       tc_fence_before();                       // this half's S reads precede the other's P writes
-      named_bar_sync(1 + quarter, 64);
+      // exchange with the other half's warp of this quarter through an mbarrier
+      // (a bounded wait: neither half can be left waiting on the other)
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar + BAR_MX + quarter * 2 + (int)(n & 1));
+      if (!mbar_wait(bar + BAR_MX + quarter * 2 + (int)(n & 1), (uint32_t)((n >> 1) & 1),
+                     abort_flag, err, wait_lim))
+        break;
       tc_fence_after();
       float mx = fmaxf(mloc, mxn[(1 - h) * 128 + row]);
       if (!valid) mx = 0.f;
@@ -564,10 +611,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       // piece row of (b, qi, g, slot, hr): the R head rows of one entry are adjacent
       const int64_t pidx =
           valid ? ((((int64_t)b * a.n_q + qi) * a.G + g) * kTopK + (e & 15)) * R + hr : 0;
-      if (valid)
-        *reinterpret_cast<float2*>(a.part_ml + pidx * 2) = make_float2(ml0.x, ml0.y + ml1.y);
+      const float l_sum = ml0.y + ml1.y;
+      if (valid) *reinterpret_cast<float2*>(a.part_ml + pidx * 2) = make_float2(ml0.x, l_sum);
+      // compact pieces: acc / l (l >= 1 on a valid row: the row maximum's weight is 1)
+      const float inv_l = (kCompact && valid && l_sum > 0.f) ? 1.0f / l_sum : 0.f;
       const uint32_t o_addr = tmem + lane_base + 256 + ob * 128;
-      float* acc = a.part_acc + pidx * kHeadDim;
+      float* acc = reinterpret_cast<float*>(a.part_acc) + pidx * kHeadDim;
+      __nv_bfloat16* acc16 = reinterpret_cast<__nv_bfloat16*>(a.part_acc) + pidx * kHeadDim;
 #pragma unroll 1
       for (int half = 0; half < 2; ++half) {
         uint32_t r0[32], r1[32];
@@ -578,7 +628,50 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           tc_fence_before();
           mbar_arrive(bar + BAR_O_EMPTY + ob);   // O buffer ob is free
         }
-        if constexpr (kTmaStore) {
+        if constexpr (kCompact) {
+          // the half row as 64 bf16 values = 128 bytes = 8 chunks of 16 bytes
+          uint32_t w[32];
+#pragma unroll
+          for (int x = 0; x < 16; ++x) {
+            w[x] = pack_bf16x2(u2f(r0[2 * x]) * inv_l, u2f(r0[2 * x + 1]) * inv_l);
+            w[16 + x] = pack_bf16x2(u2f(r1[2 * x]) * inv_l, u2f(r1[2 * x + 1]) * inv_l);
+          }
+          if constexpr (kTmaStore) {
+            bulk_wait_read();                    // the previous stores have read the panel
+            __syncwarp();
+            const int sw = lane & 7;
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              *reinterpret_cast<uint4*>(stage + lane * 128 + ((j ^ sw) << 4)) =
+                  make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (valid && hr == 0)                // first row of an entry: R rows per store
+              tma_store_2d_hint(&tm_o, stage + lane * 128, half * 64, (int32_t)pidx, pol_st);
+            bulk_commit();
+          } else {
+#pragma unroll
+            for (int x = 0; x < 8; ++x)
+              *reinterpret_cast<uint4*>(srow + x * 16) =
+                  make_uint4(w[4 * x], w[4 * x + 1], w[4 * x + 2], w[4 * x + 3]);
+            __syncwarp();
+            // four half rows (128 bytes each) per instruction: lane -> (row 4i + lane / 8,
+            // 16-byte chunk lane % 8)
+#pragma unroll 4
+            for (int i = 0; i < 8; ++i) {
+              const int rr = 4 * i + (lane >> 3);
+              const __nv_bfloat16* dst_row = (const __nv_bfloat16*)__shfl_sync(
+                  0xffffffffu, (unsigned long long)acc16, rr);
+              const bool rv = __shfl_sync(0xffffffffu, valid ? 1 : 0, rr) != 0;
+              const uint4 v =
+                  *reinterpret_cast<const uint4*>(swarp + rr * kStageRow + (lane & 7) * 16);
+              if (rv)
+                *reinterpret_cast<uint4*>(const_cast<__nv_bfloat16*>(dst_row) + half * 64 +
+                                          (lane & 7) * 8) = v;
+            }
+            __syncwarp();
+          }
+        } else if constexpr (kTmaStore) {
           bulk_wait_read();                      // the previous stores have read the panels
           __syncwarp();
           const int sw = lane & 7;
@@ -635,12 +728,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   }
 }
 
-template <int R>
+// Time limit of the attention kernel's barrier waits (a debug setting of the C
+// ABI; 2 s by default).
+static std::atomic<uint64_t> g_attn_wait_limit_ns{kWaitLimitNs};
+
+uint64_t set_attn_wait_limit(uint64_t ns) { return g_attn_wait_limit_ns.exchange(ns); }
+
+template <int R, bool kCompact>
 static cudaError_t launch_attn_r(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
                                  const CUtensorMap& tm_v, const CUtensorMap& tm_o, AttnArgs a,
                                  cudaStream_t st) {
   constexpr int CH = 128 / R;
-  auto k = sparse_attn_fwd_kernel<R>;
+  auto k = sparse_attn_fwd_kernel<R, kCompact>;
   // the register split above is only safe with exactly this many registers
   // per thread at launch
   cudaFuncAttributes fa;
@@ -665,13 +764,28 @@ static cudaError_t launch_attn_r(const CUtensorMap& tm_q, const CUtensorMap& tm_
   return cudaGetLastError();
 }
 
+template <bool kCompact>
+static cudaError_t launch_attn_c(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
+                                 const CUtensorMap& tm_v, const CUtensorMap& tm_o,
+                                 const AttnArgs& a, cudaStream_t st) {
+  switch (a.H / a.G) {
+    case 1: return launch_attn_r<1, kCompact>(tm_q, tm_k, tm_v, tm_o, a, st);
+    case 2: return launch_attn_r<2, kCompact>(tm_q, tm_k, tm_v, tm_o, a, st);
+    case 4: return launch_attn_r<4, kCompact>(tm_q, tm_k, tm_v, tm_o, a, st);
+    case 8: return launch_attn_r<8, kCompact>(tm_q, tm_k, tm_v, tm_o, a, st);
+    case 16: return launch_attn_r<16, kCompact>(tm_q, tm_k, tm_v, tm_o, a, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
 cudaError_t launch_sparse_attn(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
                                const CUtensorMap& tm_v, const CUtensorMap& tm_o, const void* q,
                                int64_t qs_b, int64_t qs_t, int64_t qs_h,
                                const int32_t* blk_offsets, const int32_t* entries,
                                int64_t n_seg, int64_t n_entries, int64_t n_q, int64_t q_pos0,
-                               int32_t G, int32_t H, int32_t nblk, float scale, float* part_ml,
-                               float* part_acc, int32_t* err, cudaStream_t st) {
+                               int32_t G, int32_t H, int32_t nblk, int32_t nwin, float scale,
+                               float* part_ml, void* part_acc, bool compact, int32_t* err,
+                               cudaStream_t st) {
   AttnArgs a;
   a.q = reinterpret_cast<const __nv_bfloat16*>(q);
   a.qs_b = qs_b;
@@ -688,18 +802,14 @@ cudaError_t launch_sparse_attn(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
   a.G = G;
   a.H = H;
   a.nblk = nblk;
+  a.nwin = nwin;
   a.scale = scale;
   a.part_ml = part_ml;
   a.part_acc = part_acc;
   a.err = err;
-  switch (H / G) {
-    case 1: return launch_attn_r<1>(tm_q, tm_k, tm_v, tm_o, a, st);
-    case 2: return launch_attn_r<2>(tm_q, tm_k, tm_v, tm_o, a, st);
-    case 4: return launch_attn_r<4>(tm_q, tm_k, tm_v, tm_o, a, st);
-    case 8: return launch_attn_r<8>(tm_q, tm_k, tm_v, tm_o, a, st);
-    case 16: return launch_attn_r<16>(tm_q, tm_k, tm_v, tm_o, a, st);
-    default: return cudaErrorInvalidValue;
-  }
+  a.wait_limit_ns = g_attn_wait_limit_ns.load();
+  return compact ? launch_attn_c<true>(tm_q, tm_k, tm_v, tm_o, a, st)
+                 : launch_attn_c<false>(tm_q, tm_k, tm_v, tm_o, a, st);
 }
 
 }  // namespace msa

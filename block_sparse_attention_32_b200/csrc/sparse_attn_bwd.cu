@@ -52,7 +52,7 @@ struct BwdArgs {
   float* dk;                  // [B, G, n_kv, 128]
   float* dv;
   int64_t n_q, n_kv, q_pos0, nseg, total, chunk_entries;
-  int32_t G, H, nblk;
+  int32_t G, H, nblk, nwin;   // segments are (batch, group, query window, block)
   float scale;
   int32_t* err;
 };
@@ -165,7 +165,7 @@ __device__ __forceinline__ bool walk_next(PieceWalk& w, const BwdArgs& a, Piece&
   pc.e1 = p_end;
   w.e = p_end;
   pc.c = (int32_t)(w.seg % a.nblk);
-  const int64_t bg = w.seg / a.nblk;
+  const int64_t bg = w.seg / a.nblk / a.nwin;
   pc.g = (int32_t)(bg % a.G);
   pc.b = bg / a.G;
   return true;
@@ -550,7 +550,8 @@ cudaError_t launch_sparse_attn_bwd(const CUtensorMap& tm_k, const CUtensorMap& t
                                    const float* lse, const int32_t* offsets,
                                    const int32_t* entries, int64_t total_entries, int64_t batch,
                                    int64_t n_q, int64_t n_kv, int64_t q_pos0, int32_t G,
-                                   int32_t H, int32_t nblk, float scale, float* delta,
+                                   int32_t H, int32_t nblk, int32_t nwin, float scale,
+                                   float* delta,
                                    float* part_dq, float* dq, float* dk, float* dv,
                                    int32_t* err, cudaStream_t st) {
   const int32_t R = H / G;
@@ -587,11 +588,12 @@ cudaError_t launch_sparse_attn_bwd(const CUtensorMap& tm_k, const CUtensorMap& t
   a.n_q = n_q;
   a.n_kv = n_kv;
   a.q_pos0 = q_pos0;
-  a.nseg = batch * G * nblk;
+  a.nseg = batch * G * nwin * nblk;
   a.total = total_entries;
   a.G = G;
   a.H = H;
   a.nblk = nblk;
+  a.nwin = nwin;
   a.scale = scale;
   a.err = err;
   // equal runs of entries, whole 128-row tiles each, about 8 per SM

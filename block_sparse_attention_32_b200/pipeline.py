@@ -41,9 +41,13 @@ class Buffers:
     out: torch.Tensor
     lse: torch.Tensor
     dev_err: torch.Tensor
+    compact: bool = False
 
     @staticmethod
-    def allocate(d: capi.Dims, device="cuda") -> "Buffers":
+    def allocate(d: capi.Dims, device="cuda", compact: bool = False) -> "Buffers":
+        """Intermediate buffers of one problem.  compact=True: the pieces' acc
+        in bf16 (acc / l), read and written by the compact attention and merge
+        calls."""
         B, n_q, G, H = d.batch, d.n_q, d.h_kv, d.h_q
         nblk = capi.msa_num_blocks(d)
         stride = (nblk + 3) // 4 * 4
@@ -55,23 +59,25 @@ class Buffers:
             pooled=torch.empty((B, G, n_q, stride), dtype=torch.float32, device=dev),
             pooled_stride=stride,
             sel=torch.empty((B, G, n_q, capi.TOPK), dtype=torch.int32, device=dev),
-            blk_offsets=torch.empty((B * G * nblk + 1,), dtype=torch.int32, device=dev),
+            blk_offsets=torch.empty((capi.msa_num_segments(d) + 1,), dtype=torch.int32,
+                                    device=dev),
             entries=torch.empty((max(n_ent, 1),), dtype=torch.int32, device=dev),
             ws=torch.empty(((ws_bytes + 15) // 16 * 4,), dtype=torch.int32, device=dev),
             part_ml=torch.empty((B, n_q, G, capi.TOPK, H // G, 2), dtype=torch.float32,
                                 device=dev),
             part_acc=torch.empty((B, n_q, G, capi.TOPK, H // G, capi.HEAD_DIM),
-                                 dtype=torch.float32, device=dev),
+                                 dtype=torch.bfloat16 if compact else torch.float32, device=dev),
             out=torch.empty((B, n_q, H, capi.HEAD_DIM), dtype=torch.bfloat16, device=dev),
             lse=torch.empty((B, n_q, H), dtype=torch.float32, device=dev),
             dev_err=torch.zeros((4,), dtype=torch.int32, device=dev),
+            compact=compact,
         )
 
 
 def dims_for(w) -> capi.Dims:
     """Dims of a workloads.Workload."""
     return capi.make_dims(w.batch, w.n_q, w.n_kv, w.q_pos0, w.h_q, w.h_kv, w.d_idx,
-                          h_kidx=w.h_kidx, scale=w.scale)
+                          h_kidx=w.h_kidx, scale=w.scale, q_window=w.q_window)
 
 
 def select(buf: Buffers, q_idx, k_idx):
@@ -103,9 +109,15 @@ def attend(buf: Buffers, q, k, v, sel=None):
     d = buf.dims
     s = buf.sel if sel is None else sel
     capi.msa_build_block_query_lists(d, s, buf.blk_offsets, buf.entries, buf.ws, buf.dev_err)
-    capi.msa_sparse_attn_fwd(d, q, k, v, buf.blk_offsets, buf.entries, buf.part_ml,
-                             buf.part_acc, buf.dev_err)
-    capi.msa_merge_partials(d, s, buf.part_ml, buf.part_acc, buf.out, buf.lse, buf.dev_err)
+    if buf.compact:
+        capi.msa_sparse_attn_fwd_compact(d, q, k, v, buf.blk_offsets, buf.entries, buf.part_ml,
+                                         buf.part_acc, buf.dev_err)
+        capi.msa_merge_partials_compact(d, s, buf.part_ml, buf.part_acc, buf.out, buf.lse,
+                                        buf.dev_err)
+    else:
+        capi.msa_sparse_attn_fwd(d, q, k, v, buf.blk_offsets, buf.entries, buf.part_ml,
+                                 buf.part_acc, buf.dev_err)
+        capi.msa_merge_partials(d, s, buf.part_ml, buf.part_acc, buf.out, buf.lse, buf.dev_err)
 
 
 def forward(buf: Buffers, q, k, v, q_idx, k_idx):
@@ -137,7 +149,11 @@ class Grads:
 def backward(buf: Buffers, grads: Grads, q, k, v, d_out):
     """Gradients of the attention for upstream d_out (bf16 [B,n_q,H,128]) after a
     forward on the same buffers (its out, lse and block lists; the selection is
-    fixed).  The forward's piece buffer holds the dQ pieces.  Returns (dq, dk, dv)."""
+    fixed).  The forward's piece buffer holds the dQ pieces, so it must be the
+    fp32 one (Buffers allocated with compact=False).  Returns (dq, dk, dv)."""
+    if buf.compact:
+        raise ValueError("the backward keeps fp32 dq pieces in the piece buffer: "
+                         "allocate the Buffers with compact=False")
     capi.msa_sparse_attn_bwd(buf.dims, q, k, v, buf.out, d_out, buf.lse, buf.blk_offsets,
                              buf.entries, grads.delta, buf.part_acc, grads.dq, grads.dk,
                              grads.dv, buf.dev_err)

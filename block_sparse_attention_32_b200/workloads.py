@@ -51,6 +51,7 @@ class Workload:
     sink: bool = False
     recency: bool = False
     q_scale: float = 1.0           # >1 gives peaked softmax rows
+    q_window: int = 0              # query window of the block->query lists (0: library default)
 
     @property
     def nblk(self) -> int:

@@ -83,11 +83,17 @@ typedef enum {
  * G = h_kv GQA groups; h_q / h_kv query heads per group (a power of two
  * <= 128); head h belongs to group h / (h_q / h_kv).  h_kidx is 1 (one index
  * key head shared by all groups) or h_kv (one per group).  scale multiplies
- * q.k in the main branch (1/sqrt(128) for the textbook softmax). */
+ * q.k in the main branch (1/sqrt(128) for the textbook softmax).
+ * q_window is a layout choice of the block->query lists, not of the method:
+ * the query indices are cut into windows of q_window consecutive queries
+ * and each block's list is split by window (see msa_build_block_query_lists).
+ * 0 selects the default (msa_query_window); otherwise a positive multiple of
+ * 128.  Results other than the lists' layout do not depend on it. */
 typedef struct {
   int64_t batch, n_q, n_kv, q_pos0;
   int32_t h_q, h_kv, h_kidx, d_idx;
   float scale;
+  int32_t q_window;
 } msa_dims;
 
 /* A strided bf16 tensor: element strides of the batch, token and head
@@ -105,6 +111,17 @@ MSA_API int64_t msa_num_blocks(const msa_dims* dims);
  * batch * h_kv * sum_i min(16, own(q_pos0 + i) + 1), own(t) = t / 128.
  * It sizes the `entries` array of msa_build_block_query_lists. */
 MSA_API int64_t msa_num_entries(const msa_dims* dims);
+
+/* The query window W of the block->query lists: dims->q_window when it is
+ * positive, else the largest power of two W >= 128 with
+ * W * (h_q / h_kv) * 256 <= 32 MiB (the bf16 query rows one window gathers
+ * for one group: about a quarter of B200's L2).  0 for invalid dims. */
+MSA_API int64_t msa_query_window(const msa_dims* dims);
+
+/* Number of segments of the block->query lists,
+ * batch * h_kv * ceil(n_q / W) * msa_num_blocks(dims); blk_offsets holds one
+ * more value.  0 for invalid dims. */
+MSA_API int64_t msa_num_segments(const msa_dims* dims);
 
 /* Step 1+2a: index scores and causal block max-pool
  * (first page, "第一步：粗筛" items 1-2: score each token, a block's score is
@@ -139,10 +156,16 @@ MSA_API size_t msa_block_query_lists_workspace(const msa_dims* dims);
 /* Step 3a: inversion of the query->block lists into block->query lists, the
  * index a KV-block-outer kernel walks (first page, "Kernel 创新：Outer Gather
  * Q": the queries that chose a block are gathered and computed together).
+ * Each block's list is split by query window (W = msa_query_window(dims)
+ * consecutive query indices): the attention kernel walks the segments in
+ * order, so at any time it gathers the query rows of one window, which stay
+ * in L2, while each K/V block is still read once per window.
  *   sel         [B, G, n_q, 16] int32 (as written by msa_topk_blocks; any
  *               valid selection works)
- *   blk_offsets [B * G * nblk + 1] int32: segment s = (b * G + g) * nblk + c
- *               holds entries[blk_offsets[s] .. blk_offsets[s+1])
+ *   blk_offsets [msa_num_segments(dims) + 1] int32: segment
+ *               s = ((b * G + g) * nwin + w) * nblk + c, nwin = ceil(n_q / W),
+ *               holds entries[blk_offsets[s] .. blk_offsets[s+1]), the
+ *               queries i of window w (w * W <= i < (w + 1) * W) that chose c
  *   entries     [msa_num_entries(dims)] int32: (i << 4) | slot for each query
  *               index i (within its batch) and the slot of c in sel[b,g,i,:],
  *               ascending in i inside a segment (deterministic counting sort)
@@ -191,7 +214,7 @@ MSA_API msa_status msa_build_block_query_lists_noalloc(const msa_dims* dims, con
 /* Step 3b: KV-block-outer sparse attention (first page "第二步：精算": full
  * attention over the selected blocks only; "稀疏注意力速览" page: exact softmax
  * attention; softmax(Q K^T * scale) V from the "稀疏注意力架构革命" page, section 1.1).  For every
- * segment (b, g, c) each K/V block is brought into shared memory once and the
+ * segment (b, g, window, c) each K/V block is brought into shared memory once and the
  * R = h_q / h_kv head rows of every listed query are gathered into 128-row
  * tensor-core tiles.  For each (query i, group g, slot, head r of the group,
  * i.e. head h = g * R + r) it writes the piece over the tokens j of block c
@@ -210,6 +233,21 @@ MSA_API msa_status msa_sparse_attn_fwd(const msa_dims* dims, msa_tensor q, msa_t
                                float* part_ml, float* part_acc,
                                int32_t* dev_err, void* stream);
 
+/* Step 3b with compact pieces (an opt-in of this library; the pages fix no
+ * piece format, and the default above keeps every piece in fp32).  Same
+ * arguments and part_ml as msa_sparse_attn_fwd, but part_acc_bf16 is
+ * [B, n_q, G, 16, R, 128] bf16 and holds acc / l: the piece's weighted mean
+ * of the V rows, a convex combination of them, so it cannot overflow; it is
+ * rounded to bf16 once.  This halves the bytes the pieces move (264 instead
+ * of 520 per (query, head, block)); merge with msa_merge_partials_compact.
+ * One query per sequence with h_q / h_kv <= 8 (the warp-level decode kernel)
+ * returns MSA_ERR_UNSUPPORTED: use the fp32 pieces there. */
+MSA_API msa_status msa_sparse_attn_fwd_compact(const msa_dims* dims, msa_tensor q, msa_tensor k,
+                                               msa_tensor v, const int32_t* blk_offsets,
+                                               const int32_t* entries, float* part_ml,
+                                               void* part_acc_bf16, int32_t* dev_err,
+                                               void* stream);
+
 /* Step 3c: log-sum-exp merge of the pieces, in slot order:
  *   M = max_s m_s, L = sum_s l_s e^{m_s - M}, o = sum_s acc_s e^{m_s - M} / L,
  *   lse = M + ln L, over the slots s with sel[b, g, i, s] >= 0.
@@ -217,6 +255,14 @@ MSA_API msa_status msa_sparse_attn_fwd(const msa_dims* dims, msa_tensor q, msa_t
 MSA_API msa_status msa_merge_partials(const msa_dims* dims, const int32_t* sel,
                               const float* part_ml, const float* part_acc,
                               void* out, float* lse, int32_t* dev_err, void* stream);
+
+/* Step 3c on compact pieces (msa_sparse_attn_fwd_compact): with
+ * accn_s = part_acc_bf16 of slot s, o = sum_s l_s e^{m_s - M} accn_s / L and
+ * lse as in msa_merge_partials. */
+MSA_API msa_status msa_merge_partials_compact(const msa_dims* dims, const int32_t* sel,
+                                              const float* part_ml, const void* part_acc_bf16,
+                                              void* out, float* lse, int32_t* dev_err,
+                                              void* stream);
 
 /* Backward of step 3b/3c for training through the sparse attention ("MSA 稀疏
  * 注意力三国杀" page, section "MSA 能力不掉：3T token 对照实验": a model trained
@@ -325,6 +371,18 @@ MSA_API msa_status msa_token_select_attention(const msa_dims* dims, msa_tensor q
                                               int64_t budget, int32_t* tokens, float* out,
                                               float* lse, void* ws, size_t ws_bytes,
                                               int32_t* dev_err, void* stream);
+
+/* Debug setting (the pages have no counterpart): the time limit, in
+ * nanoseconds, of every barrier wait inside the kernels that
+ * msa_sparse_attn_fwd and msa_sparse_attn_fwd_compact launch from now on, in
+ * this process (2 s by default; 0 restores the default, larger values are
+ * capped at it).  A wait that runs out stops its block: the block drains the
+ * loads and tensor-core work it has in flight, frees its tensor memory,
+ * stores MSA_DEVERR_TIMEOUT in *dev_err and returns, leaving the outputs
+ * incomplete.  A tiny limit (e.g. 1000) makes a valid call time out, which is
+ * how the tests exercise that path without a fault.  Returns the previous
+ * limit.  Not thread-safe against concurrent attention calls. */
+MSA_API uint64_t msa_debug_set_attn_wait_limit_ns(uint64_t ns);
 
 /* Human-readable name of a status code (static storage). */
 MSA_API const char* msa_status_string(msa_status status);

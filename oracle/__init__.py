@@ -78,7 +78,7 @@ def _load():
             lib.msa_oracle_topk_f32.argtypes = [I64, I64, P, P, P]
             lib.msa_oracle_attention.argtypes = [I64, I32, I32, I64, P, P, P, P, P, P, F64, P, P]
             lib.msa_oracle_merge.argtypes = [I64, I32, I32, P, P, P, P, P, P]
-            lib.msa_oracle_block_query_lists.argtypes = [I64, I32, I64, I64, P, P, P]
+            lib.msa_oracle_block_query_lists.argtypes = [I64, I32, I64, I64, I64, P, P, P]
             lib.msa_oracle_e4m3_value.argtypes = [ctypes.c_uint8]
             lib.msa_oracle_e4m3_value.restype = F64
             lib.msa_oracle_quantize_e4m3.argtypes = [I64, P, P, P]
@@ -210,16 +210,34 @@ def merge(valid, m, l, acc):
     return out, lse
 
 
-def block_query_lists(sel, nblk):
-    """CSR inversion of sel [B, G, n_q, 16] -> (offsets int64 [B*G*nblk+1], entries int32)."""
+def query_window(h_q, h_kv, q_window=0):
+    """The query window of the block->query lists: q_window when positive,
+    else the largest power of two W >= 128 with W * (h_q / h_kv) * 256 bytes
+    <= 32 MiB (one window's gathered query rows of one group), the rule the
+    library's header states."""
+    if q_window > 0:
+        return int(q_window)
+    R = h_q // h_kv
+    w = 128
+    while 2 * w * R * 256 <= (32 << 20):
+        w *= 2
+    return w
+
+
+def block_query_lists(sel, nblk, window=None):
+    """CSR inversion of sel [B, G, n_q, 16] with query windows of `window`
+    (default: one window over all queries) -> (offsets int64
+    [B*G*nwin*nblk+1], entries int32)."""
     lib = _load()
     s = _c(sel, np.int32)
     B, G, n_q, T = s.shape
     assert T == TOPK
-    offsets = np.empty((B * G * nblk + 1,), np.int64)
+    window = int(window or n_q)
+    nwin = (n_q + window - 1) // window
+    offsets = np.empty((B * G * nwin * nblk + 1,), np.int64)
     n_ent = int((s >= 0).sum())
     entries = np.empty((max(n_ent, 1),), np.int32)
-    lib.msa_oracle_block_query_lists(B, G, n_q, nblk, _p(s), _p(offsets), _p(entries))
+    lib.msa_oracle_block_query_lists(B, G, n_q, nblk, window, _p(s), _p(offsets), _p(entries))
     return offsets, entries[:n_ent]
 
 

@@ -269,23 +269,28 @@ void msa_oracle_merge(int64_t n, int32_t nslot, int32_t dim,
 /* Inversion of the query -> block lists into block -> query lists, the    */
 /* data structure a KV-block-outer kernel walks ([P1] "Outer Gather Q":    */
 /* all queries that chose a block are gathered and computed together).    */
-/* Segments are ordered by (batch, group, block); inside a segment the     */
+/* The query range is cut into windows of `window` consecutive query       */
+/* indices (window w holds q in [w*window, (w+1)*window)); segments are    */
+/* ordered by (batch, group, window, block), and inside a segment the      */
 /* entries are (q << 4) | slot with q ascending.  offsets has              */
-/* B*G*nblk + 1 entries, offsets[seg] .. offsets[seg+1] bound segment seg. */
+/* B*G*nwin*nblk + 1 entries, nwin = ceil(n_q / window); offsets[seg] ..   */
+/* offsets[seg+1] bound segment seg.                                       */
 /* ---------------------------------------------------------------------- */
 void msa_oracle_block_query_lists(int64_t B, int32_t G, int64_t n_q, int64_t nblk,
+                                  int64_t window,
                                   const int32_t* sel, /* [B,G,n_q,16] */
-                                  int64_t* offsets,   /* [B*G*nblk+1] */
+                                  int64_t* offsets,   /* [B*G*nwin*nblk+1] */
                                   int32_t* entries)
 {
-  const int64_t nseg = B * G * nblk;
+  const int64_t nwin = (n_q + window - 1) / window;
+  const int64_t nseg = B * G * nwin * nblk;
   int64_t* cursor = (int64_t*)calloc((size_t)nseg, sizeof(int64_t));
   for (int64_t i = 0; i <= nseg; ++i) offsets[i] = 0;
   for (int64_t bg = 0; bg < B * G; ++bg)
     for (int64_t q = 0; q < n_q; ++q)
       for (int32_t s = 0; s < MSA_TOPK; ++s) {
         const int32_t c = sel[(bg * n_q + q) * MSA_TOPK + s];
-        if (c >= 0) offsets[bg * nblk + c + 1] += 1;
+        if (c >= 0) offsets[(bg * nwin + q / window) * nblk + c + 1] += 1;
       }
   for (int64_t i = 0; i < nseg; ++i) offsets[i + 1] += offsets[i];
   for (int64_t i = 0; i < nseg; ++i) cursor[i] = offsets[i];
@@ -294,7 +299,7 @@ void msa_oracle_block_query_lists(int64_t B, int32_t G, int64_t n_q, int64_t nbl
       for (int32_t s = 0; s < MSA_TOPK; ++s) {
         const int32_t c = sel[(bg * n_q + q) * MSA_TOPK + s];
         if (c < 0) continue;
-        entries[cursor[bg * nblk + c]++] = (int32_t)((q << 4) | s);
+        entries[cursor[(bg * nwin + q / window) * nblk + c]++] = (int32_t)((q << 4) | s);
       }
   free(cursor);
 }

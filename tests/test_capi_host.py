@@ -57,7 +57,33 @@ def test_workspace_size(lib):
     nblk, ntiles = 8, 3
     nseg = 2 * 2 * nblk
     nchunks = (nseg + 4095) // 4096
+    assert capi.msa_num_segments(d) == nseg
     assert capi.msa_block_query_lists_workspace(d) == 4 * (nseg * (ntiles + 1) + nchunks)
+    # 3 query windows of 128: tile histograms + per-(window, block) totals
+    d = capi.make_dims(2, 300, 1000, 700, 8, 2, 64, q_window=128)
+    nseg = 2 * 2 * 3 * nblk
+    assert capi.msa_num_segments(d) == nseg
+    assert capi.msa_block_query_lists_workspace(d) == 4 * (2 * 2 * ntiles * nblk + nseg + 1)
+
+
+def test_query_window(lib):
+    """The default window follows the rule the header states (the same rule
+    the oracle writes out); an explicit window must be a positive multiple of
+    128."""
+    import oracle
+    for h_q, h_kv in ((64, 8), (32, 8), (32, 2), (8, 8), (4, 1)):
+        d = capi.make_dims(1, 131072, 131072, 0, h_q, h_kv, 128)
+        assert capi.msa_query_window(d) == oracle.query_window(h_q, h_kv)
+    d = capi.make_dims(1, 131072, 131072, 0, 64, 8, 128)
+    assert capi.msa_query_window(d) == 16384
+    assert capi.msa_num_segments(d) == 8 * 8 * 1024
+    assert capi.msa_query_window(capi.make_dims(1, 1000, 1000, 0, 8, 2, 64, q_window=256)) == 256
+    t = capi.Tensor(0x100000, 0, 256, 128)
+    for qw in (100, -128, 1):
+        d = capi.make_dims(1, 1000, 4096, 0, 8, 2, 128, q_window=qw)
+        assert capi.msa_query_window(d) == 0
+        assert lib.msa_index_score_maxpool(ctypes.byref(d), t, t, ctypes.c_void_p(0x200000), 32,
+                                           None, None) == 1
 
 
 BAD_DIMS = [
@@ -72,7 +98,7 @@ def test_invalid_dims_are_rejected(lib, bad):
                 scale=0.088)
     args.update(bad)
     d = capi.Dims(args["batch"], args["n_q"], args["n_kv"], args["q_pos0"], args["h_q"],
-                  args["h_kv"], args["h_kidx"], args["d_idx"], args["scale"])
+                  args["h_kv"], args["h_kidx"], args["d_idx"], args["scale"], 0)
     t = capi.Tensor(0x100000, 0, 256, 128)
     st = lib.msa_index_score_maxpool(ctypes.byref(d), t, t, ctypes.c_void_p(0x200000), 32, None,
                                      None)

@@ -5,8 +5,14 @@ The whole path runs on the GPU for every query; the oracle recomputes a
 stratified sample of query rows (first rows, the 16-block boundary, planted
 targets, random rows) from the same inputs: pooled scores, the selected set
 (bit-exact apart from counted near-ties) and the attention output.
-Selection invariants are checked on every row of the GPU result.
+Selection invariants are checked on every row of the GPU result.  Near-tie
+rows are not dropped: once the oracle's own scores show that the GPU kept one
+of the correct sets, the oracle evaluates the attention over that set.  The
+32K workload also runs with peaked softmax rows (q scaled by 4), where the
+outputs are O(1) and the absolute bars bite.
 """
+import dataclasses
+
 import numpy as np
 import pytest
 import torch
@@ -14,8 +20,8 @@ import torch
 import oracle
 from block_sparse_attention_32_b200 import pipeline, workloads as wl
 
-from _helpers import (OUT_MAX_ABS, OUT_MEAN_ABS, bits, compare_out, compare_pooled,
-                      compare_sets, pooled_tolerance, sample_rows)
+from _helpers import (assert_rows_ok, bits, compare_pooled, compare_rows, compare_sets,
+                      pooled_tolerance, rows_to_recheck, sample_rows)
 
 pytestmark = pytest.mark.gpu
 
@@ -34,19 +40,28 @@ def _invariants_all_rows(sel: torch.Tensor, w):
     assert torch.equal(last.squeeze(-1), own.expand(sel.shape[:-1]).to(sel.dtype))
 
 
-@pytest.mark.parametrize("name,n_rows,batches", [
-    ("prefill_32k", 40, None),
-    ("prefill_128k", 28, None),
-    ("chunked_prefill_1m", 12, None),
-    ("decode_64x256k", 1, [0, 37]),
+# the 32K workload with q scaled by 4: peaked softmax rows
+P32_PEAKED = dataclasses.replace(wl.P32, name="prefill_32k_peaked", q_scale=4.0)
+FULL = dict(wl.CONFIGS, **{P32_PEAKED.name: P32_PEAKED})
+
+
+@pytest.mark.parametrize("name,n_rows,batches,compact", [
+    ("prefill_32k", 40, None, False),
+    ("prefill_32k_peaked", 24, None, False),
+    ("prefill_32k_peaked", 24, None, True),
+    ("prefill_128k", 28, None, False),
+    ("prefill_128k", 20, None, True),
+    ("chunked_prefill_1m", 12, None, False),
+    ("decode_64x256k", 1, [0, 37], False),
 ])
-def test_full_size_sampled_parity(name, n_rows, batches):
+def test_full_size_sampled_parity(name, n_rows, batches, compact):
+    """compact=True runs the attention and merge on compact (bf16 acc / l) pieces."""
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
-    w = wl.CONFIGS[name]
+    w = FULL[name]
     torch.cuda.empty_cache()
     inp = wl.make_inputs(w, "cuda")
-    buf = pipeline.Buffers.allocate(pipeline.dims_for(w))
+    buf = pipeline.Buffers.allocate(pipeline.dims_for(w), compact=compact)
     out, lse = pipeline.forward(buf, inp["q"], inp["k"], inp["v"], inp["q_idx"], inp["k_idx"])
     torch.cuda.synchronize()
     assert int(buf.dev_err[0]) == 0
@@ -56,26 +71,30 @@ def test_full_size_sampled_parity(name, n_rows, batches):
     rows = sample_rows(w.n_q, w.q_pos0, n_rows, seed=1)
     pos = np.concatenate([w.q_pos0 + rows for _ in bsel])
     bat = np.concatenate([np.full(len(rows), i, np.int64) for i in range(len(bsel))])
-    qi = np.concatenate([rows for _ in bsel])
     bt = torch.tensor(bsel)
     rt = torch.tensor(rows)
     q_rows = bits(inp["q"][bt][:, rt].reshape(-1, w.h_q, 128))
     qidx_rows = bits(inp["q_idx"][bt][:, rt].reshape(-1, w.h_kv, w.d_idx))
     k_b, v_b, ki_b = (bits(inp[n][bt]) for n in ("k", "v", "k_idx"))
-    pooled_o, sel_o, out_o, _ = oracle.forward_rows(q_rows, qidx_rows, pos, bat, k_b, v_b, ki_b,
-                                                    w.scale)
     gp = buf.pooled[bt][:, :, rt].permute(0, 2, 1, 3).reshape(len(pos), w.h_kv, -1).cpu().numpy()
+    gs = buf.sel[bt][:, :, rt].permute(0, 2, 1, 3).reshape(len(pos), w.h_kv, 16).cpu().numpy()
+    go = out[bt][:, rt].float().reshape(len(pos), w.h_q, 128).cpu().numpy()
+    gl = lse[bt][:, rt].reshape(len(pos), w.h_q).cpu().numpy()
+    del inp, buf, out, lse
+    torch.cuda.empty_cache()
+    pooled_o, sel_o, out_o, lse_o = oracle.forward_rows(q_rows, qidx_rows, pos, bat, k_b, v_b,
+                                                        ki_b, w.scale)
     tol = pooled_tolerance(qidx_rows, ki_b, pos, bat, w.h_kidx)
     worst = compare_pooled(gp, pooled_o, tol, pos)
-    gs = buf.sel[bt][:, :, rt].permute(0, 2, 1, 3).reshape(len(pos), w.h_kv, 16).cpu().numpy()
-    bad, ties, bad_cert, ok = compare_sets(gs, sel_o, pooled_o, pos)
-    go = out[bt][:, rt].float().reshape(len(pos), w.h_q, 128).cpu().numpy()
-    mx, mean = compare_out(go[ok], out_o[ok])
-    print(f"{name}: rows={len(pos)} pooled_err/tol={worst:.3f} near_ties={ties} "
-          f"set_mismatch={bad} out_max={mx:.3g} out_mean={mean:.3g}")
-    del inp, buf
-    torch.cuda.empty_cache()
+    bad, ties, bad_tie, eval_sel = compare_sets(gs, sel_o, pooled_o, pos)
+    redo = rows_to_recheck(eval_sel, sel_o)
+    if len(redo):
+        o2, l2 = oracle.attention(q_rows[redo], pos[redo], bat[redo], k_b, v_b, eval_sel[redo],
+                                  w.scale)
+        out_o[redo], lse_o[redo] = o2, l2
+    res = compare_rows(go, gl, out_o, lse_o)
+    print(f"{name} compact={compact}: rows={len(pos)} pooled_err/tol={worst:.3f} near_ties={ties} "
+          f"set_mismatch={bad} rechecked_rows={len(redo)} {res}")
     assert worst <= 1.0
-    assert bad == 0 and bad_cert == 0
-    assert ok.sum() >= len(pos) - ties
-    assert mx <= OUT_MAX_ABS and mean <= OUT_MEAN_ABS
+    assert bad == 0 and bad_tie == 0
+    assert_rows_ok(res, name)

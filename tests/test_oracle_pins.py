@@ -304,7 +304,8 @@ def test_merge_of_per_block_pieces_equals_attention_over_the_union():
 # ----------------------------------------------------------------------------
 # block -> query lists
 # ----------------------------------------------------------------------------
-def test_block_query_lists_against_a_stable_sort():
+@pytest.mark.parametrize("window", [None, 128, 100, 37])
+def test_block_query_lists_against_a_stable_sort(window):
     rng = np.random.default_rng(9)
     B, G, n_q, nblk = 2, 3, 300, 7
     sel = np.full((B, G, n_q, 16), -1, np.int32)
@@ -313,17 +314,35 @@ def test_block_query_lists_against_a_stable_sort():
             for q in range(n_q):
                 k = rng.integers(1, 8)
                 sel[b, g, q, :k] = np.sort(rng.choice(nblk, size=k, replace=False))
-    offsets, entries = oracle.block_query_lists(sel, nblk)
-    # independent construction: sort all (segment, q, slot) triples
+    offsets, entries = oracle.block_query_lists(sel, nblk, window)
+    # independent construction: sort all (segment, q, slot) triples, the
+    # segment numbering (batch, group, query window, block)
+    win = window or n_q
+    nwin = -(-n_q // win)
     bb, gg, qq, ss = np.nonzero(sel >= 0)
     cc = sel[bb, gg, qq, ss]
-    seg = (bb * G + gg) * nblk + cc
+    seg = ((bb * G + gg) * nwin + qq // win) * nblk + cc
     order = np.lexsort((ss, qq, seg))
     want = (qq[order] << 4) | ss[order]
     np.testing.assert_array_equal(entries, want.astype(np.int32))
-    counts = np.bincount(seg, minlength=B * G * nblk)
+    counts = np.bincount(seg, minlength=B * G * nwin * nblk)
     np.testing.assert_array_equal(offsets, np.concatenate([[0], np.cumsum(counts)]))
     assert len(entries) == (sel >= 0).sum()
+    # each segment's queries lie in its window
+    for sgi in range(B * G * nwin * nblk):
+        w = (sgi // nblk) % nwin
+        qs = entries[offsets[sgi]:offsets[sgi + 1]] >> 4
+        assert ((qs >= w * win) & (qs < (w + 1) * win)).all()
+
+
+def test_query_window_rule():
+    """Default window: the largest power of two (>= 128) whose gathered query
+    rows of one group, window x R x 256 bytes, fit in 32 MiB."""
+    assert oracle.query_window(64, 8) == 16384      # R = 8
+    assert oracle.query_window(32, 8) == 32768      # R = 4
+    assert oracle.query_window(32, 2) == 8192       # R = 16
+    assert oracle.query_window(8, 8) == 131072      # R = 1
+    assert oracle.query_window(64, 8, 384) == 384
 
 
 # ----------------------------------------------------------------------------

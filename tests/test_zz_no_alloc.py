@@ -30,8 +30,7 @@ def _lists_with_workspace(d, sel):
 
 
 def _lists_without_workspace(d, sel):
-    nblk = capi.msa_num_blocks(d)
-    offsets = torch.full((d.batch * d.h_kv * nblk + 1,), -7, dtype=torch.int32, device="cuda")
+    offsets = torch.full((capi.msa_num_segments(d) + 1,), -7, dtype=torch.int32, device="cuda")
     entries = torch.full((max(capi.msa_num_entries(d), 1),), -7, dtype=torch.int32, device="cuda")
     err = torch.zeros((4,), dtype=torch.int32, device="cuda")
     capi.msa_build_block_query_lists_noalloc(d, sel, offsets, entries, err)
@@ -44,6 +43,7 @@ def _lists_without_workspace(d, sel):
     wl.small("ragged_r4", 1, 2500, 2500, 0, 8, 2, 128, seed=31),
     wl.small("chunk_unaligned", 2, 1600, 2600, 1000, 4, 2, 64, seed=32),
     wl.small("decode_like", 16, 1, 40000, 39999, 64, 8, 128, seed=33),
+    wl.small("windows_of_256", 1, 2000, 2000, 0, 16, 2, 128, seed=34, q_window=256),
 ], ids=lambda w: w.name)
 def test_noalloc_lists_match_the_workspace_version_twice(w):
     if not torch.cuda.is_available():
