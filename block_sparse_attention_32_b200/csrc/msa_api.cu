@@ -191,6 +191,26 @@ msa_status make_map_rows_bf16(CUtensorMap* map, void* ptr, uint64_t rows, uint32
 
 msa_status from_cuda(cudaError_t e) { return e == cudaSuccess ? MSA_OK : MSA_ERR_CUDA; }
 
+// 5-D bf16 view of q [B, n_q, H, 128] for the attention kernel's gather: dims
+// {64 columns, H heads, 2 panels of 64 columns, n_q, B} with byte strides
+// {head, 128, token, batch}; box {64, 8, 2, 1, 1} = eight heads of one query,
+// both panels, 2 KB, landing as [panel][8 rows][128 B] (128-byte swizzle).
+msa_status make_map_q_groups(CUtensorMap* map, const msa_dims* d, const msa_tensor& q) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return MSA_ERR_CUDA;
+  cuuint64_t dims[5] = {64, (cuuint64_t)d->h_q, 2, (cuuint64_t)d->n_q, (cuuint64_t)d->batch};
+  cuuint64_t strides[4] = {(cuuint64_t)q.s_head * 2, 128, (cuuint64_t)q.s_tok * 2,
+                           (cuuint64_t)q.s_batch * 2};
+  for (int i = 0; i < 4; ++i)
+    if (strides[i] == 0) strides[i] = 16;      // a dimension of extent 1 still needs a stride
+  cuuint32_t box[5] = {64, 8, 2, 1, 1};
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(q.ptr), dims,
+                  strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? MSA_OK : MSA_ERR_CUDA;
+}
+
 // 4-D uint8 map (e4m3 codes): dims {inner, d1, d2, d3}, byte strides, box
 // {128, b1, b2, 1}, 128-byte swizzle, zero fill out of bounds.
 msa_status make_map_u8(CUtensorMap* map, const void* ptr, uint64_t inner, uint64_t d1,
@@ -376,10 +396,8 @@ msa_status sparse_attn_fwd(const msa_dims* d, msa_tensor q, msa_tensor k, msa_te
         reinterpret_cast<cudaStream_t>(stream)));
   }
   if (R >= 8) {
-    // q [B, n_q, H, 128]: dims {128, H, n_q, B}, box {64, R, 1, 1} (one entry's heads)
-    if ((s = make_map(&tq, q.ptr, MSA_HEAD_DIM, d->h_q, d->n_q, d->batch, q.s_head, q.s_tok,
-                      q.s_batch, (uint32_t)R, 1)) != MSA_OK)
-      return s;
+    // q: one box per group of eight heads of an entry (both 64-column panels)
+    if ((s = make_map_q_groups(&tq, d, q)) != MSA_OK) return s;
     const int64_t rows = d->batch * d->n_q * d->h_kv * MSA_TOPK_BLOCKS * R;
     if (rows >= (int64_t(1) << 31)) return MSA_ERR_UNSUPPORTED;
     s = compact ? make_map_rows_bf16(&to, part_acc, (uint64_t)rows, (uint32_t)R)

@@ -30,17 +30,16 @@
 //                             one is done, V as soon as its last P V is done
 //   warp 3      idle (fills the control warpgroup)
 //   warps 4-7   gather:       the chunk's Q rows into a 3-deep ring: for R >= 8
-//                             warp 4 alone, one TMA box per entry and
-//                             64-column panel (an entry's R head rows are
-//                             contiguous), otherwise 16-byte cp.async by all
-//                             four warps
-//   warps 8-15  softmax:      two warpgroups, one per half of the keys; each
-//                             holds its 64 S values of a row in registers,
-//                             the halves exchange row maxima through shared
-//                             memory (an mbarrier per quarter and chunk
-//                             parity), and P = bf16(e^{s-m}) goes back into
-//                             the first 64 columns of the S buffer in TMEM
-//                             (the A operand of O = P V)
+//                             warp 4 alone, one 2 KB TMA box per eight heads
+//                             of an entry (both 64-column panels; a 5-D view
+//                             of q), otherwise 16-byte cp.async by all four
+//                             warps
+//   warps 8-15  softmax:      two warpgroups in ping-pong, warpgroup h on
+//                             the chunks n % 2 == h (S buffer h); thread =
+//                             row: the row maximum over the 128 keys, then
+//                             P = bf16(e^{s-m}) back into the first 64
+//                             columns of the S buffer in TMEM (the A operand
+//                             of O = P V)
 //   warps 16-19 epilogue:     O from TMEM half a row at a time, then the
 //                             (m, l, acc) pieces to global memory.  R >= 8:
 //                             the half rows are staged in 128B-swizzled
@@ -50,7 +49,8 @@
 //                             writes two whole half rows (coalesced)
 // The five warpgroups split the register file unevenly (setmaxnreg).
 // Shared memory: K 32 KB, V 32 KB, 3 x 32 KB Q tiles (128B-swizzled K-major;
-// V is read N-major for P V), 34 KB output staging, (m, l) slots and the row
+// a Q tile gathered by TMA is laid out [8-row group][panel][8 rows][128 B] so
+// that one box brings eight heads of an entry; V is read N-major for P V), 34 KB output staging, (m, l) slots and the row
 // maxima the two softmax halves exchange.  TMEM: S/P in columns [0,256), O in
 // [256,512), two buffers of 128 columns each; a Q tile is released as soon as
 // its S MMA is done, S(n+2) waits for O(n) = P(n) V, which reads P(n) from
@@ -91,11 +91,10 @@ constexpr int kOffV = 32768;           // 32768: [V lo | V hi]
 constexpr int kOffQP = 65536;          // kQRing x 32768: Q tile, then P
 constexpr int kStageRow = 272;                           // staged half row (256 B + pad)
 constexpr int kOffStage = kOffQP + kQRing * 32768;       // 128 staged rows
-constexpr int kOffML = kOffStage + 128 * kStageRow;      // [2 slots][2 halves][128] float2 (m, l)
-constexpr int kOffMX = kOffML + 4096;                    // [2][2 halves][128] float row maxima
-constexpr int kOffDesc = kOffMX + 2048;                  // kDescRing descriptors
+constexpr int kOffML = kOffStage + 128 * kStageRow;      // [2 slots][128] float2 (m, l)
+constexpr int kOffDesc = kOffML + 2048;                  // kDescRing descriptors
 constexpr int kOffBar = kOffDesc + kDescRing * (int)sizeof(ChunkDesc);
-constexpr int kNumBars = 4 + 3 * kQRing + 6 + 2 * kDescRing + 2 + 1 + 8;
+constexpr int kNumBars = 4 + 3 * kQRing + 6 + 2 * kDescRing + 2 + 1;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;         // TMEM base, abort flag
 constexpr int kAttnSmemBytes = 1024 + kOffMisc + 64;
 
@@ -105,9 +104,7 @@ enum {
   BAR_S_FULL = 4 + 3 * kQRing, BAR_O_FULL = BAR_S_FULL + 2, BAR_O_EMPTY = BAR_S_FULL + 4,
   BAR_D_FULL = BAR_S_FULL + 6, BAR_D_EMPTY = BAR_D_FULL + kDescRing,
   BAR_ML_EMPTY = BAR_D_EMPTY + kDescRing,
-  BAR_DRAIN = BAR_ML_EMPTY + 2,     // the MMA issuer's last commit (all its MMAs done)
-  BAR_MX = BAR_DRAIN + 1            // [quarter][chunk parity]: the two softmax halves'
-                                    // row maxima of a chunk are written
+  BAR_DRAIN = BAR_ML_EMPTY + 2      // the MMA issuer's last commit (all its MMAs done)
 };
 
 struct AttnArgs {
@@ -158,7 +155,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                                              ~uintptr_t(1023));
   uint64_t* bar = reinterpret_cast<uint64_t*>(base + kOffBar);
   float2* ml_s = reinterpret_cast<float2*>(base + kOffML);
-  float* mx_x = reinterpret_cast<float*>(base + kOffMX);
   ChunkDesc* desc = reinterpret_cast<ChunkDesc*>(base + kOffDesc);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(base + kOffMisc + 4);
@@ -172,7 +168,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     for (int i = 0; i < kQRing; ++i) {
       mbar_init(bar + BAR_Q_FULL + i, kTmaGather ? 1 : 128);
       mbar_init(bar + BAR_QP_EMPTY + i, 1);
-      mbar_init(bar + BAR_P_FULL + i, 256);
+      mbar_init(bar + BAR_P_FULL + i, 128);       // the chunk's softmax warpgroup
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar + BAR_S_FULL + i, 1);
@@ -185,7 +181,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_init(bar + BAR_D_EMPTY + i, 128 + 1);   // epilogue threads + TMA producer
     }
     mbar_init(bar + BAR_DRAIN, 1);
-    for (int i = 0; i < 8; ++i) mbar_init(bar + BAR_MX + i, 2);   // one warp of each half
     *abort_flag = 0;
     fence_mbarrier_init();
   }
@@ -211,6 +206,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   auto Wfree = [&](int id, int depth, int64_t n) {
     return n < depth || mbar_wait(bar + id + (int)(n % depth),
                                   (uint32_t)(((n / depth) + 1) & 1), abort_flag, err, wait_lim);
+  };
+  // The same for roles whose whole warp goes on to warp-collective instructions
+  // (tcgen05.ld/st .sync.aligned, votes, shuffles): every lane waits, then the
+  // warp votes, so that after a timeout no lane carries on while another has
+  // left (a lane still waiting returns once the abort flag is set).
+  auto WuseW = [&](int id, int depth, int64_t n) {
+    return __all_sync(0xffffffffu, Wuse(id, depth, n) ? 1 : 0) != 0;
+  };
+  auto WfreeW = [&](int id, int depth, int64_t n) {
+    return __all_sync(0xffffffffu, Wfree(id, depth, n) ? 1 : 0) != 0;
   };
 
   // Roles by warpgroup; each warpgroup first resizes its registers (all four
@@ -272,11 +277,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           if (pos < e1) seg = warp_find_segment(a.blk_offsets, seg + 1, a.n_seg, pos, lane);
         }
       }
-      if (ok && claim(chunk)) {          // end marker
+      // end markers in two consecutive slots: the softmax warpgroups each look
+      // at every other chunk, so each must find one
+      for (int k = 0; ok && k < 2; ++k) {
+        if (!claim(chunk)) break;
         if (lane == 0) {
           desc[chunk % kDescRing].cnt = -1;
           mbar_arrive(bar + BAR_D_FULL + (int)(chunk % kDescRing));
         }
+        ++chunk;
       }
     } else if (warp == 1) {
       // ---------------- MMA issuer ----------------
@@ -327,9 +336,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           const uint32_t ka = smem_u32(base + kOffK);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-            umma_bf16(tmem + sb * 128, smem_desc_sw128(qa + off, 16, 1024),
-                      smem_desc_sw128(ka + off, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
+            // K: [panel][128 rows][128 B] (8-row groups 1024 B apart); Q for R >= 8:
+            // [8-row group][panel][8 rows][128 B] (groups 2048 B apart), else as K
+            const uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32;
+            const uint32_t qoff = kTmaGather ? (kk >> 2) * 1024 + (kk & 3) * 32 : koff;
+            umma_bf16(tmem + sb * 128, smem_desc_sw128(qa + qoff, 16, kTmaGather ? 2048 : 1024),
+                      smem_desc_sw128(ka + koff, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
           }
           umma_commit(bar + BAR_S_FULL + sb);
           umma_commit(bar + BAR_QP_EMPTY + qb);
@@ -394,13 +406,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     setmaxnreg_dec<kRegsGather>();
     if constexpr (kTmaGather) {
       // warp 4 alone: lane 0 arms Q_FULL with the chunk's bytes, then lane l
-      // issues the TMA boxes (R rows x 64 columns) of entries l, l+32, ... for
-      // both 128-byte panels.  One thread arms each phase, so on an abort it
-      // knows which loads are in flight and drains exactly those.
+      // issues the box of 8-row group l: eight heads of one entry, both
+      // 64-column panels (2 KB), into [group][panel][8 rows][128 B] of the Q
+      // tile.  One thread arms each phase, so on an abort it knows which loads
+      // are in flight and drains exactly those.
       if (warp == 4) {
+        constexpr int kGroups = R / 8;           // 8-row groups per entry
         int64_t armed = -1;                      // last chunk whose loads were issued
         for (int64_t n = 0;; ++n) {
-          if (!Wuse(BAR_D_FULL, kDescRing, n)) break;
+          if (!WuseW(BAR_D_FULL, kDescRing, n)) break;
           const ChunkDesc& d = desc[n % kDescRing];
           if (d.cnt < 0) break;
           const int qb = (int)(n % kQRing);
@@ -420,12 +434,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           if (!__shfl_sync(0xffffffffu, ok, 0)) break;
           armed = n;
           uint8_t* sq = base + kOffQP + qb * 32768;
-          for (int t = lane; t < 2 * CH; t += 32) {
-            const int k = t >> 1, p = t & 1;
+          if (lane < 16) {                       // 16 groups of 8 rows per tile
+            const int k = lane / kGroups, j = lane % kGroups;
             const int e = d.ent[k];
-            if (e < 0 || (int64_t)(e >> 4) >= a.n_q) continue;
-            tma_load_4d(sq + p * 16384 + k * R * 128, &tm_q, bar + BAR_Q_FULL + qb, p * 64,
-                        d.g * R, e >> 4, d.b);
+            if (e >= 0 && (int64_t)(e >> 4) < a.n_q)
+              tma_load_5d(sq + lane * 2048, &tm_q, bar + BAR_Q_FULL + qb, 0, d.g * R + 8 * j, 0,
+                          e >> 4, d.b);
           }
         }
         if (lane == 0 && armed >= 0)
@@ -465,29 +479,29 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
   } else if (warp < 16) {
     // ---------------- softmax: S -> P, (m, l) ----------------
-    // warpgroup h (0, 1) takes keys 64h .. 64h+63 of every row; the two
-    // halves of a row exchange their maxima through shared memory (an
-    // mbarrier per quarter and chunk parity, one arrival per warp) and each
-    // writes its own sum.
+    // Ping-pong: warpgroup h takes the chunks n with n % 2 == h, whose S lives
+    // in TMEM buffer h, so the two warpgroups work on neighbouring chunks at
+    // once and never wait on each other.  Thread = row = TMEM lane: a first
+    // pass over the row's 128 keys takes the maximum, a second computes
+    // e^{s-m} 32 keys at a time and writes P as bf16 into the first 64
+    // columns of the same buffer (keys 32j.. -> columns 16j..; columns are
+    // overwritten only after they were read), the A operand of O = P V.
     setmaxnreg_inc<kRegsSoftmax>();
     const int h = (warp >> 2) - 2;
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     const float scale_log2 = a.scale * 1.4426950408889634f;
-    for (int64_t n = 0;; ++n) {
-      if (!Wuse(BAR_D_FULL, kDescRing, n)) break;
+    for (int64_t n = h;; n += 2) {
+      if (!WuseW(BAR_D_FULL, kDescRing, n)) break;
       const ChunkDesc& d = desc[n % kDescRing];
       if (d.cnt < 0) break;
       const int qb = (int)(n % kQRing), sb = (int)(n & 1);
       const int e = d.ent[row / R];
       const int32_t c = d.c;
-      if (!Wuse(BAR_S_FULL, 2, n)) break;
+      if (!WuseW(BAR_S_FULL, 2, n)) break;
       tc_fence_after();
       const uint32_t s_addr = tmem + lane_base + sb * 128;
-      uint32_t r0[32], r1[32];
-      tmem_ld_32x32b_x32(s_addr + 64 * h, r0);
-      tmem_ld_32x32b_x32(s_addr + 64 * h + 32, r1);
       const int64_t qi = (int64_t)(e >> 4);
       bool valid = (e >= 0) && (qi < a.n_q);
       int lim = 127;
@@ -495,54 +509,47 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const int64_t rel = a.q_pos0 + qi - (int64_t)c * kBlock;
         if (rel < 0) {
           valid = false;
-          if (h == 0) report(err, MSA_DEVERR_BAD_ENTRY);
+          report(err, MSA_DEVERR_BAD_ENTRY);
         } else if (rel < 127) {
           lim = (int)rel;
         }
       }
       if (!valid) lim = -1;                   // every weight of the row is zero
-      const int k0 = 64 * h;
       // only rows of the query's own block mask keys (past the query); a warp
       // with no such row skips every per-key compare
       const bool masked = __any_sync(0xffffffffu, lim >= 0 && lim < 127);
-      tmem_ld_wait();
       float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-      if (!masked) {
+#pragma unroll 1
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t r0[32], r1[32];
+        tmem_ld_32x32b_x32(s_addr + 64 * hh, r0);
+        tmem_ld_32x32b_x32(s_addr + 64 * hh + 32, r1);
+        tmem_ld_wait();
+        const int k0 = 64 * hh;
+        if (!masked) {
 #pragma unroll
-        for (int x = 0; x < 32; x += 2) {
-          m4[0] = fmaxf(m4[0], u2f(r0[x]));
-          m4[1] = fmaxf(m4[1], u2f(r0[x + 1]));
-          m4[2] = fmaxf(m4[2], u2f(r1[x]));
-          m4[3] = fmaxf(m4[3], u2f(r1[x + 1]));
-        }
-      } else {
+          for (int x = 0; x < 32; x += 2) {
+            m4[0] = fmaxf(m4[0], u2f(r0[x]));
+            m4[1] = fmaxf(m4[1], u2f(r0[x + 1]));
+            m4[2] = fmaxf(m4[2], u2f(r1[x]));
+            m4[3] = fmaxf(m4[3], u2f(r1[x + 1]));
+          }
+        } else {
 #pragma unroll
-        for (int x = 0; x < 32; x += 2) {
-          m4[0] = fmaxf(m4[0], k0 + x <= lim ? u2f(r0[x]) : -INFINITY);
-          m4[1] = fmaxf(m4[1], k0 + x + 1 <= lim ? u2f(r0[x + 1]) : -INFINITY);
-          m4[2] = fmaxf(m4[2], k0 + 32 + x <= lim ? u2f(r1[x]) : -INFINITY);
-          m4[3] = fmaxf(m4[3], k0 + 33 + x <= lim ? u2f(r1[x + 1]) : -INFINITY);
+          for (int x = 0; x < 32; x += 2) {
+            m4[0] = fmaxf(m4[0], k0 + x <= lim ? u2f(r0[x]) : -INFINITY);
+            m4[1] = fmaxf(m4[1], k0 + x + 1 <= lim ? u2f(r0[x + 1]) : -INFINITY);
+            m4[2] = fmaxf(m4[2], k0 + 32 + x <= lim ? u2f(r1[x]) : -INFINITY);
+            m4[3] = fmaxf(m4[3], k0 + 33 + x <= lim ? u2f(r1[x + 1]) : -INFINITY);
+          }
         }
       }
-      const float mloc = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-      float* mxn = mx_x + (int)(n & 1) * 256;   // by parity: the partner reads it before n+2
-      mxn[h * 128 + row] = mloc;
-      tc_fence_before();                       // this half's S reads precede the other's P writes
-      // exchange with the other half's warp of this quarter through an mbarrier
-      // (a bounded wait: neither half can be left waiting on the other)
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar + BAR_MX + quarter * 2 + (int)(n & 1));
-      if (!mbar_wait(bar + BAR_MX + quarter * 2 + (int)(n & 1), (uint32_t)((n >> 1) & 1),
-                     abort_flag, err, wait_lim))
-        break;
-      tc_fence_after();
-      float mx = fmaxf(mloc, mxn[(1 - h) * 128 + row]);
+      float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
       if (!valid) mx = 0.f;
       // e^{s-m} = 2^{s log2(e) scale - m log2(e) scale}; a row with no valid
       // key gets weight 2^-inf = 0 everywhere
       const float mneg = valid ? -mx * scale_log2 : -INFINITY;
       float lsum[4] = {0.f, 0.f, 0.f, 0.f};
-      // keys 32j..32j+31 -> columns 16j..16j+15 of this S buffer (already read).
       // P is rounded to bf16 for the P V product; l sums the fp32 weights.
       auto exp_pack_store = [&](const uint32_t (&r)[32], int j, bool mask) {
         uint32_t w[16];
@@ -560,19 +567,26 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
         tmem_st_32x32b_x16(s_addr + j * 16, w);
       };
-      if (!masked) {
-        exp_pack_store(r0, 2 * h, false);
-        exp_pack_store(r1, 2 * h + 1, false);
-      } else {
-        exp_pack_store(r0, 2 * h, true);
-        exp_pack_store(r1, 2 * h + 1, true);
+      // keys 32j .. 32j+31: the next block of S is loaded while this one is
+      // exponentiated (a load waits for every earlier load of the thread)
+      uint32_t ra[32], rb[32];
+      tmem_ld_32x32b_x32(s_addr, ra);
+      tmem_ld_wait();
+#pragma unroll
+      for (int j = 0; j < 4; j += 2) {
+        tmem_ld_32x32b_x32(s_addr + 32 * (j + 1), rb);
+        if (!masked) exp_pack_store(ra, j, false); else exp_pack_store(ra, j, true);
+        tmem_ld_wait();
+        if (j + 2 < 4) tmem_ld_32x32b_x32(s_addr + 32 * (j + 2), ra);
+        if (!masked) exp_pack_store(rb, j + 1, false); else exp_pack_store(rb, j + 1, true);
+        if (j + 2 < 4) tmem_ld_wait();
       }
       tmem_st_wait();
       const float l = (lsum[0] + lsum[1]) + (lsum[2] + lsum[3]);
       // (m, l) slot sb is free once the epilogue of n-2 has read it; P V(n)
-      // is issued only after both halves arrive
-      if (!Wfree(BAR_ML_EMPTY, 2, n)) break;
-      ml_s[(sb * 2 + h) * 128 + row] = make_float2(mx * a.scale, l);
+      // is issued only after the warpgroup arrives
+      if (!WfreeW(BAR_ML_EMPTY, 2, n)) break;
+      ml_s[sb * 128 + row] = make_float2(mx * a.scale, l);
       tc_fence_before();
       mbar_arrive(bar + BAR_P_FULL + qb);
     }
@@ -593,17 +607,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     uint8_t* srow = base + kOffStage + row * kStageRow;
     uint8_t* swarp = base + kOffStage + (quarter * 32) * kStageRow;
     for (int64_t n = 0;; ++n) {
-      if (!Wuse(BAR_D_FULL, kDescRing, n)) break;
+      if (!WuseW(BAR_D_FULL, kDescRing, n)) break;
       const ChunkDesc& d = desc[n % kDescRing];
       if (d.cnt < 0) break;
       const int ob = (int)(n & 1);
       const int e = d.ent[row / R];
       const int32_t b = d.b, g = d.g, c = d.c;
-      if (!Wuse(BAR_O_FULL, 2, n)) break;
-      if (!Wuse(BAR_P_FULL, kQRing, n)) break;   // acquire the softmax's (m, l)
+      if (!WuseW(BAR_O_FULL, 2, n)) break;
+      if (!WuseW(BAR_P_FULL, kQRing, n)) break;  // acquire the softmax's (m, l)
       tc_fence_after();
-      const float2 ml0 = ml_s[(ob * 2) * 128 + row];
-      const float2 ml1 = ml_s[(ob * 2 + 1) * 128 + row];
+      const float2 ml = ml_s[ob * 128 + row];
       mbar_arrive(bar + BAR_ML_EMPTY + ob);      // (m, l) slot ob is free
       const int hr = row % R;
       const int64_t qi = (int64_t)(e >> 4);
@@ -611,8 +624,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       // piece row of (b, qi, g, slot, hr): the R head rows of one entry are adjacent
       const int64_t pidx =
           valid ? ((((int64_t)b * a.n_q + qi) * a.G + g) * kTopK + (e & 15)) * R + hr : 0;
-      const float l_sum = ml0.y + ml1.y;
-      if (valid) *reinterpret_cast<float2*>(a.part_ml + pidx * 2) = make_float2(ml0.x, l_sum);
+      const float l_sum = ml.y;
+      if (valid) *reinterpret_cast<float2*>(a.part_ml + pidx * 2) = make_float2(ml.x, l_sum);
       // compact pieces: acc / l (l >= 1 on a valid row: the row maximum's weight is 1)
       const float inv_l = (kCompact && valid && l_sum > 0.f) ? 1.0f / l_sum : 0.f;
       const uint32_t o_addr = tmem + lane_base + 256 + ob * 128;

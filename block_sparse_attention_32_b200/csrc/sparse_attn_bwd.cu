@@ -17,10 +17,13 @@
 //
 // Three kernels:
 //  * bwd_delta_kernel      -- D = dO.o per (query, head), one warp each;
-//  * sparse_attn_bwd_tc_kernel<R> -- the entries of the block->query lists
-//    are cut into equal runs ("chunks", strided over a grid of at most one
-//    CTA per SM), a chunk into pieces (one per segment = KV block) and a
-//    piece into 128-row tiles (128 / R entries x R heads).  Warp roles
+//  * sparse_attn_bwd_tc_kernel<R> -- every (batch, group, KV block) is one
+//    work item, owned by one CTA (items dealt to a grid of at most one CTA
+//    per SM in snake order: round j gives CTA k item j * grid + k for even
+//    j, j * grid + grid - 1 - k for odd j, which evens out the sizes, large
+//    for early blocks).  A piece is an item with entries: its query-window
+//    segments in window order, each cut into 128-row tiles (128 / R
+//    entries x R heads).  Warp roles
 //    (512 threads): a TMA warp loads each piece's K and V; four gather warps
 //    bring each tile's Q and dO rows by cp.async into two buffers; an MMA
 //    warp issues, per tile, S^T = K Q^T and dP^T = V dO^T (tcgen05, M = 128
@@ -28,9 +31,8 @@
 //    turned them into P^T and dS^T (bf16, back into TMEM, and dS^T also into
 //    shared memory) -- dV += P^T dO and dK += dS^T Q with A read from TMEM,
 //    and dQ = dS K with A read from shared memory; four epilogue warps store
-//    the dQ pieces and, at the end of a piece, add dK and dV into the fp32
-//    outputs (vector atomics: a block split over several chunks sums its
-//    parts there);
+//    the dQ pieces and, at the end of a piece, store the block's dK and dV
+//    (one CTA owns a block: no atomics, bit-identical from run to run);
 //  * bwd_dq_reduce_kernel  -- dQ = sum over the slots of the pieces, one warp
 //    per (query, head).
 #include "common.cuh"
@@ -51,7 +53,7 @@ struct BwdArgs {
   float* part_dq;             // [B, n_q, G, 16, R, 128]
   float* dk;                  // [B, G, n_kv, 128]
   float* dv;
-  int64_t n_q, n_kv, q_pos0, nseg, total, chunk_entries;
+  int64_t n_q, n_kv, q_pos0, nseg, total, nitems;   // items: (batch, group, block)
   int32_t G, H, nblk, nwin;   // segments are (batch, group, query window, block)
   float scale;
   int32_t* err;
@@ -125,50 +127,61 @@ constexpr uint32_t idesc_tc(int a_mn, int b_mn) {
          ((uint32_t)(128 >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
 }
 
-// The CTA's sequence of pieces: runs of chunk_entries entries (chunks
-// blockIdx.x, + gridDim.x, ...), each cut at segment boundaries.  Every role
-// walks the same sequence.
+// The CTA's sequence of pieces: its items in snake order, skipping blocks no
+// query selected.  Every role walks the same sequence.
 struct PieceWalk {
-  int64_t chunk, c_end, e, seg;
+  int64_t round;
 };
 struct Piece {
-  int64_t b, e0, e1;
-  int32_t g, c;
+  int64_t b, seg0, nt;   // seg0: the segment of window 0 (window w: seg0 + w * nblk)
+  int32_t g, c;          // nt: 128-row tiles of the piece
 };
-__device__ __forceinline__ void walk_start(PieceWalk& w, const BwdArgs& a) {
-  w.chunk = blockIdx.x;
-  w.e = w.chunk * a.chunk_entries;
-  w.c_end = min64(w.e + a.chunk_entries, a.total);
-  w.seg = -1;
+// the tiles of one piece: window by window, kEnt entries each
+struct TileWalk {
+  int64_t e, e_end;
+  int32_t w;
+};
+__device__ __forceinline__ void walk_start(PieceWalk& w) { w.round = 0; }
+__device__ __forceinline__ bool walk_next(PieceWalk& w, const BwdArgs& a, Piece& pc, int kEnt) {
+  for (;;) {
+    const int64_t j = w.round++;
+    const int64_t k = (j & 1) ? (int64_t)(gridDim.x - 1 - blockIdx.x) : (int64_t)blockIdx.x;
+    const int64_t i = j * gridDim.x + k;                 // grows with j: the last item ends it
+    if (i >= a.nitems) return false;
+    const int64_t bg = i / a.nblk;
+    const int32_t c = (int32_t)(i - bg * a.nblk);
+    const int64_t seg0 = bg * a.nwin * a.nblk + c;
+    int64_t nt = 0;
+    for (int32_t win = 0; win < a.nwin; ++win) {
+      const int64_t sg = seg0 + (int64_t)win * a.nblk;
+      nt += ((int64_t)__ldg(a.offsets + sg + 1) - __ldg(a.offsets + sg) + kEnt - 1) / kEnt;
+    }
+    if (nt <= 0) continue;
+    pc.b = bg / a.G;
+    pc.g = (int32_t)(bg - pc.b * a.G);
+    pc.c = c;
+    pc.seg0 = seg0;
+    pc.nt = nt;
+    return true;
+  }
 }
-// false at the end of the CTA's work, or (with *bad set) when the lists hold
-// fewer entries than the sizes imply
-__device__ __forceinline__ bool walk_next(PieceWalk& w, const BwdArgs& a, Piece& pc, bool* bad) {
-  *bad = false;
-  while (w.e >= w.c_end) {
-    w.chunk += gridDim.x;
-    if (w.chunk * a.chunk_entries >= a.total) return false;
-    w.e = w.chunk * a.chunk_entries;
-    w.c_end = min64(w.e + a.chunk_entries, a.total);
-    w.seg = -1;
+__device__ __forceinline__ void tiles_start(TileWalk& t) {
+  t.e = 0;
+  t.e_end = 0;
+  t.w = -1;
+}
+// entries [e0, e1) of the piece's next tile (called exactly pc.nt times)
+__device__ __forceinline__ void tiles_next(TileWalk& t, const BwdArgs& a, const Piece& pc,
+                                           int kEnt, int64_t& e0, int64_t& e1) {
+  while (t.e >= t.e_end && t.w + 1 < a.nwin) {
+    ++t.w;
+    const int64_t sg = pc.seg0 + (int64_t)t.w * a.nblk;
+    t.e = __ldg(a.offsets + sg);
+    t.e_end = __ldg(a.offsets + sg + 1);
   }
-  int64_t s2 = w.seg + 1;
-  const int64_t lim = w.seg < 0 ? 0 : min64(w.seg + 5, a.nseg);
-  while (s2 < lim && a.offsets[s2 + 1] <= w.e) ++s2;
-  w.seg = (s2 < lim) ? s2 : segment_of(a.offsets, a.nseg, w.e);
-  const int64_t p_end = min64((int64_t)a.offsets[w.seg + 1], w.c_end);
-  if (p_end <= w.e) {
-    *bad = true;
-    return false;
-  }
-  pc.e0 = w.e;
-  pc.e1 = p_end;
-  w.e = p_end;
-  pc.c = (int32_t)(w.seg % a.nblk);
-  const int64_t bg = w.seg / a.nblk / a.nwin;
-  pc.g = (int32_t)(bg % a.G);
-  pc.b = bg / a.G;
-  return true;
+  e0 = t.e;
+  e1 = min64(t.e + kEnt, t.e_end);
+  t.e = e1;
 }
 }  // namespace
 
@@ -223,19 +236,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   auto W = [&](int id, int64_t k) {
     return mbar_wait(bar + id, (uint32_t)(k & 1), abort_flag, err);
   };
-  auto ntiles_of = [](const Piece& pc) { return (pc.e1 - pc.e0 + kEnt - 1) / kEnt; };
-
   PieceWalk wk;
-  walk_start(wk, a);
+  walk_start(wk);
   Piece pc;
-  bool bad = false;
+  TileWalk tw;
+  // lists with fewer entries than the sizes imply (a malformed selection): the
+  // dq slot sums would read pieces nobody wrote
+  if (blockIdx.x == 0 && tid == 0 && (int64_t)a.offsets[a.nseg] != a.total)
+    report(err, MSA_DEVERR_BAD_ENTRY);
 
   if (warp == 0) {
     // ---------------- K, V of every piece by TMA ----------------
     if (lane == 0) {
       prefetch_tensormap(&tm_k);
       prefetch_tensormap(&tm_v);
-      for (int64_t p = 0; walk_next(wk, a, pc, &bad); ++p) {
+      for (int64_t p = 0; walk_next(wk, a, pc, kEnt); ++p) {
         if (p > 0 && !W(TB_KV_EMPTY, p - 1)) break;
         mbar_arrive_expect_tx(bar + TB_KV_FULL, 65536u);
         for (int h = 0; h < 2; ++h) {
@@ -245,10 +260,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                       pc.g, (int32_t)pc.b);
         }
       }
-      if (bad) {
-        report(err, MSA_DEVERR_BAD_ENTRY);
-        *abort_flag = 1;
-      }
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
@@ -257,9 +268,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       bool ok = true;
       const uint32_t ka = smem_u32(base + kTcOffK), va = smem_u32(base + kTcOffV);
       const uint32_t dsa = smem_u32(base + kTcOffDS);
-      for (; ok && walk_next(wk, a, pc, &bad); ++p) {
+      for (; ok && walk_next(wk, a, pc, kEnt); ++p) {
         if (!W(TB_KV_FULL, p)) { ok = false; break; }
-        const int64_t nt = ntiles_of(pc);
+        const int64_t nt = pc.nt;
         // S^T(n) = K Q(n)^T into [0,128): for the first tile of a piece here, for
         // the others right after dQ(n-1) (it only needs P^T(n-1) consumed)
         auto issue_s = [&](int64_t nn) {
@@ -331,8 +342,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int ch = gt & 15;
     int64_t n = 0;
     bool ok = true;
-    for (int64_t p = 0; ok && walk_next(wk, a, pc, &bad); ++p) {
-      const int64_t nt = ntiles_of(pc);
+    for (int64_t p = 0; ok && walk_next(wk, a, pc, kEnt); ++p) {
+      const int64_t nt = pc.nt;
+      tiles_start(tw);
       const __nv_bfloat16* qb = a.q + pc.b * a.qs_b + (int64_t)(pc.g * R) * a.qs_h + ch * 8;
       const __nv_bfloat16* db = a.dout + pc.b * a.ds_b + (int64_t)(pc.g * R) * a.ds_h + ch * 8;
       for (int64_t t = 0; t < nt; ++t, ++n) {
@@ -340,13 +352,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (n >= 2 && !W(TB_QDO_EMPTY0 + buf, (n >> 1) - 1)) { ok = false; break; }
         uint8_t* sq = base + kTcOffQ + buf * 32768;
         uint8_t* sd = base + kTcOffDO + buf * 32768;
-        const int64_t et = pc.e0 + t * kEnt;
+        int64_t et, te;
+        tiles_next(tw, a, pc, kEnt, et, te);
 #pragma unroll 4
         for (int it = 0; it < 16; ++it) {
           const int row = it * 8 + (gt >> 4);
           const int64_t ei = et + row / R;
-          const int32_t ent = ei < pc.e1 ? __ldg(a.entries + ei) : -1;
-          const bool v = ent >= 0;
+          const int32_t ent = ei < te ? __ldg(a.entries + ei) : -1;
+          const bool v = ent >= 0 && (int64_t)(ent >> 4) < a.n_q;
           const int64_t qi = v ? (int64_t)(ent >> 4) : 0;
           const int64_t hoff = (int64_t)(row % R);
           const uint32_t off = (uint32_t)((ch >> 3) * 16384 + row * 128 + (((ch & 7) ^ (row & 7)) << 4));
@@ -370,16 +383,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     uint8_t* ds = base + kTcOffDS;
     int64_t n = 0;
     bool ok = true;
-    for (int64_t p = 0; ok && walk_next(wk, a, pc, &bad); ++p) {
-      const int64_t nt = ntiles_of(pc);
+    for (int64_t p = 0; ok && walk_next(wk, a, pc, kEnt); ++p) {
+      const int64_t nt = pc.nt;
+      tiles_start(tw);
       const int64_t key_abs = (int64_t)pc.c * kBlock + key;
       for (int64_t t = 0; t < nt; ++t, ++n) {
         // this thread's row (row = key index) data for the tile
-        const int64_t ei = pc.e0 + t * kEnt + key / R;
-        const int32_t ent = ei < pc.e1 ? __ldg(a.entries + ei) : -1;
+        int64_t et, te;
+        tiles_next(tw, a, pc, kEnt, et, te);
+        const int64_t ei = et + key / R;
+        const int32_t ent = ei < te ? __ldg(a.entries + ei) : -1;
         int32_t trow = -1;
         float lse_r = 0.f, d_r = 0.f;
-        if (ent >= 0) {
+        if (ent >= 0 && (int64_t)(ent >> 4) < a.n_q) {
           const int64_t qi = (int64_t)(ent >> 4);
           const int64_t mrow = (pc.b * a.n_q + qi) * a.H + pc.g * R + (key % R);
           trow = (int32_t)(a.q_pos0 + qi);
@@ -444,13 +460,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     int64_t n = 0;
     bool ok = true;
-    for (int64_t p = 0; ok && walk_next(wk, a, pc, &bad); ++p) {
-      const int64_t nt = ntiles_of(pc);
+    for (int64_t p = 0; ok && walk_next(wk, a, pc, kEnt); ++p) {
+      const int64_t nt = pc.nt;
+      tiles_start(tw);
       for (int64_t t = 0; t < nt; ++t, ++n) {
-        const int64_t ei = pc.e0 + t * kEnt + row / R;
-        const int32_t ent = ei < pc.e1 ? __ldg(a.entries + ei) : -1;
+        int64_t et, te;
+        tiles_next(tw, a, pc, kEnt, et, te);
+        const int64_t ei = et + row / R;
+        const int32_t ent = ei < te ? __ldg(a.entries + ei) : -1;
         float* dst = nullptr;
-        if (ent >= 0) {
+        if (ent >= 0 && (int64_t)(ent >> 4) < a.n_q) {
           const int64_t prow = ((pc.b * a.n_q + (ent >> 4)) * a.G + pc.g) * (int64_t)kTopK * R +
                                (int64_t)(ent & 15) * R + (row % R);
           dst = a.part_dq + prow * kHeadDim;
@@ -487,12 +506,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               uint32_t r[32];
               tmem_ld_32x32b_x32(tmem + lane_base + 256 + 128 * which + 32 * cc, r);
               tmem_ld_wait();
-              if (live) {
+              if (live) {                // this CTA owns the block: plain stores
 #pragma unroll
                 for (int x = 0; x < 8; ++x)
-                  atomicAdd(reinterpret_cast<float4*>(outp + kb + 32 * cc + 4 * x),
-                            make_float4(f * u2f(r[4 * x]), f * u2f(r[4 * x + 1]),
-                                        f * u2f(r[4 * x + 2]), f * u2f(r[4 * x + 3])));
+                  *reinterpret_cast<float4*>(outp + kb + 32 * cc + 4 * x) =
+                      make_float4(f * u2f(r[4 * x]), f * u2f(r[4 * x + 1]),
+                                  f * u2f(r[4 * x + 2]), f * u2f(r[4 * x + 3]));
               }
             }
           }
@@ -596,13 +615,9 @@ cudaError_t launch_sparse_attn_bwd(const CUtensorMap& tm_k, const CUtensorMap& t
   a.nwin = nwin;
   a.scale = scale;
   a.err = err;
-  // equal runs of entries, whole 128-row tiles each, about 8 per SM
-  const int64_t ent_per_tile = 128 / R;
-  const int64_t tiles = (total_entries + ent_per_tile - 1) / ent_per_tile;
-  const int64_t tiles_per_chunk = max64(4, (tiles + 8LL * sms - 1) / (8LL * sms));
-  a.chunk_entries = tiles_per_chunk * ent_per_tile;
-  const int64_t nchunks = (total_entries + a.chunk_entries - 1) / a.chunk_entries;
-  const int grid = (int)min64(nchunks, sms);
+  // one item per (batch, group, KV block); at most one CTA per SM
+  a.nitems = batch * G * (int64_t)nblk;
+  const int grid = total_entries > 0 ? (int)min64(a.nitems, sms) : 0;
   if (grid > 0) {
     switch (R) {
       case 1: e = launch_bwd_tc_r<1>(tm_k, tm_v, a, grid, st); break;

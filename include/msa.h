@@ -33,8 +33,7 @@
  *     that detects a problem at run time (an out-of-range block id, a wait
  *     that ran past its time limit) stores an MSA_DEVERR_* code there and
  *     returns early.  Nothing traps.
- *   - Results are deterministic: bit-identical from run to run (except dk
- *     and dv of msa_sparse_attn_bwd, summed with atomic adds).
+ *   - Results are deterministic: bit-identical from run to run.
  *   - Fixed sizes: block B_k = 128 tokens, top-k = 16 blocks (own included),
  *     head_dim = 128, d_idx in {64, 128}.
  *   - Layouts are given as [outer, ..., inner]; the innermost dimension is
@@ -284,8 +283,10 @@ MSA_API msa_status msa_merge_partials_compact(const msa_dims* dims, const int32_
  *   dq          [B, n_q, h_q, 128] fp32, contiguous
  *   dk, dv      [B, h_kv, n_kv, 128] fp32, contiguous; zeroed by the call
  * Blocks and keys that no query selected get zero gradients.  dq is summed in
- * slot order (deterministic); a KV block whose queries span several work
- * chunks sums their parts of dk, dv by atomic adds (order not fixed). */
+ * slot order; each KV block's dk and dv are accumulated by the one block of
+ * threads that owns the block (all its query windows) and stored once, so all
+ * three are bit-identical from run to run.  Lists with fewer entries than the
+ * sizes imply set MSA_DEVERR_BAD_ENTRY. */
 MSA_API msa_status msa_sparse_attn_bwd(const msa_dims* dims, msa_tensor q, msa_tensor k,
                                        msa_tensor v, msa_tensor o, msa_tensor d_o,
                                        const float* lse, const int32_t* blk_offsets,
