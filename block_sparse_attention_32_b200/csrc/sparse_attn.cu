@@ -34,10 +34,11 @@
 //                             of an entry (both 64-column panels; a 5-D view
 //                             of q), otherwise 16-byte cp.async by all four
 //                             warps
-//   warps 8-15  softmax:      two warpgroups in ping-pong, warpgroup h on
-//                             the chunks n % 2 == h (S buffer h); thread =
-//                             row: the row maximum over the 128 keys, then
-//                             P = bf16(e^{s-m}) back into the first 64
+//   warps 8-15  softmax:      two warpgroups, one per half of the keys; each
+//                             holds its 64 S values of a row in registers,
+//                             the halves exchange row maxima (and whether to
+//                             go on) at a named barrier per quarter, and
+//                             P = bf16(e^{s-m}) goes back into the first 64
 //                             columns of the S buffer in TMEM (the A operand
 //                             of O = P V)
 //   warps 16-19 epilogue:     O from TMEM half a row at a time, then the
@@ -91,8 +92,10 @@ constexpr int kOffV = 32768;           // 32768: [V lo | V hi]
 constexpr int kOffQP = 65536;          // kQRing x 32768: Q tile, then P
 constexpr int kStageRow = 272;                           // staged half row (256 B + pad)
 constexpr int kOffStage = kOffQP + kQRing * 32768;       // 128 staged rows
-constexpr int kOffML = kOffStage + 128 * kStageRow;      // [2 slots][128] float2 (m, l)
-constexpr int kOffDesc = kOffML + 2048;                  // kDescRing descriptors
+constexpr int kOffML = kOffStage + 128 * kStageRow;      // [2 slots][2 halves][128] float2 (m, l)
+constexpr int kOffMX = kOffML + 4096;                    // [2][2 halves][128] float row maxima
+constexpr int kOffVerdict = kOffMX + 2048;               // [2][2 halves][4 quarters] int
+constexpr int kOffDesc = kOffVerdict + 64;               // kDescRing descriptors
 constexpr int kOffBar = kOffDesc + kDescRing * (int)sizeof(ChunkDesc);
 constexpr int kNumBars = 4 + 3 * kQRing + 6 + 2 * kDescRing + 2 + 1;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;         // TMEM base, abort flag
@@ -156,6 +159,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint64_t* bar = reinterpret_cast<uint64_t*>(base + kOffBar);
   float2* ml_s = reinterpret_cast<float2*>(base + kOffML);
   ChunkDesc* desc = reinterpret_cast<ChunkDesc*>(base + kOffDesc);
+  float* mx_x = reinterpret_cast<float*>(base + kOffMX);
+  int* verdict = reinterpret_cast<int*>(base + kOffVerdict);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(base + kOffMisc + 4);
 
@@ -168,7 +173,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     for (int i = 0; i < kQRing; ++i) {
       mbar_init(bar + BAR_Q_FULL + i, kTmaGather ? 1 : 128);
       mbar_init(bar + BAR_QP_EMPTY + i, 1);
-      mbar_init(bar + BAR_P_FULL + i, 128);       // the chunk's softmax warpgroup
+      mbar_init(bar + BAR_P_FULL + i, 256);       // both softmax warpgroups
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar + BAR_S_FULL + i, 1);
@@ -277,15 +282,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           if (pos < e1) seg = warp_find_segment(a.blk_offsets, seg + 1, a.n_seg, pos, lane);
         }
       }
-      // end markers in two consecutive slots: the softmax warpgroups each look
-      // at every other chunk, so each must find one
-      for (int k = 0; ok && k < 2; ++k) {
-        if (!claim(chunk)) break;
+      if (ok && claim(chunk)) {          // end marker
         if (lane == 0) {
           desc[chunk % kDescRing].cnt = -1;
           mbar_arrive(bar + BAR_D_FULL + (int)(chunk % kDescRing));
         }
-        ++chunk;
       }
     } else if (warp == 1) {
       // ---------------- MMA issuer ----------------
@@ -296,6 +297,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (lane == 0) {
         int64_t pn = -1, pp = -1, v_ready = -1, last_s_piece = -1;
         bool plast = false, ok = true;
+        // shared-memory descriptors of the operands' first slices
+        const uint64_t kdesc0 = smem_desc_sw128(smem_u32(base + kOffK), 16, 1024);
+        const uint64_t vdesc0 = smem_desc_sw128(smem_u32(base + kOffV), 16384, 1024);
+        const uint64_t qdesc_ring0 =
+            smem_desc_sw128(smem_u32(base + kOffQP), 16, kTmaGather ? 2048 : 1024);
         auto issue_pv = [&](int64_t n, int64_t p, bool last) {
           if (p != v_ready) {
             if (!Wuse(BAR_V_FULL, 1, p)) return false;
@@ -306,12 +312,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           if (!Wfree(BAR_O_EMPTY, 2, n)) return false;
           const int ob = (int)(n & 1);
           tc_fence_after();
-          const uint32_t va = smem_u32(base + kOffV);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
             umma_bf16_ts(tmem + 256 + ob * 128, tmem + ob * 128 + kk * 8,
-                         smem_desc_sw128(va + kk * 2048, 16384, 1024), kIdescPV,
-                         kk > 0 ? 1u : 0u);
+                         vdesc0 + (uint64_t)((kk * 2048) >> 4), kIdescPV, kk > 0 ? 1u : 0u);
           umma_commit(bar + BAR_O_FULL + ob);
           if (last) umma_commit(bar + BAR_V_EMPTY);
           return true;
@@ -332,16 +336,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           if (n >= 2 && !Wuse(BAR_O_FULL, 2, n - 2)) { ok = false; break; }
           if (!Wuse(BAR_Q_FULL, kQRing, n)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t qa = smem_u32(base + kOffQP + qb * 32768);
-          const uint32_t ka = smem_u32(base + kOffK);
+          const uint64_t qdesc0 = qdesc_ring0 + (uint64_t)((qb * 32768) >> 4);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
             // K: [panel][128 rows][128 B] (8-row groups 1024 B apart); Q for R >= 8:
-            // [8-row group][panel][8 rows][128 B] (groups 2048 B apart), else as K
+            // [8-row group][panel][8 rows][128 B] (groups 2048 B apart), else as K.
+            // A descriptor's low 14 bits hold the address / 16, so the step to
+            // the kk-th 16-column slice is a plain add.
             const uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32;
             const uint32_t qoff = kTmaGather ? (kk >> 2) * 1024 + (kk & 3) * 32 : koff;
-            umma_bf16(tmem + sb * 128, smem_desc_sw128(qa + qoff, 16, kTmaGather ? 2048 : 1024),
-                      smem_desc_sw128(ka + koff, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
+            umma_bf16(tmem + sb * 128, qdesc0 + (uint64_t)(qoff >> 4),
+                      kdesc0 + (uint64_t)(koff >> 4), kIdescQK, kk > 0 ? 1u : 0u);
           }
           umma_commit(bar + BAR_S_FULL + sb);
           umma_commit(bar + BAR_QP_EMPTY + qb);
@@ -479,60 +484,66 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
   } else if (warp < 16) {
     // ---------------- softmax: S -> P, (m, l) ----------------
-    // Ping-pong: warpgroup h takes the chunks n with n % 2 == h, whose S lives
-    // in TMEM buffer h, so the two warpgroups work on neighbouring chunks at
-    // once and never wait on each other.  Thread = row = TMEM lane: a first
-    // pass over the row's 128 keys takes the maximum, a second computes
-    // e^{s-m} 32 keys at a time and writes P as bf16 into the first 64
-    // columns of the same buffer (keys 32j.. -> columns 16j..; columns are
-    // overwritten only after they were read), the A operand of O = P V.
+    // Warpgroup h (0, 1) takes keys 64h .. 64h+63 of every row of every chunk
+    // (thread = row = TMEM lane), so a chunk's softmax takes half the time of
+    // a whole row's.  Per chunk every wait comes first; then the two warps of
+    // a quarter (one per half) meet once at a named barrier, exchanging their
+    // row maxima and their verdict (all waits done / end of work), and both
+    // go on or both leave on the exchanged verdicts: after a timeout neither
+    // half can be left waiting at the barrier for the other.
     setmaxnreg_inc<kRegsSoftmax>();
     const int h = (warp >> 2) - 2;
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     const float scale_log2 = a.scale * 1.4426950408889634f;
-    for (int64_t n = h;; n += 2) {
-      if (!WuseW(BAR_D_FULL, kDescRing, n)) break;
-      const ChunkDesc& d = desc[n % kDescRing];
-      if (d.cnt < 0) break;
+    const uint64_t scale2 = pack_f32x2(__float_as_uint(scale_log2), __float_as_uint(scale_log2));
+    for (int64_t n = 0;; ++n) {
       const int qb = (int)(n % kQRing), sb = (int)(n & 1);
-      const int e = d.ent[row / R];
-      const int32_t c = d.c;
-      if (!WuseW(BAR_S_FULL, 2, n)) break;
-      tc_fence_after();
+      bool ok = WuseW(BAR_D_FULL, kDescRing, n);
+      const ChunkDesc& d = desc[n % kDescRing];
+      const bool end = ok && d.cnt < 0;
+      if (ok && !end) ok = WuseW(BAR_S_FULL, 2, n);
+      // the (m, l) slot sb is free once the epilogue of n-2 has read it
+      if (ok && !end) ok = WfreeW(BAR_ML_EMPTY, 2, n);
+      const bool work = ok && !end;
       const uint32_t s_addr = tmem + lane_base + sb * 128;
-      const int64_t qi = (int64_t)(e >> 4);
-      bool valid = (e >= 0) && (qi < a.n_q);
-      int lim = 127;
-      if (valid) {
-        const int64_t rel = a.q_pos0 + qi - (int64_t)c * kBlock;
-        if (rel < 0) {
-          valid = false;
-          report(err, MSA_DEVERR_BAD_ENTRY);
-        } else if (rel < 127) {
-          lim = (int)rel;
+      bool valid = false;
+      int lim = -1;
+      uint32_t r0[32], r1[32];
+      float mloc = -INFINITY;
+      bool masked = false;
+      if (work) {
+        tc_fence_after();
+        tmem_ld_32x32b_x32(s_addr + 64 * h, r0);
+        tmem_ld_32x32b_x32(s_addr + 64 * h + 32, r1);
+        const int e = d.ent[row / R];
+        const int64_t qi = (int64_t)(e >> 4);
+        valid = (e >= 0) && (qi < a.n_q);
+        lim = 127;
+        if (valid) {
+          const int64_t rel = a.q_pos0 + qi - (int64_t)d.c * kBlock;
+          if (rel < 0) {
+            valid = false;
+            if (h == 0) report(err, MSA_DEVERR_BAD_ENTRY);
+          } else if (rel < 127) {
+            lim = (int)rel;
+          }
         }
-      }
-      if (!valid) lim = -1;                   // every weight of the row is zero
-      // only rows of the query's own block mask keys (past the query); a warp
-      // with no such row skips every per-key compare
-      const bool masked = __any_sync(0xffffffffu, lim >= 0 && lim < 127);
-      float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll 1
-      for (int hh = 0; hh < 2; ++hh) {
-        uint32_t r0[32], r1[32];
-        tmem_ld_32x32b_x32(s_addr + 64 * hh, r0);
-        tmem_ld_32x32b_x32(s_addr + 64 * hh + 32, r1);
+        if (!valid) lim = -1;                 // every weight of the row is zero
+        // only rows of the query's own block mask keys (past the query); a warp
+        // with no such row skips every per-key compare
+        masked = __any_sync(0xffffffffu, lim >= 0 && lim < 127);
         tmem_ld_wait();
-        const int k0 = 64 * hh;
+        const int k0 = 64 * h;
+        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
         if (!masked) {
 #pragma unroll
-          for (int x = 0; x < 32; x += 2) {
-            m4[0] = fmaxf(m4[0], u2f(r0[x]));
-            m4[1] = fmaxf(m4[1], u2f(r0[x + 1]));
-            m4[2] = fmaxf(m4[2], u2f(r1[x]));
-            m4[3] = fmaxf(m4[3], u2f(r1[x + 1]));
+          for (int x = 0; x < 32; x += 4) {
+            m4[0] = fmax3f(m4[0], u2f(r0[x]), u2f(r0[x + 1]));
+            m4[1] = fmax3f(m4[1], u2f(r0[x + 2]), u2f(r0[x + 3]));
+            m4[2] = fmax3f(m4[2], u2f(r1[x]), u2f(r1[x + 1]));
+            m4[3] = fmax3f(m4[3], u2f(r1[x + 2]), u2f(r1[x + 3]));
           }
         } else {
 #pragma unroll
@@ -543,52 +554,63 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             m4[3] = fmaxf(m4[3], k0 + 33 + x <= lim ? u2f(r1[x + 1]) : -INFINITY);
           }
         }
+        mloc = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
       }
-      float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+      // exchange with the other half's warp of this quarter (by parity: the
+      // partner reads a slot before it is written again two chunks later)
+      float* mxn = mx_x + (int)(n & 1) * 256;
+      mxn[h * 128 + row] = mloc;
+      if (lane == 0) verdict[((int)(n & 1) * 2 + h) * 4 + quarter] = (ok ? 1 : 0) | (end ? 2 : 0);
+      tc_fence_before();                       // this half's S reads precede the other's P writes
+      named_bar_sync(1 + quarter, 64);
+      tc_fence_after();
+      const int pv = verdict[((int)(n & 1) * 2 + (1 - h)) * 4 + quarter];
+      if (!work || !(pv & 1) || (pv & 2)) break;
+      float mx = fmaxf(mloc, mxn[(1 - h) * 128 + row]);
       if (!valid) mx = 0.f;
       // e^{s-m} = 2^{s log2(e) scale - m log2(e) scale}; a row with no valid
       // key gets weight 2^-inf = 0 everywhere
       const float mneg = valid ? -mx * scale_log2 : -INFINITY;
-      float lsum[4] = {0.f, 0.f, 0.f, 0.f};
-      // P is rounded to bf16 for the P V product; l sums the fp32 weights.
+      const uint64_t mneg2 = pack_f32x2(__float_as_uint(mneg), __float_as_uint(mneg));
+      // two packed (f32x2) partial sums of the weights
+      uint64_t lsum2[2] = {0ull, 0ull};
+      // keys 32j..32j+31 -> columns 16j..16j+15 of this S buffer (already
+      // read).  P is rounded to bf16 for the P V product; l sums the fp32
+      // weights.  The exponents of a pair of keys are one packed FMA, their
+      // weights one packed add into the row sum.
       auto exp_pack_store = [&](const uint32_t (&r)[32], int j, bool mask) {
         uint32_t w[16];
 #pragma unroll
         for (int x = 0; x < 16; ++x) {
-          float p0 = ex2_approx(fmaf(u2f(r[2 * x]), scale_log2, mneg));
-          float p1 = ex2_approx(fmaf(u2f(r[2 * x + 1]), scale_log2, mneg));
+          float x0, x1;
+          unpack_f32x2(fma_f32x2(pack_f32x2(r[2 * x], r[2 * x + 1]), scale2, mneg2), x0, x1);
+          float p0 = ex2_approx(x0);
+          float p1 = ex2_approx(x1);
           if (mask) {
             const int kk = j * 32 + 2 * x;
             p0 = (kk <= lim) ? p0 : 0.f;
             p1 = (kk + 1 <= lim) ? p1 : 0.f;
           }
-          lsum[x & 3] += p0 + p1;
+          lsum2[x & 1] =
+              add_f32x2(lsum2[x & 1], pack_f32x2(__float_as_uint(p0), __float_as_uint(p1)));
           w[x] = pack_bf16x2(p0, p1);
         }
         tmem_st_32x32b_x16(s_addr + j * 16, w);
       };
-      // keys 32j .. 32j+31: the next block of S is loaded while this one is
-      // exponentiated (a load waits for every earlier load of the thread)
-      uint32_t ra[32], rb[32];
-      tmem_ld_32x32b_x32(s_addr, ra);
-      tmem_ld_wait();
-#pragma unroll
-      for (int j = 0; j < 4; j += 2) {
-        tmem_ld_32x32b_x32(s_addr + 32 * (j + 1), rb);
-        if (!masked) exp_pack_store(ra, j, false); else exp_pack_store(ra, j, true);
-        tmem_ld_wait();
-        if (j + 2 < 4) tmem_ld_32x32b_x32(s_addr + 32 * (j + 2), ra);
-        if (!masked) exp_pack_store(rb, j + 1, false); else exp_pack_store(rb, j + 1, true);
-        if (j + 2 < 4) tmem_ld_wait();
+      if (!masked) {
+        exp_pack_store(r0, 2 * h, false);
+        exp_pack_store(r1, 2 * h + 1, false);
+      } else {
+        exp_pack_store(r0, 2 * h, true);
+        exp_pack_store(r1, 2 * h + 1, true);
       }
       tmem_st_wait();
-      const float l = (lsum[0] + lsum[1]) + (lsum[2] + lsum[3]);
-      // (m, l) slot sb is free once the epilogue of n-2 has read it; P V(n)
-      // is issued only after the warpgroup arrives
-      if (!WfreeW(BAR_ML_EMPTY, 2, n)) break;
-      ml_s[sb * 128 + row] = make_float2(mx * a.scale, l);
+      float la, lb, lc, ld;
+      unpack_f32x2(lsum2[0], la, lb);
+      unpack_f32x2(lsum2[1], lc, ld);
+      ml_s[(sb * 2 + h) * 128 + row] = make_float2(mx * a.scale, (la + lb) + (lc + ld));
       tc_fence_before();
-      mbar_arrive(bar + BAR_P_FULL + qb);
+      mbar_arrive(bar + BAR_P_FULL + qb);      // P V(n) is issued once both halves arrive
     }
   } else {
     // ---------------- epilogue: O -> pieces ----------------
@@ -616,7 +638,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (!WuseW(BAR_O_FULL, 2, n)) break;
       if (!WuseW(BAR_P_FULL, kQRing, n)) break;  // acquire the softmax's (m, l)
       tc_fence_after();
-      const float2 ml = ml_s[ob * 128 + row];
+      const float2 ml0 = ml_s[(ob * 2) * 128 + row];
+      const float2 ml1 = ml_s[(ob * 2 + 1) * 128 + row];
       mbar_arrive(bar + BAR_ML_EMPTY + ob);      // (m, l) slot ob is free
       const int hr = row % R;
       const int64_t qi = (int64_t)(e >> 4);
@@ -624,8 +647,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       // piece row of (b, qi, g, slot, hr): the R head rows of one entry are adjacent
       const int64_t pidx =
           valid ? ((((int64_t)b * a.n_q + qi) * a.G + g) * kTopK + (e & 15)) * R + hr : 0;
-      const float l_sum = ml.y;
-      if (valid) *reinterpret_cast<float2*>(a.part_ml + pidx * 2) = make_float2(ml.x, l_sum);
+      const float l_sum = ml0.y + ml1.y;
+      if (valid) *reinterpret_cast<float2*>(a.part_ml + pidx * 2) = make_float2(ml0.x, l_sum);
       // compact pieces: acc / l (l >= 1 on a valid row: the row maximum's weight is 1)
       const float inv_l = (kCompact && valid && l_sum > 0.f) ? 1.0f / l_sum : 0.f;
       const uint32_t o_addr = tmem + lane_base + 256 + ob * 128;
