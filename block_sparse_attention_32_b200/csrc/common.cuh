@@ -176,6 +176,16 @@ __device__ __forceinline__ void tma_store_2d_hint(const CUtensorMap* map, const 
       : "memory");
 }
 
+__device__ __forceinline__ void tma_store_3d_hint(const CUtensorMap* map, const void* src,
+                                                  int32_t x, int32_t y, int32_t z,
+                                                  uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group.L2::cache_hint [%0, {%2, %3, %4}], "
+      "[%1], %5;" ::"l"(reinterpret_cast<uint64_t>(map)),
+      "r"(smem_u32(src)), "r"(x), "r"(y), "r"(z), "l"(policy)
+      : "memory");
+}
+
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }

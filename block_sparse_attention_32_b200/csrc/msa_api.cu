@@ -158,34 +158,24 @@ msa_status make_map(CUtensorMap* map, const void* ptr, uint64_t inner, uint64_t 
   return r == CUDA_SUCCESS ? MSA_OK : MSA_ERR_CUDA;
 }
 
-// 2-D fp32 map over rows of 128 floats (512-byte rows): dims {128, rows}, box
-// {32, box_rows}, 128-byte swizzle (the layout the writer stages in shared memory)
-msa_status make_map_rows_f32(CUtensorMap* map, void* ptr, uint64_t rows, uint32_t box_rows) {
+// 3-D map over the pieces' rows of 128 values (fp32: 512-byte rows; bf16:
+// 256-byte rows) seen as {128 bytes of a row, rows, 128-byte panels of a row},
+// box {128 bytes, box_rows, panels}: one store writes box_rows consecutive
+// rows (an entry's heads) across `panels` panels, from shared memory staged
+// [panel][row][128 B] with the 128-byte swizzle.
+msa_status make_map_piece_rows(CUtensorMap* map, void* ptr, uint64_t rows, bool bf16,
+                               uint32_t box_rows, uint32_t panels) {
   auto fn = encode_fn();
   if (fn == nullptr) return MSA_ERR_CUDA;
-  cuuint64_t dims[2] = {128, rows};
-  cuuint64_t strides[1] = {128 * sizeof(float)};
-  cuuint32_t box[2] = {32, box_rows};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, ptr, dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                  CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? MSA_OK : MSA_ERR_CUDA;
-}
-
-// 2-D bf16 map over rows of 128 values (256-byte rows): dims {128, rows}, box
-// {64, box_rows}, 128-byte swizzle (compact pieces, staged by the writer in
-// that layout)
-msa_status make_map_rows_bf16(CUtensorMap* map, void* ptr, uint64_t rows, uint32_t box_rows) {
-  auto fn = encode_fn();
-  if (fn == nullptr) return MSA_ERR_CUDA;
-  cuuint64_t dims[2] = {128, rows};
-  cuuint64_t strides[1] = {128 * 2};
-  cuuint32_t box[2] = {64, box_rows};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ptr, dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                  CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  const uint64_t row_bytes = bf16 ? 256 : 512;
+  cuuint64_t dims[3] = {bf16 ? 64u : 32u, rows, row_bytes / 128};
+  cuuint64_t strides[2] = {row_bytes, 128};
+  cuuint32_t box[3] = {bf16 ? 64u : 32u, box_rows, panels};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                  3, ptr, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? MSA_OK : MSA_ERR_CUDA;
 }
 
@@ -400,8 +390,8 @@ msa_status sparse_attn_fwd(const msa_dims* d, msa_tensor q, msa_tensor k, msa_te
     if ((s = make_map_q_groups(&tq, d, q)) != MSA_OK) return s;
     const int64_t rows = d->batch * d->n_q * d->h_kv * MSA_TOPK_BLOCKS * R;
     if (rows >= (int64_t(1) << 31)) return MSA_ERR_UNSUPPORTED;
-    s = compact ? make_map_rows_bf16(&to, part_acc, (uint64_t)rows, (uint32_t)R)
-                : make_map_rows_f32(&to, part_acc, (uint64_t)rows, (uint32_t)R);
+    // fp32: an entry's half rows (2 panels) per store; bf16: its whole rows
+    s = make_map_piece_rows(&to, part_acc, (uint64_t)rows, compact, (uint32_t)R, 2);
     if (s != MSA_OK) return s;
   }
   return from_cuda(msa::launch_sparse_attn(

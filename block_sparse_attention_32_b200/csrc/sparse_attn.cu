@@ -618,10 +618,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
-    // R >= 8: each warp stages half rows in two 32-column panels (32 rows x
-    // 128 B, 128-byte swizzle) and the first lane of each entry writes the
-    // entry's R rows with one TMA store per panel.  R < 8: half rows padded
-    // to 272 B, read back transposed, two half rows per store instruction.
+    // R >= 8: each warp stages its entries' rows as blocks [2 panels][R rows]
+    // [128 B] (128-byte swizzle; fp32: the two 32-column panels of a half row,
+    // compact: the row's two 64-column halves) and the first lane of each
+    // entry writes the block with one TMA store (a 3-D view of the pieces).
+    // R < 8: rows padded to 272 B, read back transposed, two half rows (fp32)
+    // or four (compact) per store instruction.
     constexpr bool kTmaStore = R >= 8;
     // pieces are read back only by the merge kernel: keep them from displacing Q rows in L2
     const uint64_t pol_st = l2_policy_evict_first();
@@ -673,18 +675,25 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             w[16 + x] = pack_bf16x2(u2f(r1[2 * x]) * inv_l, u2f(r1[2 * x + 1]) * inv_l);
           }
           if constexpr (kTmaStore) {
-            bulk_wait_read();                    // the previous stores have read the panel
-            __syncwarp();
+            // half `half` of the row is panel `half` of the entry's staging
+            // block [2 panels][R rows][128 B]; the block leaves by one store
+            if (half == 0) {
+              bulk_wait_read();                  // the previous stores have read the block
+              __syncwarp();
+            }
             const int sw = lane & 7;
+            uint8_t* mine = stage + (lane / R) * (2 * R * 128) + (lane % R) * 128;
 #pragma unroll
             for (int j = 0; j < 8; ++j)
-              *reinterpret_cast<uint4*>(stage + lane * 128 + ((j ^ sw) << 4)) =
+              *reinterpret_cast<uint4*>(mine + half * R * 128 + ((j ^ sw) << 4)) =
                   make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (valid && hr == 0)                // first row of an entry: R rows per store
-              tma_store_2d_hint(&tm_o, stage + lane * 128, half * 64, (int32_t)pidx, pol_st);
-            bulk_commit();
+            if (half == 1) {
+              fence_proxy_async_smem();
+              __syncwarp();
+              if (valid && hr == 0)              // first row of an entry: its R rows, both panels
+                tma_store_3d_hint(&tm_o, mine, 0, (int32_t)pidx, 0, pol_st);
+              bulk_commit();
+            }
           } else {
 #pragma unroll
             for (int x = 0; x < 8; ++x)
@@ -708,23 +717,23 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             __syncwarp();
           }
         } else if constexpr (kTmaStore) {
-          bulk_wait_read();                      // the previous stores have read the panels
+          // the half row's two 32-column panels into the entry's staging block
+          // [2 panels][R rows][128 B]; one store writes the entry's R half rows
+          bulk_wait_read();                      // the previous stores have read the block
           __syncwarp();
           const int sw = lane & 7;
+          uint8_t* mine = stage + (lane / R) * (2 * R * 128) + (lane % R) * 128;
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
-            *reinterpret_cast<uint4*>(stage + lane * 128 + ((j ^ sw) << 4)) =
+            *reinterpret_cast<uint4*>(mine + ((j ^ sw) << 4)) =
                 make_uint4(r0[4 * j], r0[4 * j + 1], r0[4 * j + 2], r0[4 * j + 3]);
-            *reinterpret_cast<uint4*>(stage + 4096 + lane * 128 + ((j ^ sw) << 4)) =
+            *reinterpret_cast<uint4*>(mine + R * 128 + ((j ^ sw) << 4)) =
                 make_uint4(r1[4 * j], r1[4 * j + 1], r1[4 * j + 2], r1[4 * j + 3]);
           }
           fence_proxy_async_smem();
           __syncwarp();
-          if (valid && hr == 0) {                // first row of an entry: R rows per store
-            tma_store_2d_hint(&tm_o, stage + lane * 128, half * 64, (int32_t)pidx, pol_st);
-            tma_store_2d_hint(&tm_o, stage + 4096 + lane * 128, half * 64 + 32,
-                              (int32_t)pidx, pol_st);
-          }
+          if (valid && hr == 0)                  // first row of an entry: its R half rows
+            tma_store_3d_hint(&tm_o, mine, 0, (int32_t)pidx, half * 2, pol_st);
           bulk_commit();
         } else {
 #pragma unroll
