@@ -94,8 +94,10 @@ def source_digest(paths):
     return h.hexdigest()
 
 
-def measured_traffic(kernel_files, record):
-    """DRAM bytes per launch from a committed ncu summary, or None when the
+def measured_traffic(kernel_files, record, units):
+    """DRAM bytes per launch from a committed ncu summary taken on a small case
+    of the same kernel: its bytes per unit (a list entry of the attention)
+    times the units one launch of this workload processes.  None when the
     kernel sources changed since the counters were taken."""
     path = os.path.join(ROOT, "profiles", record)
     try:
@@ -107,7 +109,7 @@ def measured_traffic(kernel_files, record):
     if kv.get("source_sha256", "").strip() != digest:
         return None
     try:
-        return float(kv["dram_bytes_per_launch"].strip())
+        return float(kv["dram_bytes_per_entry"].strip()) * units
     except (KeyError, ValueError):
         return None
 
@@ -376,7 +378,8 @@ def bench_recall(w, n_rows=64, reps=3):
     return out
 
 
-def attention_roofline(w, stage_mean, attn_flops, n_pieces, nbytes, peaks, peak_src):
+def attention_roofline(w, stage_mean, attn_flops, n_ent, n_pieces, nbytes, peaks, peak_src,
+                       compact=False):
     """Roofline of the KV-block-outer attention (A4) on the basis the scope
     table fixes: a dense bf16 contraction, so tensor-bound, achieved =
     selected-token FLOPs / its mean event time against the sustained bf16 peak
@@ -394,8 +397,9 @@ def attention_roofline(w, stage_mean, attn_flops, n_pieces, nbytes, peaks, peak_
     ach_m = attn_flops / secs_m / 1e12
     qo = float(w.batch * w.n_q * w.h_q * 128 * 2)
     algo = 2 * qo + float(n_pieces) * 65536
-    traffic = measured_traffic(["sparse_attn.cu", "common.cuh"],
-                               "sparse_attn_dram_traffic_prefill_128k.txt")
+    # counters of the fp32-piece kernel on the 8K profiling case, scaled by entries
+    traffic = None if compact else measured_traffic(
+        ["sparse_attn.cu", "common.cuh"], "sparse_attn_fwd_profile_8k_r8.md", n_ent)
     return {"bound": "tensor", "achieved": ach, "peak": sustained, "unit": "TFLOP/s",
             "frac": ach / sustained, "frac_of_burst": ach / burst,
             "peak_source": f"{peak_src} bf16_tflops_sustained",
@@ -418,7 +422,8 @@ def bench_compact(w, steps, warmup, peaks, peak_src):
                                                       compact=True)
     idx_flops, attn_flops, n_ent = work_counts(w)
     nbytes = bytes_model(w, n_ent, n_pieces, piece_bytes=264)
-    roof = attention_roofline(w, mean, attn_flops, n_pieces, nbytes, peaks, peak_src)
+    roof = attention_roofline(w, mean, attn_flops, n_ent, n_pieces, nbytes, peaks, peak_src,
+                              compact=True)
     roof["traffic"] = None
     roof["traffic_over_algorithmic"] = None
     ms = total_ms / steps
@@ -716,10 +721,11 @@ def main():
     burst = peaks.get("bf16_tflops", FALLBACK["bf16_tflops"])
     hbm = peaks.get("hbm_gbs", FALLBACK["hbm_gbs"])
     nbytes = bytes_model(w, n_ent, n_pieces)
-    attn_roof = attention_roofline(w, stage_mean, attn_flops, n_pieces, nbytes, peaks, peak_src)
+    attn_roof = attention_roofline(w, stage_mean, attn_flops, n_ent, n_pieces, nbytes, peaks,
+                                   peak_src)
     # dominant kernel: the longest stage.  Index scoring and the attention are
-    # dense bf16 contractions (tensor-bound by the algorithmic work, SURVEY-style
-    # FLOP counts); the other stages are HBM-bound on the bytes they must move.
+    # dense bf16 contractions (tensor-bound by the algorithmic work: the FLOPs
+    # of the selected tokens); the other stages are HBM-bound on the bytes they must move.
     dom = max(stage_mean, key=stage_mean.get)
     if dom == "attn":
         roof = dict(attn_roof)
