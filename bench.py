@@ -68,8 +68,9 @@ def bytes_model(w, n_entries, n_pieces_nonempty, piece_bytes=520):
 
     attention: per (query, block) entry the R gathered Q rows (256 B each) and
     the R pieces written (fp32: 512 B acc + 8 B (m, l); compact: 256 + 8); per selected (batch,
-    group, block) the 64 KB K/V tile once; the entry list.  merge: the pieces
-    read once, sel, and the bf16 output + lse written."""
+    group, block) the 64 KB K/V tile once; the entry list.  block lists: sel
+    read twice, the entries and their position map written.  merge: the pieces
+    read once, the position map, and the bf16 output + lse written."""
     B, G, R = w.batch, w.h_kv, w.h_q // w.h_kv
     t = w.q_pos0 + np.arange(w.n_q, dtype=np.int64)
     own = t // 128
@@ -78,7 +79,7 @@ def bytes_model(w, n_entries, n_pieces_nonempty, piece_bytes=520):
         "index": float(B * w.n_q * G * w.d_idx * 2 + B * w.h_kidx * w.n_kv * w.d_idx * 2
                        + 4 * B * G * own.sum()),
         "topk": float(4 * B * G * own[own >= 16].sum() + 64 * rows),
-        "block_lists": float(64 * rows * 2 + 4 * n_entries * 2),
+        "block_lists": float(64 * rows * 3 + 4 * n_entries * 2),
         "attn": float(n_entries * R * (256 + piece_bytes) + n_pieces_nonempty * 65536
                       + 4 * n_entries),
         "merge": float(n_entries * R * piece_bytes + 64 * rows + B * w.n_q * w.h_q * (256 + 4)),
@@ -189,15 +190,15 @@ def run_step(pipeline, capi, buf, inp, stages=None):
     if ev: ev[1].record()
     capi.msa_topk_blocks(d, buf.pooled, buf.pooled_stride, buf.sel, buf.dev_err)
     if ev: ev[2].record()
-    capi.msa_build_block_query_lists(d, buf.sel, buf.blk_offsets, buf.entries, buf.ws,
-                                     buf.dev_err)
+    capi.msa_build_block_query_lists(d, buf.sel, buf.blk_offsets, buf.entries, buf.entry_pos,
+                                     buf.ws, buf.dev_err)
     if ev: ev[3].record()
     fwd = capi.msa_sparse_attn_fwd_compact if buf.compact else capi.msa_sparse_attn_fwd
     merge = capi.msa_merge_partials_compact if buf.compact else capi.msa_merge_partials
     fwd(d, inp["q"], inp["k"], inp["v"], buf.blk_offsets, buf.entries, buf.part_ml, buf.part_acc,
         buf.dev_err)
     if ev: ev[4].record()
-    merge(d, buf.sel, buf.part_ml, buf.part_acc, buf.out, buf.lse, buf.dev_err)
+    merge(d, buf.entry_pos, buf.part_ml, buf.part_acc, buf.out, buf.lse, buf.dev_err)
     if ev: ev[5].record()
 
 

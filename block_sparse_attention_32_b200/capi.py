@@ -70,8 +70,8 @@ def load_library(path: str) -> ctypes.CDLL:
     L.msa_topk_blocks.argtypes = [_PD, _P, ctypes.c_int64, _P, _P, _P]
     L.msa_block_query_lists_workspace.argtypes = [_PD]
     L.msa_block_query_lists_workspace.restype = ctypes.c_size_t
-    L.msa_build_block_query_lists.argtypes = [_PD, _P, _P, _P, _P, ctypes.c_size_t, _P, _P]
-    L.msa_build_block_query_lists_noalloc.argtypes = [_PD, _P, _P, _P, _P, _P]
+    L.msa_build_block_query_lists.argtypes = [_PD, _P, _P, _P, _P, _P, ctypes.c_size_t, _P, _P]
+    L.msa_build_block_query_lists_noalloc.argtypes = [_PD, _P, _P, _P, _P, _P, _P]
     L.msa_sparse_attn_fwd.argtypes = [_PD, Tensor, Tensor, Tensor, _P, _P, _P, _P, _P, _P]
     L.msa_merge_partials.argtypes = [_PD, _P, _P, _P, _P, _P, _P, _P]
     L.msa_sparse_attn_fwd_compact.argtypes = [_PD, Tensor, Tensor, Tensor, _P, _P, _P, _P, _P,
@@ -184,20 +184,24 @@ def msa_topk_blocks(d: Dims, pooled, pooled_row_stride, sel, dev_err=None):
                                  _ptr(dev_err), _stream()))
 
 
-def msa_build_block_query_lists(d: Dims, sel, blk_offsets, entries, ws, dev_err=None):
+def msa_build_block_query_lists(d: Dims, sel, blk_offsets, entries, entry_pos, ws, dev_err=None):
+    """entry_pos (int32, the shape of sel) receives the position in entries of
+    each (b, g, query, slot), -1 for an empty slot."""
     nbytes = 0 if ws is None else ws.numel() * ws.element_size()
     _check("msa_build_block_query_lists",
            lib().msa_build_block_query_lists(ctypes.byref(d), _ptr(sel), _ptr(blk_offsets),
-                                             _ptr(entries), _ptr(ws), nbytes, _ptr(dev_err),
-                                             _stream()))
+                                             _ptr(entries), _ptr(entry_pos), _ptr(ws), nbytes,
+                                             _ptr(dev_err), _stream()))
 
 
-def msa_build_block_query_lists_noalloc(d: Dims, sel, blk_offsets, entries, dev_err=None):
+def msa_build_block_query_lists_noalloc(d: Dims, sel, blk_offsets, entries, entry_pos,
+                                        dev_err=None):
     """Same lists as msa_build_block_query_lists, with the library's built-in
     device scratch instead of a caller workspace (nothing is allocated)."""
     _check("msa_build_block_query_lists_noalloc",
            lib().msa_build_block_query_lists_noalloc(ctypes.byref(d), _ptr(sel), _ptr(blk_offsets),
-                                                     _ptr(entries), _ptr(dev_err), _stream()))
+                                                     _ptr(entries), _ptr(entry_pos),
+                                                     _ptr(dev_err), _stream()))
 
 
 def msa_sparse_attn_fwd(d: Dims, q, k, v, blk_offsets, entries, part_ml, part_acc, dev_err=None):
@@ -209,7 +213,7 @@ def msa_sparse_attn_fwd(d: Dims, q, k, v, blk_offsets, entries, part_ml, part_ac
 
 def msa_sparse_attn_fwd_compact(d: Dims, q, k, v, blk_offsets, entries, part_ml, part_acc16,
                                 dev_err=None):
-    """As msa_sparse_attn_fwd with compact pieces: part_acc16 bf16 [B,n_q,G,16,R,128]
+    """As msa_sparse_attn_fwd with compact pieces: part_acc16 bf16 [entries, R, 128]
     holds acc / l."""
     assert part_acc16.dtype == torch.bfloat16
     _check("msa_sparse_attn_fwd_compact",
@@ -219,10 +223,10 @@ def msa_sparse_attn_fwd_compact(d: Dims, q, k, v, blk_offsets, entries, part_ml,
                                              _stream()))
 
 
-def msa_merge_partials_compact(d: Dims, sel, part_ml, part_acc16, out, lse, dev_err=None):
+def msa_merge_partials_compact(d: Dims, entry_pos, part_ml, part_acc16, out, lse, dev_err=None):
     assert part_acc16.dtype == torch.bfloat16
     _check("msa_merge_partials_compact",
-           lib().msa_merge_partials_compact(ctypes.byref(d), _ptr(sel), _ptr(part_ml),
+           lib().msa_merge_partials_compact(ctypes.byref(d), _ptr(entry_pos), _ptr(part_ml),
                                             _ptr(part_acc16), _ptr(out), _ptr(lse),
                                             _ptr(dev_err), _stream()))
 
@@ -240,9 +244,10 @@ def msa_sparse_attn_bwd(d: Dims, q, k, v, o, d_o, lse, blk_offsets, entries, del
                                      _stream()))
 
 
-def msa_merge_partials(d: Dims, sel, part_ml, part_acc, out, lse, dev_err=None):
+def msa_merge_partials(d: Dims, entry_pos, part_ml, part_acc, out, lse, dev_err=None):
+    """Pieces in list order: slot s of (b, g, query) is at row entry_pos * R + r."""
     _check("msa_merge_partials",
-           lib().msa_merge_partials(ctypes.byref(d), _ptr(sel), _ptr(part_ml), _ptr(part_acc),
+           lib().msa_merge_partials(ctypes.byref(d), _ptr(entry_pos), _ptr(part_ml), _ptr(part_acc),
                                     _ptr(out), _ptr(lse), _ptr(dev_err), _stream()))
 
 

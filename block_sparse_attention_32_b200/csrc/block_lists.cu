@@ -19,7 +19,10 @@
 //   3. offsets: exclusive scan of the totals over all segments (chunk sums,
 //      scan of the chunk sums, chunk-local scans);
 //   4. scatter: per tile, queries in ascending order claim consecutive slots
-//      of each block's range, so the order never depends on timing.
+//      of each block's range, so the order never depends on timing; each
+//      (query, slot) also records the position it claimed (entry_pos, the
+//      shape of sel, -1 for an empty slot), which is where the attention
+//      writes that entry's piece and where the merge finds it.
 // Workspace: tile histograms [B*G, ntiles, nblk] + totals [B*G*nwin*nblk] +
 // chunk sums [ceil(B*G*nwin*nblk / 4096)], int32.  One query per row (decode) takes a
 // two-launch path that needs only the per-row counts.
@@ -219,7 +222,7 @@ __global__ void __launch_bounds__(32)
                        int32_t nblk, int32_t ntiles, int32_t tw, int32_t nwin,
                        const int32_t* __restrict__ tile_counts,
                        const int32_t* __restrict__ offsets, int32_t* __restrict__ entries,
-                       int64_t cap) {
+                       int32_t* __restrict__ entry_pos, int64_t cap) {
   extern __shared__ int32_t base[];
   const int tile = blockIdx.x;
   const int64_t bg = blockIdx.y;
@@ -233,13 +236,19 @@ __global__ void __launch_bounds__(32)
   for (int64_t i = 0; i < nq; ++i) {
     const int64_t qi = q0 + i;
     if (lane < kTopK) {
-      const int32_t c = sel[(bg * n_q + qi) * kTopK + lane];
+      const int64_t r = (bg * n_q + qi) * kTopK + lane;
+      const int32_t c = sel[r];
       const int64_t own = (q_pos0 + qi) / kBlock;
+      int32_t at = -1;
       if (c >= 0 && c <= own && c < nblk) {
         const int32_t p = base[c];
         base[c] = p + 1;                // blocks within one row are distinct
-        if (p >= 0 && p < cap) entries[p] = (int32_t)((qi << 4) | lane);
+        if (p >= 0 && p < cap) {
+          entries[p] = (int32_t)((qi << 4) | lane);
+          at = p;
+        }
       }
+      entry_pos[r] = at;
     }
     __syncwarp();
   }
@@ -270,7 +279,7 @@ __global__ void __launch_bounds__(kRowWarps * 32)
     csr_rows_fill_kernel(const int32_t* __restrict__ sel, int64_t n_rows, int64_t q_pos0,
                          int32_t nblk, const int32_t* __restrict__ counts,
                          int32_t* __restrict__ offsets, int32_t* __restrict__ entries,
-                         int64_t cap) {
+                         int32_t* __restrict__ entry_pos, int64_t cap) {
   __shared__ int32_t part[kRowWarps * 32];
   __shared__ int32_t row_base[kRowWarps + 1];
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
@@ -305,12 +314,19 @@ __global__ void __launch_bounds__(kRowWarps * 32)
     for (int k = 0; k < kTopK; ++k) below += (ck[k] < c) ? 1 : 0;
     off[c] = base + below;
   }
-  if (lane < kTopK && mine != 0x7FFFFFFF) {
-    int32_t below = 0;
+  if (lane < kTopK) {
+    int32_t at = -1;
+    if (mine != 0x7FFFFFFF) {
+      int32_t below = 0;
 #pragma unroll
-    for (int k = 0; k < kTopK; ++k) below += (ck[k] < mine) ? 1 : 0;
-    const int64_t p = (int64_t)base + below;
-    if (p < cap) entries[p] = lane;          // query 0 of the row, slot `lane`
+      for (int k = 0; k < kTopK; ++k) below += (ck[k] < mine) ? 1 : 0;
+      const int64_t p = (int64_t)base + below;
+      if (p < cap) {
+        entries[p] = lane;                   // query 0 of the row, slot `lane`
+        at = (int32_t)p;
+      }
+    }
+    entry_pos[r * kTopK + lane] = at;
   }
   if (r == n_rows - 1 && lane == 0) offsets[n_rows * nblk] = row_base[w + 1];
 }
@@ -325,8 +341,8 @@ size_t block_lists_workspace(int64_t bgcount, int64_t n_q, int64_t nblk, int64_t
 
 cudaError_t launch_block_lists(const int32_t* sel, int64_t bgcount, int64_t n_q,
                                int64_t q_pos0, int64_t nblk, int64_t window, int32_t* offsets,
-                               int32_t* entries, int64_t cap, void* ws, int32_t* err,
-                               cudaStream_t st) {
+                               int32_t* entries, int32_t* entry_pos, int64_t cap, void* ws,
+                               int32_t* err, cudaStream_t st) {
   if (n_q == 1) {
     // one window: segment (bg, c) = bg * nblk + c
     int32_t* counts = reinterpret_cast<int32_t*>(ws);
@@ -334,7 +350,8 @@ cudaError_t launch_block_lists(const int32_t* sel, int64_t bgcount, int64_t n_q,
     csr_rows_count_kernel<<<grid, kRowWarps * 32, 0, st>>>(sel, bgcount, q_pos0, (int32_t)nblk,
                                                            counts, err);
     csr_rows_fill_kernel<<<grid, kRowWarps * 32, 0, st>>>(sel, bgcount, q_pos0, (int32_t)nblk,
-                                                          counts, offsets, entries, cap);
+                                                          counts, offsets, entries, entry_pos,
+                                                          cap);
     return cudaGetLastError();
   }
   const int64_t ntiles = (n_q + kCsrTile - 1) / kCsrTile;
@@ -373,7 +390,8 @@ cudaError_t launch_block_lists(const int32_t* sel, int64_t bgcount, int64_t n_q,
                                                                      offsets);
   csr_scatter_kernel<<<g1, 32, hist_bytes, st>>>(sel, n_q, q_pos0, (int32_t)nblk,
                                                  (int32_t)ntiles, tw, (int32_t)nwin,
-                                                 tile_counts, offsets, entries, cap);
+                                                 tile_counts, offsets, entries, entry_pos,
+                                                 cap);
   return cudaGetLastError();
 }
 

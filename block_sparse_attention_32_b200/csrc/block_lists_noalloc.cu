@@ -17,7 +17,8 @@
 namespace msa {
 cudaError_t launch_block_lists(const int32_t* sel, int64_t bgcount, int64_t n_q, int64_t q_pos0,
                                int64_t nblk, int64_t window, int32_t* offsets, int32_t* entries,
-                               int64_t cap, void* ws, int32_t* err, cudaStream_t st);
+                               int32_t* entry_pos, int64_t cap, void* ws, int32_t* err,
+                               cudaStream_t st);
 msa_status validate_dims(const msa_dims* d);
 }  // namespace msa
 
@@ -88,11 +89,13 @@ cudaError_t scratch_address(void** out) {
 
 extern "C" msa_status msa_build_block_query_lists_noalloc(const msa_dims* d, const int32_t* sel,
                                                           int32_t* blk_offsets, int32_t* entries,
-                                                          int32_t* dev_err, void* stream) {
+                                                          int32_t* entry_pos, int32_t* dev_err,
+                                                          void* stream) {
   // the workspace version's checks, with its status codes
   msa_status s = msa::validate_dims(d);
   if (s != MSA_OK) return s;
-  if (sel == nullptr || blk_offsets == nullptr || entries == nullptr) return MSA_ERR_INVALID_ARG;
+  if (sel == nullptr || blk_offsets == nullptr || entries == nullptr || entry_pos == nullptr)
+    return MSA_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(sel) & 15u) != 0) return MSA_ERR_ALIGNMENT;
   const size_t need = msa_block_query_lists_workspace(d);
   if (need > (size_t)MSA_NOALLOC_SCRATCH_BYTES) return MSA_ERR_SCRATCH_LIMIT;
@@ -106,6 +109,6 @@ extern "C" msa_status msa_build_block_query_lists_noalloc(const msa_dims* d, con
   }
   const cudaError_t e = msa::launch_block_lists(
       sel, d->batch * d->h_kv, d->n_q, d->q_pos0, msa_num_blocks(d), msa_query_window(d),
-      blk_offsets, entries, total, ws, dev_err, reinterpret_cast<cudaStream_t>(stream));
+      blk_offsets, entries, entry_pos, total, ws, dev_err, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? MSA_OK : MSA_ERR_CUDA;
 }

@@ -6,6 +6,10 @@
 // what lets the "Outer Gather Q" scheme (page "MSA 稀疏注意力三国杀", section
 // "Kernel 创新：Outer Gather Q") compute each selected block separately.
 //
+// Pieces are in the block->query lists' order: the piece of (b, g, i, slot)
+// and head r of the group is row entry_pos[b, g, i, slot] * R + r; an empty
+// slot has entry_pos -1.
+//
 // One warp per (batch, query, head); lane l owns output dims 4l .. 4l+3.
 // HBM-bound: it reads each piece once.  Compact pieces hold accn_s = acc_s /
 // l_s in bf16; then o = sum_s (l_s e^{m_s-M}) accn_s / L.
@@ -15,7 +19,7 @@ namespace msa {
 
 template <bool kCompact>
 __global__ void __launch_bounds__(256)
-    merge_partials_kernel(const int32_t* __restrict__ sel, const float* __restrict__ part_ml,
+    merge_partials_kernel(const int32_t* __restrict__ entry_pos, const float* __restrict__ part_ml,
                           const void* __restrict__ part_acc, __nv_bfloat16* __restrict__ out,
                           float* __restrict__ lse, int64_t n_rows, int64_t n_q, int32_t H,
                           int32_t G) {
@@ -27,16 +31,19 @@ __global__ void __launch_bounds__(256)
   const int64_t bq = r / H;            // b * n_q + qi
   const int64_t b = bq / n_q, qi = bq - b * n_q;
   const int32_t g = h / R;
-  const int32_t* srow = sel + ((b * G + g) * n_q + qi) * kTopK;
-  // pieces are [B, n_q, G, 16 slots, R, ...]: slot s of this head is row prow0 + s * R
-  const int64_t prow0 = ((b * n_q + qi) * G + g) * kTopK * R + (h - g * R);
+  const int32_t* prow = entry_pos + ((b * G + g) * n_q + qi) * kTopK;
+  const int32_t hr = h - g * R;
 
+  // lane s < 16: the piece row of slot s for this head
   float m = -INFINITY, l = 0.f;
   bool v = false;
+  int64_t row = 0;
   if (lane < kTopK) {
-    v = srow[lane] >= 0;
+    const int32_t p = prow[lane];
+    v = p >= 0;
     if (v) {
-      const float2 ml = *reinterpret_cast<const float2*>(part_ml + (prow0 + lane * R) * 2);
+      row = (int64_t)p * R + hr;
+      const float2 ml = *reinterpret_cast<const float2*>(part_ml + row * 2);
       m = ml.x;
       l = ml.y;
     }
@@ -54,13 +61,13 @@ __global__ void __launch_bounds__(256)
   if constexpr (kCompact) {
     // weight of piece s: l_s e^{m_s - M}
     const float wl = w * l;
-    const __nv_bfloat16* pa =
-        reinterpret_cast<const __nv_bfloat16*>(part_acc) + prow0 * kHeadDim + 4 * lane;
+    const __nv_bfloat16* pa = reinterpret_cast<const __nv_bfloat16*>(part_acc) + 4 * lane;
 #pragma unroll
     for (int s = 0; s < kTopK; ++s) {
       const float ws = __shfl_sync(0xffffffffu, wl, s);
+      const int64_t rs = __shfl_sync(0xffffffffu, row, s);
       if ((vmask >> s) & 1u) {
-        const uint2 u = *reinterpret_cast<const uint2*>(pa + (int64_t)s * R * kHeadDim);
+        const uint2 u = *reinterpret_cast<const uint2*>(pa + rs * kHeadDim);
         const float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
         const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
         acc.x = fmaf(ws, lo.x, acc.x);
@@ -70,12 +77,13 @@ __global__ void __launch_bounds__(256)
       }
     }
   } else {
-    const float* pa = reinterpret_cast<const float*>(part_acc) + prow0 * kHeadDim + 4 * lane;
+    const float* pa = reinterpret_cast<const float*>(part_acc) + 4 * lane;
 #pragma unroll
     for (int s = 0; s < kTopK; ++s) {
       const float ws = __shfl_sync(0xffffffffu, w, s);
+      const int64_t rs = __shfl_sync(0xffffffffu, row, s);
       if ((vmask >> s) & 1u) {
-        const float4 a = *reinterpret_cast<const float4*>(pa + (int64_t)s * R * kHeadDim);
+        const float4 a = *reinterpret_cast<const float4*>(pa + rs * kHeadDim);
         acc.x = fmaf(ws, a.x, acc.x);
         acc.y = fmaf(ws, a.y, acc.y);
         acc.z = fmaf(ws, a.z, acc.z);
@@ -93,7 +101,7 @@ __global__ void __launch_bounds__(256)
   if (lane == 0) lse[r] = M + logf(L);
 }
 
-cudaError_t launch_merge(const int32_t* sel, const float* part_ml, const void* part_acc,
+cudaError_t launch_merge(const int32_t* entry_pos, const float* part_ml, const void* part_acc,
                          bool compact, void* out, float* lse, int64_t n_rows, int64_t n_q,
                          int32_t H, int32_t G, cudaStream_t st) {
   if (n_rows == 0) return cudaSuccess;
@@ -101,10 +109,10 @@ cudaError_t launch_merge(const int32_t* sel, const float* part_ml, const void* p
   const unsigned grid = (unsigned)((threads + 255) / 256);
   __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(out);
   if (compact)
-    merge_partials_kernel<true><<<grid, 256, 0, st>>>(sel, part_ml, part_acc, o, lse, n_rows,
+    merge_partials_kernel<true><<<grid, 256, 0, st>>>(entry_pos, part_ml, part_acc, o, lse, n_rows,
                                                       n_q, H, G);
   else
-    merge_partials_kernel<false><<<grid, 256, 0, st>>>(sel, part_ml, part_acc, o, lse, n_rows,
+    merge_partials_kernel<false><<<grid, 256, 0, st>>>(entry_pos, part_ml, part_acc, o, lse, n_rows,
                                                        n_q, H, G);
   return cudaGetLastError();
 }

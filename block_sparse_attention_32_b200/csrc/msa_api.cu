@@ -20,9 +20,10 @@ cudaError_t launch_topk_blocks(const float*, int64_t, int64_t, int64_t, int64_t,
                                cudaStream_t);
 size_t block_lists_workspace(int64_t, int64_t, int64_t, int64_t);
 cudaError_t launch_block_lists(const int32_t*, int64_t, int64_t, int64_t, int64_t, int64_t,
-                               int32_t*, int32_t*, int64_t, void*, int32_t*, cudaStream_t);
+                               int32_t*, int32_t*, int32_t*, int64_t, void*, int32_t*,
+                               cudaStream_t);
 cudaError_t launch_sparse_attn(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
-                               const CUtensorMap&, const void*, int64_t,
+                               const CUtensorMap&, const CUtensorMap&, const void*, int64_t,
                                int64_t, int64_t, const int32_t*, const int32_t*, int64_t,
                                int64_t, int64_t, int64_t, int32_t, int32_t, int32_t, int32_t,
                                float, float*, void*, bool, int32_t*, cudaStream_t);
@@ -320,11 +321,13 @@ size_t msa_block_query_lists_workspace(const msa_dims* d) {
 }
 
 msa_status msa_build_block_query_lists(const msa_dims* d, const int32_t* sel,
-                                       int32_t* blk_offsets, int32_t* entries, void* ws,
-                                       size_t ws_bytes, int32_t* dev_err, void* stream) {
+                                       int32_t* blk_offsets, int32_t* entries,
+                                       int32_t* entry_pos, void* ws, size_t ws_bytes,
+                                       int32_t* dev_err, void* stream) {
   msa_status s = check_dims(d);
   if (s != MSA_OK) return s;
-  if (sel == nullptr || blk_offsets == nullptr || entries == nullptr || ws == nullptr)
+  if (sel == nullptr || blk_offsets == nullptr || entries == nullptr || entry_pos == nullptr ||
+      ws == nullptr)
     return MSA_ERR_INVALID_ARG;
   if (!aligned16(sel) || !aligned16(ws)) return MSA_ERR_ALIGNMENT;
   if (ws_bytes < msa_block_query_lists_workspace(d)) return MSA_ERR_WORKSPACE_TOO_SMALL;
@@ -332,7 +335,7 @@ msa_status msa_build_block_query_lists(const msa_dims* d, const int32_t* sel,
   if (total >= (int64_t(1) << 31)) return MSA_ERR_UNSUPPORTED;
   return from_cuda(msa::launch_block_lists(sel, d->batch * d->h_kv, d->n_q, d->q_pos0,
                                            msa_num_blocks(d), query_window(d), blk_offsets,
-                                           entries, total, ws, dev_err,
+                                           entries, entry_pos, total, ws, dev_err,
                                            reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -369,10 +372,13 @@ msa_status sparse_attn_fwd(const msa_dims* d, msa_tensor q, msa_tensor k, msa_te
   if ((s = make_map(&tv, v.ptr, MSA_HEAD_DIM, d->n_kv, d->h_kv, d->batch, v.s_tok, v.s_head,
                     v.s_batch, 128, 1)) != MSA_OK)
     return s;
-  // part_acc [B, n_q, G, 16, R, 128] as rows of 128 values; for R >= 8 one
-  // entry's R rows are written by TMA stores of R x 32 floats (or R x 64 bf16)
-  CUtensorMap to, tq;
+  // part_acc [entries, R, 128] as rows of 128-byte panels; for R >= 8 a
+  // warp's 32 adjacent rows are written by TMA stores of 32 rows x 2 panels
+  // (fp32: half rows; bf16: whole rows), a partly covered warp's by 8-row,
+  // one-panel stores
+  CUtensorMap to, to8, tq;
   std::memset(&to, 0, sizeof(to));
+  std::memset(&to8, 0, sizeof(to8));
   std::memset(&tq, 0, sizeof(tq));
   if (decode) {
     // one query per sequence: warp-level tiles, heads as the 8-wide side.
@@ -388,30 +394,31 @@ msa_status sparse_attn_fwd(const msa_dims* d, msa_tensor q, msa_tensor k, msa_te
   if (R >= 8) {
     // q: one box per group of eight heads of an entry (both 64-column panels)
     if ((s = make_map_q_groups(&tq, d, q)) != MSA_OK) return s;
-    const int64_t rows = d->batch * d->n_q * d->h_kv * MSA_TOPK_BLOCKS * R;
+    const int64_t rows = total * R;
     if (rows >= (int64_t(1) << 31)) return MSA_ERR_UNSUPPORTED;
-    // fp32: an entry's half rows (2 panels) per store; bf16: its whole rows
-    s = make_map_piece_rows(&to, part_acc, (uint64_t)rows, compact, (uint32_t)R, 2);
+    s = make_map_piece_rows(&to, part_acc, (uint64_t)rows, compact, 32, 2);
+    if (s != MSA_OK) return s;
+    s = make_map_piece_rows(&to8, part_acc, (uint64_t)rows, compact, 8, 1);
     if (s != MSA_OK) return s;
   }
   return from_cuda(msa::launch_sparse_attn(
-      tq, tk, tv, to, q.ptr, q.s_batch, q.s_tok, q.s_head, blk_offsets, entries, n_seg, total,
+      tq, tk, tv, to, to8, q.ptr, q.s_batch, q.s_tok, q.s_head, blk_offsets, entries, n_seg, total,
       d->n_q, d->q_pos0, d->h_kv, d->h_q, (int32_t)nblk, (int32_t)nwin, d->scale, part_ml,
       part_acc, compact, dev_err, reinterpret_cast<cudaStream_t>(stream)));
 }
 
-msa_status merge_partials(const msa_dims* d, const int32_t* sel, const float* part_ml,
+msa_status merge_partials(const msa_dims* d, const int32_t* entry_pos, const float* part_ml,
                           const void* part_acc, bool compact, void* out, float* lse,
                           void* stream) {
   msa_status s = check_dims(d);
   if (s != MSA_OK) return s;
-  if (sel == nullptr || part_ml == nullptr || part_acc == nullptr || out == nullptr ||
+  if (entry_pos == nullptr || part_ml == nullptr || part_acc == nullptr || out == nullptr ||
       lse == nullptr)
     return MSA_ERR_INVALID_ARG;
   if (!aligned16(part_ml) || !aligned16(part_acc) || !aligned16(out))
     return MSA_ERR_ALIGNMENT;
   const int64_t n_rows = d->batch * d->n_q * d->h_q;
-  return from_cuda(msa::launch_merge(sel, part_ml, part_acc, compact, out, lse, n_rows, d->n_q,
+  return from_cuda(msa::launch_merge(entry_pos, part_ml, part_acc, compact, out, lse, n_rows, d->n_q,
                                      d->h_q, d->h_kv, reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -435,18 +442,18 @@ msa_status msa_sparse_attn_fwd_compact(const msa_dims* d, msa_tensor q, msa_tens
                          dev_err, stream);
 }
 
-msa_status msa_merge_partials(const msa_dims* d, const int32_t* sel, const float* part_ml,
+msa_status msa_merge_partials(const msa_dims* d, const int32_t* entry_pos, const float* part_ml,
                               const float* part_acc, void* out, float* lse, int32_t* dev_err,
                               void* stream) {
   (void)dev_err;
-  return merge_partials(d, sel, part_ml, part_acc, false, out, lse, stream);
+  return merge_partials(d, entry_pos, part_ml, part_acc, false, out, lse, stream);
 }
 
-msa_status msa_merge_partials_compact(const msa_dims* d, const int32_t* sel,
+msa_status msa_merge_partials_compact(const msa_dims* d, const int32_t* entry_pos,
                                       const float* part_ml, const void* part_acc_bf16,
                                       void* out, float* lse, int32_t* dev_err, void* stream) {
   (void)dev_err;
-  return merge_partials(d, sel, part_ml, part_acc_bf16, true, out, lse, stream);
+  return merge_partials(d, entry_pos, part_ml, part_acc_bf16, true, out, lse, stream);
 }
 
 msa_status msa_quantize_e4m3(const void* x, int64_t n, void* codes, float* scale,

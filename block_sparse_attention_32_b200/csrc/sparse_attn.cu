@@ -83,7 +83,7 @@ constexpr int kDescRing = 8;           // chunk descriptors in flight
 
 struct alignas(16) ChunkDesc {
   int32_t b, g, c, cnt;                // cnt < 0: no more work
-  int32_t piece, first, last, pad;
+  int32_t piece, first, last, pos0;   // pos0: position of ent[0] in the entries array
   int32_t ent[128];
 };
 
@@ -146,6 +146,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                            const __grid_constant__ CUtensorMap tm_k,
                            const __grid_constant__ CUtensorMap tm_v,
                            const __grid_constant__ CUtensorMap tm_o,
+                           const __grid_constant__ CUtensorMap tm_o8,
                            const __grid_constant__ AttnArgs a) {
   constexpr int CH = 128 / R;
   // R >= 8: an entry's R head rows (R x 256 contiguous bytes) arrive by TMA
@@ -271,6 +272,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               d.piece = (int32_t)piece;
               d.first = cpos == pos;
               d.last = cpos + CH >= pend;
+              d.pos0 = (int32_t)cpos;
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(bar + BAR_D_FULL + (int)(chunk % kDescRing));
@@ -618,10 +620,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
-    // R >= 8: each warp stages its entries' rows as blocks [2 panels][R rows]
-    // [128 B] (128-byte swizzle; fp32: the two 32-column panels of a half row,
-    // compact: the row's two 64-column halves) and the first lane of each
-    // entry writes the block with one TMA store (a 3-D view of the pieces).
+    // Pieces follow the lists' order: row r of a chunk is piece row
+    // pos0 * R + r, so a warp's 32 rows are adjacent in memory.  R >= 8: each
+    // warp stages its rows as [2 panels][32 rows][128 B] (128-byte swizzle;
+    // fp32: the two 32-column panels of a half row, compact: the row's two
+    // 64-column halves) and one TMA store writes them (a 3-D view of the
+    // pieces); a warp only partly covered by the chunk's entries (the end of
+    // a block's list) stores its rows in 8-row groups, one panel at a time.
     // R < 8: rows padded to 272 B, read back transposed, two half rows (fp32)
     // or four (compact) per store instruction.
     constexpr bool kTmaStore = R >= 8;
@@ -636,24 +641,36 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (d.cnt < 0) break;
       const int ob = (int)(n & 1);
       const int e = d.ent[row / R];
-      const int32_t b = d.b, g = d.g, c = d.c;
+      const int32_t c = d.c;
       if (!WuseW(BAR_O_FULL, 2, n)) break;
       if (!WuseW(BAR_P_FULL, kQRing, n)) break;  // acquire the softmax's (m, l)
       tc_fence_after();
       const float2 ml0 = ml_s[(ob * 2) * 128 + row];
       const float2 ml1 = ml_s[(ob * 2 + 1) * 128 + row];
       mbar_arrive(bar + BAR_ML_EMPTY + ob);      // (m, l) slot ob is free
-      const int hr = row % R;
       const int64_t qi = (int64_t)(e >> 4);
       const bool valid = (e >= 0) && (qi < a.n_q) && (a.q_pos0 + qi >= (int64_t)c * kBlock);
-      // piece row of (b, qi, g, slot, hr): the R head rows of one entry are adjacent
-      const int64_t pidx =
-          valid ? ((((int64_t)b * a.n_q + qi) * a.G + g) * kTopK + (e & 15)) * R + hr : 0;
+      // first piece row of this warp (piece rows < 2^31, checked by the
+      // launcher), and how many of its 32 rows hold entries
+      const int32_t wrow0 = d.pos0 * R + quarter * 32;
+      const int wrows = max(0, min(32, d.cnt * R - quarter * 32));
+      const int64_t pidx = (int64_t)wrow0 + lane;
       const float l_sum = ml0.y + ml1.y;
       if (valid) *reinterpret_cast<float2*>(a.part_ml + pidx * 2) = make_float2(ml0.x, l_sum);
       // compact pieces: acc / l (l >= 1 on a valid row: the row maximum's weight is 1)
       const float inv_l = (kCompact && valid && l_sum > 0.f) ? 1.0f / l_sum : 0.f;
       const uint32_t o_addr = tmem + lane_base + 256 + ob * 128;
+      // the staged [2 panels][32 rows][128 B] -> panels z0, z0 + 1 of rows
+      // wrow0 .. wrow0 + wrows - 1: one store for a whole warp, else one per
+      // 8-row group and panel (wrows is a multiple of R >= 8)
+      auto store_rows = [&](int z0) {
+        if (wrows == 32) {
+          if (lane == 0) tma_store_3d_hint(&tm_o, stage, 0, wrow0, z0, pol_st);
+        } else if (lane < (wrows >> 3) * 2) {
+          tma_store_3d_hint(&tm_o8, stage + (lane & 1) * 4096 + (lane >> 1) * 1024, 0,
+                            wrow0 + (lane >> 1) * 8, z0 + (lane & 1), pol_st);
+        }
+      };
       float* acc = reinterpret_cast<float*>(a.part_acc) + pidx * kHeadDim;
       __nv_bfloat16* acc16 = reinterpret_cast<__nv_bfloat16*>(a.part_acc) + pidx * kHeadDim;
 #pragma unroll 1
@@ -682,16 +699,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               __syncwarp();
             }
             const int sw = lane & 7;
-            uint8_t* mine = stage + (lane / R) * (2 * R * 128) + (lane % R) * 128;
+            uint8_t* mine = stage + lane * 128;
 #pragma unroll
             for (int j = 0; j < 8; ++j)
-              *reinterpret_cast<uint4*>(mine + half * R * 128 + ((j ^ sw) << 4)) =
+              *reinterpret_cast<uint4*>(mine + half * 4096 + ((j ^ sw) << 4)) =
                   make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
             if (half == 1) {
               fence_proxy_async_smem();
               __syncwarp();
-              if (valid && hr == 0)              // first row of an entry: its R rows, both panels
-                tma_store_3d_hint(&tm_o, mine, 0, (int32_t)pidx, 0, pol_st);
+              store_rows(0);
               bulk_commit();
             }
           } else {
@@ -722,18 +738,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           bulk_wait_read();                      // the previous stores have read the block
           __syncwarp();
           const int sw = lane & 7;
-          uint8_t* mine = stage + (lane / R) * (2 * R * 128) + (lane % R) * 128;
+          uint8_t* mine = stage + lane * 128;
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
             *reinterpret_cast<uint4*>(mine + ((j ^ sw) << 4)) =
                 make_uint4(r0[4 * j], r0[4 * j + 1], r0[4 * j + 2], r0[4 * j + 3]);
-            *reinterpret_cast<uint4*>(mine + R * 128 + ((j ^ sw) << 4)) =
+            *reinterpret_cast<uint4*>(mine + 4096 + ((j ^ sw) << 4)) =
                 make_uint4(r1[4 * j], r1[4 * j + 1], r1[4 * j + 2], r1[4 * j + 3]);
           }
           fence_proxy_async_smem();
           __syncwarp();
-          if (valid && hr == 0)                  // first row of an entry: its R half rows
-            tma_store_3d_hint(&tm_o, mine, 0, (int32_t)pidx, half * 2, pol_st);
+          store_rows(half * 2);
           bulk_commit();
         } else {
 #pragma unroll
@@ -781,8 +796,8 @@ uint64_t set_attn_wait_limit(uint64_t ns) { return g_attn_wait_limit_ns.exchange
 
 template <int R, bool kCompact>
 static cudaError_t launch_attn_r(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
-                                 const CUtensorMap& tm_v, const CUtensorMap& tm_o, AttnArgs a,
-                                 cudaStream_t st) {
+                                 const CUtensorMap& tm_v, const CUtensorMap& tm_o,
+                                 const CUtensorMap& tm_o8, AttnArgs a, cudaStream_t st) {
   constexpr int CH = 128 / R;
   auto k = sparse_attn_fwd_kernel<R, kCompact>;
   // the register split above is only safe with exactly this many registers
@@ -805,26 +820,27 @@ static cudaError_t launch_attn_r(const CUtensorMap& tm_q, const CUtensorMap& tm_
   a.n_items = (a.n_entries + W - 1) / W;
   if (a.n_items == 0) return cudaSuccess;
   const int64_t grid = min64(a.n_items, sms);
-  k<<<(unsigned)grid, kAttnThreads, kAttnSmemBytes, st>>>(tm_q, tm_k, tm_v, tm_o, a);
+  k<<<(unsigned)grid, kAttnThreads, kAttnSmemBytes, st>>>(tm_q, tm_k, tm_v, tm_o, tm_o8, a);
   return cudaGetLastError();
 }
 
 template <bool kCompact>
 static cudaError_t launch_attn_c(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
                                  const CUtensorMap& tm_v, const CUtensorMap& tm_o,
-                                 const AttnArgs& a, cudaStream_t st) {
+                                 const CUtensorMap& tm_o8, const AttnArgs& a, cudaStream_t st) {
   switch (a.H / a.G) {
-    case 1: return launch_attn_r<1, kCompact>(tm_q, tm_k, tm_v, tm_o, a, st);
-    case 2: return launch_attn_r<2, kCompact>(tm_q, tm_k, tm_v, tm_o, a, st);
-    case 4: return launch_attn_r<4, kCompact>(tm_q, tm_k, tm_v, tm_o, a, st);
-    case 8: return launch_attn_r<8, kCompact>(tm_q, tm_k, tm_v, tm_o, a, st);
-    case 16: return launch_attn_r<16, kCompact>(tm_q, tm_k, tm_v, tm_o, a, st);
+    case 1: return launch_attn_r<1, kCompact>(tm_q, tm_k, tm_v, tm_o, tm_o8, a, st);
+    case 2: return launch_attn_r<2, kCompact>(tm_q, tm_k, tm_v, tm_o, tm_o8, a, st);
+    case 4: return launch_attn_r<4, kCompact>(tm_q, tm_k, tm_v, tm_o, tm_o8, a, st);
+    case 8: return launch_attn_r<8, kCompact>(tm_q, tm_k, tm_v, tm_o, tm_o8, a, st);
+    case 16: return launch_attn_r<16, kCompact>(tm_q, tm_k, tm_v, tm_o, tm_o8, a, st);
     default: return cudaErrorInvalidValue;
   }
 }
 
 cudaError_t launch_sparse_attn(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
-                               const CUtensorMap& tm_v, const CUtensorMap& tm_o, const void* q,
+                               const CUtensorMap& tm_v, const CUtensorMap& tm_o,
+                               const CUtensorMap& tm_o8, const void* q,
                                int64_t qs_b, int64_t qs_t, int64_t qs_h,
                                const int32_t* blk_offsets, const int32_t* entries,
                                int64_t n_seg, int64_t n_entries, int64_t n_q, int64_t q_pos0,
@@ -853,8 +869,8 @@ cudaError_t launch_sparse_attn(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
   a.part_acc = part_acc;
   a.err = err;
   a.wait_limit_ns = g_attn_wait_limit_ns.load();
-  return compact ? launch_attn_c<true>(tm_q, tm_k, tm_v, tm_o, a, st)
-                 : launch_attn_c<false>(tm_q, tm_k, tm_v, tm_o, a, st);
+  return compact ? launch_attn_c<true>(tm_q, tm_k, tm_v, tm_o, tm_o8, a, st)
+                 : launch_attn_c<false>(tm_q, tm_k, tm_v, tm_o, tm_o8, a, st);
 }
 
 }  // namespace msa

@@ -189,7 +189,6 @@ __global__ void __launch_bounds__(kDaThreads, 1)
       if (d.e < 0) break;
       const int32_t ent = a.entries[d.e];
       const int64_t qi = ent >> 4;
-      const int slot = ent & 15;
       const int64_t lim64 = a.q_pos0 + qi - (int64_t)d.c * kBlock;   // last visible key
       if (qi >= a.n_q || lim64 < 0) {
         report(err, MSA_DEVERR_BAD_ENTRY);
@@ -279,8 +278,8 @@ __global__ void __launch_bounds__(kDaThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(empty + s);          // K, V and Q of the stage are consumed
 
-      // pieces: the R head rows of (b, qi, g, slot) are adjacent rows of part_acc
-      const int64_t prow0 = ((((int64_t)d.b * a.n_q + qi) * a.G + d.g) * kTopK + slot) * R;
+      // pieces in list order: the R head rows of the entry at position d.e
+      const int64_t prow0 = (int64_t)d.e * R;
       if (lane == 0) bulk_wait_read();                 // the previous piece left the staging
       __syncwarp();
 #pragma unroll

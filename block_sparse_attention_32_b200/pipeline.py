@@ -35,6 +35,7 @@ class Buffers:
     sel: torch.Tensor
     blk_offsets: torch.Tensor
     entries: torch.Tensor
+    entry_pos: torch.Tensor
     ws: torch.Tensor
     part_ml: torch.Tensor
     part_acc: torch.Tensor
@@ -62,10 +63,14 @@ class Buffers:
             blk_offsets=torch.empty((capi.msa_num_segments(d) + 1,), dtype=torch.int32,
                                     device=dev),
             entries=torch.empty((max(n_ent, 1),), dtype=torch.int32, device=dev),
+            entry_pos=torch.empty((B, G, n_q, capi.TOPK), dtype=torch.int32, device=dev),
             ws=torch.empty(((ws_bytes + 15) // 16 * 4,), dtype=torch.int32, device=dev),
-            part_ml=torch.empty((B, n_q, G, capi.TOPK, H // G, 2), dtype=torch.float32,
+            # pieces in list order, [entries, R, ...]; sized for 16 slots per
+            # (query, group), so the fp32 buffer also serves as the backward's
+            # dq scratch [B, n_q, G, 16, R, 128]
+            part_ml=torch.empty((B * n_q * G * capi.TOPK, H // G, 2), dtype=torch.float32,
                                 device=dev),
-            part_acc=torch.empty((B, n_q, G, capi.TOPK, H // G, capi.HEAD_DIM),
+            part_acc=torch.empty((B * n_q * G * capi.TOPK, H // G, capi.HEAD_DIM),
                                  dtype=torch.bfloat16 if compact else torch.float32, device=dev),
             out=torch.empty((B, n_q, H, capi.HEAD_DIM), dtype=torch.bfloat16, device=dev),
             lse=torch.empty((B, n_q, H), dtype=torch.float32, device=dev),
@@ -108,16 +113,18 @@ def attend(buf: Buffers, q, k, v, sel=None):
     """Block lists + KV-block-outer attention + merge over `sel` (default buf.sel)."""
     d = buf.dims
     s = buf.sel if sel is None else sel
-    capi.msa_build_block_query_lists(d, s, buf.blk_offsets, buf.entries, buf.ws, buf.dev_err)
+    capi.msa_build_block_query_lists(d, s, buf.blk_offsets, buf.entries, buf.entry_pos, buf.ws,
+                                     buf.dev_err)
     if buf.compact:
         capi.msa_sparse_attn_fwd_compact(d, q, k, v, buf.blk_offsets, buf.entries, buf.part_ml,
                                          buf.part_acc, buf.dev_err)
-        capi.msa_merge_partials_compact(d, s, buf.part_ml, buf.part_acc, buf.out, buf.lse,
-                                        buf.dev_err)
+        capi.msa_merge_partials_compact(d, buf.entry_pos, buf.part_ml, buf.part_acc, buf.out,
+                                        buf.lse, buf.dev_err)
     else:
         capi.msa_sparse_attn_fwd(d, q, k, v, buf.blk_offsets, buf.entries, buf.part_ml,
                                  buf.part_acc, buf.dev_err)
-        capi.msa_merge_partials(d, s, buf.part_ml, buf.part_acc, buf.out, buf.lse, buf.dev_err)
+        capi.msa_merge_partials(d, buf.entry_pos, buf.part_ml, buf.part_acc, buf.out, buf.lse,
+                                buf.dev_err)
 
 
 def forward(buf: Buffers, q, k, v, q_idx, k_idx):

@@ -168,11 +168,15 @@ MSA_API size_t msa_block_query_lists_workspace(const msa_dims* dims);
  *   entries     [msa_num_entries(dims)] int32: (i << 4) | slot for each query
  *               index i (within its batch) and the slot of c in sel[b,g,i,:],
  *               ascending in i inside a segment (deterministic counting sort)
+ *   entry_pos   [B, G, n_q, 16] int32 (the shape of sel): the position in
+ *               entries of (b, g, i, slot), -1 for an empty slot.  The
+ *               attention writes the piece of the entry at position p in
+ *               piece rows p * R .. p * R + R - 1, and the merge finds it here.
  *   ws          device workspace of at least msa_block_query_lists_workspace()
  *               bytes, 16-byte aligned; contents on entry do not matter. */
 MSA_API msa_status msa_build_block_query_lists(const msa_dims* dims, const int32_t* sel,
                                        int32_t* blk_offsets, int32_t* entries,
-                                       void* ws, size_t ws_bytes,
+                                       int32_t* entry_pos, void* ws, size_t ws_bytes,
                                        int32_t* dev_err, void* stream);
 
 /* Size of the device scratch array behind msa_build_block_query_lists_noalloc
@@ -208,20 +212,24 @@ MSA_API msa_status msa_build_block_query_lists(const msa_dims* dims, const int32
  *     GPU (on different streams without ordering) race on the array. */
 MSA_API msa_status msa_build_block_query_lists_noalloc(const msa_dims* dims, const int32_t* sel,
                                                        int32_t* blk_offsets, int32_t* entries,
-                                                       int32_t* dev_err, void* stream);
+                                                       int32_t* entry_pos, int32_t* dev_err,
+                                                       void* stream);
 
 /* Step 3b: KV-block-outer sparse attention (first page "第二步：精算": full
  * attention over the selected blocks only; "稀疏注意力速览" page: exact softmax
  * attention; softmax(Q K^T * scale) V from the "稀疏注意力架构革命" page, section 1.1).  For every
  * segment (b, g, window, c) each K/V block is brought into shared memory once and the
  * R = h_q / h_kv head rows of every listed query are gathered into 128-row
- * tensor-core tiles.  For each (query i, group g, slot, head r of the group,
- * i.e. head h = g * R + r) it writes the piece over the tokens j of block c
- * with j <= t:
- *   part_ml [B, n_q, G, 16, R, 2] fp32: m = max_j scale * q.k_j,
- *                                       l = sum_j e^{scale q.k_j - m}
- *   part_acc[B, n_q, G, 16, R, 128] fp32: sum_j e^{scale q.k_j - m} v_j
- * (the R head rows of one (query, block) are adjacent, R = h_q / h_kv)
+ * tensor-core tiles.  For each list entry (query i, group g, slot) at position
+ * p of entries and each head r of the group (head h = g * R + r) it writes the
+ * piece over the tokens j of block c with j <= t into row p * R + r:
+ *   part_ml [msa_num_entries(dims), R, 2] fp32: m = max_j scale * q.k_j,
+ *                                               l = sum_j e^{scale q.k_j - m}
+ *   part_acc[msa_num_entries(dims), R, 128] fp32: sum_j e^{scale q.k_j - m} v_j
+ * Pieces follow the lists' order, so the rows of one 128-row tile of entries
+ * are adjacent in memory and leave in a few large stores; entry_pos (from the
+ * list builder) maps (b, g, i, slot) back to p.  Rows past the listed entries
+ * are not written.
  * (l sums the fp32 weights e^{...}; they are rounded to bf16 only where they
  * multiply V, as in standard flash attention).  With one query per sequence
  * (n_q = 1) and R <= 8 the work runs on warp-level tiles instead; same output.
@@ -235,7 +243,7 @@ MSA_API msa_status msa_sparse_attn_fwd(const msa_dims* dims, msa_tensor q, msa_t
 /* Step 3b with compact pieces (an opt-in of this library; the pages fix no
  * piece format, and the default above keeps every piece in fp32).  Same
  * arguments and part_ml as msa_sparse_attn_fwd, but part_acc_bf16 is
- * [B, n_q, G, 16, R, 128] bf16 and holds acc / l: the piece's weighted mean
+ * [msa_num_entries(dims), R, 128] bf16 and holds acc / l: the piece's weighted mean
  * of the V rows, a convex combination of them, so it cannot overflow; it is
  * rounded to bf16 once.  This halves the bytes the pieces move (264 instead
  * of 520 per (query, head, block)); merge with msa_merge_partials_compact.
@@ -249,16 +257,18 @@ MSA_API msa_status msa_sparse_attn_fwd_compact(const msa_dims* dims, msa_tensor 
 
 /* Step 3c: log-sum-exp merge of the pieces, in slot order:
  *   M = max_s m_s, L = sum_s l_s e^{m_s - M}, o = sum_s acc_s e^{m_s - M} / L,
- *   lse = M + ln L, over the slots s with sel[b, g, i, s] >= 0.
+ *   lse = M + ln L, over the slots s with p_s = entry_pos[b, g, i, s] >= 0,
+ *   the piece of slot s and head r being row p_s * R + r of the pieces.
+ *   entry_pos [B, G, n_q, 16] int32, as written by the list builder
  *   out [B, n_q, h_q, 128] bf16 contiguous; lse [B, n_q, h_q] fp32. */
-MSA_API msa_status msa_merge_partials(const msa_dims* dims, const int32_t* sel,
+MSA_API msa_status msa_merge_partials(const msa_dims* dims, const int32_t* entry_pos,
                               const float* part_ml, const float* part_acc,
                               void* out, float* lse, int32_t* dev_err, void* stream);
 
 /* Step 3c on compact pieces (msa_sparse_attn_fwd_compact): with
  * accn_s = part_acc_bf16 of slot s, o = sum_s l_s e^{m_s - M} accn_s / L and
  * lse as in msa_merge_partials. */
-MSA_API msa_status msa_merge_partials_compact(const msa_dims* dims, const int32_t* sel,
+MSA_API msa_status msa_merge_partials_compact(const msa_dims* dims, const int32_t* entry_pos,
                                               const float* part_ml, const void* part_acc_bf16,
                                               void* out, float* lse, int32_t* dev_err,
                                               void* stream);
@@ -278,8 +288,9 @@ MSA_API msa_status msa_merge_partials_compact(const msa_dims* dims, const int32_
  *   k, v        [B, h_kv, n_kv, 128] bf16
  *   lse         [B, n_q, h_q] fp32
  *   delta       [B, n_q, h_q] fp32 device scratch (receives D)
- *   part_dq     [B, n_q, h_kv, 16, R, 128] fp32 device scratch, the size and
- *               layout of part_acc (the forward's buffer may be reused)
+ *   part_dq     [B, n_q, h_kv, 16, R, 128] fp32 device scratch (a forward
+ *               piece buffer of B * n_q * h_kv * 16 rows of R x 128 fp32 may
+ *               be reused; the forward itself needs msa_num_entries rows)
  *   dq          [B, n_q, h_q, 128] fp32, contiguous
  *   dk, dv      [B, h_kv, n_kv, 128] fp32, contiguous; zeroed by the call
  * Blocks and keys that no query selected get zero gradients.  dq is summed in

@@ -241,6 +241,28 @@ def block_query_lists(sel, nblk, window=None):
     return offsets, entries[:n_ent]
 
 
+def entry_positions(offsets, entries, B, G, n_q, nblk, window=None):
+    """Inverse of the block->query lists: pos [B, G, n_q, 16] int32 with
+    pos[b, g, i, slot] = p where entries[p] = (i << 4) | slot lies in a
+    segment of (b, g), and -1 for every (query, slot) no entry names.
+
+    The pages have no counterpart: it is how the library finds a piece written
+    in list order (the position of its entry), written out from its
+    definition over the segments ((b * G + g) * nwin + w) * nblk + c."""
+    window = int(window or n_q)
+    nwin = (n_q + window - 1) // window
+    off = np.asarray(offsets, np.int64)
+    ent = np.asarray(entries, np.int64)
+    pos = np.full((B, G, n_q, TOPK), -1, np.int32)
+    for s in range(B * G * nwin * nblk):
+        bg = (s // nblk) // nwin
+        b, g = bg // G, bg % G
+        for p in range(int(off[s]), int(off[s + 1])):
+            e = int(ent[p])
+            pos[b, g, e >> 4, e & 15] = p
+    return pos
+
+
 def forward_rows(q_rows, q_idx_rows, row_pos, row_batch, k, v, k_idx, scale):
     """Whole path for sampled rows: pooled scores, selection, attention."""
     pooled = index_pooled(q_idx_rows, row_pos, row_batch, k_idx)

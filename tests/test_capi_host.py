@@ -131,8 +131,12 @@ def test_pointer_and_stride_checks(lib):
     assert f(None, good, good, P(0x200000), 32, None, None) == 1
     ws = capi.msa_block_query_lists_workspace(d)
     g = lib.msa_build_block_query_lists
-    assert g(ctypes.byref(d), P(0x1000), P(0x2000), P(0x3000), P(0x4000), ws - 4, None, None) == 4
-    assert g(ctypes.byref(d), P(0x1000), None, P(0x3000), P(0x4000), ws, None, None) == 1
+    assert g(ctypes.byref(d), P(0x1000), P(0x2000), P(0x3000), P(0x5000), P(0x4000), ws - 4,
+             None, None) == 4
+    assert g(ctypes.byref(d), P(0x1000), None, P(0x3000), P(0x5000), P(0x4000), ws,
+             None, None) == 1
+    assert g(ctypes.byref(d), P(0x1000), P(0x2000), P(0x3000), None, P(0x4000), ws,
+             None, None) == 1                                       # no entry_pos
     h = lib.msa_sparse_attn_fwd
     assert h(ctypes.byref(d), good, good, mis, P(0x1000), P(0x2000), P(0x3000), P(0x4000),
              None, None) == 3
@@ -152,14 +156,15 @@ def test_noalloc_builder_returns_the_workspace_builders_statuses(lib):
              capi.make_dims(0, 100, 100, 0, 8, 2, 64),        # batch 0: invalid
              capi.make_dims(1, 100, 100, 50, 8, 2, 64)]       # q_pos0 + n_q > n_kv: invalid
     for d in cases:
-        want = ws_fn(ctypes.byref(d), P(0x1000), P(0x2000), P(0x3000), P(0x4000), 1 << 30,
-                     None, None)
-        got = na_fn(ctypes.byref(d), P(0x1000), P(0x2000), P(0x3000), None, None)
+        want = ws_fn(ctypes.byref(d), P(0x1000), P(0x2000), P(0x3000), P(0x5000), P(0x4000),
+                     1 << 30, None, None)
+        got = na_fn(ctypes.byref(d), P(0x1000), P(0x2000), P(0x3000), P(0x5000), None, None)
         assert want in (1, 2) and got == want, (want, got)
-    assert na_fn(None, P(0x1000), P(0x2000), P(0x3000), None, None) == 1
+    assert na_fn(None, P(0x1000), P(0x2000), P(0x3000), P(0x5000), None, None) == 1
     d = capi.make_dims(1, 1000, 4096, 0, 8, 2, 128)
-    assert na_fn(ctypes.byref(d), P(0x1000), None, P(0x3000), None, None) == 1
-    assert na_fn(ctypes.byref(d), P(0x1004), P(0x2000), P(0x3000), None, None) == 3
+    assert na_fn(ctypes.byref(d), P(0x1000), None, P(0x3000), P(0x5000), None, None) == 1
+    assert na_fn(ctypes.byref(d), P(0x1000), P(0x2000), P(0x3000), None, None, None) == 1
+    assert na_fn(ctypes.byref(d), P(0x1004), P(0x2000), P(0x3000), P(0x5000), None, None) == 3
 
 
 def test_token_select_and_backward_validation(lib):

@@ -136,15 +136,20 @@ def test_block_query_lists_bit_exact(w):
     buf.sel.copy_(sel)
     buf.blk_offsets.fill_(-7)
     buf.entries.fill_(-7)
+    buf.entry_pos.fill_(-7)
     buf.ws.fill_(12345)                      # stale workspace must not matter
-    capi.msa_build_block_query_lists(d, buf.sel, buf.blk_offsets, buf.entries, buf.ws, buf.dev_err)
+    capi.msa_build_block_query_lists(d, buf.sel, buf.blk_offsets, buf.entries, buf.entry_pos,
+                                     buf.ws, buf.dev_err)
     torch.cuda.synchronize()
     assert int(buf.dev_err[0]) == 0
     win = oracle.query_window(w.h_q, w.h_kv, w.q_window)
-    off, ent = oracle.block_query_lists(sel.numpy(), capi.msa_num_blocks(d), win)
+    nblk = capi.msa_num_blocks(d)
+    off, ent = oracle.block_query_lists(sel.numpy(), nblk, win)
     np.testing.assert_array_equal(buf.blk_offsets.cpu().numpy(), off.astype(np.int32))
     np.testing.assert_array_equal(buf.entries.cpu().numpy()[:len(ent)], ent)
     assert len(ent) == capi.msa_num_entries(d)
+    pos = oracle.entry_positions(off, ent, w.batch, w.h_kv, w.n_q, nblk, win)
+    np.testing.assert_array_equal(buf.entry_pos.cpu().numpy(), pos)
 
 
 @pytest.mark.parametrize("compact", [False, True], ids=["fp32_pieces", "compact_pieces"])
@@ -183,8 +188,28 @@ def test_attention_on_given_selection(w, compact):
     assert_rows_ok(res, w.name)
 
 
+def _pieces_in_list_order(sel, ml, acc, g):
+    """Pieces given per (b, q, group, slot) [B, n_q, G, 16, R, ...] placed at
+    the positions of a random permutation of the selected slots, as the
+    attention writes them in list order: (entry_pos [B, G, n_q, 16],
+    ml [n, R, 2], acc [n, R, 128]); unselected rows of the buffers hold NaN."""
+    B, G, n_q, _ = sel.shape
+    valid = sel >= 0
+    n = int(valid.sum())
+    pos = torch.full(sel.shape, -1, dtype=torch.int32)
+    pos[valid] = torch.randperm(n, generator=g).to(torch.int32)
+    where = pos.permute(0, 2, 1, 3)                    # [B, n_q, G, 16]
+    sel_v = where >= 0
+    ml_l = torch.full((n + 3,) + tuple(ml.shape[4:]), float("nan"), dtype=ml.dtype)
+    acc_l = torch.full((n + 3,) + tuple(acc.shape[4:]), float("nan"), dtype=acc.dtype)
+    ml_l[where[sel_v].long()] = ml[sel_v]
+    acc_l[where[sel_v].long()] = acc[sel_v]
+    return pos, ml_l.contiguous(), acc_l.contiguous()
+
+
 def test_merge_kernel_against_oracle_merge():
-    """Random pieces (some slots unused) merged by the kernel and by the oracle."""
+    """Random pieces (some slots unused), stored in a shuffled list order,
+    merged by the kernel and by the oracle."""
     _need_gpu()
     w = wl.small("merge", 2, 300, 3000, 2700, 8, 2, 64, seed=21)
     d = pipeline.dims_for(w)
@@ -192,14 +217,14 @@ def test_merge_kernel_against_oracle_merge():
     g = torch.Generator().manual_seed(5)
     B, n_q, H, G = w.batch, w.n_q, w.h_q, w.h_kv
     R = H // G
-    # pieces in the ABI layout [B, n_q, G, 16, R, ...]
     m = torch.randn((B, n_q, G, 16, R), generator=g) * 3
     l = torch.rand((B, n_q, G, 16, R), generator=g) * 5 + 0.5
     acc = torch.randn((B, n_q, G, 16, R, 128), generator=g) * l[..., None]
     ml = torch.stack([m, l], dim=-1).contiguous()
+    pos, ml_l, acc_l = _pieces_in_list_order(sel, ml, acc, g)
     out = torch.empty((B, n_q, H, 128), dtype=torch.bfloat16, device="cuda")
     lse = torch.empty((B, n_q, H), device="cuda")
-    capi.msa_merge_partials(d, sel.cuda(), ml.cuda(), acc.contiguous().cuda(), out, lse)
+    capi.msa_merge_partials(d, pos.cuda(), ml_l.cuda(), acc_l.cuda(), out, lse)
     # oracle view: one row per (b, q, head), 16 slots each
     to_rows = lambda t: t.movedim(4, 3).reshape(B * n_q * H, 16, *t.shape[5:])
     valid = (sel.permute(0, 2, 1, 3)[:, :, torch.arange(H) // R] >= 0).reshape(-1, 16).numpy()
@@ -224,9 +249,10 @@ def test_compact_merge_kernel_against_oracle_merge():
     l = torch.rand((B, n_q, G, 16, R), generator=g) * 5 + 1.0
     accn = torch.randn((B, n_q, G, 16, R, 128), generator=g).to(torch.bfloat16)
     ml = torch.stack([m, l], dim=-1).contiguous()
+    pos, ml_l, accn_l = _pieces_in_list_order(sel, ml, accn, g)
     out = torch.empty((B, n_q, H, 128), dtype=torch.bfloat16, device="cuda")
     lse = torch.empty((B, n_q, H), device="cuda")
-    capi.msa_merge_partials_compact(d, sel.cuda(), ml.cuda(), accn.contiguous().cuda(), out, lse)
+    capi.msa_merge_partials_compact(d, pos.cuda(), ml_l.cuda(), accn_l.cuda(), out, lse)
     to_rows = lambda t: t.movedim(4, 3).reshape(B * n_q * H, 16, *t.shape[5:])
     valid = (sel.permute(0, 2, 1, 3)[:, :, torch.arange(H) // R] >= 0).reshape(-1, 16).numpy()
     acc = accn.double() * l.double()[..., None]
@@ -295,7 +321,8 @@ def test_device_error_on_bad_selection():
     sel = wl.random_selection(w, "cpu")
     sel[0, 0, 5, 1] = 2          # query 5 lives in block 0
     buf.sel.copy_(sel)
-    capi.msa_build_block_query_lists(d, buf.sel, buf.blk_offsets, buf.entries, buf.ws, buf.dev_err)
+    capi.msa_build_block_query_lists(d, buf.sel, buf.blk_offsets, buf.entries, buf.entry_pos,
+                                     buf.ws, buf.dev_err)
     torch.cuda.synchronize()
     assert int(buf.dev_err[0]) == capi.__dict__.get("MSA_DEVERR_BAD_BLOCK", 2)
 

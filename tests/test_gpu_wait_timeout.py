@@ -41,7 +41,8 @@ def test_attention_wait_timeout_is_reported_and_the_next_call_runs(w, compact):
     sel = wl.random_selection(w, "cpu")
     buf.sel.copy_(sel)
     fwd = capi.msa_sparse_attn_fwd_compact if compact else capi.msa_sparse_attn_fwd
-    capi.msa_build_block_query_lists(d, buf.sel, buf.blk_offsets, buf.entries, buf.ws, buf.dev_err)
+    capi.msa_build_block_query_lists(d, buf.sel, buf.blk_offsets, buf.entries, buf.entry_pos,
+                                     buf.ws, buf.dev_err)
     torch.cuda.synchronize()
     assert int(buf.dev_err[0]) == 0
     prev = capi.msa_debug_set_attn_wait_limit_ns(1000)

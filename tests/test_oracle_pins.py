@@ -335,6 +335,33 @@ def test_block_query_lists_against_a_stable_sort(window):
         assert ((qs >= w * win) & (qs < (w + 1) * win)).all()
 
 
+@pytest.mark.parametrize("window", [None, 128, 37])
+def test_entry_positions_invert_the_lists(window):
+    """Every selected (query, slot) points at its own entry, inside the
+    segment of its (batch, group, window, block); empty slots get -1; the
+    positions are a permutation of 0 .. entries - 1."""
+    rng = np.random.default_rng(10)
+    B, G, n_q, nblk = 2, 2, 260, 9
+    sel = np.full((B, G, n_q, 16), -1, np.int32)
+    for b in range(B):
+        for g in range(G):
+            for q in range(n_q):
+                k = rng.integers(0, 9)
+                slots = rng.choice(16, size=k, replace=False)
+                sel[b, g, q, slots] = rng.choice(nblk, size=k, replace=False)
+    offsets, entries = oracle.block_query_lists(sel, nblk, window)
+    pos = oracle.entry_positions(offsets, entries, B, G, n_q, nblk, window)
+    win = window or n_q
+    nwin = -(-n_q // win)
+    assert ((pos >= 0) == (sel >= 0)).all()
+    assert sorted(pos[pos >= 0].tolist()) == list(range(len(entries)))
+    for b, g, q, s in zip(*np.nonzero(sel >= 0)):
+        p = pos[b, g, q, s]
+        assert entries[p] == (q << 4) | s
+        seg = ((b * G + g) * nwin + q // win) * nblk + sel[b, g, q, s]
+        assert offsets[seg] <= p < offsets[seg + 1]
+
+
 def test_query_window_rule():
     """Default window: the largest power of two (>= 128) whose gathered query
     rows of one group, window x R x 256 bytes, fit in 32 MiB."""

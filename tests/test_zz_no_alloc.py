@@ -23,20 +23,22 @@ pytestmark = pytest.mark.gpu
 
 def _lists_with_workspace(d, sel):
     buf = pipeline.Buffers.allocate(d)
-    capi.msa_build_block_query_lists(d, sel, buf.blk_offsets, buf.entries, buf.ws, buf.dev_err)
+    capi.msa_build_block_query_lists(d, sel, buf.blk_offsets, buf.entries, buf.entry_pos,
+                                     buf.ws, buf.dev_err)
     torch.cuda.synchronize()
     assert int(buf.dev_err[0]) == 0
-    return buf.blk_offsets.clone(), buf.entries.clone()
+    return buf.blk_offsets.clone(), buf.entries.clone(), buf.entry_pos.clone()
 
 
 def _lists_without_workspace(d, sel):
     offsets = torch.full((capi.msa_num_segments(d) + 1,), -7, dtype=torch.int32, device="cuda")
     entries = torch.full((max(capi.msa_num_entries(d), 1),), -7, dtype=torch.int32, device="cuda")
+    entry_pos = torch.full(tuple(sel.shape), -7, dtype=torch.int32, device="cuda")
     err = torch.zeros((4,), dtype=torch.int32, device="cuda")
-    capi.msa_build_block_query_lists_noalloc(d, sel, offsets, entries, err)
+    capi.msa_build_block_query_lists_noalloc(d, sel, offsets, entries, entry_pos, err)
     torch.cuda.synchronize()
     assert int(err[0]) == 0
-    return offsets, entries
+    return offsets, entries, entry_pos
 
 
 @pytest.mark.parametrize("w", [
@@ -54,10 +56,10 @@ def test_noalloc_lists_match_the_workspace_version_twice(w):
     # two different selections, one call each, in a row
     for offset in (11, 12):
         sel = wl.random_selection(w, "cpu", seed_offset=offset).cuda()
-        want_off, want_ent = _lists_with_workspace(d, sel)
-        got_off, got_ent = _lists_without_workspace(d, sel)
-        assert torch.equal(got_off, want_off)
-        assert torch.equal(got_ent, want_ent)
+        want = _lists_with_workspace(d, sel)
+        got = _lists_without_workspace(d, sel)
+        for g_, w_ in zip(got, want):
+            assert torch.equal(g_, w_)
 
 
 def test_noalloc_refuses_problems_beyond_its_scratch():
@@ -68,5 +70,5 @@ def test_noalloc_refuses_problems_beyond_its_scratch():
     assert capi.msa_block_query_lists_workspace(d) > (32 << 20)
     dummy = torch.zeros((16,), dtype=torch.int32, device="cuda")
     with pytest.raises(capi.MSAError) as ei:
-        capi.msa_build_block_query_lists_noalloc(d, dummy, dummy, dummy)
+        capi.msa_build_block_query_lists_noalloc(d, dummy, dummy, dummy, dummy)
     assert ei.value.status == 6                    # MSA_ERR_SCRATCH_LIMIT
