@@ -78,7 +78,7 @@ static_assert(kRegsControl + kRegsGather + 2 * kRegsSoftmax + kRegsEpilogue ==
               "warpgroup register shares must add up to the launch allocation");
 static_assert(kAttnThreads * kAttnRegsAtLaunch <= 65536, "register file");
 constexpr int kAttnMaxChunksPerItem = 32;
-constexpr int kQRing = 3;              // Q/P tiles in flight
+constexpr int kQRing = 2;              // Q tiles in flight
 constexpr int kDescRing = 8;           // chunk descriptors in flight
 
 struct alignas(16) ChunkDesc {
@@ -91,8 +91,10 @@ constexpr int kOffK = 0;               // 32768: [K lo | K hi]
 constexpr int kOffV = 32768;           // 32768: [V lo | V hi]
 constexpr int kOffQP = 65536;          // kQRing x 32768: Q tile, then P
 constexpr int kStageRow = 272;                           // staged half row (256 B + pad)
-constexpr int kOffStage = kOffQP + kQRing * 32768;       // 128 staged rows
-constexpr int kOffML = kOffStage + 128 * kStageRow;      // [2 slots][2 halves][128] float2 (m, l)
+constexpr int kOffStage = kOffQP + kQRing * 32768;       // 4 warps x 16 KB of staged rows
+constexpr int kStageBytes = 65536;
+static_assert(128 * kStageRow <= kStageBytes, "padded rows of the R < 8 epilogue");
+constexpr int kOffML = kOffStage + kStageBytes;          // [2 slots][2 halves][128] float2 (m, l)
 constexpr int kOffMX = kOffML + 4096;                    // [2][2 halves][128] float row maxima
 constexpr int kOffVerdict = kOffMX + 2048;               // [2][2 halves][4 quarters] int
 constexpr int kOffDesc = kOffVerdict + 64;               // kDescRing descriptors
@@ -622,17 +624,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     // Pieces follow the lists' order: row r of a chunk is piece row
     // pos0 * R + r, so a warp's 32 rows are adjacent in memory.  R >= 8: each
-    // warp stages its rows as [2 panels][32 rows][128 B] (128-byte swizzle;
-    // fp32: the two 32-column panels of a half row, compact: the row's two
-    // 64-column halves) and one TMA store writes them (a 3-D view of the
-    // pieces); a warp only partly covered by the chunk's entries (the end of
-    // a block's list) stores its rows in 8-row groups, one panel at a time.
+    // warp stages its rows as [panels][32 rows][128 B] (128-byte swizzle;
+    // fp32: four 32-column panels, 16 KB; compact: the row's two 64-column
+    // halves in bf16, 8 KB, in one of two buffers by chunk parity) and one
+    // TMA store writes them (a 3-D view of the pieces: 128-byte panels x rows
+    // x panels); a warp only partly covered by the chunk's entries (the end
+    // of a block's list) stores its rows in 8-row groups, one panel at a time.
     // R < 8: rows padded to 272 B, read back transposed, two half rows (fp32)
     // or four (compact) per store instruction.
     constexpr bool kTmaStore = R >= 8;
     // pieces are read back only by the merge kernel: keep them from displacing Q rows in L2
     const uint64_t pol_st = l2_policy_evict_first();
-    uint8_t* stage = base + kOffStage + quarter * 8192;
+    uint8_t* stage = base + kOffStage + quarter * 16384;
     uint8_t* srow = base + kOffStage + row * kStageRow;
     uint8_t* swarp = base + kOffStage + (quarter * 32) * kStageRow;
     for (int64_t n = 0;; ++n) {
@@ -660,15 +663,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       // compact pieces: acc / l (l >= 1 on a valid row: the row maximum's weight is 1)
       const float inv_l = (kCompact && valid && l_sum > 0.f) ? 1.0f / l_sum : 0.f;
       const uint32_t o_addr = tmem + lane_base + 256 + ob * 128;
-      // the staged [2 panels][32 rows][128 B] -> panels z0, z0 + 1 of rows
-      // wrow0 .. wrow0 + wrows - 1: one store for a whole warp, else one per
-      // 8-row group and panel (wrows is a multiple of R >= 8)
-      auto store_rows = [&](int z0) {
+      // the staged [kPanels][32 rows][128 B] at sbuf -> rows wrow0 .. wrow0 +
+      // wrows - 1: one store for a whole warp, else one per 8-row group and
+      // panel (wrows is a multiple of R >= 8)
+      constexpr int kPanels = kCompact ? 2 : 4;
+      uint8_t* sbuf = kCompact ? stage + (int)(n & 1) * 8192 : stage;
+      auto store_rows = [&]() {
         if (wrows == 32) {
-          if (lane == 0) tma_store_3d_hint(&tm_o, stage, 0, wrow0, z0, pol_st);
-        } else if (lane < (wrows >> 3) * 2) {
-          tma_store_3d_hint(&tm_o8, stage + (lane & 1) * 4096 + (lane >> 1) * 1024, 0,
-                            wrow0 + (lane >> 1) * 8, z0 + (lane & 1), pol_st);
+          if (lane == 0) tma_store_3d_hint(&tm_o, sbuf, 0, wrow0, 0, pol_st);
+        } else if (lane < (wrows >> 3) * kPanels) {
+          const int grp = lane / kPanels, pan = lane % kPanels;
+          tma_store_3d_hint(&tm_o8, sbuf + pan * 4096 + grp * 1024, 0, wrow0 + grp * 8, pan,
+                            pol_st);
         }
       };
       float* acc = reinterpret_cast<float*>(a.part_acc) + pidx * kHeadDim;
@@ -692,14 +698,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             w[16 + x] = pack_bf16x2(u2f(r1[2 * x]) * inv_l, u2f(r1[2 * x + 1]) * inv_l);
           }
           if constexpr (kTmaStore) {
-            // half `half` of the row is panel `half` of the entry's staging
-            // block [2 panels][R rows][128 B]; the block leaves by one store
+            // half `half` of the row is panel `half` of this chunk's staging
+            // buffer [2 panels][32 rows][128 B] (two buffers, by chunk parity);
+            // the buffer leaves by one store
             if (half == 0) {
-              bulk_wait_read();                  // the previous stores have read the block
+              bulk_wait_read_1();                // the store of two chunks ago has read sbuf
               __syncwarp();
             }
             const int sw = lane & 7;
-            uint8_t* mine = stage + lane * 128;
+            uint8_t* mine = sbuf + lane * 128;
 #pragma unroll
             for (int j = 0; j < 8; ++j)
               *reinterpret_cast<uint4*>(mine + half * 4096 + ((j ^ sw) << 4)) =
@@ -707,7 +714,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             if (half == 1) {
               fence_proxy_async_smem();
               __syncwarp();
-              store_rows(0);
+              store_rows();
               bulk_commit();
             }
           } else {
@@ -733,12 +740,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             __syncwarp();
           }
         } else if constexpr (kTmaStore) {
-          // the half row's two 32-column panels into the entry's staging block
-          // [2 panels][R rows][128 B]; one store writes the entry's R half rows
-          bulk_wait_read();                      // the previous stores have read the block
-          __syncwarp();
+          // the half row's two 32-column panels into panels 2 half, 2 half + 1
+          // of the staging [4 panels][32 rows][128 B]; after the second half
+          // one store writes the warp's 32 whole rows
+          if (half == 0) {
+            bulk_wait_read();                    // the previous chunk's store has read it
+            __syncwarp();
+          }
           const int sw = lane & 7;
-          uint8_t* mine = stage + lane * 128;
+          uint8_t* mine = sbuf + half * 8192 + lane * 128;
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
             *reinterpret_cast<uint4*>(mine + ((j ^ sw) << 4)) =
@@ -746,10 +756,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             *reinterpret_cast<uint4*>(mine + 4096 + ((j ^ sw) << 4)) =
                 make_uint4(r1[4 * j], r1[4 * j + 1], r1[4 * j + 2], r1[4 * j + 3]);
           }
-          fence_proxy_async_smem();
-          __syncwarp();
-          store_rows(half * 2);
-          bulk_commit();
+          if (half == 1) {
+            fence_proxy_async_smem();
+            __syncwarp();
+            store_rows();
+            bulk_commit();
+          }
         } else {
 #pragma unroll
           for (int x = 0; x < 8; ++x) {
