@@ -246,6 +246,13 @@ __device__ __forceinline__ void cp_async_16(void* dst, const void* src, uint32_t
                "r"(src_bytes)
                : "memory");
 }
+// one 32-byte store (a full sector); p must be 32-byte aligned
+__device__ __forceinline__ void st_global_v8(float* p, float a0, float a1, float a2, float a3,
+                                             float a4, float a5, float a6, float a7) {
+  asm volatile("st.global.v8.f32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "f"(a0),
+               "f"(a1), "f"(a2), "f"(a3), "f"(a4), "f"(a5), "f"(a6), "f"(a7)
+               : "memory");
+}
 __device__ __forceinline__ void cp_async_commit() {
   asm volatile("cp.async.commit_group;" ::: "memory");
 }

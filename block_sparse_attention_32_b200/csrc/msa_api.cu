@@ -67,6 +67,7 @@ namespace {
 constexpr int64_t kMaxBlocks = 50000;   // shared-memory histogram bound of the inversion
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
 bool is_pow2(int64_t x) { return x > 0 && (x & (x - 1)) == 0; }
 
 // Query window of the block->query lists: dims->q_window when positive, else
@@ -554,7 +555,8 @@ msa_status msa_sparse_attn_bwd(const msa_dims* d, msa_tensor q, msa_tensor k, ms
   if (lse == nullptr || blk_offsets == nullptr || entries == nullptr || delta == nullptr ||
       part_dq == nullptr || dq == nullptr || dk == nullptr || dv == nullptr)
     return MSA_ERR_INVALID_ARG;
-  if (!aligned16(part_dq) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+  // dq pieces, dk and dv leave in 32-byte stores
+  if (!aligned32(part_dq) || !aligned16(dq) || !aligned32(dk) || !aligned32(dv))
     return MSA_ERR_ALIGNMENT;
   const int64_t nblk = msa_num_blocks(d);
   const int64_t total = msa_num_entries(d);

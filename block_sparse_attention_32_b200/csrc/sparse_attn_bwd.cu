@@ -482,11 +482,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           tmem_ld_32x32b_x32(tmem + lane_base + 128 + 32 * cc, r);
           tmem_ld_wait();
           if (dst != nullptr) {
+            // 32-byte stores: each lane writes whole sectors of its own row
 #pragma unroll
-            for (int x = 0; x < 8; ++x)
-              *reinterpret_cast<float4*>(dst + 32 * cc + 4 * x) =
-                  make_float4(a.scale * u2f(r[4 * x]), a.scale * u2f(r[4 * x + 1]),
-                              a.scale * u2f(r[4 * x + 2]), a.scale * u2f(r[4 * x + 3]));
+            for (int x = 0; x < 4; ++x)
+              st_global_v8(dst + 32 * cc + 8 * x, a.scale * u2f(r[8 * x]),
+                           a.scale * u2f(r[8 * x + 1]), a.scale * u2f(r[8 * x + 2]),
+                           a.scale * u2f(r[8 * x + 3]), a.scale * u2f(r[8 * x + 4]),
+                           a.scale * u2f(r[8 * x + 5]), a.scale * u2f(r[8 * x + 6]),
+                           a.scale * u2f(r[8 * x + 7]));
           }
         }
         tc_fence_before();
@@ -508,10 +511,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               tmem_ld_wait();
               if (live) {                // this CTA owns the block: plain stores
 #pragma unroll
-                for (int x = 0; x < 8; ++x)
-                  *reinterpret_cast<float4*>(outp + kb + 32 * cc + 4 * x) =
-                      make_float4(f * u2f(r[4 * x]), f * u2f(r[4 * x + 1]),
-                                  f * u2f(r[4 * x + 2]), f * u2f(r[4 * x + 3]));
+                for (int x = 0; x < 4; ++x)
+                  st_global_v8(outp + kb + 32 * cc + 8 * x, f * u2f(r[8 * x]),
+                               f * u2f(r[8 * x + 1]), f * u2f(r[8 * x + 2]),
+                               f * u2f(r[8 * x + 3]), f * u2f(r[8 * x + 4]),
+                               f * u2f(r[8 * x + 5]), f * u2f(r[8 * x + 6]),
+                               f * u2f(r[8 * x + 7]));
               }
             }
           }

@@ -293,6 +293,8 @@ MSA_API msa_status msa_merge_partials_compact(const msa_dims* dims, const int32_
  *               be reused; the forward itself needs msa_num_entries rows)
  *   dq          [B, n_q, h_q, 128] fp32, contiguous
  *   dk, dv      [B, h_kv, n_kv, 128] fp32, contiguous; zeroed by the call
+ *   (part_dq, dk and dv 32-byte aligned, the others 16-byte aligned:
+ *   MSA_ERR_ALIGNMENT otherwise)
  * Blocks and keys that no query selected get zero gradients.  dq is summed in
  * slot order; each KV block's dk and dv are accumulated by the one block of
  * threads that owns the block (all its query windows) and stored once, so all

@@ -197,6 +197,12 @@ def test_token_select_and_backward_validation(lib):
     bad = list(ptrs)
     bad[6] = P(0x7008)
     assert b(ctypes.byref(d), good, good, good, good, good, *bad, None, None) == 3
+    bad = list(ptrs)
+    bad[6] = P(0x7010)                                   # dk 16- but not 32-byte aligned
+    assert b(ctypes.byref(d), good, good, good, good, good, *bad, None, None) == 3
+    bad = list(ptrs)
+    bad[4] = P(0x5010)                                   # dq pieces likewise
+    assert b(ctypes.byref(d), good, good, good, good, good, *bad, None, None) == 3
     assert b(ctypes.byref(d), good, good, good, mis, good, *ptrs, None, None) == 3
     assert b(None, good, good, good, good, good, *ptrs, None, None) == 1
 
