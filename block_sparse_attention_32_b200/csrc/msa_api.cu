@@ -374,8 +374,9 @@ msa_status sparse_attn_fwd(const msa_dims* d, msa_tensor q, msa_tensor k, msa_te
                     v.s_batch, 128, 1)) != MSA_OK)
     return s;
   // part_acc [entries, R, 128] as rows of 128-byte panels; for R >= 8 a
-  // warp's 32 adjacent whole rows are written by one TMA store (fp32: 4
-  // panels, bf16: 2), a partly covered warp's by 8-row, one-panel stores
+  // warp's 32 adjacent rows are written by TMA stores of 32 rows x 2 panels
+  // (fp32: half rows; bf16: whole rows), a partly covered warp's by 8-row,
+  // one-panel stores
   CUtensorMap to, to8, tq;
   std::memset(&to, 0, sizeof(to));
   std::memset(&to8, 0, sizeof(to8));
@@ -396,7 +397,7 @@ msa_status sparse_attn_fwd(const msa_dims* d, msa_tensor q, msa_tensor k, msa_te
     if ((s = make_map_q_groups(&tq, d, q)) != MSA_OK) return s;
     const int64_t rows = total * R;
     if (rows >= (int64_t(1) << 31)) return MSA_ERR_UNSUPPORTED;
-    s = make_map_piece_rows(&to, part_acc, (uint64_t)rows, compact, 32, compact ? 2 : 4);
+    s = make_map_piece_rows(&to, part_acc, (uint64_t)rows, compact, 32, 2);
     if (s != MSA_OK) return s;
     s = make_map_piece_rows(&to8, part_acc, (uint64_t)rows, compact, 8, 1);
     if (s != MSA_OK) return s;

@@ -624,12 +624,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     // Pieces follow the lists' order: row r of a chunk is piece row
     // pos0 * R + r, so a warp's 32 rows are adjacent in memory.  R >= 8: each
-    // warp stages its rows as [panels][32 rows][128 B] (128-byte swizzle;
-    // fp32: four 32-column panels, 16 KB; compact: the row's two 64-column
-    // halves in bf16, 8 KB, in one of two buffers by chunk parity) and one
-    // TMA store writes them (a 3-D view of the pieces: 128-byte panels x rows
-    // x panels); a warp only partly covered by the chunk's entries (the end
-    // of a block's list) stores its rows in 8-row groups, one panel at a time.
+    // warp stages [2 panels][32 rows][128 B] at a time (128-byte swizzle;
+    // fp32: a half row's two 32-column panels, one buffer per half; compact:
+    // the row's two 64-column halves in bf16, one buffer per chunk parity)
+    // and one TMA store writes them (a 3-D view of the pieces: 128-byte
+    // panels x rows x panels); a warp only partly covered by the chunk's
+    // entries (the end of a block's list) stores its rows in 8-row groups,
+    // one panel at a time.
     // R < 8: rows padded to 272 B, read back transposed, two half rows (fp32)
     // or four (compact) per store instruction.
     constexpr bool kTmaStore = R >= 8;
@@ -663,17 +664,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       // compact pieces: acc / l (l >= 1 on a valid row: the row maximum's weight is 1)
       const float inv_l = (kCompact && valid && l_sum > 0.f) ? 1.0f / l_sum : 0.f;
       const uint32_t o_addr = tmem + lane_base + 256 + ob * 128;
-      // the staged [kPanels][32 rows][128 B] at sbuf -> rows wrow0 .. wrow0 +
-      // wrows - 1: one store for a whole warp, else one per 8-row group and
-      // panel (wrows is a multiple of R >= 8)
-      constexpr int kPanels = kCompact ? 2 : 4;
+      // two staged panels [2][32 rows][128 B] at src -> panels z0, z0 + 1 of
+      // rows wrow0 .. wrow0 + wrows - 1: one store for a whole warp, else one
+      // per 8-row group and panel (wrows is a multiple of R >= 8)
       uint8_t* sbuf = kCompact ? stage + (int)(n & 1) * 8192 : stage;
-      auto store_rows = [&]() {
+      auto store_rows = [&](uint8_t* src, int z0) {
         if (wrows == 32) {
-          if (lane == 0) tma_store_3d_hint(&tm_o, sbuf, 0, wrow0, 0, pol_st);
-        } else if (lane < (wrows >> 3) * kPanels) {
-          const int grp = lane / kPanels, pan = lane % kPanels;
-          tma_store_3d_hint(&tm_o8, sbuf + pan * 4096 + grp * 1024, 0, wrow0 + grp * 8, pan,
+          if (lane == 0) tma_store_3d_hint(&tm_o, src, 0, wrow0, z0, pol_st);
+        } else if (lane < (wrows >> 3) * 2) {
+          const int grp = lane >> 1, pan = lane & 1;
+          tma_store_3d_hint(&tm_o8, src + pan * 4096 + grp * 1024, 0, wrow0 + grp * 8, z0 + pan,
                             pol_st);
         }
       };
@@ -714,7 +714,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             if (half == 1) {
               fence_proxy_async_smem();
               __syncwarp();
-              store_rows();
+              store_rows(sbuf, 0);
               bulk_commit();
             }
           } else {
@@ -740,15 +740,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             __syncwarp();
           }
         } else if constexpr (kTmaStore) {
-          // the half row's two 32-column panels into panels 2 half, 2 half + 1
-          // of the staging [4 panels][32 rows][128 B]; after the second half
-          // one store writes the warp's 32 whole rows
-          if (half == 0) {
-            bulk_wait_read();                    // the previous chunk's store has read it
-            __syncwarp();
-          }
+          // the half row's two 32-column panels into its own staging buffer
+          // [2 panels][32 rows][128 B] (one per half), written by one store
+          // as soon as it is staged; a buffer is refilled once the store from
+          // the same half of the previous chunk has read it
+          bulk_wait_read_1();
+          __syncwarp();
           const int sw = lane & 7;
-          uint8_t* mine = sbuf + half * 8192 + lane * 128;
+          uint8_t* hbuf = sbuf + half * 8192;
+          uint8_t* mine = hbuf + lane * 128;
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
             *reinterpret_cast<uint4*>(mine + ((j ^ sw) << 4)) =
@@ -756,12 +756,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             *reinterpret_cast<uint4*>(mine + 4096 + ((j ^ sw) << 4)) =
                 make_uint4(r1[4 * j], r1[4 * j + 1], r1[4 * j + 2], r1[4 * j + 3]);
           }
-          if (half == 1) {
-            fence_proxy_async_smem();
-            __syncwarp();
-            store_rows();
-            bulk_commit();
-          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          store_rows(hbuf, half * 2);
+          bulk_commit();
         } else {
 #pragma unroll
           for (int x = 0; x < 8; ++x) {
