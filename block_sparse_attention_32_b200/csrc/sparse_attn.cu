@@ -3,7 +3,9 @@
 // memory by TMA once per work item, the query rows that chose the block are
 // gathered into 128-row tiles, and S = Q K^T, the softmax piece and O = P V
 // run on the tcgen05 tensor cores with fp32 accumulators in TMEM.  Each
-// (query, head, slot) gets a piece (m, l, acc) that the merge kernel combines.
+// (query, head, slot) gets a piece (m, l, acc) that the merge kernel combines;
+// pieces are stored in the order of the lists' entries (the entry at position
+// p owns rows p * R .. p * R + R - 1), so a chunk's pieces are adjacent.
 // Pieces are fp32 by default; the compact form (an opt-in of the C ABI) keeps
 // (m, l) in fp32 and stores acc / l rounded to bf16 (a convex combination of
 // V rows, so it cannot overflow), which halves the piece traffic.
@@ -29,7 +31,7 @@
 //                             loaded as soon as the last S MMA of the current
 //                             one is done, V as soon as its last P V is done
 //   warp 3      idle (fills the control warpgroup)
-//   warps 4-7   gather:       the chunk's Q rows into a 3-deep ring: for R >= 8
+//   warps 4-7   gather:       the chunk's Q rows into a 2-deep ring: for R >= 8
 //                             warp 4 alone, one 2 KB TMA box per eight heads
 //                             of an entry (both 64-column panels; a 5-D view
 //                             of q), otherwise 16-byte cp.async by all four
@@ -43,15 +45,17 @@
 //                             of O = P V)
 //   warps 16-19 epilogue:     O from TMEM half a row at a time, then the
 //                             (m, l, acc) pieces to global memory.  R >= 8:
-//                             the half rows are staged in 128B-swizzled
-//                             panels and each entry's R rows leave by TMA
-//                             tensor stores; R < 8: staged rows are read
-//                             back transposed so that one store instruction
+//                             each warp stages its 32 rows in 128B-swizzled
+//                             panels and writes them with one TMA tensor
+//                             store per half row (fp32) or per chunk
+//                             (compact); R < 8: staged rows are read back
+//                             transposed so that one store instruction
 //                             writes two whole half rows (coalesced)
 // The five warpgroups split the register file unevenly (setmaxnreg).
-// Shared memory: K 32 KB, V 32 KB, 3 x 32 KB Q tiles (128B-swizzled K-major;
+// Shared memory: K 32 KB, V 32 KB, 2 x 32 KB Q tiles (128B-swizzled K-major;
 // a Q tile gathered by TMA is laid out [8-row group][panel][8 rows][128 B] so
-// that one box brings eight heads of an entry; V is read N-major for P V), 34 KB output staging, (m, l) slots and the row
+// that one box brings eight heads of an entry; V is read N-major for P V),
+// 64 KB output staging (16 KB per epilogue warp), (m, l) slots and the row
 // maxima the two softmax halves exchange.  TMEM: S/P in columns [0,256), O in
 // [256,512), two buffers of 128 columns each; a Q tile is released as soon as
 // its S MMA is done, S(n+2) waits for O(n) = P(n) V, which reads P(n) from
@@ -89,7 +93,7 @@ struct alignas(16) ChunkDesc {
 
 constexpr int kOffK = 0;               // 32768: [K lo | K hi]
 constexpr int kOffV = 32768;           // 32768: [V lo | V hi]
-constexpr int kOffQP = 65536;          // kQRing x 32768: Q tile, then P
+constexpr int kOffQP = 65536;          // kQRing x 32768: the gathered Q tiles
 constexpr int kStageRow = 272;                           // staged half row (256 B + pad)
 constexpr int kOffStage = kOffQP + kQRing * 32768;       // 4 warps x 16 KB of staged rows
 constexpr int kStageBytes = 65536;

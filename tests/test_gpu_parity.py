@@ -177,6 +177,12 @@ def test_attention_on_given_selection(w, compact):
     pipeline.attend(buf, inp["q"], inp["k"], inp["v"])
     torch.cuda.synchronize()
     assert int(buf.dev_err[0]) == 0
+    # pieces are written in list order: every listed entry's rows, nothing past them
+    n_ent = int(buf.blk_offsets[-1])
+    assert n_ent == capi.msa_num_entries(d)
+    assert not torch.isnan(buf.part_ml[:n_ent]).any()
+    assert torch.isnan(buf.part_ml[n_ent:]).all()
+    assert torch.isnan(buf.part_acc[n_ent:].float()).all()
     idx, pos, bat = _all_rows(w)
     q_rows = bits(inp["q"]).reshape(-1, w.h_q, 128)
     sel_rows = sel.permute(0, 2, 1, 3).reshape(-1, w.h_kv, 16).numpy()
