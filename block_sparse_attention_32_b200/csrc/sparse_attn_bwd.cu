@@ -54,6 +54,7 @@ struct BwdArgs {
   float* dk;                  // [B, G, n_kv, 128]
   float* dv;
   int64_t n_q, n_kv, q_pos0, nseg, total, nitems;   // items: (batch, group, block)
+  const int32_t* perm;        // items largest first (null: in index order)
   int32_t G, H, nblk, nwin;   // segments are (batch, group, query window, block)
   float scale;
   int32_t* err;
@@ -128,7 +129,9 @@ constexpr uint32_t idesc_tc(int a_mn, int b_mn) {
 }
 
 // The CTA's sequence of pieces: its items in snake order, skipping blocks no
-// query selected.  Every role walks the same sequence.
+// query selected.  Every role walks the same sequence.  With a.perm the items
+// are dealt largest first (longest-processing-time order), which evens out
+// the CTAs' loads; results do not depend on which CTA takes an item.
 struct PieceWalk {
   int64_t round;
 };
@@ -146,8 +149,9 @@ __device__ __forceinline__ bool walk_next(PieceWalk& w, const BwdArgs& a, Piece&
   for (;;) {
     const int64_t j = w.round++;
     const int64_t k = (j & 1) ? (int64_t)(gridDim.x - 1 - blockIdx.x) : (int64_t)blockIdx.x;
-    const int64_t i = j * gridDim.x + k;                 // grows with j: the last item ends it
-    if (i >= a.nitems) return false;
+    const int64_t i0 = j * gridDim.x + k;                // grows with j: the last item ends it
+    if (i0 >= a.nitems) return false;
+    const int64_t i = a.perm != nullptr ? (int64_t)__ldg(a.perm + i0) : i0;
     const int64_t bg = i / a.nblk;
     const int32_t c = (int32_t)(i - bg * a.nblk);
     const int64_t seg0 = bg * a.nwin * a.nblk + c;
@@ -556,6 +560,57 @@ __global__ void __launch_bounds__(256)
   *reinterpret_cast<float4*>(dq + r * kHeadDim + 4 * lane) = acc;
 }
 
+// ---------------------------------------------------------------------------
+// work order: items by tile count, largest first (a counting sort over
+// kOrderBuckets buckets; the order inside a bucket is whatever the atomics
+// give, which changes only which CTA takes an item, never a result)
+// ---------------------------------------------------------------------------
+constexpr int kOrderBuckets = 1024;
+
+__device__ __forceinline__ int item_bucket(const int32_t* __restrict__ offsets, int64_t i,
+                                           int64_t nblk, int32_t nwin, int kEnt) {
+  const int64_t bg = i / nblk;
+  const int64_t seg0 = bg * nwin * nblk + (i - bg * nblk);
+  int64_t nt = 0;
+  for (int32_t w = 0; w < nwin; ++w) {
+    const int64_t sg = seg0 + (int64_t)w * nblk;
+    nt += ((int64_t)offsets[sg + 1] - offsets[sg] + kEnt - 1) / kEnt;
+  }
+  return (int)min64(nt, kOrderBuckets - 1);
+}
+
+__global__ void __launch_bounds__(256)
+    bwd_item_hist_kernel(const int32_t* __restrict__ offsets, int64_t nitems, int64_t nblk,
+                         int32_t nwin, int kEnt, int32_t* __restrict__ hist) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nitems;
+       i += (int64_t)gridDim.x * blockDim.x)
+    atomicAdd(hist + item_bucket(offsets, i, nblk, nwin, kEnt), 1);
+}
+
+// counts -> first position of each bucket, buckets in descending order
+__global__ void __launch_bounds__(kOrderBuckets) bwd_item_scan_kernel(int32_t* hist) {
+  __shared__ int32_t s[kOrderBuckets];
+  const int t = threadIdx.x;
+  s[t] = hist[kOrderBuckets - 1 - t];
+  __syncthreads();
+  for (int o = 1; o < kOrderBuckets; o <<= 1) {
+    const int32_t v = t >= o ? s[t - o] : 0;
+    __syncthreads();
+    s[t] += v;
+    __syncthreads();
+  }
+  hist[kOrderBuckets - 1 - t] = s[t] - hist[kOrderBuckets - 1 - t];   // exclusive
+}
+
+__global__ void __launch_bounds__(256)
+    bwd_item_scatter_kernel(const int32_t* __restrict__ offsets, int64_t nitems, int64_t nblk,
+                            int32_t nwin, int kEnt, int32_t* __restrict__ cursor,
+                            int32_t* __restrict__ perm) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nitems;
+       i += (int64_t)gridDim.x * blockDim.x)
+    perm[atomicAdd(cursor + item_bucket(offsets, i, nblk, nwin, kEnt), 1)] = (int32_t)i;
+}
+
 template <int R>
 static cudaError_t launch_bwd_tc_r(const CUtensorMap& tm_k, const CUtensorMap& tm_v,
                                    const BwdArgs& a, int grid, cudaStream_t st) {
@@ -622,7 +677,25 @@ cudaError_t launch_sparse_attn_bwd(const CUtensorMap& tm_k, const CUtensorMap& t
   a.err = err;
   // one item per (batch, group, KV block); at most one CTA per SM
   a.nitems = batch * G * (int64_t)nblk;
+  a.perm = nullptr;
   const int grid = total_entries > 0 ? (int)min64(a.nitems, sms) : 0;
+  // the largest-first order lives in dq's memory until the final reduction
+  // overwrites it (when dq is large enough to hold it)
+  if (grid > 0 && a.nitems > grid && a.nitems < (int64_t(1) << 31) &&
+      (int64_t)kOrderBuckets + a.nitems <= rows * kHeadDim) {
+    int32_t* hist = reinterpret_cast<int32_t*>(dq);
+    int32_t* perm = hist + kOrderBuckets;
+    const int kEnt = kBlock / R;
+    if ((e = cudaMemsetAsync(hist, 0, kOrderBuckets * sizeof(int32_t), st)) != cudaSuccess)
+      return e;
+    const unsigned og = (unsigned)min64((a.nitems + 255) / 256, (int64_t)sms * 8);
+    bwd_item_hist_kernel<<<og, 256, 0, st>>>(offsets, a.nitems, nblk, nwin, kEnt, hist);
+    bwd_item_scan_kernel<<<1, kOrderBuckets, 0, st>>>(hist);
+    bwd_item_scatter_kernel<<<og, 256, 0, st>>>(offsets, a.nitems, nblk, nwin, kEnt, hist,
+                                                perm);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    a.perm = perm;
+  }
   if (grid > 0) {
     switch (R) {
       case 1: e = launch_bwd_tc_r<1>(tm_k, tm_v, a, grid, st); break;

@@ -291,7 +291,8 @@ MSA_API msa_status msa_merge_partials_compact(const msa_dims* dims, const int32_
  *   part_dq     [B, n_q, h_kv, 16, R, 128] fp32 device scratch (a forward
  *               piece buffer of B * n_q * h_kv * 16 rows of R x 128 fp32 may
  *               be reused; the forward itself needs msa_num_entries rows)
- *   dq          [B, n_q, h_q, 128] fp32, contiguous
+ *   dq          [B, n_q, h_q, 128] fp32, contiguous (its memory also holds
+ *               the call's work order until the result overwrites it)
  *   dk, dv      [B, h_kv, n_kv, 128] fp32, contiguous; zeroed by the call
  *   (part_dq, dk and dv 32-byte aligned, the others 16-byte aligned:
  *   MSA_ERR_ALIGNMENT otherwise)
