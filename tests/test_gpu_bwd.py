@@ -41,6 +41,9 @@ CASES = [
     # block->query lists in query windows of 256: a block's gradient gathers
     # from several windows' segments
     wl.small("bwd_r8_windows", 1, 1700, 1700, 0, 16, 2, 128, seed=77, q_window=256),
+    # 2 x 2 x 80 = 320 (batch, group, block) items, more than there are SMs: the
+    # items are dealt largest first (the work order the call sorts on the device)
+    wl.small("bwd_r8_sorted_items", 2, 600, 10240, 9640, 16, 2, 128, seed=78),
 ]
 
 
@@ -78,14 +81,15 @@ def test_backward_matches_oracle(w):
     _check("delta", grads.delta.cpu().numpy(), e_delta)
 
 
-@pytest.mark.parametrize("wi", [1, 6], ids=["chunk_after_cache", "query_windows"])
+@pytest.mark.parametrize("wi", [1, 6, 7], ids=["chunk_after_cache", "query_windows",
+                                               "sorted_items"])
 def test_backward_deterministic_and_unselected_blocks_zero(wi):
     """dq is summed in slot order and every KV block's dk, dv come from the one
     CTA that owns the block: two runs give identical bits for all three, also
     when a block's queries span several query windows; the keys of a cache
     block that no query selected get exactly zero dk and dv."""
     _need_gpu()
-    w = CASES[wi]              # 700 new queries after 2400 cached tokens / windows of 256
+    w = CASES[wi]              # a chunk after cached tokens / windows of 256 / 320 items
     d = pipeline.dims_for(w)
     buf = pipeline.Buffers.allocate(d)
     inp = wl.make_inputs(w, "cuda")
