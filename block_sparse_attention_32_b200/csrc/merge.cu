@@ -8,7 +8,8 @@
 //
 // Pieces are in the block->query lists' order: the piece of (b, g, i, slot)
 // and head r of the group is row entry_pos[b, g, i, slot] * R + r; an empty
-// slot has entry_pos -1.
+// slot has entry_pos -1, and a position past the lists' entries is reported
+// (MSA_DEVERR_BAD_ENTRY) and read as an empty slot.
 //
 // One warp per (batch, query, head); lane l owns output dims 4l .. 4l+3.
 // HBM-bound: it reads each piece once.  Compact pieces hold accn_s = acc_s /
@@ -22,7 +23,7 @@ __global__ void __launch_bounds__(256)
     merge_partials_kernel(const int32_t* __restrict__ entry_pos, const float* __restrict__ part_ml,
                           const void* __restrict__ part_acc, __nv_bfloat16* __restrict__ out,
                           float* __restrict__ lse, int64_t n_rows, int64_t n_q, int32_t H,
-                          int32_t G) {
+                          int32_t G, int64_t n_ent, int32_t* err) {
   const int lane = threadIdx.x & 31;
   const int64_t r = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   if (r >= n_rows) return;
@@ -39,7 +40,11 @@ __global__ void __launch_bounds__(256)
   bool v = false;
   int64_t row = 0;
   if (lane < kTopK) {
-    const int32_t p = prow[lane];
+    int32_t p = prow[lane];
+    if (p >= n_ent) {
+      report(err, MSA_DEVERR_BAD_ENTRY);
+      p = -1;
+    }
     v = p >= 0;
     if (v) {
       row = (int64_t)p * R + hr;
@@ -103,17 +108,17 @@ __global__ void __launch_bounds__(256)
 
 cudaError_t launch_merge(const int32_t* entry_pos, const float* part_ml, const void* part_acc,
                          bool compact, void* out, float* lse, int64_t n_rows, int64_t n_q,
-                         int32_t H, int32_t G, cudaStream_t st) {
+                         int32_t H, int32_t G, int64_t n_ent, int32_t* err, cudaStream_t st) {
   if (n_rows == 0) return cudaSuccess;
   const int64_t threads = n_rows * 32;
   const unsigned grid = (unsigned)((threads + 255) / 256);
   __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(out);
   if (compact)
     merge_partials_kernel<true><<<grid, 256, 0, st>>>(entry_pos, part_ml, part_acc, o, lse, n_rows,
-                                                      n_q, H, G);
+                                                      n_q, H, G, n_ent, err);
   else
     merge_partials_kernel<false><<<grid, 256, 0, st>>>(entry_pos, part_ml, part_acc, o, lse, n_rows,
-                                                       n_q, H, G);
+                                                       n_q, H, G, n_ent, err);
   return cudaGetLastError();
 }
 

@@ -59,7 +59,7 @@ cudaError_t launch_index_score_e4m3(const CUtensorMap&, const CUtensorMap&, int6
 cudaError_t launch_quantize_e4m3(const void*, int64_t, void*, float*, cudaStream_t);
 uint64_t set_attn_wait_limit(uint64_t);
 cudaError_t launch_merge(const int32_t*, const float*, const void*, bool, void*, float*,
-                         int64_t, int64_t, int32_t, int32_t, cudaStream_t);
+                         int64_t, int64_t, int32_t, int32_t, int64_t, int32_t*, cudaStream_t);
 }  // namespace msa
 
 namespace {
@@ -410,7 +410,7 @@ msa_status sparse_attn_fwd(const msa_dims* d, msa_tensor q, msa_tensor k, msa_te
 
 msa_status merge_partials(const msa_dims* d, const int32_t* entry_pos, const float* part_ml,
                           const void* part_acc, bool compact, void* out, float* lse,
-                          void* stream) {
+                          int32_t* dev_err, void* stream) {
   msa_status s = check_dims(d);
   if (s != MSA_OK) return s;
   if (entry_pos == nullptr || part_ml == nullptr || part_acc == nullptr || out == nullptr ||
@@ -419,8 +419,9 @@ msa_status merge_partials(const msa_dims* d, const int32_t* entry_pos, const flo
   if (!aligned16(part_ml) || !aligned16(part_acc) || !aligned16(out))
     return MSA_ERR_ALIGNMENT;
   const int64_t n_rows = d->batch * d->n_q * d->h_q;
-  return from_cuda(msa::launch_merge(entry_pos, part_ml, part_acc, compact, out, lse, n_rows, d->n_q,
-                                     d->h_q, d->h_kv, reinterpret_cast<cudaStream_t>(stream)));
+  return from_cuda(msa::launch_merge(entry_pos, part_ml, part_acc, compact, out, lse, n_rows,
+                                     d->n_q, d->h_q, d->h_kv, msa_num_entries(d), dev_err,
+                                     reinterpret_cast<cudaStream_t>(stream)));
 }
 
 }  // namespace
@@ -446,15 +447,13 @@ msa_status msa_sparse_attn_fwd_compact(const msa_dims* d, msa_tensor q, msa_tens
 msa_status msa_merge_partials(const msa_dims* d, const int32_t* entry_pos, const float* part_ml,
                               const float* part_acc, void* out, float* lse, int32_t* dev_err,
                               void* stream) {
-  (void)dev_err;
-  return merge_partials(d, entry_pos, part_ml, part_acc, false, out, lse, stream);
+  return merge_partials(d, entry_pos, part_ml, part_acc, false, out, lse, dev_err, stream);
 }
 
 msa_status msa_merge_partials_compact(const msa_dims* d, const int32_t* entry_pos,
                                       const float* part_ml, const void* part_acc_bf16,
                                       void* out, float* lse, int32_t* dev_err, void* stream) {
-  (void)dev_err;
-  return merge_partials(d, entry_pos, part_ml, part_acc_bf16, true, out, lse, stream);
+  return merge_partials(d, entry_pos, part_ml, part_acc_bf16, true, out, lse, dev_err, stream);
 }
 
 msa_status msa_quantize_e4m3(const void* x, int64_t n, void* codes, float* scale,

@@ -259,7 +259,9 @@ MSA_API msa_status msa_sparse_attn_fwd_compact(const msa_dims* dims, msa_tensor 
  *   M = max_s m_s, L = sum_s l_s e^{m_s - M}, o = sum_s acc_s e^{m_s - M} / L,
  *   lse = M + ln L, over the slots s with p_s = entry_pos[b, g, i, s] >= 0,
  *   the piece of slot s and head r being row p_s * R + r of the pieces.
- *   entry_pos [B, G, n_q, 16] int32, as written by the list builder
+ *   entry_pos [B, G, n_q, 16] int32, as written by the list builder; a
+ *             position >= msa_num_entries(dims) sets MSA_DEVERR_BAD_ENTRY in
+ *             *dev_err and counts as an empty slot
  *   out [B, n_q, h_q, 128] bf16 contiguous; lse [B, n_q, h_q] fp32. */
 MSA_API msa_status msa_merge_partials(const msa_dims* dims, const int32_t* entry_pos,
                               const float* part_ml, const float* part_acc,

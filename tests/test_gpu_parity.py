@@ -241,6 +241,42 @@ def test_merge_kernel_against_oracle_merge():
     assert np.abs(lse.reshape(-1).cpu().numpy() - lse_ref).max() <= 1e-4
 
 
+def test_merge_reports_a_position_past_the_entries():
+    """An entry position at or past msa_num_entries is reported as a bad
+    entry by the merge's own bounds check and counted as an empty slot."""
+    _need_gpu()
+    w = wl.small("merge_badpos", 1, 200, 2000, 1800, 8, 2, 64, seed=24)
+    d = pipeline.dims_for(w)
+    sel = wl.random_selection(w, "cpu")
+    g = torch.Generator().manual_seed(7)
+    B, n_q, H, G = w.batch, w.n_q, w.h_q, w.h_kv
+    R = H // G
+    m = torch.randn((B, n_q, G, 16, R), generator=g)
+    l = torch.rand((B, n_q, G, 16, R), generator=g) + 0.5
+    acc = torch.randn((B, n_q, G, 16, R, 128), generator=g) * l[..., None]
+    ml = torch.stack([m, l], dim=-1).contiguous()
+    pos, ml_l, acc_l = _pieces_in_list_order(sel, ml, acc, g)
+    b0, g0, q0 = 0, 1, 17
+    s0 = int(torch.nonzero(pos[b0, g0, q0] >= 0)[0])
+    pos[b0, g0, q0, s0] = capi.msa_num_entries(d) + 5           # past every entry
+    out = torch.empty((B, n_q, H, 128), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((B, n_q, H), device="cuda")
+    err = torch.zeros((4,), dtype=torch.int32, device="cuda")
+    capi.msa_merge_partials(d, pos.cuda(), ml_l.cuda(), acc_l.cuda(), out, lse, err)
+    torch.cuda.synchronize()
+    assert int(err[0]) == 3                                      # MSA_DEVERR_BAD_ENTRY
+    # that row is the merge of its other slots
+    keep = (pos[b0, g0, q0] >= 0).numpy()
+    keep[s0] = False
+    h = g0 * R
+    o_ref, lse_ref = oracle.merge(keep[None].astype(np.int32), m[b0, q0, g0, :, 0][None].double().numpy(),
+                                  l[b0, q0, g0, :, 0][None].double().numpy(),
+                                  acc[b0, q0, g0, :, 0][None].double().numpy())
+    o = out[b0, q0, h].float().cpu().numpy()
+    assert np.abs(o - o_ref[0]).max() <= 1e-2 * max(1.0, np.abs(o_ref).max())
+    assert abs(float(lse[b0, q0, h]) - lse_ref[0]) <= 1e-4
+
+
 def test_compact_merge_kernel_against_oracle_merge():
     """Random compact pieces (bf16 acc / l, fp32 m and l; some slots unused)
     merged by the kernel and by the oracle, which gets acc = l * (acc / l)."""
