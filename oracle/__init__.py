@@ -18,6 +18,9 @@ Each function cites the page passage it follows in ``msa_oracle.c``:
     identity the KV-block-outer "Outer Gather Q" scheme relies on);
   * ``block_query_lists`` -- query->block lists inverted into block->query
     lists ("Kernel 创新：Outer Gather Q" section);
+  * ``entry_positions`` -- the inverse of those lists, (query, slot) -> entry
+    position (no counterpart on the pages: how the library finds a piece
+    stored in list order; plain Python over the lists);
   * ``e4m3_value``, ``quantize_e4m3``, ``index_pooled_e4m3`` -- the 8-bit
     (e4m3) variant of steps 1-2: per-tensor scale amax / 448, nearest code
     with ties to even, pooled scores from the codes;
