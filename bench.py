@@ -708,15 +708,29 @@ def main():
     # the side measurements and the CPU baseline run on a single-GPU run only: with
     # N > 1 every GPU of the job would stay held while rank 0 alone works
     single = world == 1
-    recall = bench_recall(w) if single and not args.no_recall else None
-    e4m3 = bench_e4m3(w) if single and not args.no_e4m3 else None
-    backward = (bench_backward(w, attn_flops, n_ent, peaks) if single and not args.no_bwd
-                else None)
-    compact = (bench_compact(w, max(3, args.steps // 2), args.warmup, peaks, peak_src)
-               if single and not args.no_compact else None)
-    configs = ({c.name: bench_config(c, max(3, args.steps // 2), args.warmup, peaks,
-                                     with_cpu=not args.no_cpu)
-                for c in (wl.P32, wl.M1)} if single and not args.no_configs else None)
+
+    def side(enabled, fn):
+        # a side measurement that fails is reported in its own key; the headline
+        # measurement above is already complete
+        if not (single and enabled):
+            return None
+        try:
+            return fn()
+        except Exception as exc:  # noqa: BLE001 -- any failure of a side measurement
+            print(f"bench: side measurement failed: {exc!r}", file=sys.stderr)
+            torch.cuda.empty_cache()
+            return {"error": repr(exc)}
+
+    recall = side(not args.no_recall, lambda: bench_recall(w))
+    e4m3 = side(not args.no_e4m3, lambda: bench_e4m3(w))
+    backward = side(not args.no_bwd, lambda: bench_backward(w, attn_flops, n_ent, peaks))
+    compact = side(not args.no_compact,
+                   lambda: bench_compact(w, max(3, args.steps // 2), args.warmup, peaks,
+                                         peak_src))
+    configs = side(not args.no_configs,
+                   lambda: {c.name: bench_config(c, max(3, args.steps // 2), args.warmup, peaks,
+                                                 with_cpu=not args.no_cpu)
+                            for c in (wl.P32, wl.M1)})
 
     sustained = peaks.get("bf16_tflops_sustained", FALLBACK["bf16_tflops_sustained"])
     burst = peaks.get("bf16_tflops", FALLBACK["bf16_tflops"])
@@ -780,7 +794,7 @@ def main():
     }
     if single and not args.no_cpu:
         line["cpu_baseline"], sample = cpu_baseline(w)
-        if recall is not None:
+        if recall is not None and "error" not in recall:
             rec_cpu, tok_cpu = sample.run_next_rows()
             recall["cpu_oracle"] = rec_cpu
             recall["token_level"]["cpu_oracle"] = tok_cpu
