@@ -63,7 +63,8 @@ typedef enum {
   MSA_OK = 0,
   MSA_ERR_INVALID_ARG = 1,        /* null pointer, bad size, inconsistent dims */
   MSA_ERR_UNSUPPORTED = 2,        /* valid but not implemented (e.g. d_idx 96) */
-  MSA_ERR_ALIGNMENT = 3,          /* pointer or stride not 16-byte aligned */
+  MSA_ERR_ALIGNMENT = 3,          /* pointer or stride not 16-byte aligned (32 where
+                                     an entry point says so) */
   MSA_ERR_WORKSPACE_TOO_SMALL = 4,
   MSA_ERR_CUDA = 5,               /* a CUDA runtime/driver call failed */
   MSA_ERR_SCRATCH_LIMIT = 6       /* needs more than the built-in scratch of the
@@ -73,7 +74,7 @@ typedef enum {
 /* device-side error codes written to *dev_err */
 #define MSA_DEVERR_TIMEOUT 1      /* a bounded wait on a barrier ran out */
 #define MSA_DEVERR_BAD_BLOCK 2    /* a selected block id outside [0, own] */
-#define MSA_DEVERR_BAD_ENTRY 3    /* a block->query entry out of range */
+#define MSA_DEVERR_BAD_ENTRY 3    /* a block->query entry or entry position out of range */
 
 /* Problem sizes.  Query i of batch b sits at absolute position
  * t = q_pos0 + i and may attend keys j <= t; keys are 0 .. n_kv-1 and
